@@ -1,0 +1,430 @@
+"""Benchmark of the weight-streaming decode GEMM on B200.
+
+One step = every GEMM of the workload once (default: the Qwen3-8B-shaped decode
+GEMMs -- fused QKV, o, fused gate_up, down -- at M = 1, 2, 4, 8, 16; 20 GEMMs,
+each with its own weight matrix, 1.93 GB of distinct weights per step, so the
+inputs are larger than L2 and no flush is needed).  The metric is achieved HBM
+bandwidth: algorithmic bytes (W + X read once) / time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl wsm|reference]
+                  [--workload qwen3_decode|single|skinny|l2_reuse|chain]
+
+Prints ONE JSON line on rank 0.  With N > 1 (launched by torchrun) every rank
+runs an independent replica of the workload on its own GPU (the GEMMs do not
+shard across GPUs); value = all ranks' bytes / the slowest rank's time.
+
+--impl reference times the fp64 CPU oracle (the only reference this method
+has) on a bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "achieved HBM GB/s (% of peak) and µs per bf16 decode GEMM at M=1–64 on 1 B200"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_cases(name):
+    if name == "qwen3_decode":
+        return synth.config_qwen3_decode()
+    if name == "single":
+        return synth.config_single()
+    if name == "skinny":
+        return synth.config_skinny()
+    if name == "l2_reuse":
+        return synth.config_l2_reuse()
+    if name == "chain":
+        return synth.chain_layout()
+    raise SystemExit(f"unknown workload {name}")
+
+
+def alg_bytes(c):
+    """Algorithmic bytes of one GEMM: W read once + X read once (bf16)."""
+    return 2 * c.N * c.K + 2 * c.M * c.K
+
+
+def out_bytes(c):
+    return 2 * c.M * c.N
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        time.sleep(0.05)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def setup_inputs(cases, dev, seed_base=0):
+    """Seeded device inputs per GEMM (generated on the device: same recipe,
+    X ~ N(0,1), W ~ N(0,1/K), fp32 rounded to bf16)."""
+    data = []
+    for i, c in enumerate(cases):
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed_base * 100003 + i * 7919 + c.seed)
+        x = torch.randn(c.M, c.K, generator=g, device=dev).to(torch.bfloat16)
+        w = (torch.randn(c.N, c.K, generator=g, device=dev) * (1.0 / c.K ** 0.5)).to(torch.bfloat16)
+        y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+        data.append((c, x, w, y))
+    return data
+
+
+def run_gpu(args, rank, world, local_rank):
+    import weight_streaming_megakernel_b200 as wsm
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cases = workload_cases(args.workload)
+    data = setup_inputs(cases, dev, seed_base=rank)
+    L = wsm.lib()
+    stream = torch.cuda.current_stream(dev)
+    s = stream.cuda_stream
+    chain = None
+
+    if args.workload == "chain":
+        tasks = [wsm.Task(x, w, y, dep=i - 1) for i, (c, x, w, y) in enumerate(data)]
+        chain = wsm.Chain(tasks)
+        launches_per_step = 1
+
+        def step(events=None):
+            if events is not None:
+                events[0].record(stream)
+            chain.run(s)
+            if events is not None:
+                events[1].record(stream)
+    else:
+        calls = []
+        for c, x, w, y in data:
+            if c.m_tile:
+                o = wsm._opts(m_tile=c.m_tile)
+                calls.append((True, x.data_ptr(), w.data_ptr(), y.data_ptr(), c.M, c.N, c.K, o))
+            else:
+                calls.append((False, x.data_ptr(), w.data_ptr(), y.data_ptr(), c.M, c.N, c.K, None))
+        launches_per_step = len(calls)
+        import ctypes
+
+        def step(events=None):
+            for i, (ex, xp, wp, yp, M, N, K, o) in enumerate(calls):
+                if events is not None:
+                    events[i].record(stream)
+                if ex:
+                    rc = L.skinny_gemm_ex(xp, wp, yp, M, N, K, ctypes.byref(o), s)
+                else:
+                    rc = L.skinny_gemm(xp, wp, yp, M, N, K, s)
+                if rc != 0:
+                    raise RuntimeError(f"skinny_gemm failed: {wsm.last_error()}")
+            if events is not None:
+                events[len(calls)].record(stream)
+
+    total_bytes = sum(alg_bytes(c) for c in cases)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+
+    # ---- timed region: K steps, events between launches
+    nev = launches_per_step + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+
+    # per-launch durations (event to event, same stream)
+    per_launch = [[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(launches_per_step)]
+                  for k in range(args.steps)]
+
+    # ---- e2e: public API, host buffers, H2D of X and D2H of Y inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        import weight_streaming_megakernel_b200 as wsm2
+        hx = [x.cpu().pin_memory() for (_, x, _, _) in data]
+        hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for (_, _, _, y) in data]
+        h2d = sum(t.numel() * 2 for t in hx)
+        d2h = sum(t.numel() * 2 for t in hy)
+
+        def e2e_step():
+            for (c, x, w, y), h in zip(data, hx):
+                x.copy_(h, non_blocking=True)
+            if chain is not None:
+                chain.run(s)
+            else:
+                for c, x, w, y in data:
+                    wsm2.skinny_gemm(x, w, y, m_tile=c.m_tile, stream=s)
+            for (c, x, w, y), h in zip(data, hy):
+                h.copy_(y, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": round(total_bytes * world / (e_ms / args.steps * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    status = wsm.stream_status(stream) if chain is None else chain.status(s)[0]
+    if status != 0:
+        raise RuntimeError(f"device-side status {status}")
+    return dict(cases=cases, total_bytes=total_bytes, ms_per_step=ms_per_step, per_launch=per_launch,
+                clocks=clk, e2e=e2e, launches_per_step=launches_per_step, chain=chain is not None)
+
+
+# ----------------------------------------------------------------------------- CPU arm
+
+def oracle_sample_rate(cases, budget_s, threads=0):
+    """Time the fp64 oracle on a bounded sample of every GEMM of the workload:
+    a fixed random subset of outputs per GEMM, sized to ~budget_s of CPU work.
+    Returns (seconds per full step extrapolated, cores, description)."""
+    import numpy as np
+    import oracle
+
+    cores = oracle.set_threads(threads or len(os.sched_getaffinity(0)))
+    macs_step = sum(c.M * c.N * c.K for c in cases)
+    # calibrate
+    c0 = max(cases, key=lambda c: c.K)
+    x, w = synth.make_xw(1, 64, c0.K, seed=0)
+    t0 = time.perf_counter()
+    oracle.gemm_ref(x, w)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    rate = 64 * c0.K / dt  # MAC/s
+    frac = min(1.0, budget_s * rate / macs_step)
+    rng = np.random.default_rng(0)
+    spent = 0.0
+    done_macs = 0
+    for i, c in enumerate(cases):
+        n_out = max(8, int(c.M * c.N * frac))
+        g = torch.Generator().manual_seed(i)
+        xs = torch.randn(c.M, c.K, generator=g).to(torch.bfloat16)
+        ws = (torch.randn(min(c.N, n_out), c.K, generator=g) / c.K ** 0.5).to(torch.bfloat16)
+        ms = rng.integers(0, c.M, n_out)
+        ns = rng.integers(0, ws.shape[0], n_out)
+        t0 = time.perf_counter()
+        oracle.gemm_ref_sampled(xs, ws, ms, ns)
+        spent += time.perf_counter() - t0
+        done_macs += n_out * c.K
+    per_step = spent * macs_step / max(done_macs, 1)
+    desc = (f"{done_macs / macs_step:.4%} of the step's outputs (random output positions of every GEMM), "
+            f"fp64 oracle, {cores} OpenMP threads, extrapolated by MAC count")
+    return per_step, cores, desc
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="wsm", choices=["wsm", "reference"])
+    ap.add_argument("--workload", default="qwen3_decode",
+                    choices=["qwen3_decode", "single", "skinny", "l2_reuse", "chain"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    hbm_peak, peak_kind = peaks()
+    cases = workload_cases(args.workload)
+    config = {"workload": {"qwen3_decode": "qwen3_8b_decode_gemms", "single": "single_gemm_m1_4096x4096",
+                           "skinny": "skinny_k7168_k8192", "l2_reuse": "l2_reuse_m32_m64",
+                           "chain": "chain_36x4_m16"}[args.workload],
+              "gemms_per_step": len(cases),
+              "M": sorted({c.M for c in cases}),
+              "shapes_KxN": sorted({f"{c.K}x{c.N}" for c in cases}),
+              "weight_bytes_per_step": sum(2 * c.N * c.K for c in cases),
+              "l2": "inputs larger than L2: every GEMM of a step has its own weights "
+                    f"({sum(2 * c.N * c.K for c in cases) / 1e9:.2f} GB per step, L2 126 MB)",
+              "parallelism": f"replicas{world}" if world > 1 else "single"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        budget = max(2.0, min(args.cpu_budget_s, 60.0 / max(1, args.steps + args.warmup)))
+        for _ in range(args.warmup):
+            oracle_sample_rate(cases, budget / 4)
+        per = []
+        for _ in range(args.steps):
+            sec, cores, desc = oracle_sample_rate(cases, budget)
+            per.append(sec)
+        per.sort()
+        sec = per[len(per) // 2]
+        tb = sum(alg_bytes(c) for c in cases)
+        val = tb / sec / 1e9
+        line = {"metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "impl": "reference",
+                "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                 "sample": desc},
+                "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local_rank))
+    r = run_gpu(args, rank, world, local_rank)
+
+    # roofline of the weight-streaming kernel: per-launch algorithmic bytes / duration
+    import statistics
+    per_case = []
+    if r["chain"]:
+        launch_ms = [row[0] for row in r["per_launch"]]
+        med = statistics.median(launch_ms)
+        fam_bytes, fam_ms = r["total_bytes"], med
+        us_per_gemm = {"chain_us": round(med * 1e3, 2), "per_gemm_us_avg": round(med * 1e3 / len(cases), 3)}
+        dominant = "wsm_umma_kernel (chain)"
+    else:
+        from weight_streaming_megakernel_b200 import plan
+        fam = {}
+        us_per_gemm = {}
+        for i, c in enumerate(r["cases"]):
+            ms = statistics.median(row[i] for row in r["per_launch"])
+            p = plan(c.M, c.N, c.K, num_sms=torch.cuda.get_device_properties(0).multi_processor_count,
+                     m_tile=c.m_tile)
+            k = "wsm_umma_kernel" if p["path"] == 2 else "wsm_stream_kernel"
+            b, t = fam.get(k, (0, 0.0))
+            fam[k] = (b + alg_bytes(c), t + ms)
+            us_per_gemm[c.name] = round(ms * 1e3, 2)
+            per_case.append((c.name, ms))
+        dominant = max(fam, key=lambda k: fam[k][1])
+        fam_bytes, fam_ms = fam[dominant]
+    achieved = fam_bytes / (fam_ms * 1e-3) / 1e9
+    value = r["total_bytes"] * world / (r["ms_per_step"] * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sec, cores, desc = oracle_sample_rate(cases, args.cpu_budget_s)
+        cpu = {"value": round(r["total_bytes"] / sec / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+                "frac_of_peak": round(value / world / hbm_peak, 4),
+                "frac_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
+                "roofline": {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": hbm_peak,
+                             "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                             "traffic": None},
+                "us_per_gemm": us_per_gemm,
+                "cpu_baseline": cpu,
+                "e2e": r["e2e"],
+                "gpu_launches": r["launches_per_step"] * args.steps,
+                "clocks": r["clocks"]}
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

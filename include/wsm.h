@@ -1,0 +1,228 @@
+/*
+ * wsm.h -- C ABI of libwsm, the weight-streaming decode GEMM library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (every entry point below computes it):
+ *
+ *     Y[m, n] = sum_k X[m, k] * W[n, k]       Y = X . W^T
+ *
+ * with X [M, K], W [N, K] and Y [M, N] bf16, row-major and contiguous (K is
+ * the contiguous dimension of X and W, N that of Y), fp32 accumulation and one
+ * round-to-nearest-even of the fp32 result to bf16.  M is the decode batch
+ * (1..64); K and N are in the thousands.  This is the decode-phase GEMM of
+ * "AMD: ROCm Low-Latency-GEMM-Kernel beschleunigen LLM-Inferenz bis zu 1,79x
+ * auf Instinct MI355X" (section "Was ist GEMM und die Decode-Phase eines
+ * LLMs?"), whose cost is streaming W from HBM once per call.  The chain entry
+ * runs a list of such GEMMs inside one resident kernel, the persistent
+ * megakernel of "Fleet: Hierarchical Task-based Abstraction for Megakernels
+ * on Multi-Die GPUs" (reading notes, sections 2a and 3d), with readiness
+ * counters in place of kernel launches.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named X, W, Y, Yf32, workspace are DEVICE pointers on the
+ *    current CUDA device, owned by the caller, and must stay valid until the
+ *    work queued on `stream` has finished.  X, W, Y must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  All work
+ *    is queued asynchronously on it; no entry point synchronises unless its
+ *    comment says so.
+ *  - Arguments are checked before anything is queued; a bad argument returns
+ *    an error code and queues nothing.  wsm_last_error() then holds a message
+ *    (per host thread).
+ *  - Shapes: 1 <= M <= 64, N >= 1, K >= 8 and K % 8 == 0 (rows must be
+ *    16-byte multiples for the tensor-memory-access engine).  Anything else
+ *    returns WSM_ERR_UNSUPPORTED; there is no slow fallback.
+ *  - Calls queued on one stream are serialised by the stream.  Calls on
+ *    different streams may run concurrently: the library keeps one scratch
+ *    workspace per (device, stream).
+ *  - The library never reads the values of Y before writing it.
+ */
+#ifndef WSM_H
+#define WSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *wsm_stream_t;
+
+typedef enum {
+    WSM_OK = 0,
+    WSM_ERR_INVALID = 1,     /* null pointer, negative size, bad option value */
+    WSM_ERR_UNSUPPORTED = 2, /* shape outside the supported range */
+    WSM_ERR_ALIGN = 3,       /* pointer not 16-byte aligned */
+    WSM_ERR_NOMEM = 4,       /* device allocation failed, or caller workspace too small */
+    WSM_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed (message has details) */
+    WSM_ERR_TIMEOUT = 6      /* a bounded device-side wait ran out (chain dependency or pipeline) */
+} wsm_status;
+
+/* Kernel path. */
+enum {
+    WSM_PATH_AUTO = 0,
+    WSM_PATH_STREAM = 1, /* fp32 FMA dot products + warp-shuffle reduction, M <= 8 */
+    WSM_PATH_UMMA = 2    /* tcgen05 MMA into tensor memory, any M (1..64) */
+};
+
+/* Order of (N-column tile, M-tile) pairs when M is split into several
+ * M-tiles (UMMA path with m_tile < M).  M-major keeps the M-tiles of one
+ * weight column adjacent in time so the column is fetched from HBM once and
+ * re-read from L2 ("Fleet ..." reading notes, section 3f, Eq.(1)). */
+enum {
+    WSM_ORDER_AUTO = 0,    /* = M-major */
+    WSM_ORDER_M_MAJOR = 1, /* column outer, M-tile inner */
+    WSM_ORDER_NAIVE = 2    /* M-tile outer, column inner (ablation) */
+};
+
+/* L2 policy of the weight stream.  Evict-first is only right when each weight
+ * byte has one reader; with several M-tiles sharing a column it would evict
+ * the column before its last reader ("Fleet ..." reading notes, section 3f,
+ * the bs = 64 shortfall of Eq.(1)). */
+enum {
+    WSM_L2_AUTO = 0,        /* evict-first when one M-tile, normal otherwise */
+    WSM_L2_EVICT_FIRST = 1,
+    WSM_L2_NORMAL = 2
+};
+
+/* Options of skinny_gemm_ex; zero-initialised = all automatic. */
+typedef struct {
+    int path;        /* WSM_PATH_* */
+    int m_tile;      /* UMMA path: rows of X per tile, 0 = all of M in one tile;
+                        otherwise a multiple of 16 in [16, 64] */
+    int order;       /* WSM_ORDER_* */
+    int l2_policy;   /* WSM_L2_* */
+    int grid;        /* persistent CTAs, 0 = one per SM; values above the
+                        number of SMs are clamped */
+    int reserved0;
+    float *Yf32;     /* optional device [M, N] fp32: the result before rounding */
+    void *workspace; /* optional caller scratch (device, >= wsm_workspace_bytes,
+                        16-byte aligned, zero-filled before its first use; the
+                        library leaves it in a reusable state after each call).
+                        NULL = library-owned per-stream scratch. */
+    size_t workspace_bytes;
+} wsm_opts;
+
+/* What the planner chose for a shape (wsm_plan). */
+typedef struct {
+    int path;          /* WSM_PATH_STREAM or WSM_PATH_UMMA */
+    int grid;          /* persistent CTAs */
+    int tile_rows;     /* rows of W (outputs along N) per tile */
+    int tile_k;        /* K elements per pipeline stage */
+    int m_tile;        /* X rows per tile (padded to the MMA width on UMMA) */
+    int m_tiles;       /* number of M-tiles */
+    int n_tiles;       /* number of N-column tiles */
+    int k_iters;       /* pipeline stages per tile */
+    int stages;        /* shared-memory ring depth */
+    int order;         /* WSM_ORDER_M_MAJOR or WSM_ORDER_NAIVE */
+    int l2_policy;     /* WSM_L2_EVICT_FIRST or WSM_L2_NORMAL */
+    int smem_bytes;    /* dynamic shared memory per CTA */
+    long long iters;   /* total stages = n_tiles * m_tiles * k_iters */
+    size_t workspace_bytes;
+} wsm_plan_info;
+
+/* Y = X . W^T, automatic plan.  Device pointers; asynchronous on `stream`. */
+wsm_status skinny_gemm(const void *X, const void *W, void *Y, int M, int N, int K,
+                       wsm_stream_t stream);
+
+/* Same with options (opts may be NULL). */
+wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, int K,
+                          const wsm_opts *opts, wsm_stream_t stream);
+
+/* Pure host function (no CUDA calls): the plan for a shape on a GPU with
+ * `num_sms` SMs.  Used by the tests and by wsm_workspace_bytes. */
+wsm_status wsm_plan(int M, int N, int K, int num_sms, const wsm_opts *opts,
+                    wsm_plan_info *out);
+
+/* Scratch a call with this shape needs on the current device (0 on error). */
+size_t wsm_workspace_bytes(int M, int N, int K, const wsm_opts *opts);
+
+/* Synchronise `stream`, then report whether a skinny_gemm call queued on it
+ * with the library-owned workspace recorded a device-side time-out of a
+ * bounded pipeline wait since the last check (which never happens in a
+ * healthy run); clears the record.  *code = 0 or WSM_ERR_TIMEOUT; the return
+ * value is WSM_ERR_TIMEOUT in the second case. */
+wsm_status wsm_stream_status(wsm_stream_t stream, int *code);
+
+/* ---------------------------------------------------------------- chains */
+
+/* One GEMM of a chain.  dep = -1, or the index of an EARLIER task whose Y
+ * must be complete before this task reads its X (dep < own index, so a chain
+ * can never deadlock: tiles are claimed in task order).  The wait covers X
+ * only: W is streamed before the dependency is met. */
+typedef struct {
+    const void *X;
+    const void *W;
+    void *Y;
+    int M, N, K;
+    int dep;
+    float *Yf32;   /* optional fp32 result, may be NULL */
+} wsm_task;
+
+typedef struct {
+    int path;                  /* WSM_PATH_* for every task (AUTO: by the largest M) */
+    int grid;                  /* 0 = one CTA per SM */
+    unsigned long long timeout_ns; /* bound on each dependency wait, 0 = 2 s */
+    int trace;                 /* nonzero: record per-CTA, per-task %globaltimer stamps */
+    int debug_unmet_dependency; /* test hook, 0 in real use: nonzero makes every dependency
+                                   target unreachable, so each dependency wait runs out after
+                                   timeout_ns and the run reports WSM_ERR_TIMEOUT */
+    int reserved[2];
+} wsm_chain_opts;
+
+typedef struct wsm_chain wsm_chain;  /* opaque prepared chain */
+
+/* Validate a task list and prepare it on the current device: device task
+ * table, tensor maps, per-task scratch and readiness counters.  Validation
+ * runs before any allocation and rejects null pointers (WSM_ERR_INVALID),
+ * shapes outside the supported range (WSM_ERR_UNSUPPORTED), misaligned
+ * pointers (WSM_ERR_ALIGN) and a dependency index outside [-1, own index)
+ * (WSM_ERR_INVALID: forward and self dependencies could deadlock).  A
+ * dependency does not have to be a data dependency; it may order tasks only.
+ * The task array is copied; the caller may free it on return. */
+wsm_status wsm_chain_create(const wsm_task *tasks, int n_tasks, const wsm_chain_opts *opts,
+                            wsm_chain **out);
+
+/* Run a prepared chain as ONE persistent kernel on `stream`. */
+wsm_status wsm_chain_run(wsm_chain *chain, wsm_stream_t stream);
+
+/* Synchronise `stream`, then report the device-side status of the chain's
+ * last run: WSM_OK, or WSM_ERR_TIMEOUT with *failed_task = the first task
+ * whose wait ran out (may be NULL). */
+wsm_status wsm_chain_status(wsm_chain *chain, wsm_stream_t stream, int *failed_task);
+
+/* Copy the trace of the last run (trace != 0 at create) into host `out`:
+ * stamps[cta][task][3] = {first stage issued, dependency met, last tile
+ * written}, %globaltimer nanoseconds, 0 where the CTA had no work for the
+ * task.  `capacity` is the number of uint64 slots in `out`; returns the number
+ * needed (grid * n_tasks * 3), or 0 when tracing was not enabled.
+ * Synchronises `stream`. */
+size_t wsm_chain_trace(wsm_chain *chain, wsm_stream_t stream, unsigned long long *out,
+                       size_t capacity);
+
+/* Free a prepared chain (synchronises the device). */
+void wsm_chain_destroy(wsm_chain *chain);
+
+/* One-shot: validate, prepare (cached by the task list's contents, per
+ * device) and run the chain on `stream`.  Equivalent to create + run. */
+wsm_status gemm_chain(const wsm_task *tasks, int n_tasks, wsm_stream_t stream);
+
+/* Validation only (pure host function, no CUDA calls). */
+wsm_status wsm_chain_validate(const wsm_task *tasks, int n_tasks);
+
+/* ---------------------------------------------------------------- misc */
+
+/* Message of the last error on this host thread ("" when none). */
+const char *wsm_last_error(void);
+
+/* ABI version of this header (bumped on any incompatible change). */
+int wsm_abi_version(void);
+
+#define WSM_ABI_VERSION 1
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WSM_H */

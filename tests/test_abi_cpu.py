@@ -1,0 +1,177 @@
+"""C-ABI library checks that need no GPU: it loads, exports every function
+include/wsm.h declares, and its pure host logic (planning, task-list
+validation) behaves as documented."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+import weight_streaming_megakernel_b200 as wsm
+from weight_streaming_megakernel_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wsm.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    _build.build()
+    yield
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while", "sizeof")))
+
+
+def test_header_parse_sees_all_entry_points():
+    names = header_functions()
+    assert set(names) == set(wsm.HEADER_SYMBOLS), names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(wsm.LIB_PATH)
+    for name in header_functions():
+        assert hasattr(lib, name), f"{name} declared in wsm.h but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", wsm.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in header_functions():
+        assert name in exported
+
+
+def test_abi_version():
+    assert wsm.abi_version() == 1
+
+
+def test_plan_paths_and_geometry():
+    p = wsm.plan(1, 4096, 4096, num_sms=148)
+    assert p["path"] == wsm.PATH_STREAM and p["tile_rows"] == 16 and p["m_tile"] == 1
+    assert p["n_tiles"] == 256 and p["k_iters"] == 4096 // p["tile_k"]
+    assert p["iters"] == p["n_tiles"] * p["k_iters"] and p["grid"] == 148
+    p = wsm.plan(16, 4096, 4096, num_sms=148)
+    assert p["path"] == wsm.PATH_UMMA and p["tile_rows"] == 128 and p["tile_k"] == 64 and p["m_tile"] == 16
+    assert p["n_tiles"] == 32 and p["k_iters"] == 64 and p["m_tiles"] == 1
+    p = wsm.plan(17, 100, 1000, num_sms=148)
+    assert p["m_tile"] == 32 and p["n_tiles"] == 1 and p["k_iters"] == 16
+    p = wsm.plan(8, 4096, 4096, num_sms=148, path=wsm.PATH_UMMA)
+    assert p["path"] == wsm.PATH_UMMA and p["m_tile"] == 16
+
+
+def test_plan_ring_fits_shared_memory():
+    for M in (1, 2, 3, 4, 8, 16, 33, 64):
+        p = wsm.plan(M, 4096, 4096, num_sms=148)
+        assert 2 <= p["stages"] <= 16
+        assert p["smem_bytes"] <= 232448 - 4096
+
+
+def test_plan_grid_clamped_to_work():
+    p = wsm.plan(1, 16, 8, num_sms=148)
+    assert p["iters"] == 1 and p["grid"] == 1
+    p = wsm.plan(1, 4096, 4096, num_sms=148, grid=7)
+    assert p["grid"] == 7
+    p = wsm.plan(1, 4096, 4096, num_sms=148, grid=1000)
+    assert p["grid"] == 148
+
+
+def test_plan_m_tiling_and_l2_policy():
+    p = wsm.plan(64, 24576, 4096, num_sms=148, m_tile=16)
+    assert p["m_tiles"] == 4 and p["m_tile"] == 16 and p["l2_policy"] == wsm.L2_NORMAL
+    assert p["order"] == wsm.ORDER_M_MAJOR
+    p = wsm.plan(64, 24576, 4096, num_sms=148, m_tile=32, order=wsm.ORDER_NAIVE)
+    assert p["m_tiles"] == 2 and p["order"] == wsm.ORDER_NAIVE
+    p = wsm.plan(32, 4096, 12288, num_sms=148)
+    assert p["m_tiles"] == 1 and p["l2_policy"] == wsm.L2_EVICT_FIRST
+
+
+def test_plan_workspace_formula():
+    p = wsm.plan(16, 4096, 4096, num_sms=148)
+    slots = 2 * p["grid"] * 128 * 16 * 4
+    assert p["workspace_bytes"] >= 256 + p["n_tiles"] * p["m_tiles"] * 4 + slots
+    assert p["workspace_bytes"] % 256 == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(0, 16, 16), (65, 16, 16), (1, 0, 16), (1, 16, 4), (1, 16, 12), (1, 16, 0)])
+def test_plan_rejects_unsupported_shapes(M, N, K):
+    with pytest.raises(wsm.WsmError) as e:
+        wsm.plan(M, N, K)
+    assert e.value.code == wsm.WSM_ERR_UNSUPPORTED
+
+
+def test_plan_rejects_bad_options():
+    with pytest.raises(wsm.WsmError) as e:
+        wsm.plan(9, 64, 64, path=wsm.PATH_STREAM)
+    assert e.value.code == wsm.WSM_ERR_UNSUPPORTED
+    for tm in (8, 24, 80):
+        with pytest.raises(wsm.WsmError) as e:
+            wsm.plan(64, 64, 64, m_tile=tm)
+        assert e.value.code == wsm.WSM_ERR_UNSUPPORTED
+    with pytest.raises(wsm.WsmError) as e:
+        wsm.plan(4, 64, 64, path=7)
+    assert e.value.code == wsm.WSM_ERR_INVALID
+    with pytest.raises(wsm.WsmError) as e:
+        wsm.plan(4, 64, 64, grid=-1)
+    assert e.value.code == wsm.WSM_ERR_INVALID
+
+
+def _task(i, M=4, N=64, K=64, dep=-1, base=0x10000000):
+    a = base + i * 0x100000
+    return {"X": a, "W": a + 0x40000, "Y": a + 0x80000, "M": M, "N": N, "K": K, "dep": dep}
+
+
+def test_chain_validation_accepts_good_lists():
+    wsm.chain_validate([_task(0), _task(1, dep=0), _task(2, dep=0), _task(3, dep=2)])
+
+
+@pytest.mark.parametrize("bad,code", [
+    ({"dep": 3}, wsm.WSM_ERR_INVALID),      # forward dependency
+    ({"dep": 1}, wsm.WSM_ERR_INVALID),      # self dependency
+    ({"dep": -2}, wsm.WSM_ERR_INVALID),
+    ({"X": 0}, wsm.WSM_ERR_INVALID),        # null pointer
+    ({"Y": 0x10000008}, wsm.WSM_ERR_ALIGN),  # misaligned
+    ({"K": 12}, wsm.WSM_ERR_UNSUPPORTED),
+    ({"M": 65}, wsm.WSM_ERR_UNSUPPORTED),
+])
+def test_chain_validation_rejects(bad, code):
+    tasks = [_task(0), _task(1, dep=0)]
+    tasks[1].update(bad)
+    with pytest.raises(wsm.WsmError) as e:
+        wsm.chain_validate(tasks)
+    assert e.value.code == code
+
+
+def test_chain_validation_empty():
+    with pytest.raises(wsm.WsmError) as e:
+        wsm.chain_validate([])
+    assert e.value.code == wsm.WSM_ERR_INVALID
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    code = (
+        "import weight_streaming_megakernel_b200 as w\n"
+        f"w.LIB_PATH = {str(tmp_path / 'nope.so')!r}\n"
+        "try:\n"
+        "    w.lib()\n"
+        "except RuntimeError as e:\n"
+        "    print('RAISED', e)\n"
+    )
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT)
+    assert "RAISED" in out.stdout and "not built" in out.stdout
+
+
+def test_product_never_touches_the_oracle():
+    """The product package shares nothing with oracle/ and never imports it."""
+    pkg = os.path.dirname(wsm.__file__)
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f
+                assert "wsmo_" not in src, f
+    oracle_src = open(os.path.join(ROOT, "oracle", "oracle.c")).read()
+    assert "wsm.h" not in oracle_src and "wsm_internal" not in oracle_src

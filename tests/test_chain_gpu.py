@@ -1,0 +1,164 @@
+"""gemm_chain: one persistent kernel runs a list of GEMMs with readiness
+counters.  Checked against the per-task oracle: a data-dependent chain (task
+t reads task t-1's Y, so a counter that fails to order them gives a wrong
+result, not an invisible race), independent tasks at the real layer shapes,
+both kernel paths, repeated runs (epoch counters), the bounded dependency
+wait (a target nothing reaches must end in WSM_ERR_TIMEOUT, not a hang), the
+trace stamps, and the one-shot entry point."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import weight_streaming_megakernel_b200 as wsm
+from parity import check_full, check_sampled
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    yield
+
+
+def dependent_chain(M, dims, seed=0):
+    """Task t: Y_t = Y_{t-1} . W_t^T with W_t [dims[t+1], dims[t]]."""
+    x0 = synth.make_x(M, dims[0], seed).to(DEV)
+    ws = [synth.make_w(dims[t + 1], dims[t], 1000 + seed + t).to(DEV) for t in range(len(dims) - 1)]
+    ys = [torch.full((M, dims[t + 1]), float("nan"), dtype=torch.bfloat16, device=DEV) for t in range(len(ws))]
+    yfs = [torch.empty(M, dims[t + 1], dtype=torch.float32, device=DEV) for t in range(len(ws))]
+    tasks = []
+    for t in range(len(ws)):
+        x = x0 if t == 0 else ys[t - 1]
+        tasks.append(wsm.Task(x, ws[t], ys[t], dep=t - 1, yf32=yfs[t]))
+    return x0, ws, ys, yfs, tasks
+
+
+def check_dependent(x0, ws, ys, yfs):
+    x = x0
+    for t in range(len(ws)):
+        # each task against the oracle on the GPU's own input, so errors do not compound
+        check_full(x.cpu(), ws[t].cpu(), ys[t], yfs[t], what=f"task {t}")
+        x = ys[t]
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_UMMA, 16), (wsm.PATH_UMMA, 64), (wsm.PATH_STREAM, 4),
+                                    (wsm.PATH_STREAM, 1)])
+def test_dependent_chain(path, M):
+    dims = [1024, 2048, 1024, 3072, 512, 1024, 4096, 1024]
+    x0, ws, ys, yfs, tasks = dependent_chain(M, dims, seed=M)
+    ch = wsm.Chain(tasks, path=path)
+    ch.run()
+    code, failed = ch.status()
+    assert code == wsm.WSM_OK, (code, failed, wsm.last_error())
+    check_dependent(x0, ws, ys, yfs)
+    # run again (next epoch) after poisoning the outputs
+    for y in ys:
+        y.fill_(float("nan"))
+    ch.run()
+    assert ch.status()[0] == wsm.WSM_OK
+    check_dependent(x0, ws, ys, yfs)
+    ch.close()
+
+
+def test_dependent_chain_small_grid_and_empty_ctas():
+    """A grid larger than some tasks' stage counts (CTAs with no work for a
+    task) and a tiny grid (long per-CTA ranges)."""
+    dims = [64, 128, 64, 256]
+    for grid in (148, 3):
+        x0, ws, ys, yfs, tasks = dependent_chain(16, dims, seed=grid)
+        ch = wsm.Chain(tasks, path=wsm.PATH_UMMA, grid=grid)
+        ch.run()
+        assert ch.status()[0] == wsm.WSM_OK
+        check_dependent(x0, ws, ys, yfs)
+        ch.close()
+        x0, ws, ys, yfs, tasks = dependent_chain(2, dims, seed=grid)
+        ch = wsm.Chain(tasks, path=wsm.PATH_STREAM, grid=grid)
+        ch.run()
+        assert ch.status()[0] == wsm.WSM_OK
+        check_dependent(x0, ws, ys, yfs)
+        ch.close()
+
+
+def test_layer_shapes_chain():
+    """Two layers of the Qwen3-8B-shaped chain at M = 16, ordering-only
+    dependencies (task t waits for task t-1), inputs independent per task."""
+    cases = synth.chain_layout(layers=2, M=16)
+    tasks, refs = [], []
+    for t, c in enumerate(cases):
+        x = synth.make_x(c.M, c.K, c.seed).to(DEV)
+        w = synth.make_w(c.N, c.K, 10000 + c.seed).to(DEV)
+        y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=DEV)
+        yf = torch.empty(c.M, c.N, dtype=torch.float32, device=DEV)
+        tasks.append(wsm.Task(x, w, y, dep=t - 1, yf32=yf))
+    ch = wsm.Chain(tasks, trace=True)
+    ch.run()
+    assert ch.status()[0] == wsm.WSM_OK
+    rng = np.random.default_rng(1)
+    for t, task in enumerate(tasks):
+        ms = rng.integers(0, 16, 2048)
+        ns = rng.integers(0, task.w.shape[0], 2048)
+        check_sampled(task.x, task.w, task.y, task.yf32, ms, ns, what=f"task {t}")
+    tr = ch.trace()
+    assert tr is not None and tr.shape[1] == len(tasks)
+    # every task's dependency was met no earlier than its predecessor's first stage
+    started = tr[:, :, 0]
+    assert (started[:, 0] > 0).any()
+    ch.close()
+
+
+def test_bounded_dependency_wait_times_out():
+    """A dependency target nothing reaches: each wait runs out after the
+    timeout, the run ends, and the status names the waiting task."""
+    dims = [256, 256, 256]
+    x0, ws, ys, yfs, tasks = dependent_chain(16, dims, seed=5)
+    ch = wsm.Chain(tasks, path=wsm.PATH_UMMA, timeout_ns=20_000_000, debug_unmet_dependency=True)
+    t0 = time.time()
+    ch.run()
+    code, failed = ch.status()
+    elapsed = time.time() - t0
+    assert code == wsm.WSM_ERR_TIMEOUT and failed in (1, 2)
+    assert elapsed < 10.0
+    ch.close()
+    # the context is still usable and a normal chain still works
+    x0, ws, ys, yfs, tasks = dependent_chain(16, dims, seed=6)
+    ch = wsm.Chain(tasks, path=wsm.PATH_UMMA)
+    ch.run()
+    assert ch.status()[0] == wsm.WSM_OK
+    check_dependent(x0, ws, ys, yfs)
+    ch.close()
+
+
+def test_gemm_chain_one_shot():
+    dims = [512, 1024, 512]
+    x0, ws, ys, yfs, tasks = dependent_chain(8, dims, seed=11)
+    wsm.gemm_chain(tasks)
+    torch.cuda.synchronize()
+    check_dependent(x0, ws, ys, yfs)
+    for y in ys:
+        y.fill_(0)
+    wsm.gemm_chain(tasks)  # cached prepared chain, next epoch
+    torch.cuda.synchronize()
+    check_dependent(x0, ws, ys, yfs)
+
+
+def test_independent_tasks_no_deps():
+    tasks = []
+    for t in range(5):
+        M, N, K = [1, 3, 8, 5, 2][t], [4096, 100, 2112, 33, 640][t], [4096, 7168, 512, 8, 1032][t]
+        x, w = synth.make_xw(M, N, K, seed=t)
+        tasks.append(wsm.Task(x.to(DEV), w.to(DEV), torch.empty(M, N, dtype=torch.bfloat16, device=DEV),
+                              yf32=torch.empty(M, N, dtype=torch.float32, device=DEV)))
+    ch = wsm.Chain(tasks)
+    ch.run()
+    assert ch.status()[0] == wsm.WSM_OK
+    for t in tasks:
+        check_full(t.x.cpu(), t.w.cpu(), t.y, t.yf32)
+    ch.close()

@@ -1,0 +1,235 @@
+"""Parity of skinny_gemm (both kernel paths) with the fp64 oracle, through the
+C ABI, on seeded inputs: small shapes spanning several tiles with ragged
+tails, every M, integer and permutation cases that must be exact, split
+patterns (grid sizes), M-tiling orders, caller workspace, determinism, CUDA
+graph capture, and the full-size workloads on sampled outputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import weight_streaming_megakernel_b200 as wsm
+from parity import check_full, check_sampled, bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    yield
+
+
+def run(x, w, **kw):
+    M, K = x.shape
+    N = w.shape[0]
+    xd, wd = x.to(DEV), w.to(DEV)
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    yf = torch.full((M, N), float("nan"), dtype=torch.float32, device=DEV)
+    wsm.skinny_gemm(xd, wd, y, yf32=yf, **kw)
+    torch.cuda.synchronize()
+    assert wsm.stream_status() == 0
+    return y, yf
+
+
+SHAPES = [(1, 8), (17, 40), (300, 1000), (129, 4104), (1024, 4096), (2112, 7168)]
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("N,K", SHAPES)
+def test_stream_path_small(M, N, K):
+    x, w = synth.make_xw(M, N, K, seed=M * 7 + N)
+    y, yf = run(x, w, path=wsm.PATH_STREAM)
+    check_full(x, w, y, yf, what=f"stream M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("M", [1, 8, 16, 17, 32, 40, 64])
+@pytest.mark.parametrize("N,K", SHAPES)
+def test_umma_path_small(M, N, K):
+    x, w = synth.make_xw(M, N, K, seed=M * 5 + N)
+    y, yf = run(x, w, path=wsm.PATH_UMMA)
+    check_full(x, w, y, yf, what=f"umma M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("path,ms", [(wsm.PATH_STREAM, range(1, 9)), (wsm.PATH_UMMA, range(1, 65))])
+def test_every_m(path, ms):
+    N, K = 520, 1032
+    for M in ms:
+        x, w = synth.make_xw(M, N, K, seed=100 + M)
+        y, yf = run(x, w, path=path)
+        check_full(x, w, y, yf, what=f"path={path} M={M}")
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 1), (wsm.PATH_STREAM, 7), (wsm.PATH_UMMA, 16),
+                                    (wsm.PATH_UMMA, 64)])
+def test_integer_inputs_exact(path, M):
+    """Small integers: every partial sum is exact in fp32, so the fp32 output
+    must equal the oracle exactly whatever the split."""
+    N, K = 777, 4096
+    x, w = synth.make_int_xw(M, N, K, seed=M)
+    Y_ref, _ = oracle.gemm_ref(x, w)
+    for grid in (0, 1, 5, 37):
+        y, yf = run(x, w, path=path, grid=grid)
+        assert np.array_equal(yf.cpu().double().numpy(), Y_ref), f"grid={grid}"
+        assert np.array_equal(bf16_bits(y), oracle.round_bf16(Y_ref))
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 4), (wsm.PATH_UMMA, 16)])
+def test_identity_and_permutation(path, M):
+    K = 512
+    x, _ = synth.make_xw(M, K, K, seed=3)
+    I = torch.eye(K, dtype=torch.bfloat16)
+    y, yf = run(x, I, path=path)
+    assert torch.equal(y.cpu(), x)
+    P, p = synth.make_permutation_w(K, seed=4)
+    y, yf = run(x, P, path=path)
+    assert torch.equal(y.cpu(), x[:, p])
+    xo, idx = synth.make_onehot_x(M, K, seed=5)
+    _, w = synth.make_xw(1, 300, K, seed=6)
+    y, _ = run(xo, w, path=path)
+    assert torch.equal(y.cpu(), w[:, idx].T.contiguous())
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 1), (wsm.PATH_STREAM, 8), (wsm.PATH_UMMA, 16),
+                                    (wsm.PATH_UMMA, 48)])
+@pytest.mark.parametrize("grid", [1, 2, 3, 7, 64, 148])
+def test_split_patterns(path, M, grid):
+    """Different grids put the split points (and the in-order reductions) in
+    different places; every one must satisfy the bound."""
+    N, K = 1000, 6144
+    x, w = synth.make_xw(M, N, K, seed=grid)
+    y, yf = run(x, w, path=path, grid=grid)
+    check_full(x, w, y, yf, what=f"grid={grid}")
+
+
+def test_all_ones_closed_form():
+    for path, M in ((wsm.PATH_STREAM, 3), (wsm.PATH_UMMA, 20)):
+        K = 256
+        x = torch.ones(M, K, dtype=torch.bfloat16)
+        w = torch.ones(130, K, dtype=torch.bfloat16)
+        y, yf = run(x, w, path=path)
+        assert (yf.cpu() == K).all() and (y.cpu().float() == K).all()
+
+
+@pytest.mark.parametrize("M,tm", [(32, 16), (64, 16), (64, 32), (40, 16)])
+@pytest.mark.parametrize("order", [wsm.ORDER_M_MAJOR, wsm.ORDER_NAIVE])
+def test_m_tiling(M, tm, order):
+    N, K = 1100, 2048
+    x, w = synth.make_xw(M, N, K, seed=M + tm)
+    y, yf = run(x, w, path=wsm.PATH_UMMA, m_tile=tm, order=order)
+    check_full(x, w, y, yf, what=f"M={M} tm={tm} order={order}")
+    xi, wi = synth.make_int_xw(M, N, K, seed=1)
+    Y_ref, _ = oracle.gemm_ref(xi, wi)
+    y, yf = run(xi, wi, path=wsm.PATH_UMMA, m_tile=tm, order=order)
+    assert np.array_equal(yf.cpu().double().numpy(), Y_ref)
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 4), (wsm.PATH_UMMA, 32)])
+def test_deterministic(path, M):
+    N, K = 4096, 4096
+    x, w = synth.make_xw(M, N, K, seed=9)
+    y1, f1 = run(x, w, path=path)
+    y2, f2 = run(x, w, path=path)
+    assert torch.equal(y1, y2) and torch.equal(f1.view(torch.int32), f2.view(torch.int32))
+
+
+def test_l2_policy_options_same_result():
+    x, w = synth.make_xw(16, 2000, 3000, seed=1)
+    outs = []
+    for pol in (wsm.L2_EVICT_FIRST, wsm.L2_NORMAL):
+        y, yf = run(x, w, path=wsm.PATH_UMMA, l2_policy=pol)
+        outs.append(yf)
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_caller_workspace():
+    M, N, K = 8, 4096, 4096
+    x, w = synth.make_xw(M, N, K, seed=2)
+    need = wsm.workspace_bytes(M, N, K)
+    ws = torch.zeros(need // 4 + 64, dtype=torch.int32, device=DEV)
+    y, yf = run(x, w, workspace=ws)
+    check_full(x, w, y, yf)
+    y2, yf2 = run(x, w, workspace=ws)  # left reusable by the first call
+    assert torch.equal(yf, yf2)
+    with pytest.raises(wsm.WsmError) as e:
+        run(x, w, workspace=ws[:8])
+    assert e.value.code == wsm.WSM_ERR_NOMEM
+
+
+def test_argument_errors():
+    x = torch.zeros(2, 64, dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros(64, 64, dtype=torch.bfloat16, device=DEV)
+    y = torch.zeros(2, 64, dtype=torch.bfloat16, device=DEV)
+    L = wsm.lib()
+    s = torch.cuda.current_stream().cuda_stream
+    assert L.skinny_gemm(0, w.data_ptr(), y.data_ptr(), 2, 64, 64, s) == wsm.WSM_ERR_INVALID
+    assert L.skinny_gemm(x.data_ptr() + 2, w.data_ptr(), y.data_ptr(), 2, 64, 64, s) == wsm.WSM_ERR_ALIGN
+    assert L.skinny_gemm(x.data_ptr(), w.data_ptr(), y.data_ptr(), 2, 64, 60, s) == wsm.WSM_ERR_UNSUPPORTED
+    assert L.skinny_gemm(x.data_ptr(), w.data_ptr(), y.data_ptr(), 65, 64, 64, s) == wsm.WSM_ERR_UNSUPPORTED
+    assert "unsupported" in wsm.last_error()
+
+
+def test_cuda_graph_capture():
+    M, N, K = 16, 4096, 4096
+    x, w = synth.make_xw(M, N, K, seed=4)
+    xd, wd = x.to(DEV), w.to(DEV)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        wsm.skinny_gemm(xd, wd, y)  # sizes the stream's workspace outside capture
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        wsm.skinny_gemm(xd, wd, y, stream=s)
+    y.fill_(0)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    check_full(x, w, y)
+
+
+def test_empty_ranges_when_fewer_stages_than_ctas():
+    """T < grid: the plan clamps the grid, and a forced-large grid on a chain
+    covers it in-kernel (see the chain tests)."""
+    x, w = synth.make_xw(3, 40, 64, seed=1)
+    y, yf = run(x, w, path=wsm.PATH_STREAM, grid=148)
+    check_full(x, w, y, yf)
+    x, w = synth.make_xw(20, 130, 128, seed=1)
+    y, yf = run(x, w, path=wsm.PATH_UMMA, grid=148)
+    check_full(x, w, y, yf)
+
+
+# ----------------------------------------------------------- full-size workloads
+
+def _full_cases():
+    cases = []
+    cases += synth.config_single()
+    cases += synth.config_qwen3_decode()
+    cases += synth.config_skinny()
+    cases += synth.config_l2_reuse()
+    return cases
+
+
+@pytest.mark.parametrize("case", _full_cases(), ids=lambda c: c.name)
+def test_full_size_sampled(case):
+    """The benchmark's shapes and launch configuration (default plan; M-tile
+    where the config names one), checked on 4096 sampled outputs."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(case.seed)
+    x = torch.randn(case.M, case.K, generator=g, device=DEV).to(torch.bfloat16)
+    w = (torch.randn(case.N, case.K, generator=g, device=DEV) / case.K ** 0.5).to(torch.bfloat16)
+    y = torch.empty(case.M, case.N, dtype=torch.bfloat16, device=DEV)
+    yf = torch.empty(case.M, case.N, dtype=torch.float32, device=DEV)
+    kw = {"m_tile": case.m_tile} if case.m_tile else {}
+    wsm.skinny_gemm(x, w, y, yf32=yf, **kw)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(0)
+    ms = rng.integers(0, case.M, 4096)
+    ns = rng.integers(0, case.N, 4096)
+    ns[:64] = np.arange(case.N - 64, case.N)  # the ragged end of N
+    check_sampled(x, w, y, yf, ms, ns, what=case.name)

@@ -1,0 +1,303 @@
+"""Python binding of libwsm, the weight-streaming decode GEMM library for B200.
+
+Thin ctypes marshalling over the C ABI declared in ``include/wsm.h``: every
+step of the computation runs in the library's CUDA kernels.  PyTorch supplies
+device memory and streams only.  If ``libwsm.so`` is missing every call raises
+(there is no fallback); build it with ``python -m
+weight_streaming_megakernel_b200._build`` or ``__graft_entry__.build()``.
+
+    Y[m, n] = sum_k X[m, k] * W[n, k]     (X [M,K], W [N,K], Y [M,N], bf16)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "LIB_PATH", "WSM_OK", "WSM_ERR_INVALID", "WSM_ERR_UNSUPPORTED", "WSM_ERR_ALIGN", "WSM_ERR_NOMEM",
+    "WSM_ERR_CUDA", "WSM_ERR_TIMEOUT", "PATH_AUTO", "PATH_STREAM", "PATH_UMMA", "ORDER_AUTO", "ORDER_M_MAJOR",
+    "ORDER_NAIVE", "L2_AUTO", "L2_EVICT_FIRST", "L2_NORMAL", "WsmError", "lib", "skinny_gemm", "plan",
+    "workspace_bytes", "stream_status", "Task", "Chain", "gemm_chain", "chain_validate", "last_error",
+    "abi_version", "HEADER_SYMBOLS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwsm.so")
+
+WSM_OK, WSM_ERR_INVALID, WSM_ERR_UNSUPPORTED, WSM_ERR_ALIGN, WSM_ERR_NOMEM, WSM_ERR_CUDA, WSM_ERR_TIMEOUT = range(7)
+_STATUS_NAMES = {0: "WSM_OK", 1: "WSM_ERR_INVALID", 2: "WSM_ERR_UNSUPPORTED", 3: "WSM_ERR_ALIGN",
+                 4: "WSM_ERR_NOMEM", 5: "WSM_ERR_CUDA", 6: "WSM_ERR_TIMEOUT"}
+PATH_AUTO, PATH_STREAM, PATH_UMMA = 0, 1, 2
+ORDER_AUTO, ORDER_M_MAJOR, ORDER_NAIVE = 0, 1, 2
+L2_AUTO, L2_EVICT_FIRST, L2_NORMAL = 0, 1, 2
+
+# Every function include/wsm.h declares (checked by the CPU tests).
+HEADER_SYMBOLS = (
+    "skinny_gemm", "skinny_gemm_ex", "wsm_plan", "wsm_workspace_bytes", "wsm_stream_status",
+    "wsm_chain_create", "wsm_chain_run", "wsm_chain_status", "wsm_chain_trace", "wsm_chain_destroy",
+    "gemm_chain", "wsm_chain_validate", "wsm_last_error", "wsm_abi_version",
+)
+
+
+class WsmError(RuntimeError):
+    def __init__(self, code: int, where: str, msg: str):
+        self.code = code
+        super().__init__(f"{where}: {_STATUS_NAMES.get(code, code)}: {msg}")
+
+
+class _Opts(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("m_tile", ctypes.c_int), ("order", ctypes.c_int),
+                ("l2_policy", ctypes.c_int), ("grid", ctypes.c_int), ("reserved0", ctypes.c_int),
+                ("Yf32", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class _PlanInfo(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("grid", ctypes.c_int), ("tile_rows", ctypes.c_int),
+                ("tile_k", ctypes.c_int), ("m_tile", ctypes.c_int), ("m_tiles", ctypes.c_int),
+                ("n_tiles", ctypes.c_int), ("k_iters", ctypes.c_int), ("stages", ctypes.c_int),
+                ("order", ctypes.c_int), ("l2_policy", ctypes.c_int), ("smem_bytes", ctypes.c_int),
+                ("iters", ctypes.c_longlong), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class _Task(ctypes.Structure):
+    _fields_ = [("X", ctypes.c_void_p), ("W", ctypes.c_void_p), ("Y", ctypes.c_void_p),
+                ("M", ctypes.c_int), ("N", ctypes.c_int), ("K", ctypes.c_int), ("dep", ctypes.c_int),
+                ("Yf32", ctypes.c_void_p)]
+
+
+class _ChainOpts(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("grid", ctypes.c_int), ("timeout_ns", ctypes.c_ulonglong),
+                ("trace", ctypes.c_int), ("debug_unmet_dependency", ctypes.c_int), ("reserved", ctypes.c_int * 2)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libwsm.so is not built ({LIB_PATH}); run "
+                               "`python -m weight_streaming_megakernel_b200._build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_int
+        L.skinny_gemm.argtypes = [vp, vp, vp, i, i, i, vp]
+        L.skinny_gemm.restype = st
+        L.skinny_gemm_ex.argtypes = [vp, vp, vp, i, i, i, ctypes.POINTER(_Opts), vp]
+        L.skinny_gemm_ex.restype = st
+        L.wsm_plan.argtypes = [i, i, i, i, ctypes.POINTER(_Opts), ctypes.POINTER(_PlanInfo)]
+        L.wsm_plan.restype = st
+        L.wsm_workspace_bytes.argtypes = [i, i, i, ctypes.POINTER(_Opts)]
+        L.wsm_workspace_bytes.restype = ctypes.c_size_t
+        L.wsm_stream_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+        L.wsm_stream_status.restype = st
+        L.wsm_chain_create.argtypes = [ctypes.POINTER(_Task), i, ctypes.POINTER(_ChainOpts), ctypes.POINTER(vp)]
+        L.wsm_chain_create.restype = st
+        L.wsm_chain_run.argtypes = [vp, vp]
+        L.wsm_chain_run.restype = st
+        L.wsm_chain_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int)]
+        L.wsm_chain_status.restype = st
+        L.wsm_chain_trace.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_size_t]
+        L.wsm_chain_trace.restype = ctypes.c_size_t
+        L.wsm_chain_destroy.argtypes = [vp]
+        L.wsm_chain_destroy.restype = None
+        L.gemm_chain.argtypes = [ctypes.POINTER(_Task), i, vp]
+        L.gemm_chain.restype = st
+        L.wsm_chain_validate.argtypes = [ctypes.POINTER(_Task), i]
+        L.wsm_chain_validate.restype = st
+        L.wsm_last_error.argtypes = []
+        L.wsm_last_error.restype = ctypes.c_char_p
+        L.wsm_abi_version.argtypes = []
+        L.wsm_abi_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    return lib().wsm_last_error().decode()
+
+
+def abi_version() -> int:
+    return lib().wsm_abi_version()
+
+
+def _check(code: int, where: str):
+    if code != WSM_OK:
+        raise WsmError(code, where, last_error())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check_operand(name, t, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _opts(path=PATH_AUTO, m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32=None, workspace=None):
+    o = _Opts()
+    o.path, o.m_tile, o.order, o.l2_policy, o.grid = path, m_tile, order, l2_policy, grid
+    o.Yf32 = _ptr(yf32)
+    if workspace is not None:
+        o.workspace = workspace.data_ptr()
+        o.workspace_bytes = workspace.numel() * workspace.element_size()
+    return o
+
+
+def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = None, *, path=PATH_AUTO,
+                m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y = X @ W.T on the current (or given) stream; returns Y."""
+    _check_operand("x", x)
+    _check_operand("w", w)
+    if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[1]:
+        raise ValueError(f"shapes x{tuple(x.shape)} w{tuple(w.shape)} do not form X[M,K] . W[N,K]^T")
+    M, K = x.shape
+    N = w.shape[0]
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _check_operand("y", y)
+    if tuple(y.shape) != (M, N):
+        raise ValueError(f"y must be [{M}, {N}]")
+    if yf32 is not None:
+        _check_operand("yf32", yf32, torch.float32)
+        if tuple(yf32.shape) != (M, N):
+            raise ValueError(f"yf32 must be [{M}, {N}]")
+    plain = (path, m_tile, order, l2_policy, grid) == (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0) \
+        and yf32 is None and workspace is None
+    s = _stream_handle(stream)
+    if plain:
+        _check(lib().skinny_gemm(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, s), "skinny_gemm")
+    else:
+        o = _opts(path, m_tile, order, l2_policy, grid, yf32, workspace)
+        _check(lib().skinny_gemm_ex(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, ctypes.byref(o), s),
+               "skinny_gemm_ex")
+    return y
+
+
+def plan(M: int, N: int, K: int, num_sms: int = 148, **opts) -> dict:
+    """The plan for a shape (pure host computation; no GPU needed)."""
+    o = _opts(**opts)
+    info = _PlanInfo()
+    _check(lib().wsm_plan(M, N, K, num_sms, ctypes.byref(o), ctypes.byref(info)), "wsm_plan")
+    return {f: getattr(info, f) for f, _ in _PlanInfo._fields_}
+
+
+def workspace_bytes(M: int, N: int, K: int, **opts) -> int:
+    o = _opts(**opts)
+    n = lib().wsm_workspace_bytes(M, N, K, ctypes.byref(o))
+    if n == 0:
+        raise WsmError(WSM_ERR_INVALID, "wsm_workspace_bytes", last_error())
+    return n
+
+
+def stream_status(stream=None) -> int:
+    """Synchronise the stream; 0, or WSM_ERR_TIMEOUT if a pipeline wait ran out."""
+    code = ctypes.c_int(0)
+    lib().wsm_stream_status(_stream_handle(stream), ctypes.byref(code))
+    return code.value
+
+
+@dataclass
+class Task:
+    x: torch.Tensor
+    w: torch.Tensor
+    y: torch.Tensor
+    dep: int = -1
+    yf32: Optional[torch.Tensor] = None
+
+
+def _tasks_array(tasks: Sequence[Task]):
+    arr = (_Task * len(tasks))()
+    for i, t in enumerate(tasks):
+        M, K = t.x.shape
+        N = t.w.shape[0]
+        arr[i].X, arr[i].W, arr[i].Y = t.x.data_ptr(), t.w.data_ptr(), t.y.data_ptr()
+        arr[i].M, arr[i].N, arr[i].K, arr[i].dep = M, N, K, t.dep
+        arr[i].Yf32 = _ptr(t.yf32)
+    return arr
+
+
+def chain_validate(tasks) -> None:
+    """Host-side validation of a raw task list: sequence of dicts with keys
+    X, W, Y (integer addresses), M, N, K, dep."""
+    arr = (_Task * len(tasks))()
+    for i, t in enumerate(tasks):
+        arr[i].X, arr[i].W, arr[i].Y = t["X"], t["W"], t["Y"]
+        arr[i].M, arr[i].N, arr[i].K, arr[i].dep = t["M"], t["N"], t["K"], t.get("dep", -1)
+        arr[i].Yf32 = t.get("Yf32")
+    _check(lib().wsm_chain_validate(arr, len(tasks)), "wsm_chain_validate")
+
+
+class Chain:
+    """A prepared chain of GEMMs run as one persistent kernel."""
+
+    def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
+                 debug_unmet_dependency=False):
+        for i, t in enumerate(tasks):
+            _check_operand(f"tasks[{i}].x", t.x)
+            _check_operand(f"tasks[{i}].w", t.w)
+            _check_operand(f"tasks[{i}].y", t.y)
+        self.tasks = list(tasks)  # keeps the tensors alive
+        arr = _tasks_array(self.tasks)
+        o = _ChainOpts()
+        o.path, o.grid, o.timeout_ns, o.trace = path, grid, timeout_ns, 1 if trace else 0
+        o.debug_unmet_dependency = 1 if debug_unmet_dependency else 0
+        h = ctypes.c_void_p()
+        _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
+        self._h = h
+
+    def run(self, stream=None):
+        _check(lib().wsm_chain_run(self._h, _stream_handle(stream)), "wsm_chain_run")
+
+    def status(self, stream=None):
+        """Synchronise; returns (code, failed_task)."""
+        ft = ctypes.c_int(-1)
+        code = lib().wsm_chain_status(self._h, _stream_handle(stream), ctypes.byref(ft))
+        return code, ft.value
+
+    def trace(self, stream=None):
+        """Per-CTA, per-task %globaltimer stamps [grid, n_tasks, 3] (uint64), or None."""
+        n = lib().wsm_chain_trace(self._h, _stream_handle(stream), None, 0)
+        if n == 0:
+            return None
+        buf = (ctypes.c_ulonglong * n)()
+        lib().wsm_chain_trace(self._h, _stream_handle(stream), buf, n)
+        t = torch.tensor(list(buf), dtype=torch.int64)
+        return t.view(-1, len(self.tasks), 3)
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib().wsm_chain_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def gemm_chain(tasks: Sequence[Task], stream=None):
+    """One-shot chain run (prepared chains are cached by the library)."""
+    arr = _tasks_array(tasks)
+    _check(lib().gemm_chain(arr, len(tasks), _stream_handle(stream)), "gemm_chain")

@@ -1,0 +1,768 @@
+// wsm_api.cu -- host runtime and C ABI of libwsm (declared in include/wsm.h).
+//
+// Responsibilities: argument checks (before anything is queued), the plan
+// (kernel path, tile geometry, ring depth, L2 policy), TMA tensor maps, the
+// per-(device, stream) scratch workspace, chain preparation (device task
+// table, per-task partial slots and readiness counters) and kernel launches.
+#include "wsm_internal.cuh"
+#include "../../include/wsm.h"
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <string>
+#include <vector>
+
+namespace wsm {
+
+__global__ void wsm_umma_kernel(const __grid_constant__ KParams p);
+const void *stream_kernel_ptr(int mmax);  // wsm_stream.cu
+
+namespace {
+
+thread_local std::string g_err;
+
+wsm_status fail(wsm_status code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+wsm_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(WSM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+#define WSM_CUDA(call)                                      \
+    do {                                                    \
+        cudaError_t e_ = (call);                            \
+        if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+    } while (0)
+
+std::mutex g_mu;
+
+// sm_100 opt-in limit of dynamic + static shared memory per block.
+constexpr int kSmemOptin = 232448;
+constexpr int kRingBudget = kSmemOptin - 8192;  // static shared memory + 1 KB alignment slack
+
+constexpr unsigned long long kDefaultDepTimeoutNs = 2000000000ull;
+constexpr unsigned long long kPipeTimeoutNs = 4000000000ull;
+
+// ------------------------------------------------------------------ geometry
+
+struct Geo {
+    int path = 0;
+    int mmax = 0;              // stream path register width (1, 2, 4, 8)
+    int rw = 0, rg = 0, kw = 0;
+    int tile_rows = 0;         // rows of W per tile
+    int tile_k = 0;            // K per stage
+    int t_m = 0, t_mpad = 0, n_mt = 1;
+    int n_g = 0, kb = 0;
+    int stage_bytes = 0, x_off = 0, stages = 0;
+    int slot_elems = 0;
+    int order = WSM_ORDER_M_MAJOR;
+    int l2 = WSM_L2_EVICT_FIRST;
+    int grid = 0;
+    int threads = 0;
+    long long iters() const { return (long long)n_g * n_mt * kb; }
+};
+
+int pow2ceil(int v) {
+    int p = 1;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+bool shape_ok(int M, int N, int K) { return M >= 1 && M <= 64 && N >= 1 && K >= 8 && (K % 8) == 0; }
+
+// Stream (FMA) geometry per register width; see wsm_stream.cu.
+void stream_geo(int mmax, Geo &g) {
+    g.mmax = mmax;
+    if (mmax <= 2) {
+        g.rw = 4; g.rg = 4; g.kw = 2;
+    } else {
+        g.rw = 8; g.rg = 2; g.kw = 4;
+    }
+    g.tile_rows = g.rg * g.rw;                 // 16
+    g.tile_k = g.kw * kStreamBoxK;             // 512 or 1024
+    g.x_off = g.kw * g.tile_rows * 512;        // W part of a stage
+    g.stage_bytes = g.x_off + g.kw * mmax * 512;
+    g.slot_elems = g.tile_rows * mmax;
+    g.threads = 32 * (1 + g.rg * g.kw);
+}
+
+wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g) {
+    if (!shape_ok(M, N, K))
+        return fail(WSM_ERR_UNSUPPORTED, "unsupported shape M=%d N=%d K=%d (need 1<=M<=64, N>=1, K>=8, K%%8==0)", M,
+                    N, K);
+    if (num_sms < 1) return fail(WSM_ERR_INVALID, "num_sms must be positive");
+    wsm_opts z{};
+    if (!o) o = &z;
+    int path = o->path;
+    if (path < 0 || path > WSM_PATH_UMMA) return fail(WSM_ERR_INVALID, "bad path %d", path);
+    if (o->order < 0 || o->order > WSM_ORDER_NAIVE) return fail(WSM_ERR_INVALID, "bad order %d", o->order);
+    if (o->l2_policy < 0 || o->l2_policy > WSM_L2_NORMAL) return fail(WSM_ERR_INVALID, "bad l2_policy %d", o->l2_policy);
+    if (o->grid < 0) return fail(WSM_ERR_INVALID, "bad grid %d", o->grid);
+    if (path == WSM_PATH_AUTO) path = (M <= 8) ? WSM_PATH_STREAM : WSM_PATH_UMMA;
+    g = Geo{};
+    g.path = path;
+    g.grid = (o->grid > 0) ? std::min(o->grid, num_sms) : num_sms;
+    g.order = (o->order == WSM_ORDER_NAIVE) ? WSM_ORDER_NAIVE : WSM_ORDER_M_MAJOR;
+    if (path == WSM_PATH_STREAM) {
+        if (M > 8) return fail(WSM_ERR_UNSUPPORTED, "the FMA path takes M <= 8 (M=%d)", M);
+        if (o->m_tile != 0 && o->m_tile != M) return fail(WSM_ERR_UNSUPPORTED, "the FMA path has no M-tiling");
+        stream_geo(pow2ceil(M), g);
+        g.t_m = M;
+        g.t_mpad = M;
+        g.n_mt = 1;
+        g.n_g = (N + g.tile_rows - 1) / g.tile_rows;
+        g.kb = (K + g.tile_k - 1) / g.tile_k;
+    } else {
+        int tm = o->m_tile;
+        if (tm == 0) {
+            g.t_m = M;
+            g.t_mpad = (M + 15) / 16 * 16;
+        } else {
+            if (tm % 16 != 0 || tm < 16 || tm > kUmmaMaxN)
+                return fail(WSM_ERR_UNSUPPORTED, "m_tile must be a multiple of 16 in [16, 64] (got %d)", tm);
+            g.t_m = std::min(tm, M);
+            g.t_mpad = (g.t_m + 15) / 16 * 16;
+        }
+        g.n_mt = (M + g.t_m - 1) / g.t_m;
+        g.tile_rows = kUmmaRows;
+        g.tile_k = kUmmaBK;
+        g.n_g = (N + kUmmaRows - 1) / kUmmaRows;
+        g.kb = (K + kUmmaBK - 1) / kUmmaBK;
+        g.x_off = kUmmaRows * kUmmaBK * 2;                 // 16 KB of W
+        g.stage_bytes = g.x_off + g.t_mpad * kUmmaBK * 2;  // + X rows x 128 B (multiple of 1024)
+        g.slot_elems = kUmmaRows * g.t_mpad;
+        g.threads = 192;
+    }
+    g.stages = std::min(kMaxStages, kRingBudget / g.stage_bytes);
+    // no more CTAs than stages: every CTA then has work
+    if ((long long)g.grid > g.iters()) g.grid = (int)g.iters();
+    if (g.l2 = o->l2_policy, g.l2 == WSM_L2_AUTO) g.l2 = (g.n_mt > 1) ? WSM_L2_NORMAL : WSM_L2_EVICT_FIRST;
+    return WSM_OK;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace of one GEMM: [status 256 B][tile counters][partial slots].
+struct WsLayout {
+    size_t status_off = 0, cnt_off = 0, part_off = 0, total = 0;
+};
+WsLayout ws_layout(const Geo &g) {
+    WsLayout L;
+    L.status_off = 0;
+    L.cnt_off = 256;
+    const size_t n_tiles = (size_t)g.n_g * g.n_mt;
+    L.part_off = round_up(L.cnt_off + n_tiles * 4, 256);
+    L.total = round_up(L.part_off + (size_t)2 * g.grid * g.slot_elems * 4, 256);
+    return L;
+}
+
+void fill_plan_info(const Geo &g, wsm_plan_info *out) {
+    out->path = g.path;
+    out->grid = g.grid;
+    out->tile_rows = g.tile_rows;
+    out->tile_k = g.tile_k;
+    out->m_tile = g.t_mpad;
+    out->m_tiles = g.n_mt;
+    out->n_tiles = g.n_g;
+    out->k_iters = g.kb;
+    out->stages = g.stages;
+    out->order = g.order;
+    out->l2_policy = g.l2;
+    out->smem_bytes = g.stages * g.stage_bytes + 1024;
+    out->iters = g.iters();
+    out->workspace_bytes = ws_layout(g).total;
+}
+
+// ------------------------------------------------------------------ device state
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn g_encode = nullptr;
+
+wsm_status get_encode(EncodeTiledFn *fn) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+            return fail(WSM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+        g_encode = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    *fn = g_encode;
+    return WSM_OK;
+}
+
+struct DevInfo {
+    int sms = 0;
+    int smem_optin = 0;
+    bool attr_set[8] = {};
+};
+std::map<int, DevInfo> g_dev;
+
+wsm_status dev_info(int dev, DevInfo **out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_dev.find(dev);
+    if (it == g_dev.end()) {
+        DevInfo d;
+        WSM_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+        WSM_CUDA(cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+        int major = 0, minor = 0;
+        WSM_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+        WSM_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+        if (major != 10 || minor != 0)
+            return fail(WSM_ERR_UNSUPPORTED, "libwsm is built for sm_100a (B200); device %d is sm_%d%d", dev, major,
+                        minor);
+        it = g_dev.emplace(dev, d).first;
+    }
+    *out = &it->second;
+    return WSM_OK;
+}
+
+// Kernel for a geometry, and its slot in DevInfo::attr_set.
+const void *kernel_for(const Geo &g, int *slot) {
+    if (g.path == WSM_PATH_UMMA) {
+        *slot = 0;
+        return reinterpret_cast<const void *>(&wsm_umma_kernel);
+    }
+    *slot = g.mmax == 1 ? 1 : g.mmax == 2 ? 2 : g.mmax == 4 ? 3 : 4;
+    return stream_kernel_ptr(g.mmax);
+}
+
+wsm_status prepare_kernel(DevInfo *d, const Geo &g, const void **fn) {
+    int slot = 0;
+    *fn = kernel_for(g, &slot);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!d->attr_set[slot]) {
+        WSM_CUDA(cudaFuncSetAttribute(*fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingBudget + 1024));
+        d->attr_set[slot] = true;
+    }
+    return WSM_OK;
+}
+
+wsm_status encode_2d(CUtensorMap *map, const void *base, int rows, int cols, int box_cols, int box_rows,
+                     CUtensorMapSwizzle swz) {
+    EncodeTiledFn enc;
+    wsm_status st = get_encode(&enc);
+    if (st != WSM_OK) return st;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(WSM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for [%d x %d] box [%d x %d]", (int)r, rows, cols,
+                    box_rows, box_cols);
+    return WSM_OK;
+}
+
+uint32_t umma_idesc(int n) {
+    uint32_t d = 0;
+    d |= 1u << 4;                          // D format: f32
+    d |= 1u << 7;                          // A format: bf16
+    d |= 1u << 10;                         // B format: bf16
+    // bits 15/16 = 0: A and B K-major
+    d |= (uint32_t)(n >> 3) << 17;         // N / 8
+    d |= (uint32_t)(kUmmaRows >> 4) << 24; // M / 16
+    return d;
+}
+
+// Fill a TaskDev for (X, W, Y) under geometry g.
+wsm_status fill_task(TaskDev &T, const Geo &g, const void *X, const void *W, void *Y, float *Yf32, int M, int N,
+                     int K) {
+    memset(&T, 0, sizeof T);
+    wsm_status st;
+    if (g.path == WSM_PATH_UMMA) {
+        if ((st = encode_2d(&T.tmW, W, N, K, kUmmaBK, kUmmaRows, CU_TENSOR_MAP_SWIZZLE_128B)) != WSM_OK) return st;
+        if ((st = encode_2d(&T.tmX, X, M, K, kUmmaBK, g.t_mpad, CU_TENSOR_MAP_SWIZZLE_128B)) != WSM_OK) return st;
+        T.tx_bytes = (uint32_t)(kUmmaRows * kUmmaBK * 2 + g.t_mpad * kUmmaBK * 2);
+        T.idesc = umma_idesc(g.t_mpad);
+    } else {
+        if ((st = encode_2d(&T.tmW, W, N, K, kStreamBoxK, g.tile_rows, CU_TENSOR_MAP_SWIZZLE_NONE)) != WSM_OK)
+            return st;
+        if ((st = encode_2d(&T.tmX, X, M, K, kStreamBoxK, M, CU_TENSOR_MAP_SWIZZLE_NONE)) != WSM_OK) return st;
+        T.tx_bytes = (uint32_t)(g.kw * (g.tile_rows * 512 + M * 512));
+    }
+    T.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
+    T.Yf32 = Yf32;
+    T.M = M;
+    T.N = N;
+    T.K = K;
+    T.dep = -1;
+    T.n_g = g.n_g;
+    T.n_mt = g.n_mt;
+    T.t_m = g.t_m;
+    T.t_mpad = g.t_mpad;
+    T.kb = g.kb;
+    T.order = (g.order == WSM_ORDER_NAIVE) ? 1 : 0;
+    T.notify = 0;
+    T.w_evict_first = (g.l2 == WSM_L2_EVICT_FIRST) ? 1 : 0;
+    T.slot_elems = g.slot_elems;
+    return WSM_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+wsm_status check_ptrs(const void *X, const void *W, const void *Y, const float *Yf32) {
+    if (!X || !W || !Y) return fail(WSM_ERR_INVALID, "X, W and Y must be non-null device pointers");
+    if (!aligned16(X) || !aligned16(W) || !aligned16(Y))
+        return fail(WSM_ERR_ALIGN, "X, W and Y must be 16-byte aligned");
+    if (Yf32 && (reinterpret_cast<uintptr_t>(Yf32) & 3u)) return fail(WSM_ERR_ALIGN, "Yf32 must be 4-byte aligned");
+    return WSM_OK;
+}
+
+// ------------------------------------------------------------------ per-stream workspace
+
+struct Workspace {
+    void *ptr = nullptr;
+    size_t bytes = 0;
+};
+std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
+
+wsm_status stream_workspace(int dev, cudaStream_t stream, size_t need, void **out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace &w = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
+    if (w.bytes >= need) {
+        *out = w.ptr;
+        return WSM_OK;
+    }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    WSM_CUDA(cudaStreamIsCapturing(stream, &cs));
+    if (cs != cudaStreamCaptureStatusNone)
+        return fail(WSM_ERR_NOMEM,
+                    "the stream's scratch workspace must grow to %zu bytes, which cannot happen during graph capture: "
+                    "run the same call once outside capture first",
+                    need);
+    size_t bytes = std::max(need, (size_t)1 << 20);
+    if (w.ptr) {
+        WSM_CUDA(cudaStreamSynchronize(stream));
+        WSM_CUDA(cudaFree(w.ptr));
+        w.ptr = nullptr;
+        w.bytes = 0;
+    }
+    void *p = nullptr;
+    cudaError_t e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) return fail(WSM_ERR_NOMEM, "cudaMalloc(%zu) for the workspace failed: %s", bytes, cudaGetErrorString(e));
+    WSM_CUDA(cudaMemsetAsync(p, 0, bytes, stream));
+    w.ptr = p;
+    w.bytes = bytes;
+    *out = p;
+    return WSM_OK;
+}
+
+wsm_status launch(const void *fn, const Geo &g, const KParams &kp, cudaStream_t stream, bool cooperative) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g.grid);
+    cfg.blockDim = dim3((unsigned)g.threads);
+    cfg.dynamicSmemBytes = (size_t)kp.stages * kp.stage_bytes + 1024;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    int na = 0;
+    if (cooperative) {
+        attr[na].id = cudaLaunchAttributeCooperative;
+        attr[na].val.cooperative = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    void *args[1] = {const_cast<KParams *>(&kp)};
+    WSM_CUDA(cudaLaunchKernelExC(&cfg, fn, args));
+    return WSM_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ chains
+
+}  // namespace wsm
+
+struct wsm_chain {
+    int device = 0;
+    int n = 0;
+    wsm::Geo geo;                      // ring geometry shared by all tasks
+    std::vector<wsm_task> tasks;
+    std::vector<wsm::TaskDev> host_table;
+    wsm::TaskDev *d_table = nullptr;
+    void *d_buf = nullptr;             // status + counters + partials
+    size_t buf_bytes = 0;
+    int *d_status = nullptr;
+    unsigned int *d_counters = nullptr;
+    size_t counter_bytes = 0;
+    unsigned long long *d_trace = nullptr;
+    size_t trace_elems = 0;
+    uint32_t epoch = 0;
+    bool needs_reset = false;
+    bool any_dep = false;
+    unsigned long long dep_timeout_ns = 0;
+    uint32_t dep_target_extra = 0;
+    const void *fn = nullptr;
+};
+
+namespace wsm {
+namespace {
+
+std::map<std::pair<int, std::string>, wsm_chain *> g_chain_cache;
+
+wsm_status validate_tasks(const wsm_task *tasks, int n) {
+    if (!tasks || n < 1) return fail(WSM_ERR_INVALID, "task list must be non-null with n_tasks >= 1");
+    for (int i = 0; i < n; ++i) {
+        const wsm_task &t = tasks[i];
+        if (!shape_ok(t.M, t.N, t.K))
+            return fail(WSM_ERR_UNSUPPORTED, "task %d: unsupported shape M=%d N=%d K=%d", i, t.M, t.N, t.K);
+        wsm_status st = check_ptrs(t.X, t.W, t.Y, t.Yf32);
+        if (st != WSM_OK) return fail(st, "task %d: %s", i, g_err.c_str());
+        if (t.dep < -1 || t.dep >= i)
+            return fail(WSM_ERR_INVALID, "task %d: dependency %d must be -1 or an earlier task", i, t.dep);
+    }
+    return WSM_OK;
+}
+
+}  // namespace
+}  // namespace wsm
+
+using namespace wsm;
+
+extern "C" {
+
+const char *wsm_last_error(void) { return g_err.c_str(); }
+
+int wsm_abi_version(void) { return WSM_ABI_VERSION; }
+
+wsm_status wsm_plan(int M, int N, int K, int num_sms, const wsm_opts *opts, wsm_plan_info *out) {
+    if (!out) return fail(WSM_ERR_INVALID, "out must be non-null");
+    Geo g;
+    wsm_status st = make_geo(M, N, K, num_sms, opts, g);
+    if (st != WSM_OK) return st;
+    fill_plan_info(g, out);
+    g_err.clear();
+    return WSM_OK;
+}
+
+size_t wsm_workspace_bytes(int M, int N, int K, const wsm_opts *opts) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        fail(WSM_ERR_CUDA, "no CUDA device");
+        return 0;
+    }
+    DevInfo *d;
+    if (dev_info(dev, &d) != WSM_OK) return 0;
+    Geo g;
+    if (make_geo(M, N, K, d->sms, opts, g) != WSM_OK) return 0;
+    return ws_layout(g).total;
+}
+
+wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, int K, const wsm_opts *opts,
+                          wsm_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    wsm_opts z{};
+    if (!opts) opts = &z;
+    wsm_status st = check_ptrs(X, W, Y, opts->Yf32);
+    if (st != WSM_OK) return st;
+    if (!shape_ok(M, N, K))
+        return fail(WSM_ERR_UNSUPPORTED, "unsupported shape M=%d N=%d K=%d (need 1<=M<=64, N>=1, K>=8, K%%8==0)", M,
+                    N, K);
+    int dev = 0;
+    WSM_CUDA(cudaGetDevice(&dev));
+    DevInfo *d;
+    if ((st = dev_info(dev, &d)) != WSM_OK) return st;
+    Geo g;
+    if ((st = make_geo(M, N, K, d->sms, opts, g)) != WSM_OK) return st;
+    const WsLayout L = ws_layout(g);
+    void *ws = nullptr;
+    if (opts->workspace) {
+        if (opts->workspace_bytes < L.total)
+            return fail(WSM_ERR_NOMEM, "caller workspace of %zu bytes is smaller than the %zu needed",
+                        opts->workspace_bytes, L.total);
+        if (!aligned16(opts->workspace)) return fail(WSM_ERR_ALIGN, "workspace must be 16-byte aligned");
+        ws = opts->workspace;
+    } else if ((st = stream_workspace(dev, stream, L.total, &ws)) != WSM_OK) {
+        return st;
+    }
+    KParams kp;
+    memset(&kp, 0, sizeof kp);
+    if ((st = fill_task(kp.single, g, X, W, Y, opts->Yf32, M, N, K)) != WSM_OK) return st;
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    kp.single.tile_cnt = reinterpret_cast<unsigned int *>(wsb + L.cnt_off);
+    kp.single.part = reinterpret_cast<float *>(wsb + L.part_off);
+    kp.tasks = nullptr;
+    kp.n_tasks = 1;
+    kp.stages = g.stages;
+    kp.stage_bytes = g.stage_bytes;
+    kp.x_off = g.x_off;
+    kp.epoch = 1;
+    kp.status = reinterpret_cast<int *>(wsb + L.status_off);
+    kp.dep_timeout_ns = kDefaultDepTimeoutNs;
+    kp.wait_timeout_ns = kPipeTimeoutNs;
+    kp.trace = nullptr;
+    const void *fn;
+    if ((st = prepare_kernel(d, g, &fn)) != WSM_OK) return st;
+    if ((st = launch(fn, g, kp, stream, false)) != WSM_OK) return st;
+    return WSM_OK;
+}
+
+wsm_status skinny_gemm(const void *X, const void *W, void *Y, int M, int N, int K, wsm_stream_t stream) {
+    return skinny_gemm_ex(X, W, Y, M, N, K, nullptr, stream);
+}
+
+wsm_status wsm_stream_status(wsm_stream_t stream_, int *code) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int dev = 0;
+    WSM_CUDA(cudaGetDevice(&dev));
+    void *ptr = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
+        if (it != g_ws.end()) ptr = it->second.ptr;
+    }
+    if (code) *code = 0;
+    if (!ptr) return WSM_OK;
+    WSM_CUDA(cudaStreamSynchronize(stream));
+    int h[kStatusWords] = {};
+    WSM_CUDA(cudaMemcpy(h, ptr, sizeof h, cudaMemcpyDeviceToHost));
+    if (code) *code = h[0];
+    if (h[0] != 0) {
+        WSM_CUDA(cudaMemset(ptr, 0, sizeof h));
+        return fail(WSM_ERR_TIMEOUT, "device-side wait ran out (task %d, cta %d, site %d)", h[1], h[2], h[3]);
+    }
+    return WSM_OK;
+}
+
+wsm_status wsm_chain_validate(const wsm_task *tasks, int n_tasks) {
+    wsm_status st = validate_tasks(tasks, n_tasks);
+    if (st == WSM_OK) g_err.clear();
+    return st;
+}
+
+wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *opts, wsm_chain **out) {
+    if (!out) return fail(WSM_ERR_INVALID, "out must be non-null");
+    *out = nullptr;
+    wsm_status st = validate_tasks(tasks, n);
+    if (st != WSM_OK) return st;
+    wsm_chain_opts zo{};
+    if (!opts) opts = &zo;
+    if (opts->path < 0 || opts->path > WSM_PATH_UMMA) return fail(WSM_ERR_INVALID, "bad chain path %d", opts->path);
+    int dev = 0;
+    WSM_CUDA(cudaGetDevice(&dev));
+    DevInfo *d;
+    if ((st = dev_info(dev, &d)) != WSM_OK) return st;
+    int maxM = 0;
+    for (int i = 0; i < n; ++i) maxM = std::max(maxM, tasks[i].M);
+    int path = opts->path == WSM_PATH_AUTO ? (maxM <= 8 ? WSM_PATH_STREAM : WSM_PATH_UMMA) : opts->path;
+    if (path == WSM_PATH_STREAM && maxM > 8) return fail(WSM_ERR_UNSUPPORTED, "the FMA path takes M <= 8 (max M=%d)", maxM);
+
+    std::unique_ptr<wsm_chain> ch(new wsm_chain());
+    ch->device = dev;
+    ch->n = n;
+    ch->tasks.assign(tasks, tasks + n);
+    ch->dep_timeout_ns = opts->timeout_ns ? opts->timeout_ns : kDefaultDepTimeoutNs;
+    ch->dep_target_extra = opts->debug_unmet_dependency ? 0x40000000u : 0u;
+
+    // per-task geometry; the ring is sized for the widest task
+    std::vector<Geo> geos(n);
+    wsm_opts to{};
+    to.path = path;
+    to.grid = opts->grid;
+    for (int i = 0; i < n; ++i) {
+        wsm_opts oi = to;
+        if (path == WSM_PATH_STREAM) oi.m_tile = 0;
+        if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, d->sms, &oi, geos[i])) != WSM_OK)
+            return fail(st, "task %d: %s", i, g_err.c_str());
+    }
+    Geo ring = geos[0];
+    if (path == WSM_PATH_STREAM) {
+        stream_geo(pow2ceil(maxM), ring);
+    } else {
+        int tmp = 16;
+        for (auto &g : geos) tmp = std::max(tmp, g.t_mpad);
+        ring.x_off = kUmmaRows * kUmmaBK * 2;
+        ring.stage_bytes = ring.x_off + tmp * kUmmaBK * 2;
+    }
+    ring.stages = std::min(kMaxStages, kRingBudget / ring.stage_bytes);
+    ch->geo = ring;
+
+    // scratch: status | counters (tile counters of all tasks, then done counters) | partials
+    std::vector<size_t> cnt_off(n), part_off(n);
+    size_t ncnt = 0;
+    for (int i = 0; i < n; ++i) {
+        cnt_off[i] = ncnt;
+        ncnt += (size_t)geos[i].n_g * geos[i].n_mt;
+    }
+    const size_t done_off = ncnt;
+    ncnt += n;
+    const size_t counters_at = 256;
+    ch->counter_bytes = round_up(ncnt * 4, 256);
+    size_t part_at = counters_at + ch->counter_bytes;
+    for (int i = 0; i < n; ++i) {
+        part_off[i] = part_at;
+        part_at += round_up((size_t)2 * ring.grid * geos[i].slot_elems * 4, 256);
+    }
+    ch->buf_bytes = part_at;
+    cudaError_t e = cudaMalloc(&ch->d_buf, ch->buf_bytes);
+    if (e != cudaSuccess) return fail(WSM_ERR_NOMEM, "cudaMalloc(%zu) for chain scratch failed", ch->buf_bytes);
+    e = cudaMalloc(reinterpret_cast<void **>(&ch->d_table), sizeof(TaskDev) * n);
+    if (e != cudaSuccess) {
+        cudaFree(ch->d_buf);
+        return fail(WSM_ERR_NOMEM, "cudaMalloc for the task table failed");
+    }
+    auto cleanup = [&]() {
+        cudaFree(ch->d_buf);
+        cudaFree(ch->d_table);
+        if (ch->d_trace) cudaFree(ch->d_trace);
+    };
+    uint8_t *base = static_cast<uint8_t *>(ch->d_buf);
+    ch->d_status = reinterpret_cast<int *>(base);
+    ch->d_counters = reinterpret_cast<unsigned int *>(base + counters_at);
+    e = cudaMemset(ch->d_buf, 0, ch->buf_bytes);
+    if (e != cudaSuccess) {
+        cleanup();
+        return cuda_fail(e, "cudaMemset(chain scratch)");
+    }
+    std::vector<char> depended(n, 0);
+    for (int i = 0; i < n; ++i)
+        if (tasks[i].dep >= 0) depended[tasks[i].dep] = 1, ch->any_dep = true;
+    ch->host_table.resize(n);
+    for (int i = 0; i < n; ++i) {
+        TaskDev &T = ch->host_table[i];
+        Geo gi = geos[i];
+        if ((st = fill_task(T, gi, tasks[i].X, tasks[i].W, tasks[i].Y, tasks[i].Yf32, tasks[i].M, tasks[i].N,
+                            tasks[i].K)) != WSM_OK) {
+            cleanup();
+            return fail(st, "task %d: %s", i, g_err.c_str());
+        }
+        T.dep = tasks[i].dep;
+        T.tile_cnt = ch->d_counters + cnt_off[i];
+        T.done = ch->d_counters + done_off + i;
+        T.notify = depended[i];
+        T.part = reinterpret_cast<float *>(base + part_off[i]);
+    }
+    e = cudaMemcpy(ch->d_table, ch->host_table.data(), sizeof(TaskDev) * n, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cleanup();
+        return cuda_fail(e, "cudaMemcpy(task table)");
+    }
+    if (opts->trace) {
+        ch->trace_elems = (size_t)ring.grid * n * 3;
+        e = cudaMalloc(reinterpret_cast<void **>(&ch->d_trace), ch->trace_elems * 8);
+        if (e != cudaSuccess) {
+            cleanup();
+            return fail(WSM_ERR_NOMEM, "cudaMalloc for the trace failed");
+        }
+        cudaMemset(ch->d_trace, 0, ch->trace_elems * 8);
+    }
+    if ((st = prepare_kernel(d, ring, &ch->fn)) != WSM_OK) {
+        cleanup();
+        return st;
+    }
+    *out = ch.release();
+    g_err.clear();
+    return WSM_OK;
+}
+
+wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
+    if (!ch) return fail(WSM_ERR_INVALID, "chain is null");
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int dev = 0;
+    WSM_CUDA(cudaGetDevice(&dev));
+    if (dev != ch->device) return fail(WSM_ERR_INVALID, "chain was prepared on device %d, current is %d", ch->device, dev);
+    if (ch->needs_reset) {
+        WSM_CUDA(cudaMemsetAsync(ch->d_counters, 0, ch->counter_bytes, stream));
+        ch->epoch = 0;
+        ch->needs_reset = false;
+    }
+    if (ch->d_trace) WSM_CUDA(cudaMemsetAsync(ch->d_trace, 0, ch->trace_elems * 8, stream));
+    ch->epoch += 1;
+    KParams kp;
+    memset(&kp, 0, sizeof kp);
+    kp.tasks = ch->d_table;
+    kp.n_tasks = ch->n;
+    kp.stages = ch->geo.stages;
+    kp.stage_bytes = ch->geo.stage_bytes;
+    kp.x_off = ch->geo.x_off;
+    kp.epoch = ch->epoch;
+    kp.dep_target_extra = ch->dep_target_extra;
+    kp.status = ch->d_status;
+    kp.dep_timeout_ns = ch->dep_timeout_ns;
+    kp.wait_timeout_ns = ch->dep_timeout_ns + kPipeTimeoutNs;
+    kp.trace = ch->d_trace;
+    return launch(ch->fn, ch->geo, kp, stream, ch->any_dep);
+}
+
+wsm_status wsm_chain_status(wsm_chain *ch, wsm_stream_t stream_, int *failed_task) {
+    if (!ch) return fail(WSM_ERR_INVALID, "chain is null");
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    WSM_CUDA(cudaStreamSynchronize(stream));
+    int h[kStatusWords] = {};
+    WSM_CUDA(cudaMemcpy(h, ch->d_status, sizeof h, cudaMemcpyDeviceToHost));
+    if (failed_task) *failed_task = -1;
+    if (h[0] == 0) return WSM_OK;
+    if (failed_task) *failed_task = h[1];
+    WSM_CUDA(cudaMemset(ch->d_status, 0, sizeof h));
+    ch->needs_reset = true;
+    return fail(WSM_ERR_TIMEOUT, "chain wait ran out at task %d (cta %d, site %d)", h[1], h[2], h[3]);
+}
+
+size_t wsm_chain_trace(wsm_chain *ch, wsm_stream_t stream_, unsigned long long *out, size_t capacity) {
+    if (!ch || !ch->d_trace) return 0;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return 0;
+    if (out && capacity >= ch->trace_elems) {
+        if (cudaMemcpy(out, ch->d_trace, ch->trace_elems * 8, cudaMemcpyDeviceToHost) != cudaSuccess) return 0;
+    }
+    return ch->trace_elems;
+}
+
+void wsm_chain_destroy(wsm_chain *ch) {
+    if (!ch) return;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(ch->device);
+    cudaDeviceSynchronize();
+    cudaFree(ch->d_buf);
+    cudaFree(ch->d_table);
+    if (ch->d_trace) cudaFree(ch->d_trace);
+    cudaSetDevice(prev);
+    delete ch;
+}
+
+wsm_status gemm_chain(const wsm_task *tasks, int n_tasks, wsm_stream_t stream) {
+    wsm_status st = validate_tasks(tasks, n_tasks);
+    if (st != WSM_OK) return st;
+    int dev = 0;
+    WSM_CUDA(cudaGetDevice(&dev));
+    std::string key(reinterpret_cast<const char *>(tasks), sizeof(wsm_task) * (size_t)n_tasks);
+    wsm_chain *ch = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_chain_cache.find({dev, key});
+        if (it != g_chain_cache.end()) ch = it->second;
+    }
+    if (!ch) {
+        if ((st = wsm_chain_create(tasks, n_tasks, nullptr, &ch)) != WSM_OK) return st;
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_chain_cache.size() >= 16) {
+            // bounded cache: drop everything (rare; prepared chains are cheap to rebuild)
+            for (auto &kv : g_chain_cache) wsm_chain_destroy(kv.second);
+            g_chain_cache.clear();
+        }
+        g_chain_cache[{dev, key}] = ch;
+    }
+    return wsm_chain_run(ch, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,376 @@
+// wsm_stream.cu -- weight-streaming decode GEMM for M <= 8 on the fp32 FMA
+// pipes: the weight stream lands in shared memory through TMA and each output
+// is a dot product finished by a warp-shuffle reduction.  Persistent, one CTA
+// per SM; same stream-K split, partials and chain readiness as the tcgen05
+// path (wsm_internal.cuh).
+//
+// The three techniques of the FlyDSL article ("AMD: ROCm Low-Latency-GEMM-
+// Kernel ... MI355X"), as they land on B200:
+//   1. inter-CTA split-K      -> the stream-K split over persistent CTAs;
+//   2. intra-CTA K-slicing    -> KW consumer warps own disjoint 256-wide K
+//                                slices of every stage, lanes own 8-wide
+//                                pieces; slices are summed once per tile;
+//   3. multi-stage LDS pipe   -> a ring of TMA stages with mbarriers, filled
+//                                by one producer warp while 8 warps compute.
+//
+// Stage layout (one pipeline stage = T_N rows of W x T_K columns, plus the
+// matching X slice): KW boxes of W [T_N][256] then KW boxes of X [MMAX][256],
+// bf16, 512-byte rows.  A lane reads 16 bytes per row, so each LDS.128 of a
+// warp covers 512 contiguous bytes (no bank conflicts).
+//
+// Consumer warp (kw, rg): K slice kw, rows rg*RW .. rg*RW+RW-1.  Per stage a
+// lane converts its 8 X values of every row m once and reuses them for RW
+// rows of W: RW*8*MMAX FMAs per RW+MMAX shared loads.
+#include "wsm_internal.cuh"
+
+namespace wsm {
+
+namespace {
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
+    // a bf16 value is the upper half of a binary32 value
+    f[0] = __uint_as_float(u.x << 16);
+    f[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(u.y << 16);
+    f[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    f[4] = __uint_as_float(u.z << 16);
+    f[5] = __uint_as_float(u.z & 0xFFFF0000u);
+    f[6] = __uint_as_float(u.w << 16);
+    f[7] = __uint_as_float(u.w & 0xFFFF0000u);
+}
+
+__device__ __forceinline__ const TaskDev &task_at(const KParams &p, int t) {
+    return p.tasks ? p.tasks[t] : p.single;
+}
+
+constexpr int kConsBar = 1;
+
+// Transposed butterfly reduction over the 32 lanes of V values per lane.
+// While more than one value is left, each step hands half of them to the
+// partner lane (the half the partner keeps) and adds the half it receives, so
+// the whole reduction costs about V shuffles instead of 5V.  On return each
+// lane holds `V >> h` sums (h = min(5, log2 V) halving steps) starting at
+// index base(lane); when V < 32 the lanes with equal halving bits hold equal
+// copies.
+template <int V>
+struct LaneReduce {
+    static constexpr int H = (V >= 32) ? 5 : (V >= 16 ? 4 : (V >= 8 ? 3 : (V >= 4 ? 2 : (V >= 2 ? 1 : 0))));
+    static constexpr int OUT = V >> H;
+
+    __device__ __forceinline__ static int run(float (&v)[V], int lane) {
+        int base = 0;
+        int cnt = V;
+#pragma unroll
+        for (int step = 0; step < 5; ++step) {
+            const int o = 16 >> step;
+            if (step < H) {
+                const int half = cnt >> 1;
+                const bool upper = (lane & o) != 0;
+#pragma unroll
+                for (int i = 0; i < V / 2; ++i) {
+                    if (i < half) {
+                        const float send = upper ? v[i] : v[i + half];
+                        const float keep = upper ? v[i + half] : v[i];
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+                        v[i] = keep + recv;
+                    }
+                }
+                if (upper) base += half;
+                cnt = half;
+            } else {
+                v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+            }
+        }
+        return base;
+    }
+};
+
+}  // namespace
+
+// MMAX: largest M handled (register arrays); RW rows per warp; RG row groups;
+// KW K-slices.  Consumer warps = RG*KW = 8; T_N = RG*RW; T_K = KW*256.
+template <int MMAX, int RW, int RG, int KW>
+__global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const __grid_constant__ KParams p) {
+    constexpr int NCW = RG * KW;
+    constexpr int NCT = NCW * 32;
+    constexpr int TN = RG * RW;
+    constexpr int V = RW * MMAX;
+    using LR = LaneReduce<V>;
+    static_assert(NCW == 8, "eight consumer warps");
+
+    extern __shared__ __align__(1024) uint8_t smem_dyn[];
+    __shared__ __align__(8) uint64_t full_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
+    __shared__ float red[2][RG][KW][V];
+    __shared__ volatile int abort_flag;
+    __shared__ int last_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = gridDim.x;
+    const int c = blockIdx.x;
+    const int S = p.stages;
+    uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], NCW);
+        }
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const unsigned long long wlim = p.wait_timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t pol_x = policy_evict_last();
+            int s = 0;
+            uint32_t ph = 0;
+            long long issued = 0;
+            bool aborted = false;
+            for (int t = 0; t < p.n_tasks && !aborted; ++t) {
+                const TaskDev &T = task_at(p, t);
+                const long long Tt = (long long)T.n_g * T.kb;
+                const long long lo = range_lo(Tt, c, G), hi = range_lo(Tt, c + 1, G);
+                if (lo >= hi) continue;
+                prefetch_tmap(&T.tmW);
+                prefetch_tmap(&T.tmX);
+                const uint64_t pol_w = T.w_evict_first ? policy_evict_first() : policy_evict_normal();
+                bool dep_ok = T.dep < 0;
+                int pend_s[kMaxStages], pend_k[kMaxStages];
+                int np = 0;
+                if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 0] = globaltimer();
+                auto flush = [&]() {
+                    wait_dependency(p, task_at(p, T.dep), t, p.status);
+                    if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
+                    for (int i = 0; i < np; ++i) {
+                        uint8_t *xs = ring + (size_t)pend_s[i] * p.stage_bytes + p.x_off;
+#pragma unroll
+                        for (int kw = 0; kw < KW; ++kw)
+                            tma_load_2d(xs + kw * MMAX * 512, &T.tmX, &full_bar[pend_s[i]],
+                                        pend_k[i] + kw * kStreamBoxK, 0, pol_x);
+                    }
+                    np = 0;
+                    dep_ok = true;
+                };
+                for (long long it = lo; it < hi; ++it) {
+                    const int g = (int)(it / T.kb);
+                    const int kk = (int)(it - (long long)g * T.kb);
+                    if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
+                    if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
+                        if (np > 0) flush();
+                        aborted = true;
+                        break;
+                    }
+                    uint8_t *st = ring + (size_t)s * p.stage_bytes;
+                    mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
+                    const int k0 = kk * (KW * kStreamBoxK);
+#pragma unroll
+                    for (int kw = 0; kw < KW; ++kw)
+                        tma_load_2d(st + kw * TN * 512, &T.tmW, &full_bar[s], k0 + kw * kStreamBoxK, g * TN, pol_w);
+                    if (dep_ok) {
+#pragma unroll
+                        for (int kw = 0; kw < KW; ++kw)
+                            tma_load_2d(st + p.x_off + kw * MMAX * 512, &T.tmX, &full_bar[s], k0 + kw * kStreamBoxK, 0,
+                                        pol_x);
+                    } else {
+                        pend_s[np] = s;
+                        pend_k[np] = k0;
+                        ++np;
+                    }
+                    ++issued;
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (np > 0) flush();
+                if (p.trace && T.dep < 0) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
+            }
+            // copies in flight must land before exit, abort or not
+            drain_issued(full_bar, S, issued, wlim, p.status);
+        }
+    } else {
+        // ------------------------------------------------------------ consumers
+        const int cw = warp - 1;
+        const int kw = cw % KW;
+        const int rg = cw / KW;
+        const int ctid = threadIdx.x - 32;
+        const bool leader = (ctid == 0);
+        int s = 0;
+        uint32_t ph = 0;
+        uint32_t seg = 0;
+        bool aborted = false;
+        for (int t = 0; t < p.n_tasks; ++t) {
+            const TaskDev &T = task_at(p, t);
+            const long long Tt = (long long)T.n_g * T.kb;
+            const long long lo = range_lo(Tt, c, G), hi = range_lo(Tt, c + 1, G);
+            const int M = T.M;
+            long long it = lo;
+            bool wrote_any = false;
+            while (it < hi) {
+                const int g = (int)(it / T.kb);
+                const long long tile_lo = (long long)g * T.kb, tile_hi = tile_lo + T.kb;
+                const long long seg_start = it;
+                const long long seg_end = tile_hi < hi ? tile_hi : hi;
+                float acc[RW][MMAX];
+#pragma unroll
+                for (int r = 0; r < RW; ++r)
+#pragma unroll
+                    for (int m = 0; m < MMAX; ++m) acc[r][m] = 0.f;
+                for (; it < seg_end; ++it) {
+                    if (!aborted &&
+                        !mbar_wait_bounded(&full_bar[s], ph, &abort_flag, wlim, p.status, t, kSiteFull))
+                        aborted = true;
+                    aborted = __any_sync(0xffffffffu, aborted);
+                    if (!aborted) {
+                        const uint8_t *st = ring + (size_t)s * p.stage_bytes;
+                        const uint8_t *xs = st + p.x_off + kw * MMAX * 512 + lane * 16;
+                        const uint8_t *ws = st + kw * TN * 512 + (rg * RW) * 512 + lane * 16;
+                        float xv[MMAX][8];
+#pragma unroll
+                        for (int m = 0; m < MMAX; ++m) {
+                            if (m < M) {
+                                const uint4 u = *reinterpret_cast<const uint4 *>(xs + m * 512);
+                                bf16x8_to_f32(u, xv[m]);
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) xv[m][j] = 0.f;
+                            }
+                        }
+#pragma unroll
+                        for (int r = 0; r < RW; ++r) {
+                            const uint4 u = *reinterpret_cast<const uint4 *>(ws + r * 512);
+                            float wf[8];
+                            bf16x8_to_f32(u, wf);
+#pragma unroll
+                            for (int m = 0; m < MMAX; ++m) {
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) acc[r][m] = fmaf(wf[j], xv[m][j], acc[r][m]);
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0 && !aborted) mbar_arrive(&empty_bar[s]);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                // ---- end of segment: lanes -> warps -> tile outputs
+                float v[V];
+#pragma unroll
+                for (int r = 0; r < RW; ++r)
+#pragma unroll
+                    for (int m = 0; m < MMAX; ++m) v[r * MMAX + m] = acc[r][m];
+                const int base = LR::run(v, lane);
+                const int rb = seg & 1;
+                ++seg;
+                constexpr int lane_mask = (V >= 32) ? 0 : (31 >> LR::H);
+                if ((lane & lane_mask) == 0) {
+#pragma unroll
+                    for (int i = 0; i < LR::OUT; ++i) red[rb][rg][kw][base + i] = v[i];
+                }
+                named_bar_sync(kConsBar, NCT);
+                // thread ctid < TN*MMAX owns output (row, m) of this tile
+                const int o_m = ctid / TN;
+                const int o_row = ctid - o_m * TN;
+                const bool owner = ctid < TN * MMAX;
+                float val = 0.f;
+                if (owner) {
+                    const int org = o_row / RW, orr = o_row - org * RW;
+#pragma unroll
+                    for (int k = 0; k < KW; ++k) {
+                        const float x = red[rb][org][k][orr * MMAX + o_m];
+                        val = (k == 0) ? x : val + x;
+                    }
+                }
+                const int n = g * TN + o_row;
+                const bool live = owner && o_m < M && n < T.N;
+                const bool full_tile = (seg_start == tile_lo) && (seg_end == tile_hi);
+                if (full_tile) {
+                    if (live && !aborted) {
+                        const size_t o = (size_t)o_m * T.N + n;
+                        T.Y[o] = __float2bfloat16_rn(val);
+                        if (T.Yf32) T.Yf32[o] = val;
+                    }
+                    if (T.notify) {
+                        named_bar_sync(kConsBar, NCT);
+                        if (leader && !aborted) {
+                            __threadfence();
+                            red_release_gpu_add(T.done, 1u);
+                        }
+                    }
+                } else {
+                    int c_first, c_last;
+                    const int n_c = tile_contributors(tile_lo, tile_hi, Tt, G, c_first, c_last);
+                    const int my_slot = partial_slot(c, seg_start, lo);
+                    if (owner && !aborted) T.part[(size_t)my_slot * T.slot_elems + ctid] = val;
+                    named_bar_sync(kConsBar, NCT);
+                    if (leader) {
+                        int last = 0;
+                        if (!aborted) {
+                            __threadfence();
+                            const unsigned int old = atom_add_acqrel_gpu(&T.tile_cnt[g], 1u);
+                            last = (old == (unsigned int)(n_c - 1)) ? 1 : 0;
+                        }
+                        last_flag = last;
+                    }
+                    named_bar_sync(kConsBar, NCT);
+                    if (last_flag) {
+                        __threadfence();
+                        if (owner) {
+                            float sum = 0.f;
+                            for (int cj = c_first, j = 0; cj <= c_last; ++cj) {
+                                if (!cta_has_work(Tt, cj, G)) continue;
+                                float x;
+                                if (cj == c) {
+                                    x = val;
+                                } else {
+                                    const long long lo_j = range_lo(Tt, cj, G);
+                                    const int sj = (cj == c_first && lo_j < tile_lo) ? 2 * cj + 1 : 2 * cj;
+                                    x = ld_cg_f32(T.part + (size_t)sj * T.slot_elems + ctid);
+                                }
+                                sum = (j == 0) ? x : sum + x;
+                                ++j;
+                            }
+                            if (live) {
+                                const size_t o = (size_t)o_m * T.N + n;
+                                T.Y[o] = __float2bfloat16_rn(sum);
+                                if (T.Yf32) T.Yf32[o] = sum;
+                            }
+                        }
+                        named_bar_sync(kConsBar, NCT);
+                        if (leader) {
+                            T.tile_cnt[g] = 0u;
+                            if (T.notify) {
+                                __threadfence();
+                                red_release_gpu_add(T.done, 1u);
+                            }
+                        }
+                    }
+                }
+                wrote_any = true;
+            }
+            if (p.trace && wrote_any && leader) p.trace[((size_t)c * p.n_tasks + t) * 3 + 2] = globaltimer();
+        }
+    }
+    __syncthreads();
+}
+
+// Kernel for a register width; geometry per MMAX (see the file comment),
+// T_N = 16 rows for all.  Must agree with stream_geo() in wsm_api.cu.
+const void *stream_kernel_ptr(int mmax) {
+    switch (mmax) {
+        case 1: return reinterpret_cast<const void *>(&wsm_stream_kernel<1, 4, 4, 2>);
+        case 2: return reinterpret_cast<const void *>(&wsm_stream_kernel<2, 4, 4, 2>);
+        case 4: return reinterpret_cast<const void *>(&wsm_stream_kernel<4, 8, 2, 4>);
+        case 8: return reinterpret_cast<const void *>(&wsm_stream_kernel<8, 8, 2, 4>);
+        default: return nullptr;
+    }
+}
+
+}  // namespace wsm
