@@ -67,9 +67,10 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
         : "memory");
 }
 
-// 32 lanes x 16 consecutive fp32 columns -> 16 registers per thread
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
+// 32 lanes x 16 consecutive fp32 columns -> 16 registers per thread.  The
+// registers are written asynchronously: nothing may read them before
+// tmem_ld_wait16() on the same array.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
@@ -77,11 +78,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr)
         : "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Wait for this thread's outstanding tcgen05.ld; the array is a read-write
+// operand so the compiler cannot touch it before the wait has executed.
+__device__ __forceinline__ void tmem_ld_wait16(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), Blackwell
@@ -310,16 +318,19 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 if (!aborted) {
                     tc_fence_after();
                     const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kUmmaMaxN);
+                    uint32_t r[kUmmaMaxN / 16][16];
 #pragma unroll
                     for (int c16 = 0; c16 < kUmmaMaxN / 16; ++c16) {
-                        if (c16 * 16 < T.t_mpad) {
-                            float v[16];
-                            tmem_ld16(taddr + (uint32_t)(c16 * 16), v);
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) acc[c16 * 16 + i] = v[i];
-                        }
+                        for (int i = 0; i < 16; ++i) r[c16][i] = 0u;
+                        if (c16 * 16 < T.t_mpad) tmem_ld16(taddr + (uint32_t)(c16 * 16), r[c16]);
                     }
-                    tmem_ld_wait();
+#pragma unroll
+                    for (int c16 = 0; c16 < kUmmaMaxN / 16; ++c16) tmem_ld_wait16(r[c16]);
+#pragma unroll
+                    for (int c16 = 0; c16 < kUmmaMaxN / 16; ++c16)
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) acc[c16 * 16 + i] = __uint_as_float(r[c16][i]);
                 }
                 tc_fence_before();
                 __syncwarp();
