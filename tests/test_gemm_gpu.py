@@ -233,3 +233,21 @@ def test_full_size_sampled(case):
     ns = rng.integers(0, case.N, 4096)
     ns[:64] = np.arange(case.N - 64, case.N)  # the ragged end of N
     check_sampled(x, w, y, yf, ms, ns, what=case.name)
+
+
+def test_workspace_reused_across_shapes():
+    """One scratch buffer (the stream's, then a caller's) serves shapes with
+    very different tile counts and partial sizes in turn: the counters of
+    one shape must never sit on another shape's partial sums."""
+    seq = [(64, 1000, 8192, wsm.PATH_UMMA), (1, 8192, 4096, wsm.PATH_STREAM), (48, 300, 12288, wsm.PATH_UMMA),
+           (2, 16384, 1024, wsm.PATH_STREAM), (8, 4096, 7168, wsm.PATH_STREAM), (64, 6000, 2048, wsm.PATH_UMMA)]
+    for M, N, K, path in seq:
+        x, w = synth.make_xw(M, N, K, seed=N)
+        y, yf = run(x, w, path=path)
+        check_full(x, w, y, yf, what=f"stream workspace M={M} N={N} K={K}")
+    need = max(wsm.workspace_bytes(M, N, K, path=path) for M, N, K, path in seq)
+    ws = torch.zeros(need // 4, dtype=torch.int32, device=DEV)
+    for M, N, K, path in seq:
+        x, w = synth.make_xw(M, N, K, seed=N + 1)
+        y, yf = run(x, w, path=path, workspace=ws)
+        check_full(x, w, y, yf, what=f"caller workspace M={M} N={N} K={K}")

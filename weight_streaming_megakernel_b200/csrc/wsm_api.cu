@@ -98,7 +98,8 @@ void stream_geo(int mmax, Geo &g) {
     g.threads = 32 * (1 + g.rg * g.kw);
 }
 
-wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g) {
+// force_mmax: a chain's FMA kernel has one register width for all tasks.
+wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g, int force_mmax = 0) {
     if (!shape_ok(M, N, K))
         return fail(WSM_ERR_UNSUPPORTED, "unsupported shape M=%d N=%d K=%d (need 1<=M<=64, N>=1, K>=8, K%%8==0)", M,
                     N, K);
@@ -118,7 +119,7 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g)
     if (path == WSM_PATH_STREAM) {
         if (M > 8) return fail(WSM_ERR_UNSUPPORTED, "the FMA path takes M <= 8 (M=%d)", M);
         if (o->m_tile != 0 && o->m_tile != M) return fail(WSM_ERR_UNSUPPORTED, "the FMA path has no M-tiling");
-        stream_geo(pow2ceil(M), g);
+        stream_geo(force_mmax ? force_mmax : pow2ceil(M), g);
         g.t_m = M;
         g.t_mpad = M;
         g.n_mt = 1;
@@ -154,18 +155,38 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g)
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Workspace of one GEMM: [status 256 B][tile counters][partial slots].
+// Scratch of one GEMM: [status 256 B][tile counters][partial slots].  Where
+// the counters end depends ONLY on the buffer's size (1/16 of it), never on
+// the shape: a buffer reused for calls of different shapes then never finds
+// one call's partial sums where another call expects zeroed counters.  Every
+// completed call leaves the counters it used at zero.
 struct WsLayout {
     size_t status_off = 0, cnt_off = 0, part_off = 0, total = 0;
 };
-WsLayout ws_layout(const Geo &g) {
+WsLayout ws_layout_of(size_t bytes) {
     WsLayout L;
     L.status_off = 0;
     L.cnt_off = 256;
-    const size_t n_tiles = (size_t)g.n_g * g.n_mt;
-    L.part_off = round_up(L.cnt_off + n_tiles * 4, 256);
-    L.total = round_up(L.part_off + (size_t)2 * g.grid * g.slot_elems * 4, 256);
+    const size_t rest = bytes > 256 ? bytes - 256 : 0;
+    L.part_off = 256 + (rest / 16) / 256 * 256;
+    L.total = bytes;
     return L;
+}
+bool ws_fits(const Geo &g, size_t bytes) {
+    if (bytes < 512) return false;
+    const WsLayout L = ws_layout_of(bytes);
+    const size_t n_tiles = (size_t)g.n_g * g.n_mt;
+    const size_t parts = (size_t)2 * g.grid * g.slot_elems * 4;
+    return L.cnt_off + n_tiles * 4 <= L.part_off && L.part_off + parts <= bytes;
+}
+size_t ws_required(const Geo &g) {
+    const size_t n_tiles = (size_t)g.n_g * g.n_mt;
+    const size_t parts = (size_t)2 * g.grid * g.slot_elems * 4;
+    // smallest multiple of 256 that fits, from a close lower bound upwards
+    size_t z = round_up(256 + std::max(16 * (n_tiles * 4 + 256), parts + parts / 15 + 16 * 256), 256);
+    while (!ws_fits(g, z)) z += 256;
+    while (z > 512 && ws_fits(g, z - 256)) z -= 256;
+    return z;
 }
 
 void fill_plan_info(const Geo &g, wsm_plan_info *out) {
@@ -182,7 +203,7 @@ void fill_plan_info(const Geo &g, wsm_plan_info *out) {
     out->l2_policy = g.l2;
     out->smem_bytes = g.stages * g.stage_bytes + 1024;
     out->iters = g.iters();
-    out->workspace_bytes = ws_layout(g).total;
+    out->workspace_bytes = ws_required(g);
 }
 
 // ------------------------------------------------------------------ device state
@@ -335,13 +356,15 @@ struct Workspace {
 };
 std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
 
-wsm_status stream_workspace(int dev, cudaStream_t stream, size_t need, void **out) {
+wsm_status stream_workspace(int dev, cudaStream_t stream, const Geo &g, void **out, size_t *out_bytes) {
     std::lock_guard<std::mutex> lk(g_mu);
     Workspace &w = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
-    if (w.bytes >= need) {
+    if (w.ptr && ws_fits(g, w.bytes)) {
         *out = w.ptr;
+        *out_bytes = w.bytes;
         return WSM_OK;
     }
+    const size_t need = std::max(ws_required(g), 2 * w.bytes);
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     WSM_CUDA(cudaStreamIsCapturing(stream, &cs));
     if (cs != cudaStreamCaptureStatusNone)
@@ -349,7 +372,7 @@ wsm_status stream_workspace(int dev, cudaStream_t stream, size_t need, void **ou
                     "the stream's scratch workspace must grow to %zu bytes, which cannot happen during graph capture: "
                     "run the same call once outside capture first",
                     need);
-    size_t bytes = std::max(need, (size_t)1 << 20);
+    size_t bytes = round_up(std::max(need, (size_t)1 << 20), 256);
     if (w.ptr) {
         WSM_CUDA(cudaStreamSynchronize(stream));
         WSM_CUDA(cudaFree(w.ptr));
@@ -363,6 +386,7 @@ wsm_status stream_workspace(int dev, cudaStream_t stream, size_t need, void **ou
     w.ptr = p;
     w.bytes = bytes;
     *out = p;
+    *out_bytes = bytes;
     return WSM_OK;
 }
 
@@ -464,7 +488,7 @@ size_t wsm_workspace_bytes(int M, int N, int K, const wsm_opts *opts) {
     if (dev_info(dev, &d) != WSM_OK) return 0;
     Geo g;
     if (make_geo(M, N, K, d->sms, opts, g) != WSM_OK) return 0;
-    return ws_layout(g).total;
+    return ws_required(g);
 }
 
 wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, int K, const wsm_opts *opts,
@@ -483,17 +507,19 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     if ((st = dev_info(dev, &d)) != WSM_OK) return st;
     Geo g;
     if ((st = make_geo(M, N, K, d->sms, opts, g)) != WSM_OK) return st;
-    const WsLayout L = ws_layout(g);
     void *ws = nullptr;
+    size_t ws_bytes = 0;
     if (opts->workspace) {
-        if (opts->workspace_bytes < L.total)
+        if (!ws_fits(g, opts->workspace_bytes))
             return fail(WSM_ERR_NOMEM, "caller workspace of %zu bytes is smaller than the %zu needed",
-                        opts->workspace_bytes, L.total);
+                        opts->workspace_bytes, ws_required(g));
         if (!aligned16(opts->workspace)) return fail(WSM_ERR_ALIGN, "workspace must be 16-byte aligned");
         ws = opts->workspace;
-    } else if ((st = stream_workspace(dev, stream, L.total, &ws)) != WSM_OK) {
+        ws_bytes = opts->workspace_bytes;
+    } else if ((st = stream_workspace(dev, stream, g, &ws, &ws_bytes)) != WSM_OK) {
         return st;
     }
+    const WsLayout L = ws_layout_of(ws_bytes);
     KParams kp;
     memset(&kp, 0, sizeof kp);
     if ((st = fill_task(kp.single, g, X, W, Y, opts->Yf32, M, N, K)) != WSM_OK) return st;
@@ -578,12 +604,14 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     wsm_opts to{};
     to.path = path;
     to.grid = opts->grid;
+    const int chain_mmax = (path == WSM_PATH_STREAM) ? pow2ceil(maxM) : 0;
     for (int i = 0; i < n; ++i) {
-        wsm_opts oi = to;
-        if (path == WSM_PATH_STREAM) oi.m_tile = 0;
-        if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, d->sms, &oi, geos[i])) != WSM_OK)
+        if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, d->sms, &to, geos[i], chain_mmax)) != WSM_OK)
             return fail(st, "task %d: %s", i, g_err.c_str());
     }
+    // one grid for the whole chain (make_geo clamps it per task to the task's stages)
+    int chain_grid = (opts->grid > 0) ? std::min(opts->grid, d->sms) : d->sms;
+    for (auto &g : geos) g.grid = chain_grid;
     Geo ring = geos[0];
     if (path == WSM_PATH_STREAM) {
         stream_geo(pow2ceil(maxM), ring);
