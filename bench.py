@@ -126,7 +126,8 @@ class ClockSampler:
         if not sm:
             return None
         sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm),
+                "window": "loaded window containing the timed region"}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -146,14 +147,21 @@ def setup_inputs(cases, dev, seed_base=0):
 
 
 def run_gpu(args, rank, world, local_rank):
+    """Timed region: K steps, each one replay of a CUDA graph holding every
+    GEMM launch of the step with an external timing event between launches
+    (so per-launch durations come from the same timed replays)."""
+    import ctypes
     import weight_streaming_megakernel_b200 as wsm
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     cases = workload_cases(args.workload)
+    if args.only:
+        cases = [c for c in cases if c.name in args.only.split(",")]
+        assert cases, f"no case named {args.only}"
     data = setup_inputs(cases, dev, seed_base=rank)
     L = wsm.lib()
-    stream = torch.cuda.current_stream(dev)
+    stream = torch.cuda.Stream(dev)
     s = stream.cuda_stream
     chain = None
 
@@ -162,61 +170,83 @@ def run_gpu(args, rank, world, local_rank):
         chain = wsm.Chain(tasks)
         launches_per_step = 1
 
-        def step(events=None):
-            if events is not None:
-                events[0].record(stream)
+        def launch(i):
             chain.run(s)
-            if events is not None:
-                events[1].record(stream)
     else:
         calls = []
         for c, x, w, y in data:
-            if c.m_tile:
-                o = wsm._opts(m_tile=c.m_tile)
-                calls.append((True, x.data_ptr(), w.data_ptr(), y.data_ptr(), c.M, c.N, c.K, o))
-            else:
-                calls.append((False, x.data_ptr(), w.data_ptr(), y.data_ptr(), c.M, c.N, c.K, None))
+            o = wsm._opts(m_tile=c.m_tile) if c.m_tile else None
+            calls.append((x.data_ptr(), w.data_ptr(), y.data_ptr(), c.M, c.N, c.K, o))
         launches_per_step = len(calls)
-        import ctypes
 
-        def step(events=None):
-            for i, (ex, xp, wp, yp, M, N, K, o) in enumerate(calls):
-                if events is not None:
-                    events[i].record(stream)
-                if ex:
-                    rc = L.skinny_gemm_ex(xp, wp, yp, M, N, K, ctypes.byref(o), s)
-                else:
-                    rc = L.skinny_gemm(xp, wp, yp, M, N, K, s)
-                if rc != 0:
-                    raise RuntimeError(f"skinny_gemm failed: {wsm.last_error()}")
+        def launch(i):
+            xp, wp, yp, M, N, K, o = calls[i]
+            rc = L.skinny_gemm_ex(xp, wp, yp, M, N, K, ctypes.byref(o), s) if o is not None else \
+                L.skinny_gemm(xp, wp, yp, M, N, K, s)
+            if rc != 0:
+                raise RuntimeError(f"skinny_gemm failed: {wsm.last_error()}")
+
+    def step(events=None):
+        for i in range(launches_per_step):
             if events is not None:
-                events[len(calls)].record(stream)
+                events[i].record(stream)
+            launch(i)
+        if events is not None:
+            events[launches_per_step].record(stream)
 
     total_bytes = sum(alg_bytes(c) for c in cases)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
+    # eager warm-up (also sizes the stream's scratch before any capture)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
 
-    # ---- timed region: K steps, events between launches
+    # one graph per timed step, each with its own in-graph timing events
     nev = launches_per_step + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nev)] for _ in range(args.steps)]
+    graphs = []
+    for k in range(args.steps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(evs[k])
+        graphs.append(g)
+    plain = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(plain, stream=stream):
+        step()
+    with torch.cuda.stream(stream):
+        for g in graphs[: min(3, len(graphs))]:
+            g.replay()
+    stream.synchronize()
+
+    # clocks: the sampler runs over a loaded window that contains the timed region
     clocks = ClockSampler(local_rank)
     clocks.start()
-    torch.cuda.synchronize(dev)
+    t_pre = time.time()
+    with torch.cuda.stream(stream):
+        while len(clocks.lines) < 2 and time.time() - t_pre < 3.0:
+            plain.replay()
+            stream.synchronize()
     if world > 1:
         torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for k in range(args.steps):
-        step(evs[k])
-    t_end.record(stream)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for g in graphs:
+            g.replay()
+        t_end.record(stream)
+    stream.synchronize()
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
+    # keep the load on briefly so the window closes under load
+    t_post = time.time()
+    with torch.cuda.stream(stream):
+        while time.time() - t_post < 0.3:
+            plain.replay()
+            stream.synchronize()
     clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
     if world > 1:
@@ -224,15 +254,23 @@ def run_gpu(args, rank, world, local_rank):
         torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(tt.item())
     ms_per_step = total_ms / args.steps
-
-    # per-launch durations (event to event, same stream)
     per_launch = [[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(launches_per_step)]
                   for k in range(args.steps)]
+
+    # uninstrumented graph, for reference (not the headline)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(args.steps):
+            plain.replay()
+        b.record(stream)
+    stream.synchronize()
+    plain_ms = a.elapsed_time(b) / args.steps
 
     # ---- e2e: public API, host buffers, H2D of X and D2H of Y inside the timed region
     e2e = None
     if not args.no_e2e:
-        import weight_streaming_megakernel_b200 as wsm2
         hx = [x.cpu().pin_memory() for (_, x, _, _) in data]
         hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for (_, _, _, y) in data]
         h2d = sum(t.numel() * 2 for t in hx)
@@ -245,22 +283,24 @@ def run_gpu(args, rank, world, local_rank):
                 chain.run(s)
             else:
                 for c, x, w, y in data:
-                    wsm2.skinny_gemm(x, w, y, m_tile=c.m_tile, stream=s)
+                    wsm.skinny_gemm(x, w, y, m_tile=c.m_tile, stream=s)
             for (c, x, w, y), h in zip(data, hy):
                 h.copy_(y, non_blocking=True)
 
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
-        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, args.warmup)):
+                e2e_step()
+        stream.synchronize()
         if world > 1:
             torch.distributed.barrier()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            for _ in range(args.steps):
+                e2e_step()
+            b.record(stream)
+        stream.synchronize()
         e_ms = a.elapsed_time(b)
         if world > 1:
             tt = torch.tensor([e_ms], device=dev)
@@ -272,8 +312,10 @@ def run_gpu(args, rank, world, local_rank):
     status = wsm.stream_status(stream) if chain is None else chain.status(s)[0]
     if status != 0:
         raise RuntimeError(f"device-side status {status}")
+    del graphs, plain
     return dict(cases=cases, total_bytes=total_bytes, ms_per_step=ms_per_step, per_launch=per_launch,
-                clocks=clk, e2e=e2e, launches_per_step=launches_per_step, chain=chain is not None)
+                clocks=clk, e2e=e2e, launches_per_step=launches_per_step, chain=chain is not None,
+                plain_ms=plain_ms)
 
 
 # ----------------------------------------------------------------------------- CPU arm
@@ -326,6 +368,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
+    ap.add_argument("--only", default="", help="comma-separated case names (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -335,6 +378,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     hbm_peak, peak_kind = peaks()
     cases = workload_cases(args.workload)
+    if args.only:
+        cases = [c for c in cases if c.name in args.only.split(",")]
     config = {"workload": {"qwen3_decode": "qwen3_8b_decode_gemms", "single": "single_gemm_m1_4096x4096",
                            "skinny": "skinny_k7168_k8192", "l2_reuse": "l2_reuse_m32_m64",
                            "chain": "chain_36x4_m16"}[args.workload],
@@ -420,6 +465,7 @@ def main():
                 "cpu_baseline": cpu,
                 "e2e": r["e2e"],
                 "gpu_launches": r["launches_per_step"] * args.steps,
+                "ms_per_step_without_timing_events": round(r["plain_ms"], 4),
                 "clocks": r["clocks"]}
         print(json.dumps(line))
     if world > 1:

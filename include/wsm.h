@@ -95,7 +95,8 @@ typedef struct {
     int l2_policy;   /* WSM_L2_* */
     int grid;        /* persistent CTAs, 0 = one per SM; values above the
                         number of SMs are clamped */
-    int reserved0;
+    int stage_k;     /* UMMA path: K elements per pipeline stage, 0 = auto,
+                        else 64, 128 or 256 */
     float *Yf32;     /* optional device [M, N] fp32: the result before rounding */
     void *workspace; /* optional caller scratch (device, >= wsm_workspace_bytes,
                         16-byte aligned, zero-filled before its first use; the

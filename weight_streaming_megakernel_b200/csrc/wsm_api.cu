@@ -71,6 +71,8 @@ struct Geo {
     int l2 = WSM_L2_EVICT_FIRST;
     int grid = 0;
     int threads = 0;
+    int kps = 1;               // UMMA: 64-wide K boxes per stage
+    int x_stride = 0;          // UMMA: bytes between X boxes inside a stage
     long long iters() const { return (long long)n_g * n_mt * kb; }
 };
 
@@ -118,6 +120,7 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
     g.order = (o->order == WSM_ORDER_NAIVE) ? WSM_ORDER_NAIVE : WSM_ORDER_M_MAJOR;
     if (path == WSM_PATH_STREAM) {
         if (M > 8) return fail(WSM_ERR_UNSUPPORTED, "the FMA path takes M <= 8 (M=%d)", M);
+        if (o->stage_k != 0) return fail(WSM_ERR_UNSUPPORTED, "stage_k applies to the UMMA path only");
         if (o->m_tile != 0 && o->m_tile != M) return fail(WSM_ERR_UNSUPPORTED, "the FMA path has no M-tiling");
         stream_geo(force_mmax ? force_mmax : pow2ceil(M), g);
         g.t_m = M;
@@ -137,12 +140,18 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
             g.t_mpad = (g.t_m + 15) / 16 * 16;
         }
         g.n_mt = (M + g.t_m - 1) / g.t_m;
+        int sk = o->stage_k;
+        if (sk == 0) sk = kUmmaBK;
+        if (sk != 64 && sk != 128 && sk != 256)
+            return fail(WSM_ERR_UNSUPPORTED, "stage_k must be 64, 128 or 256 on the UMMA path (got %d)", sk);
+        g.kps = sk / kUmmaBK;
         g.tile_rows = kUmmaRows;
-        g.tile_k = kUmmaBK;
+        g.tile_k = sk;
         g.n_g = (N + kUmmaRows - 1) / kUmmaRows;
-        g.kb = (K + kUmmaBK - 1) / kUmmaBK;
-        g.x_off = kUmmaRows * kUmmaBK * 2;                 // 16 KB of W
-        g.stage_bytes = g.x_off + g.t_mpad * kUmmaBK * 2;  // + X rows x 128 B (multiple of 1024)
+        g.kb = (K + g.tile_k - 1) / g.tile_k;
+        g.x_stride = g.t_mpad * kUmmaBK * 2;                        // X rows x 128 B (multiple of 1024)
+        g.x_off = g.kps * kUmmaRows * kUmmaBK * 2;                  // W boxes, 16 KB each
+        g.stage_bytes = g.x_off + g.kps * g.x_stride;
         g.slot_elems = kUmmaRows * g.t_mpad;
         g.threads = 192;
     }
@@ -312,7 +321,7 @@ wsm_status fill_task(TaskDev &T, const Geo &g, const void *X, const void *W, voi
     if (g.path == WSM_PATH_UMMA) {
         if ((st = encode_2d(&T.tmW, W, N, K, kUmmaBK, kUmmaRows, CU_TENSOR_MAP_SWIZZLE_128B)) != WSM_OK) return st;
         if ((st = encode_2d(&T.tmX, X, M, K, kUmmaBK, g.t_mpad, CU_TENSOR_MAP_SWIZZLE_128B)) != WSM_OK) return st;
-        T.tx_bytes = (uint32_t)(kUmmaRows * kUmmaBK * 2 + g.t_mpad * kUmmaBK * 2);
+        T.tx_bytes = (uint32_t)(g.kps * (kUmmaRows * kUmmaBK * 2 + g.t_mpad * kUmmaBK * 2));
         T.idesc = umma_idesc(g.t_mpad);
     } else {
         if ((st = encode_2d(&T.tmW, W, N, K, kStreamBoxK, g.tile_rows, CU_TENSOR_MAP_SWIZZLE_NONE)) != WSM_OK)
@@ -531,6 +540,8 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     kp.stages = g.stages;
     kp.stage_bytes = g.stage_bytes;
     kp.x_off = g.x_off;
+    kp.kps = g.kps;
+    kp.x_stride = g.x_stride;
     kp.epoch = 1;
     kp.status = reinterpret_cast<int *>(wsb + L.status_off);
     kp.dep_timeout_ns = kDefaultDepTimeoutNs;
@@ -618,8 +629,9 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     } else {
         int tmp = 16;
         for (auto &g : geos) tmp = std::max(tmp, g.t_mpad);
-        ring.x_off = kUmmaRows * kUmmaBK * 2;
-        ring.stage_bytes = ring.x_off + tmp * kUmmaBK * 2;
+        ring.x_stride = tmp * kUmmaBK * 2;
+        ring.x_off = ring.kps * kUmmaRows * kUmmaBK * 2;
+        ring.stage_bytes = ring.x_off + ring.kps * ring.x_stride;
     }
     ring.stages = std::min(kMaxStages, kRingBudget / ring.stage_bytes);
     ch->geo = ring;
@@ -722,6 +734,8 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     kp.stages = ch->geo.stages;
     kp.stage_bytes = ch->geo.stage_bytes;
     kp.x_off = ch->geo.x_off;
+    kp.kps = ch->geo.kps;
+    kp.x_stride = ch->geo.x_stride;
     kp.epoch = ch->epoch;
     kp.dep_target_extra = ch->dep_target_extra;
     kp.status = ch->d_status;

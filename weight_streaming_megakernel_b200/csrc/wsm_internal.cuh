@@ -68,6 +68,9 @@ struct KParams {
     int x_off;                      // offset of the X part inside a stage
     uint32_t epoch;                 // chain run number (>= 1)
     uint32_t dep_target_extra;      // 0; a test hook makes every dependency unreachable with it
+    int kps;                        // UMMA path: 64-wide K boxes per stage
+    int x_stride;                   // UMMA path: bytes between the X boxes of a stage
+    int pad2_[2];
     int *status;                    // kStatusWords ints
     unsigned long long dep_timeout_ns;
     unsigned long long wait_timeout_ns;
@@ -283,6 +286,28 @@ __device__ __forceinline__ void tile_coords(const TaskDev &T, int tile, int &g, 
         g = tile - mt * T.n_g;
     }
 }
+
+// Incremental walk over a CTA's iterations [lo, hi) in tile-major order:
+// (tile, k-stage kk, column tile g, M-tile mt) with no division per step.
+struct IterWalk {
+    int tile, kk, g, mt;
+    __device__ __forceinline__ void start(const TaskDev &T, long long lo) {
+        tile = (int)(lo / T.kb);
+        kk = (int)(lo - (long long)tile * T.kb);
+        tile_coords(T, tile, g, mt);
+    }
+    __device__ __forceinline__ void next(const TaskDev &T) {
+        if (++kk == T.kb) {
+            kk = 0;
+            ++tile;
+            if (T.order == 0) {
+                if (++mt == T.n_mt) { mt = 0; ++g; }
+            } else {
+                if (++g == T.n_g) { g = 0; ++mt; }
+            }
+        }
+    }
+};
 
 // Bounded wait for task `dep` of a chain to have finished all its tiles in
 // this run.  On time-out (or an error elsewhere) records it and returns; the

@@ -156,9 +156,10 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     np = 0;
                     dep_ok = true;
                 };
-                for (long long it = lo; it < hi; ++it) {
-                    const int g = (int)(it / T.kb);
-                    const int kk = (int)(it - (long long)g * T.kb);
+                IterWalk wk;
+                wk.start(T, lo);
+                for (long long it = lo; it < hi; ++it, wk.next(T)) {
+                    const int g = wk.g, kk = wk.kk;
                     if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
                     if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
                         if (np > 0) flush();
@@ -211,8 +212,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
             const int M = T.M;
             long long it = lo;
             bool wrote_any = false;
-            while (it < hi) {
-                const int g = (int)(it / T.kb);
+            for (int g = (int)(lo / T.kb); it < hi; ++g) {
                 const long long tile_lo = (long long)g * T.kb, tile_hi = tile_lo + T.kb;
                 const long long seg_start = it;
                 const long long seg_end = tile_hi < hi ? tile_hi : hi;

@@ -181,16 +181,16 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     wait_dependency(p, task_at(p, T.dep), t, p.status);
                     if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
                     for (int i = 0; i < np; ++i)
-                        tma_load_2d(ring + (size_t)pend_s[i] * p.stage_bytes + p.x_off, &T.tmX, &full_bar[pend_s[i]],
-                                    pend_k[i], pend_y[i], pol_x);
+                        for (int j = 0; j < p.kps; ++j)
+                            tma_load_2d(ring + (size_t)pend_s[i] * p.stage_bytes + p.x_off + j * p.x_stride, &T.tmX,
+                                        &full_bar[pend_s[i]], pend_k[i] + j * kUmmaBK, pend_y[i], pol_x);
                     np = 0;
                     dep_ok = true;
                 };
-                for (long long it = lo; it < hi; ++it) {
-                    const int tile = (int)(it / T.kb);
-                    const int kk = (int)(it - (long long)tile * T.kb);
-                    int g, mt;
-                    tile_coords(T, tile, g, mt);
+                IterWalk w;
+                w.start(T, lo);
+                for (long long it = lo; it < hi; ++it, w.next(T)) {
+                    const int kk = w.kk, g = w.g, mt = w.mt;
                     // W loads may run ahead of the dependency until the ring is full
                     if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
                     if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
@@ -200,13 +200,18 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     }
                     uint8_t *st = ring + (size_t)s * p.stage_bytes;
                     mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
-                    tma_load_2d(st, &T.tmW, &full_bar[s], kk * kUmmaBK, g * kUmmaRows, pol_w);
+                    const int k0 = kk * p.kps * kUmmaBK;
+                    for (int j = 0; j < p.kps; ++j)
+                        tma_load_2d(st + j * (kUmmaRows * kUmmaBK * 2), &T.tmW, &full_bar[s], k0 + j * kUmmaBK,
+                                    g * kUmmaRows, pol_w);
                     const int xy = mt * T.t_m;
                     if (dep_ok) {
-                        tma_load_2d(st + p.x_off, &T.tmX, &full_bar[s], kk * kUmmaBK, xy, pol_x);
+                        for (int j = 0; j < p.kps; ++j)
+                            tma_load_2d(st + p.x_off + j * p.x_stride, &T.tmX, &full_bar[s], k0 + j * kUmmaBK, xy,
+                                        pol_x);
                     } else {
                         pend_s[np] = s;
-                        pend_k[np] = kk * kUmmaBK;
+                        pend_k[np] = k0;
                         pend_y[np] = xy;
                         ++np;
                     }
@@ -238,8 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 const long long lo = range_lo(Tt, c, G), hi = range_lo(Tt, c + 1, G);
                 const uint32_t idesc = T.idesc;
                 long long it = lo;
-                while (it < hi && !aborted) {
-                    const int tile = (int)(it / T.kb);
+                int tile = (int)(lo / T.kb);
+                for (; it < hi && !aborted; ++tile) {
+                    const long long seg_start = it;
                     const long long seg_end = ((long long)tile + 1) * T.kb < hi ? ((long long)tile + 1) * T.kb : hi;
                     const int buf = seg & 1;
                     const uint32_t aph = (seg >> 1) & 1;
@@ -255,14 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t a0 = smem_u32(ring + (size_t)s * p.stage_bytes);
-                        const uint32_t b0 = a0 + (uint32_t)p.x_off;
-                        const bool first_stage = (it == ((long long)tile * T.kb > lo ? (long long)tile * T.kb : lo));
+                        const uint32_t st0 = smem_u32(ring + (size_t)s * p.stage_bytes);
+                        const bool first_stage = (it == seg_start);
+                        for (int j = 0; j < p.kps; ++j) {
+                            const uint32_t a0 = st0 + (uint32_t)(j * kUmmaRows * kUmmaBK * 2);
+                            const uint32_t b0 = st0 + (uint32_t)(p.x_off + j * p.x_stride);
 #pragma unroll
-                        for (int k = 0; k < kUmmaBK / 16; ++k) {
-                            // advancing K by 16 bf16 = 32 bytes inside the swizzle atom
-                            tc_mma(d_tmem, sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k), idesc,
-                                   (first_stage && k == 0) ? 0u : 1u);
+                            for (int k = 0; k < kUmmaBK / 16; ++k) {
+                                // advancing K by 16 bf16 = 32 bytes inside the swizzle atom
+                                tc_mma(d_tmem, sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k), idesc,
+                                       (first_stage && j == 0 && k == 0) ? 0u : 1u);
+                            }
                         }
                         any_mma = true;
                         tc_commit(&empty_bar[s]);  // frees the stage once these MMAs have read it
@@ -297,8 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             const long long lo = range_lo(Tt, c, G), hi = range_lo(Tt, c + 1, G);
             long long it = lo;
             bool wrote_any = false;
-            while (it < hi) {
-                const int tile = (int)(it / T.kb);
+            for (int tile = (int)(lo / T.kb); it < hi; ++tile) {
                 const long long tile_lo = (long long)tile * T.kb, tile_hi = tile_lo + T.kb;
                 const long long seg_start = it;
                 const long long seg_end = tile_hi < hi ? tile_hi : hi;
