@@ -86,6 +86,21 @@ enum {
     WSM_L2_NORMAL = 2
 };
 
+/* Flags of wsm_opts / wsm_chain_opts.
+ *
+ * Every launch uses programmatic dependent launch: the kernel may start while
+ * the kernel queued before it on the stream is finishing, and waits for it
+ * (griddepcontrol.wait) before touching global memory, so stream order is
+ * kept.  WSM_FLAG_W_READONLY relaxes that for W only: the caller promises
+ * that the kernel queued just before this call does not write W, and the
+ * weight stream (which is the whole cost of a decode GEMM) then starts
+ * before that kernel has finished; X, Y and the scratch still wait.
+ * WSM_FLAG_NO_PDL launches without programmatic dependent launch. */
+enum {
+    WSM_FLAG_W_READONLY = 1,
+    WSM_FLAG_NO_PDL = 2
+};
+
 /* Options of skinny_gemm_ex; zero-initialised = all automatic. */
 typedef struct {
     int path;        /* WSM_PATH_* */
@@ -97,6 +112,8 @@ typedef struct {
                         number of SMs are clamped */
     int stage_k;     /* UMMA path: K elements per pipeline stage, 0 = auto,
                         else 64, 128 or 256 */
+    int flags;       /* WSM_FLAG_* */
+    int reserved0;
     float *Yf32;     /* optional device [M, N] fp32: the result before rounding */
     void *workspace; /* optional caller scratch (device, >= wsm_workspace_bytes,
                         16-byte aligned, zero-filled before its first use; the
@@ -169,7 +186,8 @@ typedef struct {
     int debug_unmet_dependency; /* test hook, 0 in real use: nonzero makes every dependency
                                    target unreachable, so each dependency wait runs out after
                                    timeout_ns and the run reports WSM_ERR_TIMEOUT */
-    int reserved[2];
+    int flags;                 /* WSM_FLAG_* (for the whole chain) */
+    int stage_k;               /* as in wsm_opts (UMMA path), 0 = auto */
 } wsm_chain_opts;
 
 typedef struct wsm_chain wsm_chain;  /* opaque prepared chain */

@@ -251,3 +251,29 @@ def test_workspace_reused_across_shapes():
         x, w = synth.make_xw(M, N, K, seed=N + 1)
         y, yf = run(x, w, path=path, workspace=ws)
         check_full(x, w, y, yf, what=f"caller workspace M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("flags", [0, wsm.FLAG_W_READONLY, wsm.FLAG_NO_PDL])
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 2), (wsm.PATH_UMMA, 16)])
+def test_back_to_back_dependent_calls(flags, path, M):
+    """Calls queued back to back on one stream, each reading the previous
+    call's Y as its X: the programmatic-dependent-launch waits must keep
+    stream order for X, Y and the scratch (W may be streamed early only
+    with FLAG_W_READONLY, and W is never written here)."""
+    dims = [2048, 4096, 1024, 6144, 2048, 4096]
+    xs = [synth.make_x(M, dims[0], 1).to(DEV)]
+    ws = [synth.make_w(dims[i + 1], dims[i], 50 + i).to(DEV) for i in range(len(dims) - 1)]
+    ys = [torch.full((M, dims[i + 1]), float("nan"), dtype=torch.bfloat16, device=DEV) for i in range(len(ws))]
+    for rep in range(3):
+        for y in ys:
+            y.fill_(float("nan"))
+        x = xs[0]
+        for i, w in enumerate(ws):
+            wsm.skinny_gemm(x, w, ys[i], path=path, flags=flags)
+            x = ys[i]
+        torch.cuda.synchronize()
+        assert wsm.stream_status() == 0
+        x = xs[0]
+        for i, w in enumerate(ws):
+            check_full(x.cpu(), w.cpu(), ys[i], what=f"rep {rep} call {i} flags {flags}")
+            x = ys[i]

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "LIB_PATH", "WSM_OK", "WSM_ERR_INVALID", "WSM_ERR_UNSUPPORTED", "WSM_ERR_ALIGN", "WSM_ERR_NOMEM",
     "WSM_ERR_CUDA", "WSM_ERR_TIMEOUT", "PATH_AUTO", "PATH_STREAM", "PATH_UMMA", "ORDER_AUTO", "ORDER_M_MAJOR",
-    "ORDER_NAIVE", "L2_AUTO", "L2_EVICT_FIRST", "L2_NORMAL", "WsmError", "lib", "skinny_gemm", "plan",
+    "ORDER_NAIVE", "L2_AUTO", "L2_EVICT_FIRST", "L2_NORMAL", "FLAG_W_READONLY", "FLAG_NO_PDL", "WsmError", "lib", "skinny_gemm", "plan",
     "workspace_bytes", "stream_status", "Task", "Chain", "gemm_chain", "chain_validate", "last_error",
     "abi_version", "HEADER_SYMBOLS",
 ]
@@ -33,6 +33,7 @@ _STATUS_NAMES = {0: "WSM_OK", 1: "WSM_ERR_INVALID", 2: "WSM_ERR_UNSUPPORTED", 3:
 PATH_AUTO, PATH_STREAM, PATH_UMMA = 0, 1, 2
 ORDER_AUTO, ORDER_M_MAJOR, ORDER_NAIVE = 0, 1, 2
 L2_AUTO, L2_EVICT_FIRST, L2_NORMAL = 0, 1, 2
+FLAG_W_READONLY, FLAG_NO_PDL = 1, 2
 
 # Every function include/wsm.h declares (checked by the CPU tests).
 HEADER_SYMBOLS = (
@@ -51,7 +52,7 @@ class WsmError(RuntimeError):
 class _Opts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("m_tile", ctypes.c_int), ("order", ctypes.c_int),
                 ("l2_policy", ctypes.c_int), ("grid", ctypes.c_int), ("stage_k", ctypes.c_int),
-                ("Yf32", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+                ("flags", ctypes.c_int), ("reserved0", ctypes.c_int), ("Yf32", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
 class _PlanInfo(ctypes.Structure):
@@ -70,7 +71,8 @@ class _Task(ctypes.Structure):
 
 class _ChainOpts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("grid", ctypes.c_int), ("timeout_ns", ctypes.c_ulonglong),
-                ("trace", ctypes.c_int), ("debug_unmet_dependency", ctypes.c_int), ("reserved", ctypes.c_int * 2)]
+                ("trace", ctypes.c_int), ("debug_unmet_dependency", ctypes.c_int), ("flags", ctypes.c_int),
+                ("stage_k", ctypes.c_int)]
 
 
 _lib = None
@@ -154,9 +156,10 @@ def _check_operand(name, t, dtype=torch.bfloat16):
 
 
 def _opts(path=PATH_AUTO, m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32=None, workspace=None,
-          stage_k=0):
+          stage_k=0, flags=0):
     o = _Opts()
     o.path, o.m_tile, o.order, o.l2_policy, o.grid, o.stage_k = path, m_tile, order, l2_policy, grid, stage_k
+    o.flags = flags
     o.Yf32 = _ptr(yf32)
     if workspace is not None:
         o.workspace = workspace.data_ptr()
@@ -166,7 +169,7 @@ def _opts(path=PATH_AUTO, m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0,
 
 def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = None, *, path=PATH_AUTO,
                 m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32: Optional[torch.Tensor] = None,
-                workspace: Optional[torch.Tensor] = None, stage_k=0, stream=None) -> torch.Tensor:
+                workspace: Optional[torch.Tensor] = None, stage_k=0, flags=0, stream=None) -> torch.Tensor:
     """Y = X @ W.T on the current (or given) stream; returns Y."""
     _check_operand("x", x)
     _check_operand("w", w)
@@ -183,13 +186,13 @@ def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = No
         _check_operand("yf32", yf32, torch.float32)
         if tuple(yf32.shape) != (M, N):
             raise ValueError(f"yf32 must be [{M}, {N}]")
-    plain = (path, m_tile, order, l2_policy, grid, stage_k) == (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0, 0) \
+    plain = (path, m_tile, order, l2_policy, grid, stage_k, flags) == (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0, 0, 0) \
         and yf32 is None and workspace is None
     s = _stream_handle(stream)
     if plain:
         _check(lib().skinny_gemm(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, s), "skinny_gemm")
     else:
-        o = _opts(path, m_tile, order, l2_policy, grid, yf32, workspace, stage_k)
+        o = _opts(path, m_tile, order, l2_policy, grid, yf32, workspace, stage_k, flags)
         _check(lib().skinny_gemm_ex(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, ctypes.byref(o), s),
                "skinny_gemm_ex")
     return y
@@ -253,7 +256,7 @@ class Chain:
     """A prepared chain of GEMMs run as one persistent kernel."""
 
     def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
-                 debug_unmet_dependency=False):
+                 debug_unmet_dependency=False, flags=0, stage_k=0):
         for i, t in enumerate(tasks):
             _check_operand(f"tasks[{i}].x", t.x)
             _check_operand(f"tasks[{i}].w", t.w)
@@ -263,6 +266,7 @@ class Chain:
         o = _ChainOpts()
         o.path, o.grid, o.timeout_ns, o.trace = path, grid, timeout_ns, 1 if trace else 0
         o.debug_unmet_dependency = 1 if debug_unmet_dependency else 0
+        o.flags, o.stage_k = flags, stage_k
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

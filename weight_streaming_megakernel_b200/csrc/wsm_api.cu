@@ -113,6 +113,7 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
     if (o->order < 0 || o->order > WSM_ORDER_NAIVE) return fail(WSM_ERR_INVALID, "bad order %d", o->order);
     if (o->l2_policy < 0 || o->l2_policy > WSM_L2_NORMAL) return fail(WSM_ERR_INVALID, "bad l2_policy %d", o->l2_policy);
     if (o->grid < 0) return fail(WSM_ERR_INVALID, "bad grid %d", o->grid);
+    if (o->flags & ~(WSM_FLAG_W_READONLY | WSM_FLAG_NO_PDL)) return fail(WSM_ERR_INVALID, "bad flags %#x", o->flags);
     if (path == WSM_PATH_AUTO) path = (M <= 8) ? WSM_PATH_STREAM : WSM_PATH_UMMA;
     g = Geo{};
     g.path = path;
@@ -399,17 +400,27 @@ wsm_status stream_workspace(int dev, cudaStream_t stream, const Geo &g, void **o
     return WSM_OK;
 }
 
+int pdl_mode(int flags) {
+    if (flags & WSM_FLAG_NO_PDL) return 0;
+    return (flags & WSM_FLAG_W_READONLY) ? 2 : 1;
+}
+
 wsm_status launch(const void *fn, const Geo &g, const KParams &kp, cudaStream_t stream, bool cooperative) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)g.grid);
     cfg.blockDim = dim3((unsigned)g.threads);
     cfg.dynamicSmemBytes = (size_t)kp.stages * kp.stage_bytes + 1024;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     int na = 0;
     if (cooperative) {
         attr[na].id = cudaLaunchAttributeCooperative;
         attr[na].val.cooperative = 1;
+        ++na;
+    }
+    if (kp.pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
         ++na;
     }
     cfg.attrs = attr;
@@ -444,6 +455,7 @@ struct wsm_chain {
     bool any_dep = false;
     unsigned long long dep_timeout_ns = 0;
     uint32_t dep_target_extra = 0;
+    int pdl = 1;
     const void *fn = nullptr;
 };
 
@@ -542,6 +554,7 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     kp.x_off = g.x_off;
     kp.kps = g.kps;
     kp.x_stride = g.x_stride;
+    kp.pdl = pdl_mode(opts->flags);
     kp.epoch = 1;
     kp.status = reinterpret_cast<int *>(wsb + L.status_off);
     kp.dep_timeout_ns = kDefaultDepTimeoutNs;
@@ -609,12 +622,16 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     ch->tasks.assign(tasks, tasks + n);
     ch->dep_timeout_ns = opts->timeout_ns ? opts->timeout_ns : kDefaultDepTimeoutNs;
     ch->dep_target_extra = opts->debug_unmet_dependency ? 0x40000000u : 0u;
+    if (opts->flags & ~(WSM_FLAG_W_READONLY | WSM_FLAG_NO_PDL))
+        return fail(WSM_ERR_INVALID, "bad chain flags %#x", opts->flags);
+    ch->pdl = pdl_mode(opts->flags);
 
     // per-task geometry; the ring is sized for the widest task
     std::vector<Geo> geos(n);
     wsm_opts to{};
     to.path = path;
     to.grid = opts->grid;
+    to.stage_k = (path == WSM_PATH_UMMA) ? opts->stage_k : 0;
     const int chain_mmax = (path == WSM_PATH_STREAM) ? pow2ceil(maxM) : 0;
     for (int i = 0; i < n; ++i) {
         if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, d->sms, &to, geos[i], chain_mmax)) != WSM_OK)
@@ -736,6 +753,7 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     kp.x_off = ch->geo.x_off;
     kp.kps = ch->geo.kps;
     kp.x_stride = ch->geo.x_stride;
+    kp.pdl = ch->pdl;
     kp.epoch = ch->epoch;
     kp.dep_target_extra = ch->dep_target_extra;
     kp.status = ch->d_status;

@@ -70,7 +70,9 @@ struct KParams {
     uint32_t dep_target_extra;      // 0; a test hook makes every dependency unreachable with it
     int kps;                        // UMMA path: 64-wide K boxes per stage
     int x_stride;                   // UMMA path: bytes between the X boxes of a stage
-    int pad2_[2];
+    int pdl;                        // 0: plain launch; 1: wait for the previous kernel before any
+                                    // global access; 2: stream W before that wait, X after it
+    int pad2_;
     int *status;                    // kStatusWords ints
     unsigned long long dep_timeout_ns;
     unsigned long long wait_timeout_ns;
@@ -256,6 +258,50 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
         }
     }
 }
+
+// The slot holding contributor cj's partial of the tile whose stages start at
+// tile_lo (c_first's slot is 2c+1 when the tile is its LAST segment).
+__device__ __forceinline__ int contributor_slot(int cj, int c_first, int first_slot) {
+    return cj == c_first ? first_slot : 2 * cj;
+}
+
+// Sum, in CTA order (= K order), of the partials of rows m0 .. m0+MB-1 (those
+// below mrows) of one tile row `off` from every contributor; the loads of a
+// block of CB contributors x MB rows are issued together so the reduction
+// costs a few L2 round trips, not one per partial.  `sum` is written for the
+// rows below mrows.
+template <int MB, int CB>
+__device__ __forceinline__ void ordered_partial_sums(const float *part, int slot_elems, int row_stride, int off,
+                                                     int m0, int mrows, int c_first, int c_last, int first_slot,
+                                                     long long T, int G, float (&sum)[MB]) {
+    bool first = true;
+    for (int cb = c_first; cb <= c_last; cb += CB) {
+        float v[CB][MB];
+        bool ok[CB];
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+            const int cj = cb + u;
+            ok[u] = cj <= c_last && (T >= G || cta_has_work(T, cj, G));
+            const float *q = part + (size_t)contributor_slot(cj, c_first, first_slot) * slot_elems + off;
+#pragma unroll
+            for (int i = 0; i < MB; ++i)
+                v[u][i] = (ok[u] && m0 + i < mrows) ? ld_cg_f32(q + (size_t)(m0 + i) * row_stride) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+            if (ok[u]) {
+#pragma unroll
+                for (int i = 0; i < MB; ++i) sum[i] = first ? v[u][i] : sum[i] + v[u][i];
+                first = false;
+            }
+        }
+    }
+}
+
+// Programmatic dependent launch: let the next kernel on the stream begin its
+// prologue, and wait for the previous kernel's completion (and memory).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Before a CTA exits, every TMA copy it issued must have landed: wait for the
 // full barriers of the last min(S, issued) stages, under ONE overall

@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
         }
         abort_flag = 0;
         fence_mbar_init();
+        pdl_launch_dependents();
     }
     __syncthreads();
     const unsigned long long wlim = p.wait_timeout_ns;
@@ -131,6 +132,8 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
             uint32_t ph = 0;
             long long issued = 0;
             bool aborted = false;
+            bool grid_dep_ok = p.pdl != 2;
+            if (p.pdl == 1) pdl_wait();
             for (int t = 0; t < p.n_tasks && !aborted; ++t) {
                 const TaskDev &T = task_at(p, t);
                 const long long Tt = (long long)T.n_g * T.kb;
@@ -139,12 +142,16 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 prefetch_tmap(&T.tmW);
                 prefetch_tmap(&T.tmX);
                 const uint64_t pol_w = T.w_evict_first ? policy_evict_first() : policy_evict_normal();
-                bool dep_ok = T.dep < 0;
+                bool dep_ok = T.dep < 0 && grid_dep_ok;
                 int pend_s[kMaxStages], pend_k[kMaxStages];
                 int np = 0;
                 if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 0] = globaltimer();
                 auto flush = [&]() {
-                    wait_dependency(p, task_at(p, T.dep), t, p.status);
+                    if (!grid_dep_ok) {
+                        pdl_wait();
+                        grid_dep_ok = true;
+                    }
+                    if (T.dep >= 0) wait_dependency(p, task_at(p, T.dep), t, p.status);
                     if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
                     for (int i = 0; i < np; ++i) {
                         uint8_t *xs = ring + (size_t)pend_s[i] * p.stage_bytes + p.x_off;
@@ -191,6 +198,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 if (np > 0) flush();
                 if (p.trace && T.dep < 0) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
             }
+            if (!grid_dep_ok) pdl_wait();
             // copies in flight must land before exit, abort or not
             drain_issued(full_bar, S, issued, wlim, p.status);
         }
@@ -201,6 +209,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
         const int rg = cw / KW;
         const int ctid = threadIdx.x - 32;
         const bool leader = (ctid == 0);
+        if (p.pdl) pdl_wait();  // Y and the scratch may still be in use by the previous kernel
         int s = 0;
         uint32_t ph = 0;
         uint32_t seg = 0;
@@ -323,24 +332,15 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     if (last_flag) {
                         __threadfence();
                         if (owner) {
-                            float sum = 0.f;
-                            for (int cj = c_first, j = 0; cj <= c_last; ++cj) {
-                                if (!cta_has_work(Tt, cj, G)) continue;
-                                float x;
-                                if (cj == c) {
-                                    x = val;
-                                } else {
-                                    const long long lo_j = range_lo(Tt, cj, G);
-                                    const int sj = (cj == c_first && lo_j < tile_lo) ? 2 * cj + 1 : 2 * cj;
-                                    x = ld_cg_f32(T.part + (size_t)sj * T.slot_elems + ctid);
-                                }
-                                sum = (j == 0) ? x : sum + x;
-                                ++j;
-                            }
+                            const int first_slot =
+                                (range_lo(Tt, c_first, G) < tile_lo) ? 2 * c_first + 1 : 2 * c_first;
+                            float sum[1];
+                            ordered_partial_sums<1, 8>(T.part, T.slot_elems, 0, ctid, 0, 1, c_first, c_last,
+                                                       first_slot, Tt, G, sum);
                             if (live) {
                                 const size_t o = (size_t)o_m * T.N + n;
-                                T.Y[o] = __float2bfloat16_rn(sum);
-                                if (T.Yf32) T.Yf32[o] = sum;
+                                T.Y[o] = __float2bfloat16_rn(sum[0]);
+                                if (T.Yf32) T.Yf32[o] = sum[0];
                             }
                         }
                         named_bar_sync(kConsBar, NCT);

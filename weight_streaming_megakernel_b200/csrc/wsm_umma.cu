@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(&tmem_base_sh, kTmemCols);
+    if (threadIdx.x == 0) pdl_launch_dependents();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -165,6 +166,8 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             uint32_t ph = 0;
             long long issued = 0;
             bool aborted = false;
+            bool grid_dep_ok = p.pdl != 2;  // mode 2 streams W before the previous kernel completes
+            if (p.pdl == 1) pdl_wait();
             for (int t = 0; t < p.n_tasks && !aborted; ++t) {
                 const TaskDev &T = task_at(p, t);
                 const long long Tt = (long long)T.n_g * T.n_mt * T.kb;
@@ -173,12 +176,16 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 prefetch_tmap(&T.tmW);
                 prefetch_tmap(&T.tmX);
                 const uint64_t pol_w = T.w_evict_first ? policy_evict_first() : policy_evict_normal();
-                bool dep_ok = T.dep < 0;
+                bool dep_ok = T.dep < 0 && grid_dep_ok;
                 int pend_s[kMaxStages], pend_k[kMaxStages], pend_y[kMaxStages];
                 int np = 0;
                 if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 0] = globaltimer();
                 auto flush = [&]() {
-                    wait_dependency(p, task_at(p, T.dep), t, p.status);
+                    if (!grid_dep_ok) {
+                        pdl_wait();
+                        grid_dep_ok = true;
+                    }
+                    if (T.dep >= 0) wait_dependency(p, task_at(p, T.dep), t, p.status);
                     if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
                     for (int i = 0; i < np; ++i)
                         for (int j = 0; j < p.kps; ++j)
@@ -224,6 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 if (np > 0) flush();
                 if (p.trace && T.dep < 0) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
             }
+            if (!grid_dep_ok) pdl_wait();  // a CTA with no work still orders itself after the previous kernel
             // Drain: every stage this thread issued must have landed before the
             // CTA may exit (bounded; in a healthy run these already completed).
             // copies in flight must land before exit, abort or not
@@ -298,6 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         const int row = q * 32 + lane;          // row of the 128-row tile = TMEM lane
         const int etid = threadIdx.x - kEpiWarp0 * 32;
         const bool leader = (etid == 0);
+        if (p.pdl) pdl_wait();                  // Y and the scratch may still be in use by the previous kernel
         uint32_t seg = 0;
         bool aborted = false;
         for (int t = 0; t < p.n_tasks; ++t) {
@@ -392,36 +401,19 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     epi_bar();
                     if (last_flag) {
                         __threadfence();
-                        float sum[kUmmaMaxN];
+                        const int first_slot = (range_lo(Tt, c_first, G) < tile_lo) ? 2 * c_first + 1 : 2 * c_first;
+                        for (int mb = 0; mb < mrows; mb += 8) {
+                            float sum[8];
+                            ordered_partial_sums<8, 4>(T.part, T.slot_elems, kUmmaRows, row, mb, mrows, c_first,
+                                                       c_last, first_slot, Tt, G, sum);
+                            if (n < T.N) {
 #pragma unroll
-                        for (int m = 0; m < kUmmaMaxN; ++m) sum[m] = 0.f;
-                        for (int cj = c_first, j = 0; cj <= c_last; ++cj) {
-                            if (!cta_has_work(Tt, cj, G)) continue;  // only when the task has fewer stages than CTAs
-                            if (cj == c) {
-#pragma unroll
-                                for (int m = 0; m < kUmmaMaxN; ++m)
-                                    if (m < mrows) sum[m] = (j == 0) ? acc[m] : sum[m] + acc[m];
-                            } else {
-                                const long long lo_j = range_lo(Tt, cj, G);
-                                const int sj = (cj == c_first && lo_j < tile_lo) ? 2 * cj + 1 : 2 * cj;
-                                const float *q_ = T.part + (size_t)sj * T.slot_elems;
-#pragma unroll
-                                for (int m = 0; m < kUmmaMaxN; ++m) {
-                                    if (m < mrows) {
-                                        const float v = ld_cg_f32(q_ + m * kUmmaRows + row);
-                                        sum[m] = (j == 0) ? v : sum[m] + v;
+                                for (int i = 0; i < 8; ++i) {
+                                    if (mb + i < mrows) {
+                                        const size_t o = (size_t)(m0 + mb + i) * T.N + n;
+                                        T.Y[o] = __float2bfloat16_rn(sum[i]);
+                                        if (T.Yf32) T.Yf32[o] = sum[i];
                                     }
-                                }
-                            }
-                            ++j;
-                        }
-                        if (n < T.N) {
-#pragma unroll
-                            for (int m = 0; m < kUmmaMaxN; ++m) {
-                                if (m < mrows) {
-                                    const size_t o = (size_t)(m0 + m) * T.N + n;
-                                    T.Y[o] = __float2bfloat16_rn(sum[m]);
-                                    if (T.Yf32) T.Yf32[o] = sum[m];
                                 }
                             }
                         }
