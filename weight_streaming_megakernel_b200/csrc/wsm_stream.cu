@@ -308,10 +308,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     }
                     if (T.notify) {
                         named_bar_sync(kConsBar, NCT);
-                        if (leader && !aborted) {
-                            __threadfence();
-                            red_release_gpu_add(T.done, 1u);
-                        }
+                        if (leader && !aborted) red_release_gpu_add(T.done, 1u);  // release covers the CTA's stores (bar.sync before)
                     }
                 } else {
                     int c_first, c_last;
@@ -322,7 +319,8 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     if (leader) {
                         int last = 0;
                         if (!aborted) {
-                            __threadfence();
+                            // acq_rel: releases the partials this CTA stored before the barrier, and
+                            // acquires the others' partials for the last arriver
                             const unsigned int old = atom_add_acqrel_gpu(&T.tile_cnt[g], 1u);
                             last = (old == (unsigned int)(n_c - 1)) ? 1 : 0;
                         }
@@ -330,7 +328,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     }
                     named_bar_sync(kConsBar, NCT);
                     if (last_flag) {
-                        __threadfence();
+                        // the leader's acquire + the barrier order these loads after every partial
                         if (owner) {
                             const int first_slot =
                                 (range_lo(Tt, c_first, G) < tile_lo) ? 2 * c_first + 1 : 2 * c_first;
@@ -346,10 +344,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                         named_bar_sync(kConsBar, NCT);
                         if (leader) {
                             T.tile_cnt[g] = 0u;
-                            if (T.notify) {
-                                __threadfence();
-                                red_release_gpu_add(T.done, 1u);
-                            }
+                            if (T.notify) red_release_gpu_add(T.done, 1u);
                         }
                     }
                 }

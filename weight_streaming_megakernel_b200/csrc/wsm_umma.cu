@@ -372,10 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     }
                     if (T.notify) {
                         epi_bar();
-                        if (leader && !aborted) {
-                            __threadfence();
-                            red_release_gpu_add(T.done, 1u);
-                        }
+                        if (leader && !aborted) red_release_gpu_add(T.done, 1u);  // release covers the CTA's stores (bar.sync before)
                     }
                 } else {
                     // split tile: write this CTA's partial, then the last arriver reduces
@@ -392,7 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     if (leader) {
                         int last = 0;
                         if (!aborted) {
-                            __threadfence();
+                            // acq_rel: releases the partials this CTA stored before the barrier, and
+                            // acquires the others' partials for the last arriver
                             const unsigned int old = atom_add_acqrel_gpu(&T.tile_cnt[tile], 1u);
                             last = (old == (unsigned int)(n_c - 1)) ? 1 : 0;
                         }
@@ -400,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     }
                     epi_bar();
                     if (last_flag) {
-                        __threadfence();
+                        // the leader's acquire + the barrier order these loads after every partial
                         const int first_slot = (range_lo(Tt, c_first, G) < tile_lo) ? 2 * c_first + 1 : 2 * c_first;
                         for (int mb = 0; mb < mrows; mb += 8) {
                             float sum[8];
@@ -420,10 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         epi_bar();
                         if (leader) {
                             T.tile_cnt[tile] = 0u;  // ready for the next call
-                            if (T.notify) {
-                                __threadfence();
-                                red_release_gpu_add(T.done, 1u);
-                            }
+                            if (T.notify) red_release_gpu_add(T.done, 1u);
                         }
                     }
                 }
