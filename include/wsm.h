@@ -212,11 +212,11 @@ wsm_status wsm_chain_run(wsm_chain *chain, wsm_stream_t stream);
 wsm_status wsm_chain_status(wsm_chain *chain, wsm_stream_t stream, int *failed_task);
 
 /* Copy the trace of the last run (trace != 0 at create) into host `out`:
- * stamps[cta][task][3] = {first stage issued, dependency met, last tile
- * written}, %globaltimer nanoseconds, 0 where the CTA had no work for the
- * task.  `capacity` is the number of uint64 slots in `out`; returns the number
- * needed (grid * n_tasks * 3), or 0 when tracing was not enabled.
- * Synchronises `stream`. */
+ * stamps[cta][task][4] = {first stage issued, dependency met, last tile
+ * written (%globaltimer nanoseconds, 0 where the CTA had no work for the
+ * task), SM the CTA ran on}.  `capacity` is the number of uint64 slots in
+ * `out`; returns the number needed (grid * n_tasks * 4), or 0 when tracing
+ * was not enabled.  Synchronises `stream`. */
 size_t wsm_chain_trace(wsm_chain *chain, wsm_stream_t stream, unsigned long long *out,
                        size_t capacity);
 

@@ -714,7 +714,7 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         return cuda_fail(e, "cudaMemcpy(task table)");
     }
     if (opts->trace) {
-        ch->trace_elems = (size_t)ring.grid * n * 3;
+        ch->trace_elems = (size_t)ring.grid * n * 4;
         e = cudaMalloc(reinterpret_cast<void **>(&ch->d_trace), ch->trace_elems * 8);
         if (e != cudaSuccess) {
             cleanup();

@@ -145,14 +145,19 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 bool dep_ok = T.dep < 0 && grid_dep_ok;
                 int pend_s[kMaxStages], pend_k[kMaxStages];
                 int np = 0;
-                if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 0] = globaltimer();
+                if (p.trace) {
+                    p.trace[((size_t)c * p.n_tasks + t) * 4 + 0] = globaltimer();
+                    uint32_t smid;
+                    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+                    p.trace[((size_t)c * p.n_tasks + t) * 4 + 3] = smid;
+                }
                 auto flush = [&]() {
                     if (!grid_dep_ok) {
                         pdl_wait();
                         grid_dep_ok = true;
                     }
                     if (T.dep >= 0) wait_dependency(p, task_at(p, T.dep), t, p.status);
-                    if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
+                    if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 4 + 1] = globaltimer();
                     for (int i = 0; i < np; ++i) {
                         uint8_t *xs = ring + (size_t)pend_s[i] * p.stage_bytes + p.x_off;
 #pragma unroll
@@ -196,7 +201,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     }
                 }
                 if (np > 0) flush();
-                if (p.trace && T.dep < 0) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
+                if (p.trace && T.dep < 0) p.trace[((size_t)c * p.n_tasks + t) * 4 + 1] = globaltimer();
             }
             if (!grid_dep_ok) pdl_wait();
             // copies in flight must land before exit, abort or not
@@ -350,7 +355,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 }
                 wrote_any = true;
             }
-            if (p.trace && wrote_any && leader) p.trace[((size_t)c * p.n_tasks + t) * 3 + 2] = globaltimer();
+            if (p.trace && wrote_any && leader) p.trace[((size_t)c * p.n_tasks + t) * 4 + 2] = globaltimer();
         }
     }
     __syncthreads();

@@ -179,14 +179,19 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 bool dep_ok = T.dep < 0 && grid_dep_ok;
                 int pend_s[kMaxStages], pend_k[kMaxStages], pend_y[kMaxStages];
                 int np = 0;
-                if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 0] = globaltimer();
+                if (p.trace) {
+                    p.trace[((size_t)c * p.n_tasks + t) * 4 + 0] = globaltimer();
+                    uint32_t smid;
+                    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+                    p.trace[((size_t)c * p.n_tasks + t) * 4 + 3] = smid;
+                }
                 auto flush = [&]() {
                     if (!grid_dep_ok) {
                         pdl_wait();
                         grid_dep_ok = true;
                     }
                     if (T.dep >= 0) wait_dependency(p, task_at(p, T.dep), t, p.status);
-                    if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
+                    if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 4 + 1] = globaltimer();
                     for (int i = 0; i < np; ++i)
                         for (int j = 0; j < p.kps; ++j)
                             tma_load_2d(ring + (size_t)pend_s[i] * p.stage_bytes + p.x_off + j * p.x_stride, &T.tmX,
@@ -229,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     }
                 }
                 if (np > 0) flush();
-                if (p.trace && T.dep < 0) p.trace[((size_t)c * p.n_tasks + t) * 3 + 1] = globaltimer();
+                if (p.trace && T.dep < 0) p.trace[((size_t)c * p.n_tasks + t) * 4 + 1] = globaltimer();
             }
             if (!grid_dep_ok) pdl_wait();  // a CTA with no work still orders itself after the previous kernel
             // Drain: every stage this thread issued must have landed before the
@@ -424,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 }
                 wrote_any = true;
             }
-            if (p.trace && wrote_any && leader) p.trace[((size_t)c * p.n_tasks + t) * 3 + 2] = globaltimer();
+            if (p.trace && wrote_any && leader) p.trace[((size_t)c * p.n_tasks + t) * 4 + 2] = globaltimer();
         }
     }
 
