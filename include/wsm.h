@@ -131,6 +131,8 @@ typedef struct {
     int m_tile;        /* X rows per tile (padded to the MMA width on UMMA) */
     int m_tiles;       /* number of M-tiles */
     int n_tiles;       /* number of N-column tiles */
+    int unit_stages;   /* pipeline stages per work unit */
+    long long units;   /* work units (n_tiles * m_tiles * ceil(k_iters / unit_stages)) */
     int k_iters;       /* pipeline stages per tile */
     int stages;        /* shared-memory ring depth */
     int order;         /* WSM_ORDER_M_MAJOR or WSM_ORDER_NAIVE */

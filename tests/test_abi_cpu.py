@@ -91,9 +91,25 @@ def test_plan_m_tiling_and_l2_policy():
 
 def test_plan_workspace_formula():
     p = wsm.plan(16, 4096, 4096, num_sms=148)
-    slots = 2 * p["grid"] * 128 * 16 * 4
-    assert p["workspace_bytes"] >= 256 + p["n_tiles"] * p["m_tiles"] * 4 + slots
+    nu = -(-p["k_iters"] // p["unit_stages"])
+    assert p["units"] == p["n_tiles"] * p["m_tiles"] * nu
+    counters = (2 + p["n_tiles"] * p["m_tiles"]) * 4
+    partials = p["units"] * 128 * 16 * 4 if nu > 1 else 0
+    assert p["workspace_bytes"] >= 256 + counters + partials
     assert p["workspace_bytes"] % 256 == 0
+
+
+def test_plan_units():
+    """Enough units for every CTA to take several, none smaller than 32 KB."""
+    for M, N, K in [(1, 4096, 4096), (16, 4096, 4096), (1, 57344, 8192), (16, 24576, 4096), (4, 2112, 7168)]:
+        p = wsm.plan(M, N, K, num_sms=148)
+        stage_bytes = p["tile_rows"] * p["tile_k"] * 2
+        assert 1 <= p["unit_stages"] <= p["k_iters"]
+        assert p["unit_stages"] * stage_bytes >= min(32 << 10, p["k_iters"] * stage_bytes)
+        if p["unit_stages"] > 1 and p["unit_stages"] * stage_bytes > 64 << 10:
+            assert p["units"] >= 8 * 148 // 2
+    p = wsm.plan(1, 57344, 8192, num_sms=148)
+    assert p["units"] >= 8 * 148
 
 
 @pytest.mark.parametrize("M,N,K", [(0, 16, 16), (65, 16, 16), (1, 0, 16), (1, 16, 4), (1, 16, 12), (1, 16, 0)])

@@ -58,7 +58,8 @@ class _Opts(ctypes.Structure):
 class _PlanInfo(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("grid", ctypes.c_int), ("tile_rows", ctypes.c_int),
                 ("tile_k", ctypes.c_int), ("m_tile", ctypes.c_int), ("m_tiles", ctypes.c_int),
-                ("n_tiles", ctypes.c_int), ("k_iters", ctypes.c_int), ("stages", ctypes.c_int),
+                ("n_tiles", ctypes.c_int), ("unit_stages", ctypes.c_int), ("units", ctypes.c_longlong),
+                ("k_iters", ctypes.c_int), ("stages", ctypes.c_int),
                 ("order", ctypes.c_int), ("l2_policy", ctypes.c_int), ("smem_bytes", ctypes.c_int),
                 ("iters", ctypes.c_longlong), ("workspace_bytes", ctypes.c_size_t)]
 

@@ -67,6 +67,7 @@ struct Geo {
     int n_g = 0, kb = 0;
     int stage_bytes = 0, x_off = 0, stages = 0;
     int slot_elems = 0;
+    int ku = 1, nu = 1;        // stages per work unit, units per tile
     int order = WSM_ORDER_M_MAJOR;
     int l2 = WSM_L2_EVICT_FIRST;
     int grid = 0;
@@ -74,6 +75,8 @@ struct Geo {
     int kps = 1;               // UMMA: 64-wide K boxes per stage
     int x_stride = 0;          // UMMA: bytes between X boxes inside a stage
     long long iters() const { return (long long)n_g * n_mt * kb; }
+    long long tiles() const { return (long long)n_g * n_mt; }
+    long long units() const { return tiles() * nu; }
 };
 
 int pow2ceil(int v) {
@@ -98,6 +101,22 @@ void stream_geo(int mmax, Geo &g) {
     g.stage_bytes = g.x_off + g.kw * mmax * 512;
     g.slot_elems = g.tile_rows * mmax;
     g.threads = 32 * (1 + g.rg * g.kw);
+}
+
+// Work units: ku consecutive stages of one tile.  A unit must be big enough
+// that its partial (when the tile is split) and its claim stay small next to
+// its weight bytes (>= 32 KB and >= 8x the partial), and there should be
+// enough units for every CTA to take several (>= 8 per CTA), so SMs that
+// stream faster take more of them.  Between those, the largest unit wins.
+void plan_units(Geo &g, int ctas) {
+    const long long wstage = (long long)g.tile_rows * g.tile_k * 2;
+    const long long part_bytes = (long long)g.tile_rows * g.t_m * 4;
+    const long long min_unit = std::max<long long>(32 << 10, 8 * part_bytes);
+    const int min_ku = (int)std::min<long long>(g.kb, std::max<long long>(1, (min_unit + wstage - 1) / wstage));
+    int ku = g.kb;
+    while (ku > min_ku && g.tiles() * ((g.kb + ku - 1) / ku) < 8LL * ctas) ku = std::max(min_ku, (ku + 1) / 2);
+    g.ku = ku;
+    g.nu = (g.kb + ku - 1) / ku;
 }
 
 // force_mmax: a chain's FMA kernel has one register width for all tasks.
@@ -157,8 +176,9 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
         g.threads = 192;
     }
     g.stages = std::min(kMaxStages, kRingBudget / g.stage_bytes);
-    // no more CTAs than stages: every CTA then has work
-    if ((long long)g.grid > g.iters()) g.grid = (int)g.iters();
+    plan_units(g, g.grid);
+    // no more CTAs than work units
+    if ((long long)g.grid > g.units()) g.grid = (int)g.units();
     if (g.l2 = o->l2_policy, g.l2 == WSM_L2_AUTO) g.l2 = (g.n_mt > 1) ? WSM_L2_NORMAL : WSM_L2_EVICT_FIRST;
     return WSM_OK;
 }
@@ -182,18 +202,19 @@ WsLayout ws_layout_of(size_t bytes) {
     L.total = bytes;
     return L;
 }
+// counters: [kSchedWords claim counters][one arrival counter per tile]
+size_t ws_counter_bytes(const Geo &g) { return ((size_t)kSchedWords + (size_t)g.tiles()) * 4; }
+size_t ws_partial_bytes(const Geo &g) { return g.nu > 1 ? (size_t)g.units() * g.slot_elems * 4 : 0; }
 bool ws_fits(const Geo &g, size_t bytes) {
     if (bytes < 512) return false;
     const WsLayout L = ws_layout_of(bytes);
-    const size_t n_tiles = (size_t)g.n_g * g.n_mt;
-    const size_t parts = (size_t)2 * g.grid * g.slot_elems * 4;
-    return L.cnt_off + n_tiles * 4 <= L.part_off && L.part_off + parts <= bytes;
+    return L.cnt_off + ws_counter_bytes(g) <= L.part_off && L.part_off + ws_partial_bytes(g) <= bytes;
 }
 size_t ws_required(const Geo &g) {
-    const size_t n_tiles = (size_t)g.n_g * g.n_mt;
-    const size_t parts = (size_t)2 * g.grid * g.slot_elems * 4;
+    const size_t cnt = ws_counter_bytes(g);
+    const size_t parts = ws_partial_bytes(g);
     // smallest multiple of 256 that fits, from a close lower bound upwards
-    size_t z = round_up(256 + std::max(16 * (n_tiles * 4 + 256), parts + parts / 15 + 16 * 256), 256);
+    size_t z = round_up(256 + std::max(16 * (cnt + 256), parts + parts / 15 + 16 * 256), 256);
     while (!ws_fits(g, z)) z += 256;
     while (z > 512 && ws_fits(g, z - 256)) z -= 256;
     return z;
@@ -207,6 +228,8 @@ void fill_plan_info(const Geo &g, wsm_plan_info *out) {
     out->m_tile = g.t_mpad;
     out->m_tiles = g.n_mt;
     out->n_tiles = g.n_g;
+    out->unit_stages = g.ku;
+    out->units = g.units();
     out->k_iters = g.kb;
     out->stages = g.stages;
     out->order = g.order;
@@ -345,6 +368,9 @@ wsm_status fill_task(TaskDev &T, const Geo &g, const void *X, const void *W, voi
     T.notify = 0;
     T.w_evict_first = (g.l2 == WSM_L2_EVICT_FIRST) ? 1 : 0;
     T.slot_elems = g.slot_elems;
+    T.ku = g.ku;
+    T.nu = g.nu;
+    T.n_units = (int)g.units();
     return WSM_OK;
 }
 
@@ -545,7 +571,8 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     memset(&kp, 0, sizeof kp);
     if ((st = fill_task(kp.single, g, X, W, Y, opts->Yf32, M, N, K)) != WSM_OK) return st;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
-    kp.single.tile_cnt = reinterpret_cast<unsigned int *>(wsb + L.cnt_off);
+    kp.single.sched = reinterpret_cast<unsigned int *>(wsb + L.cnt_off);
+    kp.single.tile_cnt = kp.single.sched + kSchedWords;
     kp.single.part = reinterpret_cast<float *>(wsb + L.part_off);
     kp.tasks = nullptr;
     kp.n_tasks = 1;
@@ -587,7 +614,13 @@ wsm_status wsm_stream_status(wsm_stream_t stream_, int *code) {
     WSM_CUDA(cudaMemcpy(h, ptr, sizeof h, cudaMemcpyDeviceToHost));
     if (code) *code = h[0];
     if (h[0] != 0) {
-        WSM_CUDA(cudaMemset(ptr, 0, sizeof h));
+        // an aborted call may leave its counters mid-count: clear the whole scratch
+        size_t bytes = 0;
+        {
+            std::lock_guard<std::mutex> lk(g_mu);
+            bytes = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}].bytes;
+        }
+        WSM_CUDA(cudaMemset(ptr, 0, bytes));
         return fail(WSM_ERR_TIMEOUT, "device-side wait ran out (task %d, cta %d, site %d)", h[1], h[2], h[3]);
     }
     return WSM_OK;
@@ -653,12 +686,14 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     ring.stages = std::min(kMaxStages, kRingBudget / ring.stage_bytes);
     ch->geo = ring;
 
-    // scratch: status | counters (tile counters of all tasks, then done counters) | partials
+    // work units per task, planned for the chain's grid
+    for (auto &g : geos) plan_units(g, chain_grid);
+    // scratch: status | counters (per task: claim counters + tile counters; then done counters) | partials
     std::vector<size_t> cnt_off(n), part_off(n);
     size_t ncnt = 0;
     for (int i = 0; i < n; ++i) {
         cnt_off[i] = ncnt;
-        ncnt += (size_t)geos[i].n_g * geos[i].n_mt;
+        ncnt += kSchedWords + (size_t)geos[i].tiles();
     }
     const size_t done_off = ncnt;
     ncnt += n;
@@ -667,7 +702,7 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     size_t part_at = counters_at + ch->counter_bytes;
     for (int i = 0; i < n; ++i) {
         part_off[i] = part_at;
-        part_at += round_up((size_t)2 * ring.grid * geos[i].slot_elems * 4, 256);
+        part_at += round_up(ws_partial_bytes(geos[i]), 256);
     }
     ch->buf_bytes = part_at;
     cudaError_t e = cudaMalloc(&ch->d_buf, ch->buf_bytes);
@@ -703,7 +738,8 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
             return fail(st, "task %d: %s", i, g_err.c_str());
         }
         T.dep = tasks[i].dep;
-        T.tile_cnt = ch->d_counters + cnt_off[i];
+        T.sched = ch->d_counters + cnt_off[i];
+        T.tile_cnt = T.sched + kSchedWords;
         T.done = ch->d_counters + done_off + i;
         T.notify = depended[i];
         T.part = reinterpret_cast<float *>(base + part_off[i]);

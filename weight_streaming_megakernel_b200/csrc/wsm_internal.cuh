@@ -3,16 +3,25 @@
 //
 // Work decomposition (both kernel paths):
 //   A GEMM is cut into tiles: `tile_rows` rows of W (outputs along N) times one
-//   M-tile of X.  A tile's K range is cut into `kb` pipeline stages.  The
-//   flattened list of (tile, stage) iterations, tile-major, is divided into
-//   `grid` contiguous ranges of equal length, one per persistent CTA (a
-//   stream-K split: every CTA streams the same number of weight bytes, so the
-//   split is balanced to one stage whatever N and K are).  A tile whose stages
-//   fall into several CTAs' ranges gets one fp32 partial per CTA; the CTA that
-//   arrives last on the tile's counter adds the partials in CTA order (= K
-//   order), so the result does not depend on arrival order.  This is the
-//   inter-CTA split-K of the FlyDSL article ("AMD: ROCm Low-Latency-GEMM-Kernel
-//   ... MI355X", technique 1), balanced per stage instead of per fixed factor.
+//   M-tile of X.  A tile's K range is cut into `kb` pipeline stages, and the
+//   stages into `nu` work units of `ku` consecutive stages (the last unit may
+//   be shorter).  Units are numbered tile-major (u = tile * nu + j) and handed
+//   out IN ORDER from one atomic counter per task: each persistent CTA's
+//   producer claims the next unit when it starts the current one.  The SMs of
+//   a B200 do not stream at the same rate (measured: a 2x spread between the
+//   fastest and slowest SMs on the same access pattern), so claiming units
+//   lets every SM work until the task is done instead of the task waiting for
+//   the slowest SM's fixed share.
+//
+//   A tile split into nu > 1 units gets one fp32 partial per unit, stored in
+//   the unit's own slot; the unit that arrives last on the tile's counter adds
+//   the nu partials in unit order (= K order).  Where a unit ends is fixed by
+//   the plan, not by which CTA ran it, so the result is the same for every run
+//   and every grid size.  This is the inter-CTA split-K of the FlyDSL article
+//   ("AMD: ROCm Low-Latency-GEMM-Kernel ... MI355X", technique 1), with the
+//   split placed per unit.  Claiming in order also keeps the M-tiles of one
+//   weight column (adjacent unit numbers) in flight together, the cooperative
+//   M-major traversal of "Fleet ..." (reading notes, section 3f, Eq.(1)).
 #pragma once
 
 #include <cuda.h>
@@ -24,14 +33,20 @@ namespace wsm {
 
 constexpr int kMaxStages = 16;
 constexpr int kUmmaRows = 128;     // rows of W per UMMA tile (MMA M)
-constexpr int kUmmaBK = 64;        // K elements per UMMA stage (one 128-byte swizzle row)
+constexpr int kUmmaBK = 64;        // K elements per UMMA box (one 128-byte swizzle row)
 constexpr int kUmmaMaxN = 64;      // largest MMA N (= X rows per tile)
 constexpr int kStreamBoxK = 256;   // K elements per TMA box on the FMA path
 constexpr int kStatusWords = 4;    // [0] error code, [1] failing task, [2] failing CTA, [3] site
+constexpr int kSchedWords = 2;     // per task: [0] next unit to claim, [1] CTAs done claiming
 
 // Error sites recorded in status[3].
 enum : int { kSiteNone = 0, kSiteDep = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteAcc = 4, kSiteDrain = 5 };
 constexpr int kCodeTimeout = 6;    // == WSM_ERR_TIMEOUT
+
+// Stage / accumulator metadata flags (producer -> consumers).
+constexpr int kMetaFirst = 1;      // first stage of its unit
+constexpr int kMetaLast = 2;       // last stage of its unit
+constexpr int kMetaDone = 4;       // no more work for this CTA: the role exits
 
 // One GEMM as the kernels see it.  Lives in kernel parameter space (single
 // GEMM) or in a device table (chain); 64-byte aligned for the tensor maps.
@@ -40,8 +55,9 @@ struct __align__(64) TaskDev {
     CUtensorMap tmX;            // X [M, K] bf16
     __nv_bfloat16 *Y;           // [M, N]
     float *Yf32;                // optional [M, N]
-    float *part;                // 2 * grid partial slots of slot_elems floats
+    float *part;                // n_units partial slots of slot_elems floats
     unsigned int *tile_cnt;     // [n_tiles] arrival counters, zero between calls
+    unsigned int *sched;        // [kSchedWords] unit claim counters, zero between calls
     unsigned int *done;         // tiles finished (monotonic over runs), chain only
     int M, N, K;
     int dep;                    // -1 or index of an earlier task
@@ -50,13 +66,15 @@ struct __align__(64) TaskDev {
     int t_m;                    // X rows per M-tile
     int t_mpad;                 // X rows loaded per M-tile (UMMA: multiple of 16)
     int kb;                     // stages per tile
+    int ku;                     // stages per unit
+    int nu;                     // units per tile
+    int n_units;                // n_g * n_mt * nu
     int order;                  // 0: M-tile inner (M-major), 1: M-tile outer
     int notify;                 // bump `done` after each finished tile
     int w_evict_first;          // L2 policy of the weight loads
     uint32_t idesc;             // UMMA instruction descriptor (MMA N = t_mpad)
     uint32_t tx_bytes;          // bytes landing in one stage
     int slot_elems;             // floats per partial slot
-    int pad_[2];
 };
 
 struct KParams {
@@ -72,43 +90,12 @@ struct KParams {
     int x_stride;                   // UMMA path: bytes between the X boxes of a stage
     int pdl;                        // 0: plain launch; 1: wait for the previous kernel before any
                                     // global access; 2: stream W before that wait, X after it
-    int pad2_;
+    int pad_;
     int *status;                    // kStatusWords ints
     unsigned long long dep_timeout_ns;
     unsigned long long wait_timeout_ns;
-    unsigned long long *trace;      // [grid][n_tasks][3] or nullptr
+    unsigned long long *trace;      // [grid][n_tasks][4] or nullptr
 };
-
-// ------------------------------------------------------------------ schedule
-
-// First iteration of CTA c when T iterations are split over G CTAs.
-__host__ __device__ __forceinline__ long long range_lo(long long T, int c, int G) {
-    return (T * (long long)c) / G;
-}
-// The CTA whose range holds iteration i (the largest c with range_lo(c) <= i).
-__host__ __device__ __forceinline__ int cta_of(long long i, long long T, int G) {
-    return (int)(((i + 1) * (long long)G - 1) / T);
-}
-// True when CTA c has at least one iteration (false only when T < G).
-__host__ __device__ __forceinline__ bool cta_has_work(long long T, int c, int G) {
-    return range_lo(T, c, G) < range_lo(T, c + 1, G);
-}
-// CTAs [c_first, c_last] hold the stages [tlo, thi) of one tile; returns how
-// many of them have any work (all of them unless T < G).
-__host__ __device__ __forceinline__ int tile_contributors(long long tlo, long long thi, long long T, int G,
-                                                          int &c_first, int &c_last) {
-    c_first = cta_of(tlo, T, G);
-    c_last = cta_of(thi - 1, T, G);
-    if (T >= G) return c_last - c_first + 1;
-    int n = 0;
-    for (int c = c_first; c <= c_last; ++c) n += cta_has_work(T, c, G) ? 1 : 0;
-    return n;
-}
-// Slot of CTA c's partial for the segment starting at `seg_start`: its first
-// segment uses slot 2c, its last (if different) slot 2c+1.
-__host__ __device__ __forceinline__ int partial_slot(int c, long long seg_start, long long lo) {
-    return 2 * c + (seg_start == lo ? 0 : 1);
-}
 
 #if defined(__CUDACC__)
 
@@ -122,6 +109,12 @@ __device__ __forceinline__ unsigned long long globaltimer() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+__device__ __forceinline__ uint32_t smid() {
+    uint32_t v;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(v));
+    return v;
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
@@ -212,6 +205,16 @@ __device__ __forceinline__ unsigned int atom_add_acqrel_gpu(unsigned int *p, uns
     return old;
 }
 
+__device__ __forceinline__ unsigned int atom_add_relaxed_gpu(unsigned int *p, unsigned int v) {
+    unsigned int old;
+    asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu(unsigned int *p, unsigned int v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -225,6 +228,11 @@ __device__ __forceinline__ float ld_cg_f32(const float *p) {
     asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
     return v;
 }
+
+// Programmatic dependent launch: let the next kernel on the stream begin its
+// prologue, and wait for the previous kernel's completion (and memory).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Record the first error of a launch (code, task, cta, site).
 __device__ __forceinline__ void record_error(int *status, int code, int task, int site) {
@@ -259,50 +267,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
-// The slot holding contributor cj's partial of the tile whose stages start at
-// tile_lo (c_first's slot is 2c+1 when the tile is its LAST segment).
-__device__ __forceinline__ int contributor_slot(int cj, int c_first, int first_slot) {
-    return cj == c_first ? first_slot : 2 * cj;
-}
-
-// Sum, in CTA order (= K order), of the partials of rows m0 .. m0+MB-1 (those
-// below mrows) of one tile row `off` from every contributor; the loads of a
-// block of CB contributors x MB rows are issued together so the reduction
-// costs a few L2 round trips, not one per partial.  `sum` is written for the
-// rows below mrows.
-template <int MB, int CB>
-__device__ __forceinline__ void ordered_partial_sums(const float *part, int slot_elems, int row_stride, int off,
-                                                     int m0, int mrows, int c_first, int c_last, int first_slot,
-                                                     long long T, int G, float (&sum)[MB]) {
-    bool first = true;
-    for (int cb = c_first; cb <= c_last; cb += CB) {
-        float v[CB][MB];
-        bool ok[CB];
-#pragma unroll
-        for (int u = 0; u < CB; ++u) {
-            const int cj = cb + u;
-            ok[u] = cj <= c_last && (T >= G || cta_has_work(T, cj, G));
-            const float *q = part + (size_t)contributor_slot(cj, c_first, first_slot) * slot_elems + off;
-#pragma unroll
-            for (int i = 0; i < MB; ++i)
-                v[u][i] = (ok[u] && m0 + i < mrows) ? ld_cg_f32(q + (size_t)(m0 + i) * row_stride) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < CB; ++u) {
-            if (ok[u]) {
-#pragma unroll
-                for (int i = 0; i < MB; ++i) sum[i] = first ? v[u][i] : sum[i] + v[u][i];
-                first = false;
-            }
-        }
-    }
-}
-
-// Programmatic dependent launch: let the next kernel on the stream begin its
-// prologue, and wait for the previous kernel's completion (and memory).
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 // Before a CTA exits, every TMA copy it issued must have landed: wait for the
 // full barriers of the last min(S, issued) stages, under ONE overall
 // deadline (a healthy run finds them all complete already).
@@ -322,6 +286,12 @@ __device__ __forceinline__ void drain_issued(uint64_t *full_bars, int S, long lo
     }
 }
 
+// ------------------------------------------------------------------ scheduling
+
+__device__ __forceinline__ const TaskDev &task_at(const KParams &p, int t) {
+    return p.tasks ? p.tasks[t] : p.single;
+}
+
 // Tile index -> (column tile g, M-tile mt).
 __device__ __forceinline__ void tile_coords(const TaskDev &T, int tile, int &g, int &mt) {
     if (T.order == 0) {
@@ -333,27 +303,46 @@ __device__ __forceinline__ void tile_coords(const TaskDev &T, int tile, int &g, 
     }
 }
 
-// Incremental walk over a CTA's iterations [lo, hi) in tile-major order:
-// (tile, k-stage kk, column tile g, M-tile mt) with no division per step.
-struct IterWalk {
-    int tile, kk, g, mt;
-    __device__ __forceinline__ void start(const TaskDev &T, long long lo) {
-        tile = (int)(lo / T.kb);
-        kk = (int)(lo - (long long)tile * T.kb);
-        tile_coords(T, tile, g, mt);
+// Claim the next unit of task T (>= n_units: none left).
+__device__ __forceinline__ int claim_unit(const TaskDev &T) {
+    return (int)atom_add_relaxed_gpu(&T.sched[0], 1u);
+}
+
+// Called once per CTA after its failing claim on a task: the last CTA resets
+// the claim counters for the next call (every CTA has claimed by then).
+__device__ __forceinline__ void claims_finished(const TaskDev &T, unsigned int grid) {
+    const unsigned int old = atom_add_acqrel_gpu(&T.sched[1], 1u);
+    if (old == grid - 1) {
+        st_relaxed_gpu(&T.sched[0], 0u);
+        st_relaxed_gpu(&T.sched[1], 0u);
     }
-    __device__ __forceinline__ void next(const TaskDev &T) {
-        if (++kk == T.kb) {
-            kk = 0;
-            ++tile;
-            if (T.order == 0) {
-                if (++mt == T.n_mt) { mt = 0; ++g; }
-            } else {
-                if (++g == T.n_g) { g = 0; ++mt; }
+}
+
+// Sum, in unit order (= K order), of the partials of rows m0 .. m0+MB-1 (those
+// below mrows) of the nu units of one tile, at element `off` of row 0 of each
+// slot.  The loads of a block of CB units x MB rows are issued together, so
+// the reduction costs a few L2 round trips rather than one per partial.
+template <int MB, int CB>
+__device__ __forceinline__ void ordered_unit_sums(const float *tile_slots, int slot_elems, int row_stride, int off,
+                                                  int m0, int mrows, int nu, float (&sum)[MB]) {
+    for (int jb = 0; jb < nu; jb += CB) {
+        float v[CB][MB];
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+            const float *q = tile_slots + (size_t)(jb + u) * slot_elems + off;
+#pragma unroll
+            for (int i = 0; i < MB; ++i)
+                v[u][i] = (jb + u < nu && m0 + i < mrows) ? ld_cg_f32(q + (size_t)(m0 + i) * row_stride) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+            if (jb + u < nu) {
+#pragma unroll
+                for (int i = 0; i < MB; ++i) sum[i] = (jb + u == 0) ? v[u][i] : sum[i] + v[u][i];
             }
         }
     }
-};
+}
 
 // Bounded wait for task `dep` of a chain to have finished all its tiles in
 // this run.  On time-out (or an error elsewhere) records it and returns; the
@@ -377,6 +366,12 @@ __device__ __forceinline__ void wait_dependency(const KParams &p, const TaskDev 
         }
     }
     fence_proxy_async_global();
+}
+
+// Trace stamps: [cta][task][4] = {first stage issued, dependency met, last
+// tile written, SM id}.
+__device__ __forceinline__ void trace_stamp(const KParams &p, int task, int slot, unsigned long long v) {
+    if (p.trace) p.trace[((size_t)blockIdx.x * p.n_tasks + task) * 4 + slot] = v;
 }
 
 #endif  // __CUDACC__

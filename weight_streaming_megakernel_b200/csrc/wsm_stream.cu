@@ -1,15 +1,16 @@
 // wsm_stream.cu -- weight-streaming decode GEMM for M <= 8 on the fp32 FMA
 // pipes: the weight stream lands in shared memory through TMA and each output
 // is a dot product finished by a warp-shuffle reduction.  Persistent, one CTA
-// per SM; same stream-K split, partials and chain readiness as the tcgen05
-// path (wsm_internal.cuh).
+// per SM; same work units, partials and chain readiness as the tcgen05 path
+// (wsm_internal.cuh).
 //
 // The three techniques of the FlyDSL article ("AMD: ROCm Low-Latency-GEMM-
 // Kernel ... MI355X"), as they land on B200:
-//   1. inter-CTA split-K      -> the stream-K split over persistent CTAs;
+//   1. inter-CTA split-K      -> work units of a tile's K range, claimed by
+//                                any CTA, reduced in unit order;
 //   2. intra-CTA K-slicing    -> KW consumer warps own disjoint 256-wide K
 //                                slices of every stage, lanes own 8-wide
-//                                pieces; slices are summed once per tile;
+//                                pieces; slices are summed once per unit;
 //   3. multi-stage LDS pipe   -> a ring of TMA stages with mbarriers, filled
 //                                by one producer warp while 8 warps compute.
 //
@@ -39,11 +40,21 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
     f[7] = __uint_as_float(u.w & 0xFFFF0000u);
 }
 
-__device__ __forceinline__ const TaskDev &task_at(const KParams &p, int t) {
-    return p.tasks ? p.tasks[t] : p.single;
-}
-
 constexpr int kConsBar = 1;
+
+// Barrier among the consumer warps that also ORs a predicate over them.
+__device__ __forceinline__ bool vote_or(bool v, int id, int n) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pc, pr;\n\t"
+        "setp.ne.u32 pc, %1, 0;\n\t"
+        "bar.red.or.pred pr, %2, %3, pc;\n\t"
+        "selp.u32 %0, 1, 0, pr;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
 
 // Transposed butterfly reduction over the 32 lanes of V values per lane.
 // While more than one value is left, each step hands half of them to the
@@ -101,14 +112,13 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
+    __shared__ int stage_meta[kMaxStages][3];   // {task, unit, flags}, written by the producer
     __shared__ float red[2][RG][KW][V];
     __shared__ volatile int abort_flag;
     __shared__ int last_flag;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int G = gridDim.x;
-    const int c = blockIdx.x;
     const int S = p.stages;
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
 
@@ -136,28 +146,19 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
             if (p.pdl == 1) pdl_wait();
             for (int t = 0; t < p.n_tasks && !aborted; ++t) {
                 const TaskDev &T = task_at(p, t);
-                const long long Tt = (long long)T.n_g * T.kb;
-                const long long lo = range_lo(Tt, c, G), hi = range_lo(Tt, c + 1, G);
-                if (lo >= hi) continue;
                 prefetch_tmap(&T.tmW);
                 prefetch_tmap(&T.tmX);
                 const uint64_t pol_w = T.w_evict_first ? policy_evict_first() : policy_evict_normal();
                 bool dep_ok = T.dep < 0 && grid_dep_ok;
                 int pend_s[kMaxStages], pend_k[kMaxStages];
                 int np = 0;
-                if (p.trace) {
-                    p.trace[((size_t)c * p.n_tasks + t) * 4 + 0] = globaltimer();
-                    uint32_t smid;
-                    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-                    p.trace[((size_t)c * p.n_tasks + t) * 4 + 3] = smid;
-                }
                 auto flush = [&]() {
                     if (!grid_dep_ok) {
                         pdl_wait();
                         grid_dep_ok = true;
                     }
                     if (T.dep >= 0) wait_dependency(p, task_at(p, T.dep), t, p.status);
-                    if (p.trace) p.trace[((size_t)c * p.n_tasks + t) * 4 + 1] = globaltimer();
+                    trace_stamp(p, t, 1, globaltimer());
                     for (int i = 0; i < np; ++i) {
                         uint8_t *xs = ring + (size_t)pend_s[i] * p.stage_bytes + p.x_off;
 #pragma unroll
@@ -168,43 +169,69 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     np = 0;
                     dep_ok = true;
                 };
-                IterWalk wk;
-                wk.start(T, lo);
-                for (long long it = lo; it < hi; ++it, wk.next(T)) {
-                    const int g = wk.g, kk = wk.kk;
-                    if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
-                    if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
-                        if (np > 0) flush();
-                        aborted = true;
-                        break;
+                bool first_unit = true;
+                int u = claim_unit(T);
+                while (u < T.n_units) {
+                    if (first_unit) {
+                        trace_stamp(p, t, 0, globaltimer());
+                        trace_stamp(p, t, 3, smid());
+                        first_unit = false;
                     }
-                    uint8_t *st = ring + (size_t)s * p.stage_bytes;
-                    mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
-                    const int k0 = kk * (KW * kStreamBoxK);
-#pragma unroll
-                    for (int kw = 0; kw < KW; ++kw)
-                        tma_load_2d(st + kw * TN * 512, &T.tmW, &full_bar[s], k0 + kw * kStreamBoxK, g * TN, pol_w);
-                    if (dep_ok) {
+                    const int g = u / T.nu;
+                    const int jj = u - g * T.nu;
+                    const int k_begin = jj * T.ku;
+                    const int k_end = min(k_begin + T.ku, T.kb);
+                    int next_u = T.n_units;
+                    for (int kk = k_begin; kk < k_end; ++kk) {
+                        if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
+                        if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
+                            if (np > 0) flush();
+                            aborted = true;
+                            break;
+                        }
+                        uint8_t *st = ring + (size_t)s * p.stage_bytes;
+                        stage_meta[s][0] = t;
+                        stage_meta[s][1] = u;
+                        stage_meta[s][2] = (kk == k_begin ? kMetaFirst : 0) | (kk == k_end - 1 ? kMetaLast : 0);
+                        mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
+                        const int k0 = kk * (KW * kStreamBoxK);
 #pragma unroll
                         for (int kw = 0; kw < KW; ++kw)
-                            tma_load_2d(st + p.x_off + kw * MMAX * 512, &T.tmX, &full_bar[s], k0 + kw * kStreamBoxK, 0,
-                                        pol_x);
-                    } else {
-                        pend_s[np] = s;
-                        pend_k[np] = k0;
-                        ++np;
+                            tma_load_2d(st + kw * TN * 512, &T.tmW, &full_bar[s], k0 + kw * kStreamBoxK, g * TN,
+                                        pol_w);
+                        if (dep_ok) {
+#pragma unroll
+                            for (int kw = 0; kw < KW; ++kw)
+                                tma_load_2d(st + p.x_off + kw * MMAX * 512, &T.tmX, &full_bar[s],
+                                            k0 + kw * kStreamBoxK, 0, pol_x);
+                        } else {
+                            pend_s[np] = s;
+                            pend_k[np] = k0;
+                            ++np;
+                        }
+                        ++issued;
+                        if (++s == S) {
+                            s = 0;
+                            ph ^= 1;
+                        }
+                        if (kk == k_begin) next_u = claim_unit(T);  // claim the next unit while this one streams
                     }
-                    ++issued;
-                    if (++s == S) {
-                        s = 0;
-                        ph ^= 1;
-                    }
+                    if (aborted) break;
+                    u = next_u;
                 }
                 if (np > 0) flush();
-                if (p.trace && T.dep < 0) p.trace[((size_t)c * p.n_tasks + t) * 4 + 1] = globaltimer();
+                if (aborted) break;
+                claims_finished(T, gridDim.x);
+                if (T.dep < 0 && !first_unit) trace_stamp(p, t, 1, globaltimer());
             }
             if (!grid_dep_ok) pdl_wait();
-            // copies in flight must land before exit, abort or not
+            // end-of-work marker for the consumers (a stage with no data)
+            if (!aborted && mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, -1, kSiteEmpty)) {
+                stage_meta[s][0] = 0;
+                stage_meta[s][1] = 0;
+                stage_meta[s][2] = kMetaDone;
+                mbar_arrive(&full_bar[s]);
+            }
             drain_issued(full_bar, S, issued, wlim, p.status);
         }
     } else {
@@ -214,148 +241,136 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
         const int rg = cw / KW;
         const int ctid = threadIdx.x - 32;
         const bool leader = (ctid == 0);
+        // thread ctid < TN*MMAX owns output (row, m) of a tile
+        const int o_m = ctid / TN;
+        const int o_row = ctid - o_m * TN;
+        const bool owner = ctid < TN * MMAX;
         if (p.pdl) pdl_wait();  // Y and the scratch may still be in use by the previous kernel
         int s = 0;
         uint32_t ph = 0;
-        uint32_t seg = 0;
-        bool aborted = false;
-        for (int t = 0; t < p.n_tasks; ++t) {
+        uint32_t unit_i = 0;
+        float acc[RW][MMAX];
+        for (;;) {
+            bool ab = !mbar_wait_bounded(&full_bar[s], ph, &abort_flag, wlim, p.status, -1, kSiteFull);
+            ab = __any_sync(0xffffffffu, ab);
+            const int flags = ab ? kMetaDone : stage_meta[s][2];
+            if (ab || (flags & kMetaDone)) {
+                // every consumer warp leaves at the same point (end marker, or an abort anywhere)
+                vote_or(ab, kConsBar, NCT);
+                break;
+            }
+            const int t = stage_meta[s][0];
+            const int u = stage_meta[s][1];
             const TaskDev &T = task_at(p, t);
-            const long long Tt = (long long)T.n_g * T.kb;
-            const long long lo = range_lo(Tt, c, G), hi = range_lo(Tt, c + 1, G);
             const int M = T.M;
-            long long it = lo;
-            bool wrote_any = false;
-            for (int g = (int)(lo / T.kb); it < hi; ++g) {
-                const long long tile_lo = (long long)g * T.kb, tile_hi = tile_lo + T.kb;
-                const long long seg_start = it;
-                const long long seg_end = tile_hi < hi ? tile_hi : hi;
-                float acc[RW][MMAX];
+            if (flags & kMetaFirst) {
 #pragma unroll
                 for (int r = 0; r < RW; ++r)
 #pragma unroll
                     for (int m = 0; m < MMAX; ++m) acc[r][m] = 0.f;
-                for (; it < seg_end; ++it) {
-                    if (!aborted &&
-                        !mbar_wait_bounded(&full_bar[s], ph, &abort_flag, wlim, p.status, t, kSiteFull))
-                        aborted = true;
-                    aborted = __any_sync(0xffffffffu, aborted);
-                    if (!aborted) {
-                        const uint8_t *st = ring + (size_t)s * p.stage_bytes;
-                        const uint8_t *xs = st + p.x_off + kw * MMAX * 512 + lane * 16;
-                        const uint8_t *ws = st + kw * TN * 512 + (rg * RW) * 512 + lane * 16;
-                        float xv[MMAX][8];
+            }
+            {
+                const uint8_t *st = ring + (size_t)s * p.stage_bytes;
+                const uint8_t *xs = st + p.x_off + kw * MMAX * 512 + lane * 16;
+                const uint8_t *ws = st + kw * TN * 512 + (rg * RW) * 512 + lane * 16;
+                float xv[MMAX][8];
 #pragma unroll
-                        for (int m = 0; m < MMAX; ++m) {
-                            if (m < M) {
-                                const uint4 u = *reinterpret_cast<const uint4 *>(xs + m * 512);
-                                bf16x8_to_f32(u, xv[m]);
-                            } else {
+                for (int m = 0; m < MMAX; ++m) {
+                    if (m < M) {
+                        const uint4 q = *reinterpret_cast<const uint4 *>(xs + m * 512);
+                        bf16x8_to_f32(q, xv[m]);
+                    } else {
 #pragma unroll
-                                for (int j = 0; j < 8; ++j) xv[m][j] = 0.f;
-                            }
-                        }
-#pragma unroll
-                        for (int r = 0; r < RW; ++r) {
-                            const uint4 u = *reinterpret_cast<const uint4 *>(ws + r * 512);
-                            float wf[8];
-                            bf16x8_to_f32(u, wf);
-#pragma unroll
-                            for (int m = 0; m < MMAX; ++m) {
-#pragma unroll
-                                for (int j = 0; j < 8; ++j) acc[r][m] = fmaf(wf[j], xv[m][j], acc[r][m]);
-                            }
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0 && !aborted) mbar_arrive(&empty_bar[s]);
-                    if (++s == S) {
-                        s = 0;
-                        ph ^= 1;
+                        for (int j = 0; j < 8; ++j) xv[m][j] = 0.f;
                     }
                 }
-                // ---- end of segment: lanes -> warps -> tile outputs
-                float v[V];
 #pragma unroll
-                for (int r = 0; r < RW; ++r)
+                for (int r = 0; r < RW; ++r) {
+                    const uint4 q = *reinterpret_cast<const uint4 *>(ws + r * 512);
+                    float wf[8];
+                    bf16x8_to_f32(q, wf);
 #pragma unroll
-                    for (int m = 0; m < MMAX; ++m) v[r * MMAX + m] = acc[r][m];
-                const int base = LR::run(v, lane);
-                const int rb = seg & 1;
-                ++seg;
-                constexpr int lane_mask = (V >= 32) ? 0 : (31 >> LR::H);
-                if ((lane & lane_mask) == 0) {
+                    for (int m = 0; m < MMAX; ++m) {
 #pragma unroll
-                    for (int i = 0; i < LR::OUT; ++i) red[rb][rg][kw][base + i] = v[i];
+                        for (int j = 0; j < 8; ++j) acc[r][m] = fmaf(wf[j], xv[m][j], acc[r][m]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[s]);
+            if (++s == S) {
+                s = 0;
+                ph ^= 1;
+            }
+            if (!(flags & kMetaLast)) continue;
+
+            // ---- end of unit: lanes -> warps -> tile outputs
+            float v[V];
+#pragma unroll
+            for (int r = 0; r < RW; ++r)
+#pragma unroll
+                for (int m = 0; m < MMAX; ++m) v[r * MMAX + m] = acc[r][m];
+            const int base = LR::run(v, lane);
+            const int rb = unit_i & 1;
+            ++unit_i;
+            constexpr int lane_mask = (V >= 32) ? 0 : (31 >> LR::H);
+            if ((lane & lane_mask) == 0) {
+#pragma unroll
+                for (int i = 0; i < LR::OUT; ++i) red[rb][rg][kw][base + i] = v[i];
+            }
+            if (vote_or(false, kConsBar, NCT)) break;  // an abort elsewhere: stop with the others
+            float val = 0.f;
+            if (owner) {
+                const int org = o_row / RW, orr = o_row - org * RW;
+#pragma unroll
+                for (int k = 0; k < KW; ++k) {
+                    const float x = red[rb][org][k][orr * MMAX + o_m];
+                    val = (k == 0) ? x : val + x;
+                }
+            }
+            const int g = u / T.nu;
+            const int n = g * TN + o_row;
+            const bool live = owner && o_m < M && n < T.N;
+            if (T.nu == 1) {
+                if (live) {
+                    const size_t o = (size_t)o_m * T.N + n;
+                    T.Y[o] = __float2bfloat16_rn(val);
+                    if (T.Yf32) T.Yf32[o] = val;
+                }
+                if (T.notify) {
+                    named_bar_sync(kConsBar, NCT);
+                    if (leader) red_release_gpu_add(T.done, 1u);  // release covers the CTA's stores (bar.sync before)
+                }
+            } else {
+                if (owner) T.part[(size_t)u * T.slot_elems + ctid] = val;
+                named_bar_sync(kConsBar, NCT);
+                if (leader) {
+                    // acq_rel: releases this CTA's partial (stored before the barrier) and acquires the
+                    // others' for the last arriver
+                    const unsigned int old = atom_add_acqrel_gpu(&T.tile_cnt[g], 1u);
+                    last_flag = (old == (unsigned int)(T.nu - 1)) ? 1 : 0;
                 }
                 named_bar_sync(kConsBar, NCT);
-                // thread ctid < TN*MMAX owns output (row, m) of this tile
-                const int o_m = ctid / TN;
-                const int o_row = ctid - o_m * TN;
-                const bool owner = ctid < TN * MMAX;
-                float val = 0.f;
-                if (owner) {
-                    const int org = o_row / RW, orr = o_row - org * RW;
-#pragma unroll
-                    for (int k = 0; k < KW; ++k) {
-                        const float x = red[rb][org][k][orr * MMAX + o_m];
-                        val = (k == 0) ? x : val + x;
+                if (last_flag) {
+                    // the leader's acquire + the barrier order these loads after every partial
+                    if (owner) {
+                        float sum[1];
+                        ordered_unit_sums<1, 8>(T.part + (size_t)g * T.nu * T.slot_elems, T.slot_elems, 0, ctid, 0,
+                                                1, T.nu, sum);
+                        if (live) {
+                            const size_t o = (size_t)o_m * T.N + n;
+                            T.Y[o] = __float2bfloat16_rn(sum[0]);
+                            if (T.Yf32) T.Yf32[o] = sum[0];
+                        }
                     }
-                }
-                const int n = g * TN + o_row;
-                const bool live = owner && o_m < M && n < T.N;
-                const bool full_tile = (seg_start == tile_lo) && (seg_end == tile_hi);
-                if (full_tile) {
-                    if (live && !aborted) {
-                        const size_t o = (size_t)o_m * T.N + n;
-                        T.Y[o] = __float2bfloat16_rn(val);
-                        if (T.Yf32) T.Yf32[o] = val;
-                    }
-                    if (T.notify) {
-                        named_bar_sync(kConsBar, NCT);
-                        if (leader && !aborted) red_release_gpu_add(T.done, 1u);  // release covers the CTA's stores (bar.sync before)
-                    }
-                } else {
-                    int c_first, c_last;
-                    const int n_c = tile_contributors(tile_lo, tile_hi, Tt, G, c_first, c_last);
-                    const int my_slot = partial_slot(c, seg_start, lo);
-                    if (owner && !aborted) T.part[(size_t)my_slot * T.slot_elems + ctid] = val;
                     named_bar_sync(kConsBar, NCT);
                     if (leader) {
-                        int last = 0;
-                        if (!aborted) {
-                            // acq_rel: releases the partials this CTA stored before the barrier, and
-                            // acquires the others' partials for the last arriver
-                            const unsigned int old = atom_add_acqrel_gpu(&T.tile_cnt[g], 1u);
-                            last = (old == (unsigned int)(n_c - 1)) ? 1 : 0;
-                        }
-                        last_flag = last;
-                    }
-                    named_bar_sync(kConsBar, NCT);
-                    if (last_flag) {
-                        // the leader's acquire + the barrier order these loads after every partial
-                        if (owner) {
-                            const int first_slot =
-                                (range_lo(Tt, c_first, G) < tile_lo) ? 2 * c_first + 1 : 2 * c_first;
-                            float sum[1];
-                            ordered_partial_sums<1, 8>(T.part, T.slot_elems, 0, ctid, 0, 1, c_first, c_last,
-                                                       first_slot, Tt, G, sum);
-                            if (live) {
-                                const size_t o = (size_t)o_m * T.N + n;
-                                T.Y[o] = __float2bfloat16_rn(sum[0]);
-                                if (T.Yf32) T.Yf32[o] = sum[0];
-                            }
-                        }
-                        named_bar_sync(kConsBar, NCT);
-                        if (leader) {
-                            T.tile_cnt[g] = 0u;
-                            if (T.notify) red_release_gpu_add(T.done, 1u);
-                        }
+                        T.tile_cnt[g] = 0u;
+                        if (T.notify) red_release_gpu_add(T.done, 1u);
                     }
                 }
-                wrote_any = true;
             }
-            if (p.trace && wrote_any && leader) p.trace[((size_t)c * p.n_tasks + t) * 4 + 2] = globaltimer();
+            if (leader) trace_stamp(p, t, 2, globaltimer());
         }
     }
     __syncthreads();
