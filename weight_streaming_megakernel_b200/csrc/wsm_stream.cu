@@ -225,6 +225,9 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 if (T.dep < 0 && !first_unit) trace_stamp(p, t, 1, globaltimer());
             }
             if (!grid_dep_ok) pdl_wait();
+            // copies in flight must land before exit (checked before the end marker below advances one of
+            // these barriers again)
+            drain_issued(full_bar, S, issued, wlim, p.status);
             // end-of-work marker for the consumers (a stage with no data)
             if (!aborted && mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, -1, kSiteEmpty)) {
                 stage_meta[s][0] = 0;
@@ -232,7 +235,6 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 stage_meta[s][2] = kMetaDone;
                 mbar_arrive(&full_bar[s]);
             }
-            drain_issued(full_bar, S, issued, wlim, p.status);
         }
     } else {
         // ------------------------------------------------------------ consumers

@@ -262,6 +262,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 if (T.dep < 0 && !first_unit) trace_stamp(p, t, 1, globaltimer());
             }
             if (!grid_dep_ok) pdl_wait();  // a CTA with no work still orders itself after the previous kernel
+            // copies in flight must land before exit, abort or not (checked before the end marker below
+            // advances one of these barriers again)
+            drain_issued(full_bar, S, issued, wlim, p.status);
             // end-of-work marker for the MMA thread (a stage with no data)
             if (!aborted && mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, -1, kSiteEmpty)) {
                 stage_meta[s][0] = 0;
@@ -269,8 +272,6 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 stage_meta[s][2] = kMetaDone;
                 mbar_arrive(&full_bar[s]);
             }
-            // copies in flight must land before exit, abort or not
-            drain_issued(full_bar, S, issued, wlim, p.status);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
