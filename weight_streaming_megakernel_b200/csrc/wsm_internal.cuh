@@ -5,9 +5,10 @@
 //   A GEMM is cut into tiles: `tile_rows` rows of W (outputs along N) times one
 //   M-tile of X.  A tile's K range is cut into `kb` pipeline stages, and the
 //   stages into `nu` work units of `ku` consecutive stages (the last unit may
-//   be shorter).  Units are numbered tile-major (u = tile * nu + j) and handed
-//   out IN ORDER from one atomic counter per task: each persistent CTA's
-//   producer claims the next unit when it starts the current one.  The SMs of
+//   be shorter).  Units are numbered tile-major (u = tile * nu + j); CTA c
+//   starts with unit c, and the rest are handed out IN ORDER from one atomic
+//   counter per task: each persistent CTA's producer claims its next unit when
+//   it starts the current one.  The SMs of
 //   a B200 do not stream at the same rate (measured: a 2x spread between the
 //   fastest and slowest SMs on the same access pattern), so claiming units
 //   lets every SM work until the task is done instead of the task waiting for
@@ -303,13 +304,14 @@ __device__ __forceinline__ void tile_coords(const TaskDev &T, int tile, int &g, 
     }
 }
 
-// Claim the next unit of task T (>= n_units: none left).
+// Claim the next dynamic unit of task T: the caller adds the number of units
+// handed out statically (unit c to CTA c); a result >= n_units means none left.
 __device__ __forceinline__ int claim_unit(const TaskDev &T) {
     return (int)atom_add_relaxed_gpu(&T.sched[0], 1u);
 }
 
-// Called once per CTA after its failing claim on a task: the last CTA resets
-// the claim counters for the next call (every CTA has claimed by then).
+// Called once per CTA when it has stopped claiming units of a task: the last
+// CTA resets the claim counters for the next call (no CTA claims any more).
 __device__ __forceinline__ void claims_finished(const TaskDev &T, unsigned int grid) {
     const unsigned int old = atom_add_acqrel_gpu(&T.sched[1], 1u);
     if (old == grid - 1) {

@@ -170,7 +170,9 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     dep_ok = true;
                 };
                 bool first_unit = true;
-                int u = claim_unit(T);
+                // the first unit of each CTA is its own index (no atomic); later ones are claimed
+                const int n_static = min((int)gridDim.x, T.n_units);
+                int u = (int)blockIdx.x < T.n_units ? (int)blockIdx.x : T.n_units;
                 while (u < T.n_units) {
                     if (first_unit) {
                         trace_stamp(p, t, 0, globaltimer());
@@ -214,7 +216,12 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                             s = 0;
                             ph ^= 1;
                         }
-                        if (kk == k_begin) next_u = claim_unit(T);  // claim the next unit while this one streams
+                        // claim the next unit while this one streams; the claim counters belong to the
+                        // previous kernel until the grid dependency is resolved
+                        if (kk == k_begin) {
+                            if (!grid_dep_ok) flush();
+                            next_u = claim_unit(T) + n_static;
+                        }
                     }
                     if (aborted) break;
                     u = next_u;
