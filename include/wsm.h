@@ -113,7 +113,7 @@ typedef struct {
     int stage_k;     /* UMMA path: K elements per pipeline stage, 0 = auto,
                         else 64, 128 or 256 */
     int flags;       /* WSM_FLAG_* */
-    int reserved0;
+    int unit_stages; /* pipeline stages per work unit, 0 = auto (see wsm_plan_info) */
     float *Yf32;     /* optional device [M, N] fp32: the result before rounding */
     void *workspace; /* optional caller scratch (device, >= wsm_workspace_bytes,
                         16-byte aligned, zero-filled before its first use; the

@@ -177,6 +177,11 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
     }
     g.stages = std::min(kMaxStages, kRingBudget / g.stage_bytes);
     plan_units(g, g.grid);
+    if (o->unit_stages < 0) return fail(WSM_ERR_INVALID, "bad unit_stages %d", o->unit_stages);
+    if (o->unit_stages > 0) {
+        g.ku = std::min(o->unit_stages, g.kb);
+        g.nu = (g.kb + g.ku - 1) / g.ku;
+    }
     // no more CTAs than work units
     if ((long long)g.grid > g.units()) g.grid = (int)g.units();
     if (g.l2 = o->l2_policy, g.l2 == WSM_L2_AUTO) g.l2 = (g.n_mt > 1) ? WSM_L2_NORMAL : WSM_L2_EVICT_FIRST;
