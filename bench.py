@@ -146,13 +146,15 @@ def setup_inputs(cases, dev, seed_base=0):
     return data
 
 
-def run_gpu(args, rank, world, local_rank):
+def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
     """Timed region: K steps, each one replay of a CUDA graph holding every
     GEMM launch of the step with an external timing event between launches
     (so per-launch durations come from the same timed replays)."""
     import ctypes
     import weight_streaming_megakernel_b200 as wsm
 
+    mode = mode or args.mode
+    n_steps = steps or args.steps
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     cases = workload_cases(args.workload)
@@ -165,9 +167,11 @@ def run_gpu(args, rank, world, local_rank):
     s = stream.cuda_stream
     chain = None
 
-    if args.workload == "chain":
-        tasks = [wsm.Task(x, w, y, dep=i - 1) for i, (c, x, w, y) in enumerate(data)]
-        chain = wsm.Chain(tasks)
+    if mode == "chain":
+        # the whole step is one persistent kernel; the layer chain orders task t after t-1
+        deps = [(i - 1) if args.workload == "chain" else -1 for i in range(len(data))]
+        tasks = [wsm.Task(x, w, y, dep=deps[i]) for i, (c, x, w, y) in enumerate(data)]
+        chain = wsm.Chain(tasks, flags=wsm.FLAG_W_READONLY)
         launches_per_step = 1
 
         def launch(i):
@@ -175,7 +179,7 @@ def run_gpu(args, rank, world, local_rank):
     else:
         calls = []
         for c, x, w, y in data:
-            o = wsm._opts(m_tile=c.m_tile) if c.m_tile else None
+            o = wsm._opts(m_tile=c.m_tile, flags=wsm.FLAG_W_READONLY)
             calls.append((x.data_ptr(), w.data_ptr(), y.data_ptr(), c.M, c.N, c.K, o))
         launches_per_step = len(calls)
 
@@ -204,9 +208,9 @@ def run_gpu(args, rank, world, local_rank):
 
     # one graph per timed step, each with its own in-graph timing events
     nev = launches_per_step + 1
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nev)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nev)] for _ in range(n_steps)]
     graphs = []
-    for k in range(args.steps):
+    for k in range(n_steps):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             step(evs[k])
@@ -221,10 +225,11 @@ def run_gpu(args, rank, world, local_rank):
 
     # clocks: the sampler runs over a loaded window that contains the timed region
     clocks = ClockSampler(local_rank)
-    clocks.start()
+    if extras:
+        clocks.start()
     t_pre = time.time()
     with torch.cuda.stream(stream):
-        while len(clocks.lines) < 2 and time.time() - t_pre < 3.0:
+        while extras and len(clocks.lines) < 2 and time.time() - t_pre < 3.0:
             plain.replay()
             stream.synchronize()
     if world > 1:
@@ -244,7 +249,7 @@ def run_gpu(args, rank, world, local_rank):
     # keep the load on briefly so the window closes under load
     t_post = time.time()
     with torch.cuda.stream(stream):
-        while time.time() - t_post < 0.3:
+        while extras and time.time() - t_post < 0.3:
             plain.replay()
             stream.synchronize()
     clk = clocks.stop()
@@ -253,24 +258,24 @@ def run_gpu(args, rank, world, local_rank):
         tt = torch.tensor([total_ms], device=dev)
         torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(tt.item())
-    ms_per_step = total_ms / args.steps
+    ms_per_step = total_ms / n_steps
     per_launch = [[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(launches_per_step)]
-                  for k in range(args.steps)]
+                  for k in range(n_steps)]
 
     # uninstrumented graph, for reference (not the headline)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         a.record(stream)
-        for _ in range(args.steps):
+        for _ in range(n_steps):
             plain.replay()
         b.record(stream)
     stream.synchronize()
-    plain_ms = a.elapsed_time(b) / args.steps
+    plain_ms = a.elapsed_time(b) / n_steps
 
     # ---- e2e: public API, host buffers, H2D of X and D2H of Y inside the timed region
     e2e = None
-    if not args.no_e2e:
+    if extras and not args.no_e2e:
         hx = [x.cpu().pin_memory() for (_, x, _, _) in data]
         hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for (_, _, _, y) in data]
         h2d = sum(t.numel() * 2 for t in hx)
@@ -283,7 +288,7 @@ def run_gpu(args, rank, world, local_rank):
                 chain.run(s)
             else:
                 for c, x, w, y in data:
-                    wsm.skinny_gemm(x, w, y, m_tile=c.m_tile, stream=s)
+                    wsm.skinny_gemm(x, w, y, m_tile=c.m_tile, flags=wsm.FLAG_W_READONLY, stream=s)
             for (c, x, w, y), h in zip(data, hy):
                 h.copy_(y, non_blocking=True)
 
@@ -297,7 +302,7 @@ def run_gpu(args, rank, world, local_rank):
         b = torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             a.record(stream)
-            for _ in range(args.steps):
+            for _ in range(n_steps):
                 e2e_step()
             b.record(stream)
         stream.synchronize()
@@ -306,7 +311,7 @@ def run_gpu(args, rank, world, local_rank):
             tt = torch.tensor([e_ms], device=dev)
             torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
             e_ms = float(tt.item())
-        e2e = {"value": round(total_bytes * world / (e_ms / args.steps * 1e-3) / 1e9, 2), "unit": "GB/s",
+        e2e = {"value": round(total_bytes * world / (e_ms / n_steps * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     status = wsm.stream_status(stream) if chain is None else chain.status(s)[0]
@@ -369,6 +374,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
     ap.add_argument("--only", default="", help="comma-separated case names (profiling)")
+    ap.add_argument("--mode", default="chain", choices=["chain", "launches"],
+                    help="chain: the step is one persistent gemm_chain kernel; launches: one skinny_gemm per GEMM")
+    ap.add_argument("--no-breakdown", action="store_true", help="skip the per-GEMM single-launch breakdown")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -389,7 +397,9 @@ def main():
               "weight_bytes_per_step": sum(2 * c.N * c.K for c in cases),
               "l2": "inputs larger than L2: every GEMM of a step has its own weights "
                     f"({sum(2 * c.N * c.K for c in cases) / 1e9:.2f} GB per step, L2 126 MB)",
-              "parallelism": f"replicas{world}" if world > 1 else "single"}
+              "parallelism": f"replicas{world}" if world > 1 else "single",
+              "mode": args.mode + (" (one persistent kernel per step, W read-only flag)" if args.mode == "chain"
+                                   else " (one skinny_gemm launch per GEMM, W read-only flag)")}
 
     if args.impl == "reference":
         if rank != 0:
@@ -418,6 +428,15 @@ def main():
     if world > 1:
         torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local_rank))
     r = run_gpu(args, rank, world, local_rank)
+    breakdown = None
+    if args.mode == "chain" and not args.no_breakdown and args.workload != "chain":
+        # informational: the same GEMMs as separate skinny_gemm launches (graph-replayed)
+        rb = run_gpu(args, rank, world, local_rank, mode="launches", steps=min(args.steps, 5), extras=False)
+        import statistics as _st
+        breakdown = {"ms_per_step": round(rb["ms_per_step"], 4),
+                     "value_GBps": round(rb["total_bytes"] / (rb["ms_per_step"] * 1e-3) / 1e9, 1),
+                     "us_per_gemm": {c.name: round(_st.median(row[i] for row in rb["per_launch"]) * 1e3, 2)
+                                     for i, c in enumerate(rb["cases"])}}
 
     # roofline of the weight-streaming kernel: per-launch algorithmic bytes / duration
     import statistics
@@ -427,7 +446,7 @@ def main():
         med = statistics.median(launch_ms)
         fam_bytes, fam_ms = r["total_bytes"], med
         us_per_gemm = {"chain_us": round(med * 1e3, 2), "per_gemm_us_avg": round(med * 1e3 / len(cases), 3)}
-        dominant = "wsm_umma_kernel (chain)"
+        dominant = "wsm_umma_kernel" if max(c.M for c in cases) > 8 else "wsm_stream_kernel"
     else:
         from weight_streaming_megakernel_b200 import plan
         fam = {}
@@ -462,6 +481,7 @@ def main():
                              "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                              "traffic": None},
                 "us_per_gemm": us_per_gemm,
+                "single_launch_breakdown": breakdown,
                 "cpu_baseline": cpu,
                 "e2e": r["e2e"],
                 "gpu_launches": r["launches_per_step"] * args.steps,

@@ -55,10 +55,14 @@ def test_plan_paths_and_geometry():
     assert p["n_tiles"] == 256 and p["k_iters"] == 4096 // p["tile_k"]
     assert p["iters"] == p["n_tiles"] * p["k_iters"] and p["grid"] == 148
     p = wsm.plan(16, 4096, 4096, num_sms=148)
-    assert p["path"] == wsm.PATH_UMMA and p["tile_rows"] == 128 and p["tile_k"] == 64 and p["m_tile"] == 16
-    assert p["n_tiles"] == 32 and p["k_iters"] == 64 and p["m_tiles"] == 1
+    assert p["path"] == wsm.PATH_UMMA and p["tile_rows"] == 128 and p["tile_k"] == 256 and p["m_tile"] == 16
+    assert p["n_tiles"] == 32 and p["k_iters"] == 16 and p["m_tiles"] == 1
+    p = wsm.plan(16, 4096, 4096, num_sms=148, stage_k=64)
+    assert p["tile_k"] == 64 and p["k_iters"] == 64
+    p = wsm.plan(48, 4096, 4096, num_sms=148)
+    assert p["tile_k"] == 128 and p["m_tile"] == 48
     p = wsm.plan(17, 100, 1000, num_sms=148)
-    assert p["m_tile"] == 32 and p["n_tiles"] == 1 and p["k_iters"] == 16
+    assert p["m_tile"] == 32 and p["n_tiles"] == 1 and p["k_iters"] == 4
     p = wsm.plan(8, 4096, 4096, num_sms=148, path=wsm.PATH_UMMA)
     assert p["path"] == wsm.PATH_UMMA and p["m_tile"] == 16
 
@@ -100,16 +104,21 @@ def test_plan_workspace_formula():
 
 
 def test_plan_units():
-    """Enough units for every CTA to take several, none smaller than 32 KB."""
-    for M, N, K in [(1, 4096, 4096), (16, 4096, 4096), (1, 57344, 8192), (16, 24576, 4096), (4, 2112, 7168)]:
-        p = wsm.plan(M, N, K, num_sms=148)
-        stage_bytes = p["tile_rows"] * p["tile_k"] * 2
-        assert 1 <= p["unit_stages"] <= p["k_iters"]
-        assert p["unit_stages"] * stage_bytes >= min(32 << 10, p["k_iters"] * stage_bytes)
-        if p["unit_stages"] > 1 and p["unit_stages"] * stage_bytes > 64 << 10:
-            assert p["units"] >= 8 * 148 // 2
-    p = wsm.plan(1, 57344, 8192, num_sms=148)
-    assert p["units"] >= 8 * 148
+    """At most 4 units per tile on the tensor-core path, 2 on the FMA path;
+    the units cover every stage of a tile exactly once."""
+    for M, N, K in [(1, 4096, 4096), (16, 4096, 4096), (1, 57344, 8192), (16, 24576, 4096), (4, 2112, 7168),
+                    (16, 4096, 12288), (64, 300, 72)]:
+        for path in (wsm.PATH_STREAM, wsm.PATH_UMMA):
+            if path == wsm.PATH_STREAM and M > 8:
+                continue
+            p = wsm.plan(M, N, K, num_sms=148, path=path)
+            nu = -(-p["k_iters"] // p["unit_stages"])
+            assert 1 <= p["unit_stages"] <= p["k_iters"]
+            assert nu <= (4 if path == wsm.PATH_UMMA else 2)
+            assert (nu - 1) * p["unit_stages"] < p["k_iters"] <= nu * p["unit_stages"]
+            assert p["units"] == p["n_tiles"] * p["m_tiles"] * nu
+    p = wsm.plan(16, 4096, 4096, num_sms=148, unit_stages=3)
+    assert p["unit_stages"] == 3 and p["units"] == 32 * 6
 
 
 @pytest.mark.parametrize("M,N,K", [(0, 16, 16), (65, 16, 16), (1, 0, 16), (1, 16, 4), (1, 16, 12), (1, 16, 0)])

@@ -103,20 +103,19 @@ void stream_geo(int mmax, Geo &g) {
     g.threads = 32 * (1 + g.rg * g.kw);
 }
 
-// Work units: ku consecutive stages of one tile.  A unit must be big enough
-// that its partial (when the tile is split) and its claim stay small next to
-// its weight bytes (>= 32 KB and >= 8x the partial), and there should be
-// enough units for every CTA to take several (>= 8 per CTA), so SMs that
-// stream faster take more of them.  Between those, the largest unit wins.
+// Work units: ku consecutive stages of one tile.  Measured on B200 (decode
+// shapes, M = 1 and 16): every unit costs a claim and, when its tile is split,
+// a partial store, a tile-counter round trip and a share of the in-order
+// reduction -- all latency-bound under a saturated memory system -- so the
+// best split is the coarsest one that still spreads a task over the SMs:
+// at most 4 units per tile on the tensor-core path (2 on the FMA path, whose
+// consumer warps run the epilogue themselves).
 void plan_units(Geo &g, int ctas) {
-    const long long wstage = (long long)g.tile_rows * g.tile_k * 2;
-    const long long part_bytes = (long long)g.tile_rows * g.t_m * 4;
-    const long long min_unit = std::max<long long>(32 << 10, 8 * part_bytes);
-    const int min_ku = (int)std::min<long long>(g.kb, std::max<long long>(1, (min_unit + wstage - 1) / wstage));
-    int ku = g.kb;
-    while (ku > min_ku && g.tiles() * ((g.kb + ku - 1) / ku) < 8LL * ctas) ku = std::max(min_ku, (ku + 1) / 2);
-    g.ku = ku;
-    g.nu = (g.kb + ku - 1) / ku;
+    (void)ctas;
+    const int nu_max = (g.path == WSM_PATH_UMMA) ? 4 : 2;
+    const int nu = std::max(1, std::min(nu_max, g.kb));
+    g.ku = (g.kb + nu - 1) / nu;
+    g.nu = (g.kb + g.ku - 1) / g.ku;
 }
 
 // force_mmax: a chain's FMA kernel has one register width for all tasks.
@@ -161,7 +160,7 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
         }
         g.n_mt = (M + g.t_m - 1) / g.t_m;
         int sk = o->stage_k;
-        if (sk == 0) sk = kUmmaBK;
+        if (sk == 0) sk = (g.t_mpad <= 32) ? 256 : 128;  // measured best; wider X tiles leave room for fewer stages
         if (sk != 64 && sk != 128 && sk != 256)
             return fail(WSM_ERR_UNSUPPORTED, "stage_k must be 64, 128 or 256 on the UMMA path (got %d)", sk);
         g.kps = sk / kUmmaBK;

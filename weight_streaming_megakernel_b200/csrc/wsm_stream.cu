@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     const int jj = u - g * T.nu;
                     const int k_begin = jj * T.ku;
                     const int k_end = min(k_begin + T.ku, T.kb);
-                    int next_u = T.n_units;
+                    int next_u = T.n_units - n_static;
                     for (int kk = k_begin; kk < k_end; ++kk) {
                         if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
                         if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
@@ -220,11 +220,11 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                         // previous kernel until the grid dependency is resolved
                         if (kk == k_begin) {
                             if (!grid_dep_ok) flush();
-                            next_u = claim_unit(T) + n_static;
+                            next_u = claim_unit(T);  // first used after this unit's other stages are issued
                         }
                     }
                     if (aborted) break;
-                    u = next_u;
+                    u = next_u + n_static;
                 }
                 if (np > 0) flush();
                 if (aborted) break;

@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     const int k_begin = jj * T.ku;
                     const int k_end = min(k_begin + T.ku, T.kb);
                     const int xy = mt * T.t_m;
-                    int next_u = T.n_units;
+                    int next_u = T.n_units - n_static;
                     for (int kk = k_begin; kk < k_end; ++kk) {
                         // W loads may run ahead of the dependency until the ring is full
                         if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
@@ -256,11 +256,11 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         // previous kernel until the grid dependency is resolved
                         if (kk == k_begin) {
                             if (!grid_dep_ok) flush();
-                            next_u = claim_unit(T) + n_static;
+                            next_u = claim_unit(T);  // first used after this unit's other stages are issued
                         }
                     }
                     if (aborted) break;
-                    u = next_u;
+                    u = next_u + n_static;
                 }
                 if (np > 0) flush();
                 if (aborted) break;
