@@ -162,3 +162,28 @@ def test_independent_tasks_no_deps():
     for t in tasks:
         check_full(t.x.cpu(), t.w.cpu(), t.y, t.yf32)
     ch.close()
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_UMMA, 16), (wsm.PATH_STREAM, 2)])
+def test_dependent_chain_graph_replays(path, M):
+    """A chain captured once in a CUDA graph and replayed many times: the
+    dependency targets come from a device-side run counter, so every replay
+    still orders task t after task t-1."""
+    dims = [1024, 3072, 1024, 2048, 4096]
+    x0, ws, ys, yfs, tasks = dependent_chain(M, dims, seed=21)
+    ch = wsm.Chain(tasks, path=path, flags=wsm.FLAG_W_READONLY)
+    s = torch.cuda.Stream()
+    ch.run(s)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        ch.run(s)
+    for rep in range(4):
+        for y in ys:
+            y.fill_(float("nan"))
+        g.replay()
+        s.synchronize()
+        assert ch.status(s)[0] == wsm.WSM_OK
+        check_dependent(x0, ws, ys, yfs)
+    del g
+    ch.close()

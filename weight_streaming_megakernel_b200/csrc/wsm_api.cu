@@ -111,8 +111,8 @@ void stream_geo(int mmax, Geo &g) {
 // at most 4 units per tile on the tensor-core path (2 on the FMA path, whose
 // consumer warps run the epilogue themselves).
 void plan_units(Geo &g, int ctas) {
-    (void)ctas;
-    const int nu_max = (g.path == WSM_PATH_UMMA) ? 4 : 2;
+    // the FMA path splits a tile only when there are fewer tiles than CTAs
+    const int nu_max = (g.path == WSM_PATH_UMMA) ? 4 : (g.tiles() >= ctas ? 1 : 2);
     const int nu = std::max(1, std::min(nu_max, g.kb));
     g.ku = (g.kb + nu - 1) / nu;
     g.nu = (g.kb + g.ku - 1) / g.ku;
@@ -480,7 +480,7 @@ struct wsm_chain {
     size_t counter_bytes = 0;
     unsigned long long *d_trace = nullptr;
     size_t trace_elems = 0;
-    uint32_t epoch = 0;
+    unsigned int *d_run_ctl = nullptr;   // [runs completed, CTAs done with the current run]
     bool needs_reset = false;
     bool any_dep = false;
     unsigned long long dep_timeout_ns = 0;
@@ -586,7 +586,7 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     kp.kps = g.kps;
     kp.x_stride = g.x_stride;
     kp.pdl = pdl_mode(opts->flags);
-    kp.epoch = 1;
+    kp.run_ctl = nullptr;
     kp.status = reinterpret_cast<int *>(wsb + L.status_off);
     kp.dep_timeout_ns = kDefaultDepTimeoutNs;
     kp.wait_timeout_ns = kPipeTimeoutNs;
@@ -723,6 +723,7 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     };
     uint8_t *base = static_cast<uint8_t *>(ch->d_buf);
     ch->d_status = reinterpret_cast<int *>(base);
+    ch->d_run_ctl = reinterpret_cast<unsigned int *>(base + 64);  // inside the 256-byte status block
     ch->d_counters = reinterpret_cast<unsigned int *>(base + counters_at);
     e = cudaMemset(ch->d_buf, 0, ch->buf_bytes);
     if (e != cudaSuccess) {
@@ -779,11 +780,10 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     if (dev != ch->device) return fail(WSM_ERR_INVALID, "chain was prepared on device %d, current is %d", ch->device, dev);
     if (ch->needs_reset) {
         WSM_CUDA(cudaMemsetAsync(ch->d_counters, 0, ch->counter_bytes, stream));
-        ch->epoch = 0;
+        WSM_CUDA(cudaMemsetAsync(ch->d_run_ctl, 0, 2 * sizeof(unsigned int), stream));
         ch->needs_reset = false;
     }
     if (ch->d_trace) WSM_CUDA(cudaMemsetAsync(ch->d_trace, 0, ch->trace_elems * 8, stream));
-    ch->epoch += 1;
     KParams kp;
     memset(&kp, 0, sizeof kp);
     kp.tasks = ch->d_table;
@@ -794,7 +794,7 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     kp.kps = ch->geo.kps;
     kp.x_stride = ch->geo.x_stride;
     kp.pdl = ch->pdl;
-    kp.epoch = ch->epoch;
+    kp.run_ctl = ch->d_run_ctl;
     kp.dep_target_extra = ch->dep_target_extra;
     kp.status = ch->d_status;
     kp.dep_timeout_ns = ch->dep_timeout_ns;

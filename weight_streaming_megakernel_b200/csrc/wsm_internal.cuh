@@ -85,8 +85,9 @@ struct KParams {
     int stages;                     // ring depth
     int stage_bytes;                // bytes per ring stage
     int x_off;                      // offset of the X part inside a stage
-    uint32_t epoch;                 // chain run number (>= 1)
     uint32_t dep_target_extra;      // 0; a test hook makes every dependency unreachable with it
+    int pad0_;
+    unsigned int *run_ctl;          // chain: [0] runs completed, [1] CTAs done with this run; or nullptr
     int kps;                        // UMMA path: 64-wide K boxes per stage
     int x_stride;                   // UMMA path: bytes between the X boxes of a stage
     int pdl;                        // 0: plain launch; 1: wait for the previous kernel before any
@@ -349,8 +350,12 @@ __device__ __forceinline__ void ordered_unit_sums(const float *tile_slots, int s
 // Bounded wait for task `dep` of a chain to have finished all its tiles in
 // this run.  On time-out (or an error elsewhere) records it and returns; the
 // caller then proceeds with whatever X holds, so the kernel always ends.
+// The run number is read from device memory (not a launch parameter) so a
+// chain captured once in a CUDA graph stays correct over any number of
+// replays; the last CTA to finish a run advances it (chain_run_done).
 __device__ __forceinline__ void wait_dependency(const KParams &p, const TaskDev &D, int task, int *status) {
-    const unsigned int target = p.epoch * (unsigned int)(D.n_g * D.n_mt) + p.dep_target_extra;
+    const unsigned int run = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
+    const unsigned int target = run * (unsigned int)(D.n_g * D.n_mt) + p.dep_target_extra;
     if (ld_acquire_gpu(D.done) - target < 0x80000000u) {  // done >= target (wrap-safe)
         fence_proxy_async_global();
         return;
@@ -368,6 +373,17 @@ __device__ __forceinline__ void wait_dependency(const KParams &p, const TaskDev 
         }
     }
     fence_proxy_async_global();
+}
+
+// Called by one thread per CTA after the CTA has finished all its work of a
+// chain run: the last CTA advances the run counter for the next run.
+__device__ __forceinline__ void chain_run_done(const KParams &p) {
+    if (!p.run_ctl) return;
+    const unsigned int old = atom_add_acqrel_gpu(&p.run_ctl[1], 1u);
+    if (old == gridDim.x - 1) {
+        st_relaxed_gpu(&p.run_ctl[1], 0u);
+        red_release_gpu_add(&p.run_ctl[0], 1u);
+    }
 }
 
 // Trace stamps: [cta][task][4] = {first stage issued, dependency met, last

@@ -383,6 +383,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
         }
     }
     __syncthreads();
+    if (threadIdx.x == 0) chain_run_done(p);
 }
 
 // Kernel for a register width; geometry per MMAX (see the file comment),

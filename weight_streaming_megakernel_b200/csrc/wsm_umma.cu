@@ -455,6 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+    if (threadIdx.x == 0) chain_run_done(p);
 }
 
 }  // namespace wsm
