@@ -165,6 +165,31 @@ size_t wsm_workspace_bytes(int M, int N, int K, const wsm_opts *opts);
  * value is WSM_ERR_TIMEOUT in the second case. */
 wsm_status wsm_stream_status(wsm_stream_t stream, int *code);
 
+/* Bytes of the fixed scratch array skinny_gemm_noalloc uses on each device. */
+#define WSM_NOALLOC_SCRATCH_BYTES (16 << 20)
+
+/* skinny_gemm for callers that cannot allocate device memory after start-up:
+ * an inference loop that reserved its whole memory budget up front, a host
+ * framework whose own allocator must own every device allocation, or a
+ * latency-critical caller that cannot afford cudaMalloc's implicit
+ * synchronisation.  (No counterpart on the pages: it is an interface choice of
+ * this library, not part of the method.)  Same arguments, plan and results as
+ * skinny_gemm; it never calls cudaMalloc or cudaFree.  Its scratch is one
+ * array of WSM_NOALLOC_SCRATCH_BYTES in the library's device image, present
+ * on every GPU that loads the library until the process exits.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Shapes whose plan needs more scratch than the array holds return
+ *    WSM_ERR_UNSUPPORTED with a message naming both sizes (the tensor-core
+ *    plans of M >= 48 on wide N are the ones that do not fit).
+ *  - Every call shares the array.  Each call clears the part that must start
+ *    at zero (queued on `stream`), but calls that overlap on the GPU -- on
+ *    different streams, or on different host threads -- race on it; queue
+ *    them on one stream. */
+wsm_status skinny_gemm_noalloc(const void *X, const void *W, void *Y, int M, int N, int K,
+                               wsm_stream_t stream);
+
 /* ---------------------------------------------------------------- chains */
 
 /* One GEMM of a chain.  dep = -1, or the index of an EARLIER task whose Y

@@ -22,6 +22,7 @@ __all__ = [
     "WSM_ERR_CUDA", "WSM_ERR_TIMEOUT", "PATH_AUTO", "PATH_STREAM", "PATH_UMMA", "ORDER_AUTO", "ORDER_M_MAJOR",
     "ORDER_NAIVE", "L2_AUTO", "L2_EVICT_FIRST", "L2_NORMAL", "FLAG_W_READONLY", "FLAG_NO_PDL", "WsmError", "lib", "skinny_gemm", "plan",
     "workspace_bytes", "stream_status", "Task", "Chain", "gemm_chain", "chain_validate", "last_error",
+    "skinny_gemm_noalloc",
     "abi_version", "HEADER_SYMBOLS",
 ]
 
@@ -37,7 +38,7 @@ FLAG_W_READONLY, FLAG_NO_PDL = 1, 2
 
 # Every function include/wsm.h declares (checked by the CPU tests).
 HEADER_SYMBOLS = (
-    "skinny_gemm", "skinny_gemm_ex", "wsm_plan", "wsm_workspace_bytes", "wsm_stream_status",
+    "skinny_gemm", "skinny_gemm_ex", "wsm_plan", "wsm_workspace_bytes", "wsm_stream_status", "skinny_gemm_noalloc",
     "wsm_chain_create", "wsm_chain_run", "wsm_chain_status", "wsm_chain_trace", "wsm_chain_destroy",
     "gemm_chain", "wsm_chain_validate", "wsm_last_error", "wsm_abi_version",
 )
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
         L.skinny_gemm.restype = st
         L.skinny_gemm_ex.argtypes = [vp, vp, vp, i, i, i, ctypes.POINTER(_Opts), vp]
         L.skinny_gemm_ex.restype = st
+        L.skinny_gemm_noalloc.argtypes = [vp, vp, vp, i, i, i, vp]
+        L.skinny_gemm_noalloc.restype = st
         L.wsm_plan.argtypes = [i, i, i, i, ctypes.POINTER(_Opts), ctypes.POINTER(_PlanInfo)]
         L.wsm_plan.restype = st
         L.wsm_workspace_bytes.argtypes = [i, i, i, ctypes.POINTER(_Opts)]
@@ -197,6 +200,21 @@ def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = No
         o = _opts(path, m_tile, order, l2_policy, grid, yf32, workspace, stage_k, flags, unit_stages)
         _check(lib().skinny_gemm_ex(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, ctypes.byref(o), s),
                "skinny_gemm_ex")
+    return y
+
+
+def skinny_gemm_noalloc(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, stream=None) -> torch.Tensor:
+    """Y = X @ W.T with the library's fixed device scratch array (no device
+    allocation ever; calls that overlap on the GPU race on the array)."""
+    _check_operand("x", x)
+    _check_operand("w", w)
+    _check_operand("y", y)
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] != K or tuple(y.shape) != (M, N):
+        raise ValueError("shapes do not form Y[M,N] = X[M,K] . W[N,K]^T")
+    _check(lib().skinny_gemm_noalloc(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, _stream_handle(stream)),
+           "skinny_gemm_noalloc")
     return y
 
 

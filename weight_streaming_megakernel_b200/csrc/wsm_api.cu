@@ -511,6 +511,11 @@ wsm_status validate_tasks(const wsm_task *tasks, int n) {
 }  // namespace
 }  // namespace wsm
 
+namespace wsm {
+// Sets the message wsm_last_error() returns on this host thread.
+void set_last_error_message(const char *msg) { g_err = msg ? msg : ""; }
+}  // namespace wsm
+
 using namespace wsm;
 
 extern "C" {
