@@ -2,7 +2,7 @@
 
 Acceptance (element by element):
   * fp32 result before rounding:  |Yf32 - Y_ref| <= 1e-3 * S + 1e-6,
-    S = sum_k |X[m,k] W[n,k]| (the tolerance the task definition states);
+    S = sum_k |X[m,k] W[n,k]| (the stated fp32 tolerance of the method);
   * bf16 result: within 1 bf16 ulp of round_bf16(Y_ref), ulps counted in
     the ordered integer encoding (so power-of-two boundaries and signs count
     right; +0 and -0 are equal) -- or, where the two stated tolerances
