@@ -59,7 +59,9 @@ typedef enum {
     WSM_ERR_TIMEOUT = 6      /* a bounded device-side wait ran out (chain dependency or pipeline) */
 } wsm_status;
 
-/* Kernel path. */
+/* Kernel path.  AUTO takes the FMA path for M = 1 up to 512 MiB of weights,
+ * M = 2 up to 180 MiB and M <= 4 up to 64 MiB (measured crossovers on B200),
+ * the tensor-core path otherwise. */
 enum {
     WSM_PATH_AUTO = 0,
     WSM_PATH_STREAM = 1, /* fp32 FMA dot products + warp-shuffle reduction, M <= 8 */
@@ -114,6 +116,10 @@ typedef struct {
                         else 64, 128 or 256 */
     int flags;       /* WSM_FLAG_* */
     int unit_stages; /* pipeline stages per work unit, 0 = auto (see wsm_plan_info) */
+    int tail_tiles;  /* the last tail_tiles tiles of the schedule are split into
+                        smaller units of tail_unit_stages stages, so the end of
+                        the GEMM spreads evenly over the CTAs: 0 = auto, -1 = none */
+    int tail_unit_stages; /* pipeline stages per tail unit, 0 = auto */
     float *Yf32;     /* optional device [M, N] fp32: the result before rounding */
     void *workspace; /* optional caller scratch (device, >= wsm_workspace_bytes,
                         16-byte aligned, zero-filled before its first use; the
@@ -131,8 +137,11 @@ typedef struct {
     int m_tile;        /* X rows per tile (padded to the MMA width on UMMA) */
     int m_tiles;       /* number of M-tiles */
     int n_tiles;       /* number of N-column tiles */
-    int unit_stages;   /* pipeline stages per work unit */
-    long long units;   /* work units (n_tiles * m_tiles * ceil(k_iters / unit_stages)) */
+    int unit_stages;   /* pipeline stages per work unit (head tiles) */
+    int tail_tiles;    /* tiles split into tail units (the last ones of the schedule) */
+    int tail_unit_stages; /* pipeline stages per tail unit */
+    long long units;   /* work units: (n_tiles * m_tiles - tail_tiles) * ceil(k_iters / unit_stages)
+                          + tail_tiles * ceil(k_iters / tail_unit_stages) */
     int k_iters;       /* pipeline stages per tile */
     int stages;        /* shared-memory ring depth */
     int order;         /* WSM_ORDER_M_MAJOR or WSM_ORDER_NAIVE */
@@ -206,7 +215,8 @@ typedef struct {
 } wsm_task;
 
 typedef struct {
-    int path;                  /* WSM_PATH_* for every task (AUTO: by the largest M) */
+    int path;                  /* WSM_PATH_* for every task (AUTO: the FMA path only if AUTO
+                                  picks it for every task at the chain's largest M) */
     int grid;                  /* 0 = one CTA per SM */
     unsigned long long timeout_ns; /* bound on each dependency wait, 0 = 2 s */
     int trace;                 /* nonzero: record per-CTA, per-task %globaltimer stamps */
@@ -215,6 +225,9 @@ typedef struct {
                                    timeout_ns and the run reports WSM_ERR_TIMEOUT */
     int flags;                 /* WSM_FLAG_* (for the whole chain) */
     int stage_k;               /* as in wsm_opts (UMMA path), 0 = auto */
+    int unit_stages;           /* as in wsm_opts, for every task */
+    int tail_tiles;            /* as in wsm_opts, for every task */
+    int tail_unit_stages;      /* as in wsm_opts, for every task */
 } wsm_chain_opts;
 
 typedef struct wsm_chain wsm_chain;  /* opaque prepared chain */

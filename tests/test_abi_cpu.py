@@ -67,6 +67,22 @@ def test_plan_paths_and_geometry():
     assert p["path"] == wsm.PATH_UMMA and p["m_tile"] == 16
 
 
+def test_auto_path_crossovers():
+    """AUTO: FMA path for M = 1 up to 512 MiB of weights, M = 2 up to 180 MiB,
+    M <= 4 up to 64 MiB; tensor cores otherwise."""
+    S, U = wsm.PATH_STREAM, wsm.PATH_UMMA
+    cases = [(1, 4096, 4096, S), (1, 24576, 4096, S), (1, 57344, 8192, U), (2, 4096, 12288, S),
+             (2, 10240, 8192, S), (2, 24576, 4096, U), (4, 4096, 4096, S), (4, 4096, 7168, S),
+             (4, 4096, 12288, U), (3, 6144, 4096, S), (5, 64, 64, U), (8, 4096, 4096, U), (16, 64, 64, U)]
+    for M, N, K, want in cases:
+        assert wsm.plan(M, N, K)["path"] == want, (M, N, K)
+    # exactly at the thresholds
+    assert wsm.plan(1, 32768, 8192)["path"] == S          # 512 MiB
+    assert wsm.plan(1, 32769, 8192)["path"] == U
+    assert wsm.plan(4, 4096, 8192)["path"] == S           # 64 MiB
+    assert wsm.plan(4, 4097, 8192)["path"] == U
+
+
 def test_plan_ring_fits_shared_memory():
     for M in (1, 2, 3, 4, 8, 16, 33, 64):
         p = wsm.plan(M, 4096, 4096, num_sms=148)
@@ -119,6 +135,31 @@ def test_plan_units():
             assert p["units"] == p["n_tiles"] * p["m_tiles"] * nu
     p = wsm.plan(16, 4096, 4096, num_sms=148, unit_stages=3)
     assert p["unit_stages"] == 3 and p["units"] == 32 * 6
+
+
+def test_plan_tail_units():
+    """The last tail_tiles tiles are split into units of tail_unit_stages
+    stages; the head tiles keep unit_stages.  Units and workspace follow."""
+    M, N, K = 16, 4096, 4096          # 32 tiles x 16 stages of 256
+    base = wsm.plan(M, N, K, num_sms=148, path=wsm.PATH_UMMA, tail_tiles=-1)
+    assert base["tail_tiles"] == 0 and base["units"] == 32 * 4
+    p = wsm.plan(M, N, K, num_sms=148, path=wsm.PATH_UMMA, tail_tiles=10, tail_unit_stages=2)
+    assert p["tail_tiles"] == 10 and p["tail_unit_stages"] == 2 and p["unit_stages"] == base["unit_stages"]
+    assert p["units"] == 22 * 4 + 10 * 8
+    assert p["workspace_bytes"] >= p["units"] * 128 * 16 * 4
+    # uneven split: 16 stages in units of 3 -> 6 units per tail tile, the last one short
+    p = wsm.plan(M, N, K, num_sms=148, path=wsm.PATH_UMMA, tail_tiles=5, tail_unit_stages=3)
+    assert p["units"] == 27 * 4 + 5 * 6
+    # more tail tiles than tiles: every tile is a tail tile
+    p = wsm.plan(M, N, K, num_sms=148, path=wsm.PATH_UMMA, tail_tiles=1000, tail_unit_stages=1)
+    assert p["tail_tiles"] == 32 and p["units"] == 32 * 16
+    # the FMA path takes the same options
+    p = wsm.plan(2, 2112, 7168, num_sms=148, path=wsm.PATH_STREAM, tail_tiles=20, tail_unit_stages=1)
+    assert p["tail_tiles"] == 20 and p["units"] == (p["n_tiles"] - 20) * -(-p["k_iters"] // p["unit_stages"]) + 20 * p["k_iters"]
+    for bad in (dict(tail_tiles=-2), dict(tail_unit_stages=-1), dict(unit_stages=-1)):
+        with pytest.raises(wsm.WsmError) as e:
+            wsm.plan(M, N, K, **bad)
+        assert e.value.code == wsm.WSM_ERR_INVALID
 
 
 @pytest.mark.parametrize("M,N,K", [(0, 16, 16), (65, 16, 16), (1, 0, 16), (1, 16, 4), (1, 16, 12), (1, 16, 0)])

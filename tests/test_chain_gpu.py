@@ -68,6 +68,22 @@ def test_dependent_chain(path, M):
     ch.close()
 
 
+@pytest.mark.parametrize("path,M", [(wsm.PATH_UMMA, 16), (wsm.PATH_STREAM, 4)])
+def test_dependent_chain_tail_units(path, M):
+    """Tail units in every task of a data-dependent chain, run twice (the
+    claim counters are reset at the end of each run)."""
+    dims = [1024, 2048, 1024, 3072, 512]
+    x0, ws, ys, yfs, tasks = dependent_chain(M, dims, seed=30 + M)
+    ch = wsm.Chain(tasks, path=path, unit_stages=3, tail_tiles=6, tail_unit_stages=1)
+    for _ in range(2):
+        for y in ys:
+            y.fill_(float("nan"))
+        ch.run()
+        assert ch.status()[0] == wsm.WSM_OK
+        check_dependent(x0, ws, ys, yfs)
+    ch.close()
+
+
 def test_dependent_chain_small_grid_and_empty_ctas():
     """A grid larger than some tasks' stage counts (CTAs with no work for a
     task) and a tiny grid (long per-CTA ranges)."""

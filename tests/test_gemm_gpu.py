@@ -107,6 +107,23 @@ def test_split_patterns(path, M, grid):
     check_full(x, w, y, yf, what=f"grid={grid}")
 
 
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 2), (wsm.PATH_STREAM, 8), (wsm.PATH_UMMA, 16),
+                                    (wsm.PATH_UMMA, 64)])
+def test_tail_units(path, M):
+    """Tail tiles split into smaller units than the head tiles: exact on
+    small-integer inputs (bitwise equal to the unsplit result) and within the
+    bound on random inputs, for several tail sizes, unit sizes and grids."""
+    N, K = 1000, 6144
+    xi, wi = synth.make_int_xw(M, N, K, seed=40 + M)
+    Y_ref, _ = oracle.gemm_ref(xi, wi)
+    x, w = synth.make_xw(M, N, K, seed=50 + M)
+    for tail_tiles, tus, grid in [(1, 1, 0), (5, 2, 0), (1000, 1, 0), (7, 3, 37), (3, 1, 5)]:
+        y, yf = run(xi, wi, path=path, grid=grid, tail_tiles=tail_tiles, tail_unit_stages=tus)
+        assert np.array_equal(yf.cpu().double().numpy(), Y_ref), (tail_tiles, tus, grid)
+        y, yf = run(x, w, path=path, grid=grid, tail_tiles=tail_tiles, tail_unit_stages=tus)
+        check_full(x, w, y, yf, what=f"tail_tiles={tail_tiles} tail_unit_stages={tus} grid={grid}")
+
+
 def test_all_ones_closed_form():
     for path, M in ((wsm.PATH_STREAM, 3), (wsm.PATH_UMMA, 20)):
         K = 256

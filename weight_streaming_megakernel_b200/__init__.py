@@ -53,13 +53,16 @@ class WsmError(RuntimeError):
 class _Opts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("m_tile", ctypes.c_int), ("order", ctypes.c_int),
                 ("l2_policy", ctypes.c_int), ("grid", ctypes.c_int), ("stage_k", ctypes.c_int),
-                ("flags", ctypes.c_int), ("unit_stages", ctypes.c_int), ("Yf32", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+                ("flags", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
+                ("tail_unit_stages", ctypes.c_int), ("Yf32", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
 
 
 class _PlanInfo(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("grid", ctypes.c_int), ("tile_rows", ctypes.c_int),
                 ("tile_k", ctypes.c_int), ("m_tile", ctypes.c_int), ("m_tiles", ctypes.c_int),
-                ("n_tiles", ctypes.c_int), ("unit_stages", ctypes.c_int), ("units", ctypes.c_longlong),
+                ("n_tiles", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
+                ("tail_unit_stages", ctypes.c_int), ("units", ctypes.c_longlong),
                 ("k_iters", ctypes.c_int), ("stages", ctypes.c_int),
                 ("order", ctypes.c_int), ("l2_policy", ctypes.c_int), ("smem_bytes", ctypes.c_int),
                 ("iters", ctypes.c_longlong), ("workspace_bytes", ctypes.c_size_t)]
@@ -74,7 +77,8 @@ class _Task(ctypes.Structure):
 class _ChainOpts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("grid", ctypes.c_int), ("timeout_ns", ctypes.c_ulonglong),
                 ("trace", ctypes.c_int), ("debug_unmet_dependency", ctypes.c_int), ("flags", ctypes.c_int),
-                ("stage_k", ctypes.c_int)]
+                ("stage_k", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
+                ("tail_unit_stages", ctypes.c_int)]
 
 
 _lib = None
@@ -160,10 +164,10 @@ def _check_operand(name, t, dtype=torch.bfloat16):
 
 
 def _opts(path=PATH_AUTO, m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32=None, workspace=None,
-          stage_k=0, flags=0, unit_stages=0):
+          stage_k=0, flags=0, unit_stages=0, tail_tiles=0, tail_unit_stages=0):
     o = _Opts()
     o.path, o.m_tile, o.order, o.l2_policy, o.grid, o.stage_k = path, m_tile, order, l2_policy, grid, stage_k
-    o.flags, o.unit_stages = flags, unit_stages
+    o.flags, o.unit_stages, o.tail_tiles, o.tail_unit_stages = flags, unit_stages, tail_tiles, tail_unit_stages
     o.Yf32 = _ptr(yf32)
     if workspace is not None:
         o.workspace = workspace.data_ptr()
@@ -173,8 +177,8 @@ def _opts(path=PATH_AUTO, m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0,
 
 def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = None, *, path=PATH_AUTO,
                 m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32: Optional[torch.Tensor] = None,
-                workspace: Optional[torch.Tensor] = None, stage_k=0, flags=0, unit_stages=0,
-                stream=None) -> torch.Tensor:
+                workspace: Optional[torch.Tensor] = None, stage_k=0, flags=0, unit_stages=0, tail_tiles=0,
+                tail_unit_stages=0, stream=None) -> torch.Tensor:
     """Y = X @ W.T on the current (or given) stream; returns Y."""
     _check_operand("x", x)
     _check_operand("w", w)
@@ -191,13 +195,14 @@ def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = No
         _check_operand("yf32", yf32, torch.float32)
         if tuple(yf32.shape) != (M, N):
             raise ValueError(f"yf32 must be [{M}, {N}]")
-    plain = (path, m_tile, order, l2_policy, grid, stage_k, flags, unit_stages) == \
-        (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0, 0, 0, 0) and yf32 is None and workspace is None
+    plain = (path, m_tile, order, l2_policy, grid, stage_k, flags, unit_stages, tail_tiles, tail_unit_stages) == \
+        (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0, 0, 0, 0, 0, 0) and yf32 is None and workspace is None
     s = _stream_handle(stream)
     if plain:
         _check(lib().skinny_gemm(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, s), "skinny_gemm")
     else:
-        o = _opts(path, m_tile, order, l2_policy, grid, yf32, workspace, stage_k, flags, unit_stages)
+        o = _opts(path, m_tile, order, l2_policy, grid, yf32, workspace, stage_k, flags, unit_stages, tail_tiles,
+                  tail_unit_stages)
         _check(lib().skinny_gemm_ex(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, ctypes.byref(o), s),
                "skinny_gemm_ex")
     return y
@@ -276,7 +281,8 @@ class Chain:
     """A prepared chain of GEMMs run as one persistent kernel."""
 
     def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
-                 debug_unmet_dependency=False, flags=0, stage_k=0):
+                 debug_unmet_dependency=False, flags=0, stage_k=0, unit_stages=0, tail_tiles=0,
+                 tail_unit_stages=0):
         for i, t in enumerate(tasks):
             _check_operand(f"tasks[{i}].x", t.x)
             _check_operand(f"tasks[{i}].w", t.w)
@@ -287,6 +293,7 @@ class Chain:
         o.path, o.grid, o.timeout_ns, o.trace = path, grid, timeout_ns, 1 if trace else 0
         o.debug_unmet_dependency = 1 if debug_unmet_dependency else 0
         o.flags, o.stage_k = flags, stage_k
+        o.unit_stages, o.tail_tiles, o.tail_unit_stages = unit_stages, tail_tiles, tail_unit_stages
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

@@ -67,7 +67,9 @@ struct Geo {
     int n_g = 0, kb = 0;
     int stage_bytes = 0, x_off = 0, stages = 0;
     int slot_elems = 0;
-    int ku = 1, nu = 1;        // stages per work unit, units per tile
+    int ku = 1, nu = 1;        // head tiles: stages per work unit, units per tile
+    int ku_t = 1, nu_t = 1;    // tail tiles: the same
+    int tail = 0;              // tail tiles (the last ones of the schedule)
     int order = WSM_ORDER_M_MAJOR;
     int l2 = WSM_L2_EVICT_FIRST;
     int grid = 0;
@@ -76,7 +78,8 @@ struct Geo {
     int x_stride = 0;          // UMMA: bytes between X boxes inside a stage
     long long iters() const { return (long long)n_g * n_mt * kb; }
     long long tiles() const { return (long long)n_g * n_mt; }
-    long long units() const { return tiles() * nu; }
+    long long units() const { return (tiles() - tail) * nu + (long long)tail * nu_t; }
+    bool split() const { return nu > 1 || (tail > 0 && nu_t > 1); }
 };
 
 int pow2ceil(int v) {
@@ -90,11 +93,7 @@ bool shape_ok(int M, int N, int K) { return M >= 1 && M <= 64 && N >= 1 && K >= 
 // Stream (FMA) geometry per register width; see wsm_stream.cu.
 void stream_geo(int mmax, Geo &g) {
     g.mmax = mmax;
-    if (mmax <= 2) {
-        g.rw = 4; g.rg = 4; g.kw = 2;
-    } else {
-        g.rw = 8; g.rg = 2; g.kw = 4;
-    }
+    g.rw = 8; g.rg = 2; g.kw = 4;
     g.tile_rows = g.rg * g.rw;                 // 16
     g.tile_k = g.kw * kStreamBoxK;             // 512 or 1024
     g.x_off = g.kw * g.tile_rows * 512;        // W part of a stage
@@ -110,12 +109,43 @@ void stream_geo(int mmax, Geo &g) {
 // best split is the coarsest one that still spreads a task over the SMs:
 // at most 4 units per tile on the tensor-core path (2 on the FMA path, whose
 // consumer warps run the epilogue themselves).
-void plan_units(Geo &g, int ctas) {
-    // the FMA path splits a tile only when there are fewer tiles than CTAs
-    const int nu_max = (g.path == WSM_PATH_UMMA) ? 4 : (g.tiles() >= ctas ? 1 : 2);
-    const int nu = std::max(1, std::min(nu_max, g.kb));
-    g.ku = (g.kb + nu - 1) / nu;
+//
+// Tail: the last tiles of the schedule may be split into smaller units, so
+// the end of a GEMM (which in a chain every dependent task waits for) is
+// spread evenly over CTAs that stream at different speeds.
+wsm_status plan_units(Geo &g, int ctas, int unit_stages, int tail_tiles, int tail_unit_stages) {
+    if (unit_stages < 0) return fail(WSM_ERR_INVALID, "bad unit_stages %d", unit_stages);
+    if (tail_tiles < -1) return fail(WSM_ERR_INVALID, "bad tail_tiles %d", tail_tiles);
+    if (tail_unit_stages < 0) return fail(WSM_ERR_INVALID, "bad tail_unit_stages %d", tail_unit_stages);
+    if (unit_stages > 0) {
+        g.ku = std::min(unit_stages, g.kb);
+    } else {
+        // the FMA path splits a tile only when there are fewer tiles than CTAs
+        const int nu_max = (g.path == WSM_PATH_UMMA) ? 4 : (g.tiles() >= ctas ? 1 : 2);
+        const int nu = std::max(1, std::min(nu_max, g.kb));
+        g.ku = (g.kb + nu - 1) / nu;
+    }
     g.nu = (g.kb + g.ku - 1) / g.ku;
+    long long tt = tail_tiles > 0 ? tail_tiles : 0;  // auto: no tail
+    tt = std::min(tt, g.tiles());
+    g.tail = (int)tt;
+    g.ku_t = tail_unit_stages > 0 ? std::min(tail_unit_stages, g.kb) : std::max(1, g.ku / 4);
+    if (g.tail == 0) g.ku_t = g.ku;
+    g.nu_t = (g.kb + g.ku_t - 1) / g.ku_t;
+    return WSM_OK;
+}
+
+// Automatic path choice.  Measured on B200 (graph-replayed back-to-back
+// launches of decode shapes, M = 1..8, weights 30 MB .. 940 MB): the FMA path
+// wins while its arithmetic per weight byte stays light -- M = 1 up to about
+// 0.5 GB of weights, M = 2 up to about 180 MB, M <= 4 up to about 64 MB --
+// and the tensor-core path wins everywhere else (at M >= 5 always).
+int auto_path(int M, long long w_bytes) {
+    const long long MB = 1ll << 20;
+    if (M == 1 && w_bytes <= 512 * MB) return WSM_PATH_STREAM;
+    if (M == 2 && w_bytes <= 180 * MB) return WSM_PATH_STREAM;
+    if (M <= 4 && w_bytes <= 64 * MB) return WSM_PATH_STREAM;
+    return WSM_PATH_UMMA;
 }
 
 // force_mmax: a chain's FMA kernel has one register width for all tasks.
@@ -132,7 +162,7 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
     if (o->l2_policy < 0 || o->l2_policy > WSM_L2_NORMAL) return fail(WSM_ERR_INVALID, "bad l2_policy %d", o->l2_policy);
     if (o->grid < 0) return fail(WSM_ERR_INVALID, "bad grid %d", o->grid);
     if (o->flags & ~(WSM_FLAG_W_READONLY | WSM_FLAG_NO_PDL)) return fail(WSM_ERR_INVALID, "bad flags %#x", o->flags);
-    if (path == WSM_PATH_AUTO) path = (M <= 8) ? WSM_PATH_STREAM : WSM_PATH_UMMA;
+    if (path == WSM_PATH_AUTO) path = auto_path(M, 2ll * N * K);
     g = Geo{};
     g.path = path;
     g.grid = (o->grid > 0) ? std::min(o->grid, num_sms) : num_sms;
@@ -172,15 +202,11 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
         g.x_off = g.kps * kUmmaRows * kUmmaBK * 2;                  // W boxes, 16 KB each
         g.stage_bytes = g.x_off + g.kps * g.x_stride;
         g.slot_elems = kUmmaRows * g.t_mpad;
-        g.threads = 192;
+        g.threads = 64 + 2 * 128;   // producer, MMA, two epilogue warp sets
     }
     g.stages = std::min(kMaxStages, kRingBudget / g.stage_bytes);
-    plan_units(g, g.grid);
-    if (o->unit_stages < 0) return fail(WSM_ERR_INVALID, "bad unit_stages %d", o->unit_stages);
-    if (o->unit_stages > 0) {
-        g.ku = std::min(o->unit_stages, g.kb);
-        g.nu = (g.kb + g.ku - 1) / g.ku;
-    }
+    wsm_status st = plan_units(g, g.grid, o->unit_stages, o->tail_tiles, o->tail_unit_stages);
+    if (st != WSM_OK) return st;
     // no more CTAs than work units
     if ((long long)g.grid > g.units()) g.grid = (int)g.units();
     if (g.l2 = o->l2_policy, g.l2 == WSM_L2_AUTO) g.l2 = (g.n_mt > 1) ? WSM_L2_NORMAL : WSM_L2_EVICT_FIRST;
@@ -208,7 +234,7 @@ WsLayout ws_layout_of(size_t bytes) {
 }
 // counters: [kSchedWords claim counters][one arrival counter per tile]
 size_t ws_counter_bytes(const Geo &g) { return ((size_t)kSchedWords + (size_t)g.tiles()) * 4; }
-size_t ws_partial_bytes(const Geo &g) { return g.nu > 1 ? (size_t)g.units() * g.slot_elems * 4 : 0; }
+size_t ws_partial_bytes(const Geo &g) { return g.split() ? (size_t)g.units() * g.slot_elems * 4 : 0; }
 bool ws_fits(const Geo &g, size_t bytes) {
     if (bytes < 512) return false;
     const WsLayout L = ws_layout_of(bytes);
@@ -233,6 +259,8 @@ void fill_plan_info(const Geo &g, wsm_plan_info *out) {
     out->m_tiles = g.n_mt;
     out->n_tiles = g.n_g;
     out->unit_stages = g.ku;
+    out->tail_tiles = g.tail;
+    out->tail_unit_stages = g.ku_t;
     out->units = g.units();
     out->k_iters = g.kb;
     out->stages = g.stages;
@@ -374,6 +402,10 @@ wsm_status fill_task(TaskDev &T, const Geo &g, const void *X, const void *W, voi
     T.slot_elems = g.slot_elems;
     T.ku = g.ku;
     T.nu = g.nu;
+    T.t_head = (int)(g.tiles() - g.tail);
+    T.u_head = T.t_head * g.nu;
+    T.ku_t = g.ku_t;
+    T.nu_t = g.nu_t;
     T.n_units = (int)g.units();
     return WSM_OK;
 }
@@ -655,7 +687,13 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     if ((st = dev_info(dev, &d)) != WSM_OK) return st;
     int maxM = 0;
     for (int i = 0; i < n; ++i) maxM = std::max(maxM, tasks[i].M);
-    int path = opts->path == WSM_PATH_AUTO ? (maxM <= 8 ? WSM_PATH_STREAM : WSM_PATH_UMMA) : opts->path;
+    // AUTO: the FMA path only if it is the automatic choice for every task at the chain's largest M
+    int path = opts->path;
+    if (path == WSM_PATH_AUTO) {
+        path = WSM_PATH_STREAM;
+        for (int i = 0; i < n; ++i)
+            if (auto_path(maxM, 2ll * tasks[i].N * tasks[i].K) != WSM_PATH_STREAM) path = WSM_PATH_UMMA;
+    }
     if (path == WSM_PATH_STREAM && maxM > 8) return fail(WSM_ERR_UNSUPPORTED, "the FMA path takes M <= 8 (max M=%d)", maxM);
 
     std::unique_ptr<wsm_chain> ch(new wsm_chain());
@@ -696,7 +734,10 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     ch->geo = ring;
 
     // work units per task, planned for the chain's grid
-    for (auto &g : geos) plan_units(g, chain_grid);
+    for (int i = 0; i < n; ++i)
+        if ((st = plan_units(geos[i], chain_grid, opts->unit_stages, opts->tail_tiles, opts->tail_unit_stages)) !=
+            WSM_OK)
+            return fail(st, "task %d: %s", i, g_err.c_str());
     // scratch: status | counters (per task: claim counters + tile counters; then done counters) | partials
     std::vector<size_t> cnt_off(n), part_off(n);
     size_t ncnt = 0;

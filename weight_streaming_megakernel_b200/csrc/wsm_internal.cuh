@@ -39,6 +39,7 @@ constexpr int kUmmaMaxN = 64;      // largest MMA N (= X rows per tile)
 constexpr int kStreamBoxK = 256;   // K elements per TMA box on the FMA path
 constexpr int kStatusWords = 4;    // [0] error code, [1] failing task, [2] failing CTA, [3] site
 constexpr int kSchedWords = 2;     // per task: [0] next unit to claim, [1] CTAs done claiming
+constexpr int kClaimLead = 4;      // a CTA claims its next unit this many stages before its unit ends
 
 // Error sites recorded in status[3].
 enum : int { kSiteNone = 0, kSiteDep = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteAcc = 4, kSiteDrain = 5 };
@@ -67,9 +68,17 @@ struct __align__(64) TaskDev {
     int t_m;                    // X rows per M-tile
     int t_mpad;                 // X rows loaded per M-tile (UMMA: multiple of 16)
     int kb;                     // stages per tile
-    int ku;                     // stages per unit
-    int nu;                     // units per tile
-    int n_units;                // n_g * n_mt * nu
+    // Work units.  The first t_head tiles of the schedule are split into nu
+    // units of ku stages (u_head = t_head * nu units), the remaining tiles
+    // into nu_t units of ku_t stages: big units first, small ones last, so the
+    // end of a task is spread evenly over the CTAs.
+    int ku;                     // stages per head unit
+    int nu;                     // units per head tile
+    int t_head;                 // head tiles
+    int u_head;                 // t_head * nu
+    int ku_t;                   // stages per tail unit
+    int nu_t;                   // units per tail tile
+    int n_units;                // u_head + (n_g * n_mt - t_head) * nu_t
     int order;                  // 0: M-tile inner (M-major), 1: M-tile outer
     int notify;                 // bump `done` after each finished tile
     int w_evict_first;          // L2 policy of the weight loads
@@ -305,14 +314,43 @@ __device__ __forceinline__ void tile_coords(const TaskDev &T, int tile, int &g, 
     }
 }
 
+// Work unit u of task T: its tile, the tile's first unit and unit count (its
+// partial slots are u0 .. u0 + nu - 1, in K order) and its stage range.
+struct UnitSpan {
+    int tile, u0, nu, k_begin, k_end;
+};
+__device__ __forceinline__ UnitSpan unit_span(const TaskDev &T, int u) {
+    UnitSpan r;
+    int j, ku;
+    if (u < T.u_head) {
+        r.tile = u / T.nu;
+        j = u - r.tile * T.nu;
+        r.nu = T.nu;
+        ku = T.ku;
+    } else {
+        const int v = u - T.u_head;
+        const int tt = v / T.nu_t;
+        r.tile = T.t_head + tt;
+        j = v - tt * T.nu_t;
+        r.nu = T.nu_t;
+        ku = T.ku_t;
+    }
+    r.u0 = u - j;
+    r.k_begin = j * ku;
+    r.k_end = min(r.k_begin + ku, T.kb);
+    return r;
+}
+
 // Claim the next dynamic unit of task T: the caller adds the number of units
 // handed out statically (unit c to CTA c); a result >= n_units means none left.
 __device__ __forceinline__ int claim_unit(const TaskDev &T) {
     return (int)atom_add_relaxed_gpu(&T.sched[0], 1u);
 }
 
-// Called once per CTA when it has stopped claiming units of a task: the last
-// CTA resets the claim counters for the next call (no CTA claims any more).
+// Single GEMM: called once per CTA when it has stopped claiming units; the
+// last CTA resets the claim counters for the next call (no CTA claims any
+// more).  A chain resets all its tasks' claim counters at the end of the run
+// instead (chain_run_done), so no CTA waits on this atomic between tasks.
 __device__ __forceinline__ void claims_finished(const TaskDev &T, unsigned int grid) {
     const unsigned int old = atom_add_acqrel_gpu(&T.sched[1], 1u);
     if (old == grid - 1) {
@@ -376,11 +414,13 @@ __device__ __forceinline__ void wait_dependency(const KParams &p, const TaskDev 
 }
 
 // Called by one thread per CTA after the CTA has finished all its work of a
-// chain run: the last CTA advances the run counter for the next run.
+// chain run: the last CTA (every other CTA has stopped claiming) resets the
+// tasks' claim counters and advances the run counter for the next run.
 __device__ __forceinline__ void chain_run_done(const KParams &p) {
     if (!p.run_ctl) return;
     const unsigned int old = atom_add_acqrel_gpu(&p.run_ctl[1], 1u);
     if (old == gridDim.x - 1) {
+        for (int t = 0; t < p.n_tasks; ++t) st_relaxed_gpu(&task_at(p, t).sched[0], 0u);
         st_relaxed_gpu(&p.run_ctl[1], 0u);
         red_release_gpu_add(&p.run_ctl[0], 1u);
     }

@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
             uint32_t ph = 0;
             long long issued = 0;
             bool aborted = false;
+            bool slot_ok = false;  // the wait for ring slot s has already succeeded
             bool grid_dep_ok = p.pdl != 2;
             if (p.pdl == 1) pdl_wait();
             for (int t = 0; t < p.n_tasks && !aborted; ++t) {
@@ -169,6 +170,19 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     np = 0;
                     dep_ok = true;
                 };
+                // Wait for ring slot s.  W loads may run ahead of the dependency until the ring is full;
+                // then the pending X loads go out first (every issued stage must be able to complete).
+                auto take_slot = [&]() -> bool {
+                    if (slot_ok) return true;
+                    if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
+                    if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
+                        if (np > 0) flush();
+                        aborted = true;
+                        return false;
+                    }
+                    slot_ok = true;
+                    return true;
+                };
                 bool first_unit = true;
                 // the first unit of each CTA is its own index (no atomic); later ones are claimed
                 const int n_static = min((int)gridDim.x, T.n_units);
@@ -179,18 +193,15 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                         trace_stamp(p, t, 3, smid());
                         first_unit = false;
                     }
-                    const int g = u / T.nu;
-                    const int jj = u - g * T.nu;
-                    const int k_begin = jj * T.ku;
-                    const int k_end = min(k_begin + T.ku, T.kb);
+                    const UnitSpan us = unit_span(T, u);
+                    const int g = us.tile;
+                    const int k_begin = us.k_begin;
+                    const int k_end = us.k_end;
                     int next_u = T.n_units - n_static;
+                    bool claimed = false;
                     for (int kk = k_begin; kk < k_end; ++kk) {
-                        if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
-                        if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
-                            if (np > 0) flush();
-                            aborted = true;
-                            break;
-                        }
+                        if (!take_slot()) break;
+                        slot_ok = false;
                         uint8_t *st = ring + (size_t)s * p.stage_bytes;
                         stage_meta[s][0] = t;
                         stage_meta[s][1] = u;
@@ -216,19 +227,29 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                             s = 0;
                             ph ^= 1;
                         }
-                        // claim the next unit while this one streams; the claim counters belong to the
-                        // previous kernel until the grid dependency is resolved
-                        if (kk == k_begin) {
-                            if (!grid_dep_ok) flush();
-                            next_u = claim_unit(T);  // first used after this unit's other stages are issued
+                        // claim the next unit kClaimLead stages before this one ends: early enough to
+                        // hide the claim's round trip, late enough not to hold work a faster CTA could
+                        // take (the claim counters belong to the previous kernel until the grid
+                        // dependency is resolved)
+                        if (!claimed && grid_dep_ok && k_end - kk <= kClaimLead) {
+                            next_u = claim_unit(T);
+                            claimed = true;
                         }
                     }
                     if (aborted) break;
+                    if (!claimed) {
+                        // the first unit streamed completely before the grid dependency was resolved
+                        if (!grid_dep_ok) flush();
+                        next_u = claim_unit(T);
+                    }
+                    // whatever comes next needs a free slot: wait for it before the claim's result is used,
+                    // so the claim's round trip overlaps the wait
+                    if (!take_slot()) break;
                     u = next_u + n_static;
                 }
                 if (np > 0) flush();
                 if (aborted) break;
-                claims_finished(T, gridDim.x);
+                if (!p.run_ctl) claims_finished(T, gridDim.x);
                 if (T.dep < 0 && !first_unit) trace_stamp(p, t, 1, globaltimer());
             }
             if (!grid_dep_ok) pdl_wait();
@@ -236,7 +257,8 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
             // these barriers again)
             drain_issued(full_bar, S, issued, wlim, p.status);
             // end-of-work marker for the consumers (a stage with no data)
-            if (!aborted && mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, -1, kSiteEmpty)) {
+            if (!aborted && (slot_ok || mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, -1,
+                                                          kSiteEmpty))) {
                 stage_meta[s][0] = 0;
                 stage_meta[s][1] = 0;
                 stage_meta[s][2] = kMetaDone;
@@ -337,10 +359,11 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     val = (k == 0) ? x : val + x;
                 }
             }
-            const int g = u / T.nu;
+            const UnitSpan us = unit_span(T, u);
+            const int g = us.tile;
             const int n = g * TN + o_row;
             const bool live = owner && o_m < M && n < T.N;
-            if (T.nu == 1) {
+            if (us.nu == 1) {
                 if (live) {
                     const size_t o = (size_t)o_m * T.N + n;
                     T.Y[o] = __float2bfloat16_rn(val);
@@ -357,15 +380,15 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     // acq_rel: releases this CTA's partial (stored before the barrier) and acquires the
                     // others' for the last arriver
                     const unsigned int old = atom_add_acqrel_gpu(&T.tile_cnt[g], 1u);
-                    last_flag = (old == (unsigned int)(T.nu - 1)) ? 1 : 0;
+                    last_flag = (old == (unsigned int)(us.nu - 1)) ? 1 : 0;
                 }
                 named_bar_sync(kConsBar, NCT);
                 if (last_flag) {
                     // the leader's acquire + the barrier order these loads after every partial
                     if (owner) {
                         float sum[1];
-                        ordered_unit_sums<1, 8>(T.part + (size_t)g * T.nu * T.slot_elems, T.slot_elems, 0, ctid, 0,
-                                                1, T.nu, sum);
+                        ordered_unit_sums<1, 8>(T.part + (size_t)us.u0 * T.slot_elems, T.slot_elems, 0, ctid, 0,
+                                                1, us.nu, sum);
                         if (live) {
                             const size_t o = (size_t)o_m * T.N + n;
                             T.Y[o] = __float2bfloat16_rn(sum[0]);
@@ -386,12 +409,14 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
     if (threadIdx.x == 0) chain_run_done(p);
 }
 
-// Kernel for a register width; geometry per MMAX (see the file comment),
-// T_N = 16 rows for all.  Must agree with stream_geo() in wsm_api.cu.
+// Kernel for a register width: 8 rows per warp, 2 row groups, 4 K-slices
+// (T_N = 16 rows, T_K = 1024) for every MMAX; measured on B200, the wide
+// stage beats 4 x 4 x 2 (T_K = 512) at M = 1 and 2 as well.  Must agree with
+// stream_geo() in wsm_api.cu.
 const void *stream_kernel_ptr(int mmax) {
     switch (mmax) {
-        case 1: return reinterpret_cast<const void *>(&wsm_stream_kernel<1, 4, 4, 2>);
-        case 2: return reinterpret_cast<const void *>(&wsm_stream_kernel<2, 4, 4, 2>);
+        case 1: return reinterpret_cast<const void *>(&wsm_stream_kernel<1, 8, 2, 4>);
+        case 2: return reinterpret_cast<const void *>(&wsm_stream_kernel<2, 8, 2, 4>);
         case 4: return reinterpret_cast<const void *>(&wsm_stream_kernel<4, 8, 2, 4>);
         case 8: return reinterpret_cast<const void *>(&wsm_stream_kernel<8, 8, 2, 4>);
         default: return nullptr;

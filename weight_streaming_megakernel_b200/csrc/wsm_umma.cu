@@ -120,13 +120,64 @@ __device__ __forceinline__ bool vote_or(bool v, int id, int n) {
     return r != 0;
 }
 
-constexpr int kThreads = 192;
 constexpr int kEpiWarp0 = 2;
-constexpr int kEpiThreads = 128;
-constexpr int kEpiBar = 1;          // named barrier id of the epilogue warps
-constexpr uint32_t kTmemCols = 2 * kUmmaMaxN;   // two accumulator buffers
+constexpr int kEpiSets = 2;         // two independent epilogue warp sets (units alternate between them)
+constexpr int kEpiThreads = 128;    // per set: four warps, one per TMEM lane quadrant
+constexpr int kThreads = 64 + kEpiSets * kEpiThreads;
+constexpr int kAccBufs = 4;         // accumulators in TMEM: the MMA can run up to three units ahead
+constexpr uint32_t kTmemCols = kAccBufs * kUmmaMaxN;
 
-__device__ __forceinline__ void epi_bar() { named_bar_sync(kEpiBar, kEpiThreads); }
+__device__ __forceinline__ void epi_bar(int set) { named_bar_sync(1 + set, kEpiThreads); }
+
+// The last unit of a split tile adds the tile's nu partials (slots u0 ..
+// u0 + nu - 1) for its row, in unit order (= K order).  Partial slots are
+// [128 rows][t_mpad] floats, so a thread's values are contiguous: 16-byte
+// loads, CB units x MB rows in flight.
+template <int MB, int CB>
+__device__ __forceinline__ void reduce_row_partials(const TaskDev &T, int u0, int nu, int row, int mrows, int m0,
+                                                    int n) {
+    const float *base = T.part + (size_t)u0 * T.slot_elems + (size_t)row * T.t_mpad;
+    for (int mb = 0; mb < mrows; mb += MB) {
+        float sum[MB];
+#pragma unroll
+        for (int i = 0; i < MB; ++i) sum[i] = 0.f;
+        for (int jb = 0; jb < nu; jb += CB) {
+            float4 v[CB][MB / 4];
+#pragma unroll
+            for (int u = 0; u < CB; ++u) {
+                const float4 *q = reinterpret_cast<const float4 *>(base + (size_t)(jb + u) * T.slot_elems + mb);
+#pragma unroll
+                for (int i = 0; i < MB / 4; ++i)
+                    v[u][i] = (jb + u < nu && mb + 4 * i < mrows) ? __ldcg(q + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < CB; ++u) {
+                if (jb + u < nu) {
+#pragma unroll
+                    for (int i = 0; i < MB / 4; ++i) {
+                        if (jb + u == 0) {
+                            sum[4 * i] = v[u][i].x; sum[4 * i + 1] = v[u][i].y;
+                            sum[4 * i + 2] = v[u][i].z; sum[4 * i + 3] = v[u][i].w;
+                        } else {
+                            sum[4 * i] += v[u][i].x; sum[4 * i + 1] += v[u][i].y;
+                            sum[4 * i + 2] += v[u][i].z; sum[4 * i + 3] += v[u][i].w;
+                        }
+                    }
+                }
+            }
+        }
+        if (n < T.N) {
+#pragma unroll
+            for (int i = 0; i < MB; ++i) {
+                if (mb + i < mrows) {
+                    const size_t o = (size_t)(m0 + mb + i) * T.N + n;
+                    T.Y[o] = __float2bfloat16_rn(sum[i]);
+                    if (T.Yf32) T.Yf32[o] = sum[i];
+                }
+            }
+        }
+    }
+}
 
 }  // namespace
 
@@ -134,14 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
-    __shared__ __align__(8) uint64_t accf_bar[2];
-    __shared__ __align__(8) uint64_t acce_bar[2];
+    __shared__ __align__(8) uint64_t accf_bar[kAccBufs];
+    __shared__ __align__(8) uint64_t acce_bar[kAccBufs];
     __shared__ __align__(8) uint64_t drain_bar;
     __shared__ int stage_meta[kMaxStages][3];   // {task, unit, flags}, written by the producer
-    __shared__ int acc_meta[2][3];              // {task, unit, flags}, written by the MMA thread
+    __shared__ int acc_meta[kAccBufs][3];       // {task, unit, flags}, written by the MMA thread
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_flag;
-    __shared__ int last_flag;
+    __shared__ int last_flag[kEpiSets];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -154,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kAccBufs; ++b) {
             mbar_init(&accf_bar[b], 2);                  // tcgen05.commit + the MMA thread's metadata arrive
             mbar_init(&acce_bar[b], kEpiThreads / 32);
         }
@@ -178,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             uint32_t ph = 0;
             long long issued = 0;
             bool aborted = false;
+            bool slot_ok = false;           // the wait for ring slot s has already succeeded
             bool grid_dep_ok = p.pdl != 2;  // mode 2 streams W before the previous kernel completes
             if (p.pdl == 1) pdl_wait();
             for (int t = 0; t < p.n_tasks && !aborted; ++t) {
@@ -202,6 +254,19 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     np = 0;
                     dep_ok = true;
                 };
+                // Wait for ring slot s.  W loads may run ahead of the dependency until the ring is full;
+                // then the pending X loads go out first (every issued stage must be able to complete).
+                auto take_slot = [&]() -> bool {
+                    if (slot_ok) return true;
+                    if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
+                    if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
+                        if (np > 0) flush();
+                        aborted = true;
+                        return false;
+                    }
+                    slot_ok = true;
+                    return true;
+                };
                 bool first_unit = true;
                 // the first unit of each CTA is its own index (no atomic); later ones are claimed
                 const int n_static = min((int)gridDim.x, T.n_units);
@@ -212,26 +277,19 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         trace_stamp(p, t, 3, smid());
                         first_unit = false;
                     }
-                    const int tile = u / T.nu;
-                    const int jj = u - tile * T.nu;
+                    const UnitSpan us = unit_span(T, u);
                     int g, mt;
-                    tile_coords(T, tile, g, mt);
-                    const int k_begin = jj * T.ku;
-                    const int k_end = min(k_begin + T.ku, T.kb);
+                    tile_coords(T, us.tile, g, mt);
                     const int xy = mt * T.t_m;
                     int next_u = T.n_units - n_static;
-                    for (int kk = k_begin; kk < k_end; ++kk) {
-                        // W loads may run ahead of the dependency until the ring is full
-                        if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
-                        if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
-                            if (np > 0) flush();  // every issued stage must be able to complete
-                            aborted = true;
-                            break;
-                        }
+                    bool claimed = false;
+                    for (int kk = us.k_begin; kk < us.k_end; ++kk) {
+                        if (!take_slot()) break;
+                        slot_ok = false;
                         uint8_t *st = ring + (size_t)s * p.stage_bytes;
                         stage_meta[s][0] = t;
                         stage_meta[s][1] = u;
-                        stage_meta[s][2] = (kk == k_begin ? kMetaFirst : 0) | (kk == k_end - 1 ? kMetaLast : 0);
+                        stage_meta[s][2] = (kk == us.k_begin ? kMetaFirst : 0) | (kk == us.k_end - 1 ? kMetaLast : 0);
                         mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
                         const int k0 = kk * p.kps * kUmmaBK;
                         for (int j = 0; j < p.kps; ++j)
@@ -252,19 +310,29 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                             s = 0;
                             ph ^= 1;
                         }
-                        // claim the next unit while this one streams; the claim counters belong to the
-                        // previous kernel until the grid dependency is resolved
-                        if (kk == k_begin) {
-                            if (!grid_dep_ok) flush();
-                            next_u = claim_unit(T);  // first used after this unit's other stages are issued
+                        // claim the next unit kClaimLead stages before this one ends: early enough to
+                        // hide the claim's round trip, late enough not to hold work a faster CTA could
+                        // take (the claim counters belong to the previous kernel until the grid
+                        // dependency is resolved)
+                        if (!claimed && grid_dep_ok && us.k_end - kk <= kClaimLead) {
+                            next_u = claim_unit(T);
+                            claimed = true;
                         }
                     }
                     if (aborted) break;
+                    if (!claimed) {
+                        // the first unit streamed completely before the grid dependency was resolved
+                        if (!grid_dep_ok) flush();
+                        next_u = claim_unit(T);
+                    }
+                    // whatever comes next needs a free slot: wait for it before the claim's result is used,
+                    // so the claim's round trip overlaps the wait
+                    if (!take_slot()) break;
                     u = next_u + n_static;
                 }
                 if (np > 0) flush();
                 if (aborted) break;
-                claims_finished(T, gridDim.x);
+                if (!p.run_ctl) claims_finished(T, gridDim.x);
                 if (T.dep < 0 && !first_unit) trace_stamp(p, t, 1, globaltimer());
             }
             if (!grid_dep_ok) pdl_wait();  // a CTA with no work still orders itself after the previous kernel
@@ -272,7 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             // advances one of these barriers again)
             drain_issued(full_bar, S, issued, wlim, p.status);
             // end-of-work marker for the MMA thread (a stage with no data)
-            if (!aborted && mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, -1, kSiteEmpty)) {
+            if (!aborted && (slot_ok || mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, -1,
+                                                          kSiteEmpty))) {
                 stage_meta[s][0] = 0;
                 stage_meta[s][1] = 0;
                 stage_meta[s][2] = kMetaDone;
@@ -294,21 +363,25 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 const int u = stage_meta[s][1];
                 const int flags = stage_meta[s][2];
                 if (flags & kMetaDone) {
-                    buf = acc_i & 1;
-                    if (mbar_wait_bounded(&acce_bar[buf], ((acc_i >> 1) & 1) ^ 1, &abort_flag, wlim, p.status, -1,
-                                          kSiteAcc)) {
-                        acc_meta[buf][0] = 0;
-                        acc_meta[buf][1] = 0;
-                        acc_meta[buf][2] = kMetaDone;
-                        mbar_arrive(&accf_bar[buf]);
-                        mbar_arrive(&accf_bar[buf]);
+                    // the end marker goes to the next accumulator of EACH epilogue set
+                    for (uint32_t d = 0; d < (uint32_t)kEpiSets; ++d) {
+                        const uint32_t i = acc_i + d;
+                        const int b = (int)(i % kAccBufs);
+                        if (!mbar_wait_bounded(&acce_bar[b], ((i / kAccBufs) & 1) ^ 1, &abort_flag, wlim, p.status,
+                                               -1, kSiteAcc))
+                            break;
+                        acc_meta[b][0] = 0;
+                        acc_meta[b][1] = 0;
+                        acc_meta[b][2] = kMetaDone;
+                        mbar_arrive(&accf_bar[b]);
+                        mbar_arrive(&accf_bar[b]);
                     }
                     break;
                 }
                 if (flags & kMetaFirst) {
-                    buf = acc_i & 1;
-                    if (!mbar_wait_bounded(&acce_bar[buf], ((acc_i >> 1) & 1) ^ 1, &abort_flag, wlim, p.status, t,
-                                           kSiteAcc))
+                    buf = (int)(acc_i % kAccBufs);
+                    if (!mbar_wait_bounded(&acce_bar[buf], ((acc_i / kAccBufs) & 1) ^ 1, &abort_flag, wlim, p.status,
+                                           t, kSiteAcc))
                         break;
                     tc_fence_after();
                 }
@@ -349,19 +422,21 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Two sets of four warps; set e takes accumulators e, e + 2, e + 4, ...
+        const int set = (warp - kEpiWarp0) / 4;
         const int q = warp & 3;                 // TMEM lane quadrant this warp may access
         const int row = q * 32 + lane;          // row of the 128-row tile = TMEM lane
-        const int etid = threadIdx.x - kEpiWarp0 * 32;
+        const int etid = threadIdx.x - (kEpiWarp0 + 4 * set) * 32;
         const bool leader = (etid == 0);
         if (p.pdl) pdl_wait();                  // Y and the scratch may still be in use by the previous kernel
-        uint32_t acc_i = 0;
-        for (;;) {
-            const int buf = acc_i & 1;
-            const uint32_t aph = (acc_i >> 1) & 1;
+        for (uint32_t k = 0;; ++k) {
+            const uint32_t acc_i = kEpiSets * k + (uint32_t)set;
+            const int buf = (int)(acc_i % kAccBufs);
+            const uint32_t aph = (acc_i / kAccBufs) & 1;
             const bool ab = !mbar_wait_bounded(&accf_bar[buf], aph, &abort_flag, wlim, p.status, -1, kSiteAcc);
-            // all four warps stop together (an abort anywhere, or the end marker)
+            // the four warps of the set stop together (an abort anywhere, or the end marker)
             const int flags = ab ? kMetaDone : acc_meta[buf][2];
-            if (vote_or(ab || (flags & kMetaDone), kEpiBar, kEpiThreads)) break;
+            if (vote_or(ab || (flags & kMetaDone), 1 + set, kEpiThreads)) break;
             const int t = acc_meta[buf][0];
             const int u = acc_meta[buf][1];
             const TaskDev &T = task_at(p, t);
@@ -386,15 +461,15 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acce_bar[buf]);
-            ++acc_i;
 
-            const int tile = u / T.nu;
+            const UnitSpan us = unit_span(T, u);
+            const int tile = us.tile;
             int g, mt;
             tile_coords(T, tile, g, mt);
             const int n = g * kUmmaRows + row;
             const int m0 = mt * T.t_m;
             const int mrows = min(T.t_m, T.M - m0);
-            if (T.nu == 1) {
+            if (us.nu == 1) {
                 if (n < T.N) {
 #pragma unroll
                     for (int m = 0; m < kUmmaMaxN; ++m) {
@@ -406,41 +481,30 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     }
                 }
                 if (T.notify) {
-                    epi_bar();
-                    if (leader) red_release_gpu_add(T.done, 1u);  // release covers the CTA's stores (bar.sync before)
+                    epi_bar(set);
+                    if (leader) red_release_gpu_add(T.done, 1u);  // release covers the set's stores (bar.sync before)
                 }
             } else {
-                // split tile: store this unit's partial; the last unit of the tile to arrive adds all of them
-                float *pslot = T.part + (size_t)u * T.slot_elems;
+                // split tile: store this unit's partial row; the last unit of the tile to arrive adds all of them
+                float4 *dst = reinterpret_cast<float4 *>(T.part + (size_t)u * T.slot_elems + (size_t)row * T.t_mpad);
 #pragma unroll
-                for (int m = 0; m < kUmmaMaxN; ++m)
-                    if (m < mrows) pslot[m * kUmmaRows + row] = acc[m];
-                epi_bar();
+                for (int i = 0; i < kUmmaMaxN / 4; ++i)
+                    if (4 * i < mrows) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+                epi_bar(set);
                 if (leader) {
-                    // acq_rel: releases this CTA's partial (stored before the barrier) and acquires the
+                    // acq_rel: releases this set's partial (stored before the barrier) and acquires the
                     // others' for the last arriver
                     const unsigned int old = atom_add_acqrel_gpu(&T.tile_cnt[tile], 1u);
-                    last_flag = (old == (unsigned int)(T.nu - 1)) ? 1 : 0;
+                    last_flag[set] = (old == (unsigned int)(us.nu - 1)) ? 1 : 0;
                 }
-                epi_bar();
-                if (last_flag) {
+                epi_bar(set);
+                if (last_flag[set]) {
                     // the leader's acquire + the barrier order these loads after every partial
-                    const float *tile_slots = T.part + (size_t)tile * T.nu * T.slot_elems;
-                    for (int mb = 0; mb < mrows; mb += 8) {
-                        float sum[8];
-                        ordered_unit_sums<8, 4>(tile_slots, T.slot_elems, kUmmaRows, row, mb, mrows, T.nu, sum);
-                        if (n < T.N) {
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                if (mb + i < mrows) {
-                                    const size_t o = (size_t)(m0 + mb + i) * T.N + n;
-                                    T.Y[o] = __float2bfloat16_rn(sum[i]);
-                                    if (T.Yf32) T.Yf32[o] = sum[i];
-                                }
-                            }
-                        }
-                    }
-                    epi_bar();
+                    if (mrows <= 4)
+                        reduce_row_partials<4, 16>(T, us.u0, us.nu, row, mrows, m0, n);
+                    else
+                        reduce_row_partials<16, 4>(T, us.u0, us.nu, row, mrows, m0, n);
+                    epi_bar(set);
                     if (leader) {
                         T.tile_cnt[tile] = 0u;  // ready for the next call
                         if (T.notify) red_release_gpu_add(T.done, 1u);
