@@ -39,6 +39,38 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
 
+def kernel_source_hash():
+    """sha256 over the CUDA sources (name + bytes, sorted): identifies the
+    kernel build a stored DRAM-traffic figure was taken from."""
+    import hashlib
+    d = os.path.join(ROOT, "weight_streaming_megakernel_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(name.encode())
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def stored_traffic(kernel, workload, mode):
+    """DRAM bytes (read + write) of one launch of `kernel`, from the ncu
+    summary under profiles/ -- only if it was taken from the current sources."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{kernel}_{workload}_{mode}.txt")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("csrc_sha256") != kernel_source_hash():
+            return None
+        return int(kv["dram__bytes_read.sum"]) + int(kv["dram__bytes_write.sum"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -463,13 +495,21 @@ def main():
         dominant = max(fam, key=lambda k: fam[k][1])
         fam_bytes, fam_ms = fam[dominant]
     achieved = fam_bytes / (fam_ms * 1e-3) / 1e9
+    traffic = stored_traffic(dominant, config["workload"], args.mode) if r["chain"] and not args.only else None
+    step_ms = sorted(sum(row) for row in r["per_launch"])
+
+    def pct(q):
+        return round(step_ms[min(len(step_ms) - 1, int(q * (len(step_ms) - 1) + 0.5))], 4)
     value = r["total_bytes"] * world / (r["ms_per_step"] * 1e-3) / 1e9
 
-    cpu = None
+    cpu = cpu1 = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sec, cores, desc = oracle_sample_rate(cases, args.cpu_budget_s)
         cpu = {"value": round(r["total_bytes"] / sec / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": desc}
+        sec, cores, desc = oracle_sample_rate(cases, args.cpu_budget_s / 2, threads=1)
+        cpu1 = {"value": round(r["total_bytes"] / sec / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                "sample": desc}
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -479,10 +519,13 @@ def main():
                 "frac_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
                 "roofline": {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": hbm_peak,
                              "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                             "traffic": None},
+                             "traffic": traffic,
+                             "algorithmic_bytes_per_launch": fam_bytes if r["chain"] else None},
+                "step_ms_p10_p50_p90": [pct(0.1), pct(0.5), pct(0.9)],
                 "us_per_gemm": us_per_gemm,
                 "single_launch_breakdown": breakdown,
                 "cpu_baseline": cpu,
+                "cpu_baseline_1thread": cpu1,
                 "e2e": r["e2e"],
                 "gpu_launches": r["launches_per_step"] * args.steps,
                 "ms_per_step_without_timing_events": round(r["plain_ms"], 4),
