@@ -20,6 +20,17 @@ What it computes, and from which passage:
   changes when work runs, not what it computes).
 * ``l2model`` -- Eq.(1) of the Fleet reading notes (section 3f), the L2 weight
   hit rate of M-major cooperative traversal, and AI_eff.
+* ``silu`` / ``gate_up_rows`` / ``silu_mul_ref`` -- the fused SiLU epilogue of
+  the gate+up GEMM ("Fleet ..." reading notes, sections 3f and 7b and the
+  design summary: gate and up concatenated into one GEMM sharing one
+  activation, with SiLU fused): ``H = silu(X Wg^T) * (X Wu^T)``, silu(z) =
+  z / (1 + e^-z), evaluated in fp64 from the fp64 products.  The pages do not
+  fix how gate and up rows are laid out in the one weight; the reading here
+  interleaves them in blocks of 8 rows (gate rows 8b..8b+7, then the up rows
+  8b..8b+7), so every weight tile holds matching gate and up rows.
+* ``residual_ref`` -- the residual-add epilogue, ``Y = X W^T + R`` in fp64.
+* ``fused_bounds`` -- the fp32 acceptance bounds of the fused outputs,
+  propagated from the GEMM's per-element bound (see the function).
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against
 brute-force exact rational arithmetic, integer and permutation cases, library
@@ -161,3 +172,60 @@ def chain_ref(tasks):
 def set_threads(n: int = 0) -> int:
     """Set the OpenMP thread count (0 keeps the current one); returns it."""
     return load().wsmo_set_threads(int(n))
+
+
+# --------------------------------------------------------------------------- fused epilogues
+
+def silu(z):
+    """silu(z) = z * sigmoid(z) = z / (1 + exp(-z)), fp64 (exp overflow for very
+    negative z gives z / inf = -0.0, the limit)."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def gate_up_rows(I: int):
+    """(gate, up) row indices of the fused gate+up weight [2I, K] for output
+    column j < I: blocks of 8 rows, gate rows of block b then its up rows."""
+    assert I % 8 == 0
+    j = np.arange(I)
+    gate = 16 * (j // 8) + (j % 8)
+    return gate, gate + 8
+
+
+def silu_mul_ref(X, W_gu, lib=None):
+    """Fused gate+up GEMM with SiLU: returns (H_ref, G, U, Sg, Su), all [M, I]
+    fp64: H = silu(G) * U with G, U the gate and up products and Sg, Su their
+    sums of |products| (the scale of the GEMM bound)."""
+    Y, S = gemm_ref(X, W_gu, lib)
+    gi, ui = gate_up_rows(Y.shape[1] // 2)
+    G, U = Y[:, gi], Y[:, ui]
+    return silu(G) * U, G, U, S[:, gi], S[:, ui]
+
+
+def residual_ref(X, W, R, lib=None):
+    """Y = X W^T + R in fp64 (R: bf16 [M, N]); returns (Y_ref, S) with S the
+    GEMM's sum of |products|."""
+    Y, S = gemm_ref(X, W, lib)
+    r = _u16(R)
+    Rf = np.frombuffer((r.astype(np.uint32) << 16).tobytes(), dtype=np.float32).reshape(r.shape).astype(np.float64)
+    return Y + Rf, S
+
+
+def fused_bounds(kind, *, S=None, Y=None, G=None, U=None, Sg=None, Su=None):
+    """Per-element fp32 acceptance bound of a fused output.
+
+    The GEMM part of every output may differ from its fp64 value by
+    d = 1e-3 * S + 1e-6 (the accumulation bound).  Residual: d plus one fp32
+    rounding of the sum, 2^-23 |Y|.  SiLU*mul: with dg, du the bounds of G and
+    U, and |silu'| <= 1.1 everywhere (its extremes are about 1.0998 and
+    -0.0998), |dH| <= 1.1 |U| dg + (|silu(G)| + 1.1 dg) du, plus the fp32
+    evaluation of silu and the product, 2^-19 |silu(G) U| + 1e-7."""
+    if kind == "residual":
+        return 1e-3 * S + 1e-6 + 2.0 ** -23 * np.abs(Y)
+    if kind == "silu_mul":
+        dg = 1e-3 * Sg + 1e-6
+        du = 1e-3 * Su + 1e-6
+        sg = np.abs(silu(G))
+        return 1.1 * np.abs(U) * dg + (sg + 1.1 * dg) * du + 2.0 ** -19 * sg * np.abs(U) + 1e-7
+    raise ValueError(kind)

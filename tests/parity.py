@@ -80,3 +80,24 @@ def check_sampled(x, w, y, yf32, ms, ns, what=""):
         yf = yf32.detach().cpu().double().numpy()[ms, ns]
         assert (np.abs(yf - Y_ref) <= RTOL_S * S + ATOL).all(), f"{what}: fp32 outside bound"
     return int(d.max()) if d.size else 0
+
+
+def check_bounded(y, yf32, ref, bound, what=""):
+    """Fused outputs: |yf32 - ref| <= bound element-wise, and the bf16 result
+    within 1 ulp of round_bf16(ref) or the rounding of some value inside the
+    bound (the same acceptance as the plain GEMM, with the fused bound from
+    oracle.fused_bounds)."""
+    if yf32 is not None:
+        yf = yf32.detach().cpu().double().numpy()
+        err = np.abs(yf - ref)
+        bad = np.argwhere(~(err <= bound))
+        assert bad.size == 0, (f"{what}: fp32 outside bound at {bad[:5].tolist()}: got {yf[tuple(bad[0])]}, "
+                               f"ref {ref[tuple(bad[0])]}, bound {bound[tuple(bad[0])]}")
+    got = bf16_bits(y)
+    d = ulp_distance(got, oracle.round_bf16(ref))
+    g = ordered(got)
+    ok = (d <= 1) | ((g >= ordered(oracle.round_bf16(ref - bound))) & (g <= ordered(oracle.round_bf16(ref + bound))))
+    bad = np.argwhere(~ok)
+    assert bad.size == 0, (f"{what}: bf16 off at {bad[:5].tolist()} (got {hex(int(got[tuple(bad[0])]))}, "
+                           f"ref {hex(int(oracle.round_bf16(ref)[tuple(bad[0])]))}, ulps {int(d[tuple(bad[0])])})")
+    return int(d.max()) if d.size else 0

@@ -370,3 +370,136 @@ def test_planted_mistakes_are_caught(name, tmp_path):
     subprocess.run(["gcc", *oracle.CFLAGS, "-o", str(so), str(mutated), "-lm"], check=True)
     lib = oracle.load(str(so))
     assert not _pins_pass(lib), f"planted mistake '{name}' was not caught by the pins"
+
+
+# --------------------------------------------------------------------------- fused epilogues
+#
+# The pins below take the functions under test as parameters, so the same pins
+# can be run against deliberately wrong variants (planted in the test, on the
+# CPU) to show that each plausible slip is caught.
+
+SIGMOID_1 = 0.7310585786300049          # logistic(1) = e / (1 + e), to 16 digits
+
+
+def _silu_pins(silu):
+    z = np.random.default_rng(0).normal(0, 4, 4096)
+    if silu(np.array([0.0]))[0] != 0.0:
+        return False
+    if abs(silu(np.array([1.0]))[0] - SIGMOID_1) > 1e-15:
+        return False
+    # silu(z) - silu(-z) = z  (sigmoid(z) + sigmoid(-z) = 1)
+    if np.max(np.abs(silu(z) - silu(-z) - z) / np.maximum(1.0, np.abs(z))) > 1e-14:
+        return False
+    big = silu(np.array([40.0, 1000.0, -40.0, -1000.0]))
+    if not (abs(big[0] - 40.0) < 1e-14 and big[1] == 1000.0 and abs(big[2]) < 1e-15 and big[3] == 0.0):
+        return False
+    return not np.isnan(big).any()
+
+
+def _interleave_by_reshape(Wg, Wu):
+    """Fused gate+up weight built independently of gate_up_rows: blocks of 8
+    gate rows then the matching 8 up rows."""
+    I, K = Wg.shape
+    g = Wg.reshape(I // 8, 8, K)
+    u = Wu.reshape(I // 8, 8, K)
+    return torch.stack([g, u], dim=1).reshape(2 * I, K).contiguous()
+
+
+def _silu_mul_pins(silu_mul_ref):
+    M, I, K = 3, 32, 96
+    X, Wg = synth.make_xw(M, I, K, seed=70)
+    _, Wu = synth.make_xw(1, I, K, seed=71)
+    H, G, U, Sg, Su = silu_mul_ref(X, _interleave_by_reshape(Wg, Wu))
+    Gr, Sgr = oracle.gemm_ref(X, Wg)
+    Ur, Sur = oracle.gemm_ref(X, Wu)
+    if not (np.array_equal(G, Gr) and np.array_equal(U, Ur) and np.array_equal(Sg, Sgr) and np.array_equal(Su, Sur)):
+        return False
+    return np.array_equal(H, oracle.silu(Gr) * Ur)
+
+
+def _residual_pins(residual_ref):
+    X, W = synth.make_int_xw(3, 40, 64, seed=72)
+    R = synth.make_x(3, 40, seed=73)                 # any bf16 [3, 40]
+    Y, S = residual_ref(X, W, R)
+    Y0, S0 = oracle.gemm_ref(X, W)
+    # R widened exactly (torch's bf16 -> fp64) and added once
+    if not np.array_equal(Y - Y0, R.to(torch.float64).numpy()) or not np.array_equal(S, S0):
+        return False
+    Yz, _ = residual_ref(X, W, torch.zeros(3, 40, dtype=torch.bfloat16))
+    return np.array_equal(Yz, Y0)
+
+
+def test_silu_pins():
+    assert _silu_pins(oracle.silu)
+
+
+def test_silu_mul_pins():
+    assert _silu_mul_pins(oracle.silu_mul_ref)
+
+
+def test_residual_pins():
+    assert _residual_pins(oracle.residual_ref)
+
+
+def test_gate_up_rows_cover_every_row_once():
+    gi, ui = oracle.gate_up_rows(64)
+    assert sorted(np.concatenate([gi, ui]).tolist()) == list(range(128))
+    assert np.all(ui - gi == 8) and np.all((gi % 16) < 8)
+
+
+def test_silu_derivative_bound():
+    """The constant 1.1 of fused_bounds: |silu'| <= 1.1 on a fine grid (its
+    extremes are ~1.0998 near z = 2.4 and ~-0.0998 near z = -2.4)."""
+    z = np.linspace(-30, 30, 600001)
+    d = np.gradient(oracle.silu(z), z)
+    assert d.max() < 1.1 and d.min() > -1.1
+    assert abs(d.max() - 1.0998) < 1e-3 and abs(d.min() + 0.0998) < 1e-3
+
+
+def test_fused_bound_covers_perturbed_inputs():
+    """Any G, U moved by at most their GEMM bounds changes silu(G) * U by no
+    more than the silu_mul bound (corners of the box, many random points)."""
+    rng = np.random.default_rng(5)
+    G = rng.normal(0, 3, 20000)
+    U = rng.normal(0, 3, 20000)
+    Sg = np.abs(G) * rng.uniform(1, 50, G.size)
+    Su = np.abs(U) * rng.uniform(1, 50, U.size)
+    b = oracle.fused_bounds("silu_mul", G=G, U=U, Sg=Sg, Su=Su)
+    H = oracle.silu(G) * U
+    dg, du = 1e-3 * Sg + 1e-6, 1e-3 * Su + 1e-6
+    for sg in (-1, 1):
+        for su in (-1, 1):
+            Hp = oracle.silu(G + sg * dg) * (U + su * du)
+            assert np.all(np.abs(Hp - H) <= b)
+    # the bound is not vacuous: the worst corner uses a good part of it
+    Hp = np.maximum.reduce([np.abs(oracle.silu(G + a * dg) * (U + c * du) - H) for a in (-1, 1) for c in (-1, 1)])
+    assert np.median(Hp / b) > 0.3
+
+
+FUSED_MUTATIONS = {
+    # exp(+z) instead of exp(-z)
+    "silu_sign": ("silu", lambda z: np.asarray(z, np.float64) / (1.0 + np.exp(np.asarray(z, np.float64)))),
+    # sigmoid without the factor z
+    "silu_no_z": ("silu", lambda z: 1.0 / (1.0 + np.exp(-np.asarray(z, np.float64)))),
+    # gate and up swapped
+    "swap_gate_up": ("silu_mul", lambda X, W: (lambda Y, S: (
+        oracle.silu(Y[:, oracle.gate_up_rows(Y.shape[1] // 2)[1]]) * Y[:, oracle.gate_up_rows(Y.shape[1] // 2)[0]],
+        Y[:, oracle.gate_up_rows(Y.shape[1] // 2)[1]], Y[:, oracle.gate_up_rows(Y.shape[1] // 2)[0]],
+        S[:, oracle.gate_up_rows(Y.shape[1] // 2)[1]], S[:, oracle.gate_up_rows(Y.shape[1] // 2)[0]]))(
+        *oracle.gemm_ref(X, W))),
+    # halves layout (gate rows first, then up rows) instead of blocks of 8
+    "halves_layout": ("silu_mul", lambda X, W: (lambda Y, S, I: (
+        oracle.silu(Y[:, :I]) * Y[:, I:], Y[:, :I], Y[:, I:], S[:, :I], S[:, I:]))(
+        *oracle.gemm_ref(X, W), W.shape[0] // 2)),
+    # residual dropped / subtracted
+    "residual_dropped": ("residual", lambda X, W, R: oracle.gemm_ref(X, W)),
+    "residual_sign": ("residual", lambda X, W, R: (lambda Y, S: (Y - R.to(torch.float64).numpy(), S))(
+        *oracle.gemm_ref(X, W))),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FUSED_MUTATIONS))
+def test_fused_planted_mistakes_are_caught(name):
+    kind, fn = FUSED_MUTATIONS[name]
+    pins = {"silu": _silu_pins, "silu_mul": _silu_mul_pins, "residual": _residual_pins}[kind]
+    assert not pins(fn), f"planted mistake '{name}' was not caught"
