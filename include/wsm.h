@@ -103,6 +103,24 @@ enum {
     WSM_FLAG_NO_PDL = 2
 };
 
+/* Epilogue applied to the fp32 result, before its one rounding to bf16.
+ * SILU_MUL is the gate+up projection of a gated MLP with the activation fused
+ * ("Fleet ..." reading notes, sections 3f and 7b: gate and up concatenated into
+ * one GEMM sharing one activation, SiLU fused).  W is the fused weight [N, K],
+ * N = 2I a multiple of 16, holding gate and up rows interleaved in blocks of 8:
+ * rows 16b .. 16b+7 are gate rows 8b .. 8b+7 and rows 16b+8 .. 16b+15 the
+ * matching up rows.  The output is H [M, I]:
+ *     H[m, 8b + i] = silu(G) * U,  G = (X W^T)[m, 16b + i],
+ *                                  U = (X W^T)[m, 16b + 8 + i],
+ * silu(z) = z / (1 + e^-z) in fp32.  RESIDUAL adds a bf16 [M, N] input R:
+ * Y = X W^T + R (R may be Y itself: each element is read before it is
+ * written, by the same thread). */
+enum {
+    WSM_EPI_NONE = 0,
+    WSM_EPI_SILU_MUL = 1,
+    WSM_EPI_RESIDUAL = 2
+};
+
 /* Options of skinny_gemm_ex; zero-initialised = all automatic. */
 typedef struct {
     int path;        /* WSM_PATH_* */
@@ -120,6 +138,11 @@ typedef struct {
                         smaller units of tail_unit_stages stages, so the end of
                         the GEMM spreads evenly over the CTAs: 0 = auto, -1 = none */
     int tail_unit_stages; /* pipeline stages per tail unit, 0 = auto */
+    int l2_prefetch_stages; /* W pipeline stages per CTA prefetched into L2 while the
+                               CTA waits for the previous kernel (WSM_FLAG_W_READONLY):
+                               0 = auto, -1 = none */
+    int epilogue;    /* WSM_EPI_*; with SILU_MUL, Y (and Yf32) are [M, N/2] */
+    const void *R;   /* WSM_EPI_RESIDUAL: bf16 [M, N], device */
     float *Yf32;     /* optional device [M, N] fp32: the result before rounding */
     void *workspace; /* optional caller scratch (device, >= wsm_workspace_bytes,
                         16-byte aligned, zero-filled before its first use; the
@@ -204,7 +227,14 @@ wsm_status skinny_gemm_noalloc(const void *X, const void *W, void *Y, int M, int
 /* One GEMM of a chain.  dep = -1, or the index of an EARLIER task whose Y
  * must be complete before this task reads its X (dep < own index, so a chain
  * can never deadlock: tiles are claimed in task order).  The wait covers X
- * only: W is streamed before the dependency is met. */
+ * only: W is streamed before the dependency is met.
+ *
+ * dep_cols != 0 makes the dependency a data dependency per column: X must be
+ * the dep task's output (same pointer, K = its output columns, same M), and
+ * each pipeline stage waits only until the 256-column chunks of X it reads
+ * are complete, instead of the whole dep task.  Such a task's work units are
+ * ordered K-range first (the first K-range of every tile, then the second,
+ * ...), so early units need only the columns the dep task finishes first. */
 typedef struct {
     const void *X;
     const void *W;
@@ -212,6 +242,9 @@ typedef struct {
     int M, N, K;
     int dep;
     float *Yf32;   /* optional fp32 result, may be NULL */
+    int epilogue;  /* WSM_EPI_* (as in wsm_opts) */
+    const void *R; /* WSM_EPI_RESIDUAL: bf16 [M, N] */
+    int dep_cols;  /* nonzero: per-column data dependency on task dep (see above) */
 } wsm_task;
 
 typedef struct {
@@ -228,6 +261,8 @@ typedef struct {
     int unit_stages;           /* as in wsm_opts, for every task */
     int tail_tiles;            /* as in wsm_opts, for every task */
     int tail_unit_stages;      /* as in wsm_opts, for every task */
+    int l2_prefetch_stages;    /* W stages per CTA prefetched into L2 while the CTA waits for
+                                  a dependency or the previous kernel: 0 = auto, -1 = none */
 } wsm_chain_opts;
 
 typedef struct wsm_chain wsm_chain;  /* opaque prepared chain */

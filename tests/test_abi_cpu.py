@@ -156,7 +156,7 @@ def test_plan_tail_units():
     # the FMA path takes the same options
     p = wsm.plan(2, 2112, 7168, num_sms=148, path=wsm.PATH_STREAM, tail_tiles=20, tail_unit_stages=1)
     assert p["tail_tiles"] == 20 and p["units"] == (p["n_tiles"] - 20) * -(-p["k_iters"] // p["unit_stages"]) + 20 * p["k_iters"]
-    for bad in (dict(tail_tiles=-2), dict(tail_unit_stages=-1), dict(unit_stages=-1)):
+    for bad in (dict(tail_tiles=-2), dict(tail_unit_stages=-1), dict(unit_stages=-1), dict(l2_prefetch_stages=-2)):
         with pytest.raises(wsm.WsmError) as e:
             wsm.plan(M, N, K, **bad)
         assert e.value.code == wsm.WSM_ERR_INVALID
@@ -241,3 +241,36 @@ def test_product_never_touches_the_oracle():
                 assert "wsmo_" not in src, f
     oracle_src = open(os.path.join(ROOT, "oracle", "oracle.c")).read()
     assert "wsm.h" not in oracle_src and "wsm_internal" not in oracle_src
+
+
+def test_chain_validate_epilogues_and_column_deps():
+    base = 0x20000000
+    ok = [
+        {"X": base, "W": base + 0x100000, "Y": base + 0x200000, "M": 4, "N": 64, "K": 64},
+        {"X": base + 0x200000, "W": base + 0x300000, "Y": base + 0x400000, "M": 4, "N": 128, "K": 64, "dep": 0,
+         "dep_cols": 1, "epilogue": wsm.EPI_SILU_MUL},
+        {"X": base + 0x400000, "W": base + 0x500000, "Y": base + 0x600000, "M": 4, "N": 64, "K": 64, "dep": 1,
+         "dep_cols": 1, "epilogue": wsm.EPI_RESIDUAL, "R": base + 0x200000},
+    ]
+    wsm.chain_validate(ok)
+
+    def bad(i, code, **kv):
+        ts = [dict(t) for t in ok]
+        ts[i].update(kv)
+        with pytest.raises(wsm.WsmError) as e:
+            wsm.chain_validate(ts)
+        assert e.value.code == code, kv
+
+    bad(0, wsm.WSM_ERR_INVALID, epilogue=7)
+    bad(1, wsm.WSM_ERR_UNSUPPORTED, N=120)                       # SiLU*mul needs N % 16 == 0
+    bad(2, wsm.WSM_ERR_INVALID, R=None)                          # residual without R
+    bad(2, wsm.WSM_ERR_INVALID, R=base + 0x200001)               # misaligned R
+    bad(1, wsm.WSM_ERR_INVALID, dep=-1)                          # dep_cols without a dependency
+    bad(1, wsm.WSM_ERR_INVALID, X=base + 0x700000)               # X is not the dep task's Y
+    bad(2, wsm.WSM_ERR_INVALID, K=128)                           # K != dep's output columns (128 / 2)
+    bad(2, wsm.WSM_ERR_INVALID, M=8)                             # M differs from the dep task's
+
+
+def test_plan_accepts_epilogue_options():
+    wsm.plan(4, 4096, 4096, epilogue=wsm.EPI_SILU_MUL)
+    wsm.plan(4, 4096, 4096, epilogue=wsm.EPI_RESIDUAL)

@@ -74,7 +74,7 @@ def test_dependent_chain_tail_units(path, M):
     claim counters are reset at the end of each run)."""
     dims = [1024, 2048, 1024, 3072, 512]
     x0, ws, ys, yfs, tasks = dependent_chain(M, dims, seed=30 + M)
-    ch = wsm.Chain(tasks, path=path, unit_stages=3, tail_tiles=6, tail_unit_stages=1)
+    ch = wsm.Chain(tasks, path=path, unit_stages=3, tail_tiles=6, tail_unit_stages=1, l2_prefetch_stages=8)
     for _ in range(2):
         for y in ys:
             y.fill_(float("nan"))

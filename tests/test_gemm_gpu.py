@@ -107,6 +107,27 @@ def test_split_patterns(path, M, grid):
     check_full(x, w, y, yf, what=f"grid={grid}")
 
 
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 2), (wsm.PATH_UMMA, 16)])
+@pytest.mark.parametrize("pf", [-1, 1, 64])
+def test_l2_prefetch_back_to_back(path, M, pf):
+    """The L2 prefetch issued while a launch waits for the previous kernel
+    (W read-only flag) is only a hint: back-to-back launches give the same
+    bits for every prefetch depth."""
+    N, K = 3000, 4096
+    x, w = synth.make_xw(M, N, K, seed=60 + M)
+    xd, wd = x.to(DEV), w.to(DEV)
+    ref = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    wsm.skinny_gemm(xd, wd, ref, path=path, l2_prefetch_stages=-1)
+    ys = [torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV) for _ in range(4)]
+    for y in ys:
+        wsm.skinny_gemm(xd, wd, y, path=path, flags=wsm.FLAG_W_READONLY, l2_prefetch_stages=pf)
+    torch.cuda.synchronize()
+    assert wsm.stream_status() == 0
+    for y in ys:
+        assert torch.equal(y, ref)
+    check_full(x, w, ys[-1], None, what=f"pf={pf}")
+
+
 @pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 2), (wsm.PATH_STREAM, 8), (wsm.PATH_UMMA, 16),
                                     (wsm.PATH_UMMA, 64)])
 def test_tail_units(path, M):

@@ -35,6 +35,7 @@ PATH_AUTO, PATH_STREAM, PATH_UMMA = 0, 1, 2
 ORDER_AUTO, ORDER_M_MAJOR, ORDER_NAIVE = 0, 1, 2
 L2_AUTO, L2_EVICT_FIRST, L2_NORMAL = 0, 1, 2
 FLAG_W_READONLY, FLAG_NO_PDL = 1, 2
+EPI_NONE, EPI_SILU_MUL, EPI_RESIDUAL = 0, 1, 2
 
 # Every function include/wsm.h declares (checked by the CPU tests).
 HEADER_SYMBOLS = (
@@ -54,7 +55,8 @@ class _Opts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("m_tile", ctypes.c_int), ("order", ctypes.c_int),
                 ("l2_policy", ctypes.c_int), ("grid", ctypes.c_int), ("stage_k", ctypes.c_int),
                 ("flags", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
-                ("tail_unit_stages", ctypes.c_int), ("Yf32", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int), ("epilogue", ctypes.c_int),
+                ("R", ctypes.c_void_p), ("Yf32", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t)]
 
 
@@ -71,14 +73,14 @@ class _PlanInfo(ctypes.Structure):
 class _Task(ctypes.Structure):
     _fields_ = [("X", ctypes.c_void_p), ("W", ctypes.c_void_p), ("Y", ctypes.c_void_p),
                 ("M", ctypes.c_int), ("N", ctypes.c_int), ("K", ctypes.c_int), ("dep", ctypes.c_int),
-                ("Yf32", ctypes.c_void_p)]
+                ("Yf32", ctypes.c_void_p), ("epilogue", ctypes.c_int), ("R", ctypes.c_void_p), ("dep_cols", ctypes.c_int)]
 
 
 class _ChainOpts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("grid", ctypes.c_int), ("timeout_ns", ctypes.c_ulonglong),
                 ("trace", ctypes.c_int), ("debug_unmet_dependency", ctypes.c_int), ("flags", ctypes.c_int),
                 ("stage_k", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
-                ("tail_unit_stages", ctypes.c_int)]
+                ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int)]
 
 
 _lib = None
@@ -164,10 +166,14 @@ def _check_operand(name, t, dtype=torch.bfloat16):
 
 
 def _opts(path=PATH_AUTO, m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32=None, workspace=None,
-          stage_k=0, flags=0, unit_stages=0, tail_tiles=0, tail_unit_stages=0):
+          stage_k=0, flags=0, unit_stages=0, tail_tiles=0, tail_unit_stages=0, l2_prefetch_stages=0, epilogue=0,
+          r=None):
     o = _Opts()
     o.path, o.m_tile, o.order, o.l2_policy, o.grid, o.stage_k = path, m_tile, order, l2_policy, grid, stage_k
     o.flags, o.unit_stages, o.tail_tiles, o.tail_unit_stages = flags, unit_stages, tail_tiles, tail_unit_stages
+    o.l2_prefetch_stages = l2_prefetch_stages
+    o.epilogue = epilogue
+    o.R = _ptr(r)
     o.Yf32 = _ptr(yf32)
     if workspace is not None:
         o.workspace = workspace.data_ptr()
@@ -178,31 +184,43 @@ def _opts(path=PATH_AUTO, m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0,
 def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = None, *, path=PATH_AUTO,
                 m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None, stage_k=0, flags=0, unit_stages=0, tail_tiles=0,
-                tail_unit_stages=0, stream=None) -> torch.Tensor:
-    """Y = X @ W.T on the current (or given) stream; returns Y."""
+                tail_unit_stages=0, l2_prefetch_stages=0, epilogue=EPI_NONE, r: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """Y = X @ W.T on the current (or given) stream; returns Y.  With
+    epilogue=EPI_SILU_MUL, W is the fused gate+up weight (rows interleaved in
+    blocks of 8) and Y is [M, N/2] = silu(gate) * up; with EPI_RESIDUAL,
+    Y = X @ W.T + r."""
     _check_operand("x", x)
     _check_operand("w", w)
     if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[1]:
         raise ValueError(f"shapes x{tuple(x.shape)} w{tuple(w.shape)} do not form X[M,K] . W[N,K]^T")
     M, K = x.shape
     N = w.shape[0]
+    ny = N // 2 if epilogue == EPI_SILU_MUL else N
     if y is None:
-        y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+        y = torch.empty(M, ny, dtype=torch.bfloat16, device=x.device)
     _check_operand("y", y)
-    if tuple(y.shape) != (M, N):
-        raise ValueError(f"y must be [{M}, {N}]")
+    if tuple(y.shape) != (M, ny):
+        raise ValueError(f"y must be [{M}, {ny}]")
     if yf32 is not None:
         _check_operand("yf32", yf32, torch.float32)
-        if tuple(yf32.shape) != (M, N):
-            raise ValueError(f"yf32 must be [{M}, {N}]")
-    plain = (path, m_tile, order, l2_policy, grid, stage_k, flags, unit_stages, tail_tiles, tail_unit_stages) == \
-        (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0, 0, 0, 0, 0, 0) and yf32 is None and workspace is None
+        if tuple(yf32.shape) != (M, ny):
+            raise ValueError(f"yf32 must be [{M}, {ny}]")
+    if epilogue == EPI_RESIDUAL:
+        if r is None:
+            raise ValueError("the residual epilogue needs r")
+        _check_operand("r", r)
+        if tuple(r.shape) != (M, N):
+            raise ValueError(f"r must be [{M}, {N}]")
+    plain = (path, m_tile, order, l2_policy, grid, stage_k, flags, unit_stages, tail_tiles, tail_unit_stages,
+             l2_prefetch_stages, epilogue) == (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0, 0, 0, 0, 0, 0, 0, 0) \
+        and yf32 is None and workspace is None
     s = _stream_handle(stream)
     if plain:
         _check(lib().skinny_gemm(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, s), "skinny_gemm")
     else:
         o = _opts(path, m_tile, order, l2_policy, grid, yf32, workspace, stage_k, flags, unit_stages, tail_tiles,
-                  tail_unit_stages)
+                  tail_unit_stages, l2_prefetch_stages, epilogue, r)
         _check(lib().skinny_gemm_ex(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, ctypes.byref(o), s),
                "skinny_gemm_ex")
     return y
@@ -253,6 +271,9 @@ class Task:
     y: torch.Tensor
     dep: int = -1
     yf32: Optional[torch.Tensor] = None
+    epilogue: int = EPI_NONE
+    r: Optional[torch.Tensor] = None
+    dep_cols: bool = False
 
 
 def _tasks_array(tasks: Sequence[Task]):
@@ -263,17 +284,20 @@ def _tasks_array(tasks: Sequence[Task]):
         arr[i].X, arr[i].W, arr[i].Y = t.x.data_ptr(), t.w.data_ptr(), t.y.data_ptr()
         arr[i].M, arr[i].N, arr[i].K, arr[i].dep = M, N, K, t.dep
         arr[i].Yf32 = _ptr(t.yf32)
+        arr[i].epilogue, arr[i].R, arr[i].dep_cols = t.epilogue, _ptr(t.r), 1 if t.dep_cols else 0
     return arr
 
 
 def chain_validate(tasks) -> None:
     """Host-side validation of a raw task list: sequence of dicts with keys
-    X, W, Y (integer addresses), M, N, K, dep."""
+    X, W, Y (integer addresses), M, N, K and optionally dep, Yf32, epilogue, R,
+    dep_cols."""
     arr = (_Task * len(tasks))()
     for i, t in enumerate(tasks):
         arr[i].X, arr[i].W, arr[i].Y = t["X"], t["W"], t["Y"]
         arr[i].M, arr[i].N, arr[i].K, arr[i].dep = t["M"], t["N"], t["K"], t.get("dep", -1)
         arr[i].Yf32 = t.get("Yf32")
+        arr[i].epilogue, arr[i].R, arr[i].dep_cols = t.get("epilogue", 0), t.get("R"), int(bool(t.get("dep_cols")))
     _check(lib().wsm_chain_validate(arr, len(tasks)), "wsm_chain_validate")
 
 
@@ -282,7 +306,7 @@ class Chain:
 
     def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
                  debug_unmet_dependency=False, flags=0, stage_k=0, unit_stages=0, tail_tiles=0,
-                 tail_unit_stages=0):
+                 tail_unit_stages=0, l2_prefetch_stages=0):
         for i, t in enumerate(tasks):
             _check_operand(f"tasks[{i}].x", t.x)
             _check_operand(f"tasks[{i}].w", t.w)
@@ -294,6 +318,7 @@ class Chain:
         o.debug_unmet_dependency = 1 if debug_unmet_dependency else 0
         o.flags, o.stage_k = flags, stage_k
         o.unit_stages, o.tail_tiles, o.tail_unit_stages = unit_stages, tail_tiles, tail_unit_stages
+        o.l2_prefetch_stages = l2_prefetch_stages
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

@@ -40,6 +40,10 @@ constexpr int kStreamBoxK = 256;   // K elements per TMA box on the FMA path
 constexpr int kStatusWords = 4;    // [0] error code, [1] failing task, [2] failing CTA, [3] site
 constexpr int kSchedWords = 2;     // per task: [0] next unit to claim, [1] CTAs done claiming
 constexpr int kClaimLead = 4;      // a CTA claims its next unit this many stages before its unit ends
+constexpr int kColChunk = 256;     // output columns per readiness chunk (per-column data dependencies)
+
+// Epilogues (== WSM_EPI_*).
+enum : int { kEpiNone = 0, kEpiSiluMul = 1, kEpiResidual = 2 };
 
 // Error sites recorded in status[3].
 enum : int { kSiteNone = 0, kSiteDep = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteAcc = 4, kSiteDrain = 5 };
@@ -79,8 +83,17 @@ struct __align__(64) TaskDev {
     int ku_t;                   // stages per tail unit
     int nu_t;                   // units per tail tile
     int n_units;                // u_head + (n_g * n_mt - t_head) * nu_t
+    int k_major;                // units ordered K-range first: unit u = K-range u / tiles of tile u % tiles
+                                // (no tail split); partial slot u either way
     int order;                  // 0: M-tile inner (M-major), 1: M-tile outer
     int notify;                 // bump `done` after each finished tile
+    int epi;                    // kEpi*
+    int y_cols;                 // output columns: N, or N / 2 with SiLU*mul
+    const __nv_bfloat16 *R;     // residual [M, N] (kEpiResidual)
+    unsigned int *col_cnt;      // per kColChunk output columns: tiles finished (monotonic over runs), or nullptr
+    const unsigned int *col_need;      // tiles that touch each chunk, per run
+    const unsigned int *dep_col_cnt;   // per-column dependency: the dep task's col_cnt, else nullptr
+    const unsigned int *dep_col_need;  // ... and its col_need
     int w_evict_first;          // L2 policy of the weight loads
     uint32_t idesc;             // UMMA instruction descriptor (MMA N = t_mpad)
     uint32_t tx_bytes;          // bytes landing in one stage
@@ -95,7 +108,7 @@ struct KParams {
     int stage_bytes;                // bytes per ring stage
     int x_off;                      // offset of the X part inside a stage
     uint32_t dep_target_extra;      // 0; a test hook makes every dependency unreachable with it
-    int pad0_;
+    int prefetch_stages;            // W stages a waiting CTA prefetches into L2 (0: none)
     unsigned int *run_ctl;          // chain: [0] runs completed, [1] CTAs done with this run; or nullptr
     int kps;                        // UMMA path: 64-wide K boxes per stage
     int x_stride;                   // UMMA path: bytes between the X boxes of a stage
@@ -194,6 +207,14 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
         " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
         : "memory");
+}
+
+// L2 prefetch of one box of a tensor map: no shared memory, nothing to wait for.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
+                 : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
@@ -318,10 +339,23 @@ __device__ __forceinline__ void tile_coords(const TaskDev &T, int tile, int &g, 
 // partial slots are u0 .. u0 + nu - 1, in K order) and its stage range.
 struct UnitSpan {
     int tile, u0, nu, k_begin, k_end;
+    int slot_stride;  // partial slot of the tile's unit j = u0 + j * slot_stride
 };
 __device__ __forceinline__ UnitSpan unit_span(const TaskDev &T, int u) {
     UnitSpan r;
     int j, ku;
+    r.slot_stride = 1;
+    if (T.k_major) {
+        const int tiles = T.n_g * T.n_mt;
+        j = u / tiles;
+        r.tile = u - j * tiles;
+        r.nu = T.nu;
+        r.u0 = r.tile;
+        r.slot_stride = tiles;
+        r.k_begin = j * T.ku;
+        r.k_end = min(r.k_begin + T.ku, T.kb);
+        return r;
+    }
     if (u < T.u_head) {
         r.tile = u / T.nu;
         j = u - r.tile * T.nu;
@@ -391,6 +425,52 @@ __device__ __forceinline__ void ordered_unit_sums(const float *tile_slots, int s
 // The run number is read from device memory (not a launch parameter) so a
 // chain captured once in a CUDA graph stays correct over any number of
 // replays; the last CTA to finish a run advances it (chain_run_done).
+// A finished tile of task T (column tile g, rows_per_tile rows of W) counts
+// toward every kColChunk-column chunk of the output it wrote.  Called by one
+// thread after a barrier that follows all the tile's stores (release).
+__device__ __forceinline__ void notify_columns(const TaskDev &T, int g, int rows_per_tile) {
+    int c_lo = g * rows_per_tile;
+    int c_hi = min(T.N, c_lo + rows_per_tile);
+    if (T.epi == kEpiSiluMul) {  // N and the tile heights are multiples of 16
+        c_lo >>= 1;
+        c_hi >>= 1;
+    }
+    for (int c = c_lo / kColChunk; c <= (c_hi - 1) / kColChunk; ++c) red_release_gpu_add(&T.col_cnt[c], 1u);
+}
+
+// Per-column dependency: wait (bounded) until the chunks c0 .. c1 of the dep
+// task's output are complete in run `run`; `mask` caches chunks < 64 already
+// seen complete (they stay complete for the rest of the run).
+__device__ __forceinline__ void wait_chunks(const KParams &p, const TaskDev &T, int c0, int c1, unsigned int run,
+                                            unsigned long long &mask, int task, int *status) {
+    for (int c = c0; c <= c1; ++c) {
+        if (c < 64 && ((mask >> c) & 1ull)) continue;
+        const unsigned int target = run * T.dep_col_need[c] + p.dep_target_extra;
+        if (ld_acquire_gpu(&T.dep_col_cnt[c]) - target >= 0x80000000u) {
+            const unsigned long long t0 = globaltimer();
+            for (uint32_t spin = 1;; ++spin) {
+                if (ld_acquire_gpu(&T.dep_col_cnt[c]) - target < 0x80000000u) break;
+                if ((spin & 31u) == 0) {
+                    if (status_set(status)) return;
+                    if (globaltimer() - t0 > p.dep_timeout_ns) {
+                        record_error(status, kCodeTimeout, task, kSiteDep);
+                        return;
+                    }
+                    __nanosleep(64);
+                }
+            }
+        }
+        if (c < 64) mask |= 1ull << c;
+    }
+    fence_proxy_async_global();
+}
+
+__device__ __forceinline__ bool dependency_met(const KParams &p, const TaskDev &D) {
+    const unsigned int run = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
+    const unsigned int target = run * (unsigned int)(D.n_g * D.n_mt) + p.dep_target_extra;
+    return ld_acquire_gpu(D.done) - target < 0x80000000u;  // done >= target (wrap-safe)
+}
+
 __device__ __forceinline__ void wait_dependency(const KParams &p, const TaskDev &D, int task, int *status) {
     const unsigned int run = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
     const unsigned int target = run * (unsigned int)(D.n_g * D.n_mt) + p.dep_target_extra;

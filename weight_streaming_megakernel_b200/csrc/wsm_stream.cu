@@ -42,6 +42,25 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
 
 constexpr int kConsBar = 1;
 
+// Epilogue of one output (row n of W, X row m): plain, residual add, or
+// SiLU*mul (the up value of gate row n comes from the thread owning row n + 8,
+// lane ^ 8: every lane of the warp calls this), then one rounding to bf16.
+__device__ __forceinline__ void emit_one(const TaskDev &T, int n, int m, bool live, float y) {
+    size_t o;
+    if (T.epi == kEpiSiluMul) {
+        const float up = __shfl_xor_sync(0xffffffffu, y, 8);
+        if (!live || (n & 8)) return;
+        y = y / (1.f + expf(-y)) * up;
+        o = (size_t)m * T.y_cols + ((n >> 4) << 3) + (n & 7);
+    } else {
+        if (!live) return;
+        o = (size_t)m * T.N + n;
+        if (T.epi == kEpiResidual) y += __bfloat162float(T.R[o]);
+    }
+    T.Y[o] = __float2bfloat16_rn(y);
+    if (T.Yf32) T.Yf32[o] = y;
+}
+
 // Barrier among the consumer warps that also ORs a predicate over them.
 __device__ __forceinline__ bool vote_or(bool v, int id, int n) {
     uint32_t r;
@@ -153,14 +172,59 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 bool dep_ok = T.dep < 0 && grid_dep_ok;
                 int pend_s[kMaxStages], pend_k[kMaxStages];
                 int np = 0;
+                // Per-column dependency: each stage's X waits only for the kColChunk-column chunks it
+                // reads (seen-complete chunks are cached in chunk_mask).
+                const bool col_dep = T.dep >= 0 && T.dep_col_cnt != nullptr;
+                unsigned long long chunk_mask = 0;
+                unsigned int run_no = 0;
+                auto stage_chunks = [&](int k0, int &c0, int &c1) {
+                    c0 = k0 / kColChunk;
+                    c1 = (min(k0 + KW * kStreamBoxK, T.K) - 1) / kColChunk;
+                };
+                auto x_now = [&](int k0) -> bool {  // may this stage's X load go out now?
+                    if (!dep_ok) return false;
+                    if (!col_dep) return true;
+                    int c0, c1;
+                    stage_chunks(k0, c0, c1);
+                    for (int c = c0; c <= c1; ++c)
+                        if (c >= 64 || !((chunk_mask >> c) & 1ull)) return false;
+                    return true;
+                };
+                // While this CTA waits (for the previous kernel or a dependency) HBM would idle: prefetch
+                // into L2 the W of the units it would own in a round-robin (c, c + G, ...), except the
+                // first ring-full of each first-round unit (some CTA's ring already holds it).
+                bool prefetched = p.prefetch_stages <= 0;
+                auto prefetch_l2 = [&]() {
+                    if (prefetched) return;
+                    prefetched = true;
+                    int budget = p.prefetch_stages;
+                    for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
+                        const UnitSpan ps = unit_span(T, uu);
+                        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? S : 0); kk < ps.k_end && budget > 0;
+                             ++kk, --budget)
+#pragma unroll
+                            for (int kw = 0; kw < KW; ++kw)
+                                tma_prefetch_l2_2d(&T.tmW, kk * (KW * kStreamBoxK) + kw * kStreamBoxK, ps.tile * TN);
+                    }
+                };
                 auto flush = [&]() {
                     if (!grid_dep_ok) {
+                        prefetch_l2();
                         pdl_wait();
                         grid_dep_ok = true;
                     }
-                    if (T.dep >= 0) wait_dependency(p, task_at(p, T.dep), t, p.status);
-                    trace_stamp(p, t, 1, globaltimer());
+                    if (T.dep >= 0 && !col_dep) {
+                        if (!prefetched && !dependency_met(p, task_at(p, T.dep))) prefetch_l2();
+                        wait_dependency(p, task_at(p, T.dep), t, p.status);
+                    }
+                    if (col_dep && run_no == 0) run_no = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
+                    if (!dep_ok) trace_stamp(p, t, 1, globaltimer());
                     for (int i = 0; i < np; ++i) {
+                        if (col_dep) {
+                            int c0, c1;
+                            stage_chunks(pend_k[i], c0, c1);
+                            wait_chunks(p, T, c0, c1, run_no, chunk_mask, t, p.status);
+                        }
                         uint8_t *xs = ring + (size_t)pend_s[i] * p.stage_bytes + p.x_off;
 #pragma unroll
                         for (int kw = 0; kw < KW; ++kw)
@@ -184,9 +248,21 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     return true;
                 };
                 bool first_unit = true;
-                // the first unit of each CTA is its own index (no atomic); later ones are claimed
-                const int n_static = min((int)gridDim.x, T.n_units);
-                int u = (int)blockIdx.x < T.n_units ? (int)blockIdx.x : T.n_units;
+                // The kernel's first task hands unit c to CTA c (no atomic, and it can stream before the
+                // grid dependency); later tasks hand out every unit by claim, so the CTAs that finish the
+                // previous task first take the next task's work.
+                const int n_static = (t == 0) ? min((int)gridDim.x, T.n_units) : 0;
+                int u;
+                if (t == 0) {
+                    u = (int)blockIdx.x < T.n_units ? (int)blockIdx.x : T.n_units;
+                } else {
+                    if (!grid_dep_ok) {
+                        pdl_wait();
+                        grid_dep_ok = true;
+                        dep_ok = T.dep < 0;
+                    }
+                    u = claim_unit(T);
+                }
                 while (u < T.n_units) {
                     if (first_unit) {
                         trace_stamp(p, t, 0, globaltimer());
@@ -212,7 +288,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                         for (int kw = 0; kw < KW; ++kw)
                             tma_load_2d(st + kw * TN * 512, &T.tmW, &full_bar[s], k0 + kw * kStreamBoxK, g * TN,
                                         pol_w);
-                        if (dep_ok) {
+                        if (x_now(k0)) {
 #pragma unroll
                             for (int kw = 0; kw < KW; ++kw)
                                 tma_load_2d(st + p.x_off + kw * MMAX * 512, &T.tmX, &full_bar[s],
@@ -229,17 +305,18 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                         }
                         // claim the next unit kClaimLead stages before this one ends: early enough to
                         // hide the claim's round trip, late enough not to hold work a faster CTA could
-                        // take (the claim counters belong to the previous kernel until the grid
-                        // dependency is resolved)
-                        if (!claimed && grid_dep_ok && k_end - kk <= kClaimLead) {
+                        // take -- and never while this task's dependency is unmet, when every CTA would
+                        // hold a second unit it cannot start (the claim counters belong to the previous
+                        // kernel until the grid dependency is resolved)
+                        if (!claimed && dep_ok && k_end - kk <= kClaimLead) {
                             next_u = claim_unit(T);
                             claimed = true;
                         }
                     }
                     if (aborted) break;
                     if (!claimed) {
-                        // the first unit streamed completely before the grid dependency was resolved
-                        if (!grid_dep_ok) flush();
+                        // the unit streamed completely before its dependencies were resolved
+                        if (!dep_ok) flush();
                         next_u = claim_unit(T);
                     }
                     // whatever comes next needs a free slot: wait for it before the claim's result is used,
@@ -364,14 +441,13 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
             const int n = g * TN + o_row;
             const bool live = owner && o_m < M && n < T.N;
             if (us.nu == 1) {
-                if (live) {
-                    const size_t o = (size_t)o_m * T.N + n;
-                    T.Y[o] = __float2bfloat16_rn(val);
-                    if (T.Yf32) T.Yf32[o] = val;
-                }
-                if (T.notify) {
+                emit_one(T, n, o_m, live, val);
+                if (T.notify || T.col_cnt) {
                     named_bar_sync(kConsBar, NCT);
-                    if (leader) red_release_gpu_add(T.done, 1u);  // release covers the CTA's stores (bar.sync before)
+                    if (leader) {  // release covers the CTA's stores (bar.sync before)
+                        if (T.notify) red_release_gpu_add(T.done, 1u);
+                        if (T.col_cnt) notify_columns(T, g, TN);
+                    }
                 }
             } else {
                 if (owner) T.part[(size_t)u * T.slot_elems + ctid] = val;
@@ -385,20 +461,16 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 named_bar_sync(kConsBar, NCT);
                 if (last_flag) {
                     // the leader's acquire + the barrier order these loads after every partial
-                    if (owner) {
-                        float sum[1];
-                        ordered_unit_sums<1, 8>(T.part + (size_t)us.u0 * T.slot_elems, T.slot_elems, 0, ctid, 0,
-                                                1, us.nu, sum);
-                        if (live) {
-                            const size_t o = (size_t)o_m * T.N + n;
-                            T.Y[o] = __float2bfloat16_rn(sum[0]);
-                            if (T.Yf32) T.Yf32[o] = sum[0];
-                        }
-                    }
+                    float sum[1] = {0.f};
+                    if (owner)
+                        ordered_unit_sums<1, 8>(T.part + (size_t)us.u0 * T.slot_elems,
+                                                us.slot_stride * T.slot_elems, 0, ctid, 0, 1, us.nu, sum);
+                    emit_one(T, n, o_m, live, sum[0]);
                     named_bar_sync(kConsBar, NCT);
                     if (leader) {
                         T.tile_cnt[g] = 0u;
                         if (T.notify) red_release_gpu_add(T.done, 1u);
+                        if (T.col_cnt) notify_columns(T, g, TN);
                     }
                 }
             }

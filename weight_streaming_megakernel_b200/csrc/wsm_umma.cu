@@ -129,14 +129,43 @@ constexpr uint32_t kTmemCols = kAccBufs * kUmmaMaxN;
 
 __device__ __forceinline__ void epi_bar(int set) { named_bar_sync(1 + set, kEpiThreads); }
 
-// The last unit of a split tile adds the tile's nu partials (slots u0 ..
-// u0 + nu - 1) for its row, in unit order (= K order).  Partial slots are
-// [128 rows][t_mpad] floats, so a thread's values are contiguous: 16-byte
-// loads, CB units x MB rows in flight.
+// Epilogue of one thread's outputs: row n of W (output column n), X rows
+// m0 .. m0 + cnt - 1, fp32 values v.  Plain, residual add, or SiLU*mul, then
+// one rounding to bf16.  For SiLU*mul the up value of gate row n comes from
+// the thread of row n + 8 (lane ^ 8): every lane of the warp calls this with
+// the same cnt.
+template <int MB>
+__device__ __forceinline__ void emit_outputs(const TaskDev &T, int n, int m0, int cnt, const float (&v)[MB]) {
+#pragma unroll
+    for (int i = 0; i < MB; ++i) {
+        if (i >= cnt) break;  // uniform across the warp
+        float y = v[i];
+        size_t o;
+        if (T.epi == kEpiSiluMul) {
+            const float up = __shfl_xor_sync(0xffffffffu, y, 8);
+            if ((n & 8) || n >= T.N) continue;
+            y = y / (1.f + expf(-y)) * up;
+            o = (size_t)(m0 + i) * T.y_cols + ((n >> 4) << 3) + (n & 7);
+        } else {
+            if (n >= T.N) continue;
+            o = (size_t)(m0 + i) * T.N + n;
+            if (T.epi == kEpiResidual) y += __bfloat162float(T.R[o]);
+        }
+        T.Y[o] = __float2bfloat16_rn(y);
+        if (T.Yf32) T.Yf32[o] = y;
+    }
+}
+
+// The last unit of a split tile adds the tile's nu partials (slots u0 +
+// j * stride, j = 0 .. nu - 1) for its row, in unit order (= K order), and
+// writes the outputs.  Partial slots are [128 rows][t_mpad] floats, so a
+// thread's values are contiguous: 16-byte loads, CB units x MB rows in flight.
 template <int MB, int CB>
-__device__ __forceinline__ void reduce_row_partials(const TaskDev &T, int u0, int nu, int row, int mrows, int m0,
-                                                    int n) {
-    const float *base = T.part + (size_t)u0 * T.slot_elems + (size_t)row * T.t_mpad;
+__device__ __forceinline__ void reduce_row_partials(const TaskDev &T, const UnitSpan &us, int row, int mrows,
+                                                    int m0, int n) {
+    const int nu = us.nu;
+    const size_t step = (size_t)us.slot_stride * T.slot_elems;
+    const float *base = T.part + (size_t)us.u0 * T.slot_elems + (size_t)row * T.t_mpad;
     for (int mb = 0; mb < mrows; mb += MB) {
         float sum[MB];
 #pragma unroll
@@ -145,7 +174,7 @@ __device__ __forceinline__ void reduce_row_partials(const TaskDev &T, int u0, in
             float4 v[CB][MB / 4];
 #pragma unroll
             for (int u = 0; u < CB; ++u) {
-                const float4 *q = reinterpret_cast<const float4 *>(base + (size_t)(jb + u) * T.slot_elems + mb);
+                const float4 *q = reinterpret_cast<const float4 *>(base + (size_t)(jb + u) * step + mb);
 #pragma unroll
                 for (int i = 0; i < MB / 4; ++i)
                     v[u][i] = (jb + u < nu && mb + 4 * i < mrows) ? __ldcg(q + i) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -166,16 +195,7 @@ __device__ __forceinline__ void reduce_row_partials(const TaskDev &T, int u0, in
                 }
             }
         }
-        if (n < T.N) {
-#pragma unroll
-            for (int i = 0; i < MB; ++i) {
-                if (mb + i < mrows) {
-                    const size_t o = (size_t)(m0 + mb + i) * T.N + n;
-                    T.Y[o] = __float2bfloat16_rn(sum[i]);
-                    if (T.Yf32) T.Yf32[o] = sum[i];
-                }
-            }
-        }
+        emit_outputs<MB>(T, n, m0 + mb, min(MB, mrows - mb), sum);
     }
 }
 
@@ -240,17 +260,64 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 bool dep_ok = T.dep < 0 && grid_dep_ok;
                 int pend_s[kMaxStages], pend_k[kMaxStages], pend_y[kMaxStages];
                 int np = 0;
+                // Per-column dependency: each stage's X waits only for the kColChunk-column chunks it
+                // reads (seen-complete chunks are cached in chunk_mask).
+                const bool col_dep = T.dep >= 0 && T.dep_col_cnt != nullptr;
+                unsigned long long chunk_mask = 0;
+                unsigned int run_no = 0;
+                auto stage_chunks = [&](int k0, int &c0, int &c1) {
+                    c0 = k0 / kColChunk;
+                    c1 = (min(k0 + p.kps * kUmmaBK, T.K) - 1) / kColChunk;
+                };
+                auto x_now = [&](int k0) -> bool {  // may this stage's X load go out now?
+                    if (!dep_ok) return false;
+                    if (!col_dep) return true;
+                    int c0, c1;
+                    stage_chunks(k0, c0, c1);
+                    for (int c = c0; c <= c1; ++c)
+                        if (c >= 64 || !((chunk_mask >> c) & 1ull)) return false;
+                    return true;
+                };
+                // While this CTA waits (for the previous kernel or a dependency) HBM would idle: prefetch
+                // into L2 the W of the units it would own in a round-robin (c, c + G, ...), except the
+                // first ring-full of each first-round unit (some CTA's ring already holds it).
+                bool prefetched = p.prefetch_stages <= 0;
+                auto prefetch_l2 = [&]() {
+                    if (prefetched) return;
+                    prefetched = true;
+                    int budget = p.prefetch_stages;
+                    for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
+                        const UnitSpan ps = unit_span(T, uu);
+                        int pg, pmt;
+                        tile_coords(T, ps.tile, pg, pmt);
+                        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? S : 0); kk < ps.k_end && budget > 0;
+                             ++kk, --budget)
+                            for (int j = 0; j < p.kps; ++j)
+                                tma_prefetch_l2_2d(&T.tmW, (kk * p.kps + j) * kUmmaBK, pg * kUmmaRows);
+                    }
+                };
                 auto flush = [&]() {
                     if (!grid_dep_ok) {
+                        prefetch_l2();
                         pdl_wait();
                         grid_dep_ok = true;
                     }
-                    if (T.dep >= 0) wait_dependency(p, task_at(p, T.dep), t, p.status);
-                    trace_stamp(p, t, 1, globaltimer());
-                    for (int i = 0; i < np; ++i)
+                    if (T.dep >= 0 && !col_dep) {
+                        if (!prefetched && !dependency_met(p, task_at(p, T.dep))) prefetch_l2();
+                        wait_dependency(p, task_at(p, T.dep), t, p.status);
+                    }
+                    if (col_dep && run_no == 0) run_no = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
+                    if (!dep_ok) trace_stamp(p, t, 1, globaltimer());
+                    for (int i = 0; i < np; ++i) {
+                        if (col_dep) {
+                            int c0, c1;
+                            stage_chunks(pend_k[i], c0, c1);
+                            wait_chunks(p, T, c0, c1, run_no, chunk_mask, t, p.status);
+                        }
                         for (int j = 0; j < p.kps; ++j)
                             tma_load_2d(ring + (size_t)pend_s[i] * p.stage_bytes + p.x_off + j * p.x_stride, &T.tmX,
                                         &full_bar[pend_s[i]], pend_k[i] + j * kUmmaBK, pend_y[i], pol_x);
+                    }
                     np = 0;
                     dep_ok = true;
                 };
@@ -268,9 +335,21 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     return true;
                 };
                 bool first_unit = true;
-                // the first unit of each CTA is its own index (no atomic); later ones are claimed
-                const int n_static = min((int)gridDim.x, T.n_units);
-                int u = (int)blockIdx.x < T.n_units ? (int)blockIdx.x : T.n_units;
+                // The kernel's first task hands unit c to CTA c (no atomic, and it can stream before the
+                // grid dependency); later tasks hand out every unit by claim, so the CTAs that finish the
+                // previous task first take the next task's work.
+                const int n_static = (t == 0) ? min((int)gridDim.x, T.n_units) : 0;
+                int u;
+                if (t == 0) {
+                    u = (int)blockIdx.x < T.n_units ? (int)blockIdx.x : T.n_units;
+                } else {
+                    if (!grid_dep_ok) {
+                        pdl_wait();
+                        grid_dep_ok = true;
+                        dep_ok = T.dep < 0;
+                    }
+                    u = claim_unit(T);
+                }
                 while (u < T.n_units) {
                     if (first_unit) {
                         trace_stamp(p, t, 0, globaltimer());
@@ -295,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         for (int j = 0; j < p.kps; ++j)
                             tma_load_2d(st + j * (kUmmaRows * kUmmaBK * 2), &T.tmW, &full_bar[s], k0 + j * kUmmaBK,
                                         g * kUmmaRows, pol_w);
-                        if (dep_ok) {
+                        if (x_now(k0)) {
                             for (int j = 0; j < p.kps; ++j)
                                 tma_load_2d(st + p.x_off + j * p.x_stride, &T.tmX, &full_bar[s], k0 + j * kUmmaBK, xy,
                                             pol_x);
@@ -312,17 +391,18 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         }
                         // claim the next unit kClaimLead stages before this one ends: early enough to
                         // hide the claim's round trip, late enough not to hold work a faster CTA could
-                        // take (the claim counters belong to the previous kernel until the grid
-                        // dependency is resolved)
-                        if (!claimed && grid_dep_ok && us.k_end - kk <= kClaimLead) {
+                        // take -- and never while this task's dependency is unmet, when every CTA would
+                        // hold a second unit it cannot start (the claim counters belong to the previous
+                        // kernel until the grid dependency is resolved)
+                        if (!claimed && dep_ok && us.k_end - kk <= kClaimLead) {
                             next_u = claim_unit(T);
                             claimed = true;
                         }
                     }
                     if (aborted) break;
                     if (!claimed) {
-                        // the first unit streamed completely before the grid dependency was resolved
-                        if (!grid_dep_ok) flush();
+                        // the unit streamed completely before its dependencies were resolved
+                        if (!dep_ok) flush();
                         next_u = claim_unit(T);
                     }
                     // whatever comes next needs a free slot: wait for it before the claim's result is used,
@@ -470,19 +550,13 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             const int m0 = mt * T.t_m;
             const int mrows = min(T.t_m, T.M - m0);
             if (us.nu == 1) {
-                if (n < T.N) {
-#pragma unroll
-                    for (int m = 0; m < kUmmaMaxN; ++m) {
-                        if (m < mrows) {
-                            const size_t o = (size_t)(m0 + m) * T.N + n;
-                            T.Y[o] = __float2bfloat16_rn(acc[m]);
-                            if (T.Yf32) T.Yf32[o] = acc[m];
-                        }
-                    }
-                }
-                if (T.notify) {
+                emit_outputs<kUmmaMaxN>(T, n, m0, mrows, acc);
+                if (T.notify || T.col_cnt) {
                     epi_bar(set);
-                    if (leader) red_release_gpu_add(T.done, 1u);  // release covers the set's stores (bar.sync before)
+                    if (leader) {  // release covers the set's stores (bar.sync before)
+                        if (T.notify) red_release_gpu_add(T.done, 1u);
+                        if (T.col_cnt) notify_columns(T, g, kUmmaRows);
+                    }
                 }
             } else {
                 // split tile: store this unit's partial row; the last unit of the tile to arrive adds all of them
@@ -501,13 +575,14 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 if (last_flag[set]) {
                     // the leader's acquire + the barrier order these loads after every partial
                     if (mrows <= 4)
-                        reduce_row_partials<4, 16>(T, us.u0, us.nu, row, mrows, m0, n);
+                        reduce_row_partials<4, 16>(T, us, row, mrows, m0, n);
                     else
-                        reduce_row_partials<16, 4>(T, us.u0, us.nu, row, mrows, m0, n);
+                        reduce_row_partials<16, 4>(T, us, row, mrows, m0, n);
                     epi_bar(set);
                     if (leader) {
                         T.tile_cnt[tile] = 0u;  // ready for the next call
                         if (T.notify) red_release_gpu_add(T.done, 1u);
+                        if (T.col_cnt) notify_columns(T, g, kUmmaRows);
                     }
                 }
             }
