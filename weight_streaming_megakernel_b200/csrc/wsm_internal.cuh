@@ -281,10 +281,18 @@ __device__ __forceinline__ bool status_set(const int *status) {
 }
 
 // Bounded wait on an mbarrier phase.  Returns false (and records an error)
-// when `limit_ns` of %globaltimer pass, or when `abort_flag` is raised.
+// when `limit_ns` of %globaltimer pass, or when `abort_flag` is raised.  The
+// spin loop is a real call (not inlined at the many wait sites): the
+// kernels' hot code stays small enough for the instruction caches.
+static __device__ __noinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                            unsigned long long limit_ns, int *status, int task, int site);
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                   unsigned long long limit_ns, int *status, int task, int site) {
     if (mbar_try(bar, parity)) return true;
+    return mbar_wait_spin(bar, parity, abort_flag, limit_ns, status, task, site);
+}
+static __device__ __noinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                            unsigned long long limit_ns, int *status, int task, int site) {
     unsigned long long t0 = globaltimer();
     for (uint32_t spin = 1;; ++spin) {
         if (mbar_try(bar, parity)) return true;
@@ -425,28 +433,77 @@ __device__ __forceinline__ void ordered_unit_sums(const float *tile_slots, int s
 // The run number is read from device memory (not a launch parameter) so a
 // chain captured once in a CUDA graph stays correct over any number of
 // replays; the last CTA to finish a run advances it (chain_run_done).
-// A finished tile of task T (column tile g, rows_per_tile rows of W) counts
-// toward every kColChunk-column chunk of the output it wrote.  Called by one
-// thread after a barrier that follows all the tile's stores (release).
-__device__ __forceinline__ void notify_columns(const TaskDev &T, int g, int rows_per_tile) {
+// What an epilogue writes, copied out of the task table into registers once
+// per unit: loads through the table reference cannot be hoisted over the
+// output stores (they might alias), and each reload is an L2 round trip.
+struct EpiOut {
+    __nv_bfloat16 *Y;
+    float *Yf32;
+    const __nv_bfloat16 *R;
+    int N, y_cols, epi;
+};
+__device__ __forceinline__ EpiOut epi_out(const TaskDev &T) {
+    EpiOut e;
+    e.Y = T.Y;
+    e.Yf32 = T.Yf32;
+    e.R = T.R;
+    e.N = T.N;
+    e.y_cols = T.y_cols;
+    e.epi = T.epi;
+    return e;
+}
+
+// Everything a unit's epilogue touches after its first store, in registers
+// (see EpiOut).
+struct UnitOut {
+    EpiOut e;
+    float *part;
+    unsigned int *tile_cnt;
+    unsigned int *done;     // nullptr unless some task waits for this whole task
+    unsigned int *col_cnt;  // nullptr unless some task waits for its columns
+    int slot_elems, t_mpad;
+};
+__device__ __forceinline__ UnitOut unit_out(const TaskDev &T) {
+    UnitOut o;
+    o.e = epi_out(T);
+    o.part = T.part;
+    o.tile_cnt = T.tile_cnt;
+    o.done = T.notify ? T.done : nullptr;
+    o.col_cnt = T.col_cnt;
+    o.slot_elems = T.slot_elems;
+    o.t_mpad = T.t_mpad;
+    return o;
+}
+
+// A finished tile (column tile g, rows_per_tile rows of W) counts toward every
+// kColChunk-column chunk of the output it wrote.  Called by one thread after a
+// barrier that follows all the tile's stores (release).
+__device__ __forceinline__ void notify_columns(const UnitOut &o, int g, int rows_per_tile) {
     int c_lo = g * rows_per_tile;
-    int c_hi = min(T.N, c_lo + rows_per_tile);
-    if (T.epi == kEpiSiluMul) {  // N and the tile heights are multiples of 16
+    int c_hi = min(o.e.N, c_lo + rows_per_tile);
+    if (o.e.epi == kEpiSiluMul) {  // N and the tile heights are multiples of 16
         c_lo >>= 1;
         c_hi >>= 1;
     }
-    for (int c = c_lo / kColChunk; c <= (c_hi - 1) / kColChunk; ++c) red_release_gpu_add(&T.col_cnt[c], 1u);
+    for (int c = c_lo / kColChunk; c <= (c_hi - 1) / kColChunk; ++c) red_release_gpu_add(&o.col_cnt[c], 1u);
+}
+
+// The tile is complete: whole-task and per-column readiness (leader thread,
+// after the barrier that follows the tile's last stores).
+__device__ __forceinline__ void tile_finished(const UnitOut &o, int g, int rows_per_tile) {
+    if (o.done) red_release_gpu_add(o.done, 1u);
+    if (o.col_cnt) notify_columns(o, g, rows_per_tile);
 }
 
 // Per-column dependency: wait (bounded) until the chunks c0 .. c1 of the dep
 // task's output are complete in run `run`; `mask` caches chunks < 64 already
 // seen complete (they stay complete for the rest of the run).
-__device__ __forceinline__ void wait_chunks(const KParams &p, const TaskDev &T, int c0, int c1, unsigned int run,
-                                            unsigned long long &mask, int task, int *status) {
+static __device__ __noinline__ void wait_chunks(const KParams &p, const TaskDev &T, int c0, int c1, unsigned int run,
+                                                unsigned long long &mask, int task, int *status) {
     for (int c = c0; c <= c1; ++c) {
         if (c < 64 && ((mask >> c) & 1ull)) continue;
         const unsigned int target = run * T.dep_col_need[c] + p.dep_target_extra;
-        if (ld_acquire_gpu(&T.dep_col_cnt[c]) - target >= 0x80000000u) {
+        if (ld_acquire_gpu(&T.dep_col_cnt[c]) - target >= 0x80000000u) {  // counter < target (wrap-safe)
             const unsigned long long t0 = globaltimer();
             for (uint32_t spin = 1;; ++spin) {
                 if (ld_acquire_gpu(&T.dep_col_cnt[c]) - target < 0x80000000u) break;
@@ -471,7 +528,7 @@ __device__ __forceinline__ bool dependency_met(const KParams &p, const TaskDev &
     return ld_acquire_gpu(D.done) - target < 0x80000000u;  // done >= target (wrap-safe)
 }
 
-__device__ __forceinline__ void wait_dependency(const KParams &p, const TaskDev &D, int task, int *status) {
+static __device__ __noinline__ void wait_dependency(const KParams &p, const TaskDev &D, int task, int *status) {
     const unsigned int run = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
     const unsigned int target = run * (unsigned int)(D.n_g * D.n_mt) + p.dep_target_extra;
     if (ld_acquire_gpu(D.done) - target < 0x80000000u) {  // done >= target (wrap-safe)

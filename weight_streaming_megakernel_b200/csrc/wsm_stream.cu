@@ -45,20 +45,20 @@ constexpr int kConsBar = 1;
 // Epilogue of one output (row n of W, X row m): plain, residual add, or
 // SiLU*mul (the up value of gate row n comes from the thread owning row n + 8,
 // lane ^ 8: every lane of the warp calls this), then one rounding to bf16.
-__device__ __forceinline__ void emit_one(const TaskDev &T, int n, int m, bool live, float y) {
+__device__ __forceinline__ void emit_one(const EpiOut &e, int n, int m, bool live, float y) {
     size_t o;
-    if (T.epi == kEpiSiluMul) {
+    if (e.epi == kEpiSiluMul) {
         const float up = __shfl_xor_sync(0xffffffffu, y, 8);
         if (!live || (n & 8)) return;
         y = y / (1.f + expf(-y)) * up;
-        o = (size_t)m * T.y_cols + ((n >> 4) << 3) + (n & 7);
+        o = (size_t)m * e.y_cols + ((n >> 4) << 3) + (n & 7);
     } else {
         if (!live) return;
-        o = (size_t)m * T.N + n;
-        if (T.epi == kEpiResidual) y += __bfloat162float(T.R[o]);
+        o = (size_t)m * e.N + n;
+        if (e.epi == kEpiResidual) y += __bfloat162float(e.R[o]);
     }
-    T.Y[o] = __float2bfloat16_rn(y);
-    if (T.Yf32) T.Yf32[o] = y;
+    e.Y[o] = __float2bfloat16_rn(y);
+    if (e.Yf32) e.Yf32[o] = y;
 }
 
 // Barrier among the consumer warps that also ORs a predicate over them.
@@ -117,6 +117,20 @@ struct LaneReduce {
 
 }  // namespace
 
+// L2 prefetch of the W of the units this CTA would own in a round-robin (c,
+// c + G, ...), p.prefetch_stages stages at most, skipping the first S stages
+// of each first-round unit (some CTA's ring holds them).  Out of line: it runs
+// at most once per task.
+static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDev &T, int S, int KW, int TN) {
+    int budget = p.prefetch_stages;
+    for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
+        const UnitSpan ps = unit_span(T, uu);
+        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? S : 0); kk < ps.k_end && budget > 0; ++kk, --budget)
+            for (int kw = 0; kw < KW; ++kw)
+                tma_prefetch_l2_2d(&T.tmW, kk * (KW * kStreamBoxK) + kw * kStreamBoxK, ps.tile * TN);
+    }
+}
+
 // MMAX: largest M handled (register arrays); RW rows per warp; RG row groups;
 // KW K-slices.  Consumer warps = RG*KW = 8; T_N = RG*RW; T_K = KW*256.
 template <int MMAX, int RW, int RG, int KW>
@@ -169,12 +183,14 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 prefetch_tmap(&T.tmW);
                 prefetch_tmap(&T.tmX);
                 const uint64_t pol_w = T.w_evict_first ? policy_evict_first() : policy_evict_normal();
+                const bool col_dep = T.dep >= 0 && T.dep_col_cnt != nullptr;
+                // nothing of X before the dependency is met (per column: the first chunks; after that the
+                // chunk mask decides stage by stage)
                 bool dep_ok = T.dep < 0 && grid_dep_ok;
                 int pend_s[kMaxStages], pend_k[kMaxStages];
                 int np = 0;
                 // Per-column dependency: each stage's X waits only for the kColChunk-column chunks it
                 // reads (seen-complete chunks are cached in chunk_mask).
-                const bool col_dep = T.dep >= 0 && T.dep_col_cnt != nullptr;
                 unsigned long long chunk_mask = 0;
                 unsigned int run_no = 0;
                 auto stage_chunks = [&](int k0, int &c0, int &c1) {
@@ -197,15 +213,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 auto prefetch_l2 = [&]() {
                     if (prefetched) return;
                     prefetched = true;
-                    int budget = p.prefetch_stages;
-                    for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
-                        const UnitSpan ps = unit_span(T, uu);
-                        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? S : 0); kk < ps.k_end && budget > 0;
-                             ++kk, --budget)
-#pragma unroll
-                            for (int kw = 0; kw < KW; ++kw)
-                                tma_prefetch_l2_2d(&T.tmW, kk * (KW * kStreamBoxK) + kw * kStreamBoxK, ps.tile * TN);
-                    }
+                    prefetch_w_l2(p, T, S, KW, TN);
                 };
                 auto flush = [&]() {
                     if (!grid_dep_ok) {
@@ -440,22 +448,20 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
             const int g = us.tile;
             const int n = g * TN + o_row;
             const bool live = owner && o_m < M && n < T.N;
+            const UnitOut uo = unit_out(T);  // no task-table reads after the first store below
             if (us.nu == 1) {
-                emit_one(T, n, o_m, live, val);
-                if (T.notify || T.col_cnt) {
+                emit_one(uo.e, n, o_m, live, val);
+                if (uo.done || uo.col_cnt) {
                     named_bar_sync(kConsBar, NCT);
-                    if (leader) {  // release covers the CTA's stores (bar.sync before)
-                        if (T.notify) red_release_gpu_add(T.done, 1u);
-                        if (T.col_cnt) notify_columns(T, g, TN);
-                    }
+                    if (leader) tile_finished(uo, g, TN);  // release covers the CTA's stores (bar.sync before)
                 }
             } else {
-                if (owner) T.part[(size_t)u * T.slot_elems + ctid] = val;
+                if (owner) uo.part[(size_t)u * uo.slot_elems + ctid] = val;
                 named_bar_sync(kConsBar, NCT);
                 if (leader) {
                     // acq_rel: releases this CTA's partial (stored before the barrier) and acquires the
                     // others' for the last arriver
-                    const unsigned int old = atom_add_acqrel_gpu(&T.tile_cnt[g], 1u);
+                    const unsigned int old = atom_add_acqrel_gpu(&uo.tile_cnt[g], 1u);
                     last_flag = (old == (unsigned int)(us.nu - 1)) ? 1 : 0;
                 }
                 named_bar_sync(kConsBar, NCT);
@@ -463,14 +469,13 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     // the leader's acquire + the barrier order these loads after every partial
                     float sum[1] = {0.f};
                     if (owner)
-                        ordered_unit_sums<1, 8>(T.part + (size_t)us.u0 * T.slot_elems,
-                                                us.slot_stride * T.slot_elems, 0, ctid, 0, 1, us.nu, sum);
-                    emit_one(T, n, o_m, live, sum[0]);
+                        ordered_unit_sums<1, 8>(uo.part + (size_t)us.u0 * uo.slot_elems,
+                                                us.slot_stride * uo.slot_elems, 0, ctid, 0, 1, us.nu, sum);
+                    emit_one(uo.e, n, o_m, live, sum[0]);
                     named_bar_sync(kConsBar, NCT);
                     if (leader) {
-                        T.tile_cnt[g] = 0u;
-                        if (T.notify) red_release_gpu_add(T.done, 1u);
-                        if (T.col_cnt) notify_columns(T, g, TN);
+                        uo.tile_cnt[g] = 0u;
+                        tile_finished(uo, g, TN);
                     }
                 }
             }

@@ -133,26 +133,34 @@ __device__ __forceinline__ void epi_bar(int set) { named_bar_sync(1 + set, kEpiT
 // m0 .. m0 + cnt - 1, fp32 values v.  Plain, residual add, or SiLU*mul, then
 // one rounding to bf16.  For SiLU*mul the up value of gate row n comes from
 // the thread of row n + 8 (lane ^ 8): every lane of the warp calls this with
-// the same cnt.
+// the same cnt.  The epilogue kind is branched on once, outside the loops.
 template <int MB>
-__device__ __forceinline__ void emit_outputs(const TaskDev &T, int n, int m0, int cnt, const float (&v)[MB]) {
+__device__ __forceinline__ void emit_outputs(const EpiOut &e, int n, int m0, int cnt, const float (&v)[MB]) {
+    if (e.epi == kEpiSiluMul) {
+        const bool writer = !(n & 8) && n < e.N;
+        const size_t col = ((size_t)(n >> 4) << 3) + (n & 7);
+#pragma unroll
+        for (int i = 0; i < MB; ++i) {
+            if (i >= cnt) break;  // uniform across the warp
+            const float up = __shfl_xor_sync(0xffffffffu, v[i], 8);
+            if (writer) {
+                const float y = v[i] / (1.f + expf(-v[i])) * up;
+                const size_t o = (size_t)(m0 + i) * e.y_cols + col;
+                e.Y[o] = __float2bfloat16_rn(y);
+                if (e.Yf32) e.Yf32[o] = y;
+            }
+        }
+        return;
+    }
+    if (n >= e.N) return;
+    const bool res = e.epi == kEpiResidual;
 #pragma unroll
     for (int i = 0; i < MB; ++i) {
-        if (i >= cnt) break;  // uniform across the warp
-        float y = v[i];
-        size_t o;
-        if (T.epi == kEpiSiluMul) {
-            const float up = __shfl_xor_sync(0xffffffffu, y, 8);
-            if ((n & 8) || n >= T.N) continue;
-            y = y / (1.f + expf(-y)) * up;
-            o = (size_t)(m0 + i) * T.y_cols + ((n >> 4) << 3) + (n & 7);
-        } else {
-            if (n >= T.N) continue;
-            o = (size_t)(m0 + i) * T.N + n;
-            if (T.epi == kEpiResidual) y += __bfloat162float(T.R[o]);
-        }
-        T.Y[o] = __float2bfloat16_rn(y);
-        if (T.Yf32) T.Yf32[o] = y;
+        if (i >= cnt) break;
+        const size_t o = (size_t)(m0 + i) * e.N + n;
+        const float y = res ? v[i] + __bfloat162float(e.R[o]) : v[i];
+        e.Y[o] = __float2bfloat16_rn(y);
+        if (e.Yf32) e.Yf32[o] = y;
     }
 }
 
@@ -161,11 +169,12 @@ __device__ __forceinline__ void emit_outputs(const TaskDev &T, int n, int m0, in
 // writes the outputs.  Partial slots are [128 rows][t_mpad] floats, so a
 // thread's values are contiguous: 16-byte loads, CB units x MB rows in flight.
 template <int MB, int CB>
-__device__ __forceinline__ void reduce_row_partials(const TaskDev &T, const UnitSpan &us, int row, int mrows,
+__device__ __forceinline__ void reduce_row_partials(const UnitOut &uo, const UnitSpan &us, int row, int mrows,
                                                     int m0, int n) {
     const int nu = us.nu;
-    const size_t step = (size_t)us.slot_stride * T.slot_elems;
-    const float *base = T.part + (size_t)us.u0 * T.slot_elems + (size_t)row * T.t_mpad;
+    const size_t step = (size_t)us.slot_stride * uo.slot_elems;
+    const float *base = uo.part + (size_t)us.u0 * uo.slot_elems + (size_t)row * uo.t_mpad;
+    const EpiOut &e = uo.e;
     for (int mb = 0; mb < mrows; mb += MB) {
         float sum[MB];
 #pragma unroll
@@ -195,11 +204,26 @@ __device__ __forceinline__ void reduce_row_partials(const TaskDev &T, const Unit
                 }
             }
         }
-        emit_outputs<MB>(T, n, m0 + mb, min(MB, mrows - mb), sum);
+        emit_outputs<MB>(e, n, m0 + mb, min(MB, mrows - mb), sum);
     }
 }
 
 }  // namespace
+
+// L2 prefetch of the W of the units this CTA would own in a round-robin (c,
+// c + G, ...), p.prefetch_stages stages at most, skipping the first S stages
+// of each first-round unit (some CTA's ring holds them).  Out of line: it runs
+// at most once per task.
+static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDev &T, int S) {
+    int budget = p.prefetch_stages;
+    for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
+        const UnitSpan ps = unit_span(T, uu);
+        int pg, pmt;
+        tile_coords(T, ps.tile, pg, pmt);
+        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? S : 0); kk < ps.k_end && budget > 0; ++kk, --budget)
+            for (int j = 0; j < p.kps; ++j) tma_prefetch_l2_2d(&T.tmW, (kk * p.kps + j) * kUmmaBK, pg * kUmmaRows);
+    }
+}
 
 __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_constant__ KParams p) {
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -257,12 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 prefetch_tmap(&T.tmW);
                 prefetch_tmap(&T.tmX);
                 const uint64_t pol_w = T.w_evict_first ? policy_evict_first() : policy_evict_normal();
+                const bool col_dep = T.dep >= 0 && T.dep_col_cnt != nullptr;
+                // nothing of X before the dependency is met (per column: the first chunks; after that the
+                // chunk mask decides stage by stage)
                 bool dep_ok = T.dep < 0 && grid_dep_ok;
                 int pend_s[kMaxStages], pend_k[kMaxStages], pend_y[kMaxStages];
                 int np = 0;
                 // Per-column dependency: each stage's X waits only for the kColChunk-column chunks it
                 // reads (seen-complete chunks are cached in chunk_mask).
-                const bool col_dep = T.dep >= 0 && T.dep_col_cnt != nullptr;
                 unsigned long long chunk_mask = 0;
                 unsigned int run_no = 0;
                 auto stage_chunks = [&](int k0, int &c0, int &c1) {
@@ -285,16 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 auto prefetch_l2 = [&]() {
                     if (prefetched) return;
                     prefetched = true;
-                    int budget = p.prefetch_stages;
-                    for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
-                        const UnitSpan ps = unit_span(T, uu);
-                        int pg, pmt;
-                        tile_coords(T, ps.tile, pg, pmt);
-                        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? S : 0); kk < ps.k_end && budget > 0;
-                             ++kk, --budget)
-                            for (int j = 0; j < p.kps; ++j)
-                                tma_prefetch_l2_2d(&T.tmW, (kk * p.kps + j) * kUmmaBK, pg * kUmmaRows);
-                    }
+                    prefetch_w_l2(p, T, S);
                 };
                 auto flush = [&]() {
                     if (!grid_dep_ok) {
@@ -520,28 +537,6 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             const int t = acc_meta[buf][0];
             const int u = acc_meta[buf][1];
             const TaskDev &T = task_at(p, t);
-            float acc[kUmmaMaxN];
-            {
-                tc_fence_after();
-                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kUmmaMaxN);
-                uint32_t r[kUmmaMaxN / 16][16];
-#pragma unroll
-                for (int c16 = 0; c16 < kUmmaMaxN / 16; ++c16) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) r[c16][i] = 0u;
-                    if (c16 * 16 < T.t_mpad) tmem_ld16(taddr + (uint32_t)(c16 * 16), r[c16]);
-                }
-#pragma unroll
-                for (int c16 = 0; c16 < kUmmaMaxN / 16; ++c16) tmem_ld_wait16(r[c16]);
-#pragma unroll
-                for (int c16 = 0; c16 < kUmmaMaxN / 16; ++c16)
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[c16 * 16 + i] = __uint_as_float(r[c16][i]);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acce_bar[buf]);
-
             const UnitSpan us = unit_span(T, u);
             const int tile = us.tile;
             int g, mt;
@@ -549,40 +544,58 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             const int n = g * kUmmaRows + row;
             const int m0 = mt * T.t_m;
             const int mrows = min(T.t_m, T.M - m0);
+            const UnitOut uo = unit_out(T);  // no task-table reads after the first store below
+            // The accumulator, 16 columns (X rows) at a time: TMEM -> registers -> outputs (whole tile) or
+            // this unit's partial row [row][m] (split tile).  The loop is not unrolled: one copy of the
+            // epilogue code per kind keeps the kernel small.
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kUmmaMaxN);
+            float4 *dst = reinterpret_cast<float4 *>(uo.part + (size_t)u * uo.slot_elems + (size_t)row * uo.t_mpad);
+#pragma unroll 1
+            for (int c = 0; c < mrows; c += 16) {
+                uint32_t r[16];
+                tmem_ld16(taddr + (uint32_t)c, r);
+                tmem_ld_wait16(r);
+                float v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+                if (us.nu == 1) {
+                    emit_outputs<16>(uo.e, n, m0 + c, min(16, mrows - c), v);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (c + 4 * i < mrows) dst[c / 4 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce_bar[buf]);
+
             if (us.nu == 1) {
-                emit_outputs<kUmmaMaxN>(T, n, m0, mrows, acc);
-                if (T.notify || T.col_cnt) {
+                if (uo.done || uo.col_cnt) {
                     epi_bar(set);
-                    if (leader) {  // release covers the set's stores (bar.sync before)
-                        if (T.notify) red_release_gpu_add(T.done, 1u);
-                        if (T.col_cnt) notify_columns(T, g, kUmmaRows);
-                    }
+                    if (leader) tile_finished(uo, g, kUmmaRows);  // release covers the set's stores (bar.sync before)
                 }
             } else {
-                // split tile: store this unit's partial row; the last unit of the tile to arrive adds all of them
-                float4 *dst = reinterpret_cast<float4 *>(T.part + (size_t)u * T.slot_elems + (size_t)row * T.t_mpad);
-#pragma unroll
-                for (int i = 0; i < kUmmaMaxN / 4; ++i)
-                    if (4 * i < mrows) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+                // the last unit of the tile to arrive adds all the partials
                 epi_bar(set);
                 if (leader) {
                     // acq_rel: releases this set's partial (stored before the barrier) and acquires the
                     // others' for the last arriver
-                    const unsigned int old = atom_add_acqrel_gpu(&T.tile_cnt[tile], 1u);
+                    const unsigned int old = atom_add_acqrel_gpu(&uo.tile_cnt[tile], 1u);
                     last_flag[set] = (old == (unsigned int)(us.nu - 1)) ? 1 : 0;
                 }
                 epi_bar(set);
                 if (last_flag[set]) {
                     // the leader's acquire + the barrier order these loads after every partial
                     if (mrows <= 4)
-                        reduce_row_partials<4, 16>(T, us, row, mrows, m0, n);
+                        reduce_row_partials<4, 16>(uo, us, row, mrows, m0, n);
                     else
-                        reduce_row_partials<16, 4>(T, us, row, mrows, m0, n);
+                        reduce_row_partials<16, 4>(uo, us, row, mrows, m0, n);
                     epi_bar(set);
                     if (leader) {
-                        T.tile_cnt[tile] = 0u;  // ready for the next call
-                        if (T.notify) red_release_gpu_add(T.done, 1u);
-                        if (T.col_cnt) notify_columns(T, g, kUmmaRows);
+                        uo.tile_cnt[tile] = 0u;  // ready for the next call
+                        tile_finished(uo, g, kUmmaRows);
                     }
                 }
             }
