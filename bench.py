@@ -95,6 +95,16 @@ def workload_cases(name):
     raise SystemExit(f"unknown workload {name}")
 
 
+L2_BYTES = 126 * 2 ** 20
+
+
+def n_copies(cases):
+    """Weight copies a step cycles through so that consecutive steps touch at
+    least 4x the L2 size (1 when one step's weights already do)."""
+    w = sum(2 * c.N * c.K for c in cases)
+    return max(1, -(-4 * L2_BYTES // w))
+
+
 def alg_bytes(c):
     """Algorithmic bytes of one GEMM: W read once + X read once (bf16)."""
     return 2 * c.N * c.K + 2 * c.M * c.K
@@ -193,7 +203,12 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
     if args.only:
         cases = [c for c in cases if c.name in args.only.split(",")]
         assert cases, f"no case named {args.only}"
-    data = setup_inputs(cases, dev, seed_base=rank)
+    # Inputs larger than L2 between timed steps: a step whose weights fit in
+    # L2 several times cycles through copies (step k uses copy k % copies).
+    copies = n_copies(cases)
+    datas = [setup_inputs(cases, dev, seed_base=rank * 1000 + r) for r in range(copies)]
+    data = datas[0]
+    cur = [0]  # copy the next launches use
     L = wsm.lib()
     stream = torch.cuda.Stream(dev)
     s = stream.cuda_stream
@@ -202,21 +217,25 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
     if mode == "chain":
         # the whole step is one persistent kernel; the layer chain orders task t after t-1
         deps = [(i - 1) if args.workload == "chain" else -1 for i in range(len(data))]
-        tasks = [wsm.Task(x, w, y, dep=deps[i]) for i, (c, x, w, y) in enumerate(data)]
-        chain = wsm.Chain(tasks, flags=wsm.FLAG_W_READONLY)
+        chains = [wsm.Chain([wsm.Task(x, w, y, dep=deps[i]) for i, (c, x, w, y) in enumerate(d)],
+                            flags=wsm.FLAG_W_READONLY) for d in datas]
+        chain = chains[0]
         launches_per_step = 1
 
         def launch(i):
-            chain.run(s)
+            chains[cur[0]].run(s)
     else:
-        calls = []
-        for c, x, w, y in data:
-            o = wsm._opts(m_tile=c.m_tile, flags=wsm.FLAG_W_READONLY)
-            calls.append((x.data_ptr(), w.data_ptr(), y.data_ptr(), c.M, c.N, c.K, o))
-        launches_per_step = len(calls)
+        callsets = []
+        for d in datas:
+            calls = []
+            for c, x, w, y in d:
+                o = wsm._opts(m_tile=c.m_tile, flags=wsm.FLAG_W_READONLY)
+                calls.append((x.data_ptr(), w.data_ptr(), y.data_ptr(), c.M, c.N, c.K, o))
+            callsets.append(calls)
+        launches_per_step = len(callsets[0])
 
         def launch(i):
-            xp, wp, yp, M, N, K, o = calls[i]
+            xp, wp, yp, M, N, K, o = callsets[cur[0]][i]
             rc = L.skinny_gemm_ex(xp, wp, yp, M, N, K, ctypes.byref(o), s) if o is not None else \
                 L.skinny_gemm(xp, wp, yp, M, N, K, s)
             if rc != 0:
@@ -234,7 +253,8 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
 
     # eager warm-up (also sizes the stream's scratch before any capture)
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
+        for k in range(max(args.warmup, copies)):
+            cur[0] = k % copies
             step()
     stream.synchronize()
 
@@ -243,14 +263,25 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
     evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nev)] for _ in range(n_steps)]
     graphs = []
     for k in range(n_steps):
+        cur[0] = k % copies
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             step(evs[k])
         graphs.append(g)
-    plain = torch.cuda.CUDAGraph()
+    plain = torch.cuda.CUDAGraph()  # all copies once each
     with torch.cuda.graph(plain, stream=stream):
-        step()
+        for r in range(copies):
+            cur[0] = r
+            step()
+    # the timed region: the K steps back to back in ONE graph, no events inside (launches keep their
+    # programmatic overlap across steps and pay one graph launch for all of them)
+    timed = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(timed, stream=stream):
+        for k in range(n_steps):
+            cur[0] = k % copies
+            step()
     with torch.cuda.stream(stream):
+        timed.replay()
         for g in graphs[: min(3, len(graphs))]:
             g.replay()
     stream.synchronize()
@@ -271,13 +302,17 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
     t_end = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         t_start.record(stream)
-        for g in graphs:
-            g.replay()
+        timed.replay()
         t_end.record(stream)
     stream.synchronize()
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
+    # per-launch durations (outside the timed region): the instrumented graphs, events between launches
+    with torch.cuda.stream(stream):
+        for g in graphs:
+            g.replay()
+    stream.synchronize()
     # keep the load on briefly so the window closes under load
     t_post = time.time()
     with torch.cuda.stream(stream):
@@ -303,7 +338,7 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
             plain.replay()
         b.record(stream)
     stream.synchronize()
-    plain_ms = a.elapsed_time(b) / n_steps
+    plain_ms = a.elapsed_time(b) / (n_steps * copies)
 
     # ---- e2e: public API, host buffers, H2D of X and D2H of Y inside the timed region
     e2e = None
@@ -313,20 +348,21 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
         h2d = sum(t.numel() * 2 for t in hx)
         d2h = sum(t.numel() * 2 for t in hy)
 
-        def e2e_step():
-            for (c, x, w, y), h in zip(data, hx):
+        def e2e_step(k):
+            d = datas[k % copies]
+            for (c, x, w, y), h in zip(d, hx):
                 x.copy_(h, non_blocking=True)
             if chain is not None:
-                chain.run(s)
+                chains[k % copies].run(s)
             else:
-                for c, x, w, y in data:
+                for c, x, w, y in d:
                     wsm.skinny_gemm(x, w, y, m_tile=c.m_tile, flags=wsm.FLAG_W_READONLY, stream=s)
-            for (c, x, w, y), h in zip(data, hy):
+            for (c, x, w, y), h in zip(d, hy):
                 h.copy_(y, non_blocking=True)
 
         with torch.cuda.stream(stream):
-            for _ in range(max(1, args.warmup)):
-                e2e_step()
+            for k in range(max(1, args.warmup)):
+                e2e_step(k)
         stream.synchronize()
         if world > 1:
             torch.distributed.barrier()
@@ -334,8 +370,8 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
         b = torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             a.record(stream)
-            for _ in range(n_steps):
-                e2e_step()
+            for k in range(n_steps):
+                e2e_step(k)
             b.record(stream)
         stream.synchronize()
         e_ms = a.elapsed_time(b)
@@ -346,13 +382,13 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
         e2e = {"value": round(total_bytes * world / (e_ms / n_steps * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    status = wsm.stream_status(stream) if chain is None else chain.status(s)[0]
+    status = wsm.stream_status(stream) if chain is None else max(c.status(s)[0] for c in chains)
     if status != 0:
         raise RuntimeError(f"device-side status {status}")
-    del graphs, plain
+    del graphs, plain, timed
     return dict(cases=cases, total_bytes=total_bytes, ms_per_step=ms_per_step, per_launch=per_launch,
                 clocks=clk, e2e=e2e, launches_per_step=launches_per_step, chain=chain is not None,
-                plain_ms=plain_ms)
+                plain_ms=plain_ms, copies=copies)
 
 
 # ----------------------------------------------------------------------------- CPU arm
@@ -428,7 +464,10 @@ def main():
               "shapes_KxN": sorted({f"{c.K}x{c.N}" for c in cases}),
               "weight_bytes_per_step": sum(2 * c.N * c.K for c in cases),
               "l2": "inputs larger than L2: every GEMM of a step has its own weights "
-                    f"({sum(2 * c.N * c.K for c in cases) / 1e9:.2f} GB per step, L2 126 MB)",
+                    f"({sum(2 * c.N * c.K for c in cases) / 1e9:.3f} GB per step, L2 126 MB)"
+                    + (f"; steps cycle through {n_copies(cases)} weight copies "
+                       f"({n_copies(cases) * sum(2 * c.N * c.K for c in cases) / 1e9:.2f} GB)"
+                       if n_copies(cases) > 1 else ""),
               "parallelism": f"replicas{world}" if world > 1 else "single",
               "mode": args.mode + (" (one persistent kernel per step, W read-only flag)" if args.mode == "chain"
                                    else " (one skinny_gemm launch per GEMM, W read-only flag)")}
@@ -478,7 +517,11 @@ def main():
         med = statistics.median(launch_ms)
         fam_bytes, fam_ms = r["total_bytes"], med
         us_per_gemm = {"chain_us": round(med * 1e3, 2), "per_gemm_us_avg": round(med * 1e3 / len(cases), 3)}
-        dominant = "wsm_umma_kernel" if max(c.M for c in cases) > 8 else "wsm_stream_kernel"
+        # the chain's path: FMA only if the automatic choice is FMA for every task at the largest M
+        from weight_streaming_megakernel_b200 import plan
+        mmax = max(c.M for c in cases)
+        fma = all(plan(mmax, c.N, c.K)["path"] == 1 for c in cases)
+        dominant = "wsm_stream_kernel" if fma else "wsm_umma_kernel"
     else:
         from weight_streaming_megakernel_b200 import plan
         fam = {}

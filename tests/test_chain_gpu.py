@@ -165,6 +165,28 @@ def test_gemm_chain_one_shot():
     check_dependent(x0, ws, ys, yfs)
 
 
+@pytest.mark.parametrize("deps", [False, True])
+def test_mixed_m_chain(deps):
+    """Tasks of different M in one chain share one stage geometry (the
+    widest X tile decides it): M = 1, 16, 33 and 64 mixed, with and without
+    ordering dependencies, on the tensor-core path."""
+    tasks = []
+    for t, (M, N, K) in enumerate([(16, 1024, 4096), (64, 2048, 2048), (1, 640, 3072), (33, 1000, 1032),
+                                   (64, 512, 8192), (16, 4096, 1024)]):
+        x, w = synth.make_xw(M, N, K, seed=40 + t)
+        tasks.append(wsm.Task(x.to(DEV), w.to(DEV), torch.full((M, N), float("nan"), dtype=torch.bfloat16,
+                                                               device=DEV),
+                              dep=(t - 1) if deps else -1,
+                              yf32=torch.full((M, N), float("nan"), dtype=torch.float32, device=DEV)))
+    ch = wsm.Chain(tasks, path=wsm.PATH_UMMA)
+    for _ in range(2):
+        ch.run()
+        assert ch.status()[0] == wsm.WSM_OK, wsm.last_error()
+        for t in tasks:
+            check_full(t.x.cpu(), t.w.cpu(), t.y, t.yf32)
+    ch.close()
+
+
 def test_independent_tasks_no_deps():
     tasks = []
     for t in range(5):

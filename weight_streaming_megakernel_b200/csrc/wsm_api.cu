@@ -751,7 +751,13 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     wsm_opts to{};
     to.path = path;
     to.grid = opts->grid;
-    to.stage_k = (path == WSM_PATH_UMMA) ? opts->stage_k : 0;
+    // one stage geometry for the whole chain (the ring and the kernel's boxes per stage are shared):
+    // on the UMMA path, auto stage_k follows the chain's widest X tile
+    to.stage_k = 0;
+    if (path == WSM_PATH_UMMA) {
+        to.stage_k = opts->stage_k;
+        if (to.stage_k == 0) to.stage_k = ((maxM + 15) / 16 * 16 <= 32) ? 256 : 128;
+    }
     const int chain_mmax = (path == WSM_PATH_STREAM) ? pow2ceil(maxM) : 0;
     for (int i = 0; i < n; ++i) {
         if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, d->sms, &to, geos[i], chain_mmax)) != WSM_OK)
@@ -771,6 +777,9 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         ring.stage_bytes = ring.x_off + ring.kps * ring.x_stride;
     }
     ring.stages = std::min(kMaxStages, kRingBudget / ring.stage_bytes);
+    for (int i = 0; i < n; ++i)
+        if (geos[i].kps != ring.kps || geos[i].tile_k != ring.tile_k)
+            return fail(WSM_ERR_INVALID, "task %d: stage geometry differs from the chain's", i);  // cannot happen
     ch->geo = ring;
     ch->prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, path);
 
