@@ -456,6 +456,8 @@ def main():
     cases = workload_cases(args.workload)
     if args.only:
         cases = [c for c in cases if c.name in args.only.split(",")]
+        if not cases:
+            raise SystemExit(f"--only {args.only}: no case of workload {args.workload} has these names")
     config = {"workload": {"qwen3_decode": "qwen3_8b_decode_gemms", "single": "single_gemm_m1_4096x4096",
                            "skinny": "skinny_k7168_k8192", "l2_reuse": "l2_reuse_m32_m64",
                            "chain": "chain_36x4_m16"}[args.workload],
