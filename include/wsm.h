@@ -59,8 +59,8 @@ typedef enum {
     WSM_ERR_TIMEOUT = 6      /* a bounded device-side wait ran out (chain dependency or pipeline) */
 } wsm_status;
 
-/* Kernel path.  AUTO takes the FMA path for M = 1 up to 512 MiB of weights,
- * M = 2 up to 180 MiB and M <= 4 up to 64 MiB (measured crossovers on B200),
+/* Kernel path.  AUTO takes the FMA path for M = 1 up to 180 MiB of weights,
+ * M = 2 up to 96 MiB and M <= 4 up to 64 MiB (measured crossovers on B200),
  * the tensor-core path otherwise. */
 enum {
     WSM_PATH_AUTO = 0,

@@ -68,17 +68,20 @@ def test_plan_paths_and_geometry():
 
 
 def test_auto_path_crossovers():
-    """AUTO: FMA path for M = 1 up to 512 MiB of weights, M = 2 up to 180 MiB,
+    """AUTO: FMA path for M = 1 up to 180 MiB of weights, M = 2 up to 96 MiB,
     M <= 4 up to 64 MiB; tensor cores otherwise."""
     S, U = wsm.PATH_STREAM, wsm.PATH_UMMA
-    cases = [(1, 4096, 4096, S), (1, 24576, 4096, S), (1, 57344, 8192, U), (2, 4096, 12288, S),
-             (2, 10240, 8192, S), (2, 24576, 4096, U), (4, 4096, 4096, S), (4, 4096, 7168, S),
-             (4, 4096, 12288, U), (3, 6144, 4096, S), (5, 64, 64, U), (8, 4096, 4096, U), (16, 64, 64, U)]
+    cases = [(1, 4096, 4096, S), (1, 10240, 8192, S), (1, 24576, 4096, U), (1, 57344, 8192, U),
+             (2, 4096, 12288, S), (2, 10240, 8192, U), (2, 24576, 4096, U), (4, 4096, 4096, S),
+             (4, 4096, 7168, S), (4, 4096, 12288, U), (3, 6144, 4096, S), (5, 64, 64, U), (8, 4096, 4096, U),
+             (16, 64, 64, U)]
     for M, N, K, want in cases:
         assert wsm.plan(M, N, K)["path"] == want, (M, N, K)
     # exactly at the thresholds
-    assert wsm.plan(1, 32768, 8192)["path"] == S          # 512 MiB
-    assert wsm.plan(1, 32769, 8192)["path"] == U
+    assert wsm.plan(1, 11520, 8192)["path"] == S          # 180 MiB
+    assert wsm.plan(1, 11521, 8192)["path"] == U
+    assert wsm.plan(2, 6144, 8192)["path"] == S           # 96 MiB
+    assert wsm.plan(2, 6145, 8192)["path"] == U
     assert wsm.plan(4, 4096, 8192)["path"] == S           # 64 MiB
     assert wsm.plan(4, 4097, 8192)["path"] == U
 

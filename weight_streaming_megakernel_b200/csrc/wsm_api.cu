@@ -148,14 +148,15 @@ wsm_status plan_units(Geo &g, int ctas, int unit_stages, int tail_tiles, int tai
 
 // Automatic path choice.  Measured on B200 (graph-replayed back-to-back
 // launches of decode shapes, M = 1..8, weights 30 MB .. 940 MB): the FMA path
-// wins while its arithmetic per weight byte stays light -- M = 1 up to about
-// 0.5 GB of weights, M = 2 up to about 180 MB, M <= 4 up to about 64 MB --
-// and the tensor-core path wins everywhere else (at M >= 5 always).
+// wins while its arithmetic per weight byte stays light and the weights are
+// small enough for its shorter ramp to matter -- M = 1 up to about 180 MiB of
+// weights, M = 2 up to about 96 MiB, M <= 4 up to about 64 MiB -- and the
+// tensor-core path wins everywhere else (at M >= 5 always).
 int auto_path(int M, long long w_bytes) {
-    const long long MB = 1ll << 20;
-    if (M == 1 && w_bytes <= 512 * MB) return WSM_PATH_STREAM;
-    if (M == 2 && w_bytes <= 180 * MB) return WSM_PATH_STREAM;
-    if (M <= 4 && w_bytes <= 64 * MB) return WSM_PATH_STREAM;
+    const long long MiB = 1ll << 20;
+    if (M == 1 && w_bytes <= 180 * MiB) return WSM_PATH_STREAM;
+    if (M == 2 && w_bytes <= 96 * MiB) return WSM_PATH_STREAM;
+    if (M <= 4 && w_bytes <= 64 * MiB) return WSM_PATH_STREAM;
     return WSM_PATH_UMMA;
 }
 
