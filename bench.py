@@ -19,6 +19,7 @@ has) on a bounded sample of the same workload, on rank 0 only.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import subprocess
@@ -391,6 +392,63 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
                 plain_ms=plain_ms, copies=copies)
 
 
+def run_nshard(args, rank, world, local_rank):
+    """Column-parallel step (--parallel nshard): every rank streams its block
+    of output columns of every weight (one chain kernel over the blocks), then
+    one all-gather per GEMM assembles the full Y on every rank.  Timed eagerly
+    (the collectives are not captured in a graph): K steps between a barrier
+    and a synchronize, max over ranks."""
+    import weight_streaming_megakernel_b200 as wsm
+    from weight_streaming_megakernel_b200.shard import column_shards, gather_columns, max_over_ranks
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cases = workload_cases(args.workload)
+    if args.only:
+        cases = [c for c in cases if c.name in args.only.split(",")]
+    full_bytes = sum(alg_bytes(c) for c in cases)
+    shards = [column_shards(c.N, world, 128) for c in cases]
+    local = []
+    for c, sh in zip(cases, shards):
+        n0, n1 = sh[rank]
+        local.append(synth.Case(c.name, c.M, max(n1 - n0, 1), c.K, c.seed, c.m_tile))
+    data = setup_inputs(local, dev, seed_base=rank)
+    deps = [(i - 1) if args.workload == "chain" else -1 for i in range(len(data))]
+    chain = wsm.Chain([wsm.Task(x, w, y, dep=deps[i]) for i, (c, x, w, y) in enumerate(data)],
+                      flags=wsm.FLAG_W_READONLY)
+    stream = torch.cuda.Stream(dev)
+
+    def step():
+        chain.run(stream.cuda_stream)
+        if world > 1:
+            for (c, x, w, y), sh in zip(data, shards):
+                gather_columns(y[:, : sh[rank][1] - sh[rank][0]], sh)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+    stream.synchronize()
+    total_ms = a.elapsed_time(b)
+    if world > 1:
+        torch.distributed.barrier()
+        total_ms = max_over_ranks(total_ms, device=dev)
+    if chain.status(stream.cuda_stream)[0] != 0:
+        raise RuntimeError("device-side status")
+    chain.close()
+    return full_bytes, total_ms / args.steps
+
+
 # ----------------------------------------------------------------------------- CPU arm
 
 def oracle_sample_rate(cases, budget_s, threads=0):
@@ -445,6 +503,9 @@ def main():
     ap.add_argument("--mode", default="chain", choices=["chain", "launches"],
                     help="chain: the step is one persistent gemm_chain kernel; launches: one skinny_gemm per GEMM")
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-GEMM single-launch breakdown")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "nshard"],
+                    help="N > 1: independent replicas (weak scaling) or column blocks of every weight per rank "
+                         "with an all-gather of each Y (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -499,7 +560,21 @@ def main():
         return
 
     if world > 1:
-        torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local_rank))
+        torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local_rank),
+                                             timeout=datetime.timedelta(seconds=120))
+    if args.parallel == "nshard":
+        full_bytes, ms = run_nshard(args, rank, world, local_rank)
+        if rank == 0:
+            config["parallelism"] = f"nshard{world}"
+            print(json.dumps({"metric": METRIC, "value": round(full_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "strong",
+                              "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+                              "frac_of_peak": round(full_bytes / (ms * 1e-3) / 1e9 / world / hbm_peak, 4),
+                              "gpu_launches": args.steps, "roofline": None, "cpu_baseline": None, "e2e": None}))
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     r = run_gpu(args, rank, world, local_rank)
     breakdown = None
     if args.mode == "chain" and not args.no_breakdown and args.workload != "chain":
