@@ -263,6 +263,16 @@ typedef struct {
     int tail_unit_stages;      /* as in wsm_opts, for every task */
     int l2_prefetch_stages;    /* W stages per CTA prefetched into L2 while the CTA waits for
                                   a dependency or the previous kernel: 0 = auto, -1 = none */
+    int counter_groups;        /* 0 or 1: one readiness counter per task, bumped by every
+                                  finished tile.  G >= 2: two-level readiness ("Fleet ..."
+                                  reading notes, section 3d and the two-level event
+                                  synchronisation flowchart): CTA c belongs to group c % G,
+                                  each task's tiles are split into G contiguous ranges, one
+                                  per group, a group claims only its own range, a finished
+                                  tile bumps its group's counter and the group's last tile
+                                  bumps the task's counter once.  An ablation: the pages use
+                                  it to save cross-die fences, which B200's coherent L2 does
+                                  not need.  Not with dep_cols tasks (WSM_ERR_UNSUPPORTED). */
 } wsm_chain_opts;
 
 typedef struct wsm_chain wsm_chain;  /* opaque prepared chain */

@@ -84,6 +84,49 @@ def test_dependent_chain_tail_units(path, M):
     ch.close()
 
 
+@pytest.mark.parametrize("path,M,groups", [(wsm.PATH_UMMA, 16, 2), (wsm.PATH_UMMA, 16, 7), (wsm.PATH_UMMA, 48, 3),
+                                           (wsm.PATH_STREAM, 2, 2), (wsm.PATH_STREAM, 8, 5)])
+def test_two_level_readiness(path, M, groups):
+    """Two-level readiness counters (group counters, then one global bump per
+    group): a data-dependent chain still orders every task after its
+    dependency, over repeated runs and CUDA-graph replays."""
+    dims = [1024, 2048, 1024, 3072, 512, 4096, 1024]
+    x0, ws, ys, yfs, tasks = dependent_chain(M, dims, seed=50 + groups)
+    ch = wsm.Chain(tasks, path=path, counter_groups=groups, flags=wsm.FLAG_W_READONLY)
+    for _ in range(2):
+        for y in ys:
+            y.fill_(float("nan"))
+        ch.run()
+        assert ch.status()[0] == wsm.WSM_OK, wsm.last_error()
+        check_dependent(x0, ws, ys, yfs)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    ch.run(s)
+    s.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        ch.run(s)
+    for _ in range(2):
+        for y in ys:
+            y.fill_(float("nan"))
+        g.replay()
+        s.synchronize()
+        assert ch.status(s)[0] == wsm.WSM_OK
+        check_dependent(x0, ws, ys, yfs)
+    del g
+    ch.close()
+
+
+def test_two_level_rejects_column_dependencies():
+    x = torch.zeros(4, 64, dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros(64, 64, dtype=torch.bfloat16, device=DEV)
+    y0 = torch.empty(4, 64, dtype=torch.bfloat16, device=DEV)
+    y1 = torch.empty(4, 64, dtype=torch.bfloat16, device=DEV)
+    tasks = [wsm.Task(x, w, y0), wsm.Task(y0, w, y1, dep=0, dep_cols=True)]
+    with pytest.raises(wsm.WsmError) as e:
+        wsm.Chain(tasks, counter_groups=2)
+    assert e.value.code == wsm.WSM_ERR_UNSUPPORTED
+
+
 def test_dependent_chain_small_grid_and_empty_ctas():
     """A grid larger than some tasks' stage counts (CTAs with no work for a
     task) and a tiny grid (long per-CTA ranges)."""

@@ -80,7 +80,8 @@ class _ChainOpts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("grid", ctypes.c_int), ("timeout_ns", ctypes.c_ulonglong),
                 ("trace", ctypes.c_int), ("debug_unmet_dependency", ctypes.c_int), ("flags", ctypes.c_int),
                 ("stage_k", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
-                ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int)]
+                ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int),
+                ("counter_groups", ctypes.c_int)]
 
 
 _lib = None
@@ -306,7 +307,7 @@ class Chain:
 
     def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
                  debug_unmet_dependency=False, flags=0, stage_k=0, unit_stages=0, tail_tiles=0,
-                 tail_unit_stages=0, l2_prefetch_stages=0):
+                 tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0):
         for i, t in enumerate(tasks):
             _check_operand(f"tasks[{i}].x", t.x)
             _check_operand(f"tasks[{i}].w", t.w)
@@ -319,6 +320,7 @@ class Chain:
         o.flags, o.stage_k = flags, stage_k
         o.unit_stages, o.tail_tiles, o.tail_unit_stages = unit_stages, tail_tiles, tail_unit_stages
         o.l2_prefetch_stages = l2_prefetch_stages
+        o.counter_groups = counter_groups
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

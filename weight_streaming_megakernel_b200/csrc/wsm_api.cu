@@ -746,6 +746,12 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     ch->pdl = pdl_mode(opts->flags);
     if (opts->l2_prefetch_stages < -1)
         return fail(WSM_ERR_INVALID, "bad l2_prefetch_stages %d", opts->l2_prefetch_stages);
+    if (opts->counter_groups < 0) return fail(WSM_ERR_INVALID, "bad counter_groups %d", opts->counter_groups);
+    const int groups = opts->counter_groups > 1 ? opts->counter_groups : 1;
+    if (groups > 1)
+        for (int i = 0; i < n; ++i)
+            if (tasks[i].dep_cols)
+                return fail(WSM_ERR_UNSUPPORTED, "task %d: two-level readiness does not combine with dep_cols", i);
 
     // per-task geometry; the ring is sized for the widest task
     std::vector<Geo> geos(n);
@@ -787,8 +793,9 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     // work units per task, planned for the chain's grid (K-range-first units, no tail, for a task that
     // waits per column)
     for (int i = 0; i < n; ++i)
-        if ((st = plan_units(geos[i], chain_grid, opts->unit_stages, tasks[i].dep_cols ? -1 : opts->tail_tiles,
-                             opts->tail_unit_stages)) != WSM_OK)
+        if ((st = plan_units(geos[i], chain_grid, opts->unit_stages,
+                             (tasks[i].dep_cols || groups > 1) ? -1 : opts->tail_tiles, opts->tail_unit_stages)) !=
+            WSM_OK)
             return fail(st, "task %d: %s", i, g_err.c_str());
     // per-column readiness: a task some other task reads per column publishes one counter per
     // kColChunk output columns; col_need[c] = tiles (all M-tiles) whose outputs touch chunk c
@@ -813,10 +820,13 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     // scratch: status | counters (per task: claim counters + tile counters; then done counters; then
     // column counters) | partials | column needs (constant)
     std::vector<size_t> cnt_off(n), part_off(n), col_off(n), need_off(n);
+    std::vector<int> n_groups(n, 1);
     size_t ncnt = 0;
     for (int i = 0; i < n; ++i) {
+        // every group needs at least one tile and one CTA
+        n_groups[i] = (int)std::min<long long>(groups, std::min<long long>(geos[i].tiles(), chain_grid));
         cnt_off[i] = ncnt;
-        ncnt += kSchedWords + (size_t)geos[i].tiles();
+        ncnt += kSchedWords + (size_t)geos[i].tiles() + (n_groups[i] > 1 ? 2 * (size_t)n_groups[i] : 0);
     }
     const size_t done_off = ncnt;
     ncnt += n;
@@ -882,6 +892,11 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         T.dep = tasks[i].dep;
         T.sched = ch->d_counters + cnt_off[i];
         T.tile_cnt = T.sched + kSchedWords;
+        T.n_groups = n_groups[i];
+        if (n_groups[i] > 1) {
+            T.grp_sched = T.tile_cnt + gi.tiles();
+            T.grp_done = T.grp_sched + n_groups[i];
+        }
         T.done = ch->d_counters + done_off + i;
         T.notify = depended[i];
         T.part = reinterpret_cast<float *>(base + part_off[i]);

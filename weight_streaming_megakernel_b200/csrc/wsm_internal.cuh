@@ -94,6 +94,12 @@ struct __align__(64) TaskDev {
     const unsigned int *col_need;      // tiles that touch each chunk, per run
     const unsigned int *dep_col_cnt;   // per-column dependency: the dep task's col_cnt, else nullptr
     const unsigned int *dep_col_need;  // ... and its col_need
+    // Two-level readiness (n_groups > 1): CTA c belongs to group c % n_groups, group g owns the
+    // contiguous tiles [g T / G, (g+1) T / G) and claims their units from grp_sched[g]; a finished tile
+    // bumps grp_done[g] and the group's last tile bumps `done` once: done counts groups, not tiles.
+    int n_groups;
+    unsigned int *grp_sched;    // [n_groups] claim counters, zero between runs
+    unsigned int *grp_done;     // [n_groups] finished tiles per group (monotonic over runs)
     int w_evict_first;          // L2 policy of the weight loads
     uint32_t idesc;             // UMMA instruction descriptor (MMA N = t_mpad)
     uint32_t tx_bytes;          // bytes landing in one stage
@@ -383,11 +389,36 @@ __device__ __forceinline__ UnitSpan unit_span(const TaskDev &T, int u) {
     return r;
 }
 
-// Claim the next dynamic unit of task T: the caller adds the number of units
-// handed out statically (unit c to CTA c); a result >= n_units means none left.
-__device__ __forceinline__ int claim_unit(const TaskDev &T) {
-    return (int)atom_add_relaxed_gpu(&T.sched[0], 1u);
+// The units a CTA claims from: all of the task's, or with two-level readiness
+// its group's tiles (tile-major units, so a contiguous range).
+struct ClaimRange {
+    unsigned int *ctr;
+    int lo, hi;
+};
+__device__ __forceinline__ int group_tile_lo(const TaskDev &T, int g) {
+    return (int)((long long)g * (T.n_g * T.n_mt) / T.n_groups);
 }
+__device__ __forceinline__ int group_of_tile(const TaskDev &T, int tile) {
+    return (int)(((long long)(tile + 1) * T.n_groups - 1) / (T.n_g * T.n_mt));
+}
+__device__ __forceinline__ ClaimRange claim_range(const TaskDev &T) {
+    ClaimRange r;
+    if (T.n_groups <= 1) {
+        r.ctr = &T.sched[0];
+        r.lo = 0;
+        r.hi = T.n_units;
+    } else {
+        const int g = (int)blockIdx.x % T.n_groups;
+        r.ctr = &T.grp_sched[g];
+        r.lo = group_tile_lo(T, g) * T.nu;
+        r.hi = group_tile_lo(T, g + 1) * T.nu;
+    }
+    return r;
+}
+
+// Claim the next dynamic unit: the caller adds cr.lo and the number of units
+// handed out statically (unit c to CTA c); a result >= cr.hi means none left.
+__device__ __forceinline__ int claim_unit(const ClaimRange &cr) { return (int)atom_add_relaxed_gpu(cr.ctr, 1u); }
 
 // Single GEMM: called once per CTA when it has stopped claiming units; the
 // last CTA resets the claim counters for the next call (no CTA claims any
@@ -461,7 +492,10 @@ struct UnitOut {
     unsigned int *tile_cnt;
     unsigned int *done;     // nullptr unless some task waits for this whole task
     unsigned int *col_cnt;  // nullptr unless some task waits for its columns
+    unsigned int *grp_done; // two-level readiness, else nullptr
     int slot_elems, t_mpad;
+    int grp_tiles;          // two-level: tiles of the unit's group
+    int grp;                // ... and the group
 };
 __device__ __forceinline__ UnitOut unit_out(const TaskDev &T) {
     UnitOut o;
@@ -472,7 +506,16 @@ __device__ __forceinline__ UnitOut unit_out(const TaskDev &T) {
     o.col_cnt = T.col_cnt;
     o.slot_elems = T.slot_elems;
     o.t_mpad = T.t_mpad;
+    o.grp_done = (T.notify && T.n_groups > 1) ? T.grp_done : nullptr;
+    o.grp = 0;
+    o.grp_tiles = 0;
     return o;
+}
+// Two-level readiness: the group of the unit's tile (call before the first store).
+__device__ __forceinline__ void unit_out_group(UnitOut &o, const TaskDev &T, int tile) {
+    if (!o.grp_done) return;
+    o.grp = group_of_tile(T, tile);
+    o.grp_tiles = group_tile_lo(T, o.grp + 1) - group_tile_lo(T, o.grp);
 }
 
 // A finished tile (column tile g, rows_per_tile rows of W) counts toward every
@@ -490,8 +533,15 @@ __device__ __forceinline__ void notify_columns(const UnitOut &o, int g, int rows
 
 // The tile is complete: whole-task and per-column readiness (leader thread,
 // after the barrier that follows the tile's last stores).
-__device__ __forceinline__ void tile_finished(const UnitOut &o, int g, int rows_per_tile) {
-    if (o.done) red_release_gpu_add(o.done, 1u);
+__device__ __forceinline__ void tile_finished(const UnitOut &o, int g, int rows_per_tile, unsigned int run) {
+    if (o.grp_done) {
+        // first level: the group's count of finished tiles (acq_rel: the group's last tile sees every
+        // earlier tile's stores and its release to `done` covers them); second level: once per group
+        const unsigned int old = atom_add_acqrel_gpu(&o.grp_done[o.grp], 1u);
+        if (old + 1u == run * (unsigned int)o.grp_tiles) red_release_gpu_add(o.done, 1u);
+    } else if (o.done) {
+        red_release_gpu_add(o.done, 1u);
+    }
     if (o.col_cnt) notify_columns(o, g, rows_per_tile);
 }
 
@@ -524,13 +574,13 @@ static __device__ __noinline__ void wait_chunks(const KParams &p, const TaskDev 
 
 __device__ __forceinline__ bool dependency_met(const KParams &p, const TaskDev &D) {
     const unsigned int run = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
-    const unsigned int target = run * (unsigned int)(D.n_g * D.n_mt) + p.dep_target_extra;
+    const unsigned int target = run * (unsigned int)(D.n_groups > 1 ? D.n_groups : D.n_g * D.n_mt) + p.dep_target_extra;
     return ld_acquire_gpu(D.done) - target < 0x80000000u;  // done >= target (wrap-safe)
 }
 
 static __device__ __noinline__ void wait_dependency(const KParams &p, const TaskDev &D, int task, int *status) {
     const unsigned int run = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
-    const unsigned int target = run * (unsigned int)(D.n_g * D.n_mt) + p.dep_target_extra;
+    const unsigned int target = run * (unsigned int)(D.n_groups > 1 ? D.n_groups : D.n_g * D.n_mt) + p.dep_target_extra;
     if (ld_acquire_gpu(D.done) - target < 0x80000000u) {  // done >= target (wrap-safe)
         fence_proxy_async_global();
         return;
@@ -557,7 +607,12 @@ __device__ __forceinline__ void chain_run_done(const KParams &p) {
     if (!p.run_ctl) return;
     const unsigned int old = atom_add_acqrel_gpu(&p.run_ctl[1], 1u);
     if (old == gridDim.x - 1) {
-        for (int t = 0; t < p.n_tasks; ++t) st_relaxed_gpu(&task_at(p, t).sched[0], 0u);
+        for (int t = 0; t < p.n_tasks; ++t) {
+            const TaskDev &T = task_at(p, t);
+            st_relaxed_gpu(&T.sched[0], 0u);
+            if (T.n_groups > 1)
+                for (int g = 0; g < T.n_groups; ++g) st_relaxed_gpu(&T.grp_sched[g], 0u);
+        }
         st_relaxed_gpu(&p.run_ctl[1], 0u);
         red_release_gpu_add(&p.run_ctl[0], 1u);
     }

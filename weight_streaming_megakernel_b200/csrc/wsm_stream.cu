@@ -259,9 +259,12 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 // The kernel's first task hands unit c to CTA c (no atomic, and it can stream before the
                 // grid dependency); later tasks hand out every unit by claim, so the CTAs that finish the
                 // previous task first take the next task's work.
-                const int n_static = (t == 0) ? min((int)gridDim.x, T.n_units) : 0;
+                // (with two-level readiness a CTA works only on its group's tiles, all claimed)
+                const ClaimRange cr = claim_range(T);
+                const bool static_first = t == 0 && T.n_groups <= 1;
+                const int n_static = static_first ? min((int)gridDim.x, T.n_units) : 0;
                 int u;
-                if (t == 0) {
+                if (static_first) {
                     u = (int)blockIdx.x < T.n_units ? (int)blockIdx.x : T.n_units;
                 } else {
                     if (!grid_dep_ok) {
@@ -269,9 +272,9 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                         grid_dep_ok = true;
                         dep_ok = T.dep < 0;
                     }
-                    u = claim_unit(T);
+                    u = cr.lo + claim_unit(cr);
                 }
-                while (u < T.n_units) {
+                while (u < cr.hi) {
                     if (first_unit) {
                         trace_stamp(p, t, 0, globaltimer());
                         trace_stamp(p, t, 3, smid());
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     const int g = us.tile;
                     const int k_begin = us.k_begin;
                     const int k_end = us.k_end;
-                    int next_u = T.n_units - n_static;
+                    int next_u = cr.hi - cr.lo - n_static;
                     bool claimed = false;
                     for (int kk = k_begin; kk < k_end; ++kk) {
                         if (!take_slot()) break;
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                         // hold a second unit it cannot start (the claim counters belong to the previous
                         // kernel until the grid dependency is resolved)
                         if (!claimed && dep_ok && k_end - kk <= kClaimLead) {
-                            next_u = claim_unit(T);
+                            next_u = claim_unit(cr);
                             claimed = true;
                         }
                     }
@@ -325,12 +328,12 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     if (!claimed) {
                         // the unit streamed completely before its dependencies were resolved
                         if (!dep_ok) flush();
-                        next_u = claim_unit(T);
+                        next_u = claim_unit(cr);
                     }
                     // whatever comes next needs a free slot: wait for it before the claim's result is used,
                     // so the claim's round trip overlaps the wait
                     if (!take_slot()) break;
-                    u = next_u + n_static;
+                    u = cr.lo + next_u + n_static;
                 }
                 if (np > 0) flush();
                 if (aborted) break;
@@ -362,6 +365,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
         const int o_row = ctid - o_m * TN;
         const bool owner = ctid < TN * MMAX;
         if (p.pdl) pdl_wait();  // Y and the scratch may still be in use by the previous kernel
+        const unsigned int run_no = p.run_ctl ? ld_acquire_gpu(&p.run_ctl[0]) + 1u : 0u;  // this chain run
         int s = 0;
         uint32_t ph = 0;
         uint32_t unit_i = 0;
@@ -468,12 +472,13 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
             const int g = us.tile;
             const int n = g * TN + o_row;
             const bool live = owner && o_m < M && n < T.N;
-            const UnitOut uo = unit_out(T);  // no task-table reads after the first store below
+            UnitOut uo = unit_out(T);  // no task-table reads after the first store below
+            unit_out_group(uo, T, g);
             if (us.nu == 1) {
                 emit_one(uo.e, n, o_m, live, val);
                 if (uo.done || uo.col_cnt) {
                     named_bar_sync(kConsBar, NCT);
-                    if (leader) tile_finished(uo, g, TN);  // release covers the CTA's stores (bar.sync before)
+                    if (leader) tile_finished(uo, g, TN, run_no);  // release covers the CTA's stores (bar.sync before)
                 }
             } else {
                 if (owner) uo.part[(size_t)u * uo.slot_elems + ctid] = val;
@@ -495,7 +500,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     named_bar_sync(kConsBar, NCT);
                     if (leader) {
                         uo.tile_cnt[g] = 0u;
-                        tile_finished(uo, g, TN);
+                        tile_finished(uo, g, TN, run_no);
                     }
                 }
             }

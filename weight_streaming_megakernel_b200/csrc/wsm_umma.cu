@@ -355,9 +355,12 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 // The kernel's first task hands unit c to CTA c (no atomic, and it can stream before the
                 // grid dependency); later tasks hand out every unit by claim, so the CTAs that finish the
                 // previous task first take the next task's work.
-                const int n_static = (t == 0) ? min((int)gridDim.x, T.n_units) : 0;
+                // (with two-level readiness a CTA works only on its group's tiles, all claimed)
+                const ClaimRange cr = claim_range(T);
+                const bool static_first = t == 0 && T.n_groups <= 1;
+                const int n_static = static_first ? min((int)gridDim.x, T.n_units) : 0;
                 int u;
-                if (t == 0) {
+                if (static_first) {
                     u = (int)blockIdx.x < T.n_units ? (int)blockIdx.x : T.n_units;
                 } else {
                     if (!grid_dep_ok) {
@@ -365,9 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         grid_dep_ok = true;
                         dep_ok = T.dep < 0;
                     }
-                    u = claim_unit(T);
+                    u = cr.lo + claim_unit(cr);
                 }
-                while (u < T.n_units) {
+                while (u < cr.hi) {
                     if (first_unit) {
                         trace_stamp(p, t, 0, globaltimer());
                         trace_stamp(p, t, 3, smid());
@@ -377,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     int g, mt;
                     tile_coords(T, us.tile, g, mt);
                     const int xy = mt * T.t_m;
-                    int next_u = T.n_units - n_static;
+                    int next_u = cr.hi - cr.lo - n_static;
                     bool claimed = false;
                     for (int kk = us.k_begin; kk < us.k_end; ++kk) {
                         if (!take_slot()) break;
@@ -412,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         // hold a second unit it cannot start (the claim counters belong to the previous
                         // kernel until the grid dependency is resolved)
                         if (!claimed && dep_ok && us.k_end - kk <= kClaimLead) {
-                            next_u = claim_unit(T);
+                            next_u = claim_unit(cr);
                             claimed = true;
                         }
                     }
@@ -420,12 +423,12 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     if (!claimed) {
                         // the unit streamed completely before its dependencies were resolved
                         if (!dep_ok) flush();
-                        next_u = claim_unit(T);
+                        next_u = claim_unit(cr);
                     }
                     // whatever comes next needs a free slot: wait for it before the claim's result is used,
                     // so the claim's round trip overlaps the wait
                     if (!take_slot()) break;
-                    u = next_u + n_static;
+                    u = cr.lo + next_u + n_static;
                 }
                 if (np > 0) flush();
                 if (aborted) break;
@@ -526,6 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         const int etid = threadIdx.x - (kEpiWarp0 + 4 * set) * 32;
         const bool leader = (etid == 0);
         if (p.pdl) pdl_wait();                  // Y and the scratch may still be in use by the previous kernel
+        const unsigned int run_no = p.run_ctl ? ld_acquire_gpu(&p.run_ctl[0]) + 1u : 0u;  // this chain run
         for (uint32_t k = 0;; ++k) {
             const uint32_t acc_i = kEpiSets * k + (uint32_t)set;
             const int buf = (int)(acc_i % kAccBufs);
@@ -544,7 +548,8 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             const int n = g * kUmmaRows + row;
             const int m0 = mt * T.t_m;
             const int mrows = min(T.t_m, T.M - m0);
-            const UnitOut uo = unit_out(T);  // no task-table reads after the first store below
+            UnitOut uo = unit_out(T);  // no task-table reads after the first store below
+            unit_out_group(uo, T, tile);
             // The accumulator, 16 columns (X rows) at a time: TMEM -> registers -> outputs (whole tile) or
             // this unit's partial row [row][m] (split tile).  The loop is not unrolled: one copy of the
             // epilogue code per kind keeps the kernel small.
@@ -574,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             if (us.nu == 1) {
                 if (uo.done || uo.col_cnt) {
                     epi_bar(set);
-                    if (leader) tile_finished(uo, g, kUmmaRows);  // release covers the set's stores (bar.sync before)
+                    if (leader) tile_finished(uo, g, kUmmaRows, run_no);  // release covers the set's stores (bar.sync before)
                 }
             } else {
                 // the last unit of the tile to arrive adds all the partials
@@ -595,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     epi_bar(set);
                     if (leader) {
                         uo.tile_cnt[tile] = 0u;  // ready for the next call
-                        tile_finished(uo, g, kUmmaRows);
+                        tile_finished(uo, g, kUmmaRows, run_no);
                     }
                 }
             }
