@@ -59,7 +59,7 @@ typedef enum {
     WSM_ERR_TIMEOUT = 6      /* a bounded device-side wait ran out (chain dependency or pipeline) */
 } wsm_status;
 
-/* Kernel path.  AUTO takes the FMA path for M = 1 up to 180 MiB of weights,
+/* Kernel path.  AUTO takes the FMA path for M = 1 up to 128 MiB of weights,
  * M = 2 up to 96 MiB and M <= 4 up to 64 MiB (measured crossovers on B200),
  * the tensor-core path otherwise. */
 enum {
@@ -213,8 +213,9 @@ wsm_status wsm_stream_status(wsm_stream_t stream, int *code);
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.
  *  - Shapes whose plan needs more scratch than the array holds return
- *    WSM_ERR_UNSUPPORTED with a message naming both sizes (the tensor-core
- *    plans of M >= 48 on wide N are the ones that do not fit).
+ *    WSM_ERR_UNSUPPORTED with a message naming both sizes (split-K
+ *    tensor-core plans with M > 16 on the widest N, e.g. 24..64 x 57344 x
+ *    8192, are the ones that do not fit).
  *  - Every call shares the array.  Each call clears the part that must start
  *    at zero (queued on `stream`), but calls that overlap on the GPU -- on
  *    different streams, or on different host threads -- race on it; queue
@@ -273,7 +274,22 @@ typedef struct {
                                   bumps the task's counter once.  An ablation: the pages use
                                   it to save cross-die fences, which B200's coherent L2 does
                                   not need.  Not with dep_cols tasks (WSM_ERR_UNSUPPORTED). */
+    int kernels;               /* WSM_CHAIN_KERNELS_*: hybrid dispatch.  One kernel sizes its
+                                  pipeline stages for the chain's widest X tile, which costs
+                                  tasks of M <= 32 about 5 % when M > 32 tasks share the chain;
+                                  SPLIT runs such a tensor-core chain as one kernel per run of
+                                  consecutive tasks of one kind, back to back on the stream (a
+                                  dependency on an earlier kernel is met by stream order;
+                                  wsm_chain_trace is then not available), at about 20 us per
+                                  extra kernel boundary.  AUTO splits when the narrow tasks'
+                                  weights exceed 1.5 GB per extra boundary. */
 } wsm_chain_opts;
+
+enum {
+    WSM_CHAIN_KERNELS_AUTO = 0,
+    WSM_CHAIN_KERNELS_ONE = 1,
+    WSM_CHAIN_KERNELS_SPLIT = 2
+};
 
 typedef struct wsm_chain wsm_chain;  /* opaque prepared chain */
 

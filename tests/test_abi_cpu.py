@@ -60,7 +60,7 @@ def test_plan_paths_and_geometry():
     p = wsm.plan(16, 4096, 4096, num_sms=148, stage_k=64)
     assert p["tile_k"] == 64 and p["k_iters"] == 64
     p = wsm.plan(48, 4096, 4096, num_sms=148)
-    assert p["tile_k"] == 128 and p["m_tile"] == 48
+    assert p["tile_k"] == 256 and p["m_tile"] == 48 and p["stages"] == 2
     p = wsm.plan(17, 100, 1000, num_sms=148)
     assert p["m_tile"] == 32 and p["n_tiles"] == 1 and p["k_iters"] == 4
     p = wsm.plan(8, 4096, 4096, num_sms=148, path=wsm.PATH_UMMA)
@@ -68,18 +68,18 @@ def test_plan_paths_and_geometry():
 
 
 def test_auto_path_crossovers():
-    """AUTO: FMA path for M = 1 up to 180 MiB of weights, M = 2 up to 96 MiB,
+    """AUTO: FMA path for M = 1 up to 128 MiB of weights, M = 2 up to 96 MiB,
     M <= 4 up to 64 MiB; tensor cores otherwise."""
     S, U = wsm.PATH_STREAM, wsm.PATH_UMMA
-    cases = [(1, 4096, 4096, S), (1, 10240, 8192, S), (1, 24576, 4096, U), (1, 57344, 8192, U),
+    cases = [(1, 4096, 4096, S), (1, 4096, 12288, S), (1, 10240, 8192, U), (1, 24576, 4096, U), (1, 57344, 8192, U),
              (2, 4096, 12288, S), (2, 10240, 8192, U), (2, 24576, 4096, U), (4, 4096, 4096, S),
              (4, 4096, 7168, S), (4, 4096, 12288, U), (3, 6144, 4096, S), (5, 64, 64, U), (8, 4096, 4096, U),
              (16, 64, 64, U)]
     for M, N, K, want in cases:
         assert wsm.plan(M, N, K)["path"] == want, (M, N, K)
     # exactly at the thresholds
-    assert wsm.plan(1, 11520, 8192)["path"] == S          # 180 MiB
-    assert wsm.plan(1, 11521, 8192)["path"] == U
+    assert wsm.plan(1, 8192, 8192)["path"] == S           # 128 MiB
+    assert wsm.plan(1, 8193, 8192)["path"] == U
     assert wsm.plan(2, 6144, 8192)["path"] == S           # 96 MiB
     assert wsm.plan(2, 6145, 8192)["path"] == U
     assert wsm.plan(4, 4096, 8192)["path"] == S           # 64 MiB
@@ -120,6 +120,23 @@ def test_plan_workspace_formula():
     partials = p["units"] * 128 * 16 * 4 if nu > 1 else 0
     assert p["workspace_bytes"] >= 256 + counters + partials
     assert p["workspace_bytes"] % 256 == 0
+
+
+def test_auto_units_per_tile():
+    """The automatic split of tiles into units on the tensor-core path (the
+    cost model fitted to measured B200 times): many-tile shapes split less,
+    few-tile shapes more, wider X tiles (larger partials) less."""
+    def nu(M, N, K):
+        p = wsm.plan(M, N, K, num_sms=148, path=wsm.PATH_UMMA)
+        return -(-p["k_iters"] // p["unit_stages"])
+    assert nu(16, 4096, 4096) == 4          # 32 tiles: 128 units, one round
+    assert nu(16, 4096, 12288) == 4
+    assert nu(16, 18432, 7168) == 1         # 144 tiles: one unit per CTA
+    assert nu(16, 10240, 8192) == 3         # 80 tiles: 240 units
+    assert nu(16, 57344, 8192) == 4         # 448 tiles: many rounds, small tail
+    assert nu(64, 24576, 4096) == 1         # 192 tiles at M = 64
+    assert nu(64, 57344, 8192) == 2
+    assert nu(16, 6144, 4096) == 3
 
 
 def test_plan_units():

@@ -209,10 +209,13 @@ def test_gemm_chain_one_shot():
 
 
 @pytest.mark.parametrize("deps", [False, True])
-def test_mixed_m_chain(deps):
-    """Tasks of different M in one chain share one stage geometry (the
-    widest X tile decides it): M = 1, 16, 33 and 64 mixed, with and without
-    ordering dependencies, on the tensor-core path."""
+@pytest.mark.parametrize("kernels", [wsm.CHAIN_KERNELS_SPLIT, wsm.CHAIN_KERNELS_ONE, wsm.CHAIN_KERNELS_AUTO])
+def test_mixed_m_chain(deps, kernels):
+    """Tasks of M = 1, 16, 33 and 64 in one chain on the tensor-core path,
+    with and without ordering dependencies: as one kernel sharing one stage
+    geometry (the widest X tile decides it), and with hybrid dispatch (one
+    kernel per run of tasks of one kind, dependencies across kernels met by
+    stream order)."""
     tasks = []
     for t, (M, N, K) in enumerate([(16, 1024, 4096), (64, 2048, 2048), (1, 640, 3072), (33, 1000, 1032),
                                    (64, 512, 8192), (16, 4096, 1024)]):
@@ -221,10 +224,41 @@ def test_mixed_m_chain(deps):
                                                                device=DEV),
                               dep=(t - 1) if deps else -1,
                               yf32=torch.full((M, N), float("nan"), dtype=torch.float32, device=DEV)))
-    ch = wsm.Chain(tasks, path=wsm.PATH_UMMA)
+    one = kernels != wsm.CHAIN_KERNELS_SPLIT   # AUTO keeps these small tasks in one kernel
+    ch = wsm.Chain(tasks, path=wsm.PATH_UMMA, kernels=kernels, trace=one)
     for _ in range(2):
+        for t in tasks:
+            t.y.fill_(float("nan"))
         ch.run()
         assert ch.status()[0] == wsm.WSM_OK, wsm.last_error()
+        for t in tasks:
+            check_full(t.x.cpu(), t.w.cpu(), t.y, t.yf32)
+    assert (ch.trace() is not None) == one   # split chains keep no trace
+    ch.close()
+
+
+def test_hybrid_chain_data_dependencies_across_kernels():
+    """Hybrid dispatch with data dependencies between its kernels: an M = 16
+    task writes the first 16 rows of the M = 64 task's input, whose output's
+    first 16 rows feed the next M = 16 task (three kernels; each dependency
+    is met by stream order).  Inputs are poisoned before every run."""
+    K = 512
+    B = synth.make_x(64, K, 81).to(DEV)          # rows 16..63 stay as drawn
+    x0 = synth.make_x(16, K, 82).to(DEV)
+    ws = [synth.make_w(K, K, 83 + t).to(DEV) for t in range(3)]
+    y1 = torch.empty(64, K, dtype=torch.bfloat16, device=DEV)
+    y2 = torch.empty(16, K, dtype=torch.bfloat16, device=DEV)
+    f = [torch.empty(16, K, device=DEV), torch.empty(64, K, device=DEV), torch.empty(16, K, device=DEV)]
+    tasks = [wsm.Task(x0, ws[0], B[0:16], yf32=f[0]),
+             wsm.Task(B, ws[1], y1, dep=0, yf32=f[1]),
+             wsm.Task(y1[0:16], ws[2], y2, dep=1, yf32=f[2])]
+    ch = wsm.Chain(tasks, path=wsm.PATH_UMMA, kernels=wsm.CHAIN_KERNELS_SPLIT)
+    for _ in range(2):
+        B[0:16].fill_(float("nan"))
+        y1.fill_(float("nan"))
+        y2.fill_(float("nan"))
+        ch.run()
+        assert ch.status()[0] == wsm.WSM_OK
         for t in tasks:
             check_full(t.x.cpu(), t.w.cpu(), t.y, t.yf32)
     ch.close()

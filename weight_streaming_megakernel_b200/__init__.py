@@ -36,6 +36,7 @@ ORDER_AUTO, ORDER_M_MAJOR, ORDER_NAIVE = 0, 1, 2
 L2_AUTO, L2_EVICT_FIRST, L2_NORMAL = 0, 1, 2
 FLAG_W_READONLY, FLAG_NO_PDL = 1, 2
 EPI_NONE, EPI_SILU_MUL, EPI_RESIDUAL = 0, 1, 2
+CHAIN_KERNELS_AUTO, CHAIN_KERNELS_ONE, CHAIN_KERNELS_SPLIT = 0, 1, 2
 
 # Every function include/wsm.h declares (checked by the CPU tests).
 HEADER_SYMBOLS = (
@@ -81,7 +82,7 @@ class _ChainOpts(ctypes.Structure):
                 ("trace", ctypes.c_int), ("debug_unmet_dependency", ctypes.c_int), ("flags", ctypes.c_int),
                 ("stage_k", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
                 ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int),
-                ("counter_groups", ctypes.c_int)]
+                ("counter_groups", ctypes.c_int), ("kernels", ctypes.c_int)]
 
 
 _lib = None
@@ -307,7 +308,7 @@ class Chain:
 
     def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
                  debug_unmet_dependency=False, flags=0, stage_k=0, unit_stages=0, tail_tiles=0,
-                 tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0):
+                 tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0, kernels=0):
         for i, t in enumerate(tasks):
             _check_operand(f"tasks[{i}].x", t.x)
             _check_operand(f"tasks[{i}].w", t.w)
@@ -321,6 +322,7 @@ class Chain:
         o.unit_stages, o.tail_tiles, o.tail_unit_stages = unit_stages, tail_tiles, tail_unit_stages
         o.l2_prefetch_stages = l2_prefetch_stages
         o.counter_groups = counter_groups
+        o.kernels = kernels
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

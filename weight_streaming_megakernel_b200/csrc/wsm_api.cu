@@ -8,6 +8,7 @@
 #include "../../include/wsm.h"
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -113,17 +114,40 @@ void stream_geo(int mmax, Geo &g) {
     g.threads = 32 * (1 + g.rg * g.kw);
 }
 
-// Work units: ku consecutive stages of one tile.  Measured on B200 (decode
-// shapes, M = 1 and 16): every unit costs a claim and, when its tile is split,
-// a partial store, a tile-counter round trip and a share of the in-order
-// reduction -- all latency-bound under a saturated memory system -- so the
-// best split is the coarsest one that still spreads a task over the SMs:
-// at most 4 units per tile on the tensor-core path (2 on the FMA path, whose
-// consumer warps run the epilogue themselves).
-//
+// Work units: ku consecutive stages of one tile, nu units per tile.  Every
+// unit costs a claim and, when its tile is split, a partial store, a tile
+// counter round trip and a share of the in-order reduction; and the last
+// units of a GEMM decide when it ends, with SMs that stream up to ~2x slower
+// than others.  Tensor-core path: nu in 1..4 minimising a cost in stages,
+// fitted to measured B200 times of the decode shapes (M = 8, 16, 64):
+//   units <= 2 x CTAs:  ceil(units / CTAs) x (ku + c)           (whole rounds)
+//   otherwise:          units / CTAs x (ku + c) + 2 x ku        (dynamic claims
+//                                                   smooth the rounds; a tail of
+//                                                   about two units remains)
+// with c = 1 stage of per-unit overhead at X tiles <= 32 rows, 4 above
+// (larger partials).  FMA path (consumer warps run the epilogue themselves):
+// whole tiles unless there are fewer tiles than CTAs, then 2 units per tile.
 // Tail: the last tiles of the schedule may be split into smaller units, so
 // the end of a GEMM (which in a chain every dependent task waits for) is
 // spread evenly over CTAs that stream at different speeds.
+int auto_units_per_tile(const Geo &g, int ctas) {
+    if (g.path != WSM_PATH_UMMA) return std::max(1, std::min(g.tiles() >= ctas ? 1 : 2, g.kb));
+    const double G = std::max(1, ctas);
+    const double c = (g.t_mpad <= 32) ? 1.0 : 4.0;
+    int best = 1;
+    double best_cost = 1e300;
+    for (int nu = 1; nu <= std::min(4, g.kb); ++nu) {
+        const int ku = (g.kb + nu - 1) / nu;
+        const double units = (double)g.tiles() * ((g.kb + ku - 1) / ku);
+        const double cost = units <= 2 * G ? std::ceil(units / G) * (ku + c) : units / G * (ku + c) + 2.0 * ku;
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = nu;
+        }
+    }
+    return best;
+}
+
 wsm_status plan_units(Geo &g, int ctas, int unit_stages, int tail_tiles, int tail_unit_stages) {
     if (unit_stages < 0) return fail(WSM_ERR_INVALID, "bad unit_stages %d", unit_stages);
     if (tail_tiles < -1) return fail(WSM_ERR_INVALID, "bad tail_tiles %d", tail_tiles);
@@ -131,9 +155,7 @@ wsm_status plan_units(Geo &g, int ctas, int unit_stages, int tail_tiles, int tai
     if (unit_stages > 0) {
         g.ku = std::min(unit_stages, g.kb);
     } else {
-        // the FMA path splits a tile only when there are fewer tiles than CTAs
-        const int nu_max = (g.path == WSM_PATH_UMMA) ? 4 : (g.tiles() >= ctas ? 1 : 2);
-        const int nu = std::max(1, std::min(nu_max, g.kb));
+        const int nu = auto_units_per_tile(g, ctas);
         g.ku = (g.kb + nu - 1) / nu;
     }
     g.nu = (g.kb + g.ku - 1) / g.ku;
@@ -149,12 +171,12 @@ wsm_status plan_units(Geo &g, int ctas, int unit_stages, int tail_tiles, int tai
 // Automatic path choice.  Measured on B200 (graph-replayed back-to-back
 // launches of decode shapes, M = 1..8, weights 30 MB .. 940 MB): the FMA path
 // wins while its arithmetic per weight byte stays light and the weights are
-// small enough for its shorter ramp to matter -- M = 1 up to about 180 MiB of
+// small enough for its shorter ramp to matter -- M = 1 up to about 128 MiB of
 // weights, M = 2 up to about 96 MiB, M <= 4 up to about 64 MiB -- and the
 // tensor-core path wins everywhere else (at M >= 5 always).
 int auto_path(int M, long long w_bytes) {
     const long long MiB = 1ll << 20;
-    if (M == 1 && w_bytes <= 180 * MiB) return WSM_PATH_STREAM;
+    if (M == 1 && w_bytes <= 128 * MiB) return WSM_PATH_STREAM;
     if (M == 2 && w_bytes <= 96 * MiB) return WSM_PATH_STREAM;
     if (M <= 4 && w_bytes <= 64 * MiB) return WSM_PATH_STREAM;
     return WSM_PATH_UMMA;
@@ -204,7 +226,7 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
         }
         g.n_mt = (M + g.t_m - 1) / g.t_m;
         int sk = o->stage_k;
-        if (sk == 0) sk = (g.t_mpad <= 32) ? 256 : 128;  // measured best; wider X tiles leave room for fewer stages
+        if (sk == 0) sk = 256;  // measured best at every M up to 64 on B200, even where it leaves 2 stages
         if (sk != 64 && sk != 128 && sk != 256)
             return fail(WSM_ERR_UNSUPPORTED, "stage_k must be 64, 128 or 256 on the UMMA path (got %d)", sk);
         g.kps = sk / kUmmaBK;
@@ -527,6 +549,8 @@ wsm_status launch(const void *fn, const Geo &g, const KParams &kp, cudaStream_t 
 struct wsm_chain {
     int device = 0;
     int n = 0;
+    std::vector<wsm_chain *> parts;    // hybrid dispatch: one chain per run of tasks of one kind
+    std::vector<int> part_first;       // ... and the index of its first task
     wsm::Geo geo;                      // ring geometry shared by all tasks
     std::vector<wsm_task> tasks;
     std::vector<wsm::TaskDev> host_table;
@@ -735,6 +759,65 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     }
     if (path == WSM_PATH_STREAM && maxM > 8) return fail(WSM_ERR_UNSUPPORTED, "the FMA path takes M <= 8 (max M=%d)", maxM);
 
+    // Hybrid dispatch.  One kernel sizes its ring stages for the widest X tile: with M > 32 tasks in
+    // the chain, tasks of M <= 32 get 2 stages of 96 KB instead of 3 of 72 KB, about 5 % slower
+    // (measured on B200).  Split into one kernel per run of consecutive tasks of one kind, they keep
+    // their own ring; each extra kernel boundary costs up to about 20 us (the next task no longer
+    // overlaps the previous one's tail).  AUTO splits when the narrow tasks carry more than 1.5 GB of
+    // weights per extra kernel (measured: a 1.9 GB narrow run next to one M = 64 task gains 5 % from
+    // the split; 12 alternating runs of 0.3-0.4 GB lose 27 %).  A dependency that crosses kernels
+    // is met by stream order.
+    if (opts->kernels < WSM_CHAIN_KERNELS_AUTO || opts->kernels > WSM_CHAIN_KERNELS_SPLIT)
+        return fail(WSM_ERR_INVALID, "bad kernels option %d", opts->kernels);
+    if (path == WSM_PATH_UMMA && opts->kernels != WSM_CHAIN_KERNELS_ONE) {
+        auto wide = [&](int i) { return (tasks[i].M + 15) / 16 * 16 > 32; };
+        int kinds = 0, segments = 1;
+        double narrow_bytes = 0;
+        for (int i = 0; i < n; ++i) {
+            kinds |= wide(i) ? 2 : 1;
+            if (i > 0 && wide(i) != wide(i - 1)) ++segments;
+            if (!wide(i)) narrow_bytes += 2.0 * tasks[i].N * (double)tasks[i].K;
+        }
+        const bool split = kinds == 3 && (opts->kernels == WSM_CHAIN_KERNELS_SPLIT ||
+                                          narrow_bytes > 1.5e9 * (segments - 1));
+        if (split) {
+            std::unique_ptr<wsm_chain> parent(new wsm_chain());
+            parent->device = dev;
+            parent->n = n;
+            parent->tasks.assign(tasks, tasks + n);
+            auto cleanup = [&]() {
+                for (wsm_chain *c : parent->parts) wsm_chain_destroy(c);
+                parent->parts.clear();
+            };
+            for (int a = 0, b; a < n; a = b) {
+                for (b = a + 1; b < n && wide(b) == wide(a); ++b) {}
+                std::vector<wsm_task> sub(tasks + a, tasks + b);
+                for (wsm_task &t : sub) {
+                    if (t.dep >= a) {
+                        t.dep -= a;
+                    } else {  // met by stream order: the earlier kernel has completed
+                        t.dep = -1;
+                        t.dep_cols = 0;
+                    }
+                }
+                wsm_chain_opts so = *opts;
+                so.path = WSM_PATH_UMMA;
+                so.kernels = WSM_CHAIN_KERNELS_ONE;
+                so.trace = 0;
+                wsm_chain *part = nullptr;
+                if ((st = wsm_chain_create(sub.data(), b - a, &so, &part)) != WSM_OK) {
+                    cleanup();
+                    return fail(st, "tasks %d..%d: %s", a, b - 1, g_err.c_str());
+                }
+                parent->parts.push_back(part);
+                parent->part_first.push_back(a);
+            }
+            *out = parent.release();
+            g_err.clear();
+            return WSM_OK;
+        }
+    }
+
     std::unique_ptr<wsm_chain> ch(new wsm_chain());
     ch->device = dev;
     ch->n = n;
@@ -758,13 +841,8 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     wsm_opts to{};
     to.path = path;
     to.grid = opts->grid;
-    // one stage geometry for the whole chain (the ring and the kernel's boxes per stage are shared):
-    // on the UMMA path, auto stage_k follows the chain's widest X tile
-    to.stage_k = 0;
-    if (path == WSM_PATH_UMMA) {
-        to.stage_k = opts->stage_k;
-        if (to.stage_k == 0) to.stage_k = ((maxM + 15) / 16 * 16 <= 32) ? 256 : 128;
-    }
+    // one stage geometry for the whole chain (the ring and the kernel's boxes per stage are shared)
+    to.stage_k = (path == WSM_PATH_UMMA) ? (opts->stage_k ? opts->stage_k : 256) : 0;
     const int chain_mmax = (path == WSM_PATH_STREAM) ? pow2ceil(maxM) : 0;
     for (int i = 0; i < n; ++i) {
         if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, d->sms, &to, geos[i], chain_mmax)) != WSM_OK)
@@ -937,6 +1015,13 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
 
 wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     if (!ch) return fail(WSM_ERR_INVALID, "chain is null");
+    if (!ch->parts.empty()) {
+        for (wsm_chain *part : ch->parts) {
+            wsm_status st = wsm_chain_run(part, stream_);
+            if (st != WSM_OK) return st;
+        }
+        return WSM_OK;
+    }
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     int dev = 0;
     WSM_CUDA(cudaGetDevice(&dev));
@@ -969,6 +1054,19 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
 
 wsm_status wsm_chain_status(wsm_chain *ch, wsm_stream_t stream_, int *failed_task) {
     if (!ch) return fail(WSM_ERR_INVALID, "chain is null");
+    if (!ch->parts.empty()) {
+        wsm_status first = WSM_OK;
+        if (failed_task) *failed_task = -1;
+        for (size_t k = 0; k < ch->parts.size(); ++k) {
+            int ft = -1;
+            wsm_status st = wsm_chain_status(ch->parts[k], stream_, &ft);
+            if (st != WSM_OK && first == WSM_OK) {
+                first = st;
+                if (failed_task) *failed_task = ft < 0 ? -1 : ch->part_first[k] + ft;
+            }
+        }
+        return first;
+    }
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     WSM_CUDA(cudaStreamSynchronize(stream));
     int h[kStatusWords] = {};
@@ -993,6 +1091,11 @@ size_t wsm_chain_trace(wsm_chain *ch, wsm_stream_t stream_, unsigned long long *
 
 void wsm_chain_destroy(wsm_chain *ch) {
     if (!ch) return;
+    if (!ch->parts.empty()) {
+        for (wsm_chain *part : ch->parts) wsm_chain_destroy(part);
+        delete ch;
+        return;
+    }
     int prev = 0;
     cudaGetDevice(&prev);
     cudaSetDevice(ch->device);
