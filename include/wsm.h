@@ -141,6 +141,9 @@ typedef struct {
     int l2_prefetch_stages; /* W pipeline stages per CTA prefetched into L2 while the
                                CTA waits for the previous kernel (WSM_FLAG_W_READONLY):
                                0 = auto, -1 = none */
+    int tile_rows;   /* tensor-core path: W rows per tile, 0 = auto, 128, or 256 (two
+                        128-row halves share each X stage and accumulate into two
+                        TMEM accumulators, so X is re-read half as often) */
     int epilogue;    /* WSM_EPI_*; with SILU_MUL, Y (and Yf32) are [M, N/2] */
     const void *R;   /* WSM_EPI_RESIDUAL: bf16 [M, N], device */
     float *Yf32;     /* optional device [M, N] fp32: the result before rounding */
@@ -274,6 +277,7 @@ typedef struct {
                                   bumps the task's counter once.  An ablation: the pages use
                                   it to save cross-die fences, which B200's coherent L2 does
                                   not need.  Not with dep_cols tasks (WSM_ERR_UNSUPPORTED). */
+    int tile_rows;             /* as in wsm_opts; auto: 256 only if auto picks it for every task */
     int kernels;               /* WSM_CHAIN_KERNELS_*: hybrid dispatch.  One kernel sizes its
                                   pipeline stages for the chain's widest X tile, which costs
                                   tasks of M <= 32 about 5 % when M > 32 tasks share the chain;

@@ -127,6 +127,25 @@ def test_two_level_rejects_column_dependencies():
     assert e.value.code == wsm.WSM_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("M", [16, 64])
+def test_dependent_chain_wide_tiles(M):
+    """A data-dependent chain on wide tiles (two 128-row halves per tile),
+    with whole-task and per-column dependencies."""
+    dims = [1024, 2048, 1024, 3072, 768]
+    x0, ws, ys, yfs, tasks = dependent_chain(M, dims, seed=70 + M)
+    for cols in (False, True):
+        for i, t in enumerate(tasks):
+            t.dep_cols = cols and i > 0
+        ch = wsm.Chain(tasks, path=wsm.PATH_UMMA, tile_rows=256)
+        for _ in range(2):
+            for y in ys:
+                y.fill_(float("nan"))
+            ch.run()
+            assert ch.status()[0] == wsm.WSM_OK, wsm.last_error()
+            check_dependent(x0, ws, ys, yfs)
+        ch.close()
+
+
 def test_dependent_chain_small_grid_and_empty_ctas():
     """A grid larger than some tasks' stage counts (CTAs with no work for a
     task) and a tiny grid (long per-CTA ranges)."""

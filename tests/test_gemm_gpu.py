@@ -315,3 +315,45 @@ def test_back_to_back_dependent_calls(flags, path, M):
         for i, w in enumerate(ws):
             check_full(x.cpu(), w.cpu(), ys[i], what=f"rep {rep} call {i} flags {flags}")
             x = ys[i]
+
+
+# --------------------------------------------------------------------------- wide tiles
+
+
+@pytest.mark.parametrize("M", [1, 16, 33, 64])
+@pytest.mark.parametrize("N,K", [(1000, 1032), (129, 4104), (4096, 4096), (300, 256)])
+def test_wide_tiles(M, N, K):
+    """Tiles of two 128-row W halves sharing each X stage (two accumulators):
+    ragged N (the second half may lie past N), every grid split."""
+    x, w = synth.make_xw(M, N, K, seed=M * 7 + N)
+    for grid in (0, 5):
+        y, yf = run(x, w, path=wsm.PATH_UMMA, tile_rows=256, grid=grid)
+        check_full(x, w, y, yf, what=f"wide M={M} grid={grid}")
+
+
+@pytest.mark.parametrize("M", [16, 64])
+def test_wide_tiles_integer_exact_and_options(M):
+    N, K = 1000, 3072
+    x, w = synth.make_int_xw(M, N, K, seed=M)
+    Y_ref, _ = oracle.gemm_ref(x, w)
+    for kw in (dict(), dict(unit_stages=1), dict(stage_k=64), dict(stage_k=256), dict(m_tile=16),
+               dict(tail_tiles=2, tail_unit_stages=1)):
+        y, yf = run(x, w, path=wsm.PATH_UMMA, tile_rows=256, **kw)
+        assert np.array_equal(yf.cpu().double().numpy(), Y_ref), kw
+        assert np.array_equal(bf16_bits(y), oracle.round_bf16(Y_ref)), kw
+
+
+def test_wide_tiles_fused_epilogues():
+    M, N, K = 32, 1024, 2048
+    x, w = synth.make_xw(M, N, K, seed=91)
+    y = torch.full((M, N // 2), float("nan"), dtype=torch.bfloat16, device=DEV)
+    yf = torch.full((M, N // 2), float("nan"), dtype=torch.float32, device=DEV)
+    wsm.skinny_gemm(x.to(DEV), w.to(DEV), y, yf32=yf, path=wsm.PATH_UMMA, tile_rows=256, epilogue=wsm.EPI_SILU_MUL)
+    torch.cuda.synchronize()
+    H, G, U, Sg, Su = oracle.silu_mul_ref(x, w)
+    from parity import check_bounded
+    check_bounded(y, yf, H, oracle.fused_bounds("silu_mul", G=G, U=U, Sg=Sg, Su=Su), "wide silu")
+    r = synth.make_x(M, N, 92)
+    y, yf = run(x, w, path=wsm.PATH_UMMA, tile_rows=256, epilogue=wsm.EPI_RESIDUAL, r=r.to(DEV))
+    Yr, S = oracle.residual_ref(x, w, r)
+    check_bounded(y, yf, Yr, oracle.fused_bounds("residual", S=S, Y=Yr), "wide residual")

@@ -56,7 +56,8 @@ class _Opts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("m_tile", ctypes.c_int), ("order", ctypes.c_int),
                 ("l2_policy", ctypes.c_int), ("grid", ctypes.c_int), ("stage_k", ctypes.c_int),
                 ("flags", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
-                ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int), ("epilogue", ctypes.c_int),
+                ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int), ("tile_rows", ctypes.c_int),
+                ("epilogue", ctypes.c_int),
                 ("R", ctypes.c_void_p), ("Yf32", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t)]
 
@@ -82,7 +83,7 @@ class _ChainOpts(ctypes.Structure):
                 ("trace", ctypes.c_int), ("debug_unmet_dependency", ctypes.c_int), ("flags", ctypes.c_int),
                 ("stage_k", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
                 ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int),
-                ("counter_groups", ctypes.c_int), ("kernels", ctypes.c_int)]
+                ("counter_groups", ctypes.c_int), ("tile_rows", ctypes.c_int), ("kernels", ctypes.c_int)]
 
 
 _lib = None
@@ -169,13 +170,14 @@ def _check_operand(name, t, dtype=torch.bfloat16):
 
 def _opts(path=PATH_AUTO, m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32=None, workspace=None,
           stage_k=0, flags=0, unit_stages=0, tail_tiles=0, tail_unit_stages=0, l2_prefetch_stages=0, epilogue=0,
-          r=None):
+          r=None, tile_rows=0):
     o = _Opts()
     o.path, o.m_tile, o.order, o.l2_policy, o.grid, o.stage_k = path, m_tile, order, l2_policy, grid, stage_k
     o.flags, o.unit_stages, o.tail_tiles, o.tail_unit_stages = flags, unit_stages, tail_tiles, tail_unit_stages
     o.l2_prefetch_stages = l2_prefetch_stages
     o.epilogue = epilogue
     o.R = _ptr(r)
+    o.tile_rows = tile_rows
     o.Yf32 = _ptr(yf32)
     if workspace is not None:
         o.workspace = workspace.data_ptr()
@@ -187,7 +189,7 @@ def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = No
                 m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None, stage_k=0, flags=0, unit_stages=0, tail_tiles=0,
                 tail_unit_stages=0, l2_prefetch_stages=0, epilogue=EPI_NONE, r: Optional[torch.Tensor] = None,
-                stream=None) -> torch.Tensor:
+                tile_rows=0, stream=None) -> torch.Tensor:
     """Y = X @ W.T on the current (or given) stream; returns Y.  With
     epilogue=EPI_SILU_MUL, W is the fused gate+up weight (rows interleaved in
     blocks of 8) and Y is [M, N/2] = silu(gate) * up; with EPI_RESIDUAL,
@@ -215,14 +217,14 @@ def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = No
         if tuple(r.shape) != (M, N):
             raise ValueError(f"r must be [{M}, {N}]")
     plain = (path, m_tile, order, l2_policy, grid, stage_k, flags, unit_stages, tail_tiles, tail_unit_stages,
-             l2_prefetch_stages, epilogue) == (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0, 0, 0, 0, 0, 0, 0, 0) \
+             l2_prefetch_stages, epilogue, tile_rows) == (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0, 0, 0, 0, 0, 0, 0, 0, 0) \
         and yf32 is None and workspace is None
     s = _stream_handle(stream)
     if plain:
         _check(lib().skinny_gemm(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, s), "skinny_gemm")
     else:
         o = _opts(path, m_tile, order, l2_policy, grid, yf32, workspace, stage_k, flags, unit_stages, tail_tiles,
-                  tail_unit_stages, l2_prefetch_stages, epilogue, r)
+                  tail_unit_stages, l2_prefetch_stages, epilogue, r, tile_rows)
         _check(lib().skinny_gemm_ex(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, ctypes.byref(o), s),
                "skinny_gemm_ex")
     return y
@@ -308,7 +310,7 @@ class Chain:
 
     def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
                  debug_unmet_dependency=False, flags=0, stage_k=0, unit_stages=0, tail_tiles=0,
-                 tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0, kernels=0):
+                 tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0, kernels=0, tile_rows=0):
         for i, t in enumerate(tasks):
             _check_operand(f"tasks[{i}].x", t.x)
             _check_operand(f"tasks[{i}].w", t.w)
@@ -323,6 +325,7 @@ class Chain:
         o.l2_prefetch_stages = l2_prefetch_stages
         o.counter_groups = counter_groups
         o.kernels = kernels
+        o.tile_rows = tile_rows
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

@@ -81,6 +81,7 @@ struct Geo {
     int threads = 0;
     int kps = 1;               // UMMA: 64-wide K boxes per stage
     int x_stride = 0;          // UMMA: bytes between X boxes inside a stage
+    int wide = 0;              // UMMA: tiles of 2 x 128 W rows sharing each X stage
     long long iters() const { return (long long)n_g * n_mt * kb; }
     long long tiles() const { return (long long)n_g * n_mt; }
     long long units() const { return (tiles() - tail) * nu + (long long)tail * nu_t; }
@@ -182,6 +183,17 @@ int auto_path(int M, long long w_bytes) {
     return WSM_PATH_UMMA;
 }
 
+// Wide tiles (tensor-core path): two 128-row halves of W share each X stage,
+// so X is re-read by half as many tiles.  Measured on B200 (the decode shapes
+// at M = 16..64) they are slower at every shape (e.g. gate_up at M = 64:
+// 54.3 us against 52.0 us; down: 52.6 against 34.8 us): twice the W per
+// stage needs 128-wide stages, and the ring then holds fewer bytes in flight.
+// An option (tile_rows = 256), never the automatic choice.
+bool auto_wide(int t_mpad) {
+    (void)t_mpad;
+    return false;
+}
+
 // force_mmax: a chain's FMA kernel has one register width for all tasks.
 wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g, int force_mmax = 0) {
     if (!shape_ok(M, N, K))
@@ -225,19 +237,28 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
             g.t_mpad = (g.t_m + 15) / 16 * 16;
         }
         g.n_mt = (M + g.t_m - 1) / g.t_m;
+        if (o->tile_rows != 0 && o->tile_rows != kUmmaRows && o->tile_rows != 2 * kUmmaRows)
+            return fail(WSM_ERR_UNSUPPORTED, "tile_rows must be 0, 128 or 256 on the UMMA path (got %d)", o->tile_rows);
+        g.wide = (o->tile_rows == 0) ? auto_wide(g.t_mpad) : (o->tile_rows == 2 * kUmmaRows);
         int sk = o->stage_k;
-        if (sk == 0) sk = 256;  // measured best at every M up to 64 on B200, even where it leaves 2 stages
+        // measured best on B200: 256 at every M up to 64 (even where that leaves 2 stages); wide tiles
+        // carry twice the W per stage, so 128
+        if (sk == 0) sk = g.wide ? 128 : 256;
         if (sk != 64 && sk != 128 && sk != 256)
             return fail(WSM_ERR_UNSUPPORTED, "stage_k must be 64, 128 or 256 on the UMMA path (got %d)", sk);
+        const int halves = g.wide ? 2 : 1;
         g.kps = sk / kUmmaBK;
-        g.tile_rows = kUmmaRows;
+        g.tile_rows = halves * kUmmaRows;
         g.tile_k = sk;
-        g.n_g = (N + kUmmaRows - 1) / kUmmaRows;
+        g.n_g = (N + g.tile_rows - 1) / g.tile_rows;
         g.kb = (K + g.tile_k - 1) / g.tile_k;
         g.x_stride = g.t_mpad * kUmmaBK * 2;                        // X rows x 128 B (multiple of 1024)
-        g.x_off = g.kps * kUmmaRows * kUmmaBK * 2;                  // W boxes, 16 KB each
+        g.x_off = halves * g.kps * kUmmaRows * kUmmaBK * 2;         // W boxes, 16 KB each
         g.stage_bytes = g.x_off + g.kps * g.x_stride;
-        g.slot_elems = kUmmaRows * g.t_mpad;
+        g.slot_elems = g.tile_rows * g.t_mpad;
+        if (g.stage_bytes > kRingBudget)
+            return fail(WSM_ERR_UNSUPPORTED, "a pipeline stage of %d bytes does not fit in shared memory (use a "
+                                             "smaller stage_k with wide tiles)", g.stage_bytes);
         g.threads = 64 + 2 * 128;   // producer, MMA, two epilogue warp sets
     }
     g.stages = std::min(kMaxStages, kRingBudget / g.stage_bytes);
@@ -413,7 +434,7 @@ wsm_status fill_task(TaskDev &T, const Geo &g, const void *X, const void *W, voi
     if (g.path == WSM_PATH_UMMA) {
         if ((st = encode_2d(&T.tmW, W, N, K, kUmmaBK, kUmmaRows, CU_TENSOR_MAP_SWIZZLE_128B)) != WSM_OK) return st;
         if ((st = encode_2d(&T.tmX, X, M, K, kUmmaBK, g.t_mpad, CU_TENSOR_MAP_SWIZZLE_128B)) != WSM_OK) return st;
-        T.tx_bytes = (uint32_t)(g.kps * (kUmmaRows * kUmmaBK * 2 + g.t_mpad * kUmmaBK * 2));
+        T.tx_bytes = (uint32_t)(g.kps * ((g.wide ? 2 : 1) * kUmmaRows * kUmmaBK * 2 + g.t_mpad * kUmmaBK * 2));
         T.idesc = umma_idesc(g.t_mpad);
     } else {
         if ((st = encode_2d(&T.tmW, W, N, K, kStreamBoxK, g.tile_rows, CU_TENSOR_MAP_SWIZZLE_NONE)) != WSM_OK)
@@ -684,6 +705,7 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     kp.x_off = g.x_off;
     kp.kps = g.kps;
     kp.x_stride = g.x_stride;
+    kp.wide = g.wide;
     kp.pdl = pdl_mode(opts->flags);
     kp.prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, g.path);
     kp.run_ctl = nullptr;
@@ -841,8 +863,20 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     wsm_opts to{};
     to.path = path;
     to.grid = opts->grid;
-    // one stage geometry for the whole chain (the ring and the kernel's boxes per stage are shared)
-    to.stage_k = (path == WSM_PATH_UMMA) ? (opts->stage_k ? opts->stage_k : 256) : 0;
+    // one stage geometry for the whole chain (the ring and the kernel's boxes per stage are shared):
+    // wide tiles only if every task would take them
+    bool chain_wide = false;
+    if (path == WSM_PATH_UMMA) {
+        if (opts->tile_rows != 0 && opts->tile_rows != kUmmaRows && opts->tile_rows != 2 * kUmmaRows)
+            return fail(WSM_ERR_UNSUPPORTED, "tile_rows must be 0, 128 or 256 (got %d)", opts->tile_rows);
+        chain_wide = opts->tile_rows == 2 * kUmmaRows;
+        if (opts->tile_rows == 0) {
+            chain_wide = true;
+            for (int i = 0; i < n; ++i) chain_wide = chain_wide && auto_wide((tasks[i].M + 15) / 16 * 16);
+        }
+        to.tile_rows = chain_wide ? 2 * kUmmaRows : kUmmaRows;
+    }
+    to.stage_k = (path == WSM_PATH_UMMA) ? (opts->stage_k ? opts->stage_k : (chain_wide ? 128 : 256)) : 0;
     const int chain_mmax = (path == WSM_PATH_STREAM) ? pow2ceil(maxM) : 0;
     for (int i = 0; i < n; ++i) {
         if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, d->sms, &to, geos[i], chain_mmax)) != WSM_OK)
@@ -858,12 +892,15 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         int tmp = 16;
         for (auto &g : geos) tmp = std::max(tmp, g.t_mpad);
         ring.x_stride = tmp * kUmmaBK * 2;
-        ring.x_off = ring.kps * kUmmaRows * kUmmaBK * 2;
+        ring.x_off = (ring.wide ? 2 : 1) * ring.kps * kUmmaRows * kUmmaBK * 2;
         ring.stage_bytes = ring.x_off + ring.kps * ring.x_stride;
+        if (ring.stage_bytes > kRingBudget)
+            return fail(WSM_ERR_UNSUPPORTED, "the chain's pipeline stage of %d bytes does not fit in shared memory",
+                        ring.stage_bytes);
     }
     ring.stages = std::min(kMaxStages, kRingBudget / ring.stage_bytes);
     for (int i = 0; i < n; ++i)
-        if (geos[i].kps != ring.kps || geos[i].tile_k != ring.tile_k)
+        if (geos[i].kps != ring.kps || geos[i].tile_k != ring.tile_k || geos[i].wide != ring.wide)
             return fail(WSM_ERR_INVALID, "task %d: stage geometry differs from the chain's", i);  // cannot happen
     ch->geo = ring;
     ch->prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, path);
@@ -1041,6 +1078,7 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     kp.x_off = ch->geo.x_off;
     kp.kps = ch->geo.kps;
     kp.x_stride = ch->geo.x_stride;
+    kp.wide = ch->geo.wide;
     kp.pdl = ch->pdl;
     kp.prefetch_stages = ch->prefetch_stages;
     kp.run_ctl = ch->d_run_ctl;

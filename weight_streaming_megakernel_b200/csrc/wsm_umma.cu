@@ -125,7 +125,8 @@ constexpr int kEpiSets = 2;         // two independent epilogue warp sets (units
 constexpr int kEpiThreads = 128;    // per set: four warps, one per TMEM lane quadrant
 constexpr int kThreads = 64 + kEpiSets * kEpiThreads;
 constexpr int kAccBufs = 4;         // accumulators in TMEM: the MMA can run up to three units ahead
-constexpr uint32_t kTmemCols = kAccBufs * kUmmaMaxN;
+constexpr uint32_t kTmemCols = kAccBufs * kUmmaMaxN;   // 128-row tiles
+constexpr uint32_t kTmemColsWide = 2 * kTmemCols;        // wide tiles: two accumulators per buffer (all of TMEM)
 
 __device__ __forceinline__ void epi_bar(int set) { named_bar_sync(1 + set, kEpiThreads); }
 
@@ -220,8 +221,11 @@ static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDe
         const UnitSpan ps = unit_span(T, uu);
         int pg, pmt;
         tile_coords(T, ps.tile, pg, pmt);
+        const int halves = p.wide ? 2 : 1;
         for (int kk = ps.k_begin + (uu < (int)gridDim.x ? S : 0); kk < ps.k_end && budget > 0; ++kk, --budget)
-            for (int j = 0; j < p.kps; ++j) tma_prefetch_l2_2d(&T.tmW, (kk * p.kps + j) * kUmmaBK, pg * kUmmaRows);
+            for (int h = 0; h < halves; ++h)
+                for (int j = 0; j < p.kps; ++j)
+                    tma_prefetch_l2_2d(&T.tmW, (kk * p.kps + j) * kUmmaBK, (pg * halves + h) * kUmmaRows);
     }
 }
 
@@ -258,7 +262,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         fence_mbar_init();
         pdl_launch_dependents();
     }
-    if (warp == 1) tmem_alloc(&tmem_base_sh, kTmemCols);
+    const int halves = p.wide ? 2 : 1;          // 128-row W halves per tile
+    const uint32_t acc_stride = (uint32_t)(halves * kUmmaMaxN);  // TMEM columns per accumulator buffer
+    if (warp == 1) tmem_alloc(&tmem_base_sh, p.wide ? kTmemColsWide : kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -391,9 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         stage_meta[s][2] = (kk == us.k_begin ? kMetaFirst : 0) | (kk == us.k_end - 1 ? kMetaLast : 0);
                         mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
                         const int k0 = kk * p.kps * kUmmaBK;
-                        for (int j = 0; j < p.kps; ++j)
-                            tma_load_2d(st + j * (kUmmaRows * kUmmaBK * 2), &T.tmW, &full_bar[s], k0 + j * kUmmaBK,
-                                        g * kUmmaRows, pol_w);
+                        for (int h = 0; h < halves; ++h)
+                            for (int j = 0; j < p.kps; ++j)
+                                tma_load_2d(st + (h * p.kps + j) * (kUmmaRows * kUmmaBK * 2), &T.tmW, &full_bar[s],
+                                            k0 + j * kUmmaBK, (g * halves + h) * kUmmaRows, pol_w);
                         if (x_now(k0)) {
                             for (int j = 0; j < p.kps; ++j)
                                 tma_load_2d(st + p.x_off + j * p.x_stride, &T.tmX, &full_bar[s], k0 + j * kUmmaBK, xy,
@@ -486,16 +493,19 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     tc_fence_after();
                 }
                 const TaskDev &T = task_at(p, t);
-                const uint32_t d_tmem = tmem_base + (uint32_t)(buf * kUmmaMaxN);
                 const uint32_t st0 = smem_u32(ring + (size_t)s * p.stage_bytes);
-                for (int j = 0; j < p.kps; ++j) {
-                    const uint32_t a0 = st0 + (uint32_t)(j * kUmmaRows * kUmmaBK * 2);
-                    const uint32_t b0 = st0 + (uint32_t)(p.x_off + j * p.x_stride);
+                for (int h = 0; h < halves; ++h) {
+                    // half h of the tile's W rows accumulates into columns h * 64 .. of the buffer
+                    const uint32_t d_tmem = tmem_base + (uint32_t)buf * acc_stride + (uint32_t)(h * kUmmaMaxN);
+                    for (int j = 0; j < p.kps; ++j) {
+                        const uint32_t a0 = st0 + (uint32_t)((h * p.kps + j) * kUmmaRows * kUmmaBK * 2);
+                        const uint32_t b0 = st0 + (uint32_t)(p.x_off + j * p.x_stride);
 #pragma unroll
-                    for (int k = 0; k < kUmmaBK / 16; ++k) {
-                        // advancing K by 16 bf16 = 32 bytes inside the swizzle atom
-                        tc_mma(d_tmem, sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k), T.idesc,
-                               ((flags & kMetaFirst) && j == 0 && k == 0) ? 0u : 1u);
+                        for (int k = 0; k < kUmmaBK / 16; ++k) {
+                            // advancing K by 16 bf16 = 32 bytes inside the swizzle atom
+                            tc_mma(d_tmem, sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k), T.idesc,
+                                   ((flags & kMetaFirst) && j == 0 && k == 0) ? 0u : 1u);
+                        }
                     }
                 }
                 any_mma = true;
@@ -545,31 +555,37 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             const int tile = us.tile;
             int g, mt;
             tile_coords(T, tile, g, mt);
-            const int n = g * kUmmaRows + row;
             const int m0 = mt * T.t_m;
             const int mrows = min(T.t_m, T.M - m0);
             UnitOut uo = unit_out(T);  // no task-table reads after the first store below
             unit_out_group(uo, T, tile);
-            // The accumulator, 16 columns (X rows) at a time: TMEM -> registers -> outputs (whole tile) or
-            // this unit's partial row [row][m] (split tile).  The loop is not unrolled: one copy of the
-            // epilogue code per kind keeps the kernel small.
+            // The accumulator, 16 columns (X rows) at a time, per 128-row half of the tile: TMEM ->
+            // registers -> outputs (whole tile) or this unit's partial rows [row][m] (split tile).  The
+            // loops are not unrolled: one copy of the epilogue code per kind keeps the kernel small.
             tc_fence_after();
-            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kUmmaMaxN);
-            float4 *dst = reinterpret_cast<float4 *>(uo.part + (size_t)u * uo.slot_elems + (size_t)row * uo.t_mpad);
 #pragma unroll 1
-            for (int c = 0; c < mrows; c += 16) {
-                uint32_t r[16];
-                tmem_ld16(taddr + (uint32_t)c, r);
-                tmem_ld_wait16(r);
-                float v[16];
+            for (int h = 0; h < halves; ++h) {
+                const int n = (g * halves + h) * kUmmaRows + row;
+                const uint32_t taddr =
+                    tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * acc_stride + (uint32_t)(h * kUmmaMaxN);
+                float4 *dst = reinterpret_cast<float4 *>(uo.part + (size_t)u * uo.slot_elems +
+                                                         (size_t)(h * kUmmaRows + row) * uo.t_mpad);
+#pragma unroll 1
+                for (int c = 0; c < mrows; c += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(taddr + (uint32_t)c, r);
+                    tmem_ld_wait16(r);
+                    float v[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-                if (us.nu == 1) {
-                    emit_outputs<16>(uo.e, n, m0 + c, min(16, mrows - c), v);
-                } else {
+                    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+                    if (us.nu == 1) {
+                        emit_outputs<16>(uo.e, n, m0 + c, min(16, mrows - c), v);
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (c + 4 * i < mrows) dst[c / 4 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        for (int i = 0; i < 4; ++i)
+                            if (c + 4 * i < mrows)
+                                dst[c / 4 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    }
                 }
             }
             tc_fence_before();
@@ -579,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             if (us.nu == 1) {
                 if (uo.done || uo.col_cnt) {
                     epi_bar(set);
-                    if (leader) tile_finished(uo, g, kUmmaRows, run_no);  // release covers the set's stores (bar.sync before)
+                    if (leader) tile_finished(uo, g, halves * kUmmaRows, run_no);  // release covers the set's stores
                 }
             } else {
                 // the last unit of the tile to arrive adds all the partials
@@ -593,14 +609,18 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 epi_bar(set);
                 if (last_flag[set]) {
                     // the leader's acquire + the barrier order these loads after every partial
-                    if (mrows <= 4)
-                        reduce_row_partials<4, 16>(uo, us, row, mrows, m0, n);
-                    else
-                        reduce_row_partials<16, 4>(uo, us, row, mrows, m0, n);
+#pragma unroll 1
+                    for (int h = 0; h < halves; ++h) {
+                        const int n = (g * halves + h) * kUmmaRows + row;
+                        if (mrows <= 4)
+                            reduce_row_partials<4, 16>(uo, us, h * kUmmaRows + row, mrows, m0, n);
+                        else
+                            reduce_row_partials<16, 4>(uo, us, h * kUmmaRows + row, mrows, m0, n);
+                    }
                     epi_bar(set);
                     if (leader) {
                         uo.tile_cnt[tile] = 0u;  // ready for the next call
-                        tile_finished(uo, g, kUmmaRows, run_no);
+                        tile_finished(uo, g, halves * kUmmaRows, run_no);
                     }
                 }
             }
@@ -611,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+    if (warp == 1) tmem_dealloc(tmem_base, p.wide ? kTmemColsWide : kTmemCols);
     if (threadIdx.x == 0) chain_run_done(p);
 }
 
