@@ -131,7 +131,7 @@ typedef struct {
     int grid;        /* persistent CTAs, 0 = one per SM; values above the
                         number of SMs are clamped */
     int stage_k;     /* UMMA path: K elements per pipeline stage, 0 = auto,
-                        else 64, 128 or 256 */
+                        else 64, 128, 192 or 256 */
     int flags;       /* WSM_FLAG_* */
     int unit_stages; /* pipeline stages per work unit, 0 = auto (see wsm_plan_info) */
     int tail_tiles;  /* the last tail_tiles tiles of the schedule are split into
@@ -144,6 +144,9 @@ typedef struct {
     int tile_rows;   /* tensor-core path: W rows per tile, 0 = auto, 128, or 256 (two
                         128-row halves share each X stage and accumulate into two
                         TMEM accumulators, so X is re-read half as often) */
+    int k_order;     /* tensor-core path: order of a work unit's K stages: 0 = auto,
+                        1 = increasing, 2 = rotated by a tile-dependent offset (so the
+                        CTAs do not all read the same lines of X at the same time) */
     int epilogue;    /* WSM_EPI_*; with SILU_MUL, Y (and Yf32) are [M, N/2] */
     const void *R;   /* WSM_EPI_RESIDUAL: bf16 [M, N], device */
     float *Yf32;     /* optional device [M, N] fp32: the result before rounding */
@@ -278,6 +281,7 @@ typedef struct {
                                   it to save cross-die fences, which B200's coherent L2 does
                                   not need.  Not with dep_cols tasks (WSM_ERR_UNSUPPORTED). */
     int tile_rows;             /* as in wsm_opts; auto: 256 only if auto picks it for every task */
+    int k_order;               /* as in wsm_opts */
     int kernels;               /* WSM_CHAIN_KERNELS_*: hybrid dispatch.  One kernel sizes its
                                   pipeline stages for the chain's widest X tile, which costs
                                   tasks of M <= 32 about 5 % when M > 32 tasks share the chain;

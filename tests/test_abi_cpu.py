@@ -61,8 +61,8 @@ def test_plan_paths_and_geometry():
     assert p["tile_k"] == 64 and p["k_iters"] == 64
     p = wsm.plan(48, 4096, 4096, num_sms=148)
     assert p["tile_k"] == 256 and p["m_tile"] == 48 and p["stages"] == 2
-    p = wsm.plan(17, 100, 1000, num_sms=148)
-    assert p["m_tile"] == 32 and p["n_tiles"] == 1 and p["k_iters"] == 4
+    p = wsm.plan(17, 100, 1000, num_sms=148)          # 32-row X tiles: 192-wide stages
+    assert p["m_tile"] == 32 and p["n_tiles"] == 1 and p["tile_k"] == 192 and p["k_iters"] == 6
     p = wsm.plan(8, 4096, 4096, num_sms=148, path=wsm.PATH_UMMA)
     assert p["path"] == wsm.PATH_UMMA and p["m_tile"] == 16
 

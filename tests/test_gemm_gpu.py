@@ -357,3 +357,33 @@ def test_wide_tiles_fused_epilogues():
     y, yf = run(x, w, path=wsm.PATH_UMMA, tile_rows=256, epilogue=wsm.EPI_RESIDUAL, r=r.to(DEV))
     Yr, S = oracle.residual_ref(x, w, r)
     check_bounded(y, yf, Yr, oracle.fused_bounds("residual", S=S, Y=Yr), "wide residual")
+
+
+@pytest.mark.parametrize("M", [1, 16, 64])
+def test_rotated_k_order(M):
+    """Units walking their K stages from a tile-dependent offset: exact on
+    small integers, within the bound on random inputs, deterministic."""
+    N, K = 1000, 6144
+    xi, wi = synth.make_int_xw(M, N, K, seed=3 + M)
+    Y_ref, _ = oracle.gemm_ref(xi, wi)
+    for kw in (dict(), dict(unit_stages=5), dict(grid=7)):
+        y, yf = run(xi, wi, path=wsm.PATH_UMMA, k_order=2, **kw)
+        assert np.array_equal(yf.cpu().double().numpy(), Y_ref), kw
+    x, w = synth.make_xw(M, N, K, seed=4 + M)
+    y1, yf1 = run(x, w, path=wsm.PATH_UMMA, k_order=2, unit_stages=7)
+    check_full(x, w, y1, yf1)
+    y2, yf2 = run(x, w, path=wsm.PATH_UMMA, k_order=2, unit_stages=7)
+    assert torch.equal(yf1, yf2)
+
+
+@pytest.mark.parametrize("M", [16, 32, 64])
+@pytest.mark.parametrize("stage_k", [64, 128, 192, 256])
+def test_stage_widths_exact(M, stage_k):
+    """Every stage width, including 192 (three 64-wide boxes: K = 4104 leaves
+    a last stage of one partial box and two boxes past K, zero-filled)."""
+    N, K = 700, 4104
+    x, w = synth.make_int_xw(M, N, K, seed=stage_k + M)
+    Y_ref, _ = oracle.gemm_ref(x, w)
+    y, yf = run(x, w, path=wsm.PATH_UMMA, stage_k=stage_k)
+    assert np.array_equal(yf.cpu().double().numpy(), Y_ref)
+    assert np.array_equal(bf16_bits(y), oracle.round_bf16(Y_ref))

@@ -57,7 +57,7 @@ class _Opts(ctypes.Structure):
                 ("l2_policy", ctypes.c_int), ("grid", ctypes.c_int), ("stage_k", ctypes.c_int),
                 ("flags", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
                 ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int), ("tile_rows", ctypes.c_int),
-                ("epilogue", ctypes.c_int),
+                ("k_order", ctypes.c_int), ("epilogue", ctypes.c_int),
                 ("R", ctypes.c_void_p), ("Yf32", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t)]
 
@@ -83,7 +83,8 @@ class _ChainOpts(ctypes.Structure):
                 ("trace", ctypes.c_int), ("debug_unmet_dependency", ctypes.c_int), ("flags", ctypes.c_int),
                 ("stage_k", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
                 ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int),
-                ("counter_groups", ctypes.c_int), ("tile_rows", ctypes.c_int), ("kernels", ctypes.c_int)]
+                ("counter_groups", ctypes.c_int), ("tile_rows", ctypes.c_int), ("k_order", ctypes.c_int),
+                ("kernels", ctypes.c_int)]
 
 
 _lib = None
@@ -170,7 +171,7 @@ def _check_operand(name, t, dtype=torch.bfloat16):
 
 def _opts(path=PATH_AUTO, m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32=None, workspace=None,
           stage_k=0, flags=0, unit_stages=0, tail_tiles=0, tail_unit_stages=0, l2_prefetch_stages=0, epilogue=0,
-          r=None, tile_rows=0):
+          r=None, tile_rows=0, k_order=0):
     o = _Opts()
     o.path, o.m_tile, o.order, o.l2_policy, o.grid, o.stage_k = path, m_tile, order, l2_policy, grid, stage_k
     o.flags, o.unit_stages, o.tail_tiles, o.tail_unit_stages = flags, unit_stages, tail_tiles, tail_unit_stages
@@ -178,6 +179,7 @@ def _opts(path=PATH_AUTO, m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0,
     o.epilogue = epilogue
     o.R = _ptr(r)
     o.tile_rows = tile_rows
+    o.k_order = k_order
     o.Yf32 = _ptr(yf32)
     if workspace is not None:
         o.workspace = workspace.data_ptr()
@@ -189,7 +191,7 @@ def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = No
                 m_tile=0, order=ORDER_AUTO, l2_policy=L2_AUTO, grid=0, yf32: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None, stage_k=0, flags=0, unit_stages=0, tail_tiles=0,
                 tail_unit_stages=0, l2_prefetch_stages=0, epilogue=EPI_NONE, r: Optional[torch.Tensor] = None,
-                tile_rows=0, stream=None) -> torch.Tensor:
+                tile_rows=0, k_order=0, stream=None) -> torch.Tensor:
     """Y = X @ W.T on the current (or given) stream; returns Y.  With
     epilogue=EPI_SILU_MUL, W is the fused gate+up weight (rows interleaved in
     blocks of 8) and Y is [M, N/2] = silu(gate) * up; with EPI_RESIDUAL,
@@ -217,14 +219,15 @@ def skinny_gemm(x: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = No
         if tuple(r.shape) != (M, N):
             raise ValueError(f"r must be [{M}, {N}]")
     plain = (path, m_tile, order, l2_policy, grid, stage_k, flags, unit_stages, tail_tiles, tail_unit_stages,
-             l2_prefetch_stages, epilogue, tile_rows) == (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0, 0, 0, 0, 0, 0, 0, 0, 0) \
+             l2_prefetch_stages, epilogue, tile_rows, k_order) == (PATH_AUTO, 0, ORDER_AUTO, L2_AUTO, 0, 0, 0, 0, 0, 0, 0,
+                                                                    0, 0, 0) \
         and yf32 is None and workspace is None
     s = _stream_handle(stream)
     if plain:
         _check(lib().skinny_gemm(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, s), "skinny_gemm")
     else:
         o = _opts(path, m_tile, order, l2_policy, grid, yf32, workspace, stage_k, flags, unit_stages, tail_tiles,
-                  tail_unit_stages, l2_prefetch_stages, epilogue, r, tile_rows)
+                  tail_unit_stages, l2_prefetch_stages, epilogue, r, tile_rows, k_order)
         _check(lib().skinny_gemm_ex(x.data_ptr(), w.data_ptr(), y.data_ptr(), M, N, K, ctypes.byref(o), s),
                "skinny_gemm_ex")
     return y
@@ -310,7 +313,7 @@ class Chain:
 
     def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
                  debug_unmet_dependency=False, flags=0, stage_k=0, unit_stages=0, tail_tiles=0,
-                 tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0, kernels=0, tile_rows=0):
+                 tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0, kernels=0, tile_rows=0, k_order=0):
         for i, t in enumerate(tasks):
             _check_operand(f"tasks[{i}].x", t.x)
             _check_operand(f"tasks[{i}].w", t.w)
@@ -326,6 +329,7 @@ class Chain:
         o.counter_groups = counter_groups
         o.kernels = kernels
         o.tile_rows = tile_rows
+        o.k_order = k_order
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

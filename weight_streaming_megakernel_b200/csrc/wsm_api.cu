@@ -183,6 +183,15 @@ int auto_path(int M, long long w_bytes) {
     return WSM_PATH_UMMA;
 }
 
+// K per pipeline stage on the tensor-core path, measured on B200 (the decode
+// shapes, M = 1..64): 256 (4 boxes) everywhere except X tiles of 32 rows,
+// where 256 leaves 2 stages of 80 KB in the ring and 192 (3 boxes) 3 stages of
+// 60 KB, 1-4 % faster; wide tiles carry twice the W per stage, so 128.
+int auto_stage_k(int t_mpad, bool wide) {
+    if (wide) return 128;
+    return t_mpad == 32 ? 192 : 256;
+}
+
 // Wide tiles (tensor-core path): two 128-row halves of W share each X stage,
 // so X is re-read by half as many tiles.  Measured on B200 (the decode shapes
 // at M = 16..64) they are slower at every shape (e.g. gate_up at M = 64:
@@ -210,6 +219,7 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
     if (o->flags & ~(WSM_FLAG_W_READONLY | WSM_FLAG_NO_PDL)) return fail(WSM_ERR_INVALID, "bad flags %#x", o->flags);
     if (o->l2_prefetch_stages < -1)
         return fail(WSM_ERR_INVALID, "bad l2_prefetch_stages %d", o->l2_prefetch_stages);
+    if (o->k_order < 0 || o->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", o->k_order);
     if (path == WSM_PATH_AUTO) path = auto_path(M, 2ll * N * K);
     g = Geo{};
     g.path = path;
@@ -241,11 +251,9 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
             return fail(WSM_ERR_UNSUPPORTED, "tile_rows must be 0, 128 or 256 on the UMMA path (got %d)", o->tile_rows);
         g.wide = (o->tile_rows == 0) ? auto_wide(g.t_mpad) : (o->tile_rows == 2 * kUmmaRows);
         int sk = o->stage_k;
-        // measured best on B200: 256 at every M up to 64 (even where that leaves 2 stages); wide tiles
-        // carry twice the W per stage, so 128
-        if (sk == 0) sk = g.wide ? 128 : 256;
-        if (sk != 64 && sk != 128 && sk != 256)
-            return fail(WSM_ERR_UNSUPPORTED, "stage_k must be 64, 128 or 256 on the UMMA path (got %d)", sk);
+        if (sk == 0) sk = auto_stage_k(g.t_mpad, g.wide);
+        if (sk != 64 && sk != 128 && sk != 192 && sk != 256)
+            return fail(WSM_ERR_UNSUPPORTED, "stage_k must be 64, 128, 192 or 256 on the UMMA path (got %d)", sk);
         const int halves = g.wide ? 2 : 1;
         g.kps = sk / kUmmaBK;
         g.tile_rows = halves * kUmmaRows;
@@ -590,6 +598,7 @@ struct wsm_chain {
     uint32_t dep_target_extra = 0;
     int pdl = 1;
     int prefetch_stages = 0;
+    int k_rotate = 0;
     const void *fn = nullptr;
 };
 
@@ -706,6 +715,7 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     kp.kps = g.kps;
     kp.x_stride = g.x_stride;
     kp.wide = g.wide;
+    kp.k_rotate = (opts->k_order == 2) ? 1 : 0;
     kp.pdl = pdl_mode(opts->flags);
     kp.prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, g.path);
     kp.run_ctl = nullptr;
@@ -876,7 +886,9 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         }
         to.tile_rows = chain_wide ? 2 * kUmmaRows : kUmmaRows;
     }
-    to.stage_k = (path == WSM_PATH_UMMA) ? (opts->stage_k ? opts->stage_k : (chain_wide ? 128 : 256)) : 0;
+    to.stage_k = (path == WSM_PATH_UMMA) ? (opts->stage_k ? opts->stage_k
+                                                           : auto_stage_k((maxM + 15) / 16 * 16, chain_wide))
+                                          : 0;
     const int chain_mmax = (path == WSM_PATH_STREAM) ? pow2ceil(maxM) : 0;
     for (int i = 0; i < n; ++i) {
         if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, d->sms, &to, geos[i], chain_mmax)) != WSM_OK)
@@ -904,6 +916,8 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
             return fail(WSM_ERR_INVALID, "task %d: stage geometry differs from the chain's", i);  // cannot happen
     ch->geo = ring;
     ch->prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, path);
+    if (opts->k_order < 0 || opts->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", opts->k_order);
+    ch->k_rotate = (opts->k_order == 2) ? 1 : 0;
 
     // work units per task, planned for the chain's grid (K-range-first units, no tail, for a task that
     // waits per column)
@@ -1079,6 +1093,7 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     kp.kps = ch->geo.kps;
     kp.x_stride = ch->geo.x_stride;
     kp.wide = ch->geo.wide;
+    kp.k_rotate = ch->k_rotate;
     kp.pdl = ch->pdl;
     kp.prefetch_stages = ch->prefetch_stages;
     kp.run_ctl = ch->d_run_ctl;

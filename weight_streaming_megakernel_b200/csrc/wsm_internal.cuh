@@ -120,6 +120,9 @@ struct KParams {
     int x_stride;                   // UMMA path: bytes between the X boxes of a stage
     int pdl;                        // 0: plain launch; 1: wait for the previous kernel before any
                                     // global access; 2: stream W before that wait, X after it
+    int k_rotate;                   // UMMA path: each unit walks its K stages starting at a tile-dependent
+                                    // offset (wrapping), so CTAs do not all read the same X lines at once
+    int pad2_;
     int wide;                       // UMMA path: tiles of 2 x 128 W rows sharing each X stage (two MMAs into
                                     // two accumulators), so X is re-read half as often; 0: 128-row tiles
     int *status;                    // kStatusWords ints

@@ -388,6 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     const int xy = mt * T.t_m;
                     int next_u = cr.hi - cr.lo - n_static;
                     bool claimed = false;
+                    const int k_len = us.k_end - us.k_begin;
+                    const int k_rot = p.k_rotate ? (us.tile * 5) % k_len : 0;
                     for (int kk = us.k_begin; kk < us.k_end; ++kk) {
                         if (!take_slot()) break;
                         slot_ok = false;
@@ -396,7 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         stage_meta[s][1] = u;
                         stage_meta[s][2] = (kk == us.k_begin ? kMetaFirst : 0) | (kk == us.k_end - 1 ? kMetaLast : 0);
                         mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
-                        const int k0 = kk * p.kps * kUmmaBK;
+                        // the stage this iteration loads (rotated within the unit when k_rotate)
+                        const int kr = k_rot ? us.k_begin + (kk - us.k_begin + k_rot) % k_len : kk;
+                        const int k0 = kr * p.kps * kUmmaBK;
                         for (int h = 0; h < halves; ++h)
                             for (int j = 0; j < p.kps; ++j)
                                 tma_load_2d(st + (h * p.kps + j) * (kUmmaRows * kUmmaBK * 2), &T.tmW, &full_bar[s],
