@@ -177,16 +177,35 @@ class ClockSampler:
 
 def setup_inputs(cases, dev, seed_base=0):
     """Seeded device inputs per GEMM (generated on the device: same recipe,
-    X ~ N(0,1), W ~ N(0,1/K), fp32 rounded to bf16)."""
+    X ~ N(0,1), W ~ N(0,1/K), fp32 rounded to bf16).  The X of all GEMMs are
+    slices of one buffer and so are the Y (each slice 16-byte aligned), so a
+    step's inputs and results move between host and device in one copy each."""
+    def offsets(sizes):
+        out, at = [], 0
+        for n in sizes:
+            out.append(at)
+            at += -(-n // 8) * 8          # 8 bf16 = 16 bytes
+        return out, at
+    xo, xn = offsets([c.M * c.K for c in cases])
+    yo, yn = offsets([c.M * c.N for c in cases])
+    xbuf = torch.empty(xn, dtype=torch.bfloat16, device=dev)
+    ybuf = torch.empty(yn, dtype=torch.bfloat16, device=dev)
     data = []
     for i, c in enumerate(cases):
         g = torch.Generator(device=dev)
         g.manual_seed(seed_base * 100003 + i * 7919 + c.seed)
-        x = torch.randn(c.M, c.K, generator=g, device=dev).to(torch.bfloat16)
+        x = xbuf[xo[i]: xo[i] + c.M * c.K].view(c.M, c.K)
+        x.copy_(torch.randn(c.M, c.K, generator=g, device=dev).to(torch.bfloat16))
         w = (torch.randn(c.N, c.K, generator=g, device=dev) * (1.0 / c.K ** 0.5)).to(torch.bfloat16)
-        y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+        y = ybuf[yo[i]: yo[i] + c.M * c.N].view(c.M, c.N)
         data.append((c, x, w, y))
     return data
+
+
+def packed(data, which):
+    """The one buffer the X (which=1) or Y (which=3) of all GEMMs are slices of."""
+    t = data[0][which]
+    return t.as_strided((t.untyped_storage().nbytes() // 2,), (1,), 0)
 
 
 def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
@@ -344,22 +363,21 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
     # ---- e2e: public API, host buffers, H2D of X and D2H of Y inside the timed region
     e2e = None
     if extras and not args.no_e2e:
-        hx = [x.cpu().pin_memory() for (_, x, _, _) in data]
-        hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for (_, _, _, y) in data]
-        h2d = sum(t.numel() * 2 for t in hx)
-        d2h = sum(t.numel() * 2 for t in hy)
+        # one pinned host buffer per direction; one copy each way per step
+        hx = packed(data, 1).cpu().pin_memory()
+        hy = torch.empty(packed(data, 3).numel(), dtype=torch.bfloat16).pin_memory()
+        h2d = hx.numel() * 2
+        d2h = hy.numel() * 2
 
         def e2e_step(k):
             d = datas[k % copies]
-            for (c, x, w, y), h in zip(d, hx):
-                x.copy_(h, non_blocking=True)
+            packed(d, 1).copy_(hx, non_blocking=True)
             if chain is not None:
                 chains[k % copies].run(s)
             else:
                 for c, x, w, y in d:
                     wsm.skinny_gemm(x, w, y, m_tile=c.m_tile, flags=wsm.FLAG_W_READONLY, stream=s)
-            for (c, x, w, y), h in zip(d, hy):
-                h.copy_(y, non_blocking=True)
+            hy.copy_(packed(d, 3), non_blocking=True)
 
         with torch.cuda.stream(stream):
             for k in range(max(1, args.warmup)):
