@@ -282,6 +282,9 @@ typedef struct {
                                   not need.  Not with dep_cols tasks (WSM_ERR_UNSUPPORTED). */
     int tile_rows;             /* as in wsm_opts; auto: 256 only if auto picks it for every task */
     int k_order;               /* as in wsm_opts */
+    int dep_ring_stages;       /* W stages a CTA streams into its ring ahead of an unmet
+                                  dependency: 0 = auto (2 on the tensor-core path, the whole
+                                  ring on the FMA path), -1 = the whole ring */
     int kernels;               /* WSM_CHAIN_KERNELS_*: hybrid dispatch.  One kernel sizes its
                                   pipeline stages for the chain's widest X tile, which costs
                                   tasks of M <= 32 about 5 % when M > 32 tasks share the chain;

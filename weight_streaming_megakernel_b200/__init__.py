@@ -84,7 +84,7 @@ class _ChainOpts(ctypes.Structure):
                 ("stage_k", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
                 ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int),
                 ("counter_groups", ctypes.c_int), ("tile_rows", ctypes.c_int), ("k_order", ctypes.c_int),
-                ("kernels", ctypes.c_int)]
+                ("dep_ring_stages", ctypes.c_int), ("kernels", ctypes.c_int)]
 
 
 _lib = None
@@ -313,7 +313,8 @@ class Chain:
 
     def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
                  debug_unmet_dependency=False, flags=0, stage_k=0, unit_stages=0, tail_tiles=0,
-                 tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0, kernels=0, tile_rows=0, k_order=0):
+                 tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0, kernels=0, tile_rows=0, k_order=0,
+                 dep_ring_stages=0):
         for i, t in enumerate(tasks):
             _check_operand(f"tasks[{i}].x", t.x)
             _check_operand(f"tasks[{i}].w", t.w)
@@ -330,6 +331,7 @@ class Chain:
         o.kernels = kernels
         o.tile_rows = tile_rows
         o.k_order = k_order
+        o.dep_ring_stages = dep_ring_stages
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

@@ -599,6 +599,7 @@ struct wsm_chain {
     int pdl = 1;
     int prefetch_stages = 0;
     int k_rotate = 0;
+    int dep_ring_stages = 0;
     const void *fn = nullptr;
 };
 
@@ -918,6 +919,12 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     ch->prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, path);
     if (opts->k_order < 0 || opts->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", opts->k_order);
     ch->k_rotate = (opts->k_order == 2) ? 1 : 0;
+    // measured on B200 (36 x 4 dependent chain at M = 16): 2 stages ahead of the dependency instead of
+    // the whole ring (3) is 3 % faster; 1 stage gains less.  The FMA path keeps its whole ring (unmeasured).
+    if (opts->dep_ring_stages < -1)
+        return fail(WSM_ERR_INVALID, "bad dep_ring_stages %d", opts->dep_ring_stages);
+    ch->dep_ring_stages = opts->dep_ring_stages > 0 ? opts->dep_ring_stages
+                          : (opts->dep_ring_stages == 0 && path == WSM_PATH_UMMA) ? 2 : 0;
 
     // work units per task, planned for the chain's grid (K-range-first units, no tail, for a task that
     // waits per column)
@@ -1094,6 +1101,7 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     kp.x_stride = ch->geo.x_stride;
     kp.wide = ch->geo.wide;
     kp.k_rotate = ch->k_rotate;
+    kp.dep_ring_stages = ch->dep_ring_stages;
     kp.pdl = ch->pdl;
     kp.prefetch_stages = ch->prefetch_stages;
     kp.run_ctl = ch->d_run_ctl;

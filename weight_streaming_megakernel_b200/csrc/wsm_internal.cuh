@@ -122,7 +122,8 @@ struct KParams {
                                     // global access; 2: stream W before that wait, X after it
     int k_rotate;                   // UMMA path: each unit walks its K stages starting at a tile-dependent
                                     // offset (wrapping), so CTAs do not all read the same X lines at once
-    int pad2_;
+    int dep_ring_stages;            // W stages a CTA issues into its ring while its task's dependency is
+                                    // unmet (0: the whole ring)
     int wide;                       // UMMA path: tiles of 2 x 128 W rows sharing each X stage (two MMAs into
                                     // two accumulators), so X is re-read half as often; 0: 128-row tiles
     int *status;                    // kStatusWords ints

@@ -348,6 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 // then the pending X loads go out first (every issued stage must be able to complete).
                 auto take_slot = [&]() -> bool {
                     if (slot_ok) return true;
+                    // a dependent task streams at most dep_ring_stages stages of W ahead of its dependency:
+                    // more only queues in front of the round trips that end the previous task
+                    if (np > 0 && T.dep >= 0 && p.dep_ring_stages > 0 && np >= p.dep_ring_stages) flush();
                     if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
                     if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
                         if (np > 0) flush();
