@@ -9,17 +9,22 @@
 // so the wide weight fills the MMA's M = 128 rows and the few X rows its N
 // columns.  D lives in tensor memory (TMEM), fp32.
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0     producer: claims work units (wsm_internal.cuh) and loads, per
 //              stage, kps boxes of W [128 rows x 64 k] and of X with TMA into
 //              a ring of shared-memory stages (128-byte swizzle, mbarrier
 //              completion).  W is read from HBM once per call (L2 evict-first
 //              unless several M-tiles share it); X is evict-last.  In a chain
 //              it issues a task's W loads before the task's dependency is met
-//              and holds back only the X loads.
-//   warp 1     TMEM allocation + the single MMA-issuing thread.
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, bf16 rounding, stores,
-//              split-K partials and the in-order reduction.
+//              (at most dep_ring_stages of them) and holds back only the X
+//              loads.
+//   warp 1     TMEM allocation + the single MMA-issuing thread; four
+//              accumulator buffers, so the MMA runs up to three units ahead
+//              of the epilogue.
+//   warps 2-9  epilogue, two sets of four warps that take alternate units:
+//              tcgen05.ld of the accumulator, the fused epilogue (plain,
+//              residual, SiLU*mul), bf16 rounding, stores, split-K partials
+//              and the in-order reduction.
 //
 // Fleet's per-XCD scheduler workgroup ("Fleet ..." reading notes, section 2)
 // has no counterpart: one atomic counter per task hands out the units, and the
