@@ -283,7 +283,7 @@ typedef struct {
     int tile_rows;             /* as in wsm_opts; auto: 256 only if auto picks it for every task */
     int k_order;               /* as in wsm_opts */
     int dep_ring_stages;       /* W stages a CTA streams into its ring ahead of an unmet
-                                  dependency: 0 = auto (2 on the tensor-core path, the whole
+                                  dependency: 0 = auto (1 on the tensor-core path, the whole
                                   ring on the FMA path), -1 = the whole ring */
     int kernels;               /* WSM_CHAIN_KERNELS_*: hybrid dispatch.  One kernel sizes its
                                   pipeline stages for the chain's widest X tile, which costs
@@ -324,10 +324,14 @@ wsm_status wsm_chain_run(wsm_chain *chain, wsm_stream_t stream);
 wsm_status wsm_chain_status(wsm_chain *chain, wsm_stream_t stream, int *failed_task);
 
 /* Copy the trace of the last run (trace != 0 at create) into host `out`:
- * stamps[cta][task][4] = {first stage issued, dependency met, last tile
- * written (%globaltimer nanoseconds, 0 where the CTA had no work for the
- * task), SM the CTA ran on}.  `capacity` is the number of uint64 slots in
- * `out`; returns the number needed (grid * n_tasks * 4), or 0 when tracing
+ * stamps[cta][task][8] = {first stage issued, dependency met, last unit's
+ * outputs written, SM the CTA ran on, last unit's accumulator handed to the
+ * epilogue, its split-K arrival counted, its in-order reduction done (the
+ * tile's last arriver only), first stage of the task complete at the MMA
+ * issuer} -- %globaltimer nanoseconds except the SM id, 0 where the CTA had
+ * no such event for the task; the tensor-core path records all eight, the
+ * FMA path the first four.  `capacity` is the number of uint64 slots in
+ * `out`; returns the number needed (grid * n_tasks * 8), or 0 when tracing
  * was not enabled.  Synchronises `stream`. */
 size_t wsm_chain_trace(wsm_chain *chain, wsm_stream_t stream, unsigned long long *out,
                        size_t capacity);

@@ -68,6 +68,26 @@ def test_dependent_chain(path, M):
     ch.close()
 
 
+@pytest.mark.parametrize("path,M", [(wsm.PATH_UMMA, 16), (wsm.PATH_UMMA, 48), (wsm.PATH_STREAM, 4)])
+def test_dependent_chain_ahead_of_dependency(path, M):
+    """How far a dependent task streams ahead of its dependency (W stages in
+    the ring, L2 prefetch) changes only timing: every setting gives the same
+    bits, and they pass the oracle."""
+    dims = [1024, 3072, 1024, 2048, 1024]
+    outs = []
+    for ring, pf in ((1, 4), (2, -1), (-1, 8), (0, 0)):
+        x0, ws, ys, yfs, tasks = dependent_chain(M, dims, seed=3)
+        ch = wsm.Chain(tasks, path=path, dep_ring_stages=ring, l2_prefetch_stages=pf)
+        ch.run()
+        assert ch.status()[0] == wsm.WSM_OK, wsm.last_error()
+        ch.close()
+        if not outs:
+            check_dependent(x0, ws, ys, yfs)
+        outs.append(torch.cat([y.view(torch.int16).flatten() for y in ys]))
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+
+
 @pytest.mark.parametrize("path,M", [(wsm.PATH_UMMA, 16), (wsm.PATH_STREAM, 4)])
 def test_dependent_chain_tail_units(path, M):
     """Tail units in every task of a data-dependent chain, run twice (the
@@ -185,10 +205,16 @@ def test_layer_shapes_chain():
         ns = rng.integers(0, task.w.shape[0], 2048)
         check_sampled(task.x, task.w, task.y, task.yf32, ms, ns, what=f"task {t}")
     tr = ch.trace()
-    assert tr is not None and tr.shape[1] == len(tasks)
-    # every task's dependency was met no earlier than its predecessor's first stage
+    assert tr is not None and tr.shape[1] == len(tasks) and tr.shape[2] == 8
     started = tr[:, :, 0]
     assert (started[:, 0] > 0).any()
+    # tensor-core path: every task's first stage reached the MMA issuer and an accumulator the
+    # epilogue; a CTA's stamps of one task come in order
+    for t in range(len(tasks)):
+        assert (tr[:, t, 7] > 0).any() and (tr[:, t, 4] > 0).any()
+        worked = tr[:, t, 2] > 0
+        assert (tr[worked, t, 4] <= tr[worked, t, 2]).all()
+        assert (tr[worked, t, 0] <= tr[worked, t, 2]).all()
     ch.close()
 
 

@@ -346,15 +346,18 @@ class Chain:
         return code, ft.value
 
     def trace(self, stream=None):
-        """Per-CTA, per-task stamps [grid, n_tasks, 4]: first stage issued, dependency met,
-        last tile written (%globaltimer ns), SM id; or None."""
+        """Per-CTA, per-task stamps [grid, n_tasks, 8] (%globaltimer ns, 0 = no such event):
+        first stage issued, dependency met, last unit's outputs written, SM id, last unit's
+        accumulator at the epilogue, its split-K arrival counted, its reduction done (last
+        arriver), first stage complete at the MMA issuer (the last four on the tensor-core
+        path only); or None."""
         n = lib().wsm_chain_trace(self._h, _stream_handle(stream), None, 0)
         if n == 0:
             return None
         buf = (ctypes.c_ulonglong * n)()
         lib().wsm_chain_trace(self._h, _stream_handle(stream), buf, n)
         t = torch.tensor(list(buf), dtype=torch.int64)
-        return t.view(-1, len(self.tasks), 4)
+        return t.view(-1, len(self.tasks), 8)
 
     def close(self):
         if getattr(self, "_h", None) is not None and self._h.value:

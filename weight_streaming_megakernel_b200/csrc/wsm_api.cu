@@ -919,12 +919,13 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     ch->prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, path);
     if (opts->k_order < 0 || opts->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", opts->k_order);
     ch->k_rotate = (opts->k_order == 2) ? 1 : 0;
-    // measured on B200 (36 x 4 dependent chain at M = 16): 2 stages ahead of the dependency instead of
-    // the whole ring (3) is 3 % faster; 1 stage gains less.  The FMA path keeps its whole ring (unmeasured).
+    // measured on B200 (36 x 4 dependent chain at M = 16, 4 prefetch stages): 1 stage ahead of the
+    // dependency is 2 % faster than 2 and 4 % faster than the whole ring (3), and none at all is 2 %
+    // slower than 1.  The FMA path keeps its whole ring (unmeasured).
     if (opts->dep_ring_stages < -1)
         return fail(WSM_ERR_INVALID, "bad dep_ring_stages %d", opts->dep_ring_stages);
     ch->dep_ring_stages = opts->dep_ring_stages > 0 ? opts->dep_ring_stages
-                          : (opts->dep_ring_stages == 0 && path == WSM_PATH_UMMA) ? 2 : 0;
+                          : (opts->dep_ring_stages == 0 && path == WSM_PATH_UMMA) ? 1 : 0;
 
     // work units per task, planned for the chain's grid (K-range-first units, no tail, for a task that
     // waits per column)
@@ -1054,7 +1055,7 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         return cuda_fail(e, "cudaMemcpy(task table)");
     }
     if (opts->trace) {
-        ch->trace_elems = (size_t)ring.grid * n * 4;
+        ch->trace_elems = (size_t)ring.grid * n * kTraceSlots;
         e = cudaMalloc(reinterpret_cast<void **>(&ch->d_trace), ch->trace_elems * 8);
         if (e != cudaSuccess) {
             cleanup();

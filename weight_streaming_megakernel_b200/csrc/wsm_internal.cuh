@@ -41,6 +41,11 @@ constexpr int kStatusWords = 4;    // [0] error code, [1] failing task, [2] fail
 constexpr int kSchedWords = 2;     // per task: [0] next unit to claim, [1] CTAs done claiming
 constexpr int kClaimLead = 4;      // a CTA claims its next unit this many stages before its unit ends
 constexpr int kColChunk = 256;     // output columns per readiness chunk (per-column data dependencies)
+// Trace stamps per CTA and task (%globaltimer ns unless noted): [0] first stage issued, [1] dependency
+// met, [2] last unit's outputs written, [3] SM id, [4] last unit's accumulator at the epilogue, [5] its
+// split-K arrival counted, [6] its in-order reduction done (last arriver only), [7] first stage of the
+// task complete at the MMA issuer.
+constexpr int kTraceSlots = 8;
 
 // Epilogues (== WSM_EPI_*).
 enum : int { kEpiNone = 0, kEpiSiluMul = 1, kEpiResidual = 2 };
@@ -129,7 +134,7 @@ struct KParams {
     int *status;                    // kStatusWords ints
     unsigned long long dep_timeout_ns;
     unsigned long long wait_timeout_ns;
-    unsigned long long *trace;      // [grid][n_tasks][4] or nullptr
+    unsigned long long *trace;      // [grid][n_tasks][kTraceSlots] or nullptr
 };
 
 #if defined(__CUDACC__)
@@ -623,10 +628,9 @@ __device__ __forceinline__ void chain_run_done(const KParams &p) {
     }
 }
 
-// Trace stamps: [cta][task][4] = {first stage issued, dependency met, last
-// tile written, SM id}.
+// Trace stamps: [cta][task][kTraceSlots], the slots listed at kTraceSlots.
 __device__ __forceinline__ void trace_stamp(const KParams &p, int task, int slot, unsigned long long v) {
-    if (p.trace) p.trace[((size_t)blockIdx.x * p.n_tasks + task) * 4 + slot] = v;
+    if (p.trace) p.trace[((size_t)blockIdx.x * p.n_tasks + task) * kTraceSlots + slot] = v;
 }
 
 #endif  // __CUDACC__

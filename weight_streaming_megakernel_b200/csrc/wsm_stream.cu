@@ -118,14 +118,14 @@ struct LaneReduce {
 }  // namespace
 
 // L2 prefetch of the W of the units this CTA would own in a round-robin (c,
-// c + G, ...), p.prefetch_stages stages at most, skipping the first S stages
-// of each first-round unit (some CTA's ring holds them).  Out of line: it runs
-// at most once per task.
-static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDev &T, int S, int KW, int TN) {
+// c + G, ...), p.prefetch_stages stages at most, skipping the first `skip`
+// stages of each first-round unit (its claimer's ring already holds them).
+// Out of line: it runs at most once per task.
+static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDev &T, int skip, int KW, int TN) {
     int budget = p.prefetch_stages;
     for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
         const UnitSpan ps = unit_span(T, uu);
-        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? S : 0); kk < ps.k_end && budget > 0; ++kk, --budget)
+        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? skip : 0); kk < ps.k_end && budget > 0; ++kk, --budget)
             for (int kw = 0; kw < KW; ++kw)
                 tma_prefetch_l2_2d(&T.tmW, kk * (KW * kStreamBoxK) + kw * kStreamBoxK, ps.tile * TN);
     }
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 auto prefetch_l2 = [&]() {
                     if (prefetched) return;
                     prefetched = true;
-                    prefetch_w_l2(p, T, S, KW, TN);
+                    prefetch_w_l2(p, T, (T.dep >= 0 && p.dep_ring_stages > 0) ? min(S, p.dep_ring_stages) : S, KW, TN);
                 };
                 auto flush = [&]() {
                     if (!grid_dep_ok) {

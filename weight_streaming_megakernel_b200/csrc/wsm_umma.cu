@@ -217,17 +217,17 @@ __device__ __forceinline__ void reduce_row_partials(const UnitOut &uo, const Uni
 }  // namespace
 
 // L2 prefetch of the W of the units this CTA would own in a round-robin (c,
-// c + G, ...), p.prefetch_stages stages at most, skipping the first S stages
-// of each first-round unit (some CTA's ring holds them).  Out of line: it runs
-// at most once per task.
-static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDev &T, int S) {
+// c + G, ...), p.prefetch_stages stages at most, skipping the first `skip`
+// stages of each first-round unit (its claimer's ring already holds them).
+// Out of line: it runs at most once per task.
+static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDev &T, int skip) {
     int budget = p.prefetch_stages;
     for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
         const UnitSpan ps = unit_span(T, uu);
         int pg, pmt;
         tile_coords(T, ps.tile, pg, pmt);
         const int halves = p.wide ? 2 : 1;
-        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? S : 0); kk < ps.k_end && budget > 0; ++kk, --budget)
+        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? skip : 0); kk < ps.k_end && budget > 0; ++kk, --budget)
             for (int h = 0; h < halves; ++h)
                 for (int j = 0; j < p.kps; ++j)
                     tma_prefetch_l2_2d(&T.tmW, (kk * p.kps + j) * kUmmaBK, (pg * halves + h) * kUmmaRows);
@@ -322,7 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 auto prefetch_l2 = [&]() {
                     if (prefetched) return;
                     prefetched = true;
-                    prefetch_w_l2(p, T, S);
+                    // the first-round units' first stages sit in their claimers' rings: the whole ring
+                    // ahead of the grid dependency, dep_ring_stages ahead of a task dependency
+                    prefetch_w_l2(p, T, (T.dep >= 0 && p.dep_ring_stages > 0) ? min(S, p.dep_ring_stages) : S);
                 };
                 auto flush = [&]() {
                     if (!grid_dep_ok) {
@@ -475,6 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             uint32_t acc_i = 0;   // accumulators handed to the epilogue so far
             bool any_mma = false;
             int buf = 0;
+            int traced_t = -1;
             for (;;) {
                 if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag, wlim, p.status, -1, kSiteFull)) break;
                 tc_fence_after();
@@ -503,6 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                                            t, kSiteAcc))
                         break;
                     tc_fence_after();
+                    if (p.trace && t != traced_t) {
+                        trace_stamp(p, t, 7, globaltimer());
+                        traced_t = t;
+                    }
                 }
                 const TaskDev &T = task_at(p, t);
                 const uint32_t st0 = smem_u32(ring + (size_t)s * p.stage_bytes);
@@ -562,6 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             if (vote_or(ab || (flags & kMetaDone), 1 + set, kEpiThreads)) break;
             const int t = acc_meta[buf][0];
             const int u = acc_meta[buf][1];
+            if (leader) trace_stamp(p, t, 4, globaltimer());
             const TaskDev &T = task_at(p, t);
             const UnitSpan us = unit_span(T, u);
             const int tile = us.tile;
@@ -617,6 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     // others' for the last arriver
                     const unsigned int old = atom_add_acqrel_gpu(&uo.tile_cnt[tile], 1u);
                     last_flag[set] = (old == (unsigned int)(us.nu - 1)) ? 1 : 0;
+                    trace_stamp(p, t, 5, globaltimer());
                 }
                 epi_bar(set);
                 if (last_flag[set]) {
@@ -631,6 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     }
                     epi_bar(set);
                     if (leader) {
+                        trace_stamp(p, t, 6, globaltimer());
                         uo.tile_cnt[tile] = 0u;  // ready for the next call
                         tile_finished(uo, g, halves * kUmmaRows, run_no);
                     }
