@@ -348,6 +348,17 @@ __device__ __forceinline__ const TaskDev &task_at(const KParams &p, int t) {
     return p.tasks ? p.tasks[t] : p.single;
 }
 
+// Warm this SM's L1 with the part of task t's descriptor past its tensor maps
+// (the fields the epilogue reads), so a CTA's first unit of a task does not
+// wait on loaded L2 round trips for them.  Chains only: a single GEMM's
+// descriptor is a kernel parameter.
+__device__ __forceinline__ void prefetch_task_l1(const KParams &p, int t) {
+    if (!p.tasks || t >= p.n_tasks) return;
+    const char *b = reinterpret_cast<const char *>(p.tasks + t);
+    for (size_t off = 2 * sizeof(CUtensorMap); off < sizeof(TaskDev); off += 128)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(b + off));
+}
+
 // Tile index -> (column tile g, M-tile mt).
 __device__ __forceinline__ void tile_coords(const TaskDev &T, int tile, int &g, int &mt) {
     if (T.order == 0) {

@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     __shared__ __align__(8) uint64_t accf_bar[kAccBufs];
     __shared__ __align__(8) uint64_t acce_bar[kAccBufs];
     __shared__ __align__(8) uint64_t drain_bar;
-    __shared__ int stage_meta[kMaxStages][3];   // {task, unit, flags}, written by the producer
+    __shared__ int stage_meta[kMaxStages][4];   // {task, unit, flags, MMA instruction descriptor}, by the producer
     __shared__ int acc_meta[kAccBufs][3];       // {task, unit, flags}, written by the MMA thread
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_flag;
@@ -407,6 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         stage_meta[s][0] = t;
                         stage_meta[s][1] = u;
                         stage_meta[s][2] = (kk == us.k_begin ? kMetaFirst : 0) | (kk == us.k_end - 1 ? kMetaLast : 0);
+                        stage_meta[s][3] = (int)T.idesc;  // the MMA thread reads no task table
                         mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
                         // the stage this iteration loads (rotated within the unit when k_rotate)
                         const int kr = k_rot ? us.k_begin + (kk - us.k_begin + k_rot) % k_len : kk;
@@ -511,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         traced_t = t;
                     }
                 }
-                const TaskDev &T = task_at(p, t);
+                const uint32_t idesc = (uint32_t)stage_meta[s][3];
                 const uint32_t st0 = smem_u32(ring + (size_t)s * p.stage_bytes);
                 for (int h = 0; h < halves; ++h) {
                     // half h of the tile's W rows accumulates into columns h * 64 .. of the buffer
@@ -522,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
 #pragma unroll
                         for (int k = 0; k < kUmmaBK / 16; ++k) {
                             // advancing K by 16 bf16 = 32 bytes inside the swizzle atom
-                            tc_mma(d_tmem, sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k), T.idesc,
+                            tc_mma(d_tmem, sw128_desc(a0 + 32u * k), sw128_desc(b0 + 32u * k), idesc,
                                    ((flags & kMetaFirst) && j == 0 && k == 0) ? 0u : 1u);
                         }
                     }
@@ -559,16 +560,19 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         const bool leader = (etid == 0);
         if (p.pdl) pdl_wait();                  // Y and the scratch may still be in use by the previous kernel
         const unsigned int run_no = p.run_ctl ? ld_acquire_gpu(&p.run_ctl[0]) + 1u : 0u;  // this chain run
+        int warm_t = 0;                         // the task whose descriptor the set warms while it waits
         for (uint32_t k = 0;; ++k) {
             const uint32_t acc_i = kEpiSets * k + (uint32_t)set;
             const int buf = (int)(acc_i % kAccBufs);
             const uint32_t aph = (acc_i / kAccBufs) & 1;
+            if (leader) prefetch_task_l1(p, warm_t);
             const bool ab = !mbar_wait_bounded(&accf_bar[buf], aph, &abort_flag, wlim, p.status, -1, kSiteAcc);
             // the four warps of the set stop together (an abort anywhere, or the end marker)
             const int flags = ab ? kMetaDone : acc_meta[buf][2];
             if (vote_or(ab || (flags & kMetaDone), 1 + set, kEpiThreads)) break;
             const int t = acc_meta[buf][0];
             const int u = acc_meta[buf][1];
+            warm_t = t + 1;
             if (leader) trace_stamp(p, t, 4, globaltimer());
             const TaskDev &T = task_at(p, t);
             const UnitSpan us = unit_span(T, u);
