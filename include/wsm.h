@@ -323,6 +323,14 @@ wsm_status wsm_chain_run(wsm_chain *chain, wsm_stream_t stream);
  * whose wait ran out (may be NULL). */
 wsm_status wsm_chain_status(wsm_chain *chain, wsm_stream_t stream, int *failed_task);
 
+/* The plan of task `task` of a prepared chain (the chain's grid, ring and
+ * work units; workspace_bytes is 0: the chain owns its scratch).  A chain
+ * sizes each task's automatic work units for the work that can overlap them:
+ * tasks followed, before the next dependency wait, by much more work get
+ * longer units (whole tiles when there is enough), the rest the single-call
+ * choice.  WSM_ERR_INVALID for a null chain or a task out of range. */
+wsm_status wsm_chain_task_plan(wsm_chain *chain, int task, wsm_plan_info *out);
+
 /* Copy the trace of the last run (trace != 0 at create) into host `out`:
  * stamps[cta][task][8] = {first stage issued, dependency met, last unit's
  * outputs written, SM the CTA ran on, last unit's accumulator handed to the

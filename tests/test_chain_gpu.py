@@ -88,6 +88,45 @@ def test_dependent_chain_ahead_of_dependency(path, M):
         assert torch.equal(o, outs[0])
 
 
+@pytest.mark.parametrize("deps", [False, True])
+def test_chain_units_grow_with_overlapping_work(deps):
+    """Independent tasks followed by much more work take longer units (whole
+    tiles when there is enough); the last task, with nothing after it, and
+    tasks that wait on a dependency keep the single-call choice; an explicit
+    unit_stages applies to every task.  Results pass the oracle either way."""
+    shapes = [(16, 24576, 4096)] * 4 + [(16, 4096, 12288)]
+    tasks = []
+    for i, (M, N, K) in enumerate(shapes):
+        x, w = synth.make_xw(M, N, K, seed=40 + i)
+        tasks.append(wsm.Task(x.to(DEV), w.to(DEV), torch.empty(M, N, dtype=torch.bfloat16, device=DEV),
+                              dep=(i - 1) if deps else -1, yf32=torch.empty(M, N, dtype=torch.float32, device=DEV)))
+    single = [wsm.plan(M, N, K) for M, N, K in shapes]
+    ch = wsm.Chain(tasks)
+    plans = [ch.task_plan(i) for i in range(len(tasks))]
+    if deps:
+        assert [p["unit_stages"] for p in plans] == [p["unit_stages"] for p in single]
+    else:
+        # later work: 3 gate_up + down = 10752 stages over 2 x 148 CTAs -> whole tiles; 4608 -> 2 units
+        assert plans[0]["unit_stages"] == plans[0]["k_iters"] == 16
+        assert plans[2]["unit_stages"] == 8
+        assert plans[3]["unit_stages"] == single[3]["unit_stages"]
+        assert plans[4]["unit_stages"] == single[4]["unit_stages"]
+    assert all(p["grid"] == plans[0]["grid"] for p in plans)
+    ch.run()
+    assert ch.status()[0] == wsm.WSM_OK, wsm.last_error()
+    rng = np.random.default_rng(2)
+    for i, t in enumerate(tasks):
+        ms = rng.integers(0, t.x.shape[0], 1024)
+        ns = rng.integers(0, t.w.shape[0], 1024)
+        check_sampled(t.x, t.w, t.y, t.yf32, ms, ns, what=f"task {i}")
+    with pytest.raises(wsm.WsmError):
+        ch.task_plan(len(tasks))
+    ch.close()
+    ch = wsm.Chain(tasks, unit_stages=2)
+    assert all(ch.task_plan(i)["unit_stages"] == 2 for i in range(len(tasks)))
+    ch.close()
+
+
 @pytest.mark.parametrize("path,M", [(wsm.PATH_UMMA, 16), (wsm.PATH_STREAM, 4)])
 def test_dependent_chain_tail_units(path, M):
     """Tail units in every task of a data-dependent chain, run twice (the

@@ -41,7 +41,8 @@ CHAIN_KERNELS_AUTO, CHAIN_KERNELS_ONE, CHAIN_KERNELS_SPLIT = 0, 1, 2
 # Every function include/wsm.h declares (checked by the CPU tests).
 HEADER_SYMBOLS = (
     "skinny_gemm", "skinny_gemm_ex", "wsm_plan", "wsm_workspace_bytes", "wsm_stream_status", "skinny_gemm_noalloc",
-    "wsm_chain_create", "wsm_chain_run", "wsm_chain_status", "wsm_chain_trace", "wsm_chain_destroy",
+    "wsm_chain_create", "wsm_chain_run", "wsm_chain_status", "wsm_chain_task_plan", "wsm_chain_trace",
+    "wsm_chain_destroy",
     "gemm_chain", "wsm_chain_validate", "wsm_last_error", "wsm_abi_version",
 )
 
@@ -111,6 +112,8 @@ def lib() -> ctypes.CDLL:
         L.wsm_workspace_bytes.restype = ctypes.c_size_t
         L.wsm_stream_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
         L.wsm_stream_status.restype = st
+        L.wsm_chain_task_plan.argtypes = [vp, i, ctypes.POINTER(_PlanInfo)]
+        L.wsm_chain_task_plan.restype = st
         L.wsm_chain_create.argtypes = [ctypes.POINTER(_Task), i, ctypes.POINTER(_ChainOpts), ctypes.POINTER(vp)]
         L.wsm_chain_create.restype = st
         L.wsm_chain_run.argtypes = [vp, vp]
@@ -344,6 +347,12 @@ class Chain:
         ft = ctypes.c_int(-1)
         code = lib().wsm_chain_status(self._h, _stream_handle(stream), ctypes.byref(ft))
         return code, ft.value
+
+    def task_plan(self, task: int) -> dict:
+        """The plan of one task of the chain (as `plan` reports for a single call)."""
+        info = _PlanInfo()
+        _check(lib().wsm_chain_task_plan(self._h, task, ctypes.byref(info)), "wsm_chain_task_plan")
+        return {f: getattr(info, f) for f, _ in _PlanInfo._fields_}
 
     def trace(self, stream=None):
         """Per-CTA, per-task stamps [grid, n_tasks, 8] (%globaltimer ns, 0 = no such event):
