@@ -153,18 +153,22 @@ int auto_units_per_tile(const Geo &g, int ctas) {
 // chain's tasks back to back -- a CTA that finds no unit left in a task claims
 // from the next one -- so a task's units delay the kernel only where no later
 // work can fill in: at the next task that waits on a dependency, or at the end
-// of the kernel.  With `later` stages of work before that point, a unit of up
-// to later / (2 G) stages still ends before the CTAs run out of work (2: SMs
-// stream at different rates), and longer units mean fewer split-K partials and
-// reductions.  Measured on B200 (24 independent tasks of one shape, whole
-// tiles against the single-launch choice): gate_up at M = 16 30.8 us per task
-// against 33.5, qkv 8.8 against 9.1, o 6.5 against 7.0; at M = 64 qkv 10.0
-// against 12.3, o 7.5 against 9.8.  Never fewer stages per unit than the
+// of the kernel.  With `later` stages of work before that point, units of up
+// to later / G stages (X tiles <= 32 rows) or 2 later / G (larger X tiles,
+// whose partials cost 4x more per unit) keep the kernel's end short while
+// cutting split-K partials and reductions.  Measured on B200 (24 independent
+// tasks of one shape, whole tiles against the single-launch choice): gate_up
+// at M = 16 30.8 us per task against 33.5, qkv 8.8 against 9.1, o 6.5 against
+// 7.0; at M = 64 qkv 10.0 against 12.3, o 7.5 against 9.8.  The limit, swept
+// on the default decode step and the L2-reuse set (later / (d G) for d = 1..4
+// and m later / G for m = 1, 2, 4): later / G is best on the first (6.33 TB/s
+// against 6.23-6.28 for the others), 2 later / G on the second (5.54-5.65
+// against 5.31-5.37 at later / G).  Never fewer stages per unit than the
 // single-launch choice; K split evenly between a tile's units.
 int chain_unit_stages(const Geo &g, int ctas, long long later) {
     const int nu0 = auto_units_per_tile(g, ctas);
     const int ku0 = (g.kb + nu0 - 1) / nu0;
-    const long long cap = later / (2LL * std::max(1, ctas));
+    const long long cap = later * (g.t_mpad <= 32 ? 1 : 2) / std::max(1, ctas);
     if (cap <= ku0) return ku0;
     const int nu = (int)std::max<long long>(1, (g.kb + cap - 1) / cap);
     return std::max(ku0, (g.kb + nu - 1) / nu);
