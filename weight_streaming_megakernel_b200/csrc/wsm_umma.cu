@@ -159,12 +159,17 @@ __device__ __forceinline__ void emit_outputs(const EpiOut &e, int n, int m0, int
         return;
     }
     if (n >= e.N) return;
-    const bool res = e.epi == kEpiResidual;
+    // residual: all of the thread's R loads go out before its first store (Y may alias R as far as
+    // the compiler knows, so loads interleaved with the stores would each wait a round trip)
+    float r[MB];
+#pragma unroll
+    for (int i = 0; i < MB; ++i)
+        r[i] = (e.epi == kEpiResidual && i < cnt) ? __bfloat162float(e.R[(size_t)(m0 + i) * e.N + n]) : 0.f;
 #pragma unroll
     for (int i = 0; i < MB; ++i) {
         if (i >= cnt) break;
         const size_t o = (size_t)(m0 + i) * e.N + n;
-        const float y = res ? v[i] + __bfloat162float(e.R[o]) : v[i];
+        const float y = e.epi == kEpiResidual ? v[i] + r[i] : v[i];
         e.Y[o] = __float2bfloat16_rn(y);
         if (e.Yf32) e.Yf32[o] = y;
     }
