@@ -387,3 +387,35 @@ def test_dependent_chain_graph_replays(path, M):
         check_dependent(x0, ws, ys, yfs)
     del g
     ch.close()
+
+
+@pytest.mark.parametrize("config", ["qwen3_decode", "skinny", "l2_reuse"])
+def test_benchmark_chain_full_size_sampled(config):
+    """The chain bench.py times for a workload -- every GEMM of the step as an
+    independent task of one kernel, full sizes, the weights flagged read-only
+    -- checked on sampled outputs of every task, including the ragged end of
+    N.  Its tasks run with chain-position work units (longer than the same
+    GEMM alone), which this covers at the sizes that use them."""
+    cases = getattr(synth, f"config_{config}")()
+    tasks = []
+    for c in cases:
+        g = torch.Generator(device=DEV)
+        g.manual_seed(1000 + c.seed + c.M * 7 + c.N)
+        x = torch.randn(c.M, c.K, generator=g, device=DEV).to(torch.bfloat16)
+        w = (torch.randn(c.N, c.K, generator=g, device=DEV) / c.K ** 0.5).to(torch.bfloat16)
+        tasks.append(wsm.Task(x, w, torch.empty(c.M, c.N, dtype=torch.bfloat16, device=DEV),
+                              yf32=torch.empty(c.M, c.N, dtype=torch.float32, device=DEV)))
+    ch = wsm.Chain(tasks, flags=wsm.FLAG_W_READONLY)
+    plans = [ch.task_plan(i) for i in range(len(tasks))]
+    for _ in range(2):  # the second run reuses the counters and partial slots of the first
+        ch.run()
+    assert ch.status()[0] == wsm.WSM_OK, wsm.last_error()
+    rng = np.random.default_rng(5)
+    for c, t, p in zip(cases, tasks, plans):
+        ms = rng.integers(0, c.M, 1024)
+        ns = rng.integers(0, c.N, 1024)
+        ns[:32] = np.arange(c.N - 32, c.N)
+        check_sampled(t.x, t.w, t.y, t.yf32, ms, ns, what=f"{c.name} (unit_stages {p['unit_stages']})")
+    ch.close()
+    del tasks
+    torch.cuda.empty_cache()
