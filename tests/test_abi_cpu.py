@@ -134,9 +134,12 @@ def test_auto_units_per_tile():
     assert nu(16, 18432, 7168) == 1         # 144 tiles: one unit per CTA
     assert nu(16, 10240, 8192) == 3         # 80 tiles: 240 units
     assert nu(16, 57344, 8192) == 4         # 448 tiles: many rounds, small tail
-    assert nu(64, 24576, 4096) == 1         # 192 tiles at M = 64
+    assert nu(64, 24576, 4096) == 2         # 192 tiles at M = 64: three rounds of 8 stages
     assert nu(64, 57344, 8192) == 2
     assert nu(16, 6144, 4096) == 3
+    assert nu(16, 24576, 4096) == 2         # 192 tiles: 384 units in three whole rounds (measured
+    assert nu(8, 24576, 4096) == 2          # 40.0 us against 42.7 with 4 units per tile)
+    assert nu(32, 24576, 4096) == 2
 
 
 def test_plan_units():

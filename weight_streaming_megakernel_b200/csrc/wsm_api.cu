@@ -120,8 +120,10 @@ void stream_geo(int mmax, Geo &g) {
 // counter round trip and a share of the in-order reduction; and the last
 // units of a GEMM decide when it ends, with SMs that stream up to ~2x slower
 // than others.  Tensor-core path: nu in 1..4 minimising a cost in stages,
-// fitted to measured B200 times of the decode shapes (M = 8, 16, 64):
-//   units <= 2 x CTAs:  ceil(units / CTAs) x (ku + c)           (whole rounds)
+// fitted to measured B200 times of the decode shapes (9 shapes at M = 8, 16,
+// 32, 64; back-to-back launches; mean 1.5 % above the best split, 2.0 % with
+// a threshold of 2 x CTAs, which cost gate_up 5-9 % at M = 8..32):
+//   units <= 3 x CTAs:  ceil(units / CTAs) x (ku + c)           (whole rounds)
 //   otherwise:          units / CTAs x (ku + c) + 2 x ku        (dynamic claims
 //                                                   smooth the rounds; a tail of
 //                                                   about two units remains)
@@ -140,7 +142,7 @@ int auto_units_per_tile(const Geo &g, int ctas) {
     for (int nu = 1; nu <= std::min(4, g.kb); ++nu) {
         const int ku = (g.kb + nu - 1) / nu;
         const double units = (double)g.tiles() * ((g.kb + ku - 1) / ku);
-        const double cost = units <= 2 * G ? std::ceil(units / G) * (ku + c) : units / G * (ku + c) + 2.0 * ku;
+        const double cost = units <= 3 * G ? std::ceil(units / G) * (ku + c) : units / G * (ku + c) + 2.0 * ku;
         if (cost < best_cost - 1e-9) {
             best_cost = cost;
             best = nu;
