@@ -320,6 +320,15 @@ def test_mixed_m_chain(deps, kernels):
         for t in tasks:
             check_full(t.x.cpu(), t.w.cpu(), t.y, t.yf32)
     assert (ch.trace() is not None) == one   # split chains keep no trace
+    # each task's plan, from whichever kernel runs it: one kernel sizes every X tile's stages for
+    # the widest (64 rows: 2 stages of 96 KB); split, the M <= 32 kernels keep their own ring
+    plans = [ch.task_plan(i) for i in range(len(tasks))]
+    for t, p in zip(tasks, plans):
+        M = t.x.shape[0]
+        assert p["m_tile"] >= M and p["m_tile"] % 16 == 0 and p["path"] == wsm.PATH_UMMA
+        assert p["n_tiles"] == -(-t.w.shape[0] // 128) and p["k_iters"] * p["tile_k"] >= t.x.shape[1]
+    narrow = [p["stages"] for t, p in zip(tasks, plans) if t.x.shape[0] <= 16]
+    assert all(n == (2 if one else 3) for n in narrow), narrow
     ch.close()
 
 
