@@ -59,9 +59,9 @@ typedef enum {
     WSM_ERR_TIMEOUT = 6      /* a bounded device-side wait ran out (chain dependency or pipeline) */
 } wsm_status;
 
-/* Kernel path.  AUTO takes the FMA path for M = 1 up to 128 MiB of weights,
- * M = 2 up to 96 MiB and M <= 4 up to 64 MiB (measured crossovers on B200),
- * the tensor-core path otherwise. */
+/* Kernel path.  AUTO takes the FMA path for M <= 2 at any size and for
+ * M <= 4 up to 64 MiB of weights (measured crossovers on B200), the
+ * tensor-core path otherwise. */
 enum {
     WSM_PATH_AUTO = 0,
     WSM_PATH_STREAM = 1, /* fp32 FMA dot products + warp-shuffle reduction, M <= 8 */
@@ -141,9 +141,11 @@ typedef struct {
     int l2_prefetch_stages; /* W pipeline stages per CTA prefetched into L2 while the
                                CTA waits for the previous kernel (WSM_FLAG_W_READONLY):
                                0 = auto, -1 = none */
-    int tile_rows;   /* tensor-core path: W rows per tile, 0 = auto, 128, or 256 (two
+    int tile_rows;   /* W rows per tile, 0 = auto.  Tensor-core path: 128, or 256 (two
                         128-row halves share each X stage and accumulate into two
-                        TMEM accumulators, so X is re-read half as often) */
+                        TMEM accumulators, so X is re-read half as often).  FMA
+                        path: 16 or 32 (32: larger TMA boxes, a faster stream per
+                        SM; auto takes 32 unless it leaves fewer tiles than CTAs) */
     int k_order;     /* tensor-core path: order of a work unit's K stages: 0 = auto,
                         1 = increasing, 2 = rotated by a tile-dependent offset (so the
                         CTAs do not all read the same lines of X at the same time) */
@@ -280,7 +282,9 @@ typedef struct {
                                   bumps the task's counter once.  An ablation: the pages use
                                   it to save cross-die fences, which B200's coherent L2 does
                                   not need.  Not with dep_cols tasks (WSM_ERR_UNSUPPORTED). */
-    int tile_rows;             /* as in wsm_opts; auto: 256 only if auto picks it for every task */
+    int tile_rows;             /* as in wsm_opts, one value for every task; auto: tensor-core
+                                  path 256 only if auto picks it for every task, FMA path the
+                                  height with the lower modelled time over the tasks */
     int k_order;               /* as in wsm_opts */
     int dep_ring_stages;       /* W stages a CTA streams into its ring ahead of an unmet
                                   dependency: 0 = auto (1 on the tensor-core path, the whole

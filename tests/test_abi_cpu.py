@@ -68,22 +68,43 @@ def test_plan_paths_and_geometry():
 
 
 def test_auto_path_crossovers():
-    """AUTO: FMA path for M = 1 up to 128 MiB of weights, M = 2 up to 96 MiB,
-    M <= 4 up to 64 MiB; tensor cores otherwise."""
+    """AUTO: FMA path for M <= 2 at any size, M <= 4 up to 64 MiB of weights;
+    tensor cores otherwise."""
     S, U = wsm.PATH_STREAM, wsm.PATH_UMMA
-    cases = [(1, 4096, 4096, S), (1, 4096, 12288, S), (1, 10240, 8192, U), (1, 24576, 4096, U), (1, 57344, 8192, U),
-             (2, 4096, 12288, S), (2, 10240, 8192, U), (2, 24576, 4096, U), (4, 4096, 4096, S),
+    cases = [(1, 4096, 4096, S), (1, 4096, 12288, S), (1, 10240, 8192, S), (1, 24576, 4096, S), (1, 57344, 8192, S),
+             (2, 4096, 12288, S), (2, 10240, 8192, S), (2, 24576, 4096, S), (4, 4096, 4096, S),
              (4, 4096, 7168, S), (4, 4096, 12288, U), (3, 6144, 4096, S), (5, 64, 64, U), (8, 4096, 4096, U),
-             (16, 64, 64, U)]
+             (16, 64, 64, U), (3, 24576, 4096, U)]
     for M, N, K, want in cases:
         assert wsm.plan(M, N, K)["path"] == want, (M, N, K)
-    # exactly at the thresholds
-    assert wsm.plan(1, 8192, 8192)["path"] == S           # 128 MiB
-    assert wsm.plan(1, 8193, 8192)["path"] == U
-    assert wsm.plan(2, 6144, 8192)["path"] == S           # 96 MiB
-    assert wsm.plan(2, 6145, 8192)["path"] == U
+    # exactly at the threshold for M = 3, 4
     assert wsm.plan(4, 4096, 8192)["path"] == S           # 64 MiB
     assert wsm.plan(4, 4097, 8192)["path"] == U
+    assert wsm.plan(3, 4097, 8192)["path"] == U
+
+
+def test_fma_tile_rows():
+    """FMA path tile height: 32 rows (16 KB boxes, the faster stream per SM)
+    unless that leaves fewer tiles than CTAs while 16-row tiles do not (the K
+    split would then cost more); an explicit tile_rows of 16 or 32 is taken
+    as given, anything else refused on this path."""
+    def rows(M, N, K, **kw):
+        p = wsm.plan(M, N, K, num_sms=148, path=wsm.PATH_STREAM, **kw)
+        assert p["tile_k"] == (1024 if p["tile_rows"] == 16 else 512)
+        return p["tile_rows"]
+    assert rows(1, 4096, 4096) == 16          # o: 128 tiles of 32 rows < 148, 256 of 16
+    assert rows(1, 4096, 7168) == 16
+    assert rows(1, 6144, 4096) == 32          # qkv: 192 tiles of 32 rows
+    assert rows(1, 24576, 4096) == 32         # gate_up
+    assert rows(1, 4096, 12288) == 32         # down: split either way, 32 streams faster
+    assert rows(1, 2112, 7168) == 32          # 66 or 132 tiles: both split
+    assert rows(2, 57344, 8192) == 32
+    assert rows(1, 4096, 4096, tile_rows=32) == 32
+    assert rows(1, 24576, 4096, tile_rows=16) == 16
+    with pytest.raises(wsm.WsmError):
+        wsm.plan(1, 4096, 4096, path=wsm.PATH_STREAM, tile_rows=128)
+    with pytest.raises(wsm.WsmError):
+        wsm.plan(16, 4096, 4096, path=wsm.PATH_UMMA, tile_rows=32)
 
 
 def test_plan_ring_fits_shared_memory():

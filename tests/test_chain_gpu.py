@@ -129,6 +129,24 @@ def test_chain_units_grow_with_overlapping_work(deps):
     ch.close()
 
 
+@pytest.mark.parametrize("rows,M", [(0, 1), (0, 2), (16, 2), (32, 4), (32, 8)])
+def test_dependent_chain_fma_tile_rows(rows, M):
+    """FMA-path chains on either tile height (automatic: one height for the
+    whole chain), twice (counters reset per run)."""
+    dims = [1024, 2048, 1032, 3072, 520, 4096, 1024]
+    x0, ws, ys, yfs, tasks = dependent_chain(M, dims, seed=60 + M + rows)
+    ch = wsm.Chain(tasks, path=wsm.PATH_STREAM, tile_rows=rows)
+    heights = {ch.task_plan(i)["tile_rows"] for i in range(len(tasks))}
+    assert heights == {rows} if rows else len(heights) == 1 and heights <= {16, 32}
+    for _ in range(2):
+        for y in ys:
+            y.fill_(float("nan"))
+        ch.run()
+        assert ch.status()[0] == wsm.WSM_OK, wsm.last_error()
+        check_dependent(x0, ws, ys, yfs)
+    ch.close()
+
+
 @pytest.mark.parametrize("path,M", [(wsm.PATH_UMMA, 16), (wsm.PATH_STREAM, 4)])
 def test_dependent_chain_tail_units(path, M):
     """Tail units in every task of a data-dependent chain, run twice (the

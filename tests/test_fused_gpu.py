@@ -71,6 +71,20 @@ def test_silu_mul(M, N, K):
             check_silu(x, w, h, hf, what=f"path={path} grid={grid}")
 
 
+@pytest.mark.parametrize("rows", [16, 32])
+@pytest.mark.parametrize("M", [1, 2, 4, 8])
+def test_fused_epilogues_fma_tile_rows(rows, M):
+    """SiLU*mul (gate/up pairs 8 lanes apart in either tile height) and the
+    residual add on both tile heights of the FMA path, whole tiles and split."""
+    x, w = synth.make_xw(M, 2080, 1544, seed=90 + M + rows)
+    r = synth.make_x(M, 2080, seed=91 + M)
+    for us in (0, 1):
+        h, hf = run(x, w, wsm.EPI_SILU_MUL, path=wsm.PATH_STREAM, tile_rows=rows, unit_stages=us)
+        check_silu(x, w, h, hf, what=f"silu rows={rows} M={M} unit_stages={us}")
+        y, yf = run(x, w, wsm.EPI_RESIDUAL, r=r, path=wsm.PATH_STREAM, tile_rows=rows, unit_stages=us)
+        check_residual(x, w, r, y, yf, what=f"residual rows={rows} M={M} unit_stages={us}")
+
+
 def test_silu_mul_auto_and_split_patterns():
     M, N, K = 4, 6144, 4096
     x, w = synth.make_xw(M, N, K, seed=9)

@@ -48,6 +48,20 @@ def test_stream_path_small(M, N, K):
     check_full(x, w, y, yf, what=f"stream M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("rows", [16, 32])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("N,K", [(17, 40), (300, 1000), (129, 4104), (2112, 7168)])
+def test_stream_path_tile_rows(rows, M, N, K):
+    """Both tile heights of the FMA path (16 rows: 2 row groups x 4 K-slices;
+    32 rows: 4 x 2), ragged N and K, whole tiles and K split over units."""
+    x, w = synth.make_xw(M, N, K, seed=M * 11 + N + rows)
+    for us in (0, 1):
+        y, yf = run(x, w, path=wsm.PATH_STREAM, tile_rows=rows, unit_stages=us)
+        check_full(x, w, y, yf, what=f"stream rows={rows} M={M} N={N} K={K} unit_stages={us}")
+    p = wsm.plan(M, N, K, path=wsm.PATH_STREAM, tile_rows=rows)
+    assert p["tile_rows"] == rows and p["tile_k"] == (1024 if rows == 16 else 512)
+
+
 @pytest.mark.parametrize("M", [1, 8, 16, 17, 32, 40, 64])
 @pytest.mark.parametrize("N,K", SHAPES)
 def test_umma_path_small(M, N, K):

@@ -21,7 +21,7 @@
 namespace wsm {
 
 __global__ void wsm_umma_kernel(const __grid_constant__ KParams p);
-const void *stream_kernel_ptr(int mmax);  // wsm_stream.cu
+const void *stream_kernel_ptr(int mmax, int tile_rows);  // wsm_stream.cu
 
 namespace {
 
@@ -103,12 +103,13 @@ int pow2ceil(int v) {
 
 bool shape_ok(int M, int N, int K) { return M >= 1 && M <= 64 && N >= 1 && K >= 8 && (K % 8) == 0; }
 
-// Stream (FMA) geometry per register width; see wsm_stream.cu.
-void stream_geo(int mmax, Geo &g) {
+// Stream (FMA) geometry per register width and tile height (16 or 32 rows:
+// 8 rows per warp, 8 consumer warps as 2 x 4 or 4 x 2); see wsm_stream.cu.
+void stream_geo(int mmax, Geo &g, int tile_rows) {
     g.mmax = mmax;
-    g.rw = 8; g.rg = 2; g.kw = 4;
-    g.tile_rows = g.rg * g.rw;                 // 16
-    g.tile_k = g.kw * kStreamBoxK;             // 512 or 1024
+    g.rw = 8; g.rg = tile_rows / 8; g.kw = 8 / g.rg;
+    g.tile_rows = g.rg * g.rw;                 // 16 or 32
+    g.tile_k = g.kw * kStreamBoxK;             // 1024 or 512
     g.x_off = g.kw * g.tile_rows * 512;        // W part of a stage
     g.stage_bytes = g.x_off + g.kw * mmax * 512;
     g.slot_elems = g.tile_rows * mmax;
@@ -196,19 +197,44 @@ wsm_status plan_units(Geo &g, int ctas, int unit_stages, int tail_tiles, int tai
     return WSM_OK;
 }
 
-// Automatic path choice.  Measured on B200 (graph-replayed back-to-back
-// launches of decode shapes, M = 1..8, weights 30 MB .. 940 MB): the FMA path
-// wins while its arithmetic per weight byte stays light and the weights are
-// small enough for its shorter ramp to matter -- M = 1 up to about 128 MiB of
-// weights, M = 2 up to about 96 MiB, M <= 4 up to about 64 MiB -- and the
-// tensor-core path wins everywhere else (at M >= 5 always).
+// Automatic path choice.  Measured on B200 (back-to-back launches of the nine
+// decode shapes, 29-896 MiB of weights, at M = 1, 2, 4): at M <= 2 the FMA
+// path with the better of its two tile heights is fastest at every size (e.g.
+// 896 MiB at M = 1: 138 us against 144 us on the tensor cores; 192 MiB:
+// 35.8 against 39.5 us); at M = 3, 4 it wins up to about 64 MiB of weights
+// (it is ALU-bound from there: 8 FMA per weight element at M = 8); the
+// tensor-core path wins everywhere else.
 int auto_path(int M, long long w_bytes) {
     const long long MiB = 1ll << 20;
-    if (M == 1 && w_bytes <= 128 * MiB) return WSM_PATH_STREAM;
-    if (M == 2 && w_bytes <= 96 * MiB) return WSM_PATH_STREAM;
+    if (M <= 2) return WSM_PATH_STREAM;
     if (M <= 4 && w_bytes <= 64 * MiB) return WSM_PATH_STREAM;
     return WSM_PATH_UMMA;
 }
+
+// Tile height on the FMA path.  An SM streams at most ~33 GB/s with the
+// 16-row tiles' 8 KB boxes and ~45 GB/s with the 32-row tiles' 16 KB boxes
+// (under load; the rates fitted to the measured times), so 32 rows win unless
+// they leave fewer tiles than CTAs: then the units split K in two and the
+// split's partial sums and reduction (~4 us) cost more than the faster
+// stream saves.  Cost per tile height: the longer of the HBM time and the
+// busiest CTA's stream (rounds of units x unit bytes / SM rate), plus the
+// split.  It picks the faster height in all 18 measured cases at M = 1, 2 and
+// misses by 1 % in the one measured case at M = 3, 4 that stays on this path.
+// A chain on this path takes the height with the lower total over its tasks.
+double fma_cost_us(int rows, int N, int K, int ctas) {
+    const double sm_gbs = rows == 32 ? 45.0 : 33.0;
+    const double G = std::max(1, ctas);
+    const int tile_k = (8 / (rows / 8)) * kStreamBoxK;
+    const long long kb = (K + tile_k - 1) / tile_k;
+    const long long tiles = (N + rows - 1) / rows;
+    const long long nu = tiles >= ctas ? 1 : std::min<long long>(2, kb);
+    const long long ku = (kb + nu - 1) / nu;
+    const double unit_bytes = (double)rows * ku * tile_k * 2;
+    const double rounds = std::ceil((double)(tiles * nu) / G);
+    const double us = std::max(2.0 * N * K / 6.5e6, rounds * unit_bytes / (sm_gbs * 1e3));
+    return us + (nu > 1 ? 4.0 : 0.0);
+}
+int auto_fma_rows(int N, int K, int ctas) { return fma_cost_us(32, N, K, ctas) < fma_cost_us(16, N, K, ctas) ? 32 : 16; }
 
 // K per pipeline stage on the tensor-core path, measured on B200 (the decode
 // shapes, M = 1..64): 256 (4 boxes) everywhere except X tiles of 32 rows,
@@ -256,7 +282,10 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
         if (M > 8) return fail(WSM_ERR_UNSUPPORTED, "the FMA path takes M <= 8 (M=%d)", M);
         if (o->stage_k != 0) return fail(WSM_ERR_UNSUPPORTED, "stage_k applies to the UMMA path only");
         if (o->m_tile != 0 && o->m_tile != M) return fail(WSM_ERR_UNSUPPORTED, "the FMA path has no M-tiling");
-        stream_geo(force_mmax ? force_mmax : pow2ceil(M), g);
+        if (o->tile_rows != 0 && o->tile_rows != 16 && o->tile_rows != 32)
+            return fail(WSM_ERR_UNSUPPORTED, "tile_rows must be 0, 16 or 32 on the FMA path (got %d)", o->tile_rows);
+        stream_geo(force_mmax ? force_mmax : pow2ceil(M), g,
+                   o->tile_rows ? o->tile_rows : auto_fma_rows(N, K, g.grid));
         g.t_m = M;
         g.t_mpad = M;
         g.n_mt = 1;
@@ -388,7 +417,7 @@ wsm_status get_encode(EncodeTiledFn *fn) {
 struct DevInfo {
     int sms = 0;
     int smem_optin = 0;
-    bool attr_set[8] = {};
+    bool attr_set[16] = {};
 };
 std::map<int, DevInfo> g_dev;
 
@@ -417,8 +446,8 @@ const void *kernel_for(const Geo &g, int *slot) {
         *slot = 0;
         return reinterpret_cast<const void *>(&wsm_umma_kernel);
     }
-    *slot = g.mmax == 1 ? 1 : g.mmax == 2 ? 2 : g.mmax == 4 ? 3 : 4;
-    return stream_kernel_ptr(g.mmax);
+    *slot = (g.mmax == 1 ? 1 : g.mmax == 2 ? 2 : g.mmax == 4 ? 3 : 4) + (g.tile_rows == 32 ? 4 : 0);
+    return stream_kernel_ptr(g.mmax, g.tile_rows);
 }
 
 wsm_status prepare_kernel(DevInfo *d, const Geo &g, const void **fn) {
@@ -914,6 +943,21 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
             for (int i = 0; i < n; ++i) chain_wide = chain_wide && auto_wide((tasks[i].M + 15) / 16 * 16);
         }
         to.tile_rows = chain_wide ? 2 * kUmmaRows : kUmmaRows;
+    } else {
+        // FMA path: one tile height for the chain's ring, the one with the lower modelled total over the
+        // tasks (see auto_fma_rows)
+        if (opts->tile_rows != 0 && opts->tile_rows != 16 && opts->tile_rows != 32)
+            return fail(WSM_ERR_UNSUPPORTED, "tile_rows must be 0, 16 or 32 on the FMA path (got %d)", opts->tile_rows);
+        to.tile_rows = opts->tile_rows;
+        if (to.tile_rows == 0) {
+            const int ctas = (opts->grid > 0) ? std::min(opts->grid, d->sms) : d->sms;
+            double c16 = 0, c32 = 0;
+            for (int i = 0; i < n; ++i) {
+                c16 += fma_cost_us(16, tasks[i].N, tasks[i].K, ctas);
+                c32 += fma_cost_us(32, tasks[i].N, tasks[i].K, ctas);
+            }
+            to.tile_rows = c32 < c16 ? 32 : 16;
+        }
     }
     to.stage_k = (path == WSM_PATH_UMMA) ? (opts->stage_k ? opts->stage_k
                                                            : auto_stage_k((maxM + 15) / 16 * 16, chain_wide))
@@ -928,7 +972,7 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     for (auto &g : geos) g.grid = chain_grid;
     Geo ring = geos[0];
     if (path == WSM_PATH_STREAM) {
-        stream_geo(pow2ceil(maxM), ring);
+        stream_geo(pow2ceil(maxM), ring, to.tile_rows);
     } else {
         int tmp = 16;
         for (auto &g : geos) tmp = std::max(tmp, g.t_mpad);

@@ -514,11 +514,23 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
     if (threadIdx.x == 0) chain_run_done(p);
 }
 
-// Kernel for a register width: 8 rows per warp, 2 row groups, 4 K-slices
-// (T_N = 16 rows, T_K = 1024) for every MMAX; measured on B200, the wide
-// stage beats 4 x 4 x 2 (T_K = 512) at M = 1 and 2 as well.  Must agree with
-// stream_geo() in wsm_api.cu.
-const void *stream_kernel_ptr(int mmax) {
+// Kernel for a register width and a tile height, 8 rows per warp either way:
+// 16-row tiles are 2 row groups x 4 K-slices (T_K = 1024, W boxes of
+// [16 x 256], 8 KB), 32-row tiles 4 row groups x 2 K-slices (T_K = 512, boxes
+// of [32 x 256], 16 KB).  Measured on B200: one SM streams at most ~36 GB/s
+// with the 8 KB boxes and ~50 GB/s with the 16 KB ones (the same 32 KB per
+// stage); the wide stage of the 16-row tiles beats 4 x 4 x 2 (T_K = 512) at
+// M = 1 and 2.  Must agree with stream_geo() in wsm_api.cu.
+const void *stream_kernel_ptr(int mmax, int tile_rows) {
+    if (tile_rows == 32) {
+        switch (mmax) {
+            case 1: return reinterpret_cast<const void *>(&wsm_stream_kernel<1, 8, 4, 2>);
+            case 2: return reinterpret_cast<const void *>(&wsm_stream_kernel<2, 8, 4, 2>);
+            case 4: return reinterpret_cast<const void *>(&wsm_stream_kernel<4, 8, 4, 2>);
+            case 8: return reinterpret_cast<const void *>(&wsm_stream_kernel<8, 8, 4, 2>);
+            default: return nullptr;
+        }
+    }
     switch (mmax) {
         case 1: return reinterpret_cast<const void *>(&wsm_stream_kernel<1, 8, 2, 4>);
         case 2: return reinterpret_cast<const void *>(&wsm_stream_kernel<2, 8, 2, 4>);
