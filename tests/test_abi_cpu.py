@@ -51,9 +51,11 @@ def test_abi_version():
 
 def test_plan_paths_and_geometry():
     p = wsm.plan(1, 4096, 4096, num_sms=148)
-    assert p["path"] == wsm.PATH_STREAM and p["tile_rows"] == 16 and p["m_tile"] == 1
-    assert p["n_tiles"] == 256 and p["k_iters"] == 4096 // p["tile_k"]
-    assert p["iters"] == p["n_tiles"] * p["k_iters"] and p["grid"] == 148
+    assert p["path"] == wsm.PATH_STREAM and p["tile_rows"] == 32 and p["m_tile"] == 1
+    assert p["n_tiles"] == 128 and p["k_iters"] == 4096 // p["tile_k"]
+    assert p["iters"] == p["n_tiles"] * p["k_iters"] and p["grid"] == 128   # one CTA per (whole-tile) unit
+    p = wsm.plan(1, 4096, 4096, num_sms=148, tile_rows=16)
+    assert p["tile_rows"] == 16 and p["n_tiles"] == 256 and p["grid"] == 148
     p = wsm.plan(16, 4096, 4096, num_sms=148)
     assert p["path"] == wsm.PATH_UMMA and p["tile_rows"] == 128 and p["tile_k"] == 256 and p["m_tile"] == 16
     assert p["n_tiles"] == 32 and p["k_iters"] == 16 and p["m_tiles"] == 1
@@ -85,19 +87,22 @@ def test_auto_path_crossovers():
 
 def test_fma_tile_rows():
     """FMA path tile height: 32 rows (16 KB boxes, the faster stream per SM)
-    unless that leaves fewer tiles than CTAs while 16-row tiles do not (the K
-    split would then cost more); an explicit tile_rows of 16 or 32 is taken
-    as given, anything else refused on this path."""
+    unless that leaves too few tiles (fewer than half the CTAs: K split in
+    two); an explicit tile_rows of 16 or 32 is taken as given, anything else
+    refused on this path.  Units: whole tiles from half as many tiles as CTAs
+    up, 2 per tile below."""
     def rows(M, N, K, **kw):
         p = wsm.plan(M, N, K, num_sms=148, path=wsm.PATH_STREAM, **kw)
         assert p["tile_k"] == (1024 if p["tile_rows"] == 16 else 512)
+        nu = -(-p["k_iters"] // p["unit_stages"])
+        assert nu == (1 if p["n_tiles"] * 2 >= 148 else 2) or p["k_iters"] == 1
         return p["tile_rows"]
-    assert rows(1, 4096, 4096) == 16          # o: 128 tiles of 32 rows < 148, 256 of 16
-    assert rows(1, 4096, 7168) == 16
+    assert rows(1, 4096, 4096) == 32          # o: 128 whole 32-row tiles, one round
+    assert rows(1, 4096, 7168) == 32
     assert rows(1, 6144, 4096) == 32          # qkv: 192 tiles of 32 rows
     assert rows(1, 24576, 4096) == 32         # gate_up
-    assert rows(1, 4096, 12288) == 32         # down: split either way, 32 streams faster
-    assert rows(1, 2112, 7168) == 32          # 66 or 132 tiles: both split
+    assert rows(1, 4096, 12288) == 32         # down
+    assert rows(1, 2112, 7168) == 16          # 66 tiles of 32 rows would split K: 132 whole 16-row tiles
     assert rows(2, 57344, 8192) == 32
     assert rows(1, 4096, 4096, tile_rows=32) == 32
     assert rows(1, 24576, 4096, tile_rows=16) == 16
@@ -119,8 +124,10 @@ def test_plan_grid_clamped_to_work():
     assert p["iters"] == 1 and p["grid"] == 1
     p = wsm.plan(1, 4096, 4096, num_sms=148, grid=7)
     assert p["grid"] == 7
-    p = wsm.plan(1, 4096, 4096, num_sms=148, grid=1000)
+    p = wsm.plan(1, 8192, 4096, num_sms=148, grid=1000)
     assert p["grid"] == 148
+    p = wsm.plan(1, 4096, 4096, num_sms=148, grid=1000)
+    assert p["grid"] == p["units"] == 128
 
 
 def test_plan_m_tiling_and_l2_policy():

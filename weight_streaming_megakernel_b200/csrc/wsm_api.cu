@@ -130,12 +130,15 @@ void stream_geo(int mmax, Geo &g, int tile_rows) {
 //                                                   about two units remains)
 // with c = 1 stage of per-unit overhead at X tiles <= 32 rows, 4 above
 // (larger partials).  FMA path (consumer warps run the epilogue themselves):
-// whole tiles unless there are fewer tiles than CTAs, then 2 units per tile.
+// whole tiles unless there are fewer than half as many tiles as CTAs, then 2
+// units per tile (measured on B200: with 32-row tiles, o at M = 1 10.2 us
+// whole against 12.8 us split over 2 units -- the split's reduction costs
+// more than the idle SMs; the split pays only with very few tiles).
 // Tail: the last tiles of the schedule may be split into smaller units, so
 // the end of a GEMM (which in a chain every dependent task waits for) is
 // spread evenly over CTAs that stream at different speeds.
 int auto_units_per_tile(const Geo &g, int ctas) {
-    if (g.path != WSM_PATH_UMMA) return std::max(1, std::min(g.tiles() >= ctas ? 1 : 2, g.kb));
+    if (g.path != WSM_PATH_UMMA) return std::max(1, std::min(g.tiles() * 2 >= ctas ? 1 : 2, g.kb));
     const double G = std::max(1, ctas);
     const double c = (g.t_mpad <= 32) ? 1.0 : 4.0;
     int best = 1;
@@ -214,20 +217,22 @@ int auto_path(int M, long long w_bytes) {
 // Tile height on the FMA path.  An SM streams at most ~33 GB/s with the
 // 16-row tiles' 8 KB boxes and ~45 GB/s with the 32-row tiles' 16 KB boxes
 // (under load; the rates fitted to the measured times), so 32 rows win unless
-// they leave fewer tiles than CTAs: then the units split K in two and the
-// split's partial sums and reduction (~4 us) cost more than the faster
-// stream saves.  Cost per tile height: the longer of the HBM time and the
-// busiest CTA's stream (rounds of units x unit bytes / SM rate), plus the
-// split.  It picks the faster height in all 18 measured cases at M = 1, 2 and
-// misses by 1 % in the one measured case at M = 3, 4 that stays on this path.
-// A chain on this path takes the height with the lower total over its tasks.
+// they leave too few tiles: fewer than half as many as CTAs split K in two
+// (~4 us for the partial sums and their reduction), and fewer tiles than CTAs
+// mean more bytes per busy SM.  Cost per tile height: the longer of the HBM
+// time and the busiest CTA's stream (rounds of units x unit bytes / SM rate),
+// plus the split.  On the 15 measured (shape, M) cases at M = 1, 2, 4 whose
+// choice it decides (o, qkv, down, 7168 x 2112 and x 4096), it lands within
+// 1 % of the faster height; above them both heights have whole tiles and
+// 32 rows win on the stream rate.  A chain on this path takes the height
+// with the lower total over its tasks.
 double fma_cost_us(int rows, int N, int K, int ctas) {
     const double sm_gbs = rows == 32 ? 45.0 : 33.0;
     const double G = std::max(1, ctas);
     const int tile_k = (8 / (rows / 8)) * kStreamBoxK;
     const long long kb = (K + tile_k - 1) / tile_k;
     const long long tiles = (N + rows - 1) / rows;
-    const long long nu = tiles >= ctas ? 1 : std::min<long long>(2, kb);
+    const long long nu = tiles * 2 >= ctas ? 1 : std::min<long long>(2, kb);  // as auto_units_per_tile
     const long long ku = (kb + nu - 1) / nu;
     const double unit_bytes = (double)rows * ku * tile_k * 2;
     const double rounds = std::ceil((double)(tiles * nu) / G);
