@@ -8,8 +8,8 @@ shrink by `world`; the exchange is M * N * 2 bytes per GEMM (786 KB for the
 Qwen3-8B gate+up projection at M = 16), small next to the streamed weights.
 
 Block boundaries are multiples of `align` output columns: the weight tile
-height of the kernel path (128 rows on the tensor-core path, 16 on the FMA
-path), and 16 for the fused SiLU*mul weight, whose gate/up pairs come in
+height of the kernel path (128 rows on the tensor-core path, 16 or 32 on the
+FMA path), and 16 for the fused SiLU*mul weight, whose gate/up pairs come in
 blocks of 16 rows (8 output columns).
 
 This module is host logic around the library: `ShardedLinear` calls the
