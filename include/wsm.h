@@ -33,7 +33,11 @@
  *    returns WSM_ERR_UNSUPPORTED; there is no slow fallback.
  *  - Calls queued on one stream are serialised by the stream.  Calls on
  *    different streams may run concurrently: the library keeps one scratch
- *    workspace per (device, stream).
+ *    workspace per (device, stream).  A call captured into a CUDA graph keeps
+ *    the capture stream's workspace of that moment (the library never frees
+ *    a workspace it has outgrown, so the graph stays valid); replay such a
+ *    graph on that stream, or at least never concurrently with other calls
+ *    on it.
  *  - The library never reads the values of Y before writing it.
  */
 #ifndef WSM_H
@@ -352,7 +356,15 @@ size_t wsm_chain_trace(wsm_chain *chain, wsm_stream_t stream, unsigned long long
 void wsm_chain_destroy(wsm_chain *chain);
 
 /* One-shot: validate, prepare (cached by the task list's contents, per
- * device) and run the chain on `stream`.  Equivalent to create + run. */
+ * device) and run the chain on `stream`.  Equivalent to create + run.
+ *  - Every call with the same list runs the same prepared chain, whose
+ *    readiness counters and scratch are its own: queue such calls on one
+ *    stream (runs that overlap on the GPU race on the counters).
+ *  - A list is prepared on its first call, which must not be made during
+ *    stream capture (WSM_ERR_INVALID; run it once before capturing).  A chain
+ *    that ran during a capture stays prepared for the life of the process,
+ *    so the graph stays valid; up to 16 others are kept, then dropped
+ *    together (dropping synchronises the device). */
 wsm_status gemm_chain(const wsm_task *tasks, int n_tasks, wsm_stream_t stream);
 
 /* Validation only (pure host function, no CUDA calls). */

@@ -312,6 +312,43 @@ def test_gemm_chain_one_shot():
     check_dependent(x0, ws, ys, yfs)
 
 
+@pytest.mark.filterwarnings("ignore:The CUDA Graph is empty")
+def test_gemm_chain_in_graph_survives_cache_drop():
+    """gemm_chain inside a CUDA graph: a list met for the first time during
+    capture is refused (it cannot be prepared there); prepared by a call
+    outside capture, it is captured, and the graph still replays correctly
+    after more distinct lists than the cache keeps have dropped the others."""
+    # shapes no other test passes to gemm_chain: the cache is keyed by pointers and shapes, and
+    # freed buffers come back at the same addresses
+    dims = [256, 768, 512]
+    x0, ws, ys, yfs, tasks = dependent_chain(4, dims, seed=12)
+    s = torch.cuda.Stream()
+    g0 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g0, stream=s):
+        with pytest.raises(wsm.WsmError) as ei:
+            wsm.gemm_chain(tasks, stream=s)
+    assert ei.value.code == wsm.WSM_ERR_INVALID and "capture" in str(ei.value)
+    del g0
+    wsm.gemm_chain(tasks, stream=s)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        wsm.gemm_chain(tasks, stream=s)
+    # 20 other lists (distinct output buffers) fill the cache past its bound
+    extra = [torch.empty(4, 768, dtype=torch.bfloat16, device=DEV) for _ in range(20)]
+    for yx in extra:
+        wsm.gemm_chain([wsm.Task(x0, ws[0], yx)], stream=s)
+    s.synchronize()
+    for y in ys:
+        y.fill_(0)
+    with torch.cuda.stream(s):
+        g.replay()
+        g.replay()
+    s.synchronize()
+    check_dependent(x0, ws, ys, yfs)
+    check_full(x0.cpu(), ws[0].cpu(), extra[-1], what="the last extra list")
+
+
 @pytest.mark.parametrize("deps", [False, True])
 @pytest.mark.parametrize("kernels", [wsm.CHAIN_KERNELS_SPLIT, wsm.CHAIN_KERNELS_ONE, wsm.CHAIN_KERNELS_AUTO])
 def test_mixed_m_chain(deps, kernels):

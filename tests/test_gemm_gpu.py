@@ -245,6 +245,39 @@ def test_cuda_graph_capture():
     check_full(x, w, y)
 
 
+def test_graph_survives_workspace_growth():
+    """A graph captured with the stream's workspace still replays correctly
+    after a larger call on that stream has outgrown the workspace (the
+    library keeps the outgrown buffer, which the graph still points at)."""
+    M, N, K = 16, 1024, 4096
+    M2, N2, K2 = 64, 2048, 16384
+    assert wsm.workspace_bytes(M2, N2, K2) > max(1 << 20, 2 * wsm.workspace_bytes(M, N, K))
+    x, w = synth.make_xw(M, N, K, seed=5)
+    x2, w2 = synth.make_xw(M2, N2, K2, seed=6)
+    xd, wd, x2d, w2d = x.to(DEV), w.to(DEV), x2.to(DEV), w2.to(DEV)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    y2 = torch.empty(M2, N2, dtype=torch.bfloat16, device=DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        wsm.skinny_gemm(xd, wd, y)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        wsm.skinny_gemm(xd, wd, y, stream=s)
+    with torch.cuda.stream(s):
+        wsm.skinny_gemm(x2d, w2d, y2)  # grows the stream's workspace
+        y.fill_(0)
+        g.replay()
+        g.replay()
+    s.synchronize()
+    assert wsm.stream_status(s) == 0
+    check_full(x, w, y, what="graph after workspace growth")
+    rng = np.random.default_rng(0)
+    ms = rng.integers(0, M2, 2048)
+    ns = rng.integers(0, N2, 2048)
+    check_sampled(x2, w2, y2, None, ms, ns, what="the call that grew the workspace")
+
+
 def test_empty_ranges_when_fewer_stages_than_ctas():
     """T < grid: the plan clamps the grid, and a forced-large grid on a chain
     covers it in-kernel (see the chain tests)."""

@@ -565,6 +565,12 @@ struct Workspace {
     size_t bytes = 0;
 };
 std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
+// Buffers a stream's workspace has outgrown.  They stay allocated until the
+// process exits: a CUDA graph captured while one of them was current still
+// points at it, and replaying that graph must not touch freed memory.  The
+// workspace at least doubles on each growth, so they hold less than the
+// current one.
+std::vector<void *> g_ws_retired;
 
 wsm_status stream_workspace(int dev, cudaStream_t stream, const Geo &g, void **out, size_t *out_bytes) {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -583,16 +589,14 @@ wsm_status stream_workspace(int dev, cudaStream_t stream, const Geo &g, void **o
                     "run the same call once outside capture first",
                     need);
     size_t bytes = round_up(std::max(need, (size_t)1 << 20), 256);
-    if (w.ptr) {
-        WSM_CUDA(cudaStreamSynchronize(stream));
-        WSM_CUDA(cudaFree(w.ptr));
-        w.ptr = nullptr;
-        w.bytes = 0;
-    }
     void *p = nullptr;
     cudaError_t e = cudaMalloc(&p, bytes);
     if (e != cudaSuccess) return fail(WSM_ERR_NOMEM, "cudaMalloc(%zu) for the workspace failed: %s", bytes, cudaGetErrorString(e));
-    WSM_CUDA(cudaMemsetAsync(p, 0, bytes, stream));
+    if ((e = cudaMemsetAsync(p, 0, bytes, stream)) != cudaSuccess) {
+        cudaFree(p);
+        return cuda_fail(e, "cudaMemsetAsync(workspace)");
+    }
+    if (w.ptr) g_ws_retired.push_back(w.ptr);
     w.ptr = p;
     w.bytes = bytes;
     *out = p;
@@ -668,7 +672,16 @@ struct wsm_chain {
 namespace wsm {
 namespace {
 
-std::map<std::pair<int, std::string>, wsm_chain *> g_chain_cache;
+// gemm_chain's prepared chains, by device and task list.  A chain that ran
+// while its stream was being captured is pinned: a CUDA graph points at its
+// table and scratch, so it is never freed.  The others are dropped together
+// when 16 of them have accumulated.
+struct CachedChain {
+    wsm_chain *ch = nullptr;
+    bool pinned = false;
+};
+std::map<std::pair<int, std::string>, CachedChain> g_chain_cache;
+constexpr size_t kChainCacheUnpinned = 16;
 
 wsm_status validate_tasks(const wsm_task *tasks, int n) {
     if (!tasks || n < 1) return fail(WSM_ERR_INVALID, "task list must be non-null with n_tasks >= 1");
@@ -1288,22 +1301,45 @@ wsm_status gemm_chain(const wsm_task *tasks, int n_tasks, wsm_stream_t stream) {
                                (uintptr_t)(t.dep_cols != 0)};
         key.append(reinterpret_cast<const char *>(f), sizeof f);
     }
-    wsm_chain *ch = nullptr;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    WSM_CUDA(cudaStreamIsCapturing(s, &cs));
+    const bool capturing = cs != cudaStreamCaptureStatusNone;
+    // a cached chain is run under the lock, so no other thread can drop it in between (a run only
+    // queues work and takes no lock itself)
     {
         std::lock_guard<std::mutex> lk(g_mu);
         auto it = g_chain_cache.find({dev, key});
-        if (it != g_chain_cache.end()) ch = it->second;
-    }
-    if (!ch) {
-        if ((st = wsm_chain_create(tasks, n_tasks, nullptr, &ch)) != WSM_OK) return st;
-        std::lock_guard<std::mutex> lk(g_mu);
-        if (g_chain_cache.size() >= 16) {
-            // bounded cache: drop everything (rare; prepared chains are cheap to rebuild)
-            for (auto &kv : g_chain_cache) wsm_chain_destroy(kv.second);
-            g_chain_cache.clear();
+        if (it != g_chain_cache.end()) {
+            if (capturing) it->second.pinned = true;
+            return wsm_chain_run(it->second.ch, stream);
         }
-        g_chain_cache[{dev, key}] = ch;
     }
+    if (capturing)
+        return fail(WSM_ERR_INVALID, "gemm_chain: this task list is not prepared yet and cannot be prepared during "
+                                     "stream capture: run it once outside capture first (or use wsm_chain_create)");
+    wsm_chain *ch = nullptr;
+    if ((st = wsm_chain_create(tasks, n_tasks, nullptr, &ch)) != WSM_OK) return st;
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_chain_cache.find({dev, key});
+    if (it != g_chain_cache.end()) {  // another thread prepared the same list meanwhile
+        wsm_chain_destroy(ch);
+        return wsm_chain_run(it->second.ch, stream);
+    }
+    size_t unpinned = 0;
+    for (auto &kv : g_chain_cache) unpinned += kv.second.pinned ? 0 : 1;
+    if (unpinned >= kChainCacheUnpinned) {
+        // bounded cache: drop the unpinned chains (rare; a prepared chain is cheap to rebuild)
+        for (auto i = g_chain_cache.begin(); i != g_chain_cache.end();) {
+            if (i->second.pinned) {
+                ++i;
+                continue;
+            }
+            wsm_chain_destroy(i->second.ch);
+            i = g_chain_cache.erase(i);
+        }
+    }
+    g_chain_cache[{dev, key}] = CachedChain{ch, false};
     return wsm_chain_run(ch, stream);
 }
 
