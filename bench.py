@@ -655,8 +655,10 @@ def main():
         import statistics as _st
         breakdown = {"ms_per_step": round(rb["ms_per_step"], 4),
                      "value_GBps": round(rb["total_bytes"] / (rb["ms_per_step"] * 1e-3) / 1e9, 1),
-                     "us_per_gemm": {c.name: round(_st.median(row[i] for row in rb["per_launch"]) * 1e3, 2)
-                                     for i, c in enumerate(rb["cases"])}}
+                     "note": "ms_per_step: the launches back to back in one graph; us_per_gemm_isolated: each "
+                             "launch alone between two events, without the overlap with its neighbours",
+                     "us_per_gemm_isolated": {c.name: round(_st.median(row[i] for row in rb["per_launch"]) * 1e3, 2)
+                                              for i, c in enumerate(rb["cases"])}}
 
     # roofline of the weight-streaming kernel: per-launch algorithmic bytes / duration
     import statistics
