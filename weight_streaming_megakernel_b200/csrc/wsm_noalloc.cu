@@ -90,7 +90,7 @@ wsm_status skinny_gemm_noalloc(const void *X, const void *W, void *Y, int M, int
     // The array keeps the previous call's contents: clear the status word and
     // the counters this call will use (they must start at zero).  Calls whose
     // work overlaps on the GPU share the array and race.
-    const size_t counters = 256 + 4 * (2 + (size_t)info.n_tiles * (size_t)info.m_tiles);
+    const size_t counters = 256 + 4 * ((size_t)wsm::kSchedWords + (size_t)info.n_tiles * (size_t)info.m_tiles);
     e = cudaMemsetAsync(scratch, 0, counters, stream);
     if (e != cudaSuccess) return noalloc_fail(WSM_ERR_CUDA, "skinny_gemm_noalloc: clearing the scratch failed");
 
