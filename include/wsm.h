@@ -275,7 +275,9 @@ typedef struct {
     int tail_tiles;            /* as in wsm_opts, for every task */
     int tail_unit_stages;      /* as in wsm_opts, for every task */
     int l2_prefetch_stages;    /* W stages per CTA prefetched into L2 while the CTA waits for
-                                  a dependency or the previous kernel: 0 = auto, -1 = none */
+                                  a dependency or the previous kernel: 0 = auto (tensor-core
+                                  path: 12 for a chain without dependencies whose X tiles are
+                                  16 rows, 4 otherwise; FMA path: none), -1 = none */
     int counter_groups;        /* 0 or 1: one readiness counter per task, bumped by every
                                   finished tile.  G >= 2: two-level readiness ("Fleet ..."
                                   reading notes, section 3d and the two-level event

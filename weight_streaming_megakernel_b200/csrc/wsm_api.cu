@@ -55,8 +55,14 @@ constexpr int kRingBudget = kSmemOptin - 8192;  // static shared memory + 1 KB a
 
 // W stages per waiting CTA prefetched into L2 (auto).  Measured on B200: 4
 // stages gain ~4 % on a dependent layer chain and 1-4 % on back-to-back
-// tensor-core launches; on the FMA path the prefetch costs 1-8 %, so none.
+// tensor-core launches (8-16 lose up to 10 % there); on the FMA path the
+// prefetch costs 1-8 %, so none.  A chain without dependencies waits only at
+// its start, for the previous kernel: with X tiles of 16 rows 12 stages beat
+// 4 by ~1 % (the decode step of 20 GEMMs 304.3 -> 301.3 us, the K = 7168 /
+// 8192 set 635 -> 629 us), with wider X tiles 4 stay best (the M = 32 / 64
+// set 127 us against 129-132 us with 8-16).
 constexpr int kDefaultPrefetchStagesUmma = 4;
+constexpr int kDefaultPrefetchStagesIndependentChain = 12;
 constexpr unsigned long long kDefaultDepTimeoutNs = 2000000000ull;
 constexpr unsigned long long kPipeTimeoutNs = 4000000000ull;
 
@@ -1007,6 +1013,11 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
             return fail(WSM_ERR_INVALID, "task %d: stage geometry differs from the chain's", i);  // cannot happen
     ch->geo = ring;
     ch->prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, path);
+    if (opts->l2_prefetch_stages == 0 && path == WSM_PATH_UMMA) {
+        bool deps = false;
+        for (int i = 0; i < n; ++i) deps = deps || tasks[i].dep >= 0;
+        if (!deps && ring.x_stride <= 16 * kUmmaBK * 2) ch->prefetch_stages = kDefaultPrefetchStagesIndependentChain;
+    }
     if (opts->k_order < 0 || opts->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", opts->k_order);
     ch->k_rotate = (opts->k_order == 2) ? 1 : 0;
     // measured on B200 (36 x 4 dependent chain at M = 16, 4 prefetch stages): 1 stage ahead of the
