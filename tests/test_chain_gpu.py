@@ -49,12 +49,14 @@ def check_dependent(x0, ws, ys, yfs):
         x = ys[t]
 
 
-@pytest.mark.parametrize("path,M", [(wsm.PATH_UMMA, 16), (wsm.PATH_UMMA, 64), (wsm.PATH_STREAM, 4),
-                                    (wsm.PATH_STREAM, 1)])
-def test_dependent_chain(path, M):
+@pytest.mark.parametrize("path,M,k_order", [(wsm.PATH_UMMA, 16, 0), (wsm.PATH_UMMA, 16, 1), (wsm.PATH_UMMA, 64, 0),
+                                            (wsm.PATH_UMMA, 64, 1), (wsm.PATH_STREAM, 4, 0), (wsm.PATH_STREAM, 1, 0)])
+def test_dependent_chain(path, M, k_order):
+    """Data-dependent chain (task t reads task t - 1's output); on the
+    tensor-core path in both K orders (auto = rotated for a chain)."""
     dims = [1024, 2048, 1024, 3072, 512, 1024, 4096, 1024]
     x0, ws, ys, yfs, tasks = dependent_chain(M, dims, seed=M)
-    ch = wsm.Chain(tasks, path=path)
+    ch = wsm.Chain(tasks, path=path, k_order=k_order)
     ch.run()
     code, failed = ch.status()
     assert code == wsm.WSM_OK, (code, failed, wsm.last_error())

@@ -1019,7 +1019,16 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         if (!deps && ring.x_stride <= 16 * kUmmaBK * 2) ch->prefetch_stages = kDefaultPrefetchStagesIndependentChain;
     }
     if (opts->k_order < 0 || opts->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", opts->k_order);
-    ch->k_rotate = (opts->k_order == 2) ? 1 : 0;
+    // auto: rotated on the tensor-core path.  A chain's units are long (whole tiles where later work can
+    // overlap them) and start together, and in increasing order every CTA would read the same columns
+    // of its weight rows at the same time.  Measured on B200: the decode step of 20 GEMMs 308.4 ->
+    // 300.3 us, the M = 32 / 64 set 133.0 -> 128.0 us, the 36 x 4 layer chain 3335 -> 3296 us, the
+    // fused data chain 3474 -> 3448 us, the K = 7168 / 8192 set within 0.4 %.  Single launches keep
+    // the increasing order (rotated: 0.5-2.5 % slower on 8 of 10 decode shapes).  Per-column waits
+    // read their dependency's chunks in increasing order, so those chains keep it too.
+    bool any_dep_cols = false;
+    for (int i = 0; i < n; ++i) any_dep_cols = any_dep_cols || tasks[i].dep_cols;
+    ch->k_rotate = (opts->k_order == 2 || (opts->k_order == 0 && path == WSM_PATH_UMMA && !any_dep_cols)) ? 1 : 0;
     // measured on B200 (36 x 4 dependent chain at M = 16, 4 prefetch stages): 1 stage ahead of the
     // dependency is 2 % faster than 2 and 4 % faster than the whole ring (3), and none at all is 2 %
     // slower than 1.  The FMA path keeps its whole ring (unmeasured).

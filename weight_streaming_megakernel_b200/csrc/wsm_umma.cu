@@ -221,10 +221,17 @@ __device__ __forceinline__ void reduce_row_partials(const UnitOut &uo, const Uni
 
 }  // namespace
 
+// First stage a unit streams, counted from its k_begin: with k_rotate, units
+// start at a tile-dependent offset and wrap around, so CTAs that run in
+// lockstep do not all read the same columns of their weight rows at once.
+__device__ __forceinline__ int unit_k_rot(const KParams &p, const UnitSpan &us) {
+    return p.k_rotate ? (us.tile * 5) % (us.k_end - us.k_begin) : 0;
+}
+
 // L2 prefetch of the W of the units this CTA would own in a round-robin (c,
-// c + G, ...), p.prefetch_stages stages at most, skipping the first `skip`
-// stages of each first-round unit (its claimer's ring already holds them).
-// Out of line: it runs at most once per task.
+// c + G, ...), p.prefetch_stages stages at most, in each unit's stream order,
+// skipping the first `skip` stages of each first-round unit (its claimer's
+// ring already holds them).  Out of line: it runs at most once per task.
 static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDev &T, int skip) {
     int budget = p.prefetch_stages;
     for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
@@ -232,10 +239,14 @@ static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDe
         int pg, pmt;
         tile_coords(T, ps.tile, pg, pmt);
         const int halves = p.wide ? 2 : 1;
-        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? skip : 0); kk < ps.k_end && budget > 0; ++kk, --budget)
+        const int k_len = ps.k_end - ps.k_begin;
+        const int k_rot = unit_k_rot(p, ps);
+        for (int i = (uu < (int)gridDim.x ? skip : 0); i < k_len && budget > 0; ++i, --budget) {
+            const int kk = ps.k_begin + (i + k_rot) % k_len;
             for (int h = 0; h < halves; ++h)
                 for (int j = 0; j < p.kps; ++j)
                     tma_prefetch_l2_2d(&T.tmW, (kk * p.kps + j) * kUmmaBK, (pg * halves + h) * kUmmaRows);
+        }
     }
 }
 
@@ -404,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     int next_u = cr.hi - cr.lo - n_static;
                     bool claimed = false;
                     const int k_len = us.k_end - us.k_begin;
-                    const int k_rot = p.k_rotate ? (us.tile * 5) % k_len : 0;
+                    const int k_rot = unit_k_rot(p, us);
                     for (int kk = us.k_begin; kk < us.k_end; ++kk) {
                         if (!take_slot()) break;
                         slot_ok = false;
