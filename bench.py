@@ -572,8 +572,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
     ap.add_argument("--only", default="", help="comma-separated case names (profiling)")
-    ap.add_argument("--mode", default="chain", choices=["chain", "launches"],
-                    help="chain: the step is one persistent gemm_chain kernel; launches: one skinny_gemm per GEMM")
+    ap.add_argument("--mode", default=None, choices=["chain", "launches"],
+                    help="chain: the step is one persistent gemm_chain kernel; launches: one skinny_gemm per GEMM "
+                         "(default: launches for the single-GEMM workload, chain otherwise)")
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-GEMM single-launch breakdown")
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "nshard"],
                     help="N > 1: independent replicas (weak scaling) or column blocks of every weight per rank "
@@ -581,6 +582,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.mode is None:
+        args.mode = "launches" if args.workload == "single" else "chain"
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -150,10 +150,10 @@ typedef struct {
                         TMEM accumulators, so X is re-read half as often).  FMA
                         path: 16 or 32 (32: larger TMA boxes, a faster stream per
                         SM; auto takes 32 unless it leaves fewer tiles than CTAs) */
-    int k_order;     /* tensor-core path: order of a work unit's K stages: 0 = auto
-                        (increasing for a single GEMM), 1 = increasing, 2 = rotated by a
-                        tile-dependent offset (so CTAs that start together do not all
-                        read the same columns of their weight rows at once) */
+    int k_order;     /* order of a work unit's K stages: 0 = auto (increasing for a
+                        single GEMM), 1 = increasing, 2 = rotated by a tile-dependent
+                        offset (so CTAs that start together do not all read the same
+                        columns of their weight rows at once) */
     int epilogue;    /* WSM_EPI_*; with SILU_MUL, Y (and Yf32) are [M, N/2] */
     const void *R;   /* WSM_EPI_RESIDUAL: bf16 [M, N], device */
     float *Yf32;     /* optional device [M, N] fp32: the result before rounding */
@@ -293,7 +293,8 @@ typedef struct {
                                   path 256 only if auto picks it for every task, FMA path the
                                   height with the lower modelled time over the tasks */
     int k_order;               /* as in wsm_opts; auto: rotated on the tensor-core path unless a
-                                  task waits per column (dep_cols), increasing otherwise */
+                                  task waits per column (dep_cols), increasing otherwise (on the
+                                  FMA path rotation measured 4-10 % slower) */
     int dep_ring_stages;       /* W stages a CTA streams into its ring ahead of an unmet
                                   dependency: 0 = auto (1 on the tensor-core path, the whole
                                   ring on the FMA path), -1 = the whole ring */

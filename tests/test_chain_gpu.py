@@ -50,10 +50,12 @@ def check_dependent(x0, ws, ys, yfs):
 
 
 @pytest.mark.parametrize("path,M,k_order", [(wsm.PATH_UMMA, 16, 0), (wsm.PATH_UMMA, 16, 1), (wsm.PATH_UMMA, 64, 0),
-                                            (wsm.PATH_UMMA, 64, 1), (wsm.PATH_STREAM, 4, 0), (wsm.PATH_STREAM, 1, 0)])
+                                            (wsm.PATH_UMMA, 64, 1), (wsm.PATH_STREAM, 4, 0), (wsm.PATH_STREAM, 1, 0),
+                                            (wsm.PATH_STREAM, 4, 2)])
 def test_dependent_chain(path, M, k_order):
-    """Data-dependent chain (task t reads task t - 1's output); on the
-    tensor-core path in both K orders (auto = rotated for a chain)."""
+    """Data-dependent chain (task t reads task t - 1's output), in both K
+    orders (auto: rotated on the tensor-core path, increasing on the FMA
+    path)."""
     dims = [1024, 2048, 1024, 3072, 512, 1024, 4096, 1024]
     x0, ws, ys, yfs, tasks = dependent_chain(M, dims, seed=M)
     ch = wsm.Chain(tasks, path=path, k_order=k_order)

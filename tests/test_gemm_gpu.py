@@ -406,20 +406,21 @@ def test_wide_tiles_fused_epilogues():
     check_bounded(y, yf, Yr, oracle.fused_bounds("residual", S=S, Y=Yr), "wide residual")
 
 
-@pytest.mark.parametrize("M", [1, 16, 64])
-def test_rotated_k_order(M):
+@pytest.mark.parametrize("path,M", [(wsm.PATH_UMMA, 1), (wsm.PATH_UMMA, 16), (wsm.PATH_UMMA, 64),
+                                    (wsm.PATH_STREAM, 1), (wsm.PATH_STREAM, 8)])
+def test_rotated_k_order(path, M):
     """Units walking their K stages from a tile-dependent offset: exact on
     small integers, within the bound on random inputs, deterministic."""
     N, K = 1000, 6144
     xi, wi = synth.make_int_xw(M, N, K, seed=3 + M)
     Y_ref, _ = oracle.gemm_ref(xi, wi)
     for kw in (dict(), dict(unit_stages=5), dict(grid=7)):
-        y, yf = run(xi, wi, path=wsm.PATH_UMMA, k_order=2, **kw)
+        y, yf = run(xi, wi, path=path, k_order=2, **kw)
         assert np.array_equal(yf.cpu().double().numpy(), Y_ref), kw
     x, w = synth.make_xw(M, N, K, seed=4 + M)
-    y1, yf1 = run(x, w, path=wsm.PATH_UMMA, k_order=2, unit_stages=7)
+    y1, yf1 = run(x, w, path=path, k_order=2, unit_stages=7)
     check_full(x, w, y1, yf1)
-    y2, yf2 = run(x, w, path=wsm.PATH_UMMA, k_order=2, unit_stages=7)
+    y2, yf2 = run(x, w, path=path, k_order=2, unit_stages=7)
     assert torch.equal(yf1, yf2)
 
 

@@ -125,8 +125,8 @@ struct KParams {
     int x_stride;                   // UMMA path: bytes between the X boxes of a stage
     int pdl;                        // 0: plain launch; 1: wait for the previous kernel before any
                                     // global access; 2: stream W before that wait, X after it
-    int k_rotate;                   // UMMA path: each unit walks its K stages starting at a tile-dependent
-                                    // offset (wrapping), so CTAs do not all read the same X lines at once
+    int k_rotate;                   // each unit walks its K stages starting at a tile-dependent offset
+                                    // (wrapping), so CTAs do not all read the same weight columns at once
     int dep_ring_stages;            // W stages a CTA issues into its ring while its task's dependency is
                                     // unmet (0: the whole ring)
     int wide;                       // UMMA path: tiles of 2 x 128 W rows sharing each X stage (two MMAs into
@@ -408,6 +408,13 @@ __device__ __forceinline__ UnitSpan unit_span(const TaskDev &T, int u) {
     r.k_begin = j * ku;
     r.k_end = min(r.k_begin + ku, T.kb);
     return r;
+}
+
+// First stage a unit streams, counted from its k_begin: with k_rotate, units
+// start at a tile-dependent offset and wrap around, so CTAs that run in
+// lockstep do not all read the same columns of their weight rows at once.
+__device__ __forceinline__ int unit_k_rot(const KParams &p, const UnitSpan &us) {
+    return p.k_rotate ? (us.tile * 11) % (us.k_end - us.k_begin) : 0;
 }
 
 // The units a CTA claims from: all of the task's, or with two-level readiness

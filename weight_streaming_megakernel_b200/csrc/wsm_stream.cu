@@ -118,16 +118,20 @@ struct LaneReduce {
 }  // namespace
 
 // L2 prefetch of the W of the units this CTA would own in a round-robin (c,
-// c + G, ...), p.prefetch_stages stages at most, skipping the first `skip`
-// stages of each first-round unit (its claimer's ring already holds them).
-// Out of line: it runs at most once per task.
+// c + G, ...), p.prefetch_stages stages at most, in each unit's stream order,
+// skipping the first `skip` stages of each first-round unit (its claimer's
+// ring already holds them).  Out of line: it runs at most once per task.
 static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDev &T, int skip, int KW, int TN) {
     int budget = p.prefetch_stages;
     for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
         const UnitSpan ps = unit_span(T, uu);
-        for (int kk = ps.k_begin + (uu < (int)gridDim.x ? skip : 0); kk < ps.k_end && budget > 0; ++kk, --budget)
+        const int k_len = ps.k_end - ps.k_begin;
+        const int k_rot = unit_k_rot(p, ps);
+        for (int i = (uu < (int)gridDim.x ? skip : 0); i < k_len && budget > 0; ++i, --budget) {
+            const int kk = ps.k_begin + (i + k_rot) % k_len;
             for (int kw = 0; kw < KW; ++kw)
                 tma_prefetch_l2_2d(&T.tmW, kk * (KW * kStreamBoxK) + kw * kStreamBoxK, ps.tile * TN);
+        }
     }
 }
 
@@ -287,6 +291,8 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     const int g = us.tile;
                     const int k_begin = us.k_begin;
                     const int k_end = us.k_end;
+                    const int k_len = k_end - k_begin;
+                    const int k_rot = unit_k_rot(p, us);
                     int next_u = cr.hi - cr.lo - n_static;
                     bool claimed = false;
                     for (int kk = k_begin; kk < k_end; ++kk) {
@@ -297,7 +303,9 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                         stage_meta[s][1] = u;
                         stage_meta[s][2] = (kk == k_begin ? kMetaFirst : 0) | (kk == k_end - 1 ? kMetaLast : 0);
                         mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
-                        const int k0 = kk * (KW * kStreamBoxK);
+                        // the stage this iteration loads (rotated within the unit when k_rotate)
+                        const int kr = k_rot ? k_begin + (kk - k_begin + k_rot) % k_len : kk;
+                        const int k0 = kr * (KW * kStreamBoxK);
 #pragma unroll
                         for (int kw = 0; kw < KW; ++kw)
                             tma_load_2d(st + kw * TN * 512, &T.tmW, &full_bar[s], k0 + kw * kStreamBoxK, g * TN,

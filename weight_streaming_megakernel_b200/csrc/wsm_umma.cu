@@ -221,13 +221,6 @@ __device__ __forceinline__ void reduce_row_partials(const UnitOut &uo, const Uni
 
 }  // namespace
 
-// First stage a unit streams, counted from its k_begin: with k_rotate, units
-// start at a tile-dependent offset and wrap around, so CTAs that run in
-// lockstep do not all read the same columns of their weight rows at once.
-__device__ __forceinline__ int unit_k_rot(const KParams &p, const UnitSpan &us) {
-    return p.k_rotate ? (us.tile * 11) % (us.k_end - us.k_begin) : 0;
-}
-
 // L2 prefetch of the W of the units this CTA would own in a round-robin (c,
 // c + G, ...), p.prefetch_stages stages at most, in each unit's stream order,
 // skipping the first `skip` stages of each first-round unit (its claimer's
