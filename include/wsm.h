@@ -315,6 +315,34 @@ enum {
     WSM_CHAIN_KERNELS_SPLIT = 2
 };
 
+/* Values of wsm_opts.k_order / wsm_chain_opts.k_order. */
+enum {
+    WSM_K_ORDER_AUTO = 0,
+    WSM_K_ORDER_INCREASING = 1,
+    WSM_K_ORDER_ROTATED = 2
+};
+
+/* One task's part of a chain plan (wsm_chain_plan). */
+typedef struct {
+    wsm_plan_info plan;     /* the task's plan: the chain's grid and ring, its own tiles and work
+                               units (workspace_bytes 0: a chain owns its scratch) */
+    int kernel;             /* which of the chain's kernels runs the task, from 0 (hybrid
+                               dispatch runs one kernel per run of tasks of one X width) */
+    int l2_prefetch_stages; /* that kernel's settings, resolved: W stages prefetched into L2
+                               while waiting (0 = none), */
+    int k_order;            /* WSM_K_ORDER_INCREASING or WSM_K_ORDER_ROTATED, */
+    int dep_ring_stages;    /* W stages streamed ahead of an unmet dependency (0 = the whole ring) */
+} wsm_chain_task_info;
+
+/* Pure host function (no CUDA calls, no memory touched): the plan
+ * wsm_chain_create would make for this task list and these options on a GPU
+ * with `num_sms` SMs.  The task pointers are validated (non-null, aligned,
+ * dep_cols wiring) but never dereferenced, so placeholders will do.  Fills
+ * out[0 .. n_tasks - 1] and *n_kernels (may be NULL).  Errors as
+ * wsm_chain_create's. */
+wsm_status wsm_chain_plan(const wsm_task *tasks, int n_tasks, const wsm_chain_opts *opts, int num_sms,
+                          wsm_chain_task_info *out, int *n_kernels);
+
 typedef struct wsm_chain wsm_chain;  /* opaque prepared chain */
 
 /* Validate a task list and prepare it on the current device: device task

@@ -325,3 +325,103 @@ def test_chain_validate_epilogues_and_column_deps():
 def test_plan_accepts_epilogue_options():
     wsm.plan(4, 4096, 4096, epilogue=wsm.EPI_SILU_MUL)
     wsm.plan(4, 4096, 4096, epilogue=wsm.EPI_RESIDUAL)
+
+
+# ----------------------------------------------------------- chain planning (pure host)
+
+QWEN3_LAYER = ((4096, 6144), (4096, 4096), (4096, 24576), (12288, 4096))  # (K, N): qkv, o, gate_up, down
+
+
+def test_chain_plan_independent_decode_step():
+    """The decode step (20 independent GEMMs, M = 1..16) as one tensor-core
+    kernel: units grow with the work after them (whole tiles while plenty
+    follows), the last task keeps the single-call split; 12 prefetch stages
+    (no dependencies, X tiles of 16 rows) and the rotated K order."""
+    specs = [dict(M=m, N=n, K=k) for m in (1, 2, 4, 8, 16) for (k, n) in QWEN3_LAYER]
+    plans, kernels = wsm.chain_plan(specs)
+    assert kernels == 1
+    for s, p in zip(specs, plans):
+        assert p["path"] == wsm.PATH_UMMA and p["grid"] == 148 and p["kernel"] == 0
+        assert p["l2_prefetch_stages"] == 12 and p["k_order"] == wsm.K_ORDER_ROTATED and p["dep_ring_stages"] == 1
+        assert p["stages"] == 3 and p["m_tile"] == 16
+        assert p["workspace_bytes"] == 0
+    for p in plans[:12]:
+        assert p["unit_stages"] == p["k_iters"], p  # whole tiles early in the step
+    last = wsm.plan(16, 4096, 12288)
+    assert plans[-1]["unit_stages"] == last["unit_stages"] and plans[-1]["units"] == last["units"]
+
+
+def test_chain_plan_dependent_layers():
+    """Task t waits for t - 1: nothing overlaps a task's end, so every task
+    takes the single-call split; 4 prefetch stages, one ring stage ahead of
+    the dependency, rotated K order."""
+    specs = []
+    for layer in range(3):
+        for (k, n) in QWEN3_LAYER:
+            specs.append(dict(M=16, N=n, K=k, dep=len(specs) - 1))
+    plans, kernels = wsm.chain_plan(specs)
+    assert kernels == 1
+    for s, p in zip(specs, plans):
+        single = wsm.plan(16, s["N"], s["K"])
+        assert p["unit_stages"] == single["unit_stages"] and p["units"] == single["units"], (s, p, single)
+        assert p["l2_prefetch_stages"] == 4 and p["dep_ring_stages"] == 1 and p["k_order"] == wsm.K_ORDER_ROTATED
+    # explicit options pass through
+    plans, _ = wsm.chain_plan(specs, l2_prefetch_stages=-1, dep_ring_stages=-1, k_order=wsm.K_ORDER_INCREASING)
+    assert all(p["l2_prefetch_stages"] == 0 and p["dep_ring_stages"] == 0 and p["k_order"] == 1 for p in plans)
+
+
+def test_chain_plan_wide_x_and_fma():
+    """M = 32 / 64 tasks keep 4 prefetch stages (wider X tiles); a chain of
+    M = 1 GEMMs runs on the FMA path in increasing K order, without prefetch,
+    its whole ring ahead of a dependency."""
+    specs = [dict(M=m, N=n, K=k) for m in (32, 64) for (k, n) in QWEN3_LAYER[2:]]
+    plans, _ = wsm.chain_plan(specs)
+    for s, p in zip(specs, plans):
+        assert p["path"] == wsm.PATH_UMMA and p["l2_prefetch_stages"] == 4 and p["m_tile"] == s["M"]
+        assert p["stages"] == 2  # the ring is sized for the widest X tile
+    specs = [dict(M=1, N=n, K=k, dep=i - 1) for i, (k, n) in enumerate(QWEN3_LAYER)]
+    plans, kernels = wsm.chain_plan(specs)
+    assert kernels == 1
+    for p in plans:
+        assert p["path"] == wsm.PATH_STREAM and p["k_order"] == wsm.K_ORDER_INCREASING
+        assert p["l2_prefetch_stages"] == 0 and p["dep_ring_stages"] == 0 and p["tile_rows"] in (16, 32)
+
+
+def test_chain_plan_hybrid_dispatch():
+    """Tasks of M <= 32 and M > 32 in one chain: SPLIT gives one kernel per
+    run of one X width (numbered in order), ONE a single kernel sized for the
+    widest X tile; AUTO splits only when the narrow runs carry enough weight
+    bytes per extra kernel."""
+    specs = [dict(M=16, N=4096, K=4096), dict(M=16, N=6144, K=4096, dep=0), dict(M=64, N=4096, K=4096, dep=1),
+             dict(M=64, N=4096, K=4096), dict(M=8, N=4096, K=4096, dep=3)]
+    plans, kernels = wsm.chain_plan(specs, kernels=wsm.CHAIN_KERNELS_SPLIT)
+    assert kernels == 3 and [p["kernel"] for p in plans] == [0, 0, 1, 1, 2]
+    assert [p["m_tile"] for p in plans] == [16, 16, 64, 64, 16]
+    assert plans[0]["stages"] == 3 and plans[2]["stages"] == 2
+    plans, kernels = wsm.chain_plan(specs, kernels=wsm.CHAIN_KERNELS_ONE)
+    assert kernels == 1 and all(p["stages"] == 2 and p["kernel"] == 0 for p in plans)
+    _, kernels = wsm.chain_plan(specs)
+    assert kernels == 1  # 0.1 GB of narrow weights: not worth two extra kernel boundaries
+
+
+def test_chain_plan_column_dependencies_keep_increasing_order():
+    specs = [dict(M=16, N=2048, K=1024), dict(M=16, N=1024, K=2048, dep=0, dep_cols=True)]
+    plans, _ = wsm.chain_plan(specs)
+    assert all(p["k_order"] == wsm.K_ORDER_INCREASING for p in plans)
+    assert plans[1]["tail_tiles"] == 0
+
+
+def test_chain_plan_errors():
+    specs = [dict(M=16, N=4096, K=4096), dict(M=16, N=4096, K=4096, dep=0)]
+    for kw, code in ((dict(path=3), wsm.WSM_ERR_INVALID), (dict(kernels=3), wsm.WSM_ERR_INVALID),
+                     (dict(flags=4), wsm.WSM_ERR_INVALID), (dict(l2_prefetch_stages=-2), wsm.WSM_ERR_INVALID),
+                     (dict(k_order=3), wsm.WSM_ERR_INVALID), (dict(dep_ring_stages=-2), wsm.WSM_ERR_INVALID),
+                     (dict(counter_groups=-1), wsm.WSM_ERR_INVALID), (dict(tile_rows=64), wsm.WSM_ERR_UNSUPPORTED),
+                     (dict(path=wsm.PATH_STREAM), wsm.WSM_ERR_UNSUPPORTED),  # M = 16 on the FMA path
+                     (dict(num_sms=0), wsm.WSM_ERR_INVALID)):
+        with pytest.raises(wsm.WsmError) as e:
+            wsm.chain_plan(specs, **kw)
+        assert e.value.code == code, kw
+    with pytest.raises(wsm.WsmError) as e:
+        wsm.chain_plan([dict(M=16, N=4096, K=4096, dep=0)])  # a task may not wait for itself
+    assert e.value.code == wsm.WSM_ERR_INVALID

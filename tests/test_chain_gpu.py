@@ -316,6 +316,27 @@ def test_gemm_chain_one_shot():
     check_dependent(x0, ws, ys, yfs)
 
 
+@pytest.mark.parametrize("kernels", [wsm.CHAIN_KERNELS_AUTO, wsm.CHAIN_KERNELS_SPLIT])
+def test_chain_plan_matches_prepared_chain(kernels):
+    """wsm_chain_plan, computed on the host alone, reports the plan that
+    wsm_chain_create makes on this GPU, task by task."""
+    shapes = [(1, 1024, 4096, -1), (16, 3072, 1024, 0), (64, 1024, 3072, 1), (8, 2048, 1024, -1), (2, 512, 2048, 3)]
+    tasks, specs = [], []
+    for i, (M, N, K, dep) in enumerate(shapes):
+        x = synth.make_x(M, K, 50 + i).to(DEV)
+        w = synth.make_w(N, K, 60 + i).to(DEV)
+        tasks.append(wsm.Task(x, w, torch.empty(M, N, dtype=torch.bfloat16, device=DEV), dep=dep))
+        specs.append(dict(M=M, N=N, K=K, dep=dep))
+    ch = wsm.Chain(tasks, kernels=kernels)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plans, n_kernels = wsm.chain_plan(specs, num_sms=sms, kernels=kernels)
+    assert n_kernels == (3 if kernels == wsm.CHAIN_KERNELS_SPLIT else 1)
+    for i, p in enumerate(plans):
+        tp = ch.task_plan(i)
+        assert all(tp[k] == p[k] for k in tp), (i, tp, p)
+    ch.close()
+
+
 @pytest.mark.filterwarnings("ignore:The CUDA Graph is empty")
 def test_gemm_chain_in_graph_survives_cache_drop():
     """gemm_chain inside a CUDA graph: a list met for the first time during

@@ -21,7 +21,7 @@ __all__ = [
     "LIB_PATH", "WSM_OK", "WSM_ERR_INVALID", "WSM_ERR_UNSUPPORTED", "WSM_ERR_ALIGN", "WSM_ERR_NOMEM",
     "WSM_ERR_CUDA", "WSM_ERR_TIMEOUT", "PATH_AUTO", "PATH_STREAM", "PATH_UMMA", "ORDER_AUTO", "ORDER_M_MAJOR",
     "ORDER_NAIVE", "L2_AUTO", "L2_EVICT_FIRST", "L2_NORMAL", "FLAG_W_READONLY", "FLAG_NO_PDL", "WsmError", "lib", "skinny_gemm", "plan",
-    "workspace_bytes", "stream_status", "Task", "Chain", "gemm_chain", "chain_validate", "last_error",
+    "workspace_bytes", "stream_status", "Task", "Chain", "gemm_chain", "chain_validate", "chain_plan", "last_error",
     "skinny_gemm_noalloc",
     "abi_version", "HEADER_SYMBOLS",
 ]
@@ -37,11 +37,13 @@ L2_AUTO, L2_EVICT_FIRST, L2_NORMAL = 0, 1, 2
 FLAG_W_READONLY, FLAG_NO_PDL = 1, 2
 EPI_NONE, EPI_SILU_MUL, EPI_RESIDUAL = 0, 1, 2
 CHAIN_KERNELS_AUTO, CHAIN_KERNELS_ONE, CHAIN_KERNELS_SPLIT = 0, 1, 2
+K_ORDER_AUTO, K_ORDER_INCREASING, K_ORDER_ROTATED = 0, 1, 2
 
 # Every function include/wsm.h declares (checked by the CPU tests).
 HEADER_SYMBOLS = (
     "skinny_gemm", "skinny_gemm_ex", "wsm_plan", "wsm_workspace_bytes", "wsm_stream_status", "skinny_gemm_noalloc",
-    "wsm_chain_create", "wsm_chain_run", "wsm_chain_status", "wsm_chain_task_plan", "wsm_chain_trace",
+    "wsm_chain_plan", "wsm_chain_create", "wsm_chain_run", "wsm_chain_status", "wsm_chain_task_plan",
+    "wsm_chain_trace",
     "wsm_chain_destroy",
     "gemm_chain", "wsm_chain_validate", "wsm_last_error", "wsm_abi_version",
 )
@@ -77,6 +79,11 @@ class _Task(ctypes.Structure):
     _fields_ = [("X", ctypes.c_void_p), ("W", ctypes.c_void_p), ("Y", ctypes.c_void_p),
                 ("M", ctypes.c_int), ("N", ctypes.c_int), ("K", ctypes.c_int), ("dep", ctypes.c_int),
                 ("Yf32", ctypes.c_void_p), ("epilogue", ctypes.c_int), ("R", ctypes.c_void_p), ("dep_cols", ctypes.c_int)]
+
+
+class _ChainTaskInfo(ctypes.Structure):
+    _fields_ = [("plan", _PlanInfo), ("kernel", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int),
+                ("k_order", ctypes.c_int), ("dep_ring_stages", ctypes.c_int)]
 
 
 class _ChainOpts(ctypes.Structure):
@@ -126,6 +133,9 @@ def lib() -> ctypes.CDLL:
         L.wsm_chain_destroy.restype = None
         L.gemm_chain.argtypes = [ctypes.POINTER(_Task), i, vp]
         L.gemm_chain.restype = st
+        L.wsm_chain_plan.argtypes = [ctypes.POINTER(_Task), i, ctypes.POINTER(_ChainOpts), i,
+                                     ctypes.POINTER(_ChainTaskInfo), ctypes.POINTER(ctypes.c_int)]
+        L.wsm_chain_plan.restype = st
         L.wsm_chain_validate.argtypes = [ctypes.POINTER(_Task), i]
         L.wsm_chain_validate.restype = st
         L.wsm_last_error.argtypes = []
@@ -311,6 +321,57 @@ def chain_validate(tasks) -> None:
     _check(lib().wsm_chain_validate(arr, len(tasks)), "wsm_chain_validate")
 
 
+def _chain_opts(path=PATH_AUTO, grid=0, timeout_ns=0, trace=False, debug_unmet_dependency=False, flags=0,
+                stage_k=0, unit_stages=0, tail_tiles=0, tail_unit_stages=0, l2_prefetch_stages=0,
+                counter_groups=0, kernels=0, tile_rows=0, k_order=0, dep_ring_stages=0) -> "_ChainOpts":
+    o = _ChainOpts()
+    o.path, o.grid, o.timeout_ns, o.trace = path, grid, timeout_ns, 1 if trace else 0
+    o.debug_unmet_dependency = 1 if debug_unmet_dependency else 0
+    o.flags, o.stage_k = flags, stage_k
+    o.unit_stages, o.tail_tiles, o.tail_unit_stages = unit_stages, tail_tiles, tail_unit_stages
+    o.l2_prefetch_stages = l2_prefetch_stages
+    o.counter_groups = counter_groups
+    o.kernels = kernels
+    o.tile_rows = tile_rows
+    o.k_order = k_order
+    o.dep_ring_stages = dep_ring_stages
+    return o
+
+
+def chain_plan(specs, num_sms: int = 148, **opts):
+    """The plan gemm_chain / Chain would make (pure host computation, no GPU
+    needed): specs is a sequence of dicts with keys M, N, K and optionally
+    dep, epilogue, dep_cols.  The C call gets placeholder addresses (never
+    dereferenced; a dep_cols task's X is its dependency's Y).  Returns
+    (list of per-task dicts: the plan fields plus kernel, l2_prefetch_stages,
+    k_order, dep_ring_stages; number of kernels)."""
+    n = len(specs)
+    arr = (_Task * n)()
+    base = 1 << 32
+    for i, t in enumerate(specs):
+        x, w, y = base + (3 * i) * (1 << 24), base + (3 * i + 1) * (1 << 24), base + (3 * i + 2) * (1 << 24)
+        dep = t.get("dep", -1)
+        if t.get("dep_cols"):
+            x = arr[dep].Y
+        arr[i].X, arr[i].W, arr[i].Y = x, w, y
+        arr[i].M, arr[i].N, arr[i].K, arr[i].dep = t["M"], t["N"], t["K"], dep
+        arr[i].Yf32 = None
+        arr[i].epilogue = t.get("epilogue", EPI_NONE)
+        arr[i].R = base - (1 << 24) if arr[i].epilogue == EPI_RESIDUAL else None
+        arr[i].dep_cols = 1 if t.get("dep_cols") else 0
+    out = (_ChainTaskInfo * max(n, 1))()
+    nk = ctypes.c_int(0)
+    o = _chain_opts(**opts)
+    _check(lib().wsm_chain_plan(arr, n, ctypes.byref(o), num_sms, out, ctypes.byref(nk)), "wsm_chain_plan")
+    res = []
+    for i in range(n):
+        d = {f: getattr(out[i].plan, f) for f, _ in _PlanInfo._fields_}
+        d.update(kernel=out[i].kernel, l2_prefetch_stages=out[i].l2_prefetch_stages, k_order=out[i].k_order,
+                 dep_ring_stages=out[i].dep_ring_stages)
+        res.append(d)
+    return res, nk.value
+
+
 class Chain:
     """A prepared chain of GEMMs run as one persistent kernel."""
 
@@ -324,17 +385,11 @@ class Chain:
             _check_operand(f"tasks[{i}].y", t.y)
         self.tasks = list(tasks)  # keeps the tensors alive
         arr = _tasks_array(self.tasks)
-        o = _ChainOpts()
-        o.path, o.grid, o.timeout_ns, o.trace = path, grid, timeout_ns, 1 if trace else 0
-        o.debug_unmet_dependency = 1 if debug_unmet_dependency else 0
-        o.flags, o.stage_k = flags, stage_k
-        o.unit_stages, o.tail_tiles, o.tail_unit_stages = unit_stages, tail_tiles, tail_unit_stages
-        o.l2_prefetch_stages = l2_prefetch_stages
-        o.counter_groups = counter_groups
-        o.kernels = kernels
-        o.tile_rows = tile_rows
-        o.k_order = k_order
-        o.dep_ring_stages = dep_ring_stages
+        o = _chain_opts(path=path, grid=grid, timeout_ns=timeout_ns, trace=trace,
+                        debug_unmet_dependency=debug_unmet_dependency, flags=flags, stage_k=stage_k,
+                        unit_stages=unit_stages, tail_tiles=tail_tiles, tail_unit_stages=tail_unit_stages,
+                        l2_prefetch_stages=l2_prefetch_stages, counter_groups=counter_groups, kernels=kernels,
+                        tile_rows=tile_rows, k_order=k_order, dep_ring_stages=dep_ring_stages)
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

@@ -713,6 +713,206 @@ wsm_status validate_tasks(const wsm_task *tasks, int n) {
     return WSM_OK;
 }
 
+// A chain's plan, computed on the host alone (no CUDA call): kernel path,
+// hybrid split, each task's geometry and work units, the shared ring and the
+// chain-wide settings.  wsm_chain_create builds the device state from it;
+// wsm_chain_plan reports it.
+struct ChainPlan {
+    int path = 0;
+    std::vector<std::pair<int, int>> parts;  // hybrid dispatch: [first, end) of each kernel's tasks; empty: one kernel
+    std::vector<Geo> geos;                   // one kernel: each task's plan
+    Geo ring;                                // one kernel: the stage geometry all tasks share
+    int grid = 0;
+    int groups = 1;
+    int prefetch_stages = 0, k_rotate = 0, dep_ring_stages = 0;
+};
+
+// Tasks [a, b) of a chain as a chain of their own: a dependency inside the
+// range is renumbered; one on an earlier task is met by stream order (the
+// earlier kernel has completed) and dropped.
+std::vector<wsm_task> sub_chain(const wsm_task *tasks, int a, int b) {
+    std::vector<wsm_task> sub(tasks + a, tasks + b);
+    for (wsm_task &t : sub) {
+        if (t.dep >= a) {
+            t.dep -= a;
+        } else {
+            t.dep = -1;
+            t.dep_cols = 0;
+        }
+    }
+    return sub;
+}
+
+// Options of one kernel of a hybrid-dispatch chain.
+wsm_chain_opts part_opts(const wsm_chain_opts &o) {
+    wsm_chain_opts so = o;
+    so.path = WSM_PATH_UMMA;
+    so.kernels = WSM_CHAIN_KERNELS_ONE;
+    return so;
+}
+
+wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, int sms, ChainPlan &cp) {
+    cp = ChainPlan{};
+    wsm_status st;
+    if (opts->path < 0 || opts->path > WSM_PATH_UMMA) return fail(WSM_ERR_INVALID, "bad chain path %d", opts->path);
+    if (opts->kernels < WSM_CHAIN_KERNELS_AUTO || opts->kernels > WSM_CHAIN_KERNELS_SPLIT)
+        return fail(WSM_ERR_INVALID, "bad kernels option %d", opts->kernels);
+    if (opts->flags & ~(WSM_FLAG_W_READONLY | WSM_FLAG_NO_PDL))
+        return fail(WSM_ERR_INVALID, "bad chain flags %#x", opts->flags);
+    if (opts->l2_prefetch_stages < -1)
+        return fail(WSM_ERR_INVALID, "bad l2_prefetch_stages %d", opts->l2_prefetch_stages);
+    if (opts->counter_groups < 0) return fail(WSM_ERR_INVALID, "bad counter_groups %d", opts->counter_groups);
+    if (opts->k_order < 0 || opts->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", opts->k_order);
+    if (opts->dep_ring_stages < -1) return fail(WSM_ERR_INVALID, "bad dep_ring_stages %d", opts->dep_ring_stages);
+    int maxM = 0;
+    for (int i = 0; i < n; ++i) maxM = std::max(maxM, tasks[i].M);
+    // AUTO: the FMA path only if it is the automatic choice for every task at the chain's largest M
+    int path = opts->path;
+    if (path == WSM_PATH_AUTO) {
+        path = WSM_PATH_STREAM;
+        for (int i = 0; i < n; ++i)
+            if (auto_path(maxM, 2ll * tasks[i].N * tasks[i].K) != WSM_PATH_STREAM) path = WSM_PATH_UMMA;
+    }
+    if (path == WSM_PATH_STREAM && maxM > 8) return fail(WSM_ERR_UNSUPPORTED, "the FMA path takes M <= 8 (max M=%d)", maxM);
+    cp.path = path;
+
+    // Hybrid dispatch.  One kernel sizes its ring stages for the widest X tile: with M > 32 tasks in
+    // the chain, tasks of M <= 32 get 2 stages of 96 KB instead of 3 of 72 KB, about 5 % slower
+    // (measured on B200).  Split into one kernel per run of consecutive tasks of one kind, they keep
+    // their own ring; each extra kernel boundary costs up to about 20 us (the next task no longer
+    // overlaps the previous one's tail).  AUTO splits when the narrow tasks carry more than 1.5 GB of
+    // weights per extra kernel (measured: a 1.9 GB narrow run next to one M = 64 task gains 5 % from
+    // the split; 12 alternating runs of 0.3-0.4 GB lose 27 %).  A dependency that crosses kernels
+    // is met by stream order.
+    if (path == WSM_PATH_UMMA && opts->kernels != WSM_CHAIN_KERNELS_ONE) {
+        auto wide = [&](int i) { return (tasks[i].M + 15) / 16 * 16 > 32; };
+        int kinds = 0, segments = 1;
+        double narrow_bytes = 0;
+        for (int i = 0; i < n; ++i) {
+            kinds |= wide(i) ? 2 : 1;
+            if (i > 0 && wide(i) != wide(i - 1)) ++segments;
+            if (!wide(i)) narrow_bytes += 2.0 * tasks[i].N * (double)tasks[i].K;
+        }
+        const bool split = kinds == 3 && (opts->kernels == WSM_CHAIN_KERNELS_SPLIT ||
+                                          narrow_bytes > 1.5e9 * (segments - 1));
+        if (split) {
+            for (int a = 0, b; a < n; a = b) {
+                for (b = a + 1; b < n && wide(b) == wide(a); ++b) {}
+                cp.parts.push_back({a, b});
+            }
+            return WSM_OK;
+        }
+    }
+
+    const int groups = opts->counter_groups > 1 ? opts->counter_groups : 1;
+    if (groups > 1)
+        for (int i = 0; i < n; ++i)
+            if (tasks[i].dep_cols)
+                return fail(WSM_ERR_UNSUPPORTED, "task %d: two-level readiness does not combine with dep_cols", i);
+    // per-task geometry; the ring is sized for the widest task
+    std::vector<Geo> geos(n);
+    wsm_opts to{};
+    to.path = path;
+    to.grid = opts->grid;
+    // one stage geometry for the whole chain (the ring and the kernel's boxes per stage are shared):
+    // wide tiles only if every task would take them
+    bool chain_wide = false;
+    if (path == WSM_PATH_UMMA) {
+        if (opts->tile_rows != 0 && opts->tile_rows != kUmmaRows && opts->tile_rows != 2 * kUmmaRows)
+            return fail(WSM_ERR_UNSUPPORTED, "tile_rows must be 0, 128 or 256 (got %d)", opts->tile_rows);
+        chain_wide = opts->tile_rows == 2 * kUmmaRows;
+        if (opts->tile_rows == 0) {
+            chain_wide = true;
+            for (int i = 0; i < n; ++i) chain_wide = chain_wide && auto_wide((tasks[i].M + 15) / 16 * 16);
+        }
+        to.tile_rows = chain_wide ? 2 * kUmmaRows : kUmmaRows;
+    } else {
+        // FMA path: one tile height for the chain's ring, the one with the lower modelled total over the
+        // tasks (see auto_fma_rows)
+        if (opts->tile_rows != 0 && opts->tile_rows != 16 && opts->tile_rows != 32)
+            return fail(WSM_ERR_UNSUPPORTED, "tile_rows must be 0, 16 or 32 on the FMA path (got %d)", opts->tile_rows);
+        to.tile_rows = opts->tile_rows;
+        if (to.tile_rows == 0) {
+            const int ctas = (opts->grid > 0) ? std::min(opts->grid, sms) : sms;
+            double c16 = 0, c32 = 0;
+            for (int i = 0; i < n; ++i) {
+                c16 += fma_cost_us(16, tasks[i].N, tasks[i].K, ctas);
+                c32 += fma_cost_us(32, tasks[i].N, tasks[i].K, ctas);
+            }
+            to.tile_rows = c32 < c16 ? 32 : 16;
+        }
+    }
+    to.stage_k = (path == WSM_PATH_UMMA) ? (opts->stage_k ? opts->stage_k
+                                                           : auto_stage_k((maxM + 15) / 16 * 16, chain_wide))
+                                          : 0;
+    const int chain_mmax = (path == WSM_PATH_STREAM) ? pow2ceil(maxM) : 0;
+    for (int i = 0; i < n; ++i) {
+        if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, sms, &to, geos[i], chain_mmax)) != WSM_OK)
+            return fail(st, "task %d: %s", i, g_err.c_str());
+    }
+    // one grid for the whole chain (make_geo clamps it per task to the task's stages)
+    int chain_grid = (opts->grid > 0) ? std::min(opts->grid, sms) : sms;
+    for (auto &g : geos) g.grid = chain_grid;
+    Geo ring = geos[0];
+    if (path == WSM_PATH_STREAM) {
+        stream_geo(pow2ceil(maxM), ring, to.tile_rows);
+    } else {
+        int tmp = 16;
+        for (auto &g : geos) tmp = std::max(tmp, g.t_mpad);
+        ring.x_stride = tmp * kUmmaBK * 2;
+        ring.x_off = (ring.wide ? 2 : 1) * ring.kps * kUmmaRows * kUmmaBK * 2;
+        ring.stage_bytes = ring.x_off + ring.kps * ring.x_stride;
+        if (ring.stage_bytes > kRingBudget)
+            return fail(WSM_ERR_UNSUPPORTED, "the chain's pipeline stage of %d bytes does not fit in shared memory",
+                        ring.stage_bytes);
+    }
+    ring.stages = std::min(kMaxStages, kRingBudget / ring.stage_bytes);
+    for (int i = 0; i < n; ++i)
+        if (geos[i].kps != ring.kps || geos[i].tile_k != ring.tile_k || geos[i].wide != ring.wide)
+            return fail(WSM_ERR_INVALID, "task %d: stage geometry differs from the chain's", i);  // cannot happen
+    cp.prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, path);
+    if (opts->l2_prefetch_stages == 0 && path == WSM_PATH_UMMA) {
+        bool deps = false;
+        for (int i = 0; i < n; ++i) deps = deps || tasks[i].dep >= 0;
+        if (!deps && ring.x_stride <= 16 * kUmmaBK * 2) cp.prefetch_stages = kDefaultPrefetchStagesIndependentChain;
+    }
+    // auto: rotated on the tensor-core path.  A chain's units are long (whole tiles where later work can
+    // overlap them) and start together, and in increasing order every CTA would read the same columns
+    // of its weight rows at the same time.  Measured on B200: the decode step of 20 GEMMs 308.4 ->
+    // 300.3 us, the M = 32 / 64 set 133.0 -> 128.0 us, the 36 x 4 layer chain 3335 -> 3296 us, the
+    // fused data chain 3474 -> 3448 us, the K = 7168 / 8192 set within 0.4 %.  Single launches keep
+    // the increasing order (rotated: 0.5-2.5 % slower on 8 of 10 decode shapes).  Per-column waits
+    // read their dependency's chunks in increasing order, so those chains keep it too.
+    bool any_dep_cols = false;
+    for (int i = 0; i < n; ++i) any_dep_cols = any_dep_cols || tasks[i].dep_cols;
+    cp.k_rotate = (opts->k_order == 2 || (opts->k_order == 0 && path == WSM_PATH_UMMA && !any_dep_cols)) ? 1 : 0;
+    // measured on B200 (36 x 4 dependent chain at M = 16, 4 prefetch stages): 1 stage ahead of the
+    // dependency is 2 % faster than 2 and 4 % faster than the whole ring (3), and none at all is 2 %
+    // slower than 1.  The FMA path keeps its whole ring (unmeasured).
+    cp.dep_ring_stages = opts->dep_ring_stages > 0 ? opts->dep_ring_stages
+                          : (opts->dep_ring_stages == 0 && path == WSM_PATH_UMMA) ? 1 : 0;
+
+    // work units per task, planned for the chain's grid (K-range-first units, no tail, for a task that
+    // waits per column); automatic units grow with the later work a task's units can overlap: the
+    // stages of the tasks after it, up to the next one that waits on a dependency
+    std::vector<long long> later(n, 0);
+    for (int i = n - 2; i >= 0; --i)
+        later[i] = tasks[i + 1].dep >= 0 ? 0 : later[i + 1] + geos[i + 1].tiles() * (long long)geos[i + 1].kb;
+    for (int i = 0; i < n; ++i) {
+        const bool grow = opts->unit_stages == 0 && !tasks[i].dep_cols && groups <= 1;
+        const int unit_stages = grow ? chain_unit_stages(geos[i], chain_grid, later[i]) : opts->unit_stages;
+        if ((st = plan_units(geos[i], chain_grid, unit_stages,
+                             (tasks[i].dep_cols || groups > 1) ? -1 : opts->tail_tiles, opts->tail_unit_stages)) !=
+            WSM_OK)
+            return fail(st, "task %d: %s", i, g_err.c_str());
+    }
+    cp.geos = geos;
+    cp.ring = ring;
+    cp.grid = chain_grid;
+    cp.groups = groups;
+    return WSM_OK;
+}
+
 }  // namespace
 }  // namespace wsm
 
@@ -850,6 +1050,49 @@ wsm_status wsm_chain_validate(const wsm_task *tasks, int n_tasks) {
     return st;
 }
 
+wsm_status wsm_chain_plan(const wsm_task *tasks, int n, const wsm_chain_opts *opts, int num_sms,
+                          wsm_chain_task_info *out, int *n_kernels) {
+    if (!out) return fail(WSM_ERR_INVALID, "out must be non-null");
+    wsm_status st = validate_tasks(tasks, n);
+    if (st != WSM_OK) return st;
+    if (num_sms < 1) return fail(WSM_ERR_INVALID, "num_sms must be positive");
+    wsm_chain_opts zo{};
+    if (!opts) opts = &zo;
+    ChainPlan cp;
+    if ((st = plan_chain(tasks, n, opts, num_sms, cp)) != WSM_OK) return st;
+    auto report = [&](const ChainPlan &kp, int first, int k) {
+        for (size_t i = 0; i < kp.geos.size(); ++i) {
+            Geo g = kp.geos[i];
+            g.stages = kp.ring.stages;
+            g.stage_bytes = kp.ring.stage_bytes;
+            wsm_chain_task_info &o = out[first + (int)i];
+            memset(&o, 0, sizeof o);
+            fill_plan_info(g, &o.plan);
+            o.plan.workspace_bytes = 0;  // a chain owns its scratch
+            o.kernel = k;
+            o.l2_prefetch_stages = kp.prefetch_stages;
+            o.k_order = kp.k_rotate ? WSM_K_ORDER_ROTATED : WSM_K_ORDER_INCREASING;
+            o.dep_ring_stages = kp.dep_ring_stages;
+        }
+    };
+    if (cp.parts.empty()) {
+        report(cp, 0, 0);
+    } else {
+        for (size_t k = 0; k < cp.parts.size(); ++k) {
+            const int a = cp.parts[k].first, b = cp.parts[k].second;
+            std::vector<wsm_task> sub = sub_chain(tasks, a, b);
+            const wsm_chain_opts so = part_opts(*opts);
+            ChainPlan sp;
+            if ((st = plan_chain(sub.data(), b - a, &so, num_sms, sp)) != WSM_OK)
+                return fail(st, "tasks %d..%d: %s", a, b - 1, g_err.c_str());
+            report(sp, a, (int)k);
+        }
+    }
+    if (n_kernels) *n_kernels = cp.parts.empty() ? 1 : (int)cp.parts.size();
+    g_err.clear();
+    return WSM_OK;
+}
+
 wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *opts, wsm_chain **out) {
     if (!out) return fail(WSM_ERR_INVALID, "out must be non-null");
     *out = nullptr;
@@ -857,79 +1100,39 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     if (st != WSM_OK) return st;
     wsm_chain_opts zo{};
     if (!opts) opts = &zo;
-    if (opts->path < 0 || opts->path > WSM_PATH_UMMA) return fail(WSM_ERR_INVALID, "bad chain path %d", opts->path);
     int dev = 0;
     WSM_CUDA(cudaGetDevice(&dev));
     DevInfo *d;
     if ((st = dev_info(dev, &d)) != WSM_OK) return st;
-    int maxM = 0;
-    for (int i = 0; i < n; ++i) maxM = std::max(maxM, tasks[i].M);
-    // AUTO: the FMA path only if it is the automatic choice for every task at the chain's largest M
-    int path = opts->path;
-    if (path == WSM_PATH_AUTO) {
-        path = WSM_PATH_STREAM;
-        for (int i = 0; i < n; ++i)
-            if (auto_path(maxM, 2ll * tasks[i].N * tasks[i].K) != WSM_PATH_STREAM) path = WSM_PATH_UMMA;
-    }
-    if (path == WSM_PATH_STREAM && maxM > 8) return fail(WSM_ERR_UNSUPPORTED, "the FMA path takes M <= 8 (max M=%d)", maxM);
+    ChainPlan cp;
+    if ((st = plan_chain(tasks, n, opts, d->sms, cp)) != WSM_OK) return st;
 
-    // Hybrid dispatch.  One kernel sizes its ring stages for the widest X tile: with M > 32 tasks in
-    // the chain, tasks of M <= 32 get 2 stages of 96 KB instead of 3 of 72 KB, about 5 % slower
-    // (measured on B200).  Split into one kernel per run of consecutive tasks of one kind, they keep
-    // their own ring; each extra kernel boundary costs up to about 20 us (the next task no longer
-    // overlaps the previous one's tail).  AUTO splits when the narrow tasks carry more than 1.5 GB of
-    // weights per extra kernel (measured: a 1.9 GB narrow run next to one M = 64 task gains 5 % from
-    // the split; 12 alternating runs of 0.3-0.4 GB lose 27 %).  A dependency that crosses kernels
-    // is met by stream order.
-    if (opts->kernels < WSM_CHAIN_KERNELS_AUTO || opts->kernels > WSM_CHAIN_KERNELS_SPLIT)
-        return fail(WSM_ERR_INVALID, "bad kernels option %d", opts->kernels);
-    if (path == WSM_PATH_UMMA && opts->kernels != WSM_CHAIN_KERNELS_ONE) {
-        auto wide = [&](int i) { return (tasks[i].M + 15) / 16 * 16 > 32; };
-        int kinds = 0, segments = 1;
-        double narrow_bytes = 0;
-        for (int i = 0; i < n; ++i) {
-            kinds |= wide(i) ? 2 : 1;
-            if (i > 0 && wide(i) != wide(i - 1)) ++segments;
-            if (!wide(i)) narrow_bytes += 2.0 * tasks[i].N * (double)tasks[i].K;
-        }
-        const bool split = kinds == 3 && (opts->kernels == WSM_CHAIN_KERNELS_SPLIT ||
-                                          narrow_bytes > 1.5e9 * (segments - 1));
-        if (split) {
-            std::unique_ptr<wsm_chain> parent(new wsm_chain());
-            parent->device = dev;
-            parent->n = n;
-            parent->tasks.assign(tasks, tasks + n);
-            auto cleanup = [&]() {
-                for (wsm_chain *c : parent->parts) wsm_chain_destroy(c);
-                parent->parts.clear();
-            };
-            for (int a = 0, b; a < n; a = b) {
-                for (b = a + 1; b < n && wide(b) == wide(a); ++b) {}
-                std::vector<wsm_task> sub(tasks + a, tasks + b);
-                for (wsm_task &t : sub) {
-                    if (t.dep >= a) {
-                        t.dep -= a;
-                    } else {  // met by stream order: the earlier kernel has completed
-                        t.dep = -1;
-                        t.dep_cols = 0;
-                    }
-                }
-                wsm_chain_opts so = *opts;
-                so.path = WSM_PATH_UMMA;
-                so.kernels = WSM_CHAIN_KERNELS_ONE;
-                so.trace = 0;
-                wsm_chain *part = nullptr;
-                if ((st = wsm_chain_create(sub.data(), b - a, &so, &part)) != WSM_OK) {
-                    cleanup();
-                    return fail(st, "tasks %d..%d: %s", a, b - 1, g_err.c_str());
-                }
-                parent->parts.push_back(part);
-                parent->part_first.push_back(a);
+    if (!cp.parts.empty()) {
+        // hybrid dispatch: one chain per run of tasks of one X width, run back to back
+        std::unique_ptr<wsm_chain> parent(new wsm_chain());
+        parent->device = dev;
+        parent->n = n;
+        parent->tasks.assign(tasks, tasks + n);
+        auto cleanup = [&]() {
+            for (wsm_chain *c : parent->parts) wsm_chain_destroy(c);
+            parent->parts.clear();
+        };
+        for (const auto &ab : cp.parts) {
+            const int a = ab.first, b = ab.second;
+            std::vector<wsm_task> sub = sub_chain(tasks, a, b);
+            wsm_chain_opts so = part_opts(*opts);
+            so.trace = 0;
+            wsm_chain *part = nullptr;
+            if ((st = wsm_chain_create(sub.data(), b - a, &so, &part)) != WSM_OK) {
+                cleanup();
+                return fail(st, "tasks %d..%d: %s", a, b - 1, g_err.c_str());
             }
-            *out = parent.release();
-            g_err.clear();
-            return WSM_OK;
+            parent->parts.push_back(part);
+            parent->part_first.push_back(a);
         }
+        *out = parent.release();
+        g_err.clear();
+        return WSM_OK;
     }
 
     std::unique_ptr<wsm_chain> ch(new wsm_chain());
@@ -938,119 +1141,15 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     ch->tasks.assign(tasks, tasks + n);
     ch->dep_timeout_ns = opts->timeout_ns ? opts->timeout_ns : kDefaultDepTimeoutNs;
     ch->dep_target_extra = opts->debug_unmet_dependency ? 0x40000000u : 0u;
-    if (opts->flags & ~(WSM_FLAG_W_READONLY | WSM_FLAG_NO_PDL))
-        return fail(WSM_ERR_INVALID, "bad chain flags %#x", opts->flags);
     ch->pdl = pdl_mode(opts->flags);
-    if (opts->l2_prefetch_stages < -1)
-        return fail(WSM_ERR_INVALID, "bad l2_prefetch_stages %d", opts->l2_prefetch_stages);
-    if (opts->counter_groups < 0) return fail(WSM_ERR_INVALID, "bad counter_groups %d", opts->counter_groups);
-    const int groups = opts->counter_groups > 1 ? opts->counter_groups : 1;
-    if (groups > 1)
-        for (int i = 0; i < n; ++i)
-            if (tasks[i].dep_cols)
-                return fail(WSM_ERR_UNSUPPORTED, "task %d: two-level readiness does not combine with dep_cols", i);
-
-    // per-task geometry; the ring is sized for the widest task
-    std::vector<Geo> geos(n);
-    wsm_opts to{};
-    to.path = path;
-    to.grid = opts->grid;
-    // one stage geometry for the whole chain (the ring and the kernel's boxes per stage are shared):
-    // wide tiles only if every task would take them
-    bool chain_wide = false;
-    if (path == WSM_PATH_UMMA) {
-        if (opts->tile_rows != 0 && opts->tile_rows != kUmmaRows && opts->tile_rows != 2 * kUmmaRows)
-            return fail(WSM_ERR_UNSUPPORTED, "tile_rows must be 0, 128 or 256 (got %d)", opts->tile_rows);
-        chain_wide = opts->tile_rows == 2 * kUmmaRows;
-        if (opts->tile_rows == 0) {
-            chain_wide = true;
-            for (int i = 0; i < n; ++i) chain_wide = chain_wide && auto_wide((tasks[i].M + 15) / 16 * 16);
-        }
-        to.tile_rows = chain_wide ? 2 * kUmmaRows : kUmmaRows;
-    } else {
-        // FMA path: one tile height for the chain's ring, the one with the lower modelled total over the
-        // tasks (see auto_fma_rows)
-        if (opts->tile_rows != 0 && opts->tile_rows != 16 && opts->tile_rows != 32)
-            return fail(WSM_ERR_UNSUPPORTED, "tile_rows must be 0, 16 or 32 on the FMA path (got %d)", opts->tile_rows);
-        to.tile_rows = opts->tile_rows;
-        if (to.tile_rows == 0) {
-            const int ctas = (opts->grid > 0) ? std::min(opts->grid, d->sms) : d->sms;
-            double c16 = 0, c32 = 0;
-            for (int i = 0; i < n; ++i) {
-                c16 += fma_cost_us(16, tasks[i].N, tasks[i].K, ctas);
-                c32 += fma_cost_us(32, tasks[i].N, tasks[i].K, ctas);
-            }
-            to.tile_rows = c32 < c16 ? 32 : 16;
-        }
-    }
-    to.stage_k = (path == WSM_PATH_UMMA) ? (opts->stage_k ? opts->stage_k
-                                                           : auto_stage_k((maxM + 15) / 16 * 16, chain_wide))
-                                          : 0;
-    const int chain_mmax = (path == WSM_PATH_STREAM) ? pow2ceil(maxM) : 0;
-    for (int i = 0; i < n; ++i) {
-        if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, d->sms, &to, geos[i], chain_mmax)) != WSM_OK)
-            return fail(st, "task %d: %s", i, g_err.c_str());
-    }
-    // one grid for the whole chain (make_geo clamps it per task to the task's stages)
-    int chain_grid = (opts->grid > 0) ? std::min(opts->grid, d->sms) : d->sms;
-    for (auto &g : geos) g.grid = chain_grid;
-    Geo ring = geos[0];
-    if (path == WSM_PATH_STREAM) {
-        stream_geo(pow2ceil(maxM), ring, to.tile_rows);
-    } else {
-        int tmp = 16;
-        for (auto &g : geos) tmp = std::max(tmp, g.t_mpad);
-        ring.x_stride = tmp * kUmmaBK * 2;
-        ring.x_off = (ring.wide ? 2 : 1) * ring.kps * kUmmaRows * kUmmaBK * 2;
-        ring.stage_bytes = ring.x_off + ring.kps * ring.x_stride;
-        if (ring.stage_bytes > kRingBudget)
-            return fail(WSM_ERR_UNSUPPORTED, "the chain's pipeline stage of %d bytes does not fit in shared memory",
-                        ring.stage_bytes);
-    }
-    ring.stages = std::min(kMaxStages, kRingBudget / ring.stage_bytes);
-    for (int i = 0; i < n; ++i)
-        if (geos[i].kps != ring.kps || geos[i].tile_k != ring.tile_k || geos[i].wide != ring.wide)
-            return fail(WSM_ERR_INVALID, "task %d: stage geometry differs from the chain's", i);  // cannot happen
+    const int groups = cp.groups;
+    const int chain_grid = cp.grid;
+    std::vector<Geo> &geos = cp.geos;
+    const Geo &ring = cp.ring;
     ch->geo = ring;
-    ch->prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, path);
-    if (opts->l2_prefetch_stages == 0 && path == WSM_PATH_UMMA) {
-        bool deps = false;
-        for (int i = 0; i < n; ++i) deps = deps || tasks[i].dep >= 0;
-        if (!deps && ring.x_stride <= 16 * kUmmaBK * 2) ch->prefetch_stages = kDefaultPrefetchStagesIndependentChain;
-    }
-    if (opts->k_order < 0 || opts->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", opts->k_order);
-    // auto: rotated on the tensor-core path.  A chain's units are long (whole tiles where later work can
-    // overlap them) and start together, and in increasing order every CTA would read the same columns
-    // of its weight rows at the same time.  Measured on B200: the decode step of 20 GEMMs 308.4 ->
-    // 300.3 us, the M = 32 / 64 set 133.0 -> 128.0 us, the 36 x 4 layer chain 3335 -> 3296 us, the
-    // fused data chain 3474 -> 3448 us, the K = 7168 / 8192 set within 0.4 %.  Single launches keep
-    // the increasing order (rotated: 0.5-2.5 % slower on 8 of 10 decode shapes).  Per-column waits
-    // read their dependency's chunks in increasing order, so those chains keep it too.
-    bool any_dep_cols = false;
-    for (int i = 0; i < n; ++i) any_dep_cols = any_dep_cols || tasks[i].dep_cols;
-    ch->k_rotate = (opts->k_order == 2 || (opts->k_order == 0 && path == WSM_PATH_UMMA && !any_dep_cols)) ? 1 : 0;
-    // measured on B200 (36 x 4 dependent chain at M = 16, 4 prefetch stages): 1 stage ahead of the
-    // dependency is 2 % faster than 2 and 4 % faster than the whole ring (3), and none at all is 2 %
-    // slower than 1.  The FMA path keeps its whole ring (unmeasured).
-    if (opts->dep_ring_stages < -1)
-        return fail(WSM_ERR_INVALID, "bad dep_ring_stages %d", opts->dep_ring_stages);
-    ch->dep_ring_stages = opts->dep_ring_stages > 0 ? opts->dep_ring_stages
-                          : (opts->dep_ring_stages == 0 && path == WSM_PATH_UMMA) ? 1 : 0;
-
-    // work units per task, planned for the chain's grid (K-range-first units, no tail, for a task that
-    // waits per column); automatic units grow with the later work a task's units can overlap: the
-    // stages of the tasks after it, up to the next one that waits on a dependency
-    std::vector<long long> later(n, 0);
-    for (int i = n - 2; i >= 0; --i)
-        later[i] = tasks[i + 1].dep >= 0 ? 0 : later[i + 1] + geos[i + 1].tiles() * (long long)geos[i + 1].kb;
-    for (int i = 0; i < n; ++i) {
-        const bool grow = opts->unit_stages == 0 && !tasks[i].dep_cols && groups <= 1;
-        const int unit_stages = grow ? chain_unit_stages(geos[i], chain_grid, later[i]) : opts->unit_stages;
-        if ((st = plan_units(geos[i], chain_grid, unit_stages,
-                             (tasks[i].dep_cols || groups > 1) ? -1 : opts->tail_tiles, opts->tail_unit_stages)) !=
-            WSM_OK)
-            return fail(st, "task %d: %s", i, g_err.c_str());
-    }
+    ch->prefetch_stages = cp.prefetch_stages;
+    ch->k_rotate = cp.k_rotate;
+    ch->dep_ring_stages = cp.dep_ring_stages;
     ch->task_geo = geos;
     for (Geo &g : ch->task_geo) {
         g.stages = ring.stages;
