@@ -144,7 +144,8 @@ typedef struct {
     int tail_unit_stages; /* pipeline stages per tail unit, 0 = auto */
     int l2_prefetch_stages; /* W pipeline stages per CTA prefetched into L2 while the
                                CTA waits for the previous kernel (WSM_FLAG_W_READONLY):
-                               0 = auto, -1 = none */
+                               0 = auto (4 on the tensor-core path, none on the FMA
+                               path), -1 = none */
     int tile_rows;   /* W rows per tile, 0 = auto.  Tensor-core path: 128, or 256 (two
                         128-row halves share each X stage and accumulate into two
                         TMEM accumulators, so X is re-read half as often).  FMA
