@@ -188,28 +188,69 @@ typedef struct {
     size_t workspace_bytes;
 } wsm_plan_info;
 
-/* Y = X . W^T, automatic plan.  Device pointers; asynchronous on `stream`. */
+/* Y = X . W^T, automatic plan.  Device pointers; asynchronous on `stream`.
+ * The decode GEMM of the FlyDSL article (section "Was ist GEMM und die
+ * Decode-Phase eines LLMs?"), computed as inter-CTA split-K over work units
+ * with an in-order reduction, intra-CTA K-slicing and a multi-stage shared-
+ * memory pipeline (its section "Drei Techniken von FlyDSL im AITER-Framework").
+ * Errors: WSM_ERR_INVALID / _UNSUPPORTED / _ALIGN for bad arguments (nothing
+ * queued), WSM_ERR_NOMEM if the stream's scratch must grow and cannot (or must
+ * grow during graph capture), WSM_ERR_CUDA for a failed launch.  A device-side
+ * time-out is reported later by wsm_stream_status. */
 wsm_status skinny_gemm(const void *X, const void *W, void *Y, int M, int N, int K,
                        wsm_stream_t stream);
 
-/* Same with options (opts may be NULL). */
+/* Same with options (opts may be NULL); passages as skinny_gemm, plus the
+ * Fleet reading notes' section 3f for the M-tile order and L2 policy options
+ * and section 3f / 7b for the fused SiLU*mul epilogue.  With opts->workspace
+ * the caller's buffer is used and nothing is allocated; a device-side time-out
+ * of such a call is reported by wsm_workspace_status. */
 wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, int K,
                           const wsm_opts *opts, wsm_stream_t stream);
 
 /* Pure host function (no CUDA calls): the plan for a shape on a GPU with
- * `num_sms` SMs.  Used by the tests and by wsm_workspace_bytes. */
+ * `num_sms` SMs -- path, tile geometry, split of each tile's K range into work
+ * units (the per-shape split factor of the FlyDSL article's split-K), ring
+ * depth, L2 policy.  Used by the tests and by wsm_workspace_bytes.  Errors as
+ * skinny_gemm's argument errors; `out` untouched on error. */
 wsm_status wsm_plan(int M, int N, int K, int num_sms, const wsm_opts *opts,
                     wsm_plan_info *out);
 
-/* Scratch a call with this shape needs on the current device (0 on error). */
+/* Scratch a call with this shape needs on the current device (0 on error,
+ * with wsm_last_error() set).  `opts` may be NULL: the same plan as
+ * skinny_gemm. */
 size_t wsm_workspace_bytes(int M, int N, int K, const wsm_opts *opts);
 
-/* Synchronise `stream`, then report whether a skinny_gemm call queued on it
- * with the library-owned workspace recorded a device-side time-out of a
- * bounded pipeline wait since the last check (which never happens in a
- * healthy run); clears the record.  *code = 0 or WSM_ERR_TIMEOUT; the return
- * value is WSM_ERR_TIMEOUT in the second case. */
+/* Device-side time-outs.  Every wait inside the kernels is bounded.  A wait
+ * that runs out (never in a healthy run) records a sticky error in the status
+ * words of the call's scratch, and the CTA that hit it abandons its work, so
+ * that call's outputs are incomplete.  When that launch ends, its last CTA
+ * repairs the counters it left mid-count, so the next call on the same scratch
+ * computes correct results.  The error stays recorded until one of the status
+ * queries below reads and clears it: each synchronises the stream, returns
+ * WSM_ERR_TIMEOUT once per recorded time-out (*code = WSM_ERR_TIMEOUT, message
+ * in wsm_last_error()) and WSM_OK (*code = 0) otherwise.  This follows the
+ * Fleet reading notes' section 2 on the runtime: the megakernel fails the call
+ * and leaves the retry to the framework. */
+
+/* skinny_gemm / skinny_gemm_ex calls with the library-owned workspace queued
+ * on `stream`, and skinny_gemm_noalloc calls on the current device (their
+ * array is shared by all streams). */
 wsm_status wsm_stream_status(wsm_stream_t stream, int *code);
+
+/* skinny_gemm_ex calls given this caller workspace (the pointer and size
+ * passed in wsm_opts).  WSM_ERR_INVALID / WSM_ERR_ALIGN for a null, misaligned
+ * or too small buffer. */
+wsm_status wsm_workspace_status(const void *workspace, size_t workspace_bytes, wsm_stream_t stream,
+                                int *code);
+
+/* Test hook, not for real use: each of the next `calls` launches of any entry
+ * point (a hybrid chain launches one kernel per part) makes its CTA 0 wait on
+ * a flag that nothing ever sets for `limit_ns` (at most 10 s), then record
+ * WSM_ERR_TIMEOUT and abandon its work -- a device-side time-out on demand,
+ * with no fault: every other wait stays bounded and the kernel ends.  calls =
+ * 0 cancels.  WSM_ERR_INVALID for calls < 0 or a limit outside (0, 10 s]. */
+wsm_status wsm_debug_stall(int calls, unsigned long long limit_ns);
 
 /* Bytes of the fixed scratch array skinny_gemm_noalloc uses on each device. */
 #define WSM_NOALLOC_SCRATCH_BYTES (16 << 20)
@@ -233,7 +274,11 @@ wsm_status wsm_stream_status(wsm_stream_t stream, int *code);
  *  - Every call shares the array.  Each call clears the part that must start
  *    at zero (queued on `stream`), but calls that overlap on the GPU -- on
  *    different streams, or on different host threads -- race on it; queue
- *    them on one stream. */
+ *    them on one stream.
+ *  - A device-side time-out is recorded in the array's status words and kept
+ *    across later calls until wsm_stream_status (with this device current)
+ *    reads it.
+ *  - After a device reset the next call looks the array's address up again. */
 wsm_status skinny_gemm_noalloc(const void *X, const void *W, void *Y, int M, int N, int K,
                                wsm_stream_t stream);
 
@@ -361,8 +406,9 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n_tasks, const wsm_chain_
 wsm_status wsm_chain_run(wsm_chain *chain, wsm_stream_t stream);
 
 /* Synchronise `stream`, then report the device-side status of the chain's
- * last run: WSM_OK, or WSM_ERR_TIMEOUT with *failed_task = the first task
- * whose wait ran out (may be NULL). */
+ * runs since the last check: WSM_OK, or WSM_ERR_TIMEOUT with *failed_task =
+ * the task whose wait ran out first (-1 when the wait was not a task's; may be
+ * NULL), clearing the record (see "Device-side time-outs" above). */
 wsm_status wsm_chain_status(wsm_chain *chain, wsm_stream_t stream, int *failed_task);
 
 /* The plan of task `task` of a prepared chain (the chain's grid, ring and
@@ -400,6 +446,13 @@ void wsm_chain_destroy(wsm_chain *chain);
  *    so the graph stays valid; up to 16 others are kept, then dropped
  *    together (dropping synchronises the device). */
 wsm_status gemm_chain(const wsm_task *tasks, int n_tasks, wsm_stream_t stream);
+
+/* Synchronise `stream`, then report whether a gemm_chain run on the current
+ * device recorded a device-side time-out since the last check: WSM_OK, or
+ * WSM_ERR_TIMEOUT with *failed_task = the waiting task's index in its list
+ * (-1 when not a task's wait; may be NULL), clearing the record.  Runs still
+ * queued on other streams are not waited for. */
+wsm_status gemm_chain_status(wsm_stream_t stream, int *failed_task);
 
 /* Validation only (pure host function, no CUDA calls). */
 wsm_status wsm_chain_validate(const wsm_task *tasks, int n_tasks);

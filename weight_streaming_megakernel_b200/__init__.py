@@ -22,7 +22,7 @@ __all__ = [
     "WSM_ERR_CUDA", "WSM_ERR_TIMEOUT", "PATH_AUTO", "PATH_STREAM", "PATH_UMMA", "ORDER_AUTO", "ORDER_M_MAJOR",
     "ORDER_NAIVE", "L2_AUTO", "L2_EVICT_FIRST", "L2_NORMAL", "FLAG_W_READONLY", "FLAG_NO_PDL", "WsmError", "lib", "skinny_gemm", "plan",
     "workspace_bytes", "stream_status", "Task", "Chain", "gemm_chain", "chain_validate", "chain_plan", "last_error",
-    "skinny_gemm_noalloc",
+    "skinny_gemm_noalloc", "workspace_status", "gemm_chain_status", "debug_stall",
     "abi_version", "HEADER_SYMBOLS",
 ]
 
@@ -41,7 +41,8 @@ K_ORDER_AUTO, K_ORDER_INCREASING, K_ORDER_ROTATED = 0, 1, 2
 
 # Every function include/wsm.h declares (checked by the CPU tests).
 HEADER_SYMBOLS = (
-    "skinny_gemm", "skinny_gemm_ex", "wsm_plan", "wsm_workspace_bytes", "wsm_stream_status", "skinny_gemm_noalloc",
+    "skinny_gemm", "skinny_gemm_ex", "wsm_plan", "wsm_workspace_bytes", "wsm_stream_status", "wsm_workspace_status",
+    "wsm_debug_stall", "skinny_gemm_noalloc", "gemm_chain_status",
     "wsm_chain_plan", "wsm_chain_create", "wsm_chain_run", "wsm_chain_status", "wsm_chain_task_plan",
     "wsm_chain_trace",
     "wsm_chain_destroy",
@@ -119,6 +120,12 @@ def lib() -> ctypes.CDLL:
         L.wsm_workspace_bytes.restype = ctypes.c_size_t
         L.wsm_stream_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
         L.wsm_stream_status.restype = st
+        L.wsm_workspace_status.argtypes = [vp, ctypes.c_size_t, vp, ctypes.POINTER(ctypes.c_int)]
+        L.wsm_workspace_status.restype = st
+        L.wsm_debug_stall.argtypes = [i, ctypes.c_ulonglong]
+        L.wsm_debug_stall.restype = st
+        L.gemm_chain_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+        L.gemm_chain_status.restype = st
         L.wsm_chain_task_plan.argtypes = [vp, i, ctypes.POINTER(_PlanInfo)]
         L.wsm_chain_task_plan.restype = st
         L.wsm_chain_create.argtypes = [ctypes.POINTER(_Task), i, ctypes.POINTER(_ChainOpts), ctypes.POINTER(vp)]
@@ -278,10 +285,41 @@ def workspace_bytes(M: int, N: int, K: int, **opts) -> int:
 
 
 def stream_status(stream=None) -> int:
-    """Synchronise the stream; 0, or WSM_ERR_TIMEOUT if a pipeline wait ran out."""
+    """Synchronise the stream; 0, or WSM_ERR_TIMEOUT if a device-side wait of a
+    call on it (or of a skinny_gemm_noalloc call on this device) ran out since
+    the last check."""
     code = ctypes.c_int(0)
-    lib().wsm_stream_status(_stream_handle(stream), ctypes.byref(code))
+    rc = lib().wsm_stream_status(_stream_handle(stream), ctypes.byref(code))
+    if rc not in (WSM_OK, WSM_ERR_TIMEOUT):
+        raise WsmError(rc, "wsm_stream_status", last_error())
     return code.value
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream; 0, or WSM_ERR_TIMEOUT if a device-side wait of a
+    skinny_gemm_ex call given this caller workspace ran out since the last check."""
+    code = ctypes.c_int(0)
+    rc = lib().wsm_workspace_status(workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    _stream_handle(stream), ctypes.byref(code))
+    if rc not in (WSM_OK, WSM_ERR_TIMEOUT):
+        raise WsmError(rc, "wsm_workspace_status", last_error())
+    return code.value
+
+
+def gemm_chain_status(stream=None):
+    """Synchronise the stream; (code, failed_task) for the one-shot gemm_chain
+    runs on the current device since the last check."""
+    ft = ctypes.c_int(-1)
+    rc = lib().gemm_chain_status(_stream_handle(stream), ctypes.byref(ft))
+    if rc not in (WSM_OK, WSM_ERR_TIMEOUT):
+        raise WsmError(rc, "gemm_chain_status", last_error())
+    return rc, ft.value
+
+
+def debug_stall(calls: int, limit_ns: int = 50_000_000) -> None:
+    """Test hook: the next `calls` launches each stall CTA 0 on a flag nothing
+    sets for limit_ns, then record WSM_ERR_TIMEOUT (no fault); 0 cancels."""
+    _check(lib().wsm_debug_stall(calls, limit_ns), "wsm_debug_stall")
 
 
 @dataclass

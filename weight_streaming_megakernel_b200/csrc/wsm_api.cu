@@ -8,6 +8,7 @@
 #include "../../include/wsm.h"
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -22,6 +23,7 @@ namespace wsm {
 
 __global__ void wsm_umma_kernel(const __grid_constant__ KParams p);
 const void *stream_kernel_ptr(int mmax, int tile_rows);  // wsm_stream.cu
+void *noalloc_scratch_ptr(int dev);                      // wsm_noalloc.cu: nullptr until set up on `dev`
 
 namespace {
 
@@ -610,6 +612,28 @@ wsm_status stream_workspace(int dev, cudaStream_t stream, const Geo &g, void **o
     return WSM_OK;
 }
 
+// The stall test hook (wsm_debug_stall): launches left to stall, and the stall's limit.
+std::atomic<int> g_stall_calls{0};
+std::atomic<unsigned long long> g_stall_ns{0};
+
+// Called right before a launch: the stall limit for it (0 = none), consuming one stalled launch.
+unsigned long long take_stall() {
+    int c = g_stall_calls.load(std::memory_order_relaxed);
+    while (c > 0) {
+        if (g_stall_calls.compare_exchange_weak(c, c - 1)) return g_stall_ns.load();
+    }
+    return 0;
+}
+
+// Read the sticky error words of a status block after `stream` has drained, and clear them.  Returns the
+// error code (0 = none); h receives the four words.
+wsm_status read_clear_status(const void *status, cudaStream_t stream, int (&h)[kStatusWords]) {
+    WSM_CUDA(cudaStreamSynchronize(stream));
+    WSM_CUDA(cudaMemcpy(h, status, sizeof h, cudaMemcpyDeviceToHost));
+    if (h[0] != 0) WSM_CUDA(cudaMemset(const_cast<void *>(status), 0, sizeof h));
+    return WSM_OK;
+}
+
 int pdl_mode(int flags) {
     if (flags & WSM_FLAG_NO_PDL) return 0;
     return (flags & WSM_FLAG_W_READONLY) ? 2 : 1;
@@ -1007,6 +1031,7 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     kp.trace = nullptr;
     const void *fn;
     if ((st = prepare_kernel(d, g, &fn)) != WSM_OK) return st;
+    kp.debug_stall_ns = take_stall();
     if ((st = launch(fn, g, kp, stream, false)) != WSM_OK) return st;
     return WSM_OK;
 }
@@ -1017,30 +1042,54 @@ wsm_status skinny_gemm(const void *X, const void *W, void *Y, int M, int N, int 
 
 wsm_status wsm_stream_status(wsm_stream_t stream_, int *code) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (code) *code = 0;
     int dev = 0;
     WSM_CUDA(cudaGetDevice(&dev));
-    void *ptr = nullptr;
+    void *ptrs[2] = {nullptr, wsm::noalloc_scratch_ptr(dev)};
     {
         std::lock_guard<std::mutex> lk(g_mu);
         auto it = g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
-        if (it != g_ws.end()) ptr = it->second.ptr;
+        if (it != g_ws.end()) ptrs[0] = it->second.ptr;
     }
-    if (code) *code = 0;
-    if (!ptr) return WSM_OK;
     WSM_CUDA(cudaStreamSynchronize(stream));
-    int h[kStatusWords] = {};
-    WSM_CUDA(cudaMemcpy(h, ptr, sizeof h, cudaMemcpyDeviceToHost));
-    if (code) *code = h[0];
-    if (h[0] != 0) {
-        // an aborted call may leave its counters mid-count: clear the whole scratch
-        size_t bytes = 0;
-        {
-            std::lock_guard<std::mutex> lk(g_mu);
-            bytes = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}].bytes;
+    // the stream's own workspace first, then the no-alloc array of this device
+    int first[kStatusWords] = {};
+    const char *where = nullptr;
+    for (int i = 0; i < 2; ++i) {
+        if (!ptrs[i]) continue;
+        int h[kStatusWords] = {};
+        wsm_status st = read_clear_status(ptrs[i], stream, h);
+        if (st != WSM_OK) return st;
+        if (h[0] != 0 && first[0] == 0) {
+            memcpy(first, h, sizeof h);
+            where = i == 0 ? "skinny_gemm on this stream" : "skinny_gemm_noalloc on this device";
         }
-        WSM_CUDA(cudaMemset(ptr, 0, bytes));
-        return fail(WSM_ERR_TIMEOUT, "device-side wait ran out (task %d, cta %d, site %d)", h[1], h[2], h[3]);
     }
+    if (first[0] == 0) return WSM_OK;
+    if (code) *code = first[0];
+    return fail(WSM_ERR_TIMEOUT, "device-side wait ran out in %s (cta %d, site %d)", where, first[2], first[3]);
+}
+
+wsm_status wsm_workspace_status(const void *workspace, size_t workspace_bytes, wsm_stream_t stream_, int *code) {
+    if (code) *code = 0;
+    if (!workspace) return fail(WSM_ERR_INVALID, "workspace must be non-null");
+    if (!aligned16(workspace)) return fail(WSM_ERR_ALIGN, "workspace must be 16-byte aligned");
+    if (workspace_bytes < 512) return fail(WSM_ERR_INVALID, "workspace of %zu bytes is too small to be one", workspace_bytes);
+    int h[kStatusWords] = {};
+    wsm_status st = read_clear_status(workspace, reinterpret_cast<cudaStream_t>(stream_), h);
+    if (st != WSM_OK) return st;
+    if (h[0] == 0) return WSM_OK;
+    if (code) *code = h[0];
+    return fail(WSM_ERR_TIMEOUT, "device-side wait ran out in a call on this workspace (cta %d, site %d)", h[2], h[3]);
+}
+
+wsm_status wsm_debug_stall(int calls, unsigned long long limit_ns) {
+    if (calls < 0) return fail(WSM_ERR_INVALID, "calls must be >= 0 (got %d)", calls);
+    if (calls > 0 && (limit_ns == 0 || limit_ns > 10000000000ull))
+        return fail(WSM_ERR_INVALID, "the stall limit must be in (0, 10 s] (got %llu ns)", limit_ns);
+    g_stall_ns.store(limit_ns);
+    g_stall_calls.store(calls);
+    g_err.clear();
     return WSM_OK;
 }
 
@@ -1332,6 +1381,7 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     kp.dep_timeout_ns = ch->dep_timeout_ns;
     kp.wait_timeout_ns = ch->dep_timeout_ns + kPipeTimeoutNs;
     kp.trace = ch->d_trace;
+    kp.debug_stall_ns = take_stall();
     return launch(ch->fn, ch->geo, kp, stream, ch->any_dep);
 }
 
@@ -1460,6 +1510,30 @@ wsm_status gemm_chain(const wsm_task *tasks, int n_tasks, wsm_stream_t stream) {
     }
     g_chain_cache[{dev, key}] = CachedChain{ch, false};
     return wsm_chain_run(ch, stream);
+}
+
+wsm_status gemm_chain_status(wsm_stream_t stream, int *failed_task) {
+    if (failed_task) *failed_task = -1;
+    int dev = 0;
+    WSM_CUDA(cudaGetDevice(&dev));
+    WSM_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+    wsm_status first = WSM_OK;
+    std::string msg;
+    // under the lock: no other thread drops a cached chain meanwhile
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (auto &kv : g_chain_cache) {
+        if (kv.first.first != dev) continue;
+        int ft = -1;
+        const wsm_status st = wsm_chain_status(kv.second.ch, stream, &ft);
+        if (st != WSM_OK && first == WSM_OK) {
+            first = st;
+            msg = g_err;
+            if (failed_task) *failed_task = ft;
+        }
+    }
+    if (first != WSM_OK) return fail(first, "gemm_chain: %s", msg.c_str());
+    g_err.clear();
+    return WSM_OK;
 }
 
 }  // extern "C"

@@ -37,7 +37,16 @@ constexpr int kUmmaRows = 128;     // rows of W per UMMA tile (MMA M)
 constexpr int kUmmaBK = 64;        // K elements per UMMA box (one 128-byte swizzle row)
 constexpr int kUmmaMaxN = 64;      // largest MMA N (= X rows per tile)
 constexpr int kStreamBoxK = 256;   // K elements per TMA box on the FMA path
-constexpr int kStatusWords = 4;    // [0] error code, [1] failing task, [2] failing CTA, [3] site
+// Status block (the first 256 bytes of a call's scratch or a chain's buffer):
+//   [0] first error code, [1] its task, [2] its CTA, [3] its site -- sticky: kept over later calls until the
+//       host reads and clears them (wsm_stream_status, wsm_workspace_status, wsm_chain_status,
+//       gemm_chain_status);
+//   [4] an error was recorded in the CURRENT launch: bounded waits give up early on it, and the launch's
+//       last CTA repairs the counters the launch left mid-count and clears it at exit;
+//   [5] never written by anyone: the flag the stall test hook waits on.
+constexpr int kStatusWords = 4;    // words the host reads: [0] code, [1] task, [2] CTA, [3] site
+constexpr int kStatusLaunchErr = 4;
+constexpr int kStatusStallFlag = 5;
 constexpr int kSchedWords = 2;     // per task: [0] next unit to claim, [1] CTAs done claiming
 constexpr int kClaimLead = 4;      // a CTA claims its next unit this many stages before its unit ends
 constexpr int kColChunk = 256;     // output columns per readiness chunk (per-column data dependencies)
@@ -51,7 +60,7 @@ constexpr int kTraceSlots = 8;
 enum : int { kEpiNone = 0, kEpiSiluMul = 1, kEpiResidual = 2 };
 
 // Error sites recorded in status[3].
-enum : int { kSiteNone = 0, kSiteDep = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteAcc = 4, kSiteDrain = 5 };
+enum : int { kSiteNone = 0, kSiteDep = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteAcc = 4, kSiteDrain = 5, kSiteStall = 6 };
 constexpr int kCodeTimeout = 6;    // == WSM_ERR_TIMEOUT
 
 // Stage / accumulator metadata flags (producer -> consumers).
@@ -135,6 +144,8 @@ struct KParams {
     unsigned long long dep_timeout_ns;
     unsigned long long wait_timeout_ns;
     unsigned long long *trace;      // [grid][n_tasks][kTraceSlots] or nullptr
+    unsigned long long debug_stall_ns;  // test hook, 0 in real use: CTA 0's producer waits this long on a flag
+                                        // nothing sets, records a time-out and abandons its work
 };
 
 #if defined(__CUDACC__)
@@ -282,18 +293,23 @@ __device__ __forceinline__ float ld_cg_f32(const float *p) {
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Record the first error of a launch (code, task, cta, site).
+// Record an error: the first one since the host last cleared the status (code, task, cta, site), and the
+// current launch's error flag.
 __device__ __forceinline__ void record_error(int *status, int code, int task, int site) {
-    if (status && atomicCAS(status, 0, code) == 0) {
+    if (!status) return;
+    if (atomicCAS(status, 0, code) == 0) {
         status[1] = task;
         status[2] = (int)blockIdx.x;
         status[3] = site;
-        __threadfence();
     }
+    *((volatile int *)&status[kStatusLaunchErr]) = 1;
+    __threadfence();
 }
 
-__device__ __forceinline__ bool status_set(const int *status) {
-    return status && *((volatile const int *)status) != 0;
+// An error was recorded in the current launch (an earlier launch's sticky error does not count: the
+// counters that launch left were repaired when it ended).
+__device__ __forceinline__ bool launch_failed(const int *status) {
+    return status && *((volatile const int *)&status[kStatusLaunchErr]) != 0;
 }
 
 // Bounded wait on an mbarrier phase.  Returns false (and records an error)
@@ -448,16 +464,37 @@ __device__ __forceinline__ ClaimRange claim_range(const TaskDev &T) {
 // handed out statically (unit c to CTA c); a result >= cr.hi means none left.
 __device__ __forceinline__ int claim_unit(const ClaimRange &cr) { return (int)atom_add_relaxed_gpu(cr.ctr, 1u); }
 
-// Single GEMM: called once per CTA when it has stopped claiming units; the
-// last CTA resets the claim counters for the next call (no CTA claims any
-// more).  A chain resets all its tasks' claim counters at the end of the run
-// instead (chain_run_done), so no CTA waits on this atomic between tasks.
-__device__ __forceinline__ void claims_finished(const TaskDev &T, unsigned int grid) {
+// Single GEMM: called once per CTA by thread 0 after the CTA's last barrier (all its roles are done).
+// The last CTA resets the claim counters for the next call; if this launch recorded an error, some CTA
+// abandoned its work, so tile arrival counters may be left mid-count: it clears them as well, then the
+// launch's error flag.  The next call on the same scratch starts clean (stream order, or the programmatic
+// dependency its scratch accesses wait for), and the sticky error words stay for the host to read.  A
+// chain resets its claim counters at the end of the run instead (chain_run_done).
+__device__ __forceinline__ void single_call_done(const KParams &p) {
+    const TaskDev &T = p.single;
     const unsigned int old = atom_add_acqrel_gpu(&T.sched[1], 1u);
-    if (old == grid - 1) {
-        st_relaxed_gpu(&T.sched[0], 0u);
-        st_relaxed_gpu(&T.sched[1], 0u);
+    if (old != gridDim.x - 1) return;
+    st_relaxed_gpu(&T.sched[0], 0u);
+    if (launch_failed(p.status)) {
+        const int tiles = T.n_g * T.n_mt;
+        for (int i = 0; i < tiles; ++i) st_relaxed_gpu(&T.tile_cnt[i], 0u);
+        st_relaxed_gpu(reinterpret_cast<unsigned int *>(&p.status[kStatusLaunchErr]), 0u);
     }
+    st_relaxed_gpu(&T.sched[1], 0u);
+}
+
+// Test hook (KParams::debug_stall_ns): a bounded wait on a status word that nothing ever sets.  When the
+// limit passes it records a time-out and raises the CTA's abort flag; the caller then abandons its work.
+static __device__ __noinline__ void debug_stall(const KParams &p, volatile int *abort_flag) {
+    const unsigned int *flag = reinterpret_cast<const unsigned int *>(&p.status[kStatusStallFlag]);
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t spin = 1;; ++spin) {
+        if (ld_acquire_gpu(flag) != 0u) return;
+        if ((spin & 31u) == 0 && globaltimer() - t0 > p.debug_stall_ns) break;
+        __nanosleep(256);
+    }
+    record_error(p.status, kCodeTimeout, -1, kSiteStall);
+    *abort_flag = 1;
 }
 
 // Sum, in unit order (= K order), of the partials of rows m0 .. m0+MB-1 (those
@@ -586,7 +623,7 @@ static __device__ __noinline__ void wait_chunks(const KParams &p, const TaskDev 
             for (uint32_t spin = 1;; ++spin) {
                 if (ld_acquire_gpu(&T.dep_col_cnt[c]) - target < 0x80000000u) break;
                 if ((spin & 31u) == 0) {
-                    if (status_set(status)) return;
+                    if (launch_failed(status)) return;
                     if (globaltimer() - t0 > p.dep_timeout_ns) {
                         record_error(status, kCodeTimeout, task, kSiteDep);
                         return;
@@ -617,7 +654,7 @@ static __device__ __noinline__ void wait_dependency(const KParams &p, const Task
     for (uint32_t spin = 1;; ++spin) {
         if (ld_acquire_gpu(D.done) - target < 0x80000000u) break;
         if ((spin & 31u) == 0) {
-            if (status_set(status)) break;
+            if (launch_failed(status)) break;
             if (globaltimer() - t0 > p.dep_timeout_ns) {
                 record_error(status, kCodeTimeout, task, kSiteDep);
                 break;
@@ -630,17 +667,41 @@ static __device__ __noinline__ void wait_dependency(const KParams &p, const Task
 
 // Called by one thread per CTA after the CTA has finished all its work of a
 // chain run: the last CTA (every other CTA has stopped claiming) resets the
-// tasks' claim counters and advances the run counter for the next run.
+// tasks' claim counters and advances the run counter for the next run.  If
+// the run recorded an error, some CTA abandoned its work and the counters of
+// this run may be left mid-count: the last CTA first sets every readiness
+// counter to the value a completed run leaves (run x tiles, per group, per
+// column chunk) and clears the tile arrival counters, so the next run waits
+// for exactly its own work again; the sticky error words stay for the host.
 __device__ __forceinline__ void chain_run_done(const KParams &p) {
     if (!p.run_ctl) return;
     const unsigned int old = atom_add_acqrel_gpu(&p.run_ctl[1], 1u);
     if (old == gridDim.x - 1) {
+        const bool heal = launch_failed(p.status);
+        const unsigned int run = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
         for (int t = 0; t < p.n_tasks; ++t) {
             const TaskDev &T = task_at(p, t);
             st_relaxed_gpu(&T.sched[0], 0u);
             if (T.n_groups > 1)
                 for (int g = 0; g < T.n_groups; ++g) st_relaxed_gpu(&T.grp_sched[g], 0u);
+            if (!heal) continue;
+            const int tiles = T.n_g * T.n_mt;
+            for (int i = 0; i < tiles; ++i) st_relaxed_gpu(&T.tile_cnt[i], 0u);
+            if (T.notify) {
+                if (T.n_groups > 1) {
+                    for (int g = 0; g < T.n_groups; ++g)
+                        st_relaxed_gpu(&T.grp_done[g], run * (unsigned int)(group_tile_lo(T, g + 1) - group_tile_lo(T, g)));
+                    st_relaxed_gpu(T.done, run * (unsigned int)T.n_groups);
+                } else {
+                    st_relaxed_gpu(T.done, run * (unsigned int)tiles);
+                }
+            }
+            if (T.col_cnt) {
+                const int chunks = (T.y_cols + kColChunk - 1) / kColChunk;
+                for (int c = 0; c < chunks; ++c) st_relaxed_gpu(&T.col_cnt[c], run * T.col_need[c]);
+            }
         }
+        if (heal) st_relaxed_gpu(reinterpret_cast<unsigned int *>(&p.status[kStatusLaunchErr]), 0u);
         st_relaxed_gpu(&p.run_ctl[1], 0u);
         red_release_gpu_add(&p.run_ctl[0], 1u);
     }

@@ -296,6 +296,16 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             bool slot_ok = false;           // the wait for ring slot s has already succeeded
             bool grid_dep_ok = p.pdl != 2;  // mode 2 streams W before the previous kernel completes
             if (p.pdl == 1) pdl_wait();
+            if (p.debug_stall_ns && blockIdx.x == 0) {
+                // test hook: after the previous kernel (whose exit clears the launch error flag), wait on a
+                // flag nothing sets until the limit passes, then abandon all of this CTA's work
+                if (!grid_dep_ok) {
+                    pdl_wait();
+                    grid_dep_ok = true;
+                }
+                debug_stall(p, &abort_flag);
+                aborted = abort_flag != 0;
+            }
             for (int t = 0; t < p.n_tasks && !aborted; ++t) {
                 const TaskDev &T = task_at(p, t);
                 prefetch_tmap(&T.tmW);
@@ -463,7 +473,6 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 }
                 if (np > 0) flush();
                 if (aborted) break;
-                if (!p.run_ctl) claims_finished(T, gridDim.x);
                 if (T.dep < 0 && !first_unit) trace_stamp(p, t, 1, globaltimer());
             }
             if (!grid_dep_ok) pdl_wait();  // a CTA with no work still orders itself after the previous kernel
@@ -667,7 +676,10 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, p.wide ? kTmemColsWide : kTmemCols);
-    if (threadIdx.x == 0) chain_run_done(p);
+    if (threadIdx.x == 0) {
+        if (p.run_ctl) chain_run_done(p);
+        else single_call_done(p);
+    }
 }
 
 }  // namespace wsm
