@@ -29,14 +29,47 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[WSM_NOALLOC_SCR
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void *g_noalloc_ptr[kMaxDevices] = {};  // device address of g_noalloc_scratch, per device
+// Per device: the device address of g_noalloc_scratch and the context it was looked up in.  After a
+// device reset the primary context (and with it the module's memory) is new: the address is looked up
+// again when the current context differs.
+void *g_noalloc_ptr[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
 
 wsm_status noalloc_fail(wsm_status code, const char *msg) {
     wsm::set_last_error_message(msg);
     return code;
 }
 
+// The current context (nullptr if the driver entry point is unavailable).  Caller holds g_noalloc_mu.
+CUcontext current_context() {
+    if (!g_ctx_get_current) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return nullptr;
+        g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    }
+    CUcontext c = nullptr;
+    if (g_ctx_get_current(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
 }  // namespace
+
+namespace wsm {
+// The array's device address on `dev` if a call has set it up there in the current context, else nullptr
+// (wsm_stream_status reads the array's status words through it).
+void *noalloc_scratch_ptr(int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev] || g_noalloc_ctx[dev] != current_context()) return nullptr;
+    return g_noalloc_ptr[dev];
+}
+}  // namespace wsm
 
 extern "C" {
 
@@ -47,12 +80,14 @@ wsm_status skinny_gemm_noalloc(const void *X, const void *W, void *Y, int M, int
     if (e != cudaSuccess) return noalloc_fail(WSM_ERR_CUDA, "skinny_gemm_noalloc: cudaGetDevice failed");
     if (dev < 0 || dev >= kMaxDevices) return noalloc_fail(WSM_ERR_UNSUPPORTED, "skinny_gemm_noalloc: device index too large");
 
-    // Set-up, once per device, with that device current: the host-side name of
-    // the array is only a stand-in, so look up its device address.
+    // Set-up, once per device (again after a device reset), with that device
+    // current: the host-side name of the array is only a stand-in, so look up
+    // its device address.
     void *scratch = nullptr;
     {
         std::lock_guard<std::mutex> lk(g_noalloc_mu);
-        if (!g_noalloc_ptr[dev]) {
+        const CUcontext ctx = current_context();
+        if (!g_noalloc_ptr[dev] || g_noalloc_ctx[dev] != ctx) {
             void *p = nullptr;
             e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
             if (e != cudaSuccess || !p) {
@@ -62,6 +97,7 @@ wsm_status skinny_gemm_noalloc(const void *X, const void *W, void *Y, int M, int
                 return noalloc_fail(WSM_ERR_CUDA, buf);
             }
             g_noalloc_ptr[dev] = p;
+            g_noalloc_ctx[dev] = ctx;
         }
         scratch = g_noalloc_ptr[dev];
     }
@@ -87,11 +123,13 @@ wsm_status skinny_gemm_noalloc(const void *X, const void *W, void *Y, int M, int
         return noalloc_fail(WSM_ERR_UNSUPPORTED, buf);
     }
 
-    // The array keeps the previous call's contents: clear the status word and
-    // the counters this call will use (they must start at zero).  Calls whose
-    // work overlaps on the GPU share the array and race.
-    const size_t counters = 256 + 4 * ((size_t)wsm::kSchedWords + (size_t)info.n_tiles * (size_t)info.m_tiles);
-    e = cudaMemsetAsync(scratch, 0, counters, stream);
+    // The array keeps the previous call's contents: clear the counters this
+    // call will use (they must start at zero).  The status words before them
+    // are left alone: a time-out recorded by an earlier call stays there until
+    // wsm_stream_status reads it.  Calls whose work overlaps on the GPU share
+    // the array and race.
+    const size_t counters = 4 * ((size_t)wsm::kSchedWords + (size_t)info.n_tiles * (size_t)info.m_tiles);
+    e = cudaMemsetAsync(static_cast<unsigned char *>(scratch) + 256, 0, counters, stream);
     if (e != cudaSuccess) return noalloc_fail(WSM_ERR_CUDA, "skinny_gemm_noalloc: clearing the scratch failed");
 
     wsm_opts o;
