@@ -1,0 +1,147 @@
+"""Out-of-bounds writes, caught with guard canaries.
+
+Every buffer the kernels write -- Y, the fp32 copy Yf32, the residual input R
+when Y is written over it in place, and a caller workspace -- is placed in the
+middle of a larger allocation whose guard regions before and after hold a
+fixed bit pattern the kernels never produce.  After the call the guards must
+be unchanged bit for bit, and the result must still match the oracle.  The
+guards are as long as 64 rows of the output, so a store to a padding row of
+an M-tile (X rows are padded to 16 on the tensor-core path) or past the last
+column of a ragged N would land in them.
+
+Cases: ragged N (17, 129, 2112) and K (40, 1000, 4104), every M class on both
+kernel paths, the SiLU*mul output of width N/2, split-K partial slots inside
+a caller workspace, and chain tasks (plain, residual in place, SiLU*mul)."""
+import pytest
+import torch
+
+import oracle
+import synth
+import weight_streaming_megakernel_b200 as wsm
+from parity import check_bounded, check_full
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+PATTERN16 = 0x5A3C        # a bf16 value (about 1.3e16) no output here comes near
+PATTERN32 = 0x7F8A5A3C    # an fp32 signalling-NaN payload no kernel writes
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    yield
+
+
+class Guarded:
+    """A [rows, cols] tensor of `dtype` inside an allocation with `guard`
+    elements of a fixed pattern before and after it (offsets multiples of 8
+    elements, so the tensor stays 16-byte aligned)."""
+
+    def __init__(self, rows, cols, dtype, guard_rows=64, fill=None):
+        self.n = rows * cols
+        self.g = max(guard_rows * cols, 8192)
+        self.g = -(-self.g // 8) * 8
+        itype = torch.int16 if dtype == torch.bfloat16 else torch.int32
+        pat = PATTERN16 if dtype == torch.bfloat16 else PATTERN32
+        pat = pat - (1 << 16) if itype == torch.int16 and pat >= (1 << 15) else pat
+        pat = pat - (1 << 32) if itype == torch.int32 and pat >= (1 << 31) else pat
+        self.raw = torch.full((2 * self.g + -(-self.n // 8) * 8,), pat, dtype=itype, device=DEV)
+        self.pat = pat
+        self.t = self.raw[self.g: self.g + self.n].view(dtype).view(rows, cols)
+        if fill is not None:
+            self.t.copy_(fill)
+        else:
+            self.t.view(itype).fill_(0x7FC0 if itype == torch.int16 else 0x7FC00000)  # NaN
+
+    def intact(self):
+        head = self.raw[: self.g]
+        tail = self.raw[self.g + self.n:]
+        bad_h = (head != self.pat).nonzero()
+        bad_t = (tail != self.pat).nonzero()
+        assert bad_h.numel() == 0, f"{bad_h.numel()} guard elements before the buffer overwritten " \
+                                   f"(first at -{self.g - int(bad_h[0])})"
+        assert bad_t.numel() == 0, f"{bad_t.numel()} guard elements after the buffer overwritten " \
+                                   f"(first at +{int(bad_t[0])})"
+
+
+CASES = [(path, M, N, K)
+         for path, ms in ((wsm.PATH_STREAM, (1, 3, 8)), (wsm.PATH_UMMA, (1, 5, 16, 17, 40, 64)))
+         for M in ms
+         for N, K in ((17, 40), (129, 4104), (2112, 1000))]
+
+
+@pytest.mark.parametrize("path,M,N,K", CASES)
+def test_plain_outputs_and_workspace_stay_in_bounds(path, M, N, K):
+    x, w = synth.make_xw(M, N, K, seed=M * 31 + N)
+    xd, wd = x.to(DEV), w.to(DEV)
+    for unit_stages in (0, 1):  # automatic units, and one stage per unit (split tiles, partial slots)
+        y = Guarded(M, N, torch.bfloat16)
+        yf = Guarded(M, N, torch.float32)
+        nbytes = wsm.workspace_bytes(M, N, K, path=path, unit_stages=unit_stages)
+        ws = Guarded(1, nbytes // 4, torch.int32, guard_rows=1, fill=torch.zeros(1, nbytes // 4, dtype=torch.int32))
+        wsm.skinny_gemm(xd, wd, y.t, path=path, yf32=yf.t, workspace=ws.t, unit_stages=unit_stages)
+        assert wsm.workspace_status(ws.t) == 0
+        y.intact()
+        yf.intact()
+        ws.intact()
+        check_full(x, w, y.t, yf.t, what=f"path={path} M={M} N={N} K={K} unit_stages={unit_stages}")
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 2), (wsm.PATH_UMMA, 16), (wsm.PATH_UMMA, 33)])
+def test_silu_mul_half_width_output_stays_in_bounds(path, M):
+    N, K = 1040, 1032
+    x, w = synth.make_xw(M, N, K, seed=M + 5)
+    y = Guarded(M, N // 2, torch.bfloat16)
+    yf = Guarded(M, N // 2, torch.float32)
+    wsm.skinny_gemm(x.to(DEV), w.to(DEV), y.t, path=path, yf32=yf.t, epilogue=wsm.EPI_SILU_MUL)
+    assert wsm.stream_status() == 0
+    y.intact()
+    yf.intact()
+    H, G, U, Sg, Su = oracle.silu_mul_ref(x, w)
+    check_bounded(y.t, yf.t, H, oracle.fused_bounds("silu_mul", G=G, U=U, Sg=Sg, Su=Su), "silu")
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 4), (wsm.PATH_UMMA, 24)])
+def test_residual_in_place_stays_in_bounds(path, M):
+    N, K = 2112, 1000
+    x, w = synth.make_xw(M, N, K, seed=M + 9)
+    r = synth.make_x(M, N, seed=M + 10)
+    y = Guarded(M, N, torch.bfloat16, fill=r.to(DEV))  # Y written over R
+    wsm.skinny_gemm(x.to(DEV), w.to(DEV), y.t, path=path, epilogue=wsm.EPI_RESIDUAL, r=y.t)
+    assert wsm.stream_status() == 0
+    y.intact()
+    Y, S = oracle.residual_ref(x, w, r)
+    check_bounded(y.t, None, Y, oracle.fused_bounds("residual", S=S, Y=Y), "residual in place")
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 8), (wsm.PATH_UMMA, 16), (wsm.PATH_UMMA, 64)])
+def test_chain_outputs_stay_in_bounds(path, M):
+    """A layer-like chain, each output guarded: o (+R in place) -> gate_up
+    (SiLU*mul, N/2 wide) -> down, task t reading task t - 1's output."""
+    d, ff = 1032, 2080
+    x0 = synth.make_x(M, d, seed=M).to(DEV)
+    w_o = synth.make_w(d, d, seed=M + 1).to(DEV)
+    w_gu = synth.make_w(2 * ff, d, seed=M + 2).to(DEV)
+    w_dn = synth.make_w(d, ff, seed=M + 3).to(DEV)
+    r = synth.make_x(M, d, seed=M + 4).to(DEV)
+    h0 = Guarded(M, d, torch.bfloat16, fill=r)
+    h1 = Guarded(M, ff, torch.bfloat16)
+    h2 = Guarded(M, d, torch.bfloat16)
+    f2 = Guarded(M, d, torch.float32)
+    tasks = [wsm.Task(x0, w_o, h0.t, epilogue=wsm.EPI_RESIDUAL, r=h0.t),
+             wsm.Task(h0.t, w_gu, h1.t, dep=0, epilogue=wsm.EPI_SILU_MUL),
+             wsm.Task(h1.t, w_dn, h2.t, dep=1, yf32=f2.t)]
+    ch = wsm.Chain(tasks, path=path)
+    ch.run()
+    assert ch.status()[0] == wsm.WSM_OK
+    for g in (h0, h1, h2, f2):
+        g.intact()
+    Y0, S0 = oracle.residual_ref(x0.cpu(), w_o.cpu(), r.cpu())
+    check_bounded(h0.t, None, Y0, oracle.fused_bounds("residual", S=S0, Y=Y0), "chain o")
+    H, G, U, Sg, Su = oracle.silu_mul_ref(h0.t.cpu(), w_gu.cpu())
+    check_bounded(h1.t, None, H, oracle.fused_bounds("silu_mul", G=G, U=U, Sg=Sg, Su=Su), "chain gate_up")
+    check_full(h1.t.cpu(), w_dn.cpu(), h2.t, f2.t, what="chain down")
+    ch.close()
