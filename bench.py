@@ -560,6 +560,39 @@ def oracle_sample_rate(cases, budget_s, threads=0):
     return per_step, cores, desc
 
 
+# The five configurations of the metric, as (key, workload, mode, target fraction of the measured peak or
+# None).  The default run reports every one of them beside its headline (the Qwen3-8B decode step).
+CONFIGURATIONS = (
+    ("c1_single_m1_4096x4096", "single", "launches", 0.80),
+    ("c2_qwen3_8b_decode_gemms", "qwen3_decode", "chain", 0.80),
+    ("c3_skinny_k7168_k8192", "skinny", "chain", 0.80),
+    ("c4_l2_reuse_m32_m64", "l2_reuse", "chain", None),
+    ("c5_chain_36x4_m16", "chain", "chain", 0.75),
+)
+
+
+def run_configurations(args, rank, world, local_rank, hbm_peak, headline):
+    """Every configuration besides the headline one: device time per step of
+    K' = min(K, 10) steps in one graph (same protocol as the headline), GB/s of
+    algorithmic bytes, fraction of the measured peak."""
+    out = {}
+    for key, workload, mode, target in CONFIGURATIONS:
+        if workload == args.workload and mode == args.mode:
+            r = headline
+        else:
+            sub = argparse.Namespace(**vars(args))
+            sub.workload, sub.mode, sub.only = workload, mode, ""
+            r = run_gpu(sub, rank, world, local_rank, mode=mode, steps=min(args.steps, 10), extras=False)
+        gbs = r["total_bytes"] / (r["ms_per_step"] * 1e-3) / 1e9
+        n = len(r["cases"])
+        out[key] = {"workload": workload, "mode": mode, "gemms": n, "ms_per_step": round(r["ms_per_step"], 4),
+                    "us_per_gemm": round(r["ms_per_step"] * 1e3 / n, 3), "GBps": round(gbs, 1),
+                    "frac_of_peak": round(gbs / hbm_peak, 4), "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                    "target_frac": target,
+                    "bytes_per_step": r["total_bytes"]}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -576,6 +609,8 @@ def main():
                     help="chain: the step is one persistent gemm_chain kernel; launches: one skinny_gemm per GEMM "
                          "(default: launches for the single-GEMM workload, chain otherwise)")
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-GEMM single-launch breakdown")
+    ap.add_argument("--no-configurations", action="store_true",
+                    help="skip the other four configurations (reported beside the default workload)")
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "nshard"],
                     help="N > 1: independent replicas (weak scaling) or column blocks of every weight per rank "
                          "with an all-gather of each Y (strong scaling)")
@@ -663,6 +698,10 @@ def main():
                      "us_per_gemm_isolated": {c.name: round(_st.median(row[i] for row in rb["per_launch"]) * 1e3, 2)
                                               for i, c in enumerate(rb["cases"])}}
 
+    configurations = None
+    if args.workload == "qwen3_decode" and args.mode == "chain" and not args.only and not args.no_configurations:
+        configurations = run_configurations(args, rank, world, local_rank, hbm_peak, r)
+
     # roofline of the weight-streaming kernel: per-launch algorithmic bytes / duration
     import statistics
     per_case = []
@@ -721,6 +760,7 @@ def main():
                 "step_ms_p10_p50_p90": [pct(0.1), pct(0.5), pct(0.9)],
                 "us_per_gemm": us_per_gemm,
                 "single_launch_breakdown": breakdown,
+                "configurations": configurations,
                 "cpu_baseline": cpu,
                 "cpu_baseline_1thread": cpu1,
                 "e2e": r["e2e"],
