@@ -49,6 +49,22 @@ def test_abi_version():
     assert wsm.abi_version() == 1
 
 
+def test_status_queries_and_stall_hook_check_arguments_on_the_host():
+    """The time-out queries and the stall test hook reject bad arguments
+    before any CUDA call (so this runs without a GPU)."""
+    L = wsm.lib()
+    code = ctypes.c_int(-7)
+    assert L.wsm_workspace_status(None, 1 << 20, None, ctypes.byref(code)) == wsm.WSM_ERR_INVALID
+    assert code.value == 0
+    assert L.wsm_workspace_status(ctypes.c_void_p(0x1008), 1 << 20, None, ctypes.byref(code)) == wsm.WSM_ERR_ALIGN
+    assert L.wsm_workspace_status(ctypes.c_void_p(0x1000), 256, None, ctypes.byref(code)) == wsm.WSM_ERR_INVALID
+    assert L.wsm_debug_stall(-1, 1000) == wsm.WSM_ERR_INVALID
+    assert L.wsm_debug_stall(1, 0) == wsm.WSM_ERR_INVALID
+    assert L.wsm_debug_stall(1, 20_000_000_000) == wsm.WSM_ERR_INVALID
+    assert L.wsm_debug_stall(2, 1_000_000) == wsm.WSM_OK
+    assert L.wsm_debug_stall(0, 0) == wsm.WSM_OK
+
+
 def test_plan_paths_and_geometry():
     p = wsm.plan(1, 4096, 4096, num_sms=148)
     assert p["path"] == wsm.PATH_STREAM and p["tile_rows"] == 32 and p["m_tile"] == 1
