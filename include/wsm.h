@@ -353,7 +353,30 @@ typedef struct {
                                   wsm_chain_trace is then not available), at about 20 us per
                                   extra kernel boundary.  AUTO splits when the narrow tasks'
                                   weights exceed 1.5 GB per extra boundary. */
+    int cluster;               /* WSM_CHAIN_CLUSTER_*: cluster reduction.  The kernel runs as
+                                  thread-block clusters of 4 CTAs; each task's first round of
+                                  work units is handed out statically (unit c to CTA c) with 1, 2
+                                  or 4 units per tile, so a split tile's partial sums meet inside
+                                  one cluster and are added through distributed shared memory
+                                  (in unit order: the same bits as the global-memory reduction of
+                                  the same split) instead of round trips through L2 -- the part of
+                                  a dependency boundary that dominates dependent chains.  Only
+                                  clusters that the GPU keeps resident run (on B200 33 of them:
+                                  132 CTAs).  It applies to tensor-core chains in which every
+                                  task waits for the whole task before it.  Measured on B200 it
+                                  does not pay (a 36 x 4 dependent chain at M = 16: 3.41-3.51 ms
+                                  against 3.46 ms): at a dependency boundary every memory
+                                  operation waits behind the memory system's load, the exchange
+                                  included, and the 16 SMs left out cost as much as it saves.
+                                  AUTO and OFF: never; ON: always (WSM_ERR_UNSUPPORTED where it
+                                  does not apply). */
 } wsm_chain_opts;
+
+enum {
+    WSM_CHAIN_CLUSTER_AUTO = 0,
+    WSM_CHAIN_CLUSTER_OFF = 1,
+    WSM_CHAIN_CLUSTER_ON = 2
+};
 
 enum {
     WSM_CHAIN_KERNELS_AUTO = 0,
@@ -378,6 +401,7 @@ typedef struct {
                                while waiting (0 = none), */
     int k_order;            /* WSM_K_ORDER_INCREASING or WSM_K_ORDER_ROTATED, */
     int dep_ring_stages;    /* W stages streamed ahead of an unmet dependency (0 = the whole ring) */
+    int cluster;            /* CTAs per thread-block cluster with cluster reduction, 0 without */
 } wsm_chain_task_info;
 
 /* Pure host function (no CUDA calls, no memory touched): the plan
@@ -465,7 +489,7 @@ const char *wsm_last_error(void);
 /* ABI version of this header (bumped on any incompatible change). */
 int wsm_abi_version(void);
 
-#define WSM_ABI_VERSION 1
+#define WSM_ABI_VERSION 2
 
 #ifdef __cplusplus
 }

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version():
-    assert wsm.abi_version() == 1
+    assert wsm.abi_version() == 2
 
 
 def test_status_queries_and_stall_hook_check_arguments_on_the_host():
@@ -369,8 +369,11 @@ def test_chain_plan_independent_decode_step():
 
 def test_chain_plan_dependent_layers():
     """Task t waits for t - 1: nothing overlaps a task's end, so every task
-    takes the single-call split; 4 prefetch stages, one ring stage ahead of
-    the dependency, rotated K order."""
+    takes the single-call split on all 148 CTAs; 4 prefetch stages, one ring
+    stage ahead of the dependency, rotated K order.  With cluster reduction
+    requested: clusters of 4 CTAs (132 resident on 148 SMs), 1, 2 or 4 units
+    per tile from the cost model (qkv: 2, o: 4, gate_up: 2, down: 4), no
+    tail units."""
     specs = []
     for layer in range(3):
         for (k, n) in QWEN3_LAYER:
@@ -379,11 +382,46 @@ def test_chain_plan_dependent_layers():
     assert kernels == 1
     for s, p in zip(specs, plans):
         single = wsm.plan(16, s["N"], s["K"])
+        assert p["cluster"] == 0 and p["grid"] == 148
         assert p["unit_stages"] == single["unit_stages"] and p["units"] == single["units"], (s, p, single)
         assert p["l2_prefetch_stages"] == 4 and p["dep_ring_stages"] == 1 and p["k_order"] == wsm.K_ORDER_ROTATED
+    plans, _ = wsm.chain_plan(specs, cluster=wsm.CHAIN_CLUSTER_ON)
+    units_per_tile = {6144: 2, 4096: 4, 24576: 2}
+    for s, p in zip(specs, plans):
+        assert p["cluster"] == 4 and p["grid"] == 132, p
+        nu = p["units"] // (p["n_tiles"] * p["m_tiles"])
+        assert nu == units_per_tile[s["N"]], (s, p)
+        assert p["unit_stages"] * nu >= p["k_iters"] > p["unit_stages"] * (nu - 1)
+        assert p["tail_tiles"] == 0
     # explicit options pass through
     plans, _ = wsm.chain_plan(specs, l2_prefetch_stages=-1, dep_ring_stages=-1, k_order=wsm.K_ORDER_INCREASING)
     assert all(p["l2_prefetch_stages"] == 0 and p["dep_ring_stages"] == 0 and p["k_order"] == 1 for p in plans)
+
+
+def test_chain_plan_cluster_reduction_applies_only_to_linear_dependent_chains():
+    """Cluster reduction is used only on request, and only for a linear
+    dependent tensor-core chain: independent tasks, a task that skips its
+    predecessor, two-level counters, the FMA path, an explicit split of 8
+    units per tile or tail units are refused with WSM_ERR_UNSUPPORTED; a grid
+    option is rounded down to whole clusters."""
+    ON = wsm.CHAIN_CLUSTER_ON
+    lin = [dict(M=16, N=4096, K=4096, dep=i - 1) for i in range(4)]
+    assert all(p["cluster"] == 0 for p in wsm.chain_plan(lin)[0])
+    assert all(p["cluster"] == 0 for p in wsm.chain_plan(lin, cluster=wsm.CHAIN_CLUSTER_OFF)[0])
+    assert all(p["cluster"] == 4 for p in wsm.chain_plan(lin, cluster=ON)[0])
+    assert all(p["grid"] == 64 for p in wsm.chain_plan(lin, grid=66, cluster=ON)[0])
+    assert all(p["cluster"] == 4 and p["unit_stages"] == 4 for p in wsm.chain_plan(lin, unit_stages=4, cluster=ON)[0])
+    indep = [dict(M=16, N=4096, K=4096) for _ in range(4)]
+    skip = [dict(M=16, N=4096, K=4096, dep=d) for d in (-1, 0, 0, 2)]
+    lin_fma = [dict(M=2, N=4096, K=4096, dep=i - 1) for i in range(4)]
+    for bad, kw in ((indep, {}), (skip, {}), (lin, dict(counter_groups=2)), (lin_fma, {}), (lin, dict(unit_stages=2)),
+                    (lin, dict(tail_tiles=8))):
+        with pytest.raises(wsm.WsmError) as e:
+            wsm.chain_plan(bad, cluster=ON, **kw)
+        assert e.value.code == wsm.WSM_ERR_UNSUPPORTED, kw
+    with pytest.raises(wsm.WsmError) as e:
+        wsm.chain_plan(lin, cluster=7)
+    assert e.value.code == wsm.WSM_ERR_INVALID
 
 
 def test_chain_plan_wide_x_and_fma():

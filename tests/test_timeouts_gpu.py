@@ -130,12 +130,19 @@ def test_one_shot_chain_timeout_reported_once_then_correct(M):
         _check_dependent(x0, ws, ys, yfs, f"run {rep} after the time-out")
 
 
-def test_prepared_chain_graph_replays_after_timeout():
+@pytest.mark.parametrize("cluster", [wsm.CHAIN_CLUSTER_OFF, wsm.CHAIN_CLUSTER_ON])
+def test_prepared_chain_graph_replays_after_timeout(cluster):
     """A prepared chain captured in a CUDA graph: a time-out in an eager run
     is reported once by wsm_chain_status, and later graph replays (which read
-    the run counter from device memory) stay ordered and correct."""
+    the run counter from device memory) stay ordered and correct.  With
+    cluster reduction the abandoned CTA's peers give up on their exchanges
+    (tasks split 2 and 4 ways), and the waits of the failed run stop ordering
+    its tasks; the exchange must stay well defined through all of that."""
     x0, ws, ys, yfs, tasks = _dependent_tasks(16, [512, 2048, 512, 1024, 512], seed=9)
-    ch = wsm.Chain(tasks, path=wsm.PATH_UMMA)
+    ch = wsm.Chain(tasks, path=wsm.PATH_UMMA, cluster=cluster)
+    if cluster == wsm.CHAIN_CLUSTER_ON:
+        nus = {ch.task_plan(t)["units"] // ch.task_plan(t)["n_tiles"] for t in range(len(tasks))}
+        assert nus == {2, 4}
     s = torch.cuda.Stream()
     ch.run(s)
     assert ch.status(s)[0] == wsm.WSM_OK

@@ -38,6 +38,7 @@ FLAG_W_READONLY, FLAG_NO_PDL = 1, 2
 EPI_NONE, EPI_SILU_MUL, EPI_RESIDUAL = 0, 1, 2
 CHAIN_KERNELS_AUTO, CHAIN_KERNELS_ONE, CHAIN_KERNELS_SPLIT = 0, 1, 2
 K_ORDER_AUTO, K_ORDER_INCREASING, K_ORDER_ROTATED = 0, 1, 2
+CHAIN_CLUSTER_AUTO, CHAIN_CLUSTER_OFF, CHAIN_CLUSTER_ON = 0, 1, 2
 
 # Every function include/wsm.h declares (checked by the CPU tests).
 HEADER_SYMBOLS = (
@@ -84,7 +85,7 @@ class _Task(ctypes.Structure):
 
 class _ChainTaskInfo(ctypes.Structure):
     _fields_ = [("plan", _PlanInfo), ("kernel", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int),
-                ("k_order", ctypes.c_int), ("dep_ring_stages", ctypes.c_int)]
+                ("k_order", ctypes.c_int), ("dep_ring_stages", ctypes.c_int), ("cluster", ctypes.c_int)]
 
 
 class _ChainOpts(ctypes.Structure):
@@ -93,7 +94,7 @@ class _ChainOpts(ctypes.Structure):
                 ("stage_k", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
                 ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int),
                 ("counter_groups", ctypes.c_int), ("tile_rows", ctypes.c_int), ("k_order", ctypes.c_int),
-                ("dep_ring_stages", ctypes.c_int), ("kernels", ctypes.c_int)]
+                ("dep_ring_stages", ctypes.c_int), ("kernels", ctypes.c_int), ("cluster", ctypes.c_int)]
 
 
 _lib = None
@@ -361,7 +362,7 @@ def chain_validate(tasks) -> None:
 
 def _chain_opts(path=PATH_AUTO, grid=0, timeout_ns=0, trace=False, debug_unmet_dependency=False, flags=0,
                 stage_k=0, unit_stages=0, tail_tiles=0, tail_unit_stages=0, l2_prefetch_stages=0,
-                counter_groups=0, kernels=0, tile_rows=0, k_order=0, dep_ring_stages=0) -> "_ChainOpts":
+                counter_groups=0, kernels=0, tile_rows=0, k_order=0, dep_ring_stages=0, cluster=0) -> "_ChainOpts":
     o = _ChainOpts()
     o.path, o.grid, o.timeout_ns, o.trace = path, grid, timeout_ns, 1 if trace else 0
     o.debug_unmet_dependency = 1 if debug_unmet_dependency else 0
@@ -373,6 +374,7 @@ def _chain_opts(path=PATH_AUTO, grid=0, timeout_ns=0, trace=False, debug_unmet_d
     o.tile_rows = tile_rows
     o.k_order = k_order
     o.dep_ring_stages = dep_ring_stages
+    o.cluster = cluster
     return o
 
 
@@ -405,7 +407,7 @@ def chain_plan(specs, num_sms: int = 148, **opts):
     for i in range(n):
         d = {f: getattr(out[i].plan, f) for f, _ in _PlanInfo._fields_}
         d.update(kernel=out[i].kernel, l2_prefetch_stages=out[i].l2_prefetch_stages, k_order=out[i].k_order,
-                 dep_ring_stages=out[i].dep_ring_stages)
+                 dep_ring_stages=out[i].dep_ring_stages, cluster=out[i].cluster)
         res.append(d)
     return res, nk.value
 
@@ -416,7 +418,7 @@ class Chain:
     def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
                  debug_unmet_dependency=False, flags=0, stage_k=0, unit_stages=0, tail_tiles=0,
                  tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0, kernels=0, tile_rows=0, k_order=0,
-                 dep_ring_stages=0):
+                 dep_ring_stages=0, cluster=0):
         for i, t in enumerate(tasks):
             _check_operand(f"tasks[{i}].x", t.x)
             _check_operand(f"tasks[{i}].w", t.w)
@@ -427,7 +429,7 @@ class Chain:
                         debug_unmet_dependency=debug_unmet_dependency, flags=flags, stage_k=stage_k,
                         unit_stages=unit_stages, tail_tiles=tail_tiles, tail_unit_stages=tail_unit_stages,
                         l2_prefetch_stages=l2_prefetch_stages, counter_groups=counter_groups, kernels=kernels,
-                        tile_rows=tile_rows, k_order=k_order, dep_ring_stages=dep_ring_stages)
+                        tile_rows=tile_rows, k_order=k_order, dep_ring_stages=dep_ring_stages, cluster=cluster)
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

@@ -54,6 +54,16 @@ std::mutex g_mu;
 // sm_100 opt-in limit of dynamic + static shared memory per block.
 constexpr int kSmemOptin = 232448;
 constexpr int kRingBudget = kSmemOptin - 8192;  // static shared memory + 1 KB alignment slack
+constexpr int kStaticSmemMax = 2048;            // bound on the kernels' static shared memory (ptxas: 1 KB)
+// Clusters of kClusterCtas CTAs resident at once, per 148 SMs, at one CTA per SM: measured on B200
+// (cudaOccupancyMaxActiveClusters: 33, i.e. 132 CTAs; clusters never straddle a GPC, so some SMs stay
+// out).  Used only to model the grid of a cluster chain in host-only planning (wsm_chain_plan); chain
+// creation asks the device.
+constexpr int kClustersPer148Sms = 33;
+
+// Exchange buffer of a cluster-reduction chain: the quadrant rows of up to three senders, each lane's row
+// the widest X tile's values plus 4 floats (the row's flag and padding; see the kernel).
+int xbuf_bytes_of(int t_mpad) { return 3 * 32 * (t_mpad + 4) * 4; }
 
 // W stages per waiting CTA prefetched into L2 (auto).  Measured on B200: 4
 // stages gain ~4 % on a dependent layer chain and 1-4 % on back-to-back
@@ -431,6 +441,7 @@ struct DevInfo {
     int sms = 0;
     int smem_optin = 0;
     bool attr_set[16] = {};
+    int cluster_ctas = -1;  // CTAs of the tensor-core kernel resident as clusters of kClusterCtas (-1: not asked)
 };
 std::map<int, DevInfo> g_dev;
 
@@ -468,9 +479,44 @@ wsm_status prepare_kernel(DevInfo *d, const Geo &g, const void **fn) {
     *fn = kernel_for(g, &slot);
     std::lock_guard<std::mutex> lk(g_mu);
     if (!d->attr_set[slot]) {
-        WSM_CUDA(cudaFuncSetAttribute(*fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingBudget + 1024));
+        // all the shared memory a block may have, less the kernel's static part (the ring, its alignment
+        // slack and, in cluster chains, the exchange buffer are dynamic)
+        cudaFuncAttributes fa;
+        WSM_CUDA(cudaFuncGetAttributes(&fa, *fn));
+        WSM_CUDA(cudaFuncSetAttribute(*fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kSmemOptin - (int)fa.sharedSizeBytes));
         d->attr_set[slot] = true;
     }
+    return WSM_OK;
+}
+
+// CTAs of the tensor-core kernel that can be resident at once as clusters of kClusterCtas (0 if none).
+wsm_status cluster_ctas_of(DevInfo *d, int *out) {
+    Geo g;
+    g.path = WSM_PATH_UMMA;
+    const void *fn;
+    wsm_status st = prepare_kernel(d, g, &fn);
+    if (st != WSM_OK) return st;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (d->cluster_ctas < 0) {
+        cudaFuncAttributes fa;
+        WSM_CUDA(cudaFuncGetAttributes(&fa, fn));
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(d->sms / kClusterCtas * kClusterCtas));
+        cfg.blockDim = dim3(64 + 2 * 128);
+        cfg.dynamicSmemBytes = (size_t)(kSmemOptin - (int)fa.sharedSizeBytes);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kClusterCtas;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        WSM_CUDA(cudaOccupancyMaxActiveClusters(&n, fn, &cfg));
+        d->cluster_ctas = n * kClusterCtas;
+    }
+    *out = d->cluster_ctas;
     return WSM_OK;
 }
 
@@ -639,14 +685,22 @@ int pdl_mode(int flags) {
     return (flags & WSM_FLAG_W_READONLY) ? 2 : 1;
 }
 
-wsm_status launch(const void *fn, const Geo &g, const KParams &kp, cudaStream_t stream, bool cooperative) {
+wsm_status launch(const void *fn, const Geo &g, const KParams &kp, cudaStream_t stream, bool cooperative,
+                  size_t extra_smem = 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)g.grid);
     cfg.blockDim = dim3((unsigned)g.threads);
-    cfg.dynamicSmemBytes = (size_t)kp.stages * kp.stage_bytes + 1024;
+    cfg.dynamicSmemBytes = (size_t)kp.stages * kp.stage_bytes + 1024 + extra_smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[3];
     int na = 0;
+    if (kp.cluster) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)kp.cluster;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
     if (cooperative) {
         attr[na].id = cudaLaunchAttributeCooperative;
         attr[na].val.cooperative = 1;
@@ -695,6 +749,8 @@ struct wsm_chain {
     int prefetch_stages = 0;
     int k_rotate = 0;
     int dep_ring_stages = 0;
+    int cluster = 0;                   // CTAs per cluster (cluster reduction), or 0
+    int xbuf_bytes = 0;                // cluster reduction: exchange buffer behind the ring
     std::vector<wsm::Geo> task_geo;    // each task's plan (wsm_chain_task_plan)
     const void *fn = nullptr;
 };
@@ -749,7 +805,31 @@ struct ChainPlan {
     int grid = 0;
     int groups = 1;
     int prefetch_stages = 0, k_rotate = 0, dep_ring_stages = 0;
+    int cluster = 0;     // CTAs per cluster with cluster reduction, else 0
+    int xbuf_bytes = 0;  // its exchange buffer
 };
+
+// Units per tile of a task in a cluster-reduction chain: 1, 2 or 4, so the units of a tile of the static
+// first round fall on the CTAs of one cluster; the same cost in pipeline stages as auto_units_per_tile
+// (whole rounds of units plus a per-unit overhead), over the splits that are allowed.
+int cluster_unit_stages(const Geo &g, int ctas) {
+    const double G = std::max(1, ctas);
+    const double c = (g.t_mpad <= 32) ? 1.0 : 4.0;
+    int best_ku = g.kb;
+    double best_cost = 1e300;
+    for (int nu : {1, 2, 4}) {
+        const int ku = (g.kb + nu - 1) / nu;
+        const int nu_real = (g.kb + ku - 1) / ku;
+        if (nu_real != nu) continue;
+        const double units = (double)g.tiles() * nu;
+        const double cost = units <= 3 * G ? std::ceil(units / G) * (ku + c) : units / G * (ku + c) + 2.0 * ku;
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best_ku = ku;
+        }
+    }
+    return best_ku;
+}
 
 // Tasks [a, b) of a chain as a chain of their own: a dependency inside the
 // range is renumbered; one on an earlier task is met by stream order (the
@@ -775,9 +855,13 @@ wsm_chain_opts part_opts(const wsm_chain_opts &o) {
     return so;
 }
 
-wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, int sms, ChainPlan &cp) {
+// cluster_ctas: CTAs resident as clusters of kClusterCtas (from the device, or modelled), 0 if none.
+wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, int sms, ChainPlan &cp,
+                      int cluster_ctas) {
     cp = ChainPlan{};
     wsm_status st;
+    if (opts->cluster < WSM_CHAIN_CLUSTER_AUTO || opts->cluster > WSM_CHAIN_CLUSTER_ON)
+        return fail(WSM_ERR_INVALID, "bad cluster option %d", opts->cluster);
     if (opts->path < 0 || opts->path > WSM_PATH_UMMA) return fail(WSM_ERR_INVALID, "bad chain path %d", opts->path);
     if (opts->kernels < WSM_CHAIN_KERNELS_AUTO || opts->kernels > WSM_CHAIN_KERNELS_SPLIT)
         return fail(WSM_ERR_INVALID, "bad kernels option %d", opts->kernels);
@@ -876,7 +960,6 @@ wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, 
     }
     // one grid for the whole chain (make_geo clamps it per task to the task's stages)
     int chain_grid = (opts->grid > 0) ? std::min(opts->grid, sms) : sms;
-    for (auto &g : geos) g.grid = chain_grid;
     Geo ring = geos[0];
     if (path == WSM_PATH_STREAM) {
         stream_geo(pow2ceil(maxM), ring, to.tile_rows);
@@ -894,6 +977,46 @@ wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, 
     for (int i = 0; i < n; ++i)
         if (geos[i].kps != ring.kps || geos[i].tile_k != ring.tile_k || geos[i].wide != ring.wide)
             return fail(WSM_ERR_INVALID, "task %d: stage geometry differs from the chain's", i);  // cannot happen
+
+    // Cluster reduction (KParams::cluster), on request: for a linear dependent chain on the tensor-core path
+    // -- every task waits for the one before it, so the CTAs of a cluster meet each task's first round
+    // together and a CTA's exchanges never overlap.  The split tiles of each task's static first round are
+    // reduced through distributed shared memory instead of partials in L2.  Measured on B200 (36 x 4 chain
+    // at M = 16, traced): the exchange itself is not what bounds a dependency boundary -- at the boundary
+    // every memory operation waits behind the memory system's load (the exchange ~2 us after the last
+    // accumulator instead of ~0.2 us idle, the outputs' stores ~2-3 us), so it saves ~1 us per boundary,
+    // while clusters of 4 leave 16 SMs out (132 CTAs) and push qkv to a 2-way split on 96 of them: 3.41-3.51
+    // ms against 3.46 ms without.  Not the default.
+    {
+        bool linear = n >= 2;
+        for (int i = 1; i < n; ++i) linear = linear && tasks[i].dep == i - 1 && !tasks[i].dep_cols;
+        const int xb = path == WSM_PATH_UMMA ? xbuf_bytes_of((ring.x_stride / (kUmmaBK * 2))) : 0;
+        const bool fits =
+            path == WSM_PATH_UMMA && ring.stages * ring.stage_bytes + 1024 + xb + kStaticSmemMax <= kSmemOptin;
+        const int cl_grid = (opts->grid > 0 ? std::min(opts->grid, cluster_ctas) : cluster_ctas) / kClusterCtas *
+                            kClusterCtas;
+        // an explicit split must give every tile 1, 2 or 4 units, and there are no tail units
+        bool splits_ok = opts->tail_tiles <= 0;
+        for (int i = 0; i < n && splits_ok && opts->unit_stages > 0; ++i) {
+            const int ku = std::min(opts->unit_stages, geos[i].kb);
+            splits_ok = kClusterCtas % ((geos[i].kb + ku - 1) / ku) == 0;
+        }
+        const bool ok = path == WSM_PATH_UMMA && linear && groups <= 1 && !ring.wide && fits &&
+                        cl_grid >= kClusterCtas && splits_ok;
+        if (opts->cluster == WSM_CHAIN_CLUSTER_ON && !ok)
+            return fail(WSM_ERR_UNSUPPORTED,
+                        "cluster reduction needs a tensor-core chain in which every task waits for the one before "
+                        "it (whole-task waits, one counter level, 128-row tiles, 1, 2 or 4 units per tile, no tail "
+                        "units), an exchange buffer that fits, and room for clusters of %d CTAs",
+                        kClusterCtas);
+        if (ok && opts->cluster == WSM_CHAIN_CLUSTER_ON) {
+            cp.cluster = kClusterCtas;
+            cp.xbuf_bytes = xb;
+            chain_grid = cl_grid;
+        }
+    }
+    for (auto &g : geos) g.grid = chain_grid;
+    ring.grid = chain_grid;
     cp.prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, path);
     if (opts->l2_prefetch_stages == 0 && path == WSM_PATH_UMMA) {
         bool deps = false;
@@ -923,6 +1046,16 @@ wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, 
     for (int i = n - 2; i >= 0; --i)
         later[i] = tasks[i + 1].dep >= 0 ? 0 : later[i + 1] + geos[i + 1].tiles() * (long long)geos[i + 1].kb;
     for (int i = 0; i < n; ++i) {
+        if (cp.cluster) {
+            // 1, 2 or 4 units per tile, no tail units
+            const int unit_stages = opts->unit_stages ? opts->unit_stages : cluster_unit_stages(geos[i], chain_grid);
+            if ((st = plan_units(geos[i], chain_grid, unit_stages, -1, 0)) != WSM_OK)
+                return fail(st, "task %d: %s", i, g_err.c_str());
+            if (kClusterCtas % geos[i].nu != 0)
+                return fail(WSM_ERR_UNSUPPORTED, "task %d: cluster reduction needs 1, 2 or 4 units per tile (%d)", i,
+                            geos[i].nu);
+            continue;
+        }
         const bool grow = opts->unit_stages == 0 && !tasks[i].dep_cols && groups <= 1;
         const int unit_stages = grow ? chain_unit_stages(geos[i], chain_grid, later[i]) : opts->unit_stages;
         if ((st = plan_units(geos[i], chain_grid, unit_stages,
@@ -1108,7 +1241,8 @@ wsm_status wsm_chain_plan(const wsm_task *tasks, int n, const wsm_chain_opts *op
     wsm_chain_opts zo{};
     if (!opts) opts = &zo;
     ChainPlan cp;
-    if ((st = plan_chain(tasks, n, opts, num_sms, cp)) != WSM_OK) return st;
+    const int model_cluster_ctas = num_sms * kClustersPer148Sms / 148 * kClusterCtas;
+    if ((st = plan_chain(tasks, n, opts, num_sms, cp, model_cluster_ctas)) != WSM_OK) return st;
     auto report = [&](const ChainPlan &kp, int first, int k) {
         for (size_t i = 0; i < kp.geos.size(); ++i) {
             Geo g = kp.geos[i];
@@ -1122,6 +1256,7 @@ wsm_status wsm_chain_plan(const wsm_task *tasks, int n, const wsm_chain_opts *op
             o.l2_prefetch_stages = kp.prefetch_stages;
             o.k_order = kp.k_rotate ? WSM_K_ORDER_ROTATED : WSM_K_ORDER_INCREASING;
             o.dep_ring_stages = kp.dep_ring_stages;
+            o.cluster = kp.cluster;
         }
     };
     if (cp.parts.empty()) {
@@ -1132,7 +1267,7 @@ wsm_status wsm_chain_plan(const wsm_task *tasks, int n, const wsm_chain_opts *op
             std::vector<wsm_task> sub = sub_chain(tasks, a, b);
             const wsm_chain_opts so = part_opts(*opts);
             ChainPlan sp;
-            if ((st = plan_chain(sub.data(), b - a, &so, num_sms, sp)) != WSM_OK)
+            if ((st = plan_chain(sub.data(), b - a, &so, num_sms, sp, model_cluster_ctas)) != WSM_OK)
                 return fail(st, "tasks %d..%d: %s", a, b - 1, g_err.c_str());
             report(sp, a, (int)k);
         }
@@ -1153,8 +1288,10 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     WSM_CUDA(cudaGetDevice(&dev));
     DevInfo *d;
     if ((st = dev_info(dev, &d)) != WSM_OK) return st;
+    int cluster_ctas = 0;
+    if ((st = cluster_ctas_of(d, &cluster_ctas)) != WSM_OK) return st;
     ChainPlan cp;
-    if ((st = plan_chain(tasks, n, opts, d->sms, cp)) != WSM_OK) return st;
+    if ((st = plan_chain(tasks, n, opts, d->sms, cp, cluster_ctas)) != WSM_OK) return st;
 
     if (!cp.parts.empty()) {
         // hybrid dispatch: one chain per run of tasks of one X width, run back to back
@@ -1199,6 +1336,8 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     ch->prefetch_stages = cp.prefetch_stages;
     ch->k_rotate = cp.k_rotate;
     ch->dep_ring_stages = cp.dep_ring_stages;
+    ch->cluster = cp.cluster;
+    ch->xbuf_bytes = cp.xbuf_bytes;
     ch->task_geo = geos;
     for (Geo &g : ch->task_geo) {
         g.stages = ring.stages;
@@ -1382,7 +1521,10 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     kp.wait_timeout_ns = ch->dep_timeout_ns + kPipeTimeoutNs;
     kp.trace = ch->d_trace;
     kp.debug_stall_ns = take_stall();
-    return launch(ch->fn, ch->geo, kp, stream, ch->any_dep);
+    kp.cluster = ch->cluster;
+    kp.xbuf_off = ch->geo.stages * ch->geo.stage_bytes;
+    kp.xrow = ch->geo.x_stride / (kUmmaBK * 2) + 4;
+    return launch(ch->fn, ch->geo, kp, stream, ch->any_dep, ch->cluster ? (size_t)ch->xbuf_bytes : 0);
 }
 
 wsm_status wsm_chain_status(wsm_chain *ch, wsm_stream_t stream_, int *failed_task) {

@@ -50,6 +50,11 @@ constexpr int kStatusStallFlag = 5;
 constexpr int kSchedWords = 2;     // per task: [0] next unit to claim, [1] CTAs done claiming
 constexpr int kClaimLead = 4;      // a CTA claims its next unit this many stages before its unit ends
 constexpr int kColChunk = 256;     // output columns per readiness chunk (per-column data dependencies)
+// A task's `done` counter counts quarter tiles (32-row quadrants of a 128-row tile's outputs; a wide tile's
+// quarter is 64 rows): a finished tile adds 4, and in a cluster reduction each CTA adds the quadrants it
+// reduced and stored.  (With two-level readiness `done` counts groups instead.)
+constexpr int kDonePerTile = 4;
+constexpr int kClusterCtas = 4;    // CTAs per thread-block cluster in cluster-reduction chains
 // Trace stamps per CTA and task (%globaltimer ns unless noted): [0] first stage issued, [1] dependency
 // met, [2] last unit's outputs written, [3] SM id, [4] last unit's accumulator at the epilogue, [5] its
 // split-K arrival counted, [6] its in-order reduction done (last arriver only), [7] first stage of the
@@ -60,7 +65,8 @@ constexpr int kTraceSlots = 8;
 enum : int { kEpiNone = 0, kEpiSiluMul = 1, kEpiResidual = 2 };
 
 // Error sites recorded in status[3].
-enum : int { kSiteNone = 0, kSiteDep = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteAcc = 4, kSiteDrain = 5, kSiteStall = 6 };
+enum : int { kSiteNone = 0, kSiteDep = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteAcc = 4, kSiteDrain = 5, kSiteStall = 6,
+             kSiteXchg = 7 };
 constexpr int kCodeTimeout = 6;    // == WSM_ERR_TIMEOUT
 
 // Stage / accumulator metadata flags (producer -> consumers).
@@ -146,6 +152,13 @@ struct KParams {
     unsigned long long *trace;      // [grid][n_tasks][kTraceSlots] or nullptr
     unsigned long long debug_stall_ns;  // test hook, 0 in real use: CTA 0's producer waits this long on a flag
                                         // nothing sets, records a time-out and abandons its work
+    int cluster;                    // 0, or kClusterCtas: launched as clusters; every task's first round of
+                                    // units is static (unit c on CTA c) and a split tile of that round, whose
+                                    // units sit on the CTAs of one cluster, is reduced through distributed
+                                    // shared memory instead of global partials
+    int xbuf_off;                   // cluster mode: byte offset of the exchange buffer from the ring's start
+    int xrow;                       // cluster mode: floats per exchange-buffer row (widest X tile + 4, the
+                                    // last 4 holding the row's flag)
 };
 
 #if defined(__CUDACC__)
@@ -280,6 +293,59 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ------------------------------------------------------------------ thread-block clusters
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Every thread of every CTA of the cluster: all have arrived (and their earlier shared-memory writes,
+// mbarrier initialisation included, are visible cluster-wide) before any continues.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The shared::cluster address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// Arrive (count 1) on an mbarrier of another CTA of the cluster; release: this thread's earlier writes
+// (its distributed shared memory stores included) are visible to the thread that sees the phase complete.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Arrive with `count` on a local mbarrier; returns the token of the phase arrived on.
+__device__ __forceinline__ uint64_t mbar_arrive_count(uint64_t *bar, uint32_t count) {
+    uint64_t state;
+    asm volatile("mbarrier.arrive.shared::cta.b64 %0, [%1], %2;" : "=l"(state) : "r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+    return state;
+}
+
+// true once the phase of `state` has completed; acquire at cluster scope (remote writers' stores visible)
+__device__ __forceinline__ bool mbar_try_token_cluster(uint64_t *bar, uint64_t state) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "l"(state)
+        : "memory");
+    return ok != 0;
 }
 
 __device__ __forceinline__ float ld_cg_f32(const float *p) {
@@ -605,7 +671,7 @@ __device__ __forceinline__ void tile_finished(const UnitOut &o, int g, int rows_
         const unsigned int old = atom_add_acqrel_gpu(&o.grp_done[o.grp], 1u);
         if (old + 1u == run * (unsigned int)o.grp_tiles) red_release_gpu_add(o.done, 1u);
     } else if (o.done) {
-        red_release_gpu_add(o.done, 1u);
+        red_release_gpu_add(o.done, (unsigned int)kDonePerTile);
     }
     if (o.col_cnt) notify_columns(o, g, rows_per_tile);
 }
@@ -637,15 +703,20 @@ static __device__ __noinline__ void wait_chunks(const KParams &p, const TaskDev 
     fence_proxy_async_global();
 }
 
+// What a task's `done` counter reaches in each run: groups with two-level readiness, else quarter tiles.
+__device__ __forceinline__ unsigned int done_per_run(const TaskDev &D) {
+    return (unsigned int)(D.n_groups > 1 ? D.n_groups : D.n_g * D.n_mt * kDonePerTile);
+}
+
 __device__ __forceinline__ bool dependency_met(const KParams &p, const TaskDev &D) {
     const unsigned int run = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
-    const unsigned int target = run * (unsigned int)(D.n_groups > 1 ? D.n_groups : D.n_g * D.n_mt) + p.dep_target_extra;
+    const unsigned int target = run * done_per_run(D) + p.dep_target_extra;
     return ld_acquire_gpu(D.done) - target < 0x80000000u;  // done >= target (wrap-safe)
 }
 
 static __device__ __noinline__ void wait_dependency(const KParams &p, const TaskDev &D, int task, int *status) {
     const unsigned int run = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
-    const unsigned int target = run * (unsigned int)(D.n_groups > 1 ? D.n_groups : D.n_g * D.n_mt) + p.dep_target_extra;
+    const unsigned int target = run * done_per_run(D) + p.dep_target_extra;
     if (ld_acquire_gpu(D.done) - target < 0x80000000u) {  // done >= target (wrap-safe)
         fence_proxy_async_global();
         return;
@@ -693,7 +764,7 @@ __device__ __forceinline__ void chain_run_done(const KParams &p) {
                         st_relaxed_gpu(&T.grp_done[g], run * (unsigned int)(group_tile_lo(T, g + 1) - group_tile_lo(T, g)));
                     st_relaxed_gpu(T.done, run * (unsigned int)T.n_groups);
                 } else {
-                    st_relaxed_gpu(T.done, run * (unsigned int)tiles);
+                    st_relaxed_gpu(T.done, run * (unsigned int)(tiles * kDonePerTile));
                 }
             }
             if (T.col_cnt) {

@@ -219,6 +219,128 @@ __device__ __forceinline__ void reduce_row_partials(const UnitOut &uo, const Uni
     }
 }
 
+// Exchange buffer (cluster mode): for each quadrant a CTA reduces, one slot per other unit of the tile,
+// each slot 32 rows (one per lane) of p.xrow floats: the partial's t_mpad values, then a flag word.  The
+// row stride is the chain's widest X tile + 4 floats (so 16-byte accesses of 8 consecutive lanes fall in
+// distinct banks) and the flag sits at the same place in every task.
+__device__ __forceinline__ void st_release_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.release.cluster.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_cluster_u32(const void *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+
+// Bounded wait (per lane) until the flags of this lane's row in `nslots` slots reach `seq`.  Gives up when
+// this CTA aborted, when another CTA recorded an error in this launch, or after `limit_ns` (recording a
+// time-out).
+static __device__ __noinline__ bool xchg_wait(const float *row0, int slot_floats, int nslots, int flag_at,
+                                              uint32_t seq, volatile int *abort_flag, unsigned long long limit_ns,
+                                              int *status, int task) {
+    const unsigned long long t0 = globaltimer();
+    for (int sl = 0; sl < nslots; ++sl) {
+        const float *f = row0 + (size_t)sl * slot_floats + flag_at;
+        for (uint32_t spin = 0;; ++spin) {
+            if (ld_acquire_cluster_u32(f) - seq < 0x80000000u) break;  // flag >= seq
+            if ((spin & 63u) == 63u) {
+                if (*abort_flag || launch_failed(status)) return false;
+                if (globaltimer() - t0 > limit_ns) {
+                    record_error(status, kCodeTimeout, task, kSiteXchg);
+                    *abort_flag = 1;
+                    return false;
+                }
+            }
+        }
+    }
+    return true;
+}
+
+// Epilogue of a split tile whose nu units (nu = 2 or 4) run on consecutive CTAs of one cluster: a
+// reduce-scatter through distributed shared memory instead of partials in global memory.  The tile's 128
+// rows are four 32-row quadrants (one per epilogue warp, TMEM lane quadrant q); quadrant q is reduced by
+// the tile's CTA of index q % nu.  Every other CTA of the tile writes that quadrant's rows of its partial
+// into the reducing CTA's exchange buffer, each lane its own row followed by a release store of the row's
+// flag (the task's index + 1: every CTA takes part in at most one exchange per task, in task order).  The
+// reducing lane acquires the flags of its own row only, adds the nu partials in unit order (= K order, the
+// order of the global-memory reduction: the same bits), applies the epilogue and stores the outputs; the
+// CTA then counts its reduced quadrants toward the task's readiness.  No counted arrivals are involved, so
+// a failed launch, whose tasks are no longer ordered once its waits give up, can mix data but cannot put
+// any barrier in an undefined state.
+static __device__ __noinline__ void xchg_epilogue(const KParams &p, const UnitOut &uo, const UnitSpan &us, int t,
+                                                  int u, uint32_t taddr, int q, int lane, int n, int m0, int mrows,
+                                                  int set, bool leader, float *xbuf, uint64_t *acce,
+                                                  volatile int *abort_flag) {
+    const int nu = us.nu;
+    const int pj = u - us.u0;                 // this unit's index in its tile
+    const int base = (int)cluster_ctarank() - pj;  // cluster rank of the tile's unit 0
+    const int owner = q % nu;                 // the tile's CTA that reduces quadrant q
+    const int jq = q / nu;                    // which of the owner's quadrants it is
+    const int rowf = p.xrow;
+    const int slot_floats = 32 * rowf;
+    const int flag_at = rowf - 4;
+    const uint32_t seq = (uint32_t)t + 1u;
+    tc_fence_after();
+    if (owner != pj) {
+        const int sl = pj < owner ? pj : pj - 1;
+        const uint32_t dst = map_to_rank(smem_u32(xbuf + (size_t)(jq * (nu - 1) + sl) * slot_floats + lane * rowf),
+                                         (uint32_t)(base + owner));
+#pragma unroll 1
+        for (int c = 0; c < mrows; c += 16) {
+            uint32_t r[16];
+            tmem_ld16(taddr + (uint32_t)c, r);
+            tmem_ld_wait16(r);
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                st_cluster_v4(dst + (uint32_t)(c + i) * 4u, __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                              __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+        }
+        st_release_cluster_u32(dst + (uint32_t)flag_at * 4u, seq);
+    } else {
+        const float *rx = xbuf + (size_t)jq * (nu - 1) * slot_floats + lane * rowf;
+        const bool ok = __all_sync(0xffffffffu, xchg_wait(rx, slot_floats, nu - 1, flag_at, seq, abort_flag,
+                                                          p.wait_timeout_ns, p.status, t));
+        if (ok) {
+#pragma unroll 1
+            for (int c = 0; c < mrows; c += 16) {
+                uint32_t r[16];
+                tmem_ld16(taddr + (uint32_t)c, r);
+                tmem_ld_wait16(r);
+                float v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                for (int j = 0; j < nu; ++j) {
+                    float w[16];
+                    if (j == pj) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) w[i] = __uint_as_float(r[i]);
+                    } else {
+                        const float4 *src = reinterpret_cast<const float4 *>(rx + (size_t)(j < pj ? j : j - 1) *
+                                                                                       slot_floats + c);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float4 f = src[i];
+                            w[4 * i] = f.x; w[4 * i + 1] = f.y; w[4 * i + 2] = f.z; w[4 * i + 3] = f.w;
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = (j == 0) ? w[i] : v[i] + w[i];
+                }
+                emit_outputs<16>(uo.e, n, m0 + c, min(16, mrows - c), v);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acce);
+    epi_bar(set);  // the set's reducing warps have stored their outputs
+    if (leader) {
+        trace_stamp(p, t, 6, globaltimer());
+        if (uo.done) red_release_gpu_add(uo.done, (unsigned int)(kDonePerTile / nu));
+        trace_stamp(p, t, 2, globaltimer());
+    }
+}
+
 }  // namespace
 
 // L2 prefetch of the W of the units this CTA would own in a round-robin (c,
@@ -282,6 +404,12 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (p.cluster) {
+        // exchange flags start at 0 (no task's index + 1) before any peer can write them
+        float *xb = reinterpret_cast<float *>(ring + p.xbuf_off);
+        for (int i = threadIdx.x; i < 3 * 32; i += blockDim.x) xb[(size_t)i * p.xrow + p.xrow - 4] = 0.f;
+        cluster_sync_all();
+    }
     const uint32_t tmem_base = tmem_base_sh;
     const unsigned long long wlim = p.wait_timeout_ns;
 
@@ -392,7 +520,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 // previous task first take the next task's work.
                 // (with two-level readiness a CTA works only on its group's tiles, all claimed)
                 const ClaimRange cr = claim_range(T);
-                const bool static_first = t == 0 && T.n_groups <= 1;
+                // (cluster mode: every task's first round is static, so a split tile's units of that round
+                // sit on the consecutive CTAs of one cluster)
+                const bool static_first = (t == 0 || p.cluster) && T.n_groups <= 1;
                 const int n_static = static_first ? min((int)gridDim.x, T.n_units) : 0;
                 int u;
                 if (static_first) {
@@ -601,6 +731,13 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             const int mrows = min(T.t_m, T.M - m0);
             UnitOut uo = unit_out(T);  // no task-table reads after the first store below
             unit_out_group(uo, T, tile);
+            if (p.cluster && us.nu > 1 && u < min((int)gridDim.x, T.u_head)) {
+                // a split tile of a static first round: its units are on this cluster's CTAs
+                xchg_epilogue(p, uo, us, t, u, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * acc_stride, q,
+                              lane, g * kUmmaRows + row, m0, mrows, set, leader,
+                              reinterpret_cast<float *>(ring + p.xbuf_off), &acce_bar[buf], &abort_flag);
+                continue;
+            }
             // The accumulator, 16 columns (X rows) at a time, per 128-row half of the tile: TMEM ->
             // registers -> outputs (whole tile) or this unit's partial rows [row][m] (split tile).  The
             // loops are not unrolled: one copy of the epilogue code per kind keeps the kernel small.
@@ -675,6 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (p.cluster) cluster_sync_all();  // no CTA leaves while a peer may still write its exchange buffer
     if (warp == 1) tmem_dealloc(tmem_base, p.wide ? kTmemColsWide : kTmemCols);
     if (threadIdx.x == 0) {
         if (p.run_ctl) chain_run_done(p);
