@@ -91,6 +91,8 @@ def workload_cases(name):
         return synth.config_skinny()
     if name == "l2_reuse":
         return synth.config_l2_reuse()
+    if name == "l2_reuse_whole_m":
+        return synth.config_l2_reuse(m_tiles=(0,))
     if name == "chain":
         return synth.chain_layout()
     raise SystemExit(f"unknown workload {name}")
@@ -235,8 +237,8 @@ def run_e2e(args, wsm, dev, datas, copies, mode, total_bytes, world, stream, n_s
             gemms = [(c, view(xs[j], x), w, view(ys[j], y)) for c, x, w, y in datas[r]]
             if mode == "chain":
                 deps = [(i - 1) if args.workload == "chain" else -1 for i in range(len(gemms))]
-                ch = wsm.Chain([wsm.Task(x, w, y, dep=deps[i]) for i, (c, x, w, y) in enumerate(gemms)],
-                               flags=wsm.FLAG_W_READONLY)
+                ch = wsm.Chain([wsm.Task(x, w, y, dep=deps[i], m_tile=c.m_tile) for i, (c, x, w, y) in enumerate(gemms)],
+                               flags=wsm.FLAG_W_READONLY, die_groups=args.die_groups)
                 runs[j, r] = (lambda ch=ch: ch.run(s), ch)
             else:
                 def go(gemms=gemms):
@@ -327,8 +329,8 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
     if mode == "chain":
         # the whole step is one persistent kernel; the layer chain orders task t after t-1
         deps = [(i - 1) if args.workload == "chain" else -1 for i in range(len(data))]
-        chains = [wsm.Chain([wsm.Task(x, w, y, dep=deps[i]) for i, (c, x, w, y) in enumerate(d)],
-                            flags=wsm.FLAG_W_READONLY) for d in datas]
+        chains = [wsm.Chain([wsm.Task(x, w, y, dep=deps[i], m_tile=c.m_tile) for i, (c, x, w, y) in enumerate(d)],
+                            flags=wsm.FLAG_W_READONLY, die_groups=args.die_groups) for d in datas]
         chain = chains[0]
         launches_per_step = 1
 
@@ -486,7 +488,7 @@ def run_nshard(args, rank, world, local_rank):
         local.append(synth.Case(c.name, c.M, max(n1 - n0, 1), c.K, c.seed, c.m_tile))
     data = setup_inputs(local, dev, seed_base=rank)
     deps = [(i - 1) if args.workload == "chain" else -1 for i in range(len(data))]
-    chain = wsm.Chain([wsm.Task(x, w, y, dep=deps[i]) for i, (c, x, w, y) in enumerate(data)],
+    chain = wsm.Chain([wsm.Task(x, w, y, dep=deps[i], m_tile=c.m_tile) for i, (c, x, w, y) in enumerate(data)],
                       flags=wsm.FLAG_W_READONLY)
     stream = torch.cuda.Stream(dev)
 
@@ -567,6 +569,7 @@ CONFIGURATIONS = (
     ("c2_qwen3_8b_decode_gemms", "qwen3_decode", "chain", 0.80),
     ("c3_skinny_k7168_k8192", "skinny", "chain", 0.80),
     ("c4_l2_reuse_m32_m64", "l2_reuse", "chain", None),
+    ("c4_l2_reuse_m32_m64_whole_m_tile", "l2_reuse_whole_m", "chain", None),
     ("c5_chain_36x4_m16", "chain", "chain", 0.75),
 )
 
@@ -600,7 +603,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="wsm", choices=["wsm", "reference"])
     ap.add_argument("--workload", default="qwen3_decode",
-                    choices=["qwen3_decode", "single", "skinny", "l2_reuse", "chain"])
+                    choices=["qwen3_decode", "single", "skinny", "l2_reuse", "l2_reuse_whole_m", "chain"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
@@ -609,6 +612,8 @@ def main():
                     help="chain: the step is one persistent gemm_chain kernel; launches: one skinny_gemm per GEMM "
                          "(default: launches for the single-GEMM workload, chain otherwise)")
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-GEMM single-launch breakdown")
+    ap.add_argument("--die-groups", type=int, default=0, choices=[0, 1, 2],
+                    help="chains' die-grouped claims: 0 auto (M-tiled chains), 1 on, 2 off")
     ap.add_argument("--no-configurations", action="store_true",
                     help="skip the other four configurations (reported beside the default workload)")
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "nshard"],
@@ -631,6 +636,7 @@ def main():
             raise SystemExit(f"--only {args.only}: no case of workload {args.workload} has these names")
     config = {"workload": {"qwen3_decode": "qwen3_8b_decode_gemms", "single": "single_gemm_m1_4096x4096",
                            "skinny": "skinny_k7168_k8192", "l2_reuse": "l2_reuse_m32_m64",
+                           "l2_reuse_whole_m": "l2_reuse_m32_m64_whole_m_tile",
                            "chain": "chain_36x4_m16"}[args.workload],
               "gemms_per_step": len(cases),
               "M": sorted({c.M for c in cases}),

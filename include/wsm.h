@@ -282,6 +282,30 @@ wsm_status wsm_debug_stall(int calls, unsigned long long limit_ns);
 wsm_status skinny_gemm_noalloc(const void *X, const void *W, void *Y, int M, int N, int K,
                                wsm_stream_t stream);
 
+/* What the die probe found (wsm_sm_die_map). */
+typedef struct {
+    int num_sms;        /* SMs probed (all of the device's) */
+    int dies;           /* 2 when the SMs split into two groups with distinct near lines, else 1 */
+    int sms_die0;       /* SMs on die 0 (the die of the lowest SM id), */
+    int sms_die1;       /* and on die 1 */
+    float agreement;    /* mean fraction of probed lines on which an SM's near/far pattern agrees
+                           with its die's (1 = clean split, 0.5 = no structure) */
+    float near_cycles;  /* mean L2-hit latency (SM clock cycles) to lines homed on the SM's die, */
+    float far_cycles;   /* and to lines homed on the other die */
+} wsm_die_info;
+
+/* Which die of the current device each SM sits on: die_of_sm[smid] = 0 or 1
+ * (-1 past the last SM id), for smid < capacity; `info` may be NULL.  CUDA
+ * does not expose this, so it is measured: one CTA per SM times L2 hits to a
+ * set of lines; each line is nearer to the SMs of its home die, so the SMs of
+ * one die agree on which lines are near (the die of SM id 0's reference
+ * group is die 0).  Runs once per device (synchronous, a few ms, allocates
+ * ~9 MB of device memory while it runs) and is cached.  If the SMs do not
+ * split cleanly, info->dies = 1 and every SM is reported on die 0.  No
+ * counterpart API on the pages; it serves the chiplet-aware grouping of the
+ * Fleet reading notes (sections 3b and 3f). */
+wsm_status wsm_sm_die_map(int *die_of_sm, int capacity, wsm_die_info *info);
+
 /* ---------------------------------------------------------------- chains */
 
 /* One GEMM of a chain.  dep = -1, or the index of an EARLIER task whose Y
@@ -305,6 +329,8 @@ typedef struct {
     int epilogue;  /* WSM_EPI_* (as in wsm_opts) */
     const void *R; /* WSM_EPI_RESIDUAL: bf16 [M, N] */
     int dep_cols;  /* nonzero: per-column data dependency on task dep (see above) */
+    int m_tile;    /* tensor-core path: X rows per tile as in wsm_opts.m_tile (0 = all of M;
+                      else a multiple of 16 in [16, 64]); the FMA path takes 0 only */
 } wsm_task;
 
 typedef struct {
@@ -370,7 +396,28 @@ typedef struct {
                                   included, and the 16 SMs left out cost as much as it saves.
                                   AUTO and OFF: never; ON: always (WSM_ERR_UNSUPPORTED where it
                                   does not apply). */
+    int die_groups;            /* WSM_DIE_GROUPS_*: group the CTAs by the die their SM sits on
+                                  (wsm_sm_die_map) -- the chiplet-aware scheduling of the Fleet
+                                  reading notes, sections 3b and 3f.  Each task's tiles are cut
+                                  into one contiguous range per die (in proportion to the die's
+                                  SMs); a CTA claims the units of its own die's range first (in
+                                  M-major order, so the M-tiles of a weight column are read by
+                                  SMs of one die) and then helps with the other range, so no
+                                  range waits for a die without CTAs.  Tensor-core path only; not
+                                  with counter_groups, cluster reduction or dep_cols.  Measured on
+                                  B200 (M = 32 / 64 in 16-row M-tiles): 2.2 % faster, DRAM bytes
+                                  unchanged (every column is read from HBM once either way).
+                                  AUTO: on for a chain with an M-tiled task (m_tile < M) when the
+                                  probe finds two dies; ON: always (WSM_ERR_UNSUPPORTED where it
+                                  does not apply); OFF: never.  Creating the first chain that uses
+                                  it on a device runs the die probe (synchronous, a few ms). */
 } wsm_chain_opts;
+
+enum {
+    WSM_DIE_GROUPS_AUTO = 0,
+    WSM_DIE_GROUPS_ON = 1,
+    WSM_DIE_GROUPS_OFF = 2
+};
 
 enum {
     WSM_CHAIN_CLUSTER_AUTO = 0,
@@ -402,6 +449,8 @@ typedef struct {
     int k_order;            /* WSM_K_ORDER_INCREASING or WSM_K_ORDER_ROTATED, */
     int dep_ring_stages;    /* W stages streamed ahead of an unmet dependency (0 = the whole ring) */
     int cluster;            /* CTAs per thread-block cluster with cluster reduction, 0 without */
+    int die_split;          /* die-grouped claims: first tile of the second die's range (host-only
+                               planning assumes two dies of equal SM counts); 0 without */
 } wsm_chain_task_info;
 
 /* Pure host function (no CUDA calls, no memory touched): the plan

@@ -68,7 +68,8 @@ def config_skinny(ms=(1, 4, 8)):
 
 
 def config_l2_reuse(ms=(32, 64), m_tiles=(16, 32)):
-    """gate_up and down at M in {32, 64} with M-tile 16 or 32."""
+    """gate_up and down at M in {32, 64} with M-tile 16 or 32 (0: all of M in
+    one tile, for comparison)."""
     shapes = [s for s in QWEN3_8B_LAYER if s[0] in ("gate_up", "down")]
     return [Case(f"{name}_m{M}_tm{tm}", M, N, K, 0, tm)
             for M in ms for tm in m_tiles for (name, K, N) in shapes]

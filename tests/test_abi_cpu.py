@@ -424,6 +424,30 @@ def test_chain_plan_cluster_reduction_applies_only_to_linear_dependent_chains():
     assert e.value.code == wsm.WSM_ERR_INVALID
 
 
+def test_chain_plan_die_groups():
+    """Die-grouped claims: each task's tiles split in two contiguous ranges
+    (equal dies assumed by host-only planning), no tail units; refused on the
+    FMA path, with two-level counters, cluster reduction or dep_cols."""
+    specs = [dict(M=m, N=n, K=k, m_tile=0) for m in (32, 64) for (k, n) in QWEN3_LAYER[2:]]
+    specs = [dict(M=s["M"], N=s["N"], K=s["K"]) for s in specs]
+    plans, _ = wsm.chain_plan(specs, die_groups=wsm.DIE_GROUPS_ON)
+    for p in plans:
+        tiles = p["n_tiles"] * p["m_tiles"]
+        assert p["die_split"] == tiles // 2 or p["die_split"] == (tiles + 1) // 2, p
+        assert p["tail_tiles"] == 0
+    assert all(p["die_split"] == 0 for p in wsm.chain_plan(specs)[0])  # no M-tiled task: auto leaves it off
+    tiled = [dict(s, m_tile=16) for s in specs]
+    assert all(p["die_split"] > 0 for p in wsm.chain_plan(tiled)[0])   # M-tiled: auto groups
+    assert all(p["die_split"] == 0 for p in wsm.chain_plan(tiled, die_groups=wsm.DIE_GROUPS_OFF)[0])
+    lin = [dict(M=16, N=4096, K=4096, dep=i - 1) for i in range(3)]
+    for kw in (dict(path=wsm.PATH_STREAM, specs=[dict(M=2, N=4096, K=4096)]), dict(counter_groups=2),
+               dict(cluster=wsm.CHAIN_CLUSTER_ON)):
+        sp = kw.pop("specs", lin)
+        with pytest.raises(wsm.WsmError) as e:
+            wsm.chain_plan(sp, die_groups=wsm.DIE_GROUPS_ON, **kw)
+        assert e.value.code == wsm.WSM_ERR_UNSUPPORTED, kw
+
+
 def test_chain_plan_wide_x_and_fma():
     """M = 32 / 64 tasks keep 4 prefetch stages (wider X tiles); a chain of
     M = 1 GEMMs runs on the FMA path in increasing K order, without prefetch,

@@ -22,7 +22,7 @@ __all__ = [
     "WSM_ERR_CUDA", "WSM_ERR_TIMEOUT", "PATH_AUTO", "PATH_STREAM", "PATH_UMMA", "ORDER_AUTO", "ORDER_M_MAJOR",
     "ORDER_NAIVE", "L2_AUTO", "L2_EVICT_FIRST", "L2_NORMAL", "FLAG_W_READONLY", "FLAG_NO_PDL", "WsmError", "lib", "skinny_gemm", "plan",
     "workspace_bytes", "stream_status", "Task", "Chain", "gemm_chain", "chain_validate", "chain_plan", "last_error",
-    "skinny_gemm_noalloc", "workspace_status", "gemm_chain_status", "debug_stall",
+    "skinny_gemm_noalloc", "workspace_status", "gemm_chain_status", "debug_stall", "sm_die_map",
     "abi_version", "HEADER_SYMBOLS",
 ]
 
@@ -39,11 +39,12 @@ EPI_NONE, EPI_SILU_MUL, EPI_RESIDUAL = 0, 1, 2
 CHAIN_KERNELS_AUTO, CHAIN_KERNELS_ONE, CHAIN_KERNELS_SPLIT = 0, 1, 2
 K_ORDER_AUTO, K_ORDER_INCREASING, K_ORDER_ROTATED = 0, 1, 2
 CHAIN_CLUSTER_AUTO, CHAIN_CLUSTER_OFF, CHAIN_CLUSTER_ON = 0, 1, 2
+DIE_GROUPS_AUTO, DIE_GROUPS_ON, DIE_GROUPS_OFF = 0, 1, 2
 
 # Every function include/wsm.h declares (checked by the CPU tests).
 HEADER_SYMBOLS = (
     "skinny_gemm", "skinny_gemm_ex", "wsm_plan", "wsm_workspace_bytes", "wsm_stream_status", "wsm_workspace_status",
-    "wsm_debug_stall", "skinny_gemm_noalloc", "gemm_chain_status",
+    "wsm_debug_stall", "skinny_gemm_noalloc", "gemm_chain_status", "wsm_sm_die_map",
     "wsm_chain_plan", "wsm_chain_create", "wsm_chain_run", "wsm_chain_status", "wsm_chain_task_plan",
     "wsm_chain_trace",
     "wsm_chain_destroy",
@@ -80,12 +81,20 @@ class _PlanInfo(ctypes.Structure):
 class _Task(ctypes.Structure):
     _fields_ = [("X", ctypes.c_void_p), ("W", ctypes.c_void_p), ("Y", ctypes.c_void_p),
                 ("M", ctypes.c_int), ("N", ctypes.c_int), ("K", ctypes.c_int), ("dep", ctypes.c_int),
-                ("Yf32", ctypes.c_void_p), ("epilogue", ctypes.c_int), ("R", ctypes.c_void_p), ("dep_cols", ctypes.c_int)]
+                ("Yf32", ctypes.c_void_p), ("epilogue", ctypes.c_int), ("R", ctypes.c_void_p), ("dep_cols", ctypes.c_int),
+                ("m_tile", ctypes.c_int)]
 
 
 class _ChainTaskInfo(ctypes.Structure):
     _fields_ = [("plan", _PlanInfo), ("kernel", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int),
-                ("k_order", ctypes.c_int), ("dep_ring_stages", ctypes.c_int), ("cluster", ctypes.c_int)]
+                ("k_order", ctypes.c_int), ("dep_ring_stages", ctypes.c_int), ("cluster", ctypes.c_int),
+                ("die_split", ctypes.c_int)]
+
+
+class _DieInfo(ctypes.Structure):
+    _fields_ = [("num_sms", ctypes.c_int), ("dies", ctypes.c_int), ("sms_die0", ctypes.c_int),
+                ("sms_die1", ctypes.c_int), ("agreement", ctypes.c_float), ("near_cycles", ctypes.c_float),
+                ("far_cycles", ctypes.c_float)]
 
 
 class _ChainOpts(ctypes.Structure):
@@ -94,7 +103,8 @@ class _ChainOpts(ctypes.Structure):
                 ("stage_k", ctypes.c_int), ("unit_stages", ctypes.c_int), ("tail_tiles", ctypes.c_int),
                 ("tail_unit_stages", ctypes.c_int), ("l2_prefetch_stages", ctypes.c_int),
                 ("counter_groups", ctypes.c_int), ("tile_rows", ctypes.c_int), ("k_order", ctypes.c_int),
-                ("dep_ring_stages", ctypes.c_int), ("kernels", ctypes.c_int), ("cluster", ctypes.c_int)]
+                ("dep_ring_stages", ctypes.c_int), ("kernels", ctypes.c_int), ("cluster", ctypes.c_int),
+                ("die_groups", ctypes.c_int)]
 
 
 _lib = None
@@ -127,6 +137,8 @@ def lib() -> ctypes.CDLL:
         L.wsm_debug_stall.restype = st
         L.gemm_chain_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
         L.gemm_chain_status.restype = st
+        L.wsm_sm_die_map.argtypes = [ctypes.POINTER(ctypes.c_int), i, ctypes.POINTER(_DieInfo)]
+        L.wsm_sm_die_map.restype = st
         L.wsm_chain_task_plan.argtypes = [vp, i, ctypes.POINTER(_PlanInfo)]
         L.wsm_chain_task_plan.restype = st
         L.wsm_chain_create.argtypes = [ctypes.POINTER(_Task), i, ctypes.POINTER(_ChainOpts), ctypes.POINTER(vp)]
@@ -317,6 +329,16 @@ def gemm_chain_status(stream=None):
     return rc, ft.value
 
 
+def sm_die_map(capacity: int = 1024):
+    """Which die each SM of the current device sits on (measured once per
+    device): (list die_of_sm indexed by SM id, -1 past the last SM; dict of
+    the probe's findings)."""
+    arr = (ctypes.c_int * capacity)()
+    info = _DieInfo()
+    _check(lib().wsm_sm_die_map(arr, capacity, ctypes.byref(info)), "wsm_sm_die_map")
+    return list(arr), {f: getattr(info, f) for f, _ in _DieInfo._fields_}
+
+
 def debug_stall(calls: int, limit_ns: int = 50_000_000) -> None:
     """Test hook: the next `calls` launches each stall CTA 0 on a flag nothing
     sets for limit_ns, then record WSM_ERR_TIMEOUT (no fault); 0 cancels."""
@@ -333,6 +355,7 @@ class Task:
     epilogue: int = EPI_NONE
     r: Optional[torch.Tensor] = None
     dep_cols: bool = False
+    m_tile: int = 0
 
 
 def _tasks_array(tasks: Sequence[Task]):
@@ -344,6 +367,7 @@ def _tasks_array(tasks: Sequence[Task]):
         arr[i].M, arr[i].N, arr[i].K, arr[i].dep = M, N, K, t.dep
         arr[i].Yf32 = _ptr(t.yf32)
         arr[i].epilogue, arr[i].R, arr[i].dep_cols = t.epilogue, _ptr(t.r), 1 if t.dep_cols else 0
+        arr[i].m_tile = t.m_tile
     return arr
 
 
@@ -357,12 +381,14 @@ def chain_validate(tasks) -> None:
         arr[i].M, arr[i].N, arr[i].K, arr[i].dep = t["M"], t["N"], t["K"], t.get("dep", -1)
         arr[i].Yf32 = t.get("Yf32")
         arr[i].epilogue, arr[i].R, arr[i].dep_cols = t.get("epilogue", 0), t.get("R"), int(bool(t.get("dep_cols")))
+        arr[i].m_tile = t.get("m_tile", 0)
     _check(lib().wsm_chain_validate(arr, len(tasks)), "wsm_chain_validate")
 
 
 def _chain_opts(path=PATH_AUTO, grid=0, timeout_ns=0, trace=False, debug_unmet_dependency=False, flags=0,
                 stage_k=0, unit_stages=0, tail_tiles=0, tail_unit_stages=0, l2_prefetch_stages=0,
-                counter_groups=0, kernels=0, tile_rows=0, k_order=0, dep_ring_stages=0, cluster=0) -> "_ChainOpts":
+                counter_groups=0, kernels=0, tile_rows=0, k_order=0, dep_ring_stages=0, cluster=0,
+                die_groups=0) -> "_ChainOpts":
     o = _ChainOpts()
     o.path, o.grid, o.timeout_ns, o.trace = path, grid, timeout_ns, 1 if trace else 0
     o.debug_unmet_dependency = 1 if debug_unmet_dependency else 0
@@ -375,6 +401,7 @@ def _chain_opts(path=PATH_AUTO, grid=0, timeout_ns=0, trace=False, debug_unmet_d
     o.k_order = k_order
     o.dep_ring_stages = dep_ring_stages
     o.cluster = cluster
+    o.die_groups = die_groups
     return o
 
 
@@ -399,6 +426,7 @@ def chain_plan(specs, num_sms: int = 148, **opts):
         arr[i].epilogue = t.get("epilogue", EPI_NONE)
         arr[i].R = base - (1 << 24) if arr[i].epilogue == EPI_RESIDUAL else None
         arr[i].dep_cols = 1 if t.get("dep_cols") else 0
+        arr[i].m_tile = t.get("m_tile", 0)
     out = (_ChainTaskInfo * max(n, 1))()
     nk = ctypes.c_int(0)
     o = _chain_opts(**opts)
@@ -407,7 +435,7 @@ def chain_plan(specs, num_sms: int = 148, **opts):
     for i in range(n):
         d = {f: getattr(out[i].plan, f) for f, _ in _PlanInfo._fields_}
         d.update(kernel=out[i].kernel, l2_prefetch_stages=out[i].l2_prefetch_stages, k_order=out[i].k_order,
-                 dep_ring_stages=out[i].dep_ring_stages, cluster=out[i].cluster)
+                 dep_ring_stages=out[i].dep_ring_stages, cluster=out[i].cluster, die_split=out[i].die_split)
         res.append(d)
     return res, nk.value
 
@@ -418,7 +446,7 @@ class Chain:
     def __init__(self, tasks: Sequence[Task], *, path=PATH_AUTO, grid=0, timeout_ns=0, trace=False,
                  debug_unmet_dependency=False, flags=0, stage_k=0, unit_stages=0, tail_tiles=0,
                  tail_unit_stages=0, l2_prefetch_stages=0, counter_groups=0, kernels=0, tile_rows=0, k_order=0,
-                 dep_ring_stages=0, cluster=0):
+                 dep_ring_stages=0, cluster=0, die_groups=0):
         for i, t in enumerate(tasks):
             _check_operand(f"tasks[{i}].x", t.x)
             _check_operand(f"tasks[{i}].w", t.w)
@@ -429,7 +457,8 @@ class Chain:
                         debug_unmet_dependency=debug_unmet_dependency, flags=flags, stage_k=stage_k,
                         unit_stages=unit_stages, tail_tiles=tail_tiles, tail_unit_stages=tail_unit_stages,
                         l2_prefetch_stages=l2_prefetch_stages, counter_groups=counter_groups, kernels=kernels,
-                        tile_rows=tile_rows, k_order=k_order, dep_ring_stages=dep_ring_stages, cluster=cluster)
+                        tile_rows=tile_rows, k_order=k_order, dep_ring_stages=dep_ring_stages, cluster=cluster,
+                        die_groups=die_groups)
         h = ctypes.c_void_p()
         _check(lib().wsm_chain_create(arr, len(tasks), ctypes.byref(o), ctypes.byref(h)), "wsm_chain_create")
         self._h = h

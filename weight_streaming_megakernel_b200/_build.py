@@ -14,7 +14,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["wsm_api.cu", "wsm_umma.cu", "wsm_stream.cu", "wsm_noalloc.cu"]
+SOURCES = ["wsm_api.cu", "wsm_umma.cu", "wsm_stream.cu", "wsm_noalloc.cu", "wsm_die.cu"]
 HEADERS = ["wsm_internal.cuh"]
 LIB = os.path.join(PKG, "libwsm.so")
 

@@ -24,6 +24,7 @@ namespace wsm {
 __global__ void wsm_umma_kernel(const __grid_constant__ KParams p);
 const void *stream_kernel_ptr(int mmax, int tile_rows);  // wsm_stream.cu
 void *noalloc_scratch_ptr(int dev);                      // wsm_noalloc.cu: nullptr until set up on `dev`
+wsm_status die_map_of_device(int dev, const std::vector<int> **die, wsm_die_info *info);  // wsm_die.cu
 
 namespace {
 
@@ -751,6 +752,7 @@ struct wsm_chain {
     int dep_ring_stages = 0;
     int cluster = 0;                   // CTAs per cluster (cluster reduction), or 0
     int xbuf_bytes = 0;                // cluster reduction: exchange buffer behind the ring
+    signed char *d_sm_die = nullptr;   // die-grouped claims: SM id -> die table (inside d_buf), or nullptr
     std::vector<wsm::Geo> task_geo;    // each task's plan (wsm_chain_task_plan)
     const void *fn = nullptr;
 };
@@ -807,7 +809,15 @@ struct ChainPlan {
     int prefetch_stages = 0, k_rotate = 0, dep_ring_stages = 0;
     int cluster = 0;     // CTAs per cluster with cluster reduction, else 0
     int xbuf_bytes = 0;  // its exchange buffer
+    bool die_groups = false;  // claims grouped by die
 };
+
+// Die-grouped claims: the first tile of die 1's range, in proportion to the dies' SMs (0: not split).
+int die_split_of(long long tiles, int sms_die0, int sms_die1) {
+    if (tiles < 2 || sms_die0 + sms_die1 <= 0) return 0;
+    const long long s = (tiles * sms_die0 + (sms_die0 + sms_die1) / 2) / (sms_die0 + sms_die1);
+    return (int)std::min(tiles - 1, std::max(1ll, s));
+}
 
 // Units per tile of a task in a cluster-reduction chain: 1, 2 or 4, so the units of a tile of the static
 // first round fall on the CTAs of one cluster; the same cost in pipeline stages as auto_units_per_tile
@@ -862,6 +872,8 @@ wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, 
     wsm_status st;
     if (opts->cluster < WSM_CHAIN_CLUSTER_AUTO || opts->cluster > WSM_CHAIN_CLUSTER_ON)
         return fail(WSM_ERR_INVALID, "bad cluster option %d", opts->cluster);
+    if (opts->die_groups < WSM_DIE_GROUPS_AUTO || opts->die_groups > WSM_DIE_GROUPS_OFF)
+        return fail(WSM_ERR_INVALID, "bad die_groups %d", opts->die_groups);
     if (opts->path < 0 || opts->path > WSM_PATH_UMMA) return fail(WSM_ERR_INVALID, "bad chain path %d", opts->path);
     if (opts->kernels < WSM_CHAIN_KERNELS_AUTO || opts->kernels > WSM_CHAIN_KERNELS_SPLIT)
         return fail(WSM_ERR_INVALID, "bad kernels option %d", opts->kernels);
@@ -872,8 +884,15 @@ wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, 
     if (opts->counter_groups < 0) return fail(WSM_ERR_INVALID, "bad counter_groups %d", opts->counter_groups);
     if (opts->k_order < 0 || opts->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", opts->k_order);
     if (opts->dep_ring_stages < -1) return fail(WSM_ERR_INVALID, "bad dep_ring_stages %d", opts->dep_ring_stages);
-    int maxM = 0;
-    for (int i = 0; i < n; ++i) maxM = std::max(maxM, tasks[i].M);
+    int maxM = 0, max_tile_m = 0;  // largest M, and largest X tile height (M, or the task's m_tile)
+    auto tile_m = [&](int i) {
+        const int tm = tasks[i].m_tile > 0 ? std::min(tasks[i].m_tile, tasks[i].M) : tasks[i].M;
+        return (tm + 15) / 16 * 16;
+    };
+    for (int i = 0; i < n; ++i) {
+        maxM = std::max(maxM, tasks[i].M);
+        max_tile_m = std::max(max_tile_m, tile_m(i));
+    }
     // AUTO: the FMA path only if it is the automatic choice for every task at the chain's largest M
     int path = opts->path;
     if (path == WSM_PATH_AUTO) {
@@ -893,7 +912,7 @@ wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, 
     // the split; 12 alternating runs of 0.3-0.4 GB lose 27 %).  A dependency that crosses kernels
     // is met by stream order.
     if (path == WSM_PATH_UMMA && opts->kernels != WSM_CHAIN_KERNELS_ONE) {
-        auto wide = [&](int i) { return (tasks[i].M + 15) / 16 * 16 > 32; };
+        auto wide = [&](int i) { return tile_m(i) > 32; };
         int kinds = 0, segments = 1;
         double narrow_bytes = 0;
         for (int i = 0; i < n; ++i) {
@@ -931,7 +950,7 @@ wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, 
         chain_wide = opts->tile_rows == 2 * kUmmaRows;
         if (opts->tile_rows == 0) {
             chain_wide = true;
-            for (int i = 0; i < n; ++i) chain_wide = chain_wide && auto_wide((tasks[i].M + 15) / 16 * 16);
+            for (int i = 0; i < n; ++i) chain_wide = chain_wide && auto_wide(tile_m(i));
         }
         to.tile_rows = chain_wide ? 2 * kUmmaRows : kUmmaRows;
     } else {
@@ -950,12 +969,13 @@ wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, 
             to.tile_rows = c32 < c16 ? 32 : 16;
         }
     }
-    to.stage_k = (path == WSM_PATH_UMMA) ? (opts->stage_k ? opts->stage_k
-                                                           : auto_stage_k((maxM + 15) / 16 * 16, chain_wide))
+    to.stage_k = (path == WSM_PATH_UMMA) ? (opts->stage_k ? opts->stage_k : auto_stage_k(max_tile_m, chain_wide))
                                           : 0;
     const int chain_mmax = (path == WSM_PATH_STREAM) ? pow2ceil(maxM) : 0;
     for (int i = 0; i < n; ++i) {
-        if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, sms, &to, geos[i], chain_mmax)) != WSM_OK)
+        wsm_opts ti = to;
+        ti.m_tile = tasks[i].m_tile;
+        if ((st = make_geo(tasks[i].M, tasks[i].N, tasks[i].K, sms, &ti, geos[i], chain_mmax)) != WSM_OK)
             return fail(st, "task %d: %s", i, g_err.c_str());
     }
     // one grid for the whole chain (make_geo clamps it per task to the task's stages)
@@ -1017,6 +1037,21 @@ wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, 
     }
     for (auto &g : geos) g.grid = chain_grid;
     ring.grid = chain_grid;
+    // Die-grouped claims.  AUTO: for chains with an M-tiled task, where M-tiles share weight columns (the
+    // case grouping is about; measured on B200 2.2 % faster at 16-row M-tiles, 0.8 % at 32), if the device
+    // has two dies (cp.die_groups is cleared at chain creation when the probe finds one).
+    if (opts->die_groups != WSM_DIE_GROUPS_OFF) {
+        bool any_dep_cols = false, any_m_tiled = false;
+        for (int i = 0; i < n; ++i) {
+            any_dep_cols = any_dep_cols || tasks[i].dep_cols;
+            any_m_tiled = any_m_tiled || geos[i].n_mt > 1;
+        }
+        const bool ok = path == WSM_PATH_UMMA && groups <= 1 && !cp.cluster && !any_dep_cols;
+        if (opts->die_groups == WSM_DIE_GROUPS_ON && !ok)
+            return fail(WSM_ERR_UNSUPPORTED, "die-grouped claims need the tensor-core path, one counter level, no "
+                                             "cluster reduction and no dep_cols tasks");
+        cp.die_groups = ok && (opts->die_groups == WSM_DIE_GROUPS_ON || any_m_tiled);
+    }
     cp.prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, path);
     if (opts->l2_prefetch_stages == 0 && path == WSM_PATH_UMMA) {
         bool deps = false;
@@ -1059,7 +1094,8 @@ wsm_status plan_chain(const wsm_task *tasks, int n, const wsm_chain_opts *opts, 
         const bool grow = opts->unit_stages == 0 && !tasks[i].dep_cols && groups <= 1;
         const int unit_stages = grow ? chain_unit_stages(geos[i], chain_grid, later[i]) : opts->unit_stages;
         if ((st = plan_units(geos[i], chain_grid, unit_stages,
-                             (tasks[i].dep_cols || groups > 1) ? -1 : opts->tail_tiles, opts->tail_unit_stages)) !=
+                             (tasks[i].dep_cols || groups > 1 || cp.die_groups) ? -1 : opts->tail_tiles,
+                             opts->tail_unit_stages)) !=
             WSM_OK)
             return fail(st, "task %d: %s", i, g_err.c_str());
     }
@@ -1257,6 +1293,7 @@ wsm_status wsm_chain_plan(const wsm_task *tasks, int n, const wsm_chain_opts *op
             o.k_order = kp.k_rotate ? WSM_K_ORDER_ROTATED : WSM_K_ORDER_INCREASING;
             o.dep_ring_stages = kp.dep_ring_stages;
             o.cluster = kp.cluster;
+            o.die_split = kp.die_groups ? die_split_of(g.tiles(), 1, 1) : 0;
         }
     };
     if (cp.parts.empty()) {
@@ -1367,12 +1404,23 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     // column counters) | partials | column needs (constant)
     std::vector<size_t> cnt_off(n), part_off(n), col_off(n), need_off(n);
     std::vector<int> n_groups(n, 1);
+    // die-grouped claims: the measured SM -> die map, and each task's split of its tiles
+    const std::vector<int> *die_map = nullptr;
+    std::vector<int> die_split(n, 0);
+    if (cp.die_groups) {
+        wsm_die_info di;
+        if ((st = die_map_of_device(dev, &die_map, &di)) != WSM_OK) return st;
+        if (di.dies < 2 && opts->die_groups != WSM_DIE_GROUPS_ON) cp.die_groups = false;  // nothing to group
+        for (int i = 0; i < n && cp.die_groups; ++i)
+            die_split[i] = die_split_of(geos[i].tiles(), di.sms_die0, di.sms_die1);
+    }
     size_t ncnt = 0;
     for (int i = 0; i < n; ++i) {
         // every group needs at least one tile and one CTA
         n_groups[i] = (int)std::min<long long>(groups, std::min<long long>(geos[i].tiles(), chain_grid));
         cnt_off[i] = ncnt;
-        ncnt += kSchedWords + (size_t)geos[i].tiles() + (n_groups[i] > 1 ? 2 * (size_t)n_groups[i] : 0);
+        ncnt += kSchedWords + (size_t)geos[i].tiles() + (n_groups[i] > 1 ? 2 * (size_t)n_groups[i] : 0) +
+                (die_split[i] > 0 ? 2 : 0);
     }
     const size_t done_off = ncnt;
     ncnt += n;
@@ -1391,6 +1439,8 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         need_off[i] = part_at;
         part_at += round_up(n_chunks[i] * 4, 256);
     }
+    const size_t die_off = part_at;
+    if (cp.die_groups) part_at += kMaxSmIds;
     ch->buf_bytes = part_at;
     cudaError_t e = cudaMalloc(&ch->d_buf, ch->buf_bytes);
     if (e != cudaSuccess) return fail(WSM_ERR_NOMEM, "cudaMalloc(%zu) for chain scratch failed", ch->buf_bytes);
@@ -1412,6 +1462,16 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     if (e != cudaSuccess) {
         cleanup();
         return cuda_fail(e, "cudaMemset(chain scratch)");
+    }
+    if (cp.die_groups) {
+        std::vector<signed char> table(kMaxSmIds, 0);
+        for (int i = 0; i < kMaxSmIds && i < (int)die_map->size(); ++i) table[i] = (*die_map)[i] == 1 ? 1 : 0;
+        ch->d_sm_die = reinterpret_cast<signed char *>(base + die_off);
+        e = cudaMemcpy(ch->d_sm_die, table.data(), kMaxSmIds, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            cleanup();
+            return cuda_fail(e, "cudaMemcpy(SM die table)");
+        }
     }
     std::vector<char> depended(n, 0);
     for (int i = 0; i < n; ++i) {
@@ -1442,6 +1502,10 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         if (n_groups[i] > 1) {
             T.grp_sched = T.tile_cnt + gi.tiles();
             T.grp_done = T.grp_sched + n_groups[i];
+        }
+        if (die_split[i] > 0) {
+            T.die_split = die_split[i];
+            T.die_sched = T.tile_cnt + gi.tiles() + (n_groups[i] > 1 ? 2 * n_groups[i] : 0);
         }
         T.done = ch->d_counters + done_off + i;
         T.notify = depended[i];
@@ -1524,6 +1588,7 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
     kp.cluster = ch->cluster;
     kp.xbuf_off = ch->geo.stages * ch->geo.stage_bytes;
     kp.xrow = ch->geo.x_stride / (kUmmaBK * 2) + 4;
+    kp.sm_die = ch->d_sm_die;
     return launch(ch->fn, ch->geo, kp, stream, ch->any_dep, ch->cluster ? (size_t)ch->xbuf_bytes : 0);
 }
 
@@ -1609,7 +1674,7 @@ wsm_status gemm_chain(const wsm_task *tasks, int n_tasks, wsm_stream_t stream) {
                                reinterpret_cast<uintptr_t>(t.Y), reinterpret_cast<uintptr_t>(t.Yf32),
                                reinterpret_cast<uintptr_t>(t.R), (uintptr_t)(uint32_t)t.M, (uintptr_t)(uint32_t)t.N,
                                (uintptr_t)(uint32_t)t.K, (uintptr_t)(uint32_t)t.dep, (uintptr_t)(uint32_t)t.epilogue,
-                               (uintptr_t)(t.dep_cols != 0)};
+                               (uintptr_t)(t.dep_cols != 0), (uintptr_t)(uint32_t)t.m_tile};
         key.append(reinterpret_cast<const char *>(f), sizeof f);
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -55,6 +55,7 @@ constexpr int kColChunk = 256;     // output columns per readiness chunk (per-co
 // reduced and stored.  (With two-level readiness `done` counts groups instead.)
 constexpr int kDonePerTile = 4;
 constexpr int kClusterCtas = 4;    // CTAs per thread-block cluster in cluster-reduction chains
+constexpr int kMaxSmIds = 1024;    // entries of the SM-id -> die table of die-grouped chains
 // Trace stamps per CTA and task (%globaltimer ns unless noted): [0] first stage issued, [1] dependency
 // met, [2] last unit's outputs written, [3] SM id, [4] last unit's accumulator at the epilogue, [5] its
 // split-K arrival counted, [6] its in-order reduction done (last arriver only), [7] first stage of the
@@ -120,6 +121,10 @@ struct __align__(64) TaskDev {
     int n_groups;
     unsigned int *grp_sched;    // [n_groups] claim counters, zero between runs
     unsigned int *grp_done;     // [n_groups] finished tiles per group (monotonic over runs)
+    // Die-grouped claims (die_split > 0): tiles [0, die_split) belong to die 0, the rest to die 1; a CTA
+    // claims its die's range from die_sched[die], then the other range.  No tail units.
+    int die_split;
+    unsigned int *die_sched;    // [2] claim counters, zero between runs
     int w_evict_first;          // L2 policy of the weight loads
     uint32_t idesc;             // UMMA instruction descriptor (MMA N = t_mpad)
     uint32_t tx_bytes;          // bytes landing in one stage
@@ -159,6 +164,7 @@ struct KParams {
     int xbuf_off;                   // cluster mode: byte offset of the exchange buffer from the ring's start
     int xrow;                       // cluster mode: floats per exchange-buffer row (widest X tile + 4, the
                                     // last 4 holding the row's flag)
+    const signed char *sm_die;      // die-grouped claims: die of each SM id (kMaxSmIds entries), or nullptr
 };
 
 #if defined(__CUDACC__)
@@ -493,10 +499,18 @@ __device__ __forceinline__ UnitSpan unit_span(const TaskDev &T, int u) {
 }
 
 // First stage a unit streams, counted from its k_begin: with k_rotate, units
-// start at a tile-dependent offset and wrap around, so CTAs that run in
-// lockstep do not all read the same columns of their weight rows at once.
-__device__ __forceinline__ int unit_k_rot(const KParams &p, const UnitSpan &us) {
-    return p.k_rotate ? (us.tile * 11) % (us.k_end - us.k_begin) : 0;
+// start at an offset that depends on their weight column and wrap around, so
+// CTAs that run in lockstep do not all read the same columns of their weight
+// rows at once.
+// The offset depends on the tile's weight column, not on the tile: the M-tiles that share a column (M-major
+// order) then stream its stages in the same order, close together in time, so all but the first find them
+// in L2 (Eq.(1) of the Fleet reading notes, section 3f).  Measured on B200 with a per-tile offset instead
+// (L2-reuse chain, M = 32 / 64 in 16-row M-tiles): 853 MB read from DRAM for 607 MB of weights, L2 hit rate
+// 52 %.
+__device__ __forceinline__ int unit_k_rot(const KParams &p, const TaskDev &T, const UnitSpan &us) {
+    if (!p.k_rotate) return 0;
+    const int col = T.order == 0 ? us.tile / T.n_mt : us.tile % T.n_g;
+    return (col * 11) % (us.k_end - us.k_begin);
 }
 
 // The units a CTA claims from: all of the task's, or with two-level readiness
@@ -524,6 +538,20 @@ __device__ __forceinline__ ClaimRange claim_range(const TaskDev &T) {
         r.hi = group_tile_lo(T, g + 1) * T.nu;
     }
     return r;
+}
+
+// Die-grouped claims: the range of die `d` (0 or 1) of task T.
+__device__ __forceinline__ ClaimRange die_claim_range(const TaskDev &T, int d) {
+    ClaimRange r;
+    r.ctr = &T.die_sched[d];
+    r.lo = d == 0 ? 0 : T.die_split * T.nu;
+    r.hi = d == 0 ? T.die_split * T.nu : T.n_units;
+    return r;
+}
+// ... and the die of the SM this CTA runs on (0 when the table has no entry for it).
+__device__ __forceinline__ int cta_die(const KParams &p) {
+    const uint32_t sm = smid();
+    return (p.sm_die && sm < (uint32_t)kMaxSmIds && p.sm_die[sm] == 1) ? 1 : 0;
 }
 
 // Claim the next dynamic unit: the caller adds cr.lo and the number of units
@@ -755,6 +783,10 @@ __device__ __forceinline__ void chain_run_done(const KParams &p) {
             st_relaxed_gpu(&T.sched[0], 0u);
             if (T.n_groups > 1)
                 for (int g = 0; g < T.n_groups; ++g) st_relaxed_gpu(&T.grp_sched[g], 0u);
+            if (T.die_split > 0) {
+                st_relaxed_gpu(&T.die_sched[0], 0u);
+                st_relaxed_gpu(&T.die_sched[1], 0u);
+            }
             if (!heal) continue;
             const int tiles = T.n_g * T.n_mt;
             for (int i = 0; i < tiles; ++i) st_relaxed_gpu(&T.tile_cnt[i], 0u);

@@ -126,7 +126,7 @@ static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDe
     for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
         const UnitSpan ps = unit_span(T, uu);
         const int k_len = ps.k_end - ps.k_begin;
-        const int k_rot = unit_k_rot(p, ps);
+        const int k_rot = unit_k_rot(p, T, ps);
         for (int i = (uu < (int)gridDim.x ? skip : 0); i < k_len && budget > 0; ++i, --budget) {
             const int kk = ps.k_begin + (i + k_rot) % k_len;
             for (int kw = 0; kw < KW; ++kw)
@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     const int k_begin = us.k_begin;
                     const int k_end = us.k_end;
                     const int k_len = k_end - k_begin;
-                    const int k_rot = unit_k_rot(p, us);
+                    const int k_rot = unit_k_rot(p, T, us);
                     int next_u = cr.hi - cr.lo - n_static;
                     bool claimed = false;
                     for (int kk = k_begin; kk < k_end; ++kk) {

@@ -355,7 +355,7 @@ static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDe
         tile_coords(T, ps.tile, pg, pmt);
         const int halves = p.wide ? 2 : 1;
         const int k_len = ps.k_end - ps.k_begin;
-        const int k_rot = unit_k_rot(p, ps);
+        const int k_rot = unit_k_rot(p, T, ps);
         for (int i = (uu < (int)gridDim.x ? skip : 0); i < k_len && budget > 0; ++i, --budget) {
             const int kk = ps.k_begin + (i + k_rot) % k_len;
             for (int h = 0; h < halves; ++h)
@@ -519,10 +519,13 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 // grid dependency); later tasks hand out every unit by claim, so the CTAs that finish the
                 // previous task first take the next task's work.
                 // (with two-level readiness a CTA works only on its group's tiles, all claimed)
-                const ClaimRange cr = claim_range(T);
+                // (die-grouped claims: this CTA's die's range first, then the other die's)
+                const bool by_die = T.die_split > 0;
+                const int my_die = by_die ? cta_die(p) : 0;
+                ClaimRange cr = by_die ? die_claim_range(T, my_die) : claim_range(T);
                 // (cluster mode: every task's first round is static, so a split tile's units of that round
                 // sit on the consecutive CTAs of one cluster)
-                const bool static_first = (t == 0 || p.cluster) && T.n_groups <= 1;
+                const bool static_first = (t == 0 || p.cluster) && T.n_groups <= 1 && !by_die;
                 const int n_static = static_first ? min((int)gridDim.x, T.n_units) : 0;
                 int u;
                 if (static_first) {
@@ -535,71 +538,77 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     }
                     u = cr.lo + claim_unit(cr);
                 }
-                while (u < cr.hi) {
-                    if (first_unit) {
-                        trace_stamp(p, t, 0, globaltimer());
-                        trace_stamp(p, t, 3, smid());
-                        first_unit = false;
-                    }
-                    const UnitSpan us = unit_span(T, u);
-                    int g, mt;
-                    tile_coords(T, us.tile, g, mt);
-                    const int xy = mt * T.t_m;
-                    int next_u = cr.hi - cr.lo - n_static;
-                    bool claimed = false;
-                    const int k_len = us.k_end - us.k_begin;
-                    const int k_rot = unit_k_rot(p, us);
-                    for (int kk = us.k_begin; kk < us.k_end; ++kk) {
-                        if (!take_slot()) break;
-                        slot_ok = false;
-                        uint8_t *st = ring + (size_t)s * p.stage_bytes;
-                        stage_meta[s][0] = t;
-                        stage_meta[s][1] = u;
-                        stage_meta[s][2] = (kk == us.k_begin ? kMetaFirst : 0) | (kk == us.k_end - 1 ? kMetaLast : 0);
-                        stage_meta[s][3] = (int)T.idesc;  // the MMA thread reads no task table
-                        mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
-                        // the stage this iteration loads (rotated within the unit when k_rotate)
-                        const int kr = k_rot ? us.k_begin + (kk - us.k_begin + k_rot) % k_len : kk;
-                        const int k0 = kr * p.kps * kUmmaBK;
-                        for (int h = 0; h < halves; ++h)
-                            for (int j = 0; j < p.kps; ++j)
-                                tma_load_2d(st + (h * p.kps + j) * (kUmmaRows * kUmmaBK * 2), &T.tmW, &full_bar[s],
-                                            k0 + j * kUmmaBK, (g * halves + h) * kUmmaRows, pol_w);
-                        if (x_now(k0)) {
-                            for (int j = 0; j < p.kps; ++j)
-                                tma_load_2d(st + p.x_off + j * p.x_stride, &T.tmX, &full_bar[s], k0 + j * kUmmaBK, xy,
-                                            pol_x);
-                        } else {
-                            pend_s[np] = s;
-                            pend_k[np] = k0;
-                            pend_y[np] = xy;
-                            ++np;
+                for (int pass = 0;; ++pass) {
+                    while (u < cr.hi) {
+                        if (first_unit) {
+                            trace_stamp(p, t, 0, globaltimer());
+                            trace_stamp(p, t, 3, smid());
+                            first_unit = false;
                         }
-                        ++issued;
-                        if (++s == S) {
-                            s = 0;
-                            ph ^= 1;
+                        const UnitSpan us = unit_span(T, u);
+                        int g, mt;
+                        tile_coords(T, us.tile, g, mt);
+                        const int xy = mt * T.t_m;
+                        int next_u = cr.hi - cr.lo - n_static;
+                        bool claimed = false;
+                        const int k_len = us.k_end - us.k_begin;
+                        const int k_rot = unit_k_rot(p, T, us);
+                        for (int kk = us.k_begin; kk < us.k_end; ++kk) {
+                            if (!take_slot()) break;
+                            slot_ok = false;
+                            uint8_t *st = ring + (size_t)s * p.stage_bytes;
+                            stage_meta[s][0] = t;
+                            stage_meta[s][1] = u;
+                            stage_meta[s][2] = (kk == us.k_begin ? kMetaFirst : 0) | (kk == us.k_end - 1 ? kMetaLast : 0);
+                            stage_meta[s][3] = (int)T.idesc;  // the MMA thread reads no task table
+                            mbar_arrive_expect_tx(&full_bar[s], T.tx_bytes);
+                            // the stage this iteration loads (rotated within the unit when k_rotate)
+                            const int kr = k_rot ? us.k_begin + (kk - us.k_begin + k_rot) % k_len : kk;
+                            const int k0 = kr * p.kps * kUmmaBK;
+                            for (int h = 0; h < halves; ++h)
+                                for (int j = 0; j < p.kps; ++j)
+                                    tma_load_2d(st + (h * p.kps + j) * (kUmmaRows * kUmmaBK * 2), &T.tmW, &full_bar[s],
+                                                k0 + j * kUmmaBK, (g * halves + h) * kUmmaRows, pol_w);
+                            if (x_now(k0)) {
+                                for (int j = 0; j < p.kps; ++j)
+                                    tma_load_2d(st + p.x_off + j * p.x_stride, &T.tmX, &full_bar[s], k0 + j * kUmmaBK, xy,
+                                                pol_x);
+                            } else {
+                                pend_s[np] = s;
+                                pend_k[np] = k0;
+                                pend_y[np] = xy;
+                                ++np;
+                            }
+                            ++issued;
+                            if (++s == S) {
+                                s = 0;
+                                ph ^= 1;
+                            }
+                            // claim the next unit kClaimLead stages before this one ends: early enough to
+                            // hide the claim's round trip, late enough not to hold work a faster CTA could
+                            // take -- and never while this task's dependency is unmet, when every CTA would
+                            // hold a second unit it cannot start (the claim counters belong to the previous
+                            // kernel until the grid dependency is resolved)
+                            if (!claimed && dep_ok && us.k_end - kk <= kClaimLead) {
+                                next_u = claim_unit(cr);
+                                claimed = true;
+                            }
                         }
-                        // claim the next unit kClaimLead stages before this one ends: early enough to
-                        // hide the claim's round trip, late enough not to hold work a faster CTA could
-                        // take -- and never while this task's dependency is unmet, when every CTA would
-                        // hold a second unit it cannot start (the claim counters belong to the previous
-                        // kernel until the grid dependency is resolved)
-                        if (!claimed && dep_ok && us.k_end - kk <= kClaimLead) {
+                        if (aborted) break;
+                        if (!claimed) {
+                            // the unit streamed completely before its dependencies were resolved
+                            if (!dep_ok) flush();
                             next_u = claim_unit(cr);
-                            claimed = true;
                         }
+                        // whatever comes next needs a free slot: wait for it before the claim's result is used,
+                        // so the claim's round trip overlaps the wait
+                        if (!take_slot()) break;
+                        u = cr.lo + next_u + n_static;
                     }
-                    if (aborted) break;
-                    if (!claimed) {
-                        // the unit streamed completely before its dependencies were resolved
-                        if (!dep_ok) flush();
-                        next_u = claim_unit(cr);
-                    }
-                    // whatever comes next needs a free slot: wait for it before the claim's result is used,
-                    // so the claim's round trip overlaps the wait
-                    if (!take_slot()) break;
-                    u = cr.lo + next_u + n_static;
+                    if (aborted || !by_die || pass > 0) break;
+                    // own die's range done: help with the other die's
+                    cr = die_claim_range(T, my_die ^ 1);
+                    u = cr.lo + claim_unit(cr);
                 }
                 if (np > 0) flush();
                 if (aborted) break;
