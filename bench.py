@@ -238,7 +238,7 @@ def run_e2e(args, wsm, dev, datas, copies, mode, total_bytes, world, stream, n_s
             if mode == "chain":
                 deps = [(i - 1) if args.workload == "chain" else -1 for i in range(len(gemms))]
                 ch = wsm.Chain([wsm.Task(x, w, y, dep=deps[i], m_tile=c.m_tile) for i, (c, x, w, y) in enumerate(gemms)],
-                               flags=wsm.FLAG_W_READONLY, die_groups=args.die_groups)
+                               flags=wsm.FLAG_W_READONLY, die_groups=args.die_groups, cluster=args.cluster)
                 runs[j, r] = (lambda ch=ch: ch.run(s), ch)
             else:
                 def go(gemms=gemms):
@@ -330,7 +330,8 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
         # the whole step is one persistent kernel; the layer chain orders task t after t-1
         deps = [(i - 1) if args.workload == "chain" else -1 for i in range(len(data))]
         chains = [wsm.Chain([wsm.Task(x, w, y, dep=deps[i], m_tile=c.m_tile) for i, (c, x, w, y) in enumerate(d)],
-                            flags=wsm.FLAG_W_READONLY, die_groups=args.die_groups) for d in datas]
+                            flags=wsm.FLAG_W_READONLY, die_groups=args.die_groups, cluster=args.cluster)
+                  for d in datas]
         chain = chains[0]
         launches_per_step = 1
 
@@ -523,6 +524,126 @@ def run_nshard(args, rank, world, local_rank):
     return full_bytes, total_ms / args.steps
 
 
+def trace_boundaries(args):
+    """Diagnostic (not a bench line for the driver): run the dependent layer
+    chain once with per-CTA trace stamps and report, per GEMM kind, the median
+    over layers of where a task's time goes, in microseconds from the moment
+    its dependency was met (median over CTAs): the accumulators reaching the
+    epilogue (median and last CTA), the last split-K arrival, the last
+    reduction, the last outputs written, the next task's dependency met and
+    its first stage at the MMA issuer.  Prints one JSON line."""
+    import statistics
+    import weight_streaming_megakernel_b200 as wsm
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cases = workload_cases(args.workload)
+    data = setup_inputs(cases, dev)
+    tasks = [wsm.Task(x, w, y, dep=i - 1, m_tile=c.m_tile) for i, (c, x, w, y) in enumerate(data)]
+    ch = wsm.Chain(tasks, flags=wsm.FLAG_W_READONLY, trace=True, cluster=args.cluster)
+    s = torch.cuda.Stream(dev)
+    for _ in range(max(3, args.warmup)):
+        ch.run(s)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        a.record(s)
+        ch.run(s)
+        b.record(s)
+    s.synchronize()
+    tr = ch.trace(s).double()
+    if ch.status(s)[0] != 0:
+        raise RuntimeError("device-side status")
+    plan0 = ch.task_plan(0)
+    ch.close()
+
+    def col(t, i):
+        v = tr[:, t, i]
+        return v[v > 0]
+    kinds = {}
+    for t in range(1, len(cases) - 1):
+        kind = cases[t].name.split("_", 1)[1] if "_" in cases[t].name else cases[t].name
+        acc, dep, nxt, mma = col(t, 4), col(t, 1), col(t + 1, 1), col(t + 1, 7)
+        if min(len(acc), len(dep), len(nxt), len(mma)) == 0:
+            continue
+        t0 = float(dep.median())
+        us = lambda v: (float(v) - t0) / 1e3  # noqa: E731
+        row = {"acc_median": us(acc.median()), "acc_last": us(acc.max()), "outputs_last": us(col(t, 2).max()),
+               "next_dependency_met": us(nxt.median()), "next_first_stage_at_mma": us(mma.median())}
+        if len(col(t, 5)):
+            row["arrival_last"] = us(col(t, 5).max())
+        if len(col(t, 6)):
+            row["reduction_last"] = us(col(t, 6).max())
+        kinds.setdefault(kind, []).append(row)
+    out = {k: {f: round(statistics.median(r[f] for r in rows if f in r), 2) for f in rows[0]}
+           for k, rows in kinds.items()}
+    print(json.dumps({"diagnostic": "boundary_trace", "workload": args.workload, "cluster": args.cluster,
+                      "grid": plan0["grid"], "chain_ms_traced": round(a.elapsed_time(b), 4),
+                      "us_from_dependency_met": out}))
+
+
+def trace_launches(args):
+    """Diagnostic (not a bench line for the driver): back-to-back launches of
+    each GEMM of the workload, each launch a one-task chain (the same kernels,
+    plan and programmatic-launch overlap as skinny_gemm with the W read-only
+    flag, plus per-CTA trace stamps that are never cleared between runs, so no
+    memset separates the launches), cycling through weight copies larger
+    than L2 and replayed as one CUDA graph.  Reports per GEMM, in
+    microseconds, medians over the launches: the launch slot (last outputs of
+    one launch to the last outputs of the next), the span from a launch's
+    first CTA issuing its first stage to its last outputs, how long after the
+    previous launch's last outputs its first CTA and its median CTA started,
+    and each CTA's busy time (first stage to its last outputs).  Prints one
+    JSON line."""
+    import statistics
+    import weight_streaming_megakernel_b200 as wsm
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    out = {}
+    for case in workload_cases(args.workload):
+        if args.only and case.name not in args.only.split(","):
+            continue
+        copies = n_copies([case])
+        datas = [setup_inputs([case], dev, seed_base=r) for r in range(copies)]
+        chains = [wsm.Chain([wsm.Task(x, w, y, m_tile=c.m_tile)], flags=wsm.FLAG_W_READONLY, trace=2)
+                  for d in datas for (c, x, w, y) in d]
+        s = torch.cuda.Stream(dev)
+        n_launch = max(2 * copies, 16)
+        for ch in chains:
+            ch.run(s)
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for k in range(n_launch):
+                chains[k % copies].run(s)
+        with torch.cuda.stream(s):
+            g.replay()
+        s.synchronize()
+        # each chain's trace holds its last launch: the final `copies` launches of the replay, in order
+        order = [(n_launch - copies + j) % copies for j in range(copies)]
+        stamps = [chains[i].trace(s).double()[:, 0, :] for i in order]
+        plan = chains[0].task_plan(0)
+        for ch in chains:
+            if ch.status(s)[0] != 0:
+                raise RuntimeError("device-side status")
+            ch.close()
+        del g
+        rows = []
+        for j in range(1, copies):
+            prev, cur = stamps[j - 1], stamps[j]
+            pe = prev[:, 2][prev[:, 2] > 0].max()
+            c0, c2 = cur[:, 0], cur[:, 2]
+            ok = (c0 > 0) & (c2 > 0)
+            rows.append({"slot": float(c2[ok].max() - pe) / 1e3,
+                         "span": float(c2[ok].max() - c0[ok].min()) / 1e3,
+                         "first_cta_start_after_prev_end": float(c0[ok].min() - pe) / 1e3,
+                         "median_cta_start_after_prev_end": float(c0[ok].median() - pe) / 1e3,
+                         "cta_busy_median": float((c2[ok] - c0[ok]).median()) / 1e3,
+                         "ctas": int(ok.sum())})
+        out[case.name] = {k: round(statistics.median(r[k] for r in rows), 2) for k in rows[0]}
+        out[case.name].update(path="umma" if plan["path"] == 2 else "fma", units=plan["units"], grid=plan["grid"],
+                              roofline_us=round(alg_bytes(case) / (peaks()[0] * 1e3), 2))
+    print(json.dumps({"diagnostic": "launch_trace", "workload": args.workload, "us": out}))
+
+
 # ----------------------------------------------------------------------------- CPU arm
 
 def oracle_sample_rate(cases, budget_s, threads=0):
@@ -612,6 +733,14 @@ def main():
                     help="chain: the step is one persistent gemm_chain kernel; launches: one skinny_gemm per GEMM "
                          "(default: launches for the single-GEMM workload, chain otherwise)")
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-GEMM single-launch breakdown")
+    ap.add_argument("--trace-boundaries", action="store_true",
+                    help="diagnostic: one traced run of the workload as a dependent chain; prints where each task's "
+                         "time goes (not a bench line)")
+    ap.add_argument("--trace-launches", action="store_true",
+                    help="diagnostic: per-CTA timeline of back-to-back launches of each GEMM of the workload "
+                         "(not a bench line)")
+    ap.add_argument("--cluster", type=int, default=0, choices=[0, 1, 2],
+                    help="chains' cluster reduction: 0 auto (off), 1 off, 2 on")
     ap.add_argument("--die-groups", type=int, default=0, choices=[0, 1, 2],
                     help="chains' die-grouped claims: 0 auto (M-tiled chains), 1 on, 2 off")
     ap.add_argument("--no-configurations", action="store_true",
@@ -675,6 +804,10 @@ def main():
         print(json.dumps(line))
         return
 
+    if args.trace_boundaries or args.trace_launches:
+        if rank == 0:
+            (trace_boundaries if args.trace_boundaries else trace_launches)(args)
+        return
     if world > 1:
         torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local_rank),
                                              timeout=datetime.timedelta(seconds=120))

@@ -338,7 +338,12 @@ typedef struct {
                                   picks it for every task at the chain's largest M) */
     int grid;                  /* 0 = one CTA per SM */
     unsigned long long timeout_ns; /* bound on each dependency wait, 0 = 2 s */
-    int trace;                 /* nonzero: record per-CTA, per-task %globaltimer stamps */
+    int trace;                 /* nonzero: record per-CTA, per-task %globaltimer stamps
+                                  (wsm_chain_trace); 1: cleared before every run (a memset queued
+                                  on the stream, between this run and the previous kernel), 2:
+                                  never cleared after creation, so back-to-back runs keep their
+                                  programmatic overlap (a CTA that records nothing in a run keeps
+                                  its earlier stamps) */
     int debug_unmet_dependency; /* test hook, 0 in real use: nonzero makes every dependency
                                    target unreachable, so each dependency wait runs out after
                                    timeout_ns and the run reports WSM_ERR_TIMEOUT */

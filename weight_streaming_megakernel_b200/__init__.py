@@ -390,7 +390,7 @@ def _chain_opts(path=PATH_AUTO, grid=0, timeout_ns=0, trace=False, debug_unmet_d
                 counter_groups=0, kernels=0, tile_rows=0, k_order=0, dep_ring_stages=0, cluster=0,
                 die_groups=0) -> "_ChainOpts":
     o = _ChainOpts()
-    o.path, o.grid, o.timeout_ns, o.trace = path, grid, timeout_ns, 1 if trace else 0
+    o.path, o.grid, o.timeout_ns, o.trace = path, grid, timeout_ns, (trace if trace in (1, 2) else 1) if trace else 0
     o.debug_unmet_dependency = 1 if debug_unmet_dependency else 0
     o.flags, o.stage_k = flags, stage_k
     o.unit_stages, o.tail_tiles, o.tail_unit_stages = unit_stages, tail_tiles, tail_unit_stages

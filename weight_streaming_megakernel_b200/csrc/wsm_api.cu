@@ -753,6 +753,7 @@ struct wsm_chain {
     int cluster = 0;                   // CTAs per cluster (cluster reduction), or 0
     int xbuf_bytes = 0;                // cluster reduction: exchange buffer behind the ring
     signed char *d_sm_die = nullptr;   // die-grouped claims: SM id -> die table (inside d_buf), or nullptr
+    int trace_mode = 0;                // wsm_chain_opts.trace
     std::vector<wsm::Geo> task_geo;    // each task's plan (wsm_chain_task_plan)
     const void *fn = nullptr;
 };
@@ -1527,6 +1528,7 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         cleanup();
         return cuda_fail(e, "cudaMemcpy(task table)");
     }
+    ch->trace_mode = opts->trace;
     if (opts->trace) {
         ch->trace_elems = (size_t)ring.grid * n * kTraceSlots;
         e = cudaMalloc(reinterpret_cast<void **>(&ch->d_trace), ch->trace_elems * 8);
@@ -1563,7 +1565,7 @@ wsm_status wsm_chain_run(wsm_chain *ch, wsm_stream_t stream_) {
         WSM_CUDA(cudaMemsetAsync(ch->d_run_ctl, 0, 2 * sizeof(unsigned int), stream));
         ch->needs_reset = false;
     }
-    if (ch->d_trace) WSM_CUDA(cudaMemsetAsync(ch->d_trace, 0, ch->trace_elems * 8, stream));
+    if (ch->d_trace && ch->trace_mode != 2) WSM_CUDA(cudaMemsetAsync(ch->d_trace, 0, ch->trace_elems * 8, stream));
     KParams kp;
     memset(&kp, 0, sizeof kp);
     kp.tasks = ch->d_table;
