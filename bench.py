@@ -342,7 +342,9 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
         for d in datas:
             calls = []
             for c, x, w, y in d:
-                o = wsm._opts(m_tile=c.m_tile, flags=wsm.FLAG_W_READONLY)
+                # independent launches: every GEMM of a step and every copy has its own X, W and Y
+                fl = wsm.FLAG_W_READONLY | (wsm.FLAG_INDEPENDENT if args.independent else 0)
+                o = wsm._opts(m_tile=c.m_tile, flags=fl, grid=args.grid)
                 calls.append((x.data_ptr(), w.data_ptr(), y.data_ptr(), c.M, c.N, c.K, o))
             callsets.append(calls)
         launches_per_step = len(callsets[0])
@@ -686,7 +688,12 @@ def oracle_sample_rate(cases, budget_s, threads=0):
 # The five configurations of the metric, as (key, workload, mode, target fraction of the measured peak or
 # None).  The default run reports every one of them beside its headline (the Qwen3-8B decode step).
 CONFIGURATIONS = (
-    ("c1_single_m1_4096x4096", "single", "launches", 0.80),
+    ("c1_single_m1_4096x4096", "single", "launches", 0.80, {"steps": 64}),
+    # back-to-back calls on unrelated buffers with WSM_FLAG_INDEPENDENT on a quarter of the SMs: about
+    # four calls run at once; 64 launches per timed graph so that its start and end (the first call alone,
+    # the last one draining) weigh little
+    ("c1_single_m1_4096x4096_independent", "single", "launches", 0.80,
+     {"independent": True, "grid": 37, "steps": 64}),
     ("c2_qwen3_8b_decode_gemms", "qwen3_decode", "chain", 0.80),
     ("c3_skinny_k7168_k8192", "skinny", "chain", 0.80),
     ("c4_l2_reuse_m32_m64", "l2_reuse", "chain", None),
@@ -697,22 +704,31 @@ CONFIGURATIONS = (
 
 def run_configurations(args, rank, world, local_rank, hbm_peak, headline):
     """Every configuration besides the headline one: device time per step of
-    K' = min(K, 10) steps in one graph (same protocol as the headline), GB/s of
-    algorithmic bytes, fraction of the measured peak."""
+    K' = min(K, 10) steps in one graph (same protocol as the headline; the
+    single-GEMM lines take 64 launches), GB/s of algorithmic bytes, fraction
+    of the measured peak."""
     out = {}
-    for key, workload, mode, target in CONFIGURATIONS:
-        if workload == args.workload and mode == args.mode:
+    for key, workload, mode, target, *over in CONFIGURATIONS:
+        over = dict(over[0]) if over else {}
+        own_steps = "steps" in over
+        n_steps = over.pop("steps", min(args.steps, 10))
+        if workload == args.workload and mode == args.mode and (not own_steps or n_steps == args.steps) and \
+                all(getattr(args, k) == v for k, v in over.items()):
             r = headline
+            n_steps = args.steps
         else:
             sub = argparse.Namespace(**vars(args))
             sub.workload, sub.mode, sub.only = workload, mode, ""
-            r = run_gpu(sub, rank, world, local_rank, mode=mode, steps=min(args.steps, 10), extras=False)
+            sub.independent, sub.grid = False, 0
+            for k, v in over.items():
+                setattr(sub, k, v)
+            r = run_gpu(sub, rank, world, local_rank, mode=mode, steps=n_steps, extras=False)
         gbs = r["total_bytes"] / (r["ms_per_step"] * 1e-3) / 1e9
         n = len(r["cases"])
         out[key] = {"workload": workload, "mode": mode, "gemms": n, "ms_per_step": round(r["ms_per_step"], 4),
                     "us_per_gemm": round(r["ms_per_step"] * 1e3 / n, 3), "GBps": round(gbs, 1),
                     "frac_of_peak": round(gbs / hbm_peak, 4), "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
-                    "target_frac": target,
+                    "target_frac": target, "steps": n_steps, **({"options": over} if over else {}),
                     "bytes_per_step": r["total_bytes"]}
     return out
 
@@ -743,6 +759,9 @@ def main():
                     help="chains' cluster reduction: 0 auto (off), 1 off, 2 on")
     ap.add_argument("--die-groups", type=int, default=0, choices=[0, 1, 2],
                     help="chains' die-grouped claims: 0 auto (M-tiled chains), 1 on, 2 off")
+    ap.add_argument("--independent", action="store_true",
+                    help="launches mode: WSM_FLAG_INDEPENDENT on every launch (the step's GEMMs share no buffers)")
+    ap.add_argument("--grid", type=int, default=0, help="launches mode: persistent CTAs per launch (0 = auto)")
     ap.add_argument("--no-configurations", action="store_true",
                     help="skip the other four configurations (reported beside the default workload)")
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "nshard"],
@@ -778,7 +797,9 @@ def main():
                        if n_copies(cases) > 1 else ""),
               "parallelism": f"replicas{world}" if world > 1 else "single",
               "mode": args.mode + (" (one persistent kernel per step, W read-only flag)" if args.mode == "chain"
-                                   else " (one skinny_gemm launch per GEMM, W read-only flag)")}
+                                   else " (one skinny_gemm launch per GEMM, W read-only flag"
+                                        + (", independent flag" if args.independent else "")
+                                        + (f", grid {args.grid}" if args.grid else "") + ")")}
 
     if args.impl == "reference":
         if rank != 0:

@@ -97,14 +97,33 @@ enum {
  * Every launch uses programmatic dependent launch: the kernel may start while
  * the kernel queued before it on the stream is finishing, and waits for it
  * (griddepcontrol.wait) before touching global memory, so stream order is
- * kept.  WSM_FLAG_W_READONLY relaxes that for W only: the caller promises
- * that the kernel queued just before this call does not write W, and the
- * weight stream (which is the whole cost of a decode GEMM) then starts
- * before that kernel has finished; X, Y and the scratch still wait.
- * WSM_FLAG_NO_PDL launches without programmatic dependent launch. */
+ * kept; it lets the kernel after it launch only once each of its CTAs has
+ * seen that wait through.  WSM_FLAG_W_READONLY relaxes the wait for W only:
+ * the caller promises that the kernel queued just before this call does not
+ * write W, and the weight stream (which is the whole cost of a decode GEMM)
+ * then starts before that kernel has finished; X, Y and the scratch still
+ * wait.  WSM_FLAG_NO_PDL launches without programmatic dependent launch.
+ *
+ * WSM_FLAG_INDEPENDENT (single calls only) goes further.  Such a call may run
+ * at the same time as every call queued since the last library call without
+ * the flag, that call included; the caller promises that none of those writes
+ * this call's X, W or R, or reads or writes its Y or Yf32 (e.g. a q
+ * projection without the flag, then k and v with it, all reading one X; or
+ * back-to-back GEMMs on unrelated buffers).  The plan then takes whole tiles
+ * (unless unit_stages or tail_tiles ask for split ones), CTA c runs units c,
+ * c + grid, ... without claim counters or partial slots, loads and stores
+ * without waiting, lets the next kernel launch at once, and waits for the
+ * kernel before it only on exit: every call
+ * still completes after all work queued before it, so later work on the
+ * stream sees theirs.  With a grid below the SM count (wsm_opts.grid)
+ * consecutive independent calls share the GPU.  A plan that splits tiles
+ * (asked for explicitly) ignores the flag.  A device-side time-out inside an independent call can
+ * also make the calls running beside it give up (they share the stream's
+ * launch error word); the stream status reports it either way. */
 enum {
     WSM_FLAG_W_READONLY = 1,
-    WSM_FLAG_NO_PDL = 2
+    WSM_FLAG_NO_PDL = 2,
+    WSM_FLAG_INDEPENDENT = 4
 };
 
 /* Epilogue applied to the fp32 result, before its one rounding to bf16.

@@ -109,7 +109,8 @@ def test_cluster_chain_fused_epilogues_repeated_runs_and_graph():
         check_full(h1.cpu(), w_dn.cpu(), h2, f2, what=f"{what} down")
 
     for rep in range(2):
-        h0.copy_(r)
+        with torch.cuda.stream(s):
+            h0.copy_(r)
         ch.run(s)
         assert ch.status(s)[0] == wsm.WSM_OK
         check(f"run {rep}")
@@ -117,10 +118,10 @@ def test_cluster_chain_fused_epilogues_repeated_runs_and_graph():
     with torch.cuda.graph(g, stream=s):
         ch.run(s)
     for rep in range(2):
-        h0.copy_(r)
-        h1.fill_(float("nan"))
-        h2.fill_(float("nan"))
         with torch.cuda.stream(s):
+            h0.copy_(r)
+            h1.fill_(float("nan"))
+            h2.fill_(float("nan"))
             g.replay()
         s.synchronize()
         assert ch.status(s)[0] == wsm.WSM_OK

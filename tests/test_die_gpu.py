@@ -80,6 +80,7 @@ def test_die_grouped_chain_matches_oracle_and_ungrouped(deps):
         assert p["units"] == plans[i]["units"] and p["m_tiles"] == -(-M // tm)
     s = torch.cuda.Stream()
     for rep in range(2):
+        s.wait_stream(torch.cuda.current_stream())
         ch.run(s)
         assert ch.status(s)[0] == wsm.WSM_OK
         for i, ((x, w, t), (yb, yf)) in enumerate(zip(ts, ref)):
@@ -91,6 +92,7 @@ def test_die_grouped_chain_matches_oracle_and_ungrouped(deps):
     with torch.cuda.graph(g, stream=s):
         ch.run(s)
     for rep in range(2):
+        s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             g.replay()
         s.synchronize()

@@ -1,0 +1,170 @@
+"""Independent single calls (WSM_FLAG_INDEPENDENT), against the fp64 oracle.
+
+Such a call streams whole tiles in a fixed round-robin (no claim counters, no
+partial slots), loads and stores without waiting for the kernel before it, lets
+the next kernel launch at once and waits for its predecessor only on exit.
+The tests check the results and the stream-order contract of the flag:
+
+- back-to-back independent calls on unrelated buffers, both kernel paths, at
+  full and reduced grids (consecutive calls then share the GPU);
+- a producer GEMM, then q without the flag and k, v with it, all three
+  reading the producer's output (the flag allows k and v to run beside q,
+  never beside the producer), then a consumer without the flag reading v's
+  output and a plain torch op reading k's: the waits that remain must still
+  order every read after its write;
+- a chain of independent calls followed by a normal call that overwrites
+  their X: the overwrite must wait for every one of them;
+- the flag with split tiles asked for explicitly (it is then ignored);
+- a device-side time-out inside an independent call (the stall hook)."""
+import pytest
+import torch
+
+import synth
+import weight_streaming_megakernel_b200 as wsm
+from parity import check_full
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+IND = wsm.FLAG_INDEPENDENT
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    yield
+    wsm.debug_stall(0)
+
+
+def _nan(M, N, dtype=torch.bfloat16):
+    return torch.full((M, N), float("nan"), dtype=dtype, device=DEV)
+
+
+@pytest.mark.parametrize("grid", [0, 74, 37])
+@pytest.mark.parametrize("path,M,N,K", [(wsm.PATH_STREAM, 1, 4096, 4096), (wsm.PATH_STREAM, 4, 2112, 7168),
+                                        (wsm.PATH_UMMA, 16, 6144, 4096), (wsm.PATH_UMMA, 40, 1000, 2048),
+                                        (wsm.PATH_UMMA, 64, 4096, 1032)])
+def test_back_to_back_independent_calls(path, M, N, K, grid):
+    p = wsm.plan(M, N, K, path=path, grid=grid, flags=IND)
+    assert p["units"] == p["n_tiles"] * p["m_tiles"], "an independent call plans whole tiles"
+    n = 6
+    xs, ws = zip(*[synth.make_xw(M, N, K, seed=100 * i + M + grid) for i in range(n)])
+    xds = [x.to(DEV) for x in xs]
+    wds = [w.to(DEV) for w in ws]
+    ys = [_nan(M, N) for _ in range(n)]
+    yfs = [_nan(M, N, torch.float32) for _ in range(n)]
+    wo = synth.make_w(K, K, seed=7)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(n):
+            wsm.skinny_gemm(xds[i], wds[i], ys[i], yf32=yfs[i], path=path, grid=grid, flags=IND, stream=s)
+        # a call without the flag may write what the independent calls read: X of the first one
+        wsm.skinny_gemm(xds[1], wo.to(DEV), xds[0], path=path, stream=s)
+    assert wsm.stream_status(s) == 0
+    for i in range(n):
+        check_full(xs[i], ws[i], ys[i], yfs[i], what=f"independent call {i} path={path} M={M} grid={grid}")
+    check_full(xs[1], wo, xds[0], what="the call after them")
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 2), (wsm.PATH_UMMA, 16)])
+def test_group_after_producer_keeps_stream_order(path, M):
+    """x -> P (large, no flag) -> y_p; q (no flag), k, v (flag) read y_p;
+    D (no flag) reads v's output; a torch op reads k's output."""
+    d, n_kv = 2048, 512
+    x, wp = synth.make_xw(M, d, 28672, seed=M)          # a slow producer: 112 MiB of weights
+    wq = synth.make_w(d, d, seed=M + 1)
+    wk = synth.make_w(n_kv, d, seed=M + 2)
+    wv = synth.make_w(n_kv, d, seed=M + 3)
+    wd = synth.make_w(d, n_kv, seed=M + 4)
+    xd, wpd, wqd, wkd, wvd, wdd = (t.to(DEV) for t in (x, wp, wq, wk, wv, wd))
+    s = torch.cuda.Stream()
+    for rep in range(3):
+        y_p, y_q, y_k, y_v, y_d = _nan(M, d), _nan(M, d), _nan(M, n_kv), _nan(M, n_kv), _nan(M, d)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            wsm.skinny_gemm(xd, wpd, y_p, path=path, stream=s)
+            wsm.skinny_gemm(y_p, wqd, y_q, path=path, stream=s)
+            wsm.skinny_gemm(y_p, wkd, y_k, path=path, grid=48, flags=IND, stream=s)
+            wsm.skinny_gemm(y_p, wvd, y_v, path=path, grid=48, flags=IND, stream=s)
+            wsm.skinny_gemm(y_v, wdd, y_d, path=path, stream=s)
+            k_copy = y_k.clone()
+        assert wsm.stream_status(s) == 0
+        yp = y_p.cpu()
+        check_full(x, wp, y_p, what=f"rep {rep} producer")
+        check_full(yp, wq, y_q, what=f"rep {rep} q")
+        check_full(yp, wk, y_k, what=f"rep {rep} k (independent)")
+        check_full(yp, wv, y_v, what=f"rep {rep} v (independent)")
+        check_full(y_v.cpu(), wd, y_d, what=f"rep {rep} consumer of v")
+        assert torch.equal(k_copy.view(torch.int16), y_k.view(torch.int16)), "torch op read k before it was written"
+
+
+@pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 1), (wsm.PATH_UMMA, 32)])
+def test_normal_call_after_independent_calls_waits_for_all(path, M):
+    """Four independent calls read X; the normal call after them overwrites X
+    (its own output).  Every independent call must have read X before then."""
+    N, K = 4096, 4096
+    x, _ = synth.make_xw(M, K, K, seed=5)
+    ws = [synth.make_w(N, K, seed=10 + i) for i in range(4)]
+    w_over = synth.make_w(K, K, seed=20)
+    w_dev = [w.to(DEV) for w in ws]
+    wo = w_over.to(DEV)
+    s = torch.cuda.Stream()
+    for rep in range(3):
+        xd = x.to(DEV)
+        x_in = xd.clone()
+        ys = [_nan(M, N) for _ in ws]
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for wd, y in zip(w_dev, ys):
+                wsm.skinny_gemm(xd, wd, y, path=path, grid=64, flags=IND, stream=s)
+            wsm.skinny_gemm(x_in, wo, xd, path=path, stream=s)  # overwrites X
+        assert wsm.stream_status(s) == 0
+        for i, (w, y) in enumerate(zip(ws, ys)):
+            check_full(x, w, y, what=f"rep {rep} independent call {i}")
+        check_full(x, w_over, xd, what=f"rep {rep} overwrite of X")
+
+
+@pytest.mark.parametrize("path,M,N,K", [(wsm.PATH_UMMA, 16, 6144, 4096), (wsm.PATH_STREAM, 1, 1024, 8192)])
+def test_flag_with_explicit_split_tiles(path, M, N, K):
+    p = wsm.plan(M, N, K, path=path, flags=IND, unit_stages=2)
+    assert p["units"] > p["n_tiles"] * p["m_tiles"]
+    x, w = synth.make_xw(M, N, K, seed=N)
+    xd, wd = x.to(DEV), w.to(DEV)
+    y = _nan(M, N)
+    yf = _nan(M, N, torch.float32)
+    wsm.skinny_gemm(xd, wd, y, yf32=yf, path=path, flags=IND, unit_stages=2)
+    wsm.skinny_gemm(xd, wd, y, yf32=yf, path=path, flags=IND, unit_stages=2)
+    assert wsm.stream_status() == 0
+    check_full(x, w, y, yf, what="split plan with the flag")
+
+
+@pytest.mark.parametrize("path,M,N,K", [(wsm.PATH_UMMA, 16, 6144, 4096), (wsm.PATH_STREAM, 1, 4096, 4096)])
+def test_independent_timeout_reported_once_then_correct(path, M, N, K):
+    x, w = synth.make_xw(M, N, K, seed=3 + M)
+    xd, wd = x.to(DEV), w.to(DEV)
+    s = torch.cuda.Stream()
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    y2 = _nan(M, N)
+    yf2 = _nan(M, N, torch.float32)
+    y3 = _nan(M, N)
+    s.wait_stream(torch.cuda.current_stream())
+    wsm.skinny_gemm(xd, wd, y, path=path, flags=IND, stream=s)
+    assert wsm.stream_status(s) == 0
+    wsm.debug_stall(1, 50_000_000)
+    wsm.skinny_gemm(xd, wd, y, path=path, flags=IND, stream=s)
+    # runs beside the stalled call and finishes its work long before the stall's limit
+    wsm.skinny_gemm(xd, wd, y2, yf32=yf2, path=path, flags=IND, stream=s)
+    wsm.skinny_gemm(xd, wd, y3, path=path, stream=s)  # a normal call on the same workspace after it
+    assert wsm.stream_status(s) == wsm.WSM_ERR_TIMEOUT
+    assert wsm.stream_status(s) == 0
+    check_full(x, w, y2, yf2, what="independent call after the time-out")
+    check_full(x, w, y3, what="normal call after the time-out")
+
+
+def test_chain_rejects_the_flag():
+    x, w = synth.make_xw(16, 512, 512, seed=1)
+    y = torch.empty(16, 512, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(wsm.WsmError):
+        wsm.Chain([wsm.Task(x.to(DEV), w.to(DEV), y)], flags=IND)

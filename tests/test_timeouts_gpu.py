@@ -49,22 +49,25 @@ def test_stream_workspace_timeout_reported_once_then_correct(path, M, N, K):
     x, w, xd, wd = _inputs(M, N, K, seed=M + N)
     s = torch.cuda.Stream()
     y = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    s.wait_stream(torch.cuda.current_stream())
     wsm.skinny_gemm(xd, wd, y, path=path, stream=s)  # sizes the stream's workspace
     assert wsm.stream_status(s) == 0
     wsm.debug_stall(1, STALL_NS)
     t0 = time.time()
     wsm.skinny_gemm(xd, wd, y, path=path, stream=s)
     # the next call, queued before anyone looks at the status, runs on the repaired counters
-    y2 = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
-    yf2 = torch.full((M, N), float("nan"), dtype=torch.float32, device=DEV)
+    with torch.cuda.stream(s):
+        y2 = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+        yf2 = torch.full((M, N), float("nan"), dtype=torch.float32, device=DEV)
     wsm.skinny_gemm(xd, wd, y2, path=path, yf32=yf2, stream=s)
     assert wsm.stream_status(s) == wsm.WSM_ERR_TIMEOUT
     assert time.time() - t0 < 5.0
     assert "site 6" in wsm.last_error()
     assert wsm.stream_status(s) == 0, "a time-out is reported once"
     check_full(x, w, y2, yf2, what="the call queued after the time-out")
-    y.fill_(float("nan"))
-    yf = torch.full((M, N), float("nan"), dtype=torch.float32, device=DEV)
+    with torch.cuda.stream(s):
+        y.fill_(float("nan"))
+        yf = torch.full((M, N), float("nan"), dtype=torch.float32, device=DEV)
     wsm.skinny_gemm(xd, wd, y, path=path, yf32=yf, stream=s)
     assert wsm.stream_status(s) == 0
     check_full(x, w, y, yf, what="a later call")
@@ -86,6 +89,26 @@ def test_caller_workspace_timeout_reported_once_then_correct(path, M, N, K):
     # the time-out was on the caller's buffer, not on the stream's own workspace
     assert wsm.stream_status() == 0
     check_full(x, w, y, yf, what="the call queued after the time-out")
+
+
+def test_timeout_before_workspace_growth_is_reported():
+    """The call after a time-out needs a larger stream workspace: the time-out
+    recorded in the outgrown buffer is still reported."""
+    x, w, xd, wd = _inputs(16, 512, 1024, seed=4)
+    X, W, Xd, Wd = _inputs(64, 8192, 8192, seed=5)
+    s = torch.cuda.Stream()
+    y = torch.empty(16, 512, dtype=torch.bfloat16, device=DEV)
+    with torch.cuda.stream(s):
+        Y = torch.full((64, 8192), float("nan"), dtype=torch.bfloat16, device=DEV)
+    wsm.skinny_gemm(xd, wd, y, stream=s)
+    assert wsm.stream_status(s) == 0
+    assert wsm.workspace_bytes(64, 8192, 8192) > (1 << 20), "the second call must outgrow the first workspace"
+    wsm.debug_stall(1, STALL_NS)
+    wsm.skinny_gemm(xd, wd, y, stream=s)
+    wsm.skinny_gemm(Xd, Wd, Y, stream=s)
+    assert wsm.stream_status(s) == wsm.WSM_ERR_TIMEOUT
+    assert wsm.stream_status(s) == 0
+    check_full(X, W, Y, what="the call on the grown workspace")
 
 
 def _dependent_tasks(M, dims, seed):
@@ -154,9 +177,9 @@ def test_prepared_chain_graph_replays_after_timeout(cluster):
     assert ch.status(s) == (wsm.WSM_ERR_TIMEOUT, -1)
     assert ch.status(s)[0] == wsm.WSM_OK
     for rep in range(3):
-        for y in ys:
-            y.fill_(float("nan"))
         with torch.cuda.stream(s):
+            for y in ys:
+                y.fill_(float("nan"))
             g.replay()
         s.synchronize()
         assert ch.status(s)[0] == wsm.WSM_OK

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "LIB_PATH", "WSM_OK", "WSM_ERR_INVALID", "WSM_ERR_UNSUPPORTED", "WSM_ERR_ALIGN", "WSM_ERR_NOMEM",
     "WSM_ERR_CUDA", "WSM_ERR_TIMEOUT", "PATH_AUTO", "PATH_STREAM", "PATH_UMMA", "ORDER_AUTO", "ORDER_M_MAJOR",
-    "ORDER_NAIVE", "L2_AUTO", "L2_EVICT_FIRST", "L2_NORMAL", "FLAG_W_READONLY", "FLAG_NO_PDL", "WsmError", "lib", "skinny_gemm", "plan",
+    "ORDER_NAIVE", "L2_AUTO", "L2_EVICT_FIRST", "L2_NORMAL", "FLAG_W_READONLY", "FLAG_NO_PDL", "FLAG_INDEPENDENT", "WsmError", "lib", "skinny_gemm", "plan",
     "workspace_bytes", "stream_status", "Task", "Chain", "gemm_chain", "chain_validate", "chain_plan", "last_error",
     "skinny_gemm_noalloc", "workspace_status", "gemm_chain_status", "debug_stall", "sm_die_map",
     "abi_version", "HEADER_SYMBOLS",
@@ -34,7 +34,7 @@ _STATUS_NAMES = {0: "WSM_OK", 1: "WSM_ERR_INVALID", 2: "WSM_ERR_UNSUPPORTED", 3:
 PATH_AUTO, PATH_STREAM, PATH_UMMA = 0, 1, 2
 ORDER_AUTO, ORDER_M_MAJOR, ORDER_NAIVE = 0, 1, 2
 L2_AUTO, L2_EVICT_FIRST, L2_NORMAL = 0, 1, 2
-FLAG_W_READONLY, FLAG_NO_PDL = 1, 2
+FLAG_W_READONLY, FLAG_NO_PDL, FLAG_INDEPENDENT = 1, 2, 4
 EPI_NONE, EPI_SILU_MUL, EPI_RESIDUAL = 0, 1, 2
 CHAIN_KERNELS_AUTO, CHAIN_KERNELS_ONE, CHAIN_KERNELS_SPLIT = 0, 1, 2
 K_ORDER_AUTO, K_ORDER_INCREASING, K_ORDER_ROTATED = 0, 1, 2

@@ -293,7 +293,8 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
     if (o->order < 0 || o->order > WSM_ORDER_NAIVE) return fail(WSM_ERR_INVALID, "bad order %d", o->order);
     if (o->l2_policy < 0 || o->l2_policy > WSM_L2_NORMAL) return fail(WSM_ERR_INVALID, "bad l2_policy %d", o->l2_policy);
     if (o->grid < 0) return fail(WSM_ERR_INVALID, "bad grid %d", o->grid);
-    if (o->flags & ~(WSM_FLAG_W_READONLY | WSM_FLAG_NO_PDL)) return fail(WSM_ERR_INVALID, "bad flags %#x", o->flags);
+    if (o->flags & ~(WSM_FLAG_W_READONLY | WSM_FLAG_NO_PDL | WSM_FLAG_INDEPENDENT))
+        return fail(WSM_ERR_INVALID, "bad flags %#x", o->flags);
     if (o->l2_prefetch_stages < -1)
         return fail(WSM_ERR_INVALID, "bad l2_prefetch_stages %d", o->l2_prefetch_stages);
     if (o->k_order < 0 || o->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", o->k_order);
@@ -350,7 +351,10 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
         g.threads = 64 + 2 * 128;   // producer, MMA, two epilogue warp sets
     }
     g.stages = std::min(kMaxStages, kRingBudget / g.stage_bytes);
-    wsm_status st = plan_units(g, g.grid, o->unit_stages, o->tail_tiles, o->tail_unit_stages);
+    // an independent call takes whole tiles unless told otherwise: no partial slots, no claims, no waits
+    const int unit_stages = ((o->flags & WSM_FLAG_INDEPENDENT) && o->unit_stages == 0 && o->tail_tiles <= 0)
+                                ? g.kb : o->unit_stages;
+    wsm_status st = plan_units(g, g.grid, unit_stages, o->tail_tiles, o->tail_unit_stages);
     if (st != WSM_OK) return st;
     // no more CTAs than work units
     if ((long long)g.grid > g.units()) g.grid = (int)g.units();
@@ -618,14 +622,15 @@ wsm_status check_ptrs(const void *X, const void *W, const void *Y, const float *
 struct Workspace {
     void *ptr = nullptr;
     size_t bytes = 0;
+    // Buffers this workspace has outgrown.  They stay allocated until the
+    // process exits: a CUDA graph captured while one of them was current still
+    // points at it, and replaying that graph must not touch freed memory.  The
+    // workspace at least doubles on each growth, so they hold less than the
+    // current one.  Their status words are still read by wsm_stream_status:
+    // calls queued before a growth record their time-outs there.
+    std::vector<void *> retired;
 };
 std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
-// Buffers a stream's workspace has outgrown.  They stay allocated until the
-// process exits: a CUDA graph captured while one of them was current still
-// points at it, and replaying that graph must not touch freed memory.  The
-// workspace at least doubles on each growth, so they hold less than the
-// current one.
-std::vector<void *> g_ws_retired;
 
 wsm_status stream_workspace(int dev, cudaStream_t stream, const Geo &g, void **out, size_t *out_bytes) {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -651,7 +656,7 @@ wsm_status stream_workspace(int dev, cudaStream_t stream, const Geo &g, void **o
         cudaFree(p);
         return cuda_fail(e, "cudaMemsetAsync(workspace)");
     }
-    if (w.ptr) g_ws_retired.push_back(w.ptr);
+    if (w.ptr) w.retired.push_back(w.ptr);
     w.ptr = p;
     w.bytes = bytes;
     *out = p;
@@ -1194,6 +1199,8 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     kp.k_rotate = (opts->k_order == 2) ? 1 : 0;
     kp.pdl = pdl_mode(opts->flags);
     kp.prefetch_stages = prefetch_stages_of(opts->l2_prefetch_stages, g.path);
+    // an independent call whose tiles are not split needs no scratch and no claims; split plans wait as usual
+    kp.independent = (opts->flags & WSM_FLAG_INDEPENDENT) && !g.split() ? 1 : 0;
     kp.run_ctl = nullptr;
     kp.status = reinterpret_cast<int *>(wsb + L.status_off);
     kp.dep_timeout_ns = kDefaultDepTimeoutNs;
@@ -1215,24 +1222,29 @@ wsm_status wsm_stream_status(wsm_stream_t stream_, int *code) {
     if (code) *code = 0;
     int dev = 0;
     WSM_CUDA(cudaGetDevice(&dev));
-    void *ptrs[2] = {nullptr, wsm::noalloc_scratch_ptr(dev)};
+    // the stream's workspace, the buffers it has outgrown (calls queued before a growth), then the no-alloc
+    // array of this device
+    std::vector<void *> ptrs;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         auto it = g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
-        if (it != g_ws.end()) ptrs[0] = it->second.ptr;
+        if (it != g_ws.end()) {
+            if (it->second.ptr) ptrs.push_back(it->second.ptr);
+            ptrs.insert(ptrs.end(), it->second.retired.rbegin(), it->second.retired.rend());
+        }
     }
+    const size_t n_stream = ptrs.size();
+    if (void *na = wsm::noalloc_scratch_ptr(dev)) ptrs.push_back(na);
     WSM_CUDA(cudaStreamSynchronize(stream));
-    // the stream's own workspace first, then the no-alloc array of this device
     int first[kStatusWords] = {};
     const char *where = nullptr;
-    for (int i = 0; i < 2; ++i) {
-        if (!ptrs[i]) continue;
+    for (size_t i = 0; i < ptrs.size(); ++i) {
         int h[kStatusWords] = {};
         wsm_status st = read_clear_status(ptrs[i], stream, h);
         if (st != WSM_OK) return st;
         if (h[0] != 0 && first[0] == 0) {
             memcpy(first, h, sizeof h);
-            where = i == 0 ? "skinny_gemm on this stream" : "skinny_gemm_noalloc on this device";
+            where = i < n_stream ? "skinny_gemm on this stream" : "skinny_gemm_noalloc on this device";
         }
     }
     if (first[0] == 0) return WSM_OK;

@@ -165,6 +165,10 @@ struct KParams {
     int xrow;                       // cluster mode: floats per exchange-buffer row (widest X tile + 4, the
                                     // last 4 holding the row's flag)
     const signed char *sm_die;      // die-grouped claims: die of each SM id (kMaxSmIds entries), or nullptr
+    int independent;                // single call that shares no data with the kernel before it and splits no
+                                    // tile: CTA c runs units c, c + grid, ... (no claim counters, no scratch),
+                                    // loads and stores without waiting for the previous kernel, and waits for it
+                                    // only before exiting (so stream order stays transitive for later kernels)
 };
 
 #if defined(__CUDACC__)

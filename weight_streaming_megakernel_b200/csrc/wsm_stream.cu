@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
         }
         abort_flag = 0;
         fence_mbar_init();
-        pdl_launch_dependents();
+        if (p.independent) pdl_launch_dependents();  // other calls trigger once past their grid wait (consumers)
     }
     __syncthreads();
     const unsigned long long wlim = p.wait_timeout_ns;
@@ -180,12 +180,12 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
             long long issued = 0;
             bool aborted = false;
             bool slot_ok = false;  // the wait for ring slot s has already succeeded
-            bool grid_dep_ok = p.pdl != 2;
-            if (p.pdl == 1) pdl_wait();
+            bool grid_dep_ok = p.pdl != 2 || p.independent;  // an independent call never waits here
+            if (p.pdl == 1 && !p.independent) pdl_wait();
             if (p.debug_stall_ns && blockIdx.x == 0) {
                 // test hook: after the previous kernel (whose exit clears the launch error flag), wait on a
                 // flag nothing sets until the limit passes, then abandon all of this CTA's work
-                if (!grid_dep_ok) {
+                if (!grid_dep_ok || p.independent) {
                     pdl_wait();
                     grid_dep_ok = true;
                 }
@@ -340,13 +340,13 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                         // take -- and never while this task's dependency is unmet, when every CTA would
                         // hold a second unit it cannot start (the claim counters belong to the previous
                         // kernel until the grid dependency is resolved)
-                        if (!claimed && dep_ok && k_end - kk <= kClaimLead) {
+                        if (!claimed && !p.independent && dep_ok && k_end - kk <= kClaimLead) {
                             next_u = claim_unit(cr);
                             claimed = true;
                         }
                     }
                     if (aborted) break;
-                    if (!claimed) {
+                    if (!claimed && !p.independent) {
                         // the unit streamed completely before its dependencies were resolved
                         if (!dep_ok) flush();
                         next_u = claim_unit(cr);
@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                     // whatever comes next needs a free slot: wait for it before the claim's result is used,
                     // so the claim's round trip overlaps the wait
                     if (!take_slot()) break;
-                    u = cr.lo + next_u + n_static;
+                    u = p.independent ? u + (int)gridDim.x : cr.lo + next_u + n_static;
                 }
                 if (np > 0) flush();
                 if (aborted) break;
@@ -384,7 +384,12 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
         const int o_m = ctid / TN;
         const int o_row = ctid - o_m * TN;
         const bool owner = ctid < TN * MMAX;
-        if (p.pdl) pdl_wait();  // Y and the scratch may still be in use by the previous kernel
+        if (p.pdl && !p.independent) {
+            pdl_wait();  // Y and the scratch may still be in use by the previous kernel
+            // the next kernel may launch once every CTA has seen this one's predecessor complete: so at most
+            // this kernel and the independent calls queued after it can still run when one of those starts
+            if (leader) pdl_launch_dependents();
+        }
         const unsigned int run_no = p.run_ctl ? ld_acquire_gpu(&p.run_ctl[0]) + 1u : 0u;  // this chain run
         int s = 0;
         uint32_t ph = 0;
@@ -530,7 +535,12 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
     __syncthreads();
     if (threadIdx.x == 0) {
         if (p.run_ctl) chain_run_done(p);
-        else single_call_done(p);
+        else {
+            // an independent call touches the shared exit counter and completes only after the previous
+            // kernel has: later kernels rely on stream order
+            if (p.independent && p.pdl) pdl_wait();
+            single_call_done(p);
+        }
     }
 }
 

@@ -396,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         mbar_init(&drain_bar, 1);
         abort_flag = 0;
         fence_mbar_init();
-        pdl_launch_dependents();
+        if (p.independent) pdl_launch_dependents();  // other calls trigger once past their grid wait (epilogue)
     }
     const int halves = p.wide ? 2 : 1;          // 128-row W halves per tile
     const uint32_t acc_stride = (uint32_t)(halves * kUmmaMaxN);  // TMEM columns per accumulator buffer
@@ -422,12 +422,13 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             long long issued = 0;
             bool aborted = false;
             bool slot_ok = false;           // the wait for ring slot s has already succeeded
-            bool grid_dep_ok = p.pdl != 2;  // mode 2 streams W before the previous kernel completes
-            if (p.pdl == 1) pdl_wait();
+            // mode 2 streams W before the previous kernel completes; an independent call never waits here
+            bool grid_dep_ok = p.pdl != 2 || p.independent;
+            if (p.pdl == 1 && !p.independent) pdl_wait();
             if (p.debug_stall_ns && blockIdx.x == 0) {
                 // test hook: after the previous kernel (whose exit clears the launch error flag), wait on a
                 // flag nothing sets until the limit passes, then abandon all of this CTA's work
-                if (!grid_dep_ok) {
+                if (!grid_dep_ok || p.independent) {
                     pdl_wait();
                     grid_dep_ok = true;
                 }
@@ -525,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 ClaimRange cr = by_die ? die_claim_range(T, my_die) : claim_range(T);
                 // (cluster mode: every task's first round is static, so a split tile's units of that round
                 // sit on the consecutive CTAs of one cluster)
-                const bool static_first = (t == 0 || p.cluster) && T.n_groups <= 1 && !by_die;
+                const bool static_first = (t == 0 || p.cluster) && T.n_groups <= 1 && !by_die;  // (independent: t == 0)
                 const int n_static = static_first ? min((int)gridDim.x, T.n_units) : 0;
                 int u;
                 if (static_first) {
@@ -589,13 +590,13 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                             // take -- and never while this task's dependency is unmet, when every CTA would
                             // hold a second unit it cannot start (the claim counters belong to the previous
                             // kernel until the grid dependency is resolved)
-                            if (!claimed && dep_ok && us.k_end - kk <= kClaimLead) {
+                            if (!claimed && !p.independent && dep_ok && us.k_end - kk <= kClaimLead) {
                                 next_u = claim_unit(cr);
                                 claimed = true;
                             }
                         }
                         if (aborted) break;
-                        if (!claimed) {
+                        if (!claimed && !p.independent) {
                             // the unit streamed completely before its dependencies were resolved
                             if (!dep_ok) flush();
                             next_u = claim_unit(cr);
@@ -603,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         // whatever comes next needs a free slot: wait for it before the claim's result is used,
                         // so the claim's round trip overlaps the wait
                         if (!take_slot()) break;
-                        u = cr.lo + next_u + n_static;
+                        u = p.independent ? u + (int)gridDim.x : cr.lo + next_u + n_static;
                     }
                     if (aborted || !by_die || pass > 0) break;
                     // own die's range done: help with the other die's
@@ -715,7 +716,12 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         const int row = q * 32 + lane;          // row of the 128-row tile = TMEM lane
         const int etid = threadIdx.x - (kEpiWarp0 + 4 * set) * 32;
         const bool leader = (etid == 0);
-        if (p.pdl) pdl_wait();                  // Y and the scratch may still be in use by the previous kernel
+        if (p.pdl && !p.independent) {
+            pdl_wait();  // Y and the scratch may still be in use by the previous kernel
+            // the next kernel may launch once every CTA has seen this one's predecessor complete: so at most
+            // this kernel and the independent calls queued after it can still run when one of those starts
+            if (set == 0 && leader) pdl_launch_dependents();
+        }
         const unsigned int run_no = p.run_ctl ? ld_acquire_gpu(&p.run_ctl[0]) + 1u : 0u;  // this chain run
         int warm_t = 0;                         // the task whose descriptor the set warms while it waits
         for (uint32_t k = 0;; ++k) {
@@ -825,7 +831,12 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     if (warp == 1) tmem_dealloc(tmem_base, p.wide ? kTmemColsWide : kTmemCols);
     if (threadIdx.x == 0) {
         if (p.run_ctl) chain_run_done(p);
-        else single_call_done(p);
+        else {
+            // an independent call touches the shared exit counter and completes only after the previous
+            // kernel has: later kernels rely on stream order
+            if (p.independent && p.pdl) pdl_wait();
+            single_call_done(p);
+        }
     }
 }
 
