@@ -300,6 +300,55 @@ def run_e2e(args, wsm, dev, datas, copies, mode, total_bytes, world, stream, n_s
             "overlap": "copies on their own streams, double-buffered across steps"}
 
 
+def back_to_back_per_shape(args, dev, hbm_peak, independent, grid, launches=32, replays=3):
+    """Each GEMM of the workload on its own: `launches` back-to-back
+    skinny_gemm launches of that one shape in a CUDA graph, cycling through
+    weight copies larger than 4x L2 together; device time per launch (CUDA
+    events around `replays` replays) and its fraction of the measured peak.
+    With `independent`, every launch carries WSM_FLAG_INDEPENDENT (the copies
+    share no buffers) on `grid` CTAs."""
+    import ctypes
+    import weight_streaming_megakernel_b200 as wsm
+    L = wsm.lib()
+    stream = torch.cuda.Stream(dev)
+    out = {}
+    for c in workload_cases(args.workload):
+        copies = n_copies([c])
+        datas = [setup_inputs([c], dev, seed_base=7 + r) for r in range(copies)]
+        fl = wsm.FLAG_W_READONLY | (wsm.FLAG_INDEPENDENT if independent else 0)
+        o = wsm._opts(m_tile=c.m_tile, flags=fl, grid=grid)
+        ptrs = [(d[0][1].data_ptr(), d[0][2].data_ptr(), d[0][3].data_ptr()) for d in datas]
+
+        def run():
+            for i in range(launches):
+                xp, wp, yp = ptrs[i % copies]
+                if L.skinny_gemm_ex(xp, wp, yp, c.M, c.N, c.K, ctypes.byref(o), stream.cuda_stream) != 0:
+                    raise RuntimeError(f"skinny_gemm failed: {wsm.last_error()}")
+
+        stream.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(stream):
+            run()                         # eager: sizes the stream's scratch before the capture
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            g.replay()
+            e0.record(stream)
+            for _ in range(replays):
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (replays * launches)
+        out[c.name] = {"us": round(us, 2), "frac_of_peak": round(alg_bytes(c) / (us * 1e-6) / 1e9 / hbm_peak, 4)}
+        del g, datas
+    if wsm.stream_status(stream) != 0:
+        raise RuntimeError("device-side status in the per-shape runs")
+    return out
+
+
 def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
     """Timed region: K steps, each one replay of a CUDA graph holding every
     GEMM launch of the step with an external timing event between launches
@@ -853,10 +902,26 @@ def main():
         import statistics as _st
         breakdown = {"ms_per_step": round(rb["ms_per_step"], 4),
                      "value_GBps": round(rb["total_bytes"] / (rb["ms_per_step"] * 1e-3) / 1e9, 1),
+                     "frac_of_peak": round(rb["total_bytes"] / (rb["ms_per_step"] * 1e-3) / 1e9 / hbm_peak, 4),
                      "note": "ms_per_step: the launches back to back in one graph; us_per_gemm_isolated: each "
                              "launch alone between two events, without the overlap with its neighbours",
                      "us_per_gemm_isolated": {c.name: round(_st.median(row[i] for row in rb["per_launch"]) * 1e3, 2)
                                               for i, c in enumerate(rb["cases"])}}
+        # the same launches with WSM_FLAG_INDEPENDENT on half of the SMs each (the step's GEMMs share no
+        # buffers): neighbouring launches run side by side
+        sub = argparse.Namespace(**vars(args))
+        sub.independent, sub.grid = True, 74
+        ri = run_gpu(sub, rank, world, local_rank, mode="launches", steps=min(args.steps, 5), extras=False)
+        gbs = ri["total_bytes"] / (ri["ms_per_step"] * 1e-3) / 1e9
+        breakdown["independent_launches"] = {"ms_per_step": round(ri["ms_per_step"], 4), "value_GBps": round(gbs, 1),
+                                             "frac_of_peak": round(gbs / hbm_peak, 4), "grid": 74}
+        # every GEMM on its own, 32 launches of its shape back to back: plain, and independent on a
+        # quarter of the SMs
+        dev = torch.device("cuda", local_rank)
+        breakdown["per_shape_back_to_back"] = {
+            "note": "32 launches of one shape back to back in a graph, weight copies > 4x L2; us per launch",
+            "plain": back_to_back_per_shape(args, dev, hbm_peak, False, 0),
+            "independent_grid37": back_to_back_per_shape(args, dev, hbm_peak, True, 37)}
 
     configurations = None
     if args.workload == "qwen3_decode" and args.mode == "chain" and not args.only and not args.no_configurations:
