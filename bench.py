@@ -907,14 +907,14 @@ def main():
                              "launch alone between two events, without the overlap with its neighbours",
                      "us_per_gemm_isolated": {c.name: round(_st.median(row[i] for row in rb["per_launch"]) * 1e3, 2)
                                               for i, c in enumerate(rb["cases"])}}
-        # the same launches with WSM_FLAG_INDEPENDENT on half of the SMs each (the step's GEMMs share no
-        # buffers): neighbouring launches run side by side
+        # the same launches with WSM_FLAG_INDEPENDENT on a quarter of the SMs each (the step's GEMMs share
+        # no buffers): neighbouring launches run side by side
         sub = argparse.Namespace(**vars(args))
-        sub.independent, sub.grid = True, 74
+        sub.independent, sub.grid = True, 37
         ri = run_gpu(sub, rank, world, local_rank, mode="launches", steps=min(args.steps, 5), extras=False)
         gbs = ri["total_bytes"] / (ri["ms_per_step"] * 1e-3) / 1e9
         breakdown["independent_launches"] = {"ms_per_step": round(ri["ms_per_step"], 4), "value_GBps": round(gbs, 1),
-                                             "frac_of_peak": round(gbs / hbm_peak, 4), "grid": 74}
+                                             "frac_of_peak": round(gbs / hbm_peak, 4), "grid": 37}
         # every GEMM on its own, 32 launches of its shape back to back: plain, and independent on a
         # quarter of the SMs
         dev = torch.device("cuda", local_rank)

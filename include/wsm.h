@@ -113,13 +113,15 @@ enum {
  * (unless unit_stages or tail_tiles ask for split ones), CTA c runs units c,
  * c + grid, ... without claim counters or partial slots, loads and stores
  * without waiting, lets the next kernel launch at once, and waits for the
- * kernel before it only on exit: every call
- * still completes after all work queued before it, so later work on the
- * stream sees theirs.  With a grid below the SM count (wsm_opts.grid)
- * consecutive independent calls share the GPU.  A plan that splits tiles
- * (asked for explicitly) ignores the flag.  A device-side time-out inside an independent call can
- * also make the calls running beside it give up (they share the stream's
- * launch error word); the stream status reports it either way. */
+ * kernel before it only on exit (in one CTA; the others free their SMs at
+ * once): every call still completes after all work queued before it, so
+ * later work on the stream sees theirs.  With a grid below the SM count
+ * (wsm_opts.grid) consecutive independent calls share the GPU; measured on
+ * B200, a quarter of the SMs per call suits back-to-back decode GEMMs of
+ * 30-200 MB.  A plan that splits tiles (asked for explicitly) ignores the
+ * flag.  A device-side time-out inside an independent call is kept apart
+ * from the calls beside it and reported by the same status query as any
+ * other call on that stream or workspace. */
 enum {
     WSM_FLAG_W_READONLY = 1,
     WSM_FLAG_NO_PDL = 2,

@@ -1202,7 +1202,7 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     // an independent call whose tiles are not split needs no scratch and no claims; split plans wait as usual
     kp.independent = (opts->flags & WSM_FLAG_INDEPENDENT) && !g.split() ? 1 : 0;
     kp.run_ctl = nullptr;
-    kp.status = reinterpret_cast<int *>(wsb + L.status_off);
+    kp.status = reinterpret_cast<int *>(wsb + L.status_off) + (kp.independent ? kIndStatusOff : 0);
     kp.dep_timeout_ns = kDefaultDepTimeoutNs;
     kp.wait_timeout_ns = kPipeTimeoutNs;
     kp.trace = nullptr;
@@ -1229,8 +1229,13 @@ wsm_status wsm_stream_status(wsm_stream_t stream_, int *code) {
         std::lock_guard<std::mutex> lk(g_mu);
         auto it = g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
         if (it != g_ws.end()) {
-            if (it->second.ptr) ptrs.push_back(it->second.ptr);
-            ptrs.insert(ptrs.end(), it->second.retired.rbegin(), it->second.retired.rend());
+            std::vector<void *> bufs;
+            if (it->second.ptr) bufs.push_back(it->second.ptr);
+            bufs.insert(bufs.end(), it->second.retired.rbegin(), it->second.retired.rend());
+            for (void *b : bufs) {
+                ptrs.push_back(b);
+                ptrs.push_back(static_cast<int *>(b) + kIndStatusOff);  // independent calls' block
+            }
         }
     }
     const size_t n_stream = ptrs.size();
@@ -1258,8 +1263,13 @@ wsm_status wsm_workspace_status(const void *workspace, size_t workspace_bytes, w
     if (!aligned16(workspace)) return fail(WSM_ERR_ALIGN, "workspace must be 16-byte aligned");
     if (workspace_bytes < 512) return fail(WSM_ERR_INVALID, "workspace of %zu bytes is too small to be one", workspace_bytes);
     int h[kStatusWords] = {};
+    int hi[kStatusWords] = {};  // independent calls' block
     wsm_status st = read_clear_status(workspace, reinterpret_cast<cudaStream_t>(stream_), h);
     if (st != WSM_OK) return st;
+    if ((st = read_clear_status(static_cast<const int *>(workspace) + kIndStatusOff,
+                                reinterpret_cast<cudaStream_t>(stream_), hi)) != WSM_OK)
+        return st;
+    if (h[0] == 0) memcpy(h, hi, sizeof h);
     if (h[0] == 0) return WSM_OK;
     if (code) *code = h[0];
     return fail(WSM_ERR_TIMEOUT, "device-side wait ran out in a call on this workspace (cta %d, site %d)", h[2], h[3]);

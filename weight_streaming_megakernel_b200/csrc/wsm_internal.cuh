@@ -47,6 +47,11 @@ constexpr int kStreamBoxK = 256;   // K elements per TMA box on the FMA path
 constexpr int kStatusWords = 4;    // words the host reads: [0] code, [1] task, [2] CTA, [3] site
 constexpr int kStatusLaunchErr = 4;
 constexpr int kStatusStallFlag = 5;
+// Independent single calls (KParams::independent) record into a second status block in the same 256-byte
+// status region: their launch error word must not make the calls running beside them give up, and no
+// call clears it (none of their waits consult it).
+constexpr int kIndStatusOff = 32;  // ints
+static_assert(kIndStatusOff + kStatusStallFlag < 64, "the status region holds 64 ints");
 constexpr int kSchedWords = 2;     // per task: [0] next unit to claim, [1] CTAs done claiming
 constexpr int kClaimLead = 4;      // a CTA claims its next unit this many stages before its unit ends
 constexpr int kColChunk = 256;     // output columns per readiness chunk (per-column data dependencies)

@@ -535,12 +535,10 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
     __syncthreads();
     if (threadIdx.x == 0) {
         if (p.run_ctl) chain_run_done(p);
-        else {
-            // an independent call touches the shared exit counter and completes only after the previous
-            // kernel has: later kernels rely on stream order
-            if (p.independent && p.pdl) pdl_wait();
-            single_call_done(p);
-        }
+        else if (!p.independent) single_call_done(p);
+        // an independent call completes only after the kernel before it (later kernels rely on stream
+        // order): one CTA waits for it, the others leave their SMs to the calls beside this one
+        else if (blockIdx.x == 0 && p.pdl) pdl_wait();
     }
 }
 
