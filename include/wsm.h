@@ -65,7 +65,8 @@ typedef enum {
 
 /* Kernel path.  AUTO takes the FMA path for M <= 2 at any size and for
  * M <= 4 up to 64 MiB of weights (measured crossovers on B200), the
- * tensor-core path otherwise. */
+ * tensor-core path otherwise; for calls with WSM_FLAG_INDEPENDENT the
+ * tensor-core path from M = 3. */
 enum {
     WSM_PATH_AUTO = 0,
     WSM_PATH_STREAM = 1, /* fp32 FMA dot products + warp-shuffle reduction, M <= 8 */

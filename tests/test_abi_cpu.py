@@ -101,6 +101,25 @@ def test_auto_path_crossovers():
     assert wsm.plan(3, 4097, 8192)["path"] == U
 
 
+def test_independent_calls_plan():
+    """WSM_FLAG_INDEPENDENT: whole tiles (no split-K) unless split units are
+    asked for, the grid as given (at most one CTA per unit), and the tensor
+    cores from M = 3 (the FMA path up to M = 2)."""
+    IND = wsm.FLAG_INDEPENDENT
+    for M, N, K in [(1, 4096, 4096), (16, 6144, 4096), (16, 4096, 4096), (64, 8192, 2048), (2, 1024, 8192)]:
+        for grid in (0, 37, 74):
+            p = wsm.plan(M, N, K, flags=IND, grid=grid)
+            assert p["units"] == p["n_tiles"] * p["m_tiles"], (M, N, K, grid)
+            assert p["grid"] == min(grid or 148, p["units"])
+    assert wsm.plan(16, 4096, 4096)["units"] > wsm.plan(16, 4096, 4096)["n_tiles"]  # without the flag: split
+    p = wsm.plan(16, 6144, 4096, flags=IND, unit_stages=2)
+    assert p["units"] > p["n_tiles"]
+    S, U = wsm.PATH_STREAM, wsm.PATH_UMMA
+    for M, want in ((1, S), (2, S), (3, U), (4, U), (8, U)):
+        assert wsm.plan(M, 4096, 4096, flags=IND)["path"] == want, M
+    assert wsm.plan(4, 4096, 4096)["path"] == S
+
+
 def test_fma_tile_rows():
     """FMA path tile height: 32 rows (16 KB boxes, the faster stream per SM)
     unless that leaves too few tiles (fewer than half the CTAs: K split in

@@ -44,7 +44,7 @@ def _nan(M, N, dtype=torch.bfloat16):
 @pytest.mark.parametrize("grid", [0, 74, 37])
 @pytest.mark.parametrize("path,M,N,K", [(wsm.PATH_STREAM, 1, 4096, 4096), (wsm.PATH_STREAM, 4, 2112, 7168),
                                         (wsm.PATH_UMMA, 16, 6144, 4096), (wsm.PATH_UMMA, 40, 1000, 2048),
-                                        (wsm.PATH_UMMA, 64, 4096, 1032)])
+                                        (wsm.PATH_UMMA, 64, 4096, 1032), (wsm.PATH_AUTO, 3, 6144, 4096)])
 def test_back_to_back_independent_calls(path, M, N, K, grid):
     p = wsm.plan(M, N, K, path=path, grid=grid, flags=IND)
     assert p["units"] == p["n_tiles"] * p["m_tiles"], "an independent call plans whole tiles"

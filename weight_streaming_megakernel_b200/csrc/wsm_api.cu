@@ -226,9 +226,16 @@ wsm_status plan_units(Geo &g, int ctas, int unit_stages, int tail_tiles, int tai
 // 35.8 against 39.5 us); at M = 3, 4 it wins up to about 64 MiB of weights
 // (it is ALU-bound from there: 8 FMA per weight element at M = 8); the
 // tensor-core path wins everywhere else.
-int auto_path(int M, long long w_bytes) {
+// Independent calls (WSM_FLAG_INDEPENDENT, several running side by side on a
+// quarter of the SMs each) take the tensor cores from M = 3: measured with 32
+// back-to-back launches per decode shape, at M = 3-4 qkv 84-86 % of the copy
+// peak against 72-75 % on the FMA path, o 78 against 69-70, gate_up 100
+// against 87-88, down 96 against 90; at M <= 2 the FMA path stays ahead on
+// o, qkv and down (80-99 % against 76-97).
+int auto_path(int M, long long w_bytes, bool independent = false) {
     const long long MiB = 1ll << 20;
     if (M <= 2) return WSM_PATH_STREAM;
+    if (independent) return WSM_PATH_UMMA;
     if (M <= 4 && w_bytes <= 64 * MiB) return WSM_PATH_STREAM;
     return WSM_PATH_UMMA;
 }
@@ -298,7 +305,7 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
     if (o->l2_prefetch_stages < -1)
         return fail(WSM_ERR_INVALID, "bad l2_prefetch_stages %d", o->l2_prefetch_stages);
     if (o->k_order < 0 || o->k_order > 2) return fail(WSM_ERR_INVALID, "bad k_order %d", o->k_order);
-    if (path == WSM_PATH_AUTO) path = auto_path(M, 2ll * N * K);
+    if (path == WSM_PATH_AUTO) path = auto_path(M, 2ll * N * K, (o->flags & WSM_FLAG_INDEPENDENT) != 0);
     g = Geo{};
     g.path = path;
     g.grid = (o->grid > 0) ? std::min(o->grid, num_sms) : num_sms;
