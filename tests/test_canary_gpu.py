@@ -11,7 +11,8 @@ column of a ragged N would land in them.
 
 Cases: ragged N (17, 129, 2112) and K (40, 1000, 4104), every M class on both
 kernel paths, the SiLU*mul output of width N/2, split-K partial slots inside
-a caller workspace, and chain tasks (plain, residual in place, SiLU*mul)."""
+a caller workspace, independent calls (whole tiles, no waits), and chain
+tasks (plain, residual in place, SiLU*mul)."""
 import pytest
 import torch
 
@@ -88,6 +89,41 @@ def test_plain_outputs_and_workspace_stay_in_bounds(path, M, N, K):
         yf.intact()
         ws.intact()
         check_full(x, w, y.t, yf.t, what=f"path={path} M={M} N={N} K={K} unit_stages={unit_stages}")
+
+
+@pytest.mark.parametrize("path,M,N,K", [(p, M, N, K) for p, M, N, K in CASES if M in (1, 3, 5, 17, 64)])
+def test_independent_calls_stay_in_bounds(path, M, N, K):
+    """Independent calls (whole tiles in a fixed round-robin, no waits) on
+    ragged shapes, four back to back on a reduced grid, each output and its
+    fp32 copy guarded; a plain epilogue, SiLU*mul (N/2 wide) and a residual
+    written in place over R."""
+    IND = wsm.FLAG_INDEPENDENT
+    xs, ws = zip(*[synth.make_xw(M, N, K, seed=M * 7 + N + i) for i in range(4)])
+    outs = []
+    for i in range(4):
+        y = Guarded(M, N, torch.bfloat16)
+        yf = Guarded(M, N, torch.float32)
+        wsm.skinny_gemm(xs[i].to(DEV), ws[i].to(DEV), y.t, path=path, yf32=yf.t, grid=37, flags=IND)
+        outs.append((y, yf))
+    if N % 16 == 0:
+        h = Guarded(M, N // 2, torch.bfloat16)
+        wsm.skinny_gemm(xs[0].to(DEV), ws[0].to(DEV), h.t, path=path, grid=37, flags=IND, epilogue=wsm.EPI_SILU_MUL)
+    r = synth.make_x(M, N, seed=N + 1)
+    yr = Guarded(M, N, torch.bfloat16, fill=r.to(DEV))
+    wsm.skinny_gemm(xs[1].to(DEV), ws[1].to(DEV), yr.t, path=path, grid=37, flags=IND, epilogue=wsm.EPI_RESIDUAL,
+                    r=yr.t)
+    assert wsm.stream_status() == 0
+    for i, (y, yf) in enumerate(outs):
+        y.intact()
+        yf.intact()
+        check_full(xs[i], ws[i], y.t, yf.t, what=f"independent call {i} path={path} M={M} N={N} K={K}")
+    if N % 16 == 0:
+        h.intact()
+        H, G, U, Sg, Su = oracle.silu_mul_ref(xs[0], ws[0])
+        check_bounded(h.t, None, H, oracle.fused_bounds("silu_mul", G=G, U=U, Sg=Sg, Su=Su), "independent silu")
+    yr.intact()
+    Y, S = oracle.residual_ref(xs[1], ws[1], r)
+    check_bounded(yr.t, None, Y, oracle.fused_bounds("residual", S=S, Y=Y), "independent residual in place")
 
 
 @pytest.mark.parametrize("path,M", [(wsm.PATH_STREAM, 2), (wsm.PATH_UMMA, 16), (wsm.PATH_UMMA, 33)])
