@@ -101,11 +101,19 @@ def workload_cases(name):
 L2_BYTES = 126 * 2 ** 20
 
 
-def n_copies(cases):
+def n_copies(cases, min_calls=1):
     """Weight copies a step cycles through so that consecutive steps touch at
-    least 4x the L2 size (1 when one step's weights already do)."""
+    least 4x the L2 size (1 when one step's weights already do), and a GEMM's
+    weights come back only after `min_calls` launches: independent launches
+    run several at a time, and two of them on the same copy would share its
+    weights through L2."""
     w = sum(2 * c.N * c.K for c in cases)
-    return max(1, -(-4 * L2_BYTES // w))
+    return max(1, -(-4 * L2_BYTES // w), -(-min_calls // len(cases)))
+
+
+# independent launches in flight at once: about SMs / grid (4-5 at a quarter of the SMs); a weight copy
+# comes back only after twice that many
+INDEPENDENT_REUSE_CALLS = 10
 
 
 def alg_bytes(c):
@@ -313,7 +321,7 @@ def back_to_back_per_shape(args, dev, hbm_peak, independent, grid, launches=32, 
     stream = torch.cuda.Stream(dev)
     out = {}
     for c in workload_cases(args.workload):
-        copies = n_copies([c])
+        copies = n_copies([c], INDEPENDENT_REUSE_CALLS if independent else 1)
         datas = [setup_inputs([c], dev, seed_base=7 + r) for r in range(copies)]
         fl = wsm.FLAG_W_READONLY | (wsm.FLAG_INDEPENDENT if independent else 0)
         o = wsm._opts(m_tile=c.m_tile, flags=fl, grid=grid)
@@ -366,7 +374,7 @@ def run_gpu(args, rank, world, local_rank, mode=None, steps=None, extras=True):
         assert cases, f"no case named {args.only}"
     # Inputs larger than L2 between timed steps: a step whose weights fit in
     # L2 several times cycles through copies (step k uses copy k % copies).
-    copies = n_copies(cases)
+    copies = n_copies(cases, INDEPENDENT_REUSE_CALLS if mode == "launches" and args.independent else 1)
     datas = [setup_inputs(cases, dev, seed_base=rank * 1000 + r) for r in range(copies)]
     data = datas[0]
     cur = [0]  # copy the next launches use
@@ -738,15 +746,18 @@ def oracle_sample_rate(cases, budget_s, threads=0):
 # None).  The default run reports every one of them beside its headline (the Qwen3-8B decode step).
 CONFIGURATIONS = (
     ("c1_single_m1_4096x4096", "single", "launches", 0.80, {"steps": 64}),
-    # back-to-back calls on unrelated buffers with WSM_FLAG_INDEPENDENT on a quarter of the SMs: about
-    # four calls run at once; 64 launches per timed graph so that its start and end (the first call alone,
-    # the last one draining) weigh little
+    # back-to-back calls on unrelated buffers with WSM_FLAG_INDEPENDENT (automatic grid: at most a quarter
+    # of the SMs each, so about four calls run at once); 64 launches per timed graph so that its start and
+    # end (the first call alone, the last one draining) weigh little
     ("c1_single_m1_4096x4096_independent", "single", "launches", 0.80,
-     {"independent": True, "grid": 37, "steps": 64}),
+     {"independent": True, "grid": 0, "steps": 64}),
     ("c2_qwen3_8b_decode_gemms", "qwen3_decode", "chain", 0.80),
     ("c3_skinny_k7168_k8192", "skinny", "chain", 0.80),
     ("c4_l2_reuse_m32_m64", "l2_reuse", "chain", None),
     ("c4_l2_reuse_m32_m64_whole_m_tile", "l2_reuse_whole_m", "chain", None),
+    # the same four GEMMs (gate_up, down at M = 32, 64, one M-tile each) as independent single launches
+    ("c4_l2_reuse_m32_m64_independent_launches", "l2_reuse_whole_m", "launches", 0.80,
+     {"independent": True, "grid": 0}),
     ("c5_chain_36x4_m16", "chain", "chain", 0.75),
 )
 
@@ -831,6 +842,7 @@ def main():
         cases = [c for c in cases if c.name in args.only.split(",")]
         if not cases:
             raise SystemExit(f"--only {args.only}: no case of workload {args.workload} has these names")
+    n_cp = n_copies(cases, INDEPENDENT_REUSE_CALLS if args.mode == "launches" and args.independent else 1)
     config = {"workload": {"qwen3_decode": "qwen3_8b_decode_gemms", "single": "single_gemm_m1_4096x4096",
                            "skinny": "skinny_k7168_k8192", "l2_reuse": "l2_reuse_m32_m64",
                            "l2_reuse_whole_m": "l2_reuse_m32_m64_whole_m_tile",
@@ -841,9 +853,9 @@ def main():
               "weight_bytes_per_step": sum(2 * c.N * c.K for c in cases),
               "l2": "inputs larger than L2: every GEMM of a step has its own weights "
                     f"({sum(2 * c.N * c.K for c in cases) / 1e9:.3f} GB per step, L2 126 MB)"
-                    + (f"; steps cycle through {n_copies(cases)} weight copies "
-                       f"({n_copies(cases) * sum(2 * c.N * c.K for c in cases) / 1e9:.2f} GB)"
-                       if n_copies(cases) > 1 else ""),
+                    + (f"; steps cycle through {n_cp} weight copies "
+                       f"({n_cp * sum(2 * c.N * c.K for c in cases) / 1e9:.2f} GB)"
+                       if n_cp > 1 else ""),
               "parallelism": f"replicas{world}" if world > 1 else "single",
               "mode": args.mode + (" (one persistent kernel per step, W read-only flag)" if args.mode == "chain"
                                    else " (one skinny_gemm launch per GEMM, W read-only flag"
@@ -907,21 +919,22 @@ def main():
                              "launch alone between two events, without the overlap with its neighbours",
                      "us_per_gemm_isolated": {c.name: round(_st.median(row[i] for row in rb["per_launch"]) * 1e3, 2)
                                               for i, c in enumerate(rb["cases"])}}
-        # the same launches with WSM_FLAG_INDEPENDENT on a quarter of the SMs each (the step's GEMMs share
-        # no buffers): neighbouring launches run side by side
+        # the same launches with WSM_FLAG_INDEPENDENT (the step's GEMMs share no buffers; automatic grid:
+        # at most a quarter of the SMs each): neighbouring launches run side by side
         sub = argparse.Namespace(**vars(args))
-        sub.independent, sub.grid = True, 37
+        sub.independent, sub.grid = True, 0
         ri = run_gpu(sub, rank, world, local_rank, mode="launches", steps=min(args.steps, 5), extras=False)
         gbs = ri["total_bytes"] / (ri["ms_per_step"] * 1e-3) / 1e9
         breakdown["independent_launches"] = {"ms_per_step": round(ri["ms_per_step"], 4), "value_GBps": round(gbs, 1),
-                                             "frac_of_peak": round(gbs / hbm_peak, 4), "grid": 37}
-        # every GEMM on its own, 32 launches of its shape back to back: plain, and independent on a
-        # quarter of the SMs
+                                             "frac_of_peak": round(gbs / hbm_peak, 4), "grid": "auto"}
+        # every GEMM on its own, 32 launches of its shape back to back: plain, and independent
         dev = torch.device("cuda", local_rank)
         breakdown["per_shape_back_to_back"] = {
-            "note": "32 launches of one shape back to back in a graph, weight copies > 4x L2; us per launch",
+            "note": "32 launches of one shape back to back in a graph, weight copies > 4x L2 (independent: a "
+                    "copy comes back after 10 launches at the earliest); us per launch; independent = "
+                    "WSM_FLAG_INDEPENDENT with the automatic grid (at most a quarter of the SMs, even rounds)",
             "plain": back_to_back_per_shape(args, dev, hbm_peak, False, 0),
-            "independent_grid37": back_to_back_per_shape(args, dev, hbm_peak, True, 37)}
+            "independent": back_to_back_per_shape(args, dev, hbm_peak, True, 0)}
 
     configurations = None
     if args.workload == "qwen3_decode" and args.mode == "chain" and not args.only and not args.no_configurations:

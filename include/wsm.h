@@ -100,10 +100,13 @@ enum {
  * (griddepcontrol.wait) before touching global memory, so stream order is
  * kept; it lets the kernel after it launch only once each of its CTAs has
  * seen that wait through.  WSM_FLAG_W_READONLY relaxes the wait for W only:
- * the caller promises that the kernel queued just before this call does not
- * write W, and the weight stream (which is the whole cost of a decode GEMM)
- * then starts before that kernel has finished; X, Y and the scratch still
- * wait.  WSM_FLAG_NO_PDL launches without programmatic dependent launch.
+ * the caller promises that no call that may still run when this one starts
+ * writes W -- the call just before it, and when that is an independent call
+ * (below), every call back to and including the last one without
+ * WSM_FLAG_INDEPENDENT -- and the weight stream (which is the whole cost of a
+ * decode GEMM) then starts before those have finished; X, Y and the scratch
+ * still wait.  WSM_FLAG_NO_PDL launches without programmatic dependent
+ * launch.
  *
  * WSM_FLAG_INDEPENDENT (single calls only) goes further.  Such a call may run
  * at the same time as every call queued since the last library call without
@@ -116,11 +119,11 @@ enum {
  * without waiting, lets the next kernel launch at once, and waits for the
  * kernel before it only on exit (in one CTA; the others free their SMs at
  * once): every call still completes after all work queued before it, so
- * later work on the stream sees theirs.  With a grid below the SM count
- * (wsm_opts.grid) consecutive independent calls share the GPU; measured on
- * B200, a quarter of the SMs per call suits back-to-back decode GEMMs of
- * 30-200 MB.  A plan that splits tiles (asked for explicitly) ignores the
- * flag.  A device-side time-out inside an independent call is kept apart
+ * later work on the stream sees theirs.  Consecutive independent calls share
+ * the GPU: with wsm_opts.grid = 0 each takes at most a quarter of the SMs,
+ * in even rounds of its units (measured best on B200 for back-to-back decode
+ * GEMMs of 30-200 MB); a grid given explicitly is taken as it is.  A plan
+ * that splits tiles (asked for explicitly) ignores the flag.  A device-side time-out inside an independent call is kept apart
  * from the calls beside it and reported by the same status query as any
  * other call on that stream or workspace. */
 enum {

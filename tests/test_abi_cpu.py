@@ -103,14 +103,24 @@ def test_auto_path_crossovers():
 
 def test_independent_calls_plan():
     """WSM_FLAG_INDEPENDENT: whole tiles (no split-K) unless split units are
-    asked for, the grid as given (at most one CTA per unit), and the tensor
-    cores from M = 3 (the FMA path up to M = 2)."""
+    asked for; grid 0 = at most a quarter of the SMs in even rounds of units,
+    a given grid as it is (at most one CTA per unit); the tensor cores from
+    M = 3 (the FMA path up to M = 2)."""
     IND = wsm.FLAG_INDEPENDENT
-    for M, N, K in [(1, 4096, 4096), (16, 6144, 4096), (16, 4096, 4096), (64, 8192, 2048), (2, 1024, 8192)]:
+    for M, N, K in [(1, 4096, 4096), (16, 6144, 4096), (16, 4096, 4096), (64, 8192, 2048), (2, 1024, 8192),
+                    (1, 24576, 4096)]:
         for grid in (0, 37, 74):
             p = wsm.plan(M, N, K, flags=IND, grid=grid)
-            assert p["units"] == p["n_tiles"] * p["m_tiles"], (M, N, K, grid)
-            assert p["grid"] == min(grid or 148, p["units"])
+            u = p["units"]
+            assert u == p["n_tiles"] * p["m_tiles"], (M, N, K, grid)
+            if grid:
+                assert p["grid"] == min(grid, u)
+            else:  # at most a quarter of the SMs, in even rounds
+                rounds = -(-u // 37)
+                assert p["grid"] == -(-u // rounds) and p["grid"] <= 37, (M, N, K, p["grid"])
+    assert wsm.plan(1, 4096, 4096, flags=IND)["grid"] == 32      # 128 units: 4 rounds of 32
+    assert wsm.plan(16, 6144, 4096, flags=IND)["grid"] == 24     # 48 units: 2 rounds of 24
+    assert wsm.plan(16, 4096, 4096, flags=IND)["grid"] == 32     # 32 units: 1 round
     assert wsm.plan(16, 4096, 4096)["units"] > wsm.plan(16, 4096, 4096)["n_tiles"]  # without the flag: split
     p = wsm.plan(16, 6144, 4096, flags=IND, unit_stages=2)
     assert p["units"] > p["n_tiles"]

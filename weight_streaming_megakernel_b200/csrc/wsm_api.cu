@@ -363,6 +363,13 @@ wsm_status make_geo(int M, int N, int K, int num_sms, const wsm_opts *o, Geo &g,
                                 ? g.kb : o->unit_stages;
     wsm_status st = plan_units(g, g.grid, unit_stages, o->tail_tiles, o->tail_unit_stages);
     if (st != WSM_OK) return st;
+    if ((o->flags & WSM_FLAG_INDEPENDENT) && o->grid == 0 && !g.split()) {
+        // independent calls run side by side: at most a quarter of the SMs each, in even rounds of units
+        const long long u = g.units();
+        const long long q = std::max(1, num_sms / 4);
+        const long long rounds = (u + q - 1) / q;
+        g.grid = (int)((u + rounds - 1) / rounds);
+    }
     // no more CTAs than work units
     if ((long long)g.grid > g.units()) g.grid = (int)g.units();
     if (g.l2 = o->l2_policy, g.l2 == WSM_L2_AUTO) g.l2 = (g.n_mt > 1) ? WSM_L2_NORMAL : WSM_L2_EVICT_FIRST;
