@@ -509,3 +509,37 @@ def test_benchmark_chain_full_size_sampled(config):
     ch.close()
     del tasks
     torch.cuda.empty_cache()
+
+
+def test_layer_chain_full_36_layers_sampled():
+    """The 36 x 4 layer chain at M = 16 exactly as the benchmark runs it:
+    task t waits for task t - 1 (ordering only; every task has its own X),
+    the weights flagged read-only, 13.9 GB of weights in one kernel; two
+    runs (the second on the counters the first left), then sampled outputs
+    of every task against the oracle."""
+    cases = synth.chain_layout()
+    assert len(cases) == 144
+    tasks = []
+    for t, c in enumerate(cases):
+        g = torch.Generator(device=DEV)
+        g.manual_seed(3000 + t)
+        x = torch.randn(c.M, c.K, generator=g, device=DEV).to(torch.bfloat16)
+        w = (torch.randn(c.N, c.K, generator=g, device=DEV) / c.K ** 0.5).to(torch.bfloat16)
+        tasks.append(wsm.Task(x, w, torch.empty(c.M, c.N, dtype=torch.bfloat16, device=DEV), dep=t - 1,
+                              yf32=torch.empty(c.M, c.N, dtype=torch.float32, device=DEV)))
+    ch = wsm.Chain(tasks, flags=wsm.FLAG_W_READONLY)
+    for _ in range(2):
+        for t in tasks:
+            t.y.fill_(float("nan"))
+        ch.run()
+    assert ch.status()[0] == wsm.WSM_OK, wsm.last_error()
+    rng = np.random.default_rng(11)
+    for i, (c, t) in enumerate(zip(cases, tasks)):
+        ms = rng.integers(0, c.M, 256)
+        ns = rng.integers(0, c.N, 256)
+        ns[:16] = np.arange(c.N - 16, c.N)
+        check_sampled(t.x, t.w, t.y, t.yf32, ms, ns, what=f"layer chain task {i} ({c.name})")
+        assert not torch.isnan(t.y.float()).any(), f"task {i}: unwritten outputs"
+    ch.close()
+    del tasks
+    torch.cuda.empty_cache()

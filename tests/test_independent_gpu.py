@@ -16,12 +16,13 @@ The tests check the results and the stream-order contract of the flag:
   their X: the overwrite must wait for every one of them;
 - the flag with split tiles asked for explicitly (it is then ignored);
 - a device-side time-out inside an independent call (the stall hook)."""
+import numpy as np
 import pytest
 import torch
 
 import synth
 import weight_streaming_megakernel_b200 as wsm
-from parity import check_full
+from parity import check_full, check_sampled
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -168,3 +169,38 @@ def test_chain_rejects_the_flag():
     y = torch.empty(16, 512, dtype=torch.bfloat16, device=DEV)
     with pytest.raises(wsm.WsmError):
         wsm.Chain([wsm.Task(x.to(DEV), w.to(DEV), y)], flags=IND)
+
+
+@pytest.mark.parametrize("config", ["qwen3_decode", "single", "l2_reuse"])
+def test_full_size_independent_launches_sampled(config):
+    """The benchmark's independent-launch configurations at full size: every
+    GEMM of the set launched back to back with the flag and the automatic
+    grid (the weights flagged read-only too), on two weight copies so that
+    calls of the same shape run side by side; sampled outputs of every call,
+    the ragged end of N included, and no output left unwritten."""
+    cases = getattr(synth, f"config_{config}")(**({"m_tiles": (0,)} if config == "l2_reuse" else {}))
+    calls = []
+    for r in range(2):
+        for c in cases:
+            g = torch.Generator(device=DEV)
+            g.manual_seed(5000 + 97 * r + c.seed + c.M * 7 + c.N)
+            x = torch.randn(c.M, c.K, generator=g, device=DEV).to(torch.bfloat16)
+            w = (torch.randn(c.N, c.K, generator=g, device=DEV) / c.K ** 0.5).to(torch.bfloat16)
+            calls.append((c, x, w, _nan(c.M, c.N), _nan(c.M, c.N, torch.float32)))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for c, x, w, y, yf in calls:
+            p = wsm.plan(c.M, c.N, c.K, flags=IND | wsm.FLAG_W_READONLY)
+            assert p["units"] == p["n_tiles"] * p["m_tiles"] and p["grid"] <= 37
+            wsm.skinny_gemm(x, w, y, yf32=yf, flags=IND | wsm.FLAG_W_READONLY, stream=s)
+    assert wsm.stream_status(s) == 0
+    rng = np.random.default_rng(9)
+    for i, (c, x, w, y, yf) in enumerate(calls):
+        ms = rng.integers(0, c.M, 1024)
+        ns = rng.integers(0, c.N, 1024)
+        ns[:32] = np.arange(c.N - 32, c.N)
+        check_sampled(x, w, y, yf, ms, ns, what=f"independent call {i} ({c.name})")
+        assert not torch.isnan(y.float()).any(), f"call {i}: unwritten outputs"
+    del calls
+    torch.cuda.empty_cache()
