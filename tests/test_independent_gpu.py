@@ -204,3 +204,52 @@ def test_full_size_independent_launches_sampled(config):
         assert not torch.isnan(y.float()).any(), f"call {i}: unwritten outputs"
     del calls
     torch.cuda.empty_cache()
+
+
+def test_random_mix_of_independent_calls():
+    """40 seeded random calls back to back with the flag -- both paths and
+    AUTO, M 1..64 (M-tiles where the path has them), ragged N and K, the
+    three epilogues, grids automatic or given -- many of them running side
+    by side; then a call without the flag that reads one of their outputs.
+    Every output against the oracle."""
+    import oracle
+    from parity import check_bounded
+    rng = np.random.default_rng(2024)
+    calls = []
+    for i in range(40):
+        path = int(rng.choice([wsm.PATH_AUTO, wsm.PATH_STREAM, wsm.PATH_UMMA]))
+        M = int(rng.integers(1, 9)) if path == wsm.PATH_STREAM else int(rng.integers(1, 65))
+        epi = int(rng.choice([wsm.EPI_NONE, wsm.EPI_NONE, wsm.EPI_SILU_MUL, wsm.EPI_RESIDUAL]))
+        N = int(rng.integers(1, 40)) * 16 if epi == wsm.EPI_SILU_MUL else int(rng.integers(1, 700))
+        if i == 0:
+            epi, N = wsm.EPI_NONE, 8 * int(rng.integers(1, 80))  # read by the last call: K % 8 == 0 there
+        K = int(rng.integers(1, 320)) * 8
+        grid = int(rng.choice([0, 0, 5, 16, 37, 148]))
+        m_tile = int(rng.choice([0, 16, 32])) if path == wsm.PATH_UMMA and M > 16 else 0
+        x, w = synth.make_xw(M, N, K, seed=7000 + i)
+        out_n = N // 2 if epi == wsm.EPI_SILU_MUL else N
+        r = synth.make_x(M, N, seed=8000 + i) if epi == wsm.EPI_RESIDUAL else None
+        calls.append(dict(path=path, M=M, N=N, K=K, epi=epi, grid=grid, m_tile=m_tile, x=x, w=w, r=r,
+                          xd=x.to(DEV), wd=w.to(DEV), rd=None if r is None else r.to(DEV),
+                          y=_nan(M, out_n), yf=_nan(M, out_n, torch.float32)))
+    wd_last = synth.make_w(96, calls[0]["y"].shape[1], seed=9000)
+    y_last = _nan(calls[0]["M"], 96)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for c in calls:
+            wsm.skinny_gemm(c["xd"], c["wd"], c["y"], path=c["path"], yf32=c["yf"], grid=c["grid"],
+                            m_tile=c["m_tile"], flags=IND, epilogue=c["epi"], r=c["rd"], stream=s)
+        wsm.skinny_gemm(calls[0]["y"], wd_last.to(DEV), y_last, stream=s)
+    assert wsm.stream_status(s) == 0
+    for i, c in enumerate(calls):
+        what = f"call {i}: path {c['path']} M {c['M']} N {c['N']} K {c['K']} epi {c['epi']} grid {c['grid']}"
+        if c["epi"] == wsm.EPI_NONE:
+            check_full(c["x"], c["w"], c["y"], c["yf"], what=what)
+        elif c["epi"] == wsm.EPI_SILU_MUL:
+            H, G, U, Sg, Su = oracle.silu_mul_ref(c["x"], c["w"])
+            check_bounded(c["y"], c["yf"], H, oracle.fused_bounds("silu_mul", G=G, U=U, Sg=Sg, Su=Su), what)
+        else:
+            Y, S = oracle.residual_ref(c["x"], c["w"], c["r"])
+            check_bounded(c["y"], c["yf"], Y, oracle.fused_bounds("residual", S=S, Y=Y), what)
+    check_full(calls[0]["y"].cpu(), wd_last, y_last, what="the call after them")
