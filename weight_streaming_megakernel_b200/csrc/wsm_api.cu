@@ -21,7 +21,7 @@
 
 namespace wsm {
 
-__global__ void wsm_umma_kernel(const __grid_constant__ KParams p);
+const void *umma_kernel_ptr(bool ext);                   // wsm_umma.cu
 const void *stream_kernel_ptr(int mmax, int tile_rows);  // wsm_stream.cu
 void *noalloc_scratch_ptr(int dev);                      // wsm_noalloc.cu: nullptr until set up on `dev`
 wsm_status die_map_of_device(int dev, const std::vector<int> **die, wsm_die_info *info);  // wsm_die.cu
@@ -94,6 +94,7 @@ struct Geo {
     int ku = 1, nu = 1;        // head tiles: stages per work unit, units per tile
     int ku_t = 1, nu_t = 1;    // tail tiles: the same
     int tail = 0;              // tail tiles (the last ones of the schedule)
+    bool ext = false;          // tensor-core kernel with cluster reduction and die-grouped claims compiled in
     int order = WSM_ORDER_M_MAJOR;
     int l2 = WSM_L2_EVICT_FIRST;
     int grid = 0;
@@ -486,8 +487,8 @@ wsm_status dev_info(int dev, DevInfo **out) {
 // Kernel for a geometry, and its slot in DevInfo::attr_set.
 const void *kernel_for(const Geo &g, int *slot) {
     if (g.path == WSM_PATH_UMMA) {
-        *slot = 0;
-        return reinterpret_cast<const void *>(&wsm_umma_kernel);
+        *slot = g.ext ? 9 : 0;
+        return umma_kernel_ptr(g.ext);
     }
     *slot = (g.mmax == 1 ? 1 : g.mmax == 2 ? 2 : g.mmax == 4 ? 3 : 4) + (g.tile_rows == 32 ? 4 : 0);
     return stream_kernel_ptr(g.mmax, g.tile_rows);
@@ -513,6 +514,7 @@ wsm_status prepare_kernel(DevInfo *d, const Geo &g, const void **fn) {
 wsm_status cluster_ctas_of(DevInfo *d, int *out) {
     Geo g;
     g.path = WSM_PATH_UMMA;
+    g.ext = true;
     const void *fn;
     wsm_status st = prepare_kernel(d, g, &fn);
     if (st != WSM_OK) return st;
@@ -1221,6 +1223,7 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     kp.wait_timeout_ns = kPipeTimeoutNs;
     kp.trace = nullptr;
     const void *fn;
+    g.ext = g.n_mt > 1;  // M-tiled: the tensor-core kernel with the K rotation's weight-column mapping
     if ((st = prepare_kernel(d, g, &fn)) != WSM_OK) return st;
     kp.debug_stall_ns = take_stall();
     if ((st = launch(fn, g, kp, stream, false)) != WSM_OK) return st;
@@ -1574,7 +1577,12 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
         }
         cudaMemset(ch->d_trace, 0, ch->trace_elems * 8);
     }
-    if ((st = prepare_kernel(d, ring, &ch->fn)) != WSM_OK) {
+    // cluster reduction, die-grouped claims and M-tiled tasks run in the kernel instantiation that has them
+    // compiled in
+    bool any_m_tiled = false;
+    for (int i = 0; i < n; ++i) any_m_tiled = any_m_tiled || geos[i].n_mt > 1;
+    ch->geo.ext = cp.cluster != 0 || cp.die_groups || any_m_tiled;
+    if ((st = prepare_kernel(d, ch->geo, &ch->fn)) != WSM_OK) {
         cleanup();
         return st;
     }

@@ -347,6 +347,7 @@ static __device__ __noinline__ void xchg_epilogue(const KParams &p, const UnitOu
 // c + G, ...), p.prefetch_stages stages at most, in each unit's stream order,
 // skipping the first `skip` stages of each first-round unit (its claimer's
 // ring already holds them).  Out of line: it runs at most once per task.
+template <bool kExt>
 static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDev &T, int skip) {
     int budget = p.prefetch_stages;
     for (int uu = blockIdx.x; uu < T.n_units && budget > 0; uu += gridDim.x) {
@@ -355,7 +356,7 @@ static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDe
         tile_coords(T, ps.tile, pg, pmt);
         const int halves = p.wide ? 2 : 1;
         const int k_len = ps.k_end - ps.k_begin;
-        const int k_rot = unit_k_rot(p, T, ps);
+        const int k_rot = kExt ? unit_k_rot(p, T, ps) : (p.k_rotate ? (ps.tile * 11) % k_len : 0);  // as the producer
         for (int i = (uu < (int)gridDim.x ? skip : 0); i < k_len && budget > 0; ++i, --budget) {
             const int kk = ps.k_begin + (i + k_rot) % k_len;
             for (int h = 0; h < halves; ++h)
@@ -365,6 +366,12 @@ static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDe
     }
 }
 
+// kExt compiles in what only some chains and calls need: cluster reduction of split tiles (KParams::cluster),
+// die-grouped claims (TaskDev::die_split) and the K rotation's weight-column mapping for M-tiled tasks.
+// Everything else runs the instantiation without them: measured on B200, that code in the kernel (not
+// executed), and the column mapping's divisions on the producer thread and in the L2 prefetch, made the
+// dependent 36 x 4 layer chain 2.7 % (3.49 -> 3.40 ms) and the independent decode step 2-3 % slower.
+template <bool kExt>
 __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_constant__ KParams p) {
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
@@ -404,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (p.cluster) {
+    if ((kExt && p.cluster)) {
         // exchange flags start at 0 (no task's index + 1) before any peer can write them
         float *xb = reinterpret_cast<float *>(ring + p.xbuf_off);
         for (int i = threadIdx.x; i < 3 * 32; i += blockDim.x) xb[(size_t)i * p.xrow + p.xrow - 4] = 0.f;
@@ -472,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     prefetched = true;
                     // the first-round units' first stages sit in their claimers' rings: the whole ring
                     // ahead of the grid dependency, dep_ring_stages ahead of a task dependency
-                    prefetch_w_l2(p, T, (T.dep >= 0 && p.dep_ring_stages > 0) ? min(S, p.dep_ring_stages) : S);
+                    prefetch_w_l2<kExt>(p, T, (T.dep >= 0 && p.dep_ring_stages > 0) ? min(S, p.dep_ring_stages) : S);
                 };
                 auto flush = [&]() {
                     if (!grid_dep_ok) {
@@ -521,12 +528,12 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 // previous task first take the next task's work.
                 // (with two-level readiness a CTA works only on its group's tiles, all claimed)
                 // (die-grouped claims: this CTA's die's range first, then the other die's)
-                const bool by_die = T.die_split > 0;
+                const bool by_die = kExt && T.die_split > 0;
                 const int my_die = by_die ? cta_die(p) : 0;
                 ClaimRange cr = by_die ? die_claim_range(T, my_die) : claim_range(T);
                 // (cluster mode: every task's first round is static, so a split tile's units of that round
                 // sit on the consecutive CTAs of one cluster)
-                const bool static_first = (t == 0 || p.cluster) && T.n_groups <= 1 && !by_die;  // (independent: t == 0)
+                const bool static_first = (t == 0 || (kExt && p.cluster)) && T.n_groups <= 1 && !by_die;  // (independent: t == 0)
                 const int n_static = static_first ? min((int)gridDim.x, T.n_units) : 0;
                 int u;
                 if (static_first) {
@@ -553,7 +560,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         int next_u = cr.hi - cr.lo - n_static;
                         bool claimed = false;
                         const int k_len = us.k_end - us.k_begin;
-                        const int k_rot = unit_k_rot(p, T, us);
+                        // (without M-tiles a unit's weight column is its tile: kExt covers the chains with them)
+                        const int k_rot = kExt ? unit_k_rot(p, T, us)
+                                               : (p.k_rotate ? (us.tile * 11) % (us.k_end - us.k_begin) : 0);
                         for (int kk = us.k_begin; kk < us.k_end; ++kk) {
                             if (!take_slot()) break;
                             slot_ok = false;
@@ -746,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             const int mrows = min(T.t_m, T.M - m0);
             UnitOut uo = unit_out(T);  // no task-table reads after the first store below
             unit_out_group(uo, T, tile);
-            if (p.cluster && us.nu > 1 && u < min((int)gridDim.x, T.u_head)) {
+            if ((kExt && p.cluster) && us.nu > 1 && u < min((int)gridDim.x, T.u_head)) {
                 // a split tile of a static first round: its units are on this cluster's CTAs
                 xchg_epilogue(p, uo, us, t, u, tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * acc_stride, q,
                               lane, g * kUmmaRows + row, m0, mrows, set, leader,
@@ -827,7 +836,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (p.cluster) cluster_sync_all();  // no CTA leaves while a peer may still write its exchange buffer
+    if ((kExt && p.cluster)) cluster_sync_all();  // no CTA leaves while a peer may still write its exchange buffer
     if (warp == 1) tmem_dealloc(tmem_base, p.wide ? kTmemColsWide : kTmemCols);
     if (threadIdx.x == 0) {
         if (p.run_ctl) chain_run_done(p);
@@ -836,6 +845,14 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         // order): one CTA waits for it, the others leave their SMs to the calls beside this one
         else if (blockIdx.x == 0 && p.pdl) pdl_wait();
     }
+}
+
+template __global__ void wsm_umma_kernel<false>(const __grid_constant__ KParams p);
+template __global__ void wsm_umma_kernel<true>(const __grid_constant__ KParams p);
+
+const void *umma_kernel_ptr(bool ext) {
+    return ext ? reinterpret_cast<const void *>(&wsm_umma_kernel<true>)
+               : reinterpret_cast<const void *>(&wsm_umma_kernel<false>);
 }
 
 }  // namespace wsm
