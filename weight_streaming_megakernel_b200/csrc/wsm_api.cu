@@ -1204,6 +1204,7 @@ wsm_status skinny_gemm_ex(const void *X, const void *W, void *Y, int M, int N, i
     kp.single.sched = reinterpret_cast<unsigned int *>(wsb + L.cnt_off);
     kp.single.tile_cnt = kp.single.sched + kSchedWords;
     kp.single.part = reinterpret_cast<float *>(wsb + L.part_off);
+    kp.cnt_words = (int)((L.part_off - L.cnt_off) / 4);
     kp.tasks = nullptr;
     kp.n_tasks = 1;
     kp.stages = g.stages;

@@ -52,6 +52,7 @@ constexpr int kStatusStallFlag = 5;
 // call clears it (none of their waits consult it).
 constexpr int kIndStatusOff = 32;  // ints
 static_assert(kIndStatusOff + kStatusStallFlag < 64, "the status region holds 64 ints");
+
 constexpr int kSchedWords = 2;     // per task: [0] next unit to claim, [1] CTAs done claiming
 constexpr int kClaimLead = 4;      // a CTA claims its next unit this many stages before its unit ends
 constexpr int kColChunk = 256;     // output columns per readiness chunk (per-column data dependencies)
@@ -72,7 +73,7 @@ enum : int { kEpiNone = 0, kEpiSiluMul = 1, kEpiResidual = 2 };
 
 // Error sites recorded in status[3].
 enum : int { kSiteNone = 0, kSiteDep = 1, kSiteFull = 2, kSiteEmpty = 3, kSiteAcc = 4, kSiteDrain = 5, kSiteStall = 6,
-             kSiteXchg = 7 };
+             kSiteXchg = 7, kSiteRepair = 8 };
 constexpr int kCodeTimeout = 6;    // == WSM_ERR_TIMEOUT
 
 // Stage / accumulator metadata flags (producer -> consumers).
@@ -170,6 +171,8 @@ struct KParams {
     int xrow;                       // cluster mode: floats per exchange-buffer row (widest X tile + 4, the
                                     // last 4 holding the row's flag)
     const signed char *sm_die;      // die-grouped claims: die of each SM id (kMaxSmIds entries), or nullptr
+    int cnt_words;                  // single calls: words of the scratch's counter region from single.sched on
+                                    // (zeroed by the next call after a failed one)
     int independent;                // single call that shares no data with the kernel before it and splits no
                                     // tile: CTA c runs units c, c + grid, ... (no claim counters, no scratch),
                                     // loads and stores without waiting for the previous kernel, and waits for it
@@ -300,6 +303,10 @@ __device__ __forceinline__ unsigned int atom_add_relaxed_gpu(unsigned int *p, un
 
 __device__ __forceinline__ void st_relaxed_gpu(unsigned int *p, unsigned int v) {
     asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned int *p, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -567,23 +574,59 @@ __device__ __forceinline__ int cta_die(const KParams &p) {
 // handed out statically (unit c to CTA c); a result >= cr.hi means none left.
 __device__ __forceinline__ int claim_unit(const ClaimRange &cr) { return (int)atom_add_relaxed_gpu(cr.ctr, 1u); }
 
-// Single GEMM: called once per CTA by thread 0 after the CTA's last barrier (all its roles are done).
-// The last CTA resets the claim counters for the next call; if this launch recorded an error, some CTA
-// abandoned its work, so tile arrival counters may be left mid-count: it clears them as well, then the
-// launch's error flag.  The next call on the same scratch starts clean (stream order, or the programmatic
-// dependency its scratch accesses wait for), and the sticky error words stay for the host to read.  A
-// chain resets its claim counters at the end of the run instead (chain_run_done).
-__device__ __forceinline__ void single_call_done(const KParams &p) {
-    const TaskDev &T = p.single;
+// Single GEMM accounting, kept off the end of the launch (an atomic there delayed every launch's completion
+// by its round trip: measured on B200, M = 1 4096 x 4096 back to back 10.5 -> 10.8 us).
+//
+// claims_finished: called once per CTA by the producer thread after its last claim, aborted or not; the
+// last CTA to finish claiming resets the claim counters for the next call.
+//
+// A launch that records an error (some CTA abandoned its work) may leave split-tile arrival counters
+// mid-count, and its launch error flag set.  The next single call on the same scratch repairs them before
+// any of its CTAs counts an arrival: the warp of CTA 0's first epilogue leader, once the previous kernel
+// has completed, zeroes the tile counters (the whole counter region: the failed call's shape is not known)
+// and clears the flag (repair_after_failure); every other epilogue leader waits, bounded, until the flag
+// is clear (wait_repaired).  The claim counters need no repair (every CTA counts its claims' end).  The sticky error
+// words stay for the host to read.  A chain resets its counters at the end of each run (chain_run_done).
+__device__ __forceinline__ void claims_finished(const TaskDev &T, unsigned int grid) {
     const unsigned int old = atom_add_acqrel_gpu(&T.sched[1], 1u);
-    if (old != gridDim.x - 1) return;
-    st_relaxed_gpu(&T.sched[0], 0u);
-    if (launch_failed(p.status)) {
-        const int tiles = T.n_g * T.n_mt;
-        for (int i = 0; i < tiles; ++i) st_relaxed_gpu(&T.tile_cnt[i], 0u);
-        st_relaxed_gpu(reinterpret_cast<unsigned int *>(&p.status[kStatusLaunchErr]), 0u);
+    if (old == grid - 1) {
+        st_relaxed_gpu(&T.sched[0], 0u);
+        st_relaxed_gpu(&T.sched[1], 0u);
     }
-    st_relaxed_gpu(&T.sched[1], 0u);
+}
+
+// CTA 0: the warp of its (first) epilogue leader, all 32 lanes, after the grid dependency.
+__device__ __forceinline__ void repair_after_failure(const KParams &p, int lane) {
+    unsigned int *flag = reinterpret_cast<unsigned int *>(&p.status[kStatusLaunchErr]);
+    unsigned int v = lane == 0 ? ld_acquire_gpu(flag) : 0u;
+    v = __shfl_sync(0xffffffffu, v, 0);
+    if (v == 0u) return;
+    unsigned int *cnt = p.single.sched + kSchedWords;
+    for (int i = lane; i < p.cnt_words - kSchedWords; i += 32) st_relaxed_gpu(&cnt[i], 0u);
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) st_release_gpu(flag, 0u);
+}
+
+// Every other epilogue leader (the only thread that counts arrivals), after the grid dependency; false
+// (with an error recorded) if the repair did not come within the limit.
+static __device__ __noinline__ bool wait_repaired(const KParams &p) {
+    const unsigned int *flag = reinterpret_cast<const unsigned int *>(&p.status[kStatusLaunchErr]);
+    if (ld_acquire_gpu(flag) == 0u) return true;
+    // the repair follows within microseconds (CTA 0 passed the same grid dependency); a flag that stays set
+    // was set by this launch itself, whose own failure is on record already
+    const unsigned long long limit = p.wait_timeout_ns < 100000000ull ? p.wait_timeout_ns : 100000000ull;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t spin = 1;; ++spin) {
+        if (ld_acquire_gpu(flag) == 0u) return true;
+        if ((spin & 31u) == 0) {
+            if (globaltimer() - t0 > limit) {
+                record_error(p.status, kCodeTimeout, -1, kSiteRepair);
+                return false;
+            }
+            __nanosleep(256);
+        }
+    }
 }
 
 // Test hook (KParams::debug_stall_ns): a bounded wait on a status word that nothing ever sets.  When the

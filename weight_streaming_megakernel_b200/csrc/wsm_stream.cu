@@ -360,6 +360,15 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
                 if (aborted) break;
                 if (T.dep < 0 && !first_unit) trace_stamp(p, t, 1, globaltimer());
             }
+            if (!p.run_ctl && !p.independent) {
+                // every CTA counts the end of its claims, aborted or not (after the grid dependency: until
+                // then the claim counters belong to the previous kernel)
+                if (!grid_dep_ok) {
+                    pdl_wait();
+                    grid_dep_ok = true;
+                }
+                claims_finished(p.single, gridDim.x);
+            }
             if (!grid_dep_ok) pdl_wait();
             // copies in flight must land before exit (checked before the end marker below advances one of
             // these barriers again)
@@ -389,6 +398,11 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
             // the next kernel may launch once every CTA has seen this one's predecessor complete: so at most
             // this kernel and the independent calls queued after it can still run when one of those starts
             if (leader) pdl_launch_dependents();
+        }
+        if (!p.run_ctl && !p.independent && cw == 0) {
+            // a single call: the tile counters a failed call before it left mid-count are repaired first
+            if (blockIdx.x == 0) repair_after_failure(p, lane);
+            else if (leader) wait_repaired(p);
         }
         const unsigned int run_no = p.run_ctl ? ld_acquire_gpu(&p.run_ctl[0]) + 1u : 0u;  // this chain run
         int s = 0;
@@ -535,10 +549,9 @@ __global__ void __launch_bounds__(32 * (1 + RG * KW), 1) wsm_stream_kernel(const
     __syncthreads();
     if (threadIdx.x == 0) {
         if (p.run_ctl) chain_run_done(p);
-        else if (!p.independent) single_call_done(p);
         // an independent call completes only after the kernel before it (later kernels rely on stream
         // order): one CTA waits for it, the others leave their SMs to the calls beside this one
-        else if (blockIdx.x == 0 && p.pdl) pdl_wait();
+        else if (p.independent && blockIdx.x == 0 && p.pdl) pdl_wait();
     }
 }
 

@@ -624,6 +624,15 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 if (aborted) break;
                 if (T.dep < 0 && !first_unit) trace_stamp(p, t, 1, globaltimer());
             }
+            if (!p.run_ctl && !p.independent) {
+                // every CTA counts the end of its claims, aborted or not (after the grid dependency: until
+                // then the claim counters belong to the previous kernel)
+                if (!grid_dep_ok) {
+                    pdl_wait();
+                    grid_dep_ok = true;
+                }
+                claims_finished(p.single, gridDim.x);
+            }
             if (!grid_dep_ok) pdl_wait();  // a CTA with no work still orders itself after the previous kernel
             // copies in flight must land before exit, abort or not (checked before the end marker below
             // advances one of these barriers again)
@@ -730,6 +739,11 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             // the next kernel may launch once every CTA has seen this one's predecessor complete: so at most
             // this kernel and the independent calls queued after it can still run when one of those starts
             if (set == 0 && leader) pdl_launch_dependents();
+        }
+        if (!p.run_ctl && !p.independent && etid < 32) {
+            // a single call: the tile counters a failed call before it left mid-count are repaired first
+            if (blockIdx.x == 0 && set == 0) repair_after_failure(p, lane);
+            else if (leader) wait_repaired(p);
         }
         const unsigned int run_no = p.run_ctl ? ld_acquire_gpu(&p.run_ctl[0]) + 1u : 0u;  // this chain run
         int warm_t = 0;                         // the task whose descriptor the set warms while it waits
@@ -840,10 +854,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     if (warp == 1) tmem_dealloc(tmem_base, p.wide ? kTmemColsWide : kTmemCols);
     if (threadIdx.x == 0) {
         if (p.run_ctl) chain_run_done(p);
-        else if (!p.independent) single_call_done(p);
         // an independent call completes only after the kernel before it (later kernels rely on stream
         // order): one CTA waits for it, the others leave their SMs to the calls beside this one
-        else if (blockIdx.x == 0 && p.pdl) pdl_wait();
+        else if (p.independent && blockIdx.x == 0 && p.pdl) pdl_wait();
     }
 }
 
