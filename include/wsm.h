@@ -249,9 +249,10 @@ size_t wsm_workspace_bytes(int M, int N, int K, const wsm_opts *opts);
 /* Device-side time-outs.  Every wait inside the kernels is bounded.  A wait
  * that runs out (never in a healthy run) records a sticky error in the status
  * words of the call's scratch, and the CTA that hit it abandons its work, so
- * that call's outputs are incomplete.  When that launch ends, its last CTA
- * repairs the counters it left mid-count, so the next call on the same scratch
- * computes correct results.  The error stays recorded until one of the status
+ * that call's outputs are incomplete.  The counters it left mid-count are
+ * repaired on the device -- a chain's by the end of the failed run, a single
+ * call's by the next single call on the same scratch before it uses them --
+ * so the next call on the same scratch computes correct results.  The error stays recorded until one of the status
  * queries below reads and clears it: each synchronises the stream, returns
  * WSM_ERR_TIMEOUT once per recorded time-out (*code = WSM_ERR_TIMEOUT, message
  * in wsm_last_error()) and WSM_OK (*code = 0) otherwise.  This follows the
