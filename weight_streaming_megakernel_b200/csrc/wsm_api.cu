@@ -21,7 +21,7 @@
 
 namespace wsm {
 
-const void *umma_kernel_ptr(bool ext);                   // wsm_umma.cu
+const void *umma_kernel_ptr(bool chain, bool ext);       // wsm_umma.cu
 const void *stream_kernel_ptr(int mmax, int tile_rows);  // wsm_stream.cu
 void *noalloc_scratch_ptr(int dev);                      // wsm_noalloc.cu: nullptr until set up on `dev`
 wsm_status die_map_of_device(int dev, const std::vector<int> **die, wsm_die_info *info);  // wsm_die.cu
@@ -95,6 +95,7 @@ struct Geo {
     int ku_t = 1, nu_t = 1;    // tail tiles: the same
     int tail = 0;              // tail tiles (the last ones of the schedule)
     bool ext = false;          // tensor-core kernel with cluster reduction and die-grouped claims compiled in
+    bool chain = false;        // tensor-core kernel instantiated for chain runs
     int order = WSM_ORDER_M_MAJOR;
     int l2 = WSM_L2_EVICT_FIRST;
     int grid = 0;
@@ -487,8 +488,8 @@ wsm_status dev_info(int dev, DevInfo **out) {
 // Kernel for a geometry, and its slot in DevInfo::attr_set.
 const void *kernel_for(const Geo &g, int *slot) {
     if (g.path == WSM_PATH_UMMA) {
-        *slot = g.ext ? 9 : 0;
-        return umma_kernel_ptr(g.ext);
+        *slot = g.chain ? (g.ext ? 12 : 11) : (g.ext ? 10 : 0);
+        return umma_kernel_ptr(g.chain, g.ext);
     }
     *slot = (g.mmax == 1 ? 1 : g.mmax == 2 ? 2 : g.mmax == 4 ? 3 : 4) + (g.tile_rows == 32 ? 4 : 0);
     return stream_kernel_ptr(g.mmax, g.tile_rows);
@@ -515,6 +516,7 @@ wsm_status cluster_ctas_of(DevInfo *d, int *out) {
     Geo g;
     g.path = WSM_PATH_UMMA;
     g.ext = true;
+    g.chain = true;
     const void *fn;
     wsm_status st = prepare_kernel(d, g, &fn);
     if (st != WSM_OK) return st;
@@ -1583,6 +1585,7 @@ wsm_status wsm_chain_create(const wsm_task *tasks, int n, const wsm_chain_opts *
     bool any_m_tiled = false;
     for (int i = 0; i < n; ++i) any_m_tiled = any_m_tiled || geos[i].n_mt > 1;
     ch->geo.ext = cp.cluster != 0 || cp.die_groups || any_m_tiled;
+    ch->geo.chain = true;
     if ((st = prepare_kernel(d, ch->geo, &ch->fn)) != WSM_OK) {
         cleanup();
         return st;

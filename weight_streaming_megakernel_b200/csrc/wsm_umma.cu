@@ -371,8 +371,15 @@ static __device__ __noinline__ void prefetch_w_l2(const KParams &p, const TaskDe
 // Everything else runs the instantiation without them: measured on B200, that code in the kernel (not
 // executed), and the column mapping's divisions on the producer thread and in the L2 prefetch, made the
 // dependent 36 x 4 layer chain 2.7 % (3.49 -> 3.40 ms) and the independent decode step 2-3 % slower.
-template <bool kExt>
+// kChain likewise separates chain runs from single calls (back-to-back single launches on the tensor
+// cores 3-6 % faster without the chains' dependency and readiness code, e.g. o at M = 16 15.2 -> 14.3 us).
+template <bool kChain, bool kExt>
 __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_constant__ KParams p) {
+    // kChain: a chain run (run counter, task dependencies, readiness counters), else a single call; each
+    // instantiation carries only its own accounting
+    unsigned int *const run_ctl = kChain ? p.run_ctl : nullptr;
+    const bool indep = !kChain && p.independent;
+    auto tdep = [](const TaskDev &X) { return kChain ? X.dep : -1; };
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
@@ -403,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         mbar_init(&drain_bar, 1);
         abort_flag = 0;
         fence_mbar_init();
-        if (p.independent) pdl_launch_dependents();  // other calls trigger once past their grid wait (epilogue)
+        if (indep) pdl_launch_dependents();  // other calls trigger once past their grid wait (epilogue)
     }
     const int halves = p.wide ? 2 : 1;          // 128-row W halves per tile
     const uint32_t acc_stride = (uint32_t)(halves * kUmmaMaxN);  // TMEM columns per accumulator buffer
@@ -430,12 +437,12 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
             bool aborted = false;
             bool slot_ok = false;           // the wait for ring slot s has already succeeded
             // mode 2 streams W before the previous kernel completes; an independent call never waits here
-            bool grid_dep_ok = p.pdl != 2 || p.independent;
-            if (p.pdl == 1 && !p.independent) pdl_wait();
+            bool grid_dep_ok = p.pdl != 2 || indep;
+            if (p.pdl == 1 && !indep) pdl_wait();
             if (p.debug_stall_ns && blockIdx.x == 0) {
                 // test hook: after the previous kernel (whose exit clears the launch error flag), wait on a
                 // flag nothing sets until the limit passes, then abandon all of this CTA's work
-                if (!grid_dep_ok || p.independent) {
+                if (!grid_dep_ok || indep) {
                     pdl_wait();
                     grid_dep_ok = true;
                 }
@@ -447,10 +454,10 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 prefetch_tmap(&T.tmW);
                 prefetch_tmap(&T.tmX);
                 const uint64_t pol_w = T.w_evict_first ? policy_evict_first() : policy_evict_normal();
-                const bool col_dep = T.dep >= 0 && T.dep_col_cnt != nullptr;
+                const bool col_dep = tdep(T) >= 0 && T.dep_col_cnt != nullptr;
                 // nothing of X before the dependency is met (per column: the first chunks; after that the
                 // chunk mask decides stage by stage)
-                bool dep_ok = T.dep < 0 && grid_dep_ok;
+                bool dep_ok = tdep(T) < 0 && grid_dep_ok;
                 int pend_s[kMaxStages], pend_k[kMaxStages], pend_y[kMaxStages];
                 int np = 0;
                 // Per-column dependency: each stage's X waits only for the kColChunk-column chunks it
@@ -479,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     prefetched = true;
                     // the first-round units' first stages sit in their claimers' rings: the whole ring
                     // ahead of the grid dependency, dep_ring_stages ahead of a task dependency
-                    prefetch_w_l2<kExt>(p, T, (T.dep >= 0 && p.dep_ring_stages > 0) ? min(S, p.dep_ring_stages) : S);
+                    prefetch_w_l2<kExt>(p, T, (tdep(T) >= 0 && p.dep_ring_stages > 0) ? min(S, p.dep_ring_stages) : S);
                 };
                 auto flush = [&]() {
                     if (!grid_dep_ok) {
@@ -487,11 +494,11 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         pdl_wait();
                         grid_dep_ok = true;
                     }
-                    if (T.dep >= 0 && !col_dep) {
-                        if (!prefetched && !dependency_met(p, task_at(p, T.dep))) prefetch_l2();
-                        wait_dependency(p, task_at(p, T.dep), t, p.status);
+                    if (tdep(T) >= 0 && !col_dep) {
+                        if (!prefetched && !dependency_met(p, task_at(p, tdep(T)))) prefetch_l2();
+                        wait_dependency(p, task_at(p, tdep(T)), t, p.status);
                     }
-                    if (col_dep && run_no == 0) run_no = ld_acquire_gpu(&p.run_ctl[0]) + 1u;
+                    if (col_dep && run_no == 0) run_no = ld_acquire_gpu(&run_ctl[0]) + 1u;
                     if (!dep_ok) trace_stamp(p, t, 1, globaltimer());
                     for (int i = 0; i < np; ++i) {
                         if (col_dep) {
@@ -512,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     if (slot_ok) return true;
                     // a dependent task streams at most dep_ring_stages stages of W ahead of its dependency:
                     // more only queues in front of the round trips that end the previous task
-                    if (np > 0 && T.dep >= 0 && p.dep_ring_stages > 0 && np >= p.dep_ring_stages) flush();
+                    if (np > 0 && tdep(T) >= 0 && p.dep_ring_stages > 0 && np >= p.dep_ring_stages) flush();
                     if (np > 0 && !mbar_test(&empty_bar[s], ph ^ 1)) flush();
                     if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1, &abort_flag, wlim, p.status, t, kSiteEmpty)) {
                         if (np > 0) flush();
@@ -542,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                     if (!grid_dep_ok) {
                         pdl_wait();
                         grid_dep_ok = true;
-                        dep_ok = T.dep < 0;
+                        dep_ok = tdep(T) < 0;
                     }
                     u = cr.lo + claim_unit(cr);
                 }
@@ -599,13 +606,13 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                             // take -- and never while this task's dependency is unmet, when every CTA would
                             // hold a second unit it cannot start (the claim counters belong to the previous
                             // kernel until the grid dependency is resolved)
-                            if (!claimed && !p.independent && dep_ok && us.k_end - kk <= kClaimLead) {
+                            if (!claimed && !indep && dep_ok && us.k_end - kk <= kClaimLead) {
                                 next_u = claim_unit(cr);
                                 claimed = true;
                             }
                         }
                         if (aborted) break;
-                        if (!claimed && !p.independent) {
+                        if (!claimed && !indep) {
                             // the unit streamed completely before its dependencies were resolved
                             if (!dep_ok) flush();
                             next_u = claim_unit(cr);
@@ -613,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                         // whatever comes next needs a free slot: wait for it before the claim's result is used,
                         // so the claim's round trip overlaps the wait
                         if (!take_slot()) break;
-                        u = p.independent ? u + (int)gridDim.x : cr.lo + next_u + n_static;
+                        u = indep ? u + (int)gridDim.x : cr.lo + next_u + n_static;
                     }
                     if (aborted || !by_die || pass > 0) break;
                     // own die's range done: help with the other die's
@@ -622,9 +629,9 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                 }
                 if (np > 0) flush();
                 if (aborted) break;
-                if (T.dep < 0 && !first_unit) trace_stamp(p, t, 1, globaltimer());
+                if (tdep(T) < 0 && !first_unit) trace_stamp(p, t, 1, globaltimer());
             }
-            if (!p.run_ctl && !p.independent) {
+            if (!run_ctl && !indep) {
                 // every CTA counts the end of its claims, aborted or not (after the grid dependency: until
                 // then the claim counters belong to the previous kernel)
                 if (!grid_dep_ok) {
@@ -683,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
                                            t, kSiteAcc))
                         break;
                     tc_fence_after();
-                    if (p.trace && t != traced_t) {
+                    if (kChain && p.trace && t != traced_t) {
                         trace_stamp(p, t, 7, globaltimer());
                         traced_t = t;
                     }
@@ -734,18 +741,18 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
         const int row = q * 32 + lane;          // row of the 128-row tile = TMEM lane
         const int etid = threadIdx.x - (kEpiWarp0 + 4 * set) * 32;
         const bool leader = (etid == 0);
-        if (p.pdl && !p.independent) {
+        if (p.pdl && !indep) {
             pdl_wait();  // Y and the scratch may still be in use by the previous kernel
             // the next kernel may launch once every CTA has seen this one's predecessor complete: so at most
             // this kernel and the independent calls queued after it can still run when one of those starts
             if (set == 0 && leader) pdl_launch_dependents();
         }
-        if (!p.run_ctl && !p.independent && etid < 32) {
+        if (!run_ctl && !indep && etid < 32) {
             // a single call: the tile counters a failed call before it left mid-count are repaired first
             if (blockIdx.x == 0 && set == 0) repair_after_failure(p, lane);
             else if (leader) wait_repaired(p);
         }
-        const unsigned int run_no = p.run_ctl ? ld_acquire_gpu(&p.run_ctl[0]) + 1u : 0u;  // this chain run
+        const unsigned int run_no = run_ctl ? ld_acquire_gpu(&run_ctl[0]) + 1u : 0u;  // this chain run
         int warm_t = 0;                         // the task whose descriptor the set warms while it waits
         for (uint32_t k = 0;; ++k) {
             const uint32_t acc_i = kEpiSets * k + (uint32_t)set;
@@ -853,19 +860,24 @@ __global__ void __launch_bounds__(kThreads, 1) wsm_umma_kernel(const __grid_cons
     if ((kExt && p.cluster)) cluster_sync_all();  // no CTA leaves while a peer may still write its exchange buffer
     if (warp == 1) tmem_dealloc(tmem_base, p.wide ? kTmemColsWide : kTmemCols);
     if (threadIdx.x == 0) {
-        if (p.run_ctl) chain_run_done(p);
+        if (run_ctl) chain_run_done(p);
         // an independent call completes only after the kernel before it (later kernels rely on stream
         // order): one CTA waits for it, the others leave their SMs to the calls beside this one
-        else if (p.independent && blockIdx.x == 0 && p.pdl) pdl_wait();
+        else if (indep && blockIdx.x == 0 && p.pdl) pdl_wait();
     }
 }
 
-template __global__ void wsm_umma_kernel<false>(const __grid_constant__ KParams p);
-template __global__ void wsm_umma_kernel<true>(const __grid_constant__ KParams p);
+template __global__ void wsm_umma_kernel<false, false>(const __grid_constant__ KParams p);
+template __global__ void wsm_umma_kernel<false, true>(const __grid_constant__ KParams p);
+template __global__ void wsm_umma_kernel<true, false>(const __grid_constant__ KParams p);
+template __global__ void wsm_umma_kernel<true, true>(const __grid_constant__ KParams p);
 
-const void *umma_kernel_ptr(bool ext) {
-    return ext ? reinterpret_cast<const void *>(&wsm_umma_kernel<true>)
-               : reinterpret_cast<const void *>(&wsm_umma_kernel<false>);
+const void *umma_kernel_ptr(bool chain, bool ext) {
+    if (chain)
+        return ext ? reinterpret_cast<const void *>(&wsm_umma_kernel<true, true>)
+                   : reinterpret_cast<const void *>(&wsm_umma_kernel<true, false>);
+    return ext ? reinterpret_cast<const void *>(&wsm_umma_kernel<false, true>)
+               : reinterpret_cast<const void *>(&wsm_umma_kernel<false, false>);
 }
 
 }  // namespace wsm
