@@ -1,5 +1,6 @@
-"""bench.py's reference arm (the fp64 oracle timed on the host cores) runs
-without a GPU and prints the one JSON line of the benchmark contract."""
+"""bench.py on the host: its reference arm (the fp64 oracle timed on the host
+cores) runs without a GPU and prints the one JSON line of the benchmark
+contract, and its weight-copy rotation keeps timed weights out of L2."""
 import json
 import os
 import subprocess
@@ -43,3 +44,23 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1, out.stdout
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2
+
+
+def test_weight_copies_keep_steps_and_concurrent_launches_apart():
+    """Weight copies: consecutive steps touch at least 4x L2, and for
+    independent launches (several run at once) a copy comes back only after
+    INDEPENDENT_REUSE_CALLS launches, so no two calls in flight share weights
+    through L2."""
+    import bench
+    import synth
+    L2 = bench.L2_BYTES
+    for name in ("qwen3_decode", "single", "skinny", "l2_reuse", "l2_reuse_whole_m", "chain"):
+        cases = bench.workload_cases(name)
+        w = sum(2 * c.N * c.K for c in cases)
+        n = bench.n_copies(cases)
+        assert n * w >= 4 * L2 or n == 1 and w >= 4 * L2
+        ni = bench.n_copies(cases, bench.INDEPENDENT_REUSE_CALLS)
+        assert ni >= n and ni * len(cases) >= bench.INDEPENDENT_REUSE_CALLS
+    for c in synth.config_qwen3_decode():   # the per-shape runs: one GEMM per step
+        n = bench.n_copies([c], bench.INDEPENDENT_REUSE_CALLS)
+        assert n >= bench.INDEPENDENT_REUSE_CALLS and n * 2 * c.N * c.K >= 4 * L2
